@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of one DSA decode step (indexer scan -> top-k -> sparse MQA) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3] [--impl ours|reference]
+
+Default workload: batched paged decode, B=32 sequences with lengths drawn
+uniformly in [65536, 131072], 64-token blocks under a random block permutation,
+a 64-head x 128 bf16 lightning indexer, top-2048, 128-head MQA over 576-wide
+bf16 KV rows (value = first 512 columns).  Inputs are seeded synthetic data of
+that shape, resident in HBM before timing; the per-step key stream (~805 MB) is
+larger than L2, so no explicit flush is needed.
+
+Prints ONE JSON line on rank 0.  With N > 1 (torchrun, one process per GPU) each
+rank runs its own independent batch (weak scaling, no collective on the data
+path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from sparse_attention_decode_scan_b200 import synth  # noqa: E402
+
+METRIC = "decode steps/s (scan+top-k+sparse attn) at B=32,128K; % of HBM peak GB/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- host-side plumbing
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def rank_seed(cfg: int, rank: int) -> int:
+    """Each rank draws its own batch (independent units, weak scaling)."""
+    return synth.seed_of(cfg) + 7919 * rank
+
+
+def reduce_max(x: float, group=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    dev = "cuda" if dist.get_backend(group) == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def source_hash(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+SCAN_SOURCES = ["sparse_attention_decode_scan_b200/csrc/indexer_tc.cu",
+                "sparse_attention_decode_scan_b200/csrc/indexer_simt.cu",
+                "sparse_attention_decode_scan_b200/csrc/common.cuh"]
+
+
+def scan_traffic(workload: str):
+    """DRAM bytes per scan launch from the committed ncu summary, if it still
+    describes the current scan sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = t.get(workload, {}).get("scan")
+    if not e or e.get("source_hash") != source_hash(SCAN_SOURCES):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- reference arm (the oracle)
+
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_oracle_rate(case, rows, repeats: int = 1):
+    """Times the oracle's full step on `rows` (scores, top-k, attention) and
+    returns (seconds per row, rows timed)."""
+    from oracle import lsa_oracle as O
+    t0 = time.perf_counter()
+    n = 0
+    for _ in range(repeats):
+        for r in rows:
+            O.row_step(case, r)
+            n += 1
+    return (time.perf_counter() - t0) / n, n
+
+
+def run_reference(args, ws_, rank):
+    if rank != 0:
+        return
+    cfg = args.config
+    case = synth.make_case(synth.CONFIGS[cfg], rank_seed(cfg, 0))
+    B = case.rows
+    per = []
+    for i in range(args.warmup + args.steps):
+        r = i % B
+        t, _ = cpu_oracle_rate(case, [r])
+        if i >= args.warmup:
+            per.append(t)
+    sec_per_step = statistics.mean(per) * B
+    value = 1.0 / sec_per_step
+    cores = oracle_threads()
+    sample = f"{args.steps} timed steps of one sequence each (full scan, top-k, attention), scaled to B={B}"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec_per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(cfg, case),
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- our arm
+
+def workload_config(cfg, case):
+    s = case.spec
+    c = {"workload": s.name, "batch": case.rows, "seq_len_min": int(case.seq_lens.min()),
+         "seq_len_max": int(case.seq_lens.max()), "seq_len_mean": float(case.seq_lens.mean()),
+         "block_size": s.block_size, "idx_heads": s.n_idx_heads, "idx_dim": s.idx_dim,
+         "idx_key_dtype": s.idx_key_dtype, "top_k": s.top_k, "heads": s.n_heads, "kv_width": s.qk_dim,
+         "v_dim": s.v_dim, "parallelism": "replicas (independent batch per GPU)",
+         "l2": "inputs larger than L2 (indexer keys streamed from HBM every step)" if cfg in (3, 4)
+         else "L2 flushed between steps (256 MB write, outside the kernels' event windows)"}
+    return c
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase, to_device
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = args.config
+    spec = synth.CONFIGS[cfg]
+    case = synth.make_case(spec, rank_seed(cfg, rank))
+    dc = DeviceCase(case, device=dev)
+    s = case.spec
+    R = dc.rows
+    ld = (dc.max_len + 3) // 4 * 4
+    odt = torch.float32 if s.act_dtype == "f32" else torch.bfloat16
+    prefill = s.causal
+    scores = torch.empty((R, ld), dtype=torch.float32, device=dev)
+    idx = torch.empty((R, s.top_k), dtype=torch.int32, device=dev)
+    out = torch.empty((R, s.n_heads, s.v_dim), dtype=odt, device=dev)
+    lse = torch.empty((R, s.n_heads), dtype=torch.float32, device=dev)
+    ws_bytes = max(lsa.workspace_size(dc.dims, R, dc.max_len, op) for op in
+                   (lsa.LSA_OP_SCORES, lsa.LSA_OP_TOPK, lsa.LSA_OP_ATTN, lsa.LSA_OP_DECODE_STEP))
+    ws = lsa.workspace(ws_bytes, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = None if cfg in (3, 4) else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    L = int(case.seq_lens[0])
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        lsa.indexer_scores(dc.dims, dc.cache, dc.q_idx, dc.w, scores, ld, ws, row_seq=dc.row_seq,
+                           row_pos=dc.row_pos, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if prefill:
+            lsa.topk(scores, s.top_k, idx, ws, n_cols=L, ld=ld, stream=stream)
+        else:
+            lsa.topk(scores, s.top_k, idx, ws, valid_len=dc.seq_lens, n_cols=dc.max_len, ld=ld, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        lsa.sparse_attn_decode(dc.dims, dc.cache, dc.q, idx, out, lse, ws, row_seq=dc.row_seq, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+        if flush is not None:
+            flush.zero_()
+    torch.cuda.synchronize(dev)
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    with ClockSampler(gpu_index) as clk:
+        barrier()
+        torch.cuda.synchronize(dev)
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+            if flush is not None:
+                flush.zero_()
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    scan_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    topk_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    attn_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    # with a flush between steps the wall window includes it; the step time is the kernels' window
+    kernel_ms_sum = sum(step_ms)
+    timed_ms = kernel_ms_sum if flush is not None else total_ms
+    timed_ms = reduce_max(timed_ms)
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+
+    # e2e: the public decode-step call with host (pinned) inputs and outputs
+    e2e = None
+    if not prefill:
+        h_qidx = to_device(case.q_idx, s.act_dtype, pin=True)
+        h_w = torch.from_numpy(case.w).pin_memory()
+        h_q = to_device(case.q, s.act_dtype, pin=True)
+        h_out = torch.empty(out.shape, dtype=odt).pin_memory()
+        h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        d_qidx, d_w, d_q = torch.empty_like(dc.q_idx), torch.empty_like(dc.w), torch.empty_like(dc.q)
+
+        def e2e_step():
+            d_qidx.copy_(h_qidx, non_blocking=True)
+            d_w.copy_(h_w, non_blocking=True)
+            d_q.copy_(h_q, non_blocking=True)
+            lsa.decode_step(dc.dims, dc.cache, d_qidx, d_w, d_q, out, lse, ws, stream=stream)
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = reduce_max(a.elapsed_time(b))
+        h2d = h_qidx.numel() * h_qidx.element_size() + h_w.numel() * 4 + h_q.numel() * h_q.element_size()
+        d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * 4
+        e2e = {"value": world * args.steps / (e2e_ms / 1e3), "unit": "steps/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "note": "caches resident in HBM (model state); per-step queries in, outputs out"}
+
+    peaks, peak_src = load_peaks()
+    nb = synth.nbytes_decode_step(case)
+    ms_per_step = timed_ms / args.steps
+    value = world * args.steps / (timed_ms / 1e3)
+    scan_avg = statistics.mean(scan_ms)
+    if prefill:
+        fl = synth.flops_prefill_scan(case)
+        achieved = fl / (scan_avg / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": scan_traffic(s.name), "kernel": "indexer scan (prefill)",
+                "peak_source": f"{peak_src} bf16_tflops (burst)"}
+        unit = "chunk rows/s"
+        value = world * args.steps * R / (timed_ms / 1e3)
+    else:
+        scan_bytes = nb["keys"] + nb["scales"] + nb["block_table"] + nb["q_idx_w"] + nb["scores_fp32"]
+        achieved = scan_bytes / (scan_avg / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": scan_traffic(s.name), "kernel": "indexer scan",
+                "algorithmic_bytes_per_launch": scan_bytes, "peak_source": f"{peak_src} hbm_gbs"}
+        unit = "steps/s"
+    step_gbs = nb["total"] / (ms_per_step / 1e3) / 1e9
+    # launches of our kernels per step, as the library plans them for these sizes
+    per_step = sum(lsa.launch_count(dc.dims, R, dc.max_len, op, causal=prefill)
+                   for op in (lsa.LSA_OP_SCORES, lsa.LSA_OP_TOPK, lsa.LSA_OP_ATTN))
+    launches = per_step * args.steps
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        sample_rows = [0] if not prefill else [0, R - 1]
+        t, n = cpu_oracle_rate(case, sample_rows)
+        if prefill:
+            cpu_val = 1.0 / t
+            cpu_unit = "chunk rows/s"
+        else:
+            cpu_val = 1.0 / (t * R)
+            cpu_unit = "steps/s"
+        cpu = {"value": cpu_val, "unit": cpu_unit, "cores": oracle_threads(), "kind": "oracle",
+               "sample": f"{n} query row(s) of the same workload through the full oracle step, scaled to the "
+                         f"{'chunk' if prefill else 'batch'}"}
+    clocks = clk.summary()
+    line = {"metric": METRIC if not prefill else "prefill chunk rows/s (causal indexer scan + top-k + sparse attn)",
+            "value": value, "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": s.act_dtype if s.idx_key_dtype != "fp8" else "bf16+fp8",
+            "data": "synthetic (seeded, generated on host)", "config": workload_config(cfg, case),
+            "tokens_per_s": value * R if not prefill else None,
+            "step_hbm_gbs": step_gbs, "step_hbm_frac": step_gbs / peaks["hbm_gbs"],
+            "step_algorithmic_bytes": nb["total"],
+            "kernel_ms": {"scan": scan_avg, "topk": statistics.mean(topk_ms), "attn": statistics.mean(attn_ms)},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=3, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,208 @@
+/*
+ * lsa.h -- C ABI of liblsa.so: one DeepSeek-Sparse-Attention (DSA) decode step
+ * on NVIDIA B200 (sm_100a), and its causal prefill variant.
+ *
+ * What the step computes (sources are the pages this library restates):
+ *
+ *   1. Lightning-indexer scan.  Before each DSA layer a lightning indexer scores
+ *      every cached token of the sequence and the layer attends only the k best
+ *      (k = 2048 in production) -- MLI "Multi-layer Indexer" abstract
+ *      (zhuanzhiai.com), sentence 2.  At long context this scan is where decode
+ *      time goes (same abstract, sentence 3).  The score of cached token s for a
+ *      query row is DSA's lightning-indexer form
+ *          I(s) = sum_{h < H_I} w[h] * ReLU( sum_{d < d_I} q_idx[h][d] * K[s][d] )
+ *      (DeepSeek-V3.2-Exp technical report, listed as a source on the LeanSparse
+ *      episode page).  FP8 indexer keys carry a per-token scale:
+ *      K[s][d] = scale[s] * e4m3(K[s][d]) (the compact indexer keys of the
+ *      LeanSparse episode page).
+ *   2. Top-k: the k highest scores of each row; equal scores go to the lower
+ *      position; -inf and NaN are never selected.
+ *   3. Sparse MQA over the selected rows only ("reduces reads but not storage",
+ *      LeanSparse episode page): for every head h,
+ *          o[h] = sum_j softmax_j(scale * q[h] . KV[idx_j]) * KV[idx_j][0:D_v]
+ *      and lse[h] = log sum_j exp(scale * q[h] . KV[idx_j]).
+ *   Prefill: a chunk of query rows at positions p_i scores the cache under a
+ *   causal mask (s visible iff s <= p_i), then steps 2-3 run per row (the
+ *   prefill workspace concern of the LeanSparse episode page).
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument named as "device" is a CUDA device pointer on the
+ *     current device; structs (lsa_dims, lsa_cache) live in host memory and are
+ *     read during the call only.  The caller owns every buffer.
+ *   - The library never allocates device memory and never synchronises the
+ *     stream, except lsa_read_device_status, which does both a copy and a
+ *     stream synchronisation by design.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  A call returns after enqueueing.
+ *   - Host-checkable argument errors return an error code and enqueue nothing.
+ *   - Errors only the GPU can see (a block-table entry outside the pool, a
+ *     sequence length above max_len) make the kernels skip the bad access, write
+ *     NaN for affected outputs, and record the first such error in the
+ *     workspace status word; read it with lsa_read_device_status.  Kernels never
+ *     trap.
+ *   - Cache addressing: positions are logical token positions.  Paged caches
+ *     (block_size > 0) map position p of sequence b to the stored row
+ *     block_table[b][p / block_size] * block_size + p % block_size.  Contiguous
+ *     caches (block_size == 0) map it to row b * max_len + p.
+ *   - Workspace: `ws` is a device buffer of at least lsa_workspace_size(...)
+ *     bytes, 256-byte aligned.  Its first 256 bytes hold the status word; zero
+ *     them once after allocating (e.g. allocate zero-filled).  Calls that share
+ *     one workspace must be ordered on one stream.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LSA_VERSION 1
+
+typedef struct CUstream_st* lsa_stream_t; /* same handle type as cudaStream_t */
+
+typedef enum {
+  LSA_OK = 0,
+  LSA_ERR_INVALID_ARG = 1, /* host-checkable argument error; nothing enqueued */
+  LSA_ERR_UNSUPPORTED = 2, /* valid but unsupported shape/dtype combination */
+  LSA_ERR_WORKSPACE = 3,   /* ws NULL, misaligned or smaller than required */
+  LSA_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, attribute) */
+  LSA_ERR_TIMEOUT = 5,     /* device: a bounded wait gave up (status word) */
+  LSA_ERR_BOUNDS = 6       /* device: block id / length out of range (status word) */
+} lsa_status;
+
+typedef enum { LSA_F32 = 0, LSA_BF16 = 1, LSA_FP8_E4M3 = 2 } lsa_dtype;
+
+/* Shapes and element types of the step; validated on every call. */
+typedef struct {
+  int32_t n_idx_heads;   /* H_I: indexer heads (1..64)                              */
+  int32_t idx_dim;       /* d_I: indexer head dim (multiple of 8, 8..256)           */
+  int32_t n_heads;       /* H: attention query heads sharing one KV row (MQA)       */
+  int32_t qk_dim;        /* D: KV row width = q width (multiple of 8, <= 1024)      */
+  int32_t v_dim;         /* D_v <= D: the value is the first D_v columns of the row */
+  int32_t top_k;         /* k: tokens kept per query row (1..8192)                  */
+  int32_t block_size;    /* tokens per cache block, 0 = contiguous caches           */
+  float softmax_scale;   /* logit scale of the sparse attention                     */
+  int32_t act_dtype;     /* q_idx, q, kv and out: LSA_F32 or LSA_BF16               */
+  int32_t idx_key_dtype; /* indexer keys: LSA_F32, LSA_BF16 or LSA_FP8_E4M3         */
+} lsa_dims;
+
+/* Caller-owned caches of one layer (device pointers). */
+typedef struct {
+  const void* idx_keys;        /* [n_blocks, bs, d_I] or [batch, max_len, d_I], idx_key_dtype */
+  const float* idx_key_scales; /* FP8 keys only: [n_blocks, bs] or [batch, max_len]; else NULL */
+  const void* kv;              /* [n_blocks, bs, D] or [batch, max_len, D], act_dtype; may be
+                                  NULL for calls that do not read it                             */
+  const int32_t* block_table;  /* [batch, max_blocks_per_seq] (paged) or NULL (contiguous)      */
+  int32_t max_blocks_per_seq;  /* row stride of block_table (paged)                             */
+  int64_t n_blocks;            /* physical blocks in each pool (paged); bounds for block ids    */
+  int64_t max_len;             /* upper bound of seq_lens; contiguous: row stride in tokens     */
+  const int32_t* seq_lens;     /* [batch] valid cached tokens per sequence (device)             */
+  int32_t batch;               /* sequences                                                     */
+} lsa_cache;
+
+/* Operation selector for lsa_workspace_size. */
+typedef enum {
+  LSA_OP_SCORES = 0,
+  LSA_OP_TOPK = 1,
+  LSA_OP_ATTN = 2,
+  LSA_OP_DECODE_STEP = 3
+} lsa_op;
+
+/* Flags of lsa_decode_step. */
+#define LSA_STEP_UNFUSED 0 /* scan, top-k, attention as separate launches     */
+#define LSA_STEP_FUSED 1   /* reserved for the single-launch step; see below  */
+
+/*
+ * Bytes of workspace `op` needs for `rows` query rows whose score rows hold
+ * `max_len` entries (0 on invalid arguments).  For LSA_OP_TOPK, `d` is not
+ * read and may be NULL (the top-k workspace does not depend on k).
+ */
+size_t lsa_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t op);
+
+/*
+ * Lightning-indexer scores for `rows` query rows (step 1).
+ *   row_seq  [rows] device: sequence of each row, or NULL (row r -> sequence r).
+ *   row_pos  [rows] device: causal position of each row (prefill), or NULL
+ *            (decode: all seq_lens[b] positions are visible).
+ *   q_idx    [rows, H_I, d_I] device, act_dtype (bf16 or f32).
+ *   w        [rows, H_I] device fp32.
+ *   scores   [rows, ld] device fp32 out: I(s) for visible s; -inf for masked
+ *            positions (s > p_i) and for s in [seq_len, ld).  ld >= max_len.
+ * Errors: LSA_ERR_INVALID_ARG (NULL pointers, bad dims, ld < max_len),
+ *         LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA.
+ */
+lsa_status lsa_indexer_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows,
+                              const int32_t* row_seq, const int32_t* row_pos,
+                              const void* q_idx, const float* w, float* scores, int64_t ld,
+                              void* ws, size_t ws_bytes, lsa_stream_t stream);
+
+/*
+ * Top-k of each score row (step 2), exact on the fp32 values.
+ *   scores    [rows, ld] device fp32.
+ *   valid_len [rows] device: entries [0, valid_len[r]) take part, or NULL
+ *             (every row has n_cols entries).  valid_len[r] is clamped to n_cols.
+ *   idx       [rows, k] device int32 out: positions of the min(k, #selectable)
+ *             largest entries (ties -> lower position; -0.0 == +0.0; -inf and
+ *             NaN never selected), sorted ascending, padded with -1.
+ * Errors: LSA_ERR_INVALID_ARG, LSA_ERR_WORKSPACE, LSA_ERR_CUDA.
+ */
+lsa_status lsa_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len,
+                    int64_t n_cols, int32_t k, int32_t* idx,
+                    void* ws, size_t ws_bytes, lsa_stream_t stream);
+
+/*
+ * Sparse MQA over selected rows (step 3).
+ *   row_seq [rows] device or NULL (row r -> sequence r).
+ *   q       [rows, H, D] device, act_dtype.
+ *   idx     [rows, d->top_k] device int32: positions (-1 = none; any order).
+ *   out     [rows, H, D_v] device, act_dtype out; rows with no position give 0.
+ *   lse     [rows, H] device fp32 out (natural log; -inf for empty rows), or NULL.
+ * Positions >= the sequence's length are a device error (LSA_ERR_BOUNDS).
+ */
+lsa_status lsa_sparse_attn_decode(const lsa_dims* d, const lsa_cache* c, int32_t rows,
+                                  const int32_t* row_seq, const void* q, const int32_t* idx,
+                                  void* out, float* lse,
+                                  void* ws, size_t ws_bytes, lsa_stream_t stream);
+
+/*
+ * One decode step for every sequence of the cache (rows = c->batch, row b ->
+ * sequence b): scores -> top-k -> sparse attention.
+ *   q_idx [B, H_I, d_I], w [B, H_I] fp32, q [B, H, D]: device inputs.
+ *   out [B, H, D_v], lse [B, H] (or NULL): device outputs.
+ *   idx_out [B, k] device int32 or NULL: the selection, if wanted.
+ *   flags: LSA_STEP_UNFUSED (LSA_STEP_FUSED currently runs the same launches).
+ * Workspace: lsa_workspace_size(d, B, c->max_len, LSA_OP_DECODE_STEP).
+ */
+lsa_status lsa_decode_step(const lsa_dims* d, const lsa_cache* c, const void* q_idx,
+                           const float* w, const void* q, void* out, float* lse,
+                           int32_t* idx_out, int32_t flags,
+                           void* ws, size_t ws_bytes, lsa_stream_t stream);
+
+/*
+ * Copies the workspace status word to *status (an lsa_status value), clears it,
+ * and synchronises `stream`.  Returns LSA_ERR_CUDA if a CUDA call fails.
+ */
+lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream);
+
+/*
+ * Number of kernel launches `op` enqueues for `rows` query rows with score rows
+ * of `max_len` entries (`causal` != 0: prefill rows with positions), assuming
+ * 16-byte aligned buffers.  A planning aid for launch accounting and graph
+ * capture; runtime memsets are not counted.  -1 on invalid arguments.
+ */
+int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t op, int32_t causal);
+
+/* Static description of a status code. */
+const char* lsa_status_string(lsa_status s);
+
+/* LSA_VERSION of the built library. */
+int32_t lsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */

@@ -1,0 +1,325 @@
+// C ABI of liblsa.so (declared in include/lsa.h): argument validation,
+// workspace layout and kernel dispatch.  No allocation, no synchronisation
+// (except lsa_read_device_status).
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "lsa.h"
+
+namespace lsa {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// LSA_FORCE_SIMT=1 routes every call to the CUDA-core kernels (a debugging aid
+// for comparing the two GPU paths); default is the tensor-core path wherever
+// its shape is supported.
+bool force_simt() {
+  const char* e = getenv("LSA_FORCE_SIMT");
+  return e && e[0] == '1';
+}
+
+bool valid_dims(const lsa_dims* d) {
+  if (!d) return false;
+  if (d->n_idx_heads < 1 || d->n_idx_heads > 64) return false;
+  if (d->idx_dim < 8 || d->idx_dim > 256 || d->idx_dim % 8) return false;
+  if (d->n_heads < 1 || d->n_heads > 4096) return false;
+  if (d->qk_dim < 8 || d->qk_dim > 1024 || d->qk_dim % 8) return false;
+  if (d->v_dim < 1 || d->v_dim > d->qk_dim) return false;
+  if (d->top_k < 1 || d->top_k > (1 << 20)) return false;
+  if (d->block_size < 0) return false;
+  if (d->act_dtype != LSA_F32 && d->act_dtype != LSA_BF16) return false;
+  if (d->idx_key_dtype != LSA_F32 && d->idx_key_dtype != LSA_BF16 && d->idx_key_dtype != LSA_FP8_E4M3)
+    return false;
+  if (!(d->softmax_scale == d->softmax_scale)) return false;
+  return true;
+}
+
+bool valid_cache(const lsa_dims* d, const lsa_cache* c, bool need_keys, bool need_kv) {
+  if (!c || !c->seq_lens || c->batch < 0 || c->max_len < 0) return false;
+  if (d->block_size > 0) {
+    if (!c->block_table || c->max_blocks_per_seq < 1 || c->n_blocks < 1) return false;
+    if (static_cast<int64_t>(c->max_blocks_per_seq) * d->block_size < c->max_len) return false;
+  }
+  if (need_keys) {
+    if (!c->idx_keys || !aligned16(c->idx_keys)) return false;
+    if (d->idx_key_dtype == LSA_FP8_E4M3 && !c->idx_key_scales) return false;
+  }
+  if (need_kv && (!c->kv || !aligned16(c->kv))) return false;
+  return true;
+}
+
+CacheView view(const lsa_dims* d, const lsa_cache* c) {
+  CacheView v;
+  v.idx_keys = c->idx_keys;
+  v.idx_key_scales = c->idx_key_scales;
+  v.kv = c->kv;
+  v.block_table = c->block_table;
+  v.max_blocks = c->max_blocks_per_seq;
+  v.n_blocks = d->block_size > 0 ? c->n_blocks : 0;
+  v.max_len = c->max_len;
+  v.seq_lens = c->seq_lens;
+  v.batch = c->batch;
+  v.block_size = d->block_size;
+  return v;
+}
+
+size_t scores_ws(int32_t rows, bool causal) { return align_up(scores_tc_ws_bytes(rows, causal)); }
+
+size_t attn_ws(const lsa_dims* d, int32_t rows) {
+  size_t a = attn_simt_ws_bytes(rows, d->n_heads, d->v_dim, d->top_k);
+  size_t b = attn_tc_ws_bytes(rows, d->n_heads, d->qk_dim, d->v_dim, d->top_k);
+  return align_up(a > b ? a : b);
+}
+
+inline int64_t score_ld(int64_t max_len) { return (max_len + 3) / 4 * 4; }
+
+struct StepLayout {
+  size_t scores_off, idx_off, inner_off, total;
+};
+
+StepLayout step_layout(const lsa_dims* d, int32_t rows, int64_t max_len) {
+  StepLayout L;
+  L.scores_off = kStatusBytes;
+  L.idx_off = L.scores_off + align_up(static_cast<size_t>(rows) * score_ld(max_len) * 4);
+  L.inner_off = L.idx_off + align_up(static_cast<size_t>(rows) * d->top_k * 4);
+  size_t inner = topk_ws_bytes(rows, max_len);
+  size_t a = attn_ws(d, rows);
+  size_t s = scores_ws(rows, false);
+  if (a > inner) inner = a;
+  if (s > inner) inner = s;
+  L.total = L.inner_off + align_up(inner);
+  return L;
+}
+
+lsa_status ws_check(void* ws, size_t have, size_t need) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LSA_ERR_WORKSPACE;
+  if (have < need) return LSA_ERR_WORKSPACE;
+  return LSA_OK;
+}
+
+inline lsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA; }
+
+inline DevStatus* status_of(void* ws) { return reinterpret_cast<DevStatus*>(ws); }
+
+lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
+                     const int32_t* row_pos, const void* q_idx, const float* w, float* scores,
+                     int64_t ld, void* ws, void* inner_ws, size_t inner_bytes, cudaStream_t s) {
+  ScoresArgs a;
+  a.cache = view(d, c);
+  a.key_dtype = d->idx_key_dtype;
+  a.q_dtype = d->act_dtype;
+  a.H = d->n_idx_heads;
+  a.dI = d->idx_dim;
+  a.rows = rows;
+  a.row_seq = row_seq;
+  a.row_pos = row_pos;
+  a.q_idx = q_idx;
+  a.w = w;
+  a.scores = scores;
+  a.ld = ld;
+  a.status = status_of(ws);
+  a.plan_ws = inner_ws;
+  a.plan_bytes = inner_bytes;
+  if (rows == 0 || ld == 0) return LSA_OK;
+  if (!force_simt() && scores_tc_supported(a)) return cuda_status(launch_scores_tc(a, s));
+  return cuda_status(launch_scores_simt(a, s));
+}
+
+lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
+                   int32_t k, int32_t* idx, void* ws, void* inner_ws, cudaStream_t s) {
+  TopkArgs a;
+  a.scores = scores;
+  a.ld = ld;
+  a.rows = rows;
+  a.valid_len = valid_len;
+  a.n_cols = n_cols;
+  a.k = k;
+  a.idx = idx;
+  a.ws = inner_ws;
+  a.status = status_of(ws);
+  return cuda_status(launch_topk(a, s));
+}
+
+lsa_status do_attn(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq, const void* q,
+                   const int32_t* idx, void* out, float* lse, void* ws, void* inner_ws, size_t inner_bytes,
+                   cudaStream_t s) {
+  AttnArgs a;
+  a.cache = view(d, c);
+  a.dtype = d->act_dtype;
+  a.rows = rows;
+  a.row_seq = row_seq;
+  a.q = q;
+  a.idx = idx;
+  a.k = d->top_k;
+  a.H = d->n_heads;
+  a.D = d->qk_dim;
+  a.Dv = d->v_dim;
+  a.scale = d->softmax_scale;
+  a.out = out;
+  a.lse = lse;
+  a.ws = inner_ws;
+  a.ws_bytes = inner_bytes;
+  a.status = status_of(ws);
+  if (rows == 0) return LSA_OK;
+  if (!force_simt() && attn_tc_supported(a)) return cuda_status(launch_attn_tc(a, s));
+  return cuda_status(launch_attn_simt(a, s));
+}
+
+}  // namespace
+}  // namespace lsa
+
+using namespace lsa;
+
+extern "C" {
+
+size_t lsa_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t op) {
+  if (rows < 0 || max_len < 0) return 0;
+  switch (op) {
+    case LSA_OP_SCORES:
+      if (!valid_dims(d)) return 0;
+      return kStatusBytes + scores_ws(rows, true);
+    case LSA_OP_TOPK:
+      return kStatusBytes + align_up(topk_ws_bytes(rows, max_len));
+    case LSA_OP_ATTN:
+      if (!valid_dims(d)) return 0;
+      return kStatusBytes + attn_ws(d, rows);
+    case LSA_OP_DECODE_STEP:
+      if (!valid_dims(d)) return 0;
+      return step_layout(d, rows, max_len).total;
+    default:
+      return 0;
+  }
+}
+
+lsa_status lsa_indexer_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
+                              const int32_t* row_pos, const void* q_idx, const float* w, float* scores,
+                              int64_t ld, void* ws, size_t ws_bytes, lsa_stream_t stream) {
+  if (!valid_dims(d) || !valid_cache(d, c, true, false)) return LSA_ERR_INVALID_ARG;
+  if (rows < 0 || ld < c->max_len) return LSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!q_idx || !w || !scores || !aligned16(q_idx))) return LSA_ERR_INVALID_ARG;
+  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
+  if (!row_seq && rows > c->batch) return LSA_ERR_INVALID_ARG;
+  const size_t need = kStatusBytes + scores_ws(rows, row_pos != nullptr);
+  lsa_status st = ws_check(ws, ws_bytes, need);
+  if (st != LSA_OK) return st;
+  return do_scores(d, c, rows, row_seq, row_pos, q_idx, w, scores, ld, ws,
+                   static_cast<uint8_t*>(ws) + kStatusBytes, ws_bytes - kStatusBytes,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+lsa_status lsa_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
+                    int32_t k, int32_t* idx, void* ws, size_t ws_bytes, lsa_stream_t stream) {
+  if (rows < 0 || k < 1 || n_cols < 0 || ld < n_cols || (ld % 4) != 0) return LSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!scores || !idx || !aligned16(scores))) return LSA_ERR_INVALID_ARG;
+  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
+  if (n_cols > (1LL << 31) - 1) return LSA_ERR_UNSUPPORTED;
+  const size_t need = kStatusBytes + align_up(topk_ws_bytes(rows, n_cols));
+  lsa_status st = ws_check(ws, ws_bytes, need);
+  if (st != LSA_OK) return st;
+  if (rows == 0) return LSA_OK;
+  return do_topk(scores, ld, rows, valid_len, n_cols, k, idx, ws, static_cast<uint8_t*>(ws) + kStatusBytes,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+lsa_status lsa_sparse_attn_decode(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
+                                  const void* q, const int32_t* idx, void* out, float* lse, void* ws,
+                                  size_t ws_bytes, lsa_stream_t stream) {
+  if (!valid_dims(d) || !valid_cache(d, c, false, true)) return LSA_ERR_INVALID_ARG;
+  if (rows < 0) return LSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!q || !idx || !out || !aligned16(q) || !aligned16(out))) return LSA_ERR_INVALID_ARG;
+  if (!row_seq && rows > c->batch) return LSA_ERR_INVALID_ARG;
+  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
+  const size_t need = kStatusBytes + attn_ws(d, rows);
+  lsa_status st = ws_check(ws, ws_bytes, need);
+  if (st != LSA_OK) return st;
+  return do_attn(d, c, rows, row_seq, q, idx, out, lse, ws, static_cast<uint8_t*>(ws) + kStatusBytes,
+                 ws_bytes - kStatusBytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lsa_status lsa_decode_step(const lsa_dims* d, const lsa_cache* c, const void* q_idx, const float* w,
+                           const void* q, void* out, float* lse, int32_t* idx_out, int32_t flags, void* ws,
+                           size_t ws_bytes, lsa_stream_t stream) {
+  if (!valid_dims(d) || !valid_cache(d, c, true, true)) return LSA_ERR_INVALID_ARG;
+  if (flags != LSA_STEP_UNFUSED && flags != LSA_STEP_FUSED) return LSA_ERR_INVALID_ARG;
+  const int32_t B = c->batch;
+  if (B > 0 && (!q_idx || !w || !q || !out || !aligned16(q_idx) || !aligned16(q) || !aligned16(out)))
+    return LSA_ERR_INVALID_ARG;
+  if (B > 65535) return LSA_ERR_UNSUPPORTED;
+  const StepLayout L = step_layout(d, B, c->max_len);
+  lsa_status st = ws_check(ws, ws_bytes, L.total);
+  if (st != LSA_OK) return st;
+  if (B == 0) return LSA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* scores = reinterpret_cast<float*>(base + L.scores_off);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + L.idx_off);
+  void* inner = base + L.inner_off;
+  const size_t inner_bytes = L.total - L.inner_off;
+  const int64_t ld = score_ld(c->max_len);
+  st = do_scores(d, c, B, nullptr, nullptr, q_idx, w, scores, ld, ws, inner, inner_bytes, s);
+  if (st != LSA_OK) return st;
+  st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, s);
+  if (st != LSA_OK) return st;
+  return do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s);
+}
+
+lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream) {
+  if (!ws || !status) return LSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DevStatus h;
+  if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return LSA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(h), s) != cudaSuccess) return LSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LSA_ERR_CUDA;
+  *status = h.code;
+  return LSA_OK;
+}
+
+int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t op, int32_t causal) {
+  if (rows < 0 || max_len < 0) return -1;
+  if (op != LSA_OP_TOPK && !valid_dims(d)) return -1;
+  if (rows == 0) return 0;
+  const bool simt = force_simt();
+  int scan = 1;
+  int attn = 0;
+  if (op != LSA_OP_TOPK) {
+    if (!simt && scores_tc_shape_ok(d->idx_key_dtype, d->act_dtype, d->n_idx_heads, d->idx_dim, d->block_size))
+      scan = scores_tc_launches(causal != 0);
+    if (!simt && attn_tc_shape_ok(d->act_dtype, d->n_heads, d->qk_dim, d->v_dim, d->block_size))
+      attn = attn_tc_launches(rows, d->n_heads, d->top_k);
+    else
+      attn = attn_simt_launches(rows, d->n_heads, d->top_k);
+  }
+  switch (op) {
+    case LSA_OP_SCORES: return scan;
+    case LSA_OP_TOPK: return kTopkLaunches;
+    case LSA_OP_ATTN: return attn;
+    case LSA_OP_DECODE_STEP: return scan + kTopkLaunches + attn;
+    default: return -1;
+  }
+}
+
+const char* lsa_status_string(lsa_status s) {
+  switch (s) {
+    case LSA_OK: return "ok";
+    case LSA_ERR_INVALID_ARG: return "invalid argument";
+    case LSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case LSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case LSA_ERR_CUDA: return "CUDA runtime error";
+    case LSA_ERR_TIMEOUT: return "device wait timed out";
+    case LSA_ERR_BOUNDS: return "device index out of bounds";
+    default: return "unknown status";
+  }
+}
+
+int32_t lsa_version(void) { return LSA_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,106 @@
+// Internal launch interface between the C-ABI layer (abi.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lsa.h"
+
+namespace lsa {
+
+struct DevStatus;
+
+// Planning constant: B200 has 148 SMs.  Workspace sizes depend on launch plans,
+// so plans use this fixed count (not a device query) to stay host-computable.
+constexpr int kPlanSMs = 148;
+
+struct CacheView {
+  const void* idx_keys;
+  const float* idx_key_scales;
+  const void* kv;
+  const int32_t* block_table;
+  int32_t max_blocks;
+  int64_t n_blocks;
+  int64_t max_len;
+  const int32_t* seq_lens;
+  int32_t batch;
+  int32_t block_size;
+};
+
+struct ScoresArgs {
+  CacheView cache;
+  int32_t key_dtype, q_dtype;
+  int32_t H, dI;
+  int32_t rows;
+  const int32_t* row_seq;
+  const int32_t* row_pos;
+  const void* q_idx;
+  const float* w;
+  float* scores;
+  int64_t ld;
+  DevStatus* status;
+  void* plan_ws;       // tensor-core path scratch (row groups), may be null
+  size_t plan_bytes;
+};
+
+// ---- indexer
+cudaError_t launch_scores_simt(const ScoresArgs& a, cudaStream_t s);
+// shape/dtype test of the tensor-core scan (alignment is checked separately)
+bool scores_tc_shape_ok(int32_t key_dtype, int32_t q_dtype, int32_t H, int32_t dI, int32_t block_size);
+int scores_tc_launches(bool causal);
+bool scores_tc_supported(const ScoresArgs& a);
+size_t scores_tc_ws_bytes(int32_t rows, bool causal);
+cudaError_t launch_scores_tc(const ScoresArgs& a, cudaStream_t s);
+
+// ---- top-k
+struct TopkPlan {
+  int32_t nseg;
+  int64_t seg_len;
+};
+TopkPlan topk_plan(int32_t rows, int64_t n_cols);
+size_t topk_ws_bytes(int32_t rows, int64_t n_cols);
+
+struct TopkArgs {
+  const float* scores;
+  int64_t ld;
+  int32_t rows;
+  const int32_t* valid_len;
+  int64_t n_cols;
+  int32_t k;
+  int32_t* idx;
+  void* ws;            // topk_ws_bytes bytes (256-aligned)
+  DevStatus* status;
+};
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+constexpr int kTopkLaunches = 5;
+
+// ---- sparse attention
+struct AttnArgs {
+  CacheView cache;
+  int32_t dtype;
+  int32_t rows;
+  const int32_t* row_seq;
+  const void* q;
+  const int32_t* idx;
+  int32_t k;
+  int32_t H, D, Dv;
+  float scale;
+  void* out;
+  float* lse;
+  void* ws;
+  size_t ws_bytes;
+  DevStatus* status;
+};
+size_t attn_simt_ws_bytes(int32_t rows, int32_t H, int32_t Dv, int32_t k);
+cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
+int attn_simt_launches(int32_t rows, int32_t H, int32_t k);
+bool attn_tc_shape_ok(int32_t dtype, int32_t H, int32_t D, int32_t Dv, int32_t block_size);
+int attn_tc_launches(int32_t rows, int32_t H, int32_t k);
+bool attn_tc_supported(const AttnArgs& a);
+size_t attn_tc_ws_bytes(int32_t rows, int32_t H, int32_t D, int32_t Dv, int32_t k);
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);
+// exact merge of per-split softmax partials (shared by both attention paths)
+cudaError_t launch_lse_merge(const AttnArgs& a, int nsplit, const float* part_o, const float* part_lse,
+                             cudaStream_t s);
+
+}  // namespace lsa

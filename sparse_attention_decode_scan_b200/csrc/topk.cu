@@ -1,0 +1,343 @@
+// Exact top-k of fp32 score rows: three radix-histogram passes (11 + 11 + 10
+// bits of an order-preserving 32-bit key) find the k-th largest key T, then a
+// count pass and an order-preserving compaction write the positions.
+//
+// Keeps the k highest-scoring tokens of each row (MLI abstract, sentence 2):
+//   * -0.0 compares equal to +0.0 (canonicalised before the key transform);
+//   * -inf and NaN are never selected (they map to key 0, which is skipped);
+//   * among equal scores the lower position is kept;
+//   * the output holds min(k, #selectable) positions sorted ascending, then -1.
+//
+// Each row is cut into segments so that long rows with few rows (4 x 512K)
+// still spread over every SM; segments publish histograms and counts through
+// global memory between launches, so no kernel waits on another CTA.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace lsa {
+namespace {
+
+constexpr int kT = 256;            // threads per CTA
+constexpr int kRound = kT * 4;     // elements per round (one float4 per thread)
+constexpr int kBins1 = 2048, kBins2 = 2048, kBins3 = 1024;
+constexpr int kHistStride = kBins1 + kBins2 + kBins3;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (!(f == f) || f == -INFINITY) return 0u;  // NaN, -inf: never selectable
+  uint32_t u = __float_as_uint(f);
+  if (f == 0.f) u = 0u;                          // -0.0 -> +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+struct Row {
+  int64_t n;       // valid entries of this row
+  int64_t s0, s1;  // this CTA's segment [s0, s1)
+};
+
+__device__ __forceinline__ Row row_range(const TopkArgs& a, int r, int seg, int64_t seg_len) {
+  int64_t n = a.n_cols;
+  if (a.valid_len) {
+    int64_t v = __ldg(a.valid_len + r);
+    n = v < 0 ? 0 : (v < n ? v : n);
+  }
+  Row x;
+  x.n = n;
+  x.s0 = static_cast<int64_t>(seg) * seg_len;
+  x.s1 = x.s0 + seg_len < n ? x.s0 + seg_len : n;
+  return x;
+}
+
+// Loads the 4 keys of this thread for the round starting at `base` (positions
+// >= n give key 0).  Rows start 16-byte aligned (ld % 4 == 0 is checked on the host).
+__device__ __forceinline__ void load_keys(const float* row, int64_t base, int64_t n, uint32_t (&k)[4]) {
+  const int64_t p = base + threadIdx.x * 4;
+  if (p + 3 < n) {
+    float4 v = __ldg(reinterpret_cast<const float4*>(row + p));
+    k[0] = order_key(v.x); k[1] = order_key(v.y); k[2] = order_key(v.z); k[3] = order_key(v.w);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) k[j] = (p + j < n) ? order_key(__ldg(row + p + j)) : 0u;
+  }
+}
+
+// Block-wide exclusive prefix sum of v (all threads), total in *total.
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kT / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kT / 32) warp_sums[lane] = w;  // inclusive
+  }
+  __syncthreads();
+  const int before = warp ? warp_sums[warp - 1] : 0;
+  *total = warp_sums[kT / 32 - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// Finds the bin holding the k_rem-th largest key of a histogram (bins ordered
+// by key, so larger bins hold larger keys).  Returns bin (-1 if the histogram
+// holds fewer than k_rem keys) and the rank inside it; *total = sum of bins.
+struct Found {
+  int bin;
+  uint32_t rank;  // 1-based rank of the wanted key among the keys of `bin`
+  uint32_t total;
+};
+
+template <int NB>
+__device__ Found find_bin(const uint32_t* __restrict__ hist, uint32_t k_rem, int* sh) {
+  constexpr int PER = NB / kT;  // bins per thread
+  const int t = threadIdx.x;
+  uint32_t v[PER];
+  uint32_t mine = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    v[i] = __ldcg(hist + t * PER + i);
+    mine += v[i];
+  }
+  // suffix sums: keys held by threads t' > t (higher bins)
+  int tot;
+  int excl = block_excl_scan(static_cast<int>(mine), sh, &tot);
+  uint32_t above = static_cast<uint32_t>(tot) - static_cast<uint32_t>(excl) - mine;
+  __shared__ Found res;
+  if (t == 0) res = Found{-1, 0u, static_cast<uint32_t>(tot)};
+  __syncthreads();
+  if (k_rem > 0 && above < k_rem && k_rem <= above + mine) {
+    uint32_t cum = above;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i) {
+      if (cum + v[i] >= k_rem) {
+        res.bin = t * PER + i;
+        res.rank = k_rem - cum;
+        break;
+      }
+      cum += v[i];
+    }
+  }
+  __syncthreads();
+  Found f = res;
+  __syncthreads();
+  return f;
+}
+
+struct Thresh {
+  bool any;        // at least one key selected
+  uint32_t keff;   // min(k, selectable)
+  uint32_t T;      // key of the k-th selected element (valid for the last stage reached)
+  uint32_t ties;   // how many keys equal to T are selected (final stage only)
+  int b1, b2;
+};
+
+// Recomputes the threshold state from the histograms published so far.
+template <int STAGES>
+__device__ Thresh thresholds(const uint32_t* hist_row, int k, int* sh) {
+  Thresh th{};
+  Found f1 = find_bin<kBins1>(hist_row, 0xffffffffu, sh);  // only for the total
+  uint32_t keff = f1.total < static_cast<uint32_t>(k) ? f1.total : static_cast<uint32_t>(k);
+  th.keff = keff;
+  th.any = keff > 0;
+  if (!th.any) return th;
+  f1 = find_bin<kBins1>(hist_row, keff, sh);
+  th.b1 = f1.bin;
+  if (STAGES == 1) return th;
+  Found f2 = find_bin<kBins2>(hist_row + kBins1, f1.rank, sh);
+  th.b2 = f2.bin;
+  if (STAGES == 2) return th;
+  Found f3 = find_bin<kBins3>(hist_row + kBins1 + kBins2, f2.rank, sh);
+  th.T = (static_cast<uint32_t>(f1.bin) << 21) | (static_cast<uint32_t>(f2.bin) << 10) | static_cast<uint32_t>(f3.bin);
+  th.ties = f3.rank;
+  return th;
+}
+
+// PASS 1: histogram of bits [31:21]; PASS 2: bits [20:10] of keys in bin b1;
+// PASS 3: bits [9:0] of keys with prefix (b1, b2).
+template <int PASS>
+__global__ void __launch_bounds__(kT) k_topk_hist(TopkArgs a, int64_t seg_len) {
+  constexpr int NB = PASS == 3 ? kBins3 : kBins1;
+  __shared__ uint32_t h[NB];
+  __shared__ int sh[kT / 32];
+  const int r = blockIdx.y, seg = blockIdx.x;
+  const Row rr = row_range(a, r, seg, seg_len);
+  if (rr.s0 >= rr.s1) return;
+  uint32_t* hist_row = reinterpret_cast<uint32_t*>(a.ws) + static_cast<int64_t>(r) * kHistStride;
+  uint32_t prefix = 0;
+  if (PASS >= 2) {
+    Thresh th = thresholds<PASS - 1>(hist_row, a.k, sh);
+    if (!th.any) return;
+    prefix = PASS == 2 ? static_cast<uint32_t>(th.b1) : ((static_cast<uint32_t>(th.b1) << 11) | th.b2);
+  }
+  for (int i = threadIdx.x; i < NB; i += kT) h[i] = 0;
+  __syncthreads();
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  for (int64_t base = rr.s0; base < rr.s1; base += kRound) {
+    uint32_t key[4];
+    load_keys(row, base, rr.s1, key);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t x = key[j];
+      if (x == 0u) continue;
+      if (PASS == 1) atomicAdd(&h[x >> 21], 1u);
+      else if (PASS == 2) { if ((x >> 21) == prefix) atomicAdd(&h[(x >> 10) & 2047u], 1u); }
+      else { if ((x >> 10) == prefix) atomicAdd(&h[x & 1023u], 1u); }
+    }
+  }
+  __syncthreads();
+  uint32_t* dst = hist_row + (PASS == 1 ? 0 : PASS == 2 ? kBins1 : kBins1 + kBins2);
+  for (int i = threadIdx.x; i < NB; i += kT)
+    if (h[i]) atomicAdd(dst + i, h[i]);
+}
+
+__device__ __forceinline__ int32_t* seg_counts(const TopkArgs& a, int r, int nseg) {
+  uint8_t* base = reinterpret_cast<uint8_t*>(a.ws) + static_cast<size_t>(a.rows) * kHistStride * 4;
+  return reinterpret_cast<int32_t*>(base) + (static_cast<int64_t>(r) * nseg) * 2;
+}
+
+// PASS 4: per segment, the counts of keys > T and == T.
+__global__ void __launch_bounds__(kT) k_topk_count(TopkArgs a, int64_t seg_len, int nseg) {
+  __shared__ int sh[kT / 32];
+  const int r = blockIdx.y, seg = blockIdx.x;
+  const Row rr = row_range(a, r, seg, seg_len);
+  if (rr.s0 >= rr.s1) return;
+  const uint32_t* hist_row = reinterpret_cast<const uint32_t*>(a.ws) + static_cast<int64_t>(r) * kHistStride;
+  Thresh th = thresholds<3>(hist_row, a.k, sh);
+  if (!th.any) return;
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  int gt = 0, eq = 0;
+  for (int64_t base = rr.s0; base < rr.s1; base += kRound) {
+    uint32_t key[4];
+    load_keys(row, base, rr.s1, key);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      gt += key[j] > th.T;
+      eq += key[j] == th.T;
+    }
+  }
+  int tg, te;
+  block_excl_scan(gt, sh, &tg);
+  block_excl_scan(eq, sh, &te);
+  if (threadIdx.x == 0) {
+    int32_t* c = seg_counts(a, r, nseg) + seg * 2;
+    c[0] = tg;
+    c[1] = te;
+  }
+}
+
+// PASS 5: ordered compaction of the selected positions, and -1 padding.
+__global__ void __launch_bounds__(kT) k_topk_write(TopkArgs a, int64_t seg_len, int nseg) {
+  __shared__ int sh[kT / 32];
+  const int r = blockIdx.y, seg = blockIdx.x;
+  const Row rr = row_range(a, r, seg, seg_len);
+  int32_t* out = a.idx + static_cast<int64_t>(r) * a.k;
+  if (rr.s0 >= rr.s1 && seg != 0) return;
+  const uint32_t* hist_row = reinterpret_cast<const uint32_t*>(a.ws) + static_cast<int64_t>(r) * kHistStride;
+  Thresh th = thresholds<3>(hist_row, a.k, sh);
+  if (seg == 0)
+    for (int i = static_cast<int>(th.keff) + threadIdx.x; i < a.k; i += kT) out[i] = -1;
+  if (!th.any || rr.s0 >= rr.s1) return;
+  // selected before this segment, and ties (== T) seen before it
+  const int32_t* c = seg_counts(a, r, nseg);
+  int sel_before = 0, eq_before = 0;
+  for (int s = threadIdx.x; s < seg; s += kT) {
+    sel_before += c[2 * s];
+    eq_before += c[2 * s + 1];
+  }
+  // Ties (key == T) go to the lowest positions, so the earlier segments took
+  // min(ties, keys == T before this segment) of them.
+  int tsel, teq;
+  block_excl_scan(sel_before, sh, &tsel);  // totals only
+  block_excl_scan(eq_before, sh, &teq);
+  const int ties = static_cast<int>(th.ties);
+  int out_pos = tsel + (teq < ties ? teq : ties);  // positions already written by earlier segments
+  int eq_seen = teq;                              // ties (== T) at lower positions
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  for (int64_t base = rr.s0; base < rr.s1; base += kRound) {
+    uint32_t key[4];
+    load_keys(row, base, rr.s1, key);
+    int my_eq = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) my_eq += key[j] == th.T;
+    int eq_tot;
+    int eq_ex = block_excl_scan(my_eq, sh, &eq_tot);
+    bool sel[4];
+    int my_sel = 0, e = eq_seen + eq_ex;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      bool s = key[j] > th.T;
+      if (key[j] == th.T) {
+        s = e < ties;
+        ++e;
+      }
+      sel[j] = s;
+      my_sel += s;
+    }
+    int sel_tot;
+    int sel_ex = block_excl_scan(my_sel, sh, &sel_tot);
+    int o = out_pos + sel_ex;
+    const int64_t p = base + threadIdx.x * 4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (!sel[j]) continue;
+      if (o < a.k) out[o] = static_cast<int32_t>(p + j);
+      else record_error(a.status, LSA_ERR_BOUNDS, r, o);  // cannot happen if the counts agree
+      ++o;
+    }
+    out_pos += sel_tot;
+    eq_seen += eq_tot;
+  }
+}
+
+}  // namespace
+
+TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
+  TopkPlan p;
+  int64_t target = 4LL * kPlanSMs;
+  int64_t want = rows > 0 ? (target + rows - 1) / rows : 1;
+  int64_t max_seg = (n_cols + 4095) / 4096;
+  if (max_seg < 1) max_seg = 1;
+  int64_t nseg = want < max_seg ? want : max_seg;
+  if (nseg < 1) nseg = 1;
+  int64_t seg_len = (n_cols + nseg - 1) / nseg;
+  seg_len = ((seg_len + kRound - 1) / kRound) * kRound;
+  if (seg_len < kRound) seg_len = kRound;
+  p.seg_len = seg_len;
+  p.nseg = static_cast<int32_t>((n_cols + seg_len - 1) / seg_len);
+  if (p.nseg < 1) p.nseg = 1;
+  return p;
+}
+
+size_t topk_ws_bytes(int32_t rows, int64_t n_cols) {
+  TopkPlan p = topk_plan(rows, n_cols);
+  size_t b = static_cast<size_t>(rows) * kHistStride * 4 + static_cast<size_t>(rows) * p.nseg * 8;
+  return (b + 255) / 256 * 256;
+}
+
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
+  if (a.rows == 0 || a.k == 0) return cudaSuccess;
+  TopkPlan p = topk_plan(a.rows, a.n_cols);
+  size_t hist_bytes = static_cast<size_t>(a.rows) * kHistStride * 4;
+  cudaError_t e = cudaMemsetAsync(a.ws, 0, hist_bytes, s);
+  if (e != cudaSuccess) return e;
+  dim3 grid(static_cast<unsigned>(p.nseg), static_cast<unsigned>(a.rows));
+  k_topk_hist<1><<<grid, kT, 0, s>>>(a, p.seg_len);
+  k_topk_hist<2><<<grid, kT, 0, s>>>(a, p.seg_len);
+  k_topk_hist<3><<<grid, kT, 0, s>>>(a, p.seg_len);
+  k_topk_count<<<grid, kT, 0, s>>>(a, p.seg_len, p.nseg);
+  k_topk_write<<<grid, kT, 0, s>>>(a, p.seg_len, p.nseg);
+  return cudaGetLastError();
+}
+
+}  // namespace lsa

@@ -1,0 +1,161 @@
+"""Thin ctypes binding of liblsa.so (C ABI in include/lsa.h).
+
+Argument marshalling only: torch tensors are passed as raw device pointers with
+the current CUDA stream; every step of the computation runs in the library's
+CUDA kernels.  There is no fallback: if liblsa.so is missing or fails to load,
+importing the binding's entry points raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblsa.so")
+
+LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_TIMEOUT, \
+    LSA_ERR_BOUNDS = range(7)
+LSA_F32, LSA_BF16, LSA_FP8_E4M3 = 0, 1, 2
+LSA_OP_SCORES, LSA_OP_TOPK, LSA_OP_ATTN, LSA_OP_DECODE_STEP = 0, 1, 2, 3
+LSA_STEP_UNFUSED, LSA_STEP_FUSED = 0, 1
+
+DTYPE_CODE = {"f32": LSA_F32, "bf16": LSA_BF16, "fp8": LSA_FP8_E4M3}
+
+
+class LsaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (lsa_status {code})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("n_idx_heads", ctypes.c_int32), ("idx_dim", ctypes.c_int32),
+                ("n_heads", ctypes.c_int32), ("qk_dim", ctypes.c_int32), ("v_dim", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float), ("act_dtype", ctypes.c_int32),
+                ("idx_key_dtype", ctypes.c_int32)]
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [("idx_keys", ctypes.c_void_p), ("idx_key_scales", ctypes.c_void_p),
+                ("kv", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("max_blocks_per_seq", ctypes.c_int32), ("n_blocks", ctypes.c_int64),
+                ("max_len", ctypes.c_int64), ("seq_lens", ctypes.c_void_p), ("batch", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads liblsa.so once; raises if it is absent (no fallback path exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"liblsa.so not built at {LIB_PATH}; run "
+                          "`python -m sparse_attention_decode_scan_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    D, C = ctypes.POINTER(Dims), ctypes.POINTER(Cache)
+    L.lsa_workspace_size.argtypes = [D, i32, i64, i32]
+    L.lsa_workspace_size.restype = sz
+    L.lsa_indexer_scores.argtypes = [D, C, i32, vp, vp, vp, vp, vp, i64, vp, sz, vp]
+    L.lsa_topk.argtypes = [vp, i64, i32, vp, i64, i32, vp, vp, sz, vp]
+    L.lsa_sparse_attn_decode.argtypes = [D, C, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.lsa_decode_step.argtypes = [D, C, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
+    L.lsa_read_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
+    L.lsa_status_string.argtypes = [ctypes.c_int]
+    L.lsa_status_string.restype = ctypes.c_char_p
+    L.lsa_version.restype = i32
+    L.lsa_launch_count.argtypes = [D, i32, i64, i32, i32]
+    L.lsa_launch_count.restype = i32
+    for f in ("lsa_indexer_scores", "lsa_topk", "lsa_sparse_attn_decode", "lsa_decode_step",
+              "lsa_read_device_status"):
+        getattr(L, f).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().lsa_status_string(int(code)).decode()
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check(code: int, where: str, raise_on_error: bool = True) -> int:
+    if code != LSA_OK and raise_on_error:
+        raise LsaError(code, where)
+    return code
+
+
+def workspace_size(dims: Optional[Dims], rows: int, max_len: int, op: int) -> int:
+    return int(lib().lsa_workspace_size(ctypes.byref(dims) if dims is not None else None, rows, max_len, op))
+
+
+def workspace(nbytes: int, device="cuda"):
+    """A zero-filled, 256-byte aligned workspace tensor (torch's allocator aligns to 512 B)."""
+    import torch
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def indexer_scores(dims: Dims, cache: Cache, q_idx, w, scores, ld: int, ws, row_seq=None, row_pos=None,
+                   rows: Optional[int] = None, stream=None, raise_on_error=True) -> int:
+    rows = int(q_idx.shape[0]) if rows is None else rows
+    return _check(lib().lsa_indexer_scores(ctypes.byref(dims), ctypes.byref(cache), rows, _ptr(row_seq),
+                                           _ptr(row_pos), _ptr(q_idx), _ptr(w), _ptr(scores), int(ld),
+                                           _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
+                  "lsa_indexer_scores", raise_on_error)
+
+
+def topk(scores, k: int, idx, ws, valid_len=None, n_cols: Optional[int] = None, ld: Optional[int] = None,
+         rows: Optional[int] = None, stream=None, raise_on_error=True) -> int:
+    rows = int(scores.shape[0]) if rows is None else rows
+    ld = int(scores.stride(0)) if ld is None else ld
+    n_cols = int(scores.shape[1]) if n_cols is None else n_cols
+    return _check(lib().lsa_topk(_ptr(scores), ld, rows, _ptr(valid_len), n_cols, int(k), _ptr(idx), _ptr(ws),
+                                 ws.numel() if ws is not None else 0, _stream(stream)),
+                  "lsa_topk", raise_on_error)
+
+
+def sparse_attn_decode(dims: Dims, cache: Cache, q, idx, out, lse, ws, row_seq=None, rows: Optional[int] = None,
+                       stream=None, raise_on_error=True) -> int:
+    rows = int(q.shape[0]) if rows is None else rows
+    return _check(lib().lsa_sparse_attn_decode(ctypes.byref(dims), ctypes.byref(cache), rows, _ptr(row_seq),
+                                               _ptr(q), _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws),
+                                               ws.numel() if ws is not None else 0, _stream(stream)),
+                  "lsa_sparse_attn_decode", raise_on_error)
+
+
+def decode_step(dims: Dims, cache: Cache, q_idx, w, q, out, lse, ws, idx_out=None, flags: int = LSA_STEP_UNFUSED,
+                stream=None, raise_on_error=True) -> int:
+    return _check(lib().lsa_decode_step(ctypes.byref(dims), ctypes.byref(cache), _ptr(q_idx), _ptr(w), _ptr(q),
+                                        _ptr(out), _ptr(lse), _ptr(idx_out), int(flags), _ptr(ws),
+                                        ws.numel() if ws is not None else 0, _stream(stream)),
+                  "lsa_decode_step", raise_on_error)
+
+
+def read_device_status(ws, stream=None) -> int:
+    st = ctypes.c_int32(0)
+    _check(lib().lsa_read_device_status(_ptr(ws), ctypes.byref(st), _stream(stream)), "lsa_read_device_status")
+    return int(st.value)
+
+
+def launch_count(dims: Optional[Dims], rows: int, max_len: int, op: int, causal: bool = False) -> int:
+    return int(lib().lsa_launch_count(ctypes.byref(dims) if dims is not None else None, rows, max_len, op,
+                                      1 if causal else 0))
+
+
+def version() -> int:
+    return int(lib().lsa_version())

@@ -1,0 +1,84 @@
+"""Sparse MQA on the GPU vs the oracle, given the same index lists."""
+import numpy as np
+import pytest
+
+from oracle import lsa_oracle as O
+from sparse_attention_decode_scan_b200 import synth
+from tests import cases
+from tests.helpers import check_attention
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _run_attn(case, idx_np, top_k=None):
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+    dc = DeviceCase(case, top_k=top_k)
+    s = case.spec
+    rows = dc.rows
+    odt = torch.float32 if s.act_dtype == "f32" else torch.bfloat16
+    out = torch.full((rows, s.n_heads, s.v_dim), 3.0, dtype=odt, device="cuda")
+    lse = torch.full((rows, s.n_heads), 3.0, dtype=torch.float32, device="cuda")
+    idx = torch.from_numpy(np.ascontiguousarray(idx_np, dtype=np.int32)).cuda()
+    ws = lsa.workspace(lsa.workspace_size(dc.dims, rows, dc.max_len, lsa.LSA_OP_ATTN))
+    lsa.sparse_attn_decode(dc.dims, dc.cache, dc.q, idx, out, lse, ws, row_seq=dc.row_seq)
+    torch.cuda.synchronize()
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def _visible(case):
+    return np.array([O.row_visible(case, r) for r in range(case.rows)])
+
+
+@pytest.mark.parametrize("path", ["default", "simt"])
+@pytest.mark.parametrize("name", ["tiny_fp32", "bf16_L5000", "paged_B5", "prefill_3000x256", "len1"])
+def test_attention_on_given_indices(name, path, monkeypatch):
+    if path == "simt":
+        monkeypatch.setenv("LSA_FORCE_SIMT", "1")
+    case = cases.small(name)
+    k = case.spec.top_k
+    idx = synth.index_lists(case.rows, k, _visible(case), 600 + k)
+    rows = range(case.rows) if case.rows <= 8 else [0, 1, 100, case.rows - 1]
+    out, lse = _run_attn(case, idx)
+    for r in rows:
+        o_ref, l_ref = O.row_attention(case, r, idx[r])
+        check_attention(out[r], o_ref, lse[r], l_ref, what=f"{name} row {r}")
+
+
+def test_attention_index_order_and_padding_positions():
+    # indices in any order, -1 entries anywhere in the list
+    case = cases.small("paged_B5")
+    k = case.spec.top_k
+    idx = synth.index_lists(case.rows, k, _visible(case), 61)
+    g = np.random.default_rng(62)
+    for r in range(case.rows):
+        g.shuffle(idx[r])
+    out, lse = _run_attn(case, idx)
+    for r in range(case.rows):
+        o_ref, l_ref = O.row_attention(case, r, idx[r])
+        check_attention(out[r], o_ref, lse[r], l_ref, what=f"shuffled row {r}")
+
+
+def test_attention_empty_rows():
+    case = cases.small("paged_B5")
+    idx = np.full((case.rows, case.spec.top_k), -1, np.int32)
+    idx[2, :3] = [0, 5, 9]
+    out, lse = _run_attn(case, idx)
+    for r in range(case.rows):
+        if r == 2:
+            o_ref, l_ref = O.row_attention(case, r, idx[r])
+            check_attention(out[r], o_ref, lse[r], l_ref)
+        else:
+            assert (out[r] == 0).all() and np.isneginf(lse[r]).all()
+
+
+def test_attention_split_invariance():
+    # same selection, different k (pad with -1): the split count changes, the result must not
+    case = cases.small("bf16_L5000")
+    idx = synth.index_lists(1, 2048, _visible(case), 63)
+    out1, lse1 = _run_attn(case, idx)
+    idx_pad = np.concatenate([idx, np.full((1, 2048), -1, np.int32)], axis=1)
+    out2, lse2 = _run_attn(case, idx_pad, top_k=4096)
+    assert np.abs(out1 - out2).max() <= 1e-2 and np.abs(lse1 - lse2).max() <= 1e-4

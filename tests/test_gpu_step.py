@@ -1,0 +1,111 @@
+"""End-to-end decode step (scan -> top-k -> sparse MQA) and the prefill chain vs the oracle."""
+import numpy as np
+import pytest
+
+from oracle import lsa_oracle as O
+from tests import cases
+from tests.helpers import check_attention, check_selection
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _step(dc, flags=0):
+    from sparse_attention_decode_scan_b200 import lsa
+    s = dc.spec
+    B = dc.rows
+    odt = torch.float32 if s.act_dtype == "f32" else torch.bfloat16
+    out = torch.empty((B, s.n_heads, s.v_dim), dtype=odt, device="cuda")
+    lse = torch.empty((B, s.n_heads), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, s.top_k), dtype=torch.int32, device="cuda")
+    ws = lsa.workspace(lsa.workspace_size(dc.dims, B, dc.max_len, lsa.LSA_OP_DECODE_STEP))
+    lsa.decode_step(dc.dims, dc.cache, dc.q_idx, dc.w, dc.q, out, lse, ws, idx_out=idx, flags=flags)
+    torch.cuda.synchronize()
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    return out, lse, idx
+
+
+def _attn_on(dc, idx_np):
+    from sparse_attention_decode_scan_b200 import lsa
+    s = dc.spec
+    B = dc.rows
+    odt = torch.float32 if s.act_dtype == "f32" else torch.bfloat16
+    out = torch.empty((B, s.n_heads, s.v_dim), dtype=odt, device="cuda")
+    lse = torch.empty((B, s.n_heads), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.workspace_size(dc.dims, B, dc.max_len, lsa.LSA_OP_ATTN))
+    lsa.sparse_attn_decode(dc.dims, dc.cache, dc.q, torch.from_numpy(idx_np).cuda(), out, lse, ws,
+                           row_seq=dc.row_seq)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def _check_step(case, rows, flags=0):
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+    dc = DeviceCase(case)
+    out, lse, idx = _step(dc, flags)
+    out_h, lse_h, idx_h = out.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
+    ref_sel = np.stack([O.topk(O.row_scores(case, r), O.row_visible(case, r), case.spec.top_k)
+                        if r in rows else np.full(case.spec.top_k, -1, np.int32) for r in range(case.rows)])
+    # GPU attention on the oracle's selection (same selection on both sides)
+    o_gpu_on_ref, l_gpu_on_ref = _attn_on(dc, ref_sel)
+    ndiff = 0
+    for r in rows:
+        sc = O.row_scores(case, r)
+        ndiff += check_selection(idx_h[r], ref_sel[r], sc, what=f"{case.spec.name} row {r}")
+        o_ref, l_ref = O.row_attention(case, r, ref_sel[r])
+        check_attention(o_gpu_on_ref[r], o_ref, l_gpu_on_ref[r], l_ref, what=f"{case.spec.name} row {r}")
+        if np.array_equal(idx_h[r], ref_sel[r]):
+            check_attention(out_h[r], o_ref, lse_h[r], l_ref, what=f"{case.spec.name} step row {r}")
+    return ndiff
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "bf16_L5000", "paged_B5", "fp8_L6001", "len1"])
+def test_decode_step_small(name):
+    case = cases.small(name)
+    _check_step(case, list(range(case.rows)))
+
+
+def test_decode_step_fused_flag_matches_unfused():
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+    dc = DeviceCase(cases.small("paged_B5"))
+    o1, l1, i1 = _step(dc, 0)
+    o2, l2, i2 = _step(dc, 1)
+    assert torch.equal(i1, i2)
+    assert (o1.float() - o2.float()).abs().max().item() <= 1e-2
+
+
+def test_prefill_chain_small():
+    """Causal scores -> top-k over every row -> attention over each row's selection."""
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+    case = cases.small("prefill_3000x256")
+    dc = DeviceCase(case)
+    R, k = dc.rows, case.spec.top_k
+    L = int(case.seq_lens[0])
+    ld = (dc.max_len + 3) // 4 * 4
+    scores = torch.empty((R, ld), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(max(lsa.workspace_size(dc.dims, R, dc.max_len, op) for op in range(3)))
+    lsa.indexer_scores(dc.dims, dc.cache, dc.q_idx, dc.w, scores, ld, ws, row_seq=dc.row_seq, row_pos=dc.row_pos)
+    idx = torch.empty((R, k), dtype=torch.int32, device="cuda")
+    lsa.topk(scores, k, idx, ws, n_cols=L, ld=ld)
+    torch.cuda.synchronize()
+    idx_h = idx.cpu().numpy()
+    for r in [0, 1, 77, R - 1]:
+        sc = O.row_scores(case, r)
+        ref = O.topk(sc, L, k)
+        check_selection(idx_h[r], ref, sc, what=f"prefill row {r}")
+        assert (idx_h[r][idx_h[r] >= 0] <= case.row_pos[r]).all()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_decode_step_full(cfg):
+    case = cases.full(cfg)
+    rows = sorted({0, case.rows - 1, case.rows // 2})
+    _check_step(case, rows)
+
+
+@pytest.mark.slow
+def test_decode_step_full_fp8():
+    case = cases.full(4)
+    _check_step(case, [0, 3])
