@@ -1,9 +1,638 @@
-// placeholder: tensor-core indexer
+// Lightning-indexer scan on the sm_100a tensor cores (tcgen05 + TMA + TMEM).
+//
+// Before each DSA layer the lightning indexer scores every cached token of the
+// sequence, and at long context this scan is where decode time goes (MLI
+// "Multi-layer Indexer" abstract, sentences 2-3).  Score of token s for a query
+// row: I(s) = sum_h w[h] * ReLU(q[h] . K[s]) over 64 indexer heads of dim 128
+// (DSA lightning indexer, DeepSeek-V3.2-Exp report); FP8 keys carry a per-token
+// scale (the compact indexer keys of the LeanSparse episode page).
+//
+// Mapping: keys are the MMA's M side (128 tokens per tile, one TMEM lane per
+// token) and the query heads its N side, so after the MMA every epilogue thread
+// owns one token with all of its head dot products in TMEM; the ReLU-weighted
+// head reduction then runs in registers.  Decode groups one query row per tile
+// (N = 64); the causal prefill groups 4 rows of one sequence (N = 256), reusing
+// each key tile 4 times.  FP8 keys go straight to kind::f8f6f4 MMAs: the bf16
+// query is split exactly into two e4m3 terms (hi + lo, per-head power-of-two
+// scale folded into w), so N doubles and no key conversion is needed.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0  TMA producer: 64-row boxes of the key cache (block-table gather)
+//   warp 1  MMA issuer (one thread) + TMEM owner
+//   warp 2  query staging: query rows -> swizzled smem operand, weights
+//   warps 3-6 epilogue: TMEM -> registers, ReLU-weighted sum, score stores
+// Every wait is bounded; a timeout records LSA_ERR_TIMEOUT and unwinds.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
+
 namespace lsa {
-bool scores_tc_shape_ok(int32_t, int32_t, int32_t, int32_t, int32_t) { return false; }
+namespace {
+
+constexpr int kHeads = 64;       // indexer heads
+constexpr int kDim = 128;        // indexer head dim
+constexpr int kTile = 128;       // tokens per tile (MMA M, TMEM lanes)
+constexpr int kBoxRows = 64;     // rows per TMA box (one 64-token page or half tile)
+constexpr int kThreads = 224;    // 7 warps
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpQ = 2, kWarpEpi = 3;
+constexpr int kSmemLimit = 232448;
+
+template <int KDT, int QB>
+struct Cfg {
+  static constexpr bool kFp8 = KDT == LSA_FP8_E4M3;
+  static constexpr int kN = (kFp8 ? 2 * kHeads : kHeads) * QB;    // MMA N (columns per accumulator)
+  static constexpr int kKBlocks = kFp8 ? 1 : 2;                    // 128-byte K blocks per row
+  static constexpr int kKBlockBytes = kTile * 128;                 // A: 128 rows x 128 B
+  static constexpr int kTileBytes = kKBlocks * kKBlockBytes;
+  static constexpr int kBoxBytes = kBoxRows * 128;
+  static constexpr int kQKBlockBytes = kN * 128;                   // B: N rows x 128 B per K block
+  static constexpr int kQBytes = kKBlocks * kQKBlockBytes;
+  static constexpr int kNQ = QB == 1 ? 2 : 1;                      // query operand buffers
+  static constexpr int kWBytes = QB * kHeads * 4;
+  static constexpr int kFixed = kNQ * kQBytes + kNQ * kWBytes + 1024 /*barriers, scratch*/ + 1024 /*align*/;
+  static constexpr int kNSmax = (kSmemLimit - kFixed) / kTileBytes;
+  static constexpr int kNS = kNSmax > 8 ? 8 : kNSmax;              // key stages
+  static constexpr int kAccCols = kN;
+  static constexpr int kTmemCols = 2 * kN <= 32 ? 32 : 2 * kN <= 64 ? 64 : 2 * kN <= 128 ? 128
+                                   : 2 * kN <= 256 ? 256 : 512;
+  static constexpr int kSmemBytes = kNS * kTileBytes + kFixed;
+  static constexpr uint32_t kIdesc = tc::idesc(kFp8 ? tc::kFmtE4M3 : tc::kFmtBF16,
+                                               kFp8 ? tc::kFmtE4M3 : tc::kFmtBF16, kTile, kN);
+  static_assert(kNS >= 3, "too few key stages");
+  static_assert(2 * kN <= 512, "accumulators exceed TMEM");
+  static_assert(kSmemBytes <= kSmemLimit, "shared memory");
+};
+
+// ---------------------------------------------------------------- work items
+
+__device__ __forceinline__ int seq_of(const ScoresArgs& a, int r) { return a.row_seq ? __ldg(a.row_seq + r) : r; }
+
+// Visible positions of query row r (0 for an invalid row).
+__device__ __forceinline__ int64_t row_visible(const ScoresArgs& a, int r, int* b_out) {
+  const int b = seq_of(a, r);
+  *b_out = b;
+  if (b < 0 || b >= a.cache.batch) return 0;
+  int64_t L = __ldg(a.cache.seq_lens + b);
+  L = L < 0 ? 0 : (L > a.cache.max_len ? a.cache.max_len : L);
+  if (a.row_pos) {
+    int64_t p = static_cast<int64_t>(__ldg(a.row_pos + r)) + 1;
+    p = p < 0 ? 0 : p;
+    L = p < L ? p : L;
+  }
+  return L;
+}
+
+// A group is a run of up to QB consecutive query rows of one sequence that
+// does not cross a multiple of QB; its rows share every key tile.
+template <int QB>
+__device__ __forceinline__ bool is_leader(const ScoresArgs& a, int r) {
+  if (QB == 1 || r % QB == 0) return true;
+  return seq_of(a, r) != seq_of(a, r - 1);
+}
+
+struct Group {
+  int r0, nrows, b, tiles;
+  int64_t vis;  // max visible positions over the group's rows
+};
+
+template <int QB>
+__device__ Group group_at(const ScoresArgs& a, int r0) {
+  Group g;
+  g.r0 = r0;
+  int b;
+  int64_t vis = row_visible(a, r0, &b);
+  g.b = b;
+  int n = 1;
+  if (QB > 1) {
+    while (n < QB && r0 + n < a.rows && ((r0 + n) % QB) != 0 && seq_of(a, r0 + n) == b) {
+      int bb;
+      int64_t v = row_visible(a, r0 + n, &bb);
+      vis = v > vis ? v : vis;
+      ++n;
+    }
+  }
+  g.nrows = n;
+  g.vis = vis;
+  g.tiles = static_cast<int>((vis + kTile - 1) / kTile);
+  return g;
+}
+
+// Walks the CTA's items (group, tile) in global order, skipping empty groups.
+template <int QB>
+struct Walker {
+  Group g;
+  int j;
+  __device__ void start(const ScoresArgs& a, int r0, int j0) {
+    g = group_at<QB>(a, r0);
+    j = j0;
+  }
+  __device__ void next(const ScoresArgs& a) {
+    if (++j < g.tiles) return;
+    j = 0;
+    int r = g.r0 + g.nrows;
+    while (r < a.rows) {
+      g = group_at<QB>(a, r);
+      if (g.tiles > 0) return;
+      r += g.nrows;
+    }
+    g.tiles = 0;  // past the end
+  }
+};
+
+__device__ __forceinline__ int block_sum_i64_scan(int64_t v, int64_t* warp_buf, int64_t* incl, int64_t* total) {
+  // inclusive scan over the block (kThreads threads), returns nothing; used by the planner
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_buf[warp] = x;
+  __syncthreads();
+  int64_t before = 0, tot = 0;
+  for (int w = 0; w < kThreads / 32; ++w) {
+    if (w < warp) before += warp_buf[w];
+    tot += warp_buf[w];
+  }
+  *incl = before + x;
+  *total = tot;
+  __syncthreads();
+  return 0;
+}
+
+struct Plan {
+  int r_first;  // leader row of the CTA's first item
+  int j_first;
+  int64_t n_items;
+};
+
+// Every thread of the CTA takes part: total tiles, this CTA's share, and the
+// group holding its first tile.
+template <int QB>
+__device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
+  int64_t total = 0;
+  for (int base = 0; base < a.rows; base += kThreads) {
+    const int r = base + threadIdx.x;
+    int64_t t = 0;
+    if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
+    int64_t incl, tot;
+    block_sum_i64_scan(t, sbuf, &incl, &tot);
+    total += tot;
+  }
+  Plan p;
+  const int64_t t0 = total * blockIdx.x / gridDim.x;
+  const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
+  p.n_items = t1 - t0;
+  p.r_first = 0;
+  p.j_first = 0;
+  if (p.n_items <= 0) return p;
+  if (threadIdx.x == 0) sfound[0] = -1;
+  __syncthreads();
+  int64_t acc = 0;
+  for (int base = 0; base < a.rows; base += kThreads) {
+    const int r = base + threadIdx.x;
+    int64_t t = 0;
+    if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
+    int64_t incl, tot;
+    block_sum_i64_scan(t, sbuf, &incl, &tot);
+    const int64_t start = acc + incl - t;
+    if (t > 0 && start <= t0 && t0 < start + t) {
+      sfound[0] = r;
+      sfound[1] = static_cast<int>(t0 - start);
+    }
+    acc += tot;
+    __syncthreads();
+    if (sfound[0] >= 0) break;
+  }
+  p.r_first = sfound[0];
+  p.j_first = sfound[1];
+  return p;
+}
+
+// ---------------------------------------------------------------- query staging
+
+// bf16: B row n = qq * 64 + h holds q[row r0+qq][h][:] in two 128-byte K blocks.
+template <int QB>
+__device__ void stage_query_bf16(const ScoresArgs& a, const Group& g, uint8_t* qbuf, float* wbuf, int lane) {
+  constexpr int N = kHeads * QB;
+  const uint4* src = reinterpret_cast<const uint4*>(a.q_idx);
+  for (int idx = lane; idx < N * (kDim / 8); idx += 32) {
+    const int n = idx >> 4, c = idx & 15;
+    const int qq = n / kHeads, h = n % kHeads;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (qq < g.nrows) v = __ldg(src + ((static_cast<int64_t>(g.r0 + qq) * kHeads + h) * kDim) / 8 + c);
+    const int kb = c >> 3, cc = c & 7;
+    *reinterpret_cast<uint4*>(qbuf + kb * (N * 128) + tc::sw128_offset(n, cc)) = v;
+  }
+  for (int i = lane; i < QB * kHeads; i += 32) {
+    const int qq = i / kHeads;
+    wbuf[i] = qq < g.nrows ? __ldg(a.w + static_cast<int64_t>(g.r0 + qq) * kHeads + (i % kHeads)) : 0.f;
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// fp8: per (query, head) a power-of-two scale s puts max|q| into [224, 448];
+// q*s = hi + lo with hi = e4m3(q*s), lo = e4m3(q*s - hi), exact for bf16 q
+// (4 + 4 significant bits) outside the e4m3 subnormal range.  B row
+// qq*128 + h holds hi, qq*128 + 64 + h holds lo; w' = w / s.
+template <int QB>
+__device__ void stage_query_fp8(const ScoresArgs& a, const Group& g, uint8_t* qbuf, float* wbuf, int lane) {
+  const uint16_t* q = reinterpret_cast<const uint16_t*>(a.q_idx);
+  for (int n = lane; n < QB * kHeads; n += 32) {
+    const int qq = n / kHeads, h = n % kHeads;
+    const bool live = qq < g.nrows;
+    const uint16_t* src = q + (static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + h) * kDim;
+    float mx = 0.f;
+    for (int d = 0; d < kDim; ++d) mx = fmaxf(mx, fabsf(bf16_bits_to_float(__ldg(src + d))));
+    float s = 1.f;
+    if (mx > 0.f) {
+      int e;
+      frexpf(448.f / mx, &e);  // 448/mx = f * 2^e, f in [0.5, 1)
+      s = ldexpf(1.f, e - 1);  // largest power of two <= 448 / mx
+    }
+    const int row_hi = qq * 2 * kHeads + h, row_lo = row_hi + kHeads;
+    for (int c = 0; c < 8; ++c) {  // 16-byte chunks of 16 dims
+      uint32_t hw[4], lw[4];
+      for (int u = 0; u < 4; ++u) {
+        float x[4], hv[4], lv[4];
+        for (int e4 = 0; e4 < 4; ++e4) x[e4] = live ? bf16_bits_to_float(__ldg(src + c * 16 + u * 4 + e4)) * s : 0.f;
+        hw[u] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
+        for (int e4 = 0; e4 < 4; ++e4) {
+          hv[e4] = e4m3_to_float(static_cast<uint8_t>(hw[u] >> (8 * e4)));
+          lv[e4] = x[e4] - hv[e4];
+        }
+        lw[u] = pack_e4m3x4(lv[0], lv[1], lv[2], lv[3]);
+      }
+      *reinterpret_cast<uint4*>(qbuf + tc::sw128_offset(row_hi, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(qbuf + tc::sw128_offset(row_lo, c)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    wbuf[n] = live ? __ldg(a.w + static_cast<int64_t>(g.r0 + qq) * kHeads + h) / s : 0.f;
+  }
+}
+
+// ---------------------------------------------------------------- the kernel
+
+template <int KDT, int QB>
+__global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmap, const ScoresArgs a) {
+  using C = Cfg<KDT, QB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint8_t* qbufs = stages + C::kNS * C::kTileBytes;
+  float* wbufs = reinterpret_cast<float*>(qbufs + C::kNQ * C::kQBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(wbufs) + C::kNQ * C::kWBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = full + C::kNS;
+  uint64_t* qfull = empty + C::kNS;
+  uint64_t* qempty = qfull + C::kNQ;
+  uint64_t* tfull = qempty + C::kNQ;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* sfound = const_cast<int*>(abort_flag) + 1;                       // 2 ints
+  int64_t* sbuf = reinterpret_cast<int64_t*>(sfound + 2 + 1);           // kThreads/32 int64 (8-aligned below)
+  sbuf = reinterpret_cast<int64_t*>((reinterpret_cast<uintptr_t>(sbuf) + 7) & ~uintptr_t(7));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kNS; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < C::kNQ; ++s) {
+      tc::mbar_init(&qfull[s], 1);
+      tc::mbar_init(&qempty[s], 1 + 4);  // MMA commit + 4 epilogue warps
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&tfull[s], 1);
+      tc::mbar_init(&tempty[s], 4);
+    }
+    tc::mbar_init(done, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == kWarpProd && lane == 0) tc::prefetch_tmap(&tmap);
+  if (warp == kWarpMma) {
+    tc::tmem_alloc(tmem_slot, C::kTmemCols);
+    tc::tc_fence_before();
+  }
+  const Plan plan = plan_work<QB>(a, sbuf, sfound);
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  CacheAddr ad{a.cache.block_table, a.cache.max_blocks, a.cache.block_size, a.cache.n_blocks, a.cache.max_len};
+
+  if (warp == kWarpProd) {
+    if (lane == 0 && plan.n_items > 0) {
+      Walker<QB> W;
+      W.start(a, plan.r_first, plan.j_first);
+      int64_t it = 0;
+      for (; it < plan.n_items; ++it) {
+        const int s = static_cast<int>(it % C::kNS);
+        const uint32_t ph = static_cast<uint32_t>((it / C::kNS) & 1);
+        if (!tc::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+          record_error(a.status, LSA_ERR_TIMEOUT, 0, 1);
+          *abort_flag = 1;
+          break;
+        }
+        int64_t rows[2] = {-1, -1};
+        uint32_t bytes = 0;
+        for (int h = 0; h < 2; ++h) {
+          const int64_t p = static_cast<int64_t>(W.j) * kTile + h * kBoxRows;
+          if (p < W.g.vis) {
+            rows[h] = ad.row(W.g.b, p);
+            if (rows[h] >= 0) bytes += C::kKBlocks * C::kBoxBytes;
+            else record_error(a.status, LSA_ERR_BOUNDS, W.g.r0, static_cast<int>(p));
+          }
+        }
+        tc::mbar_arrive_expect_tx(&full[s], bytes);
+        uint8_t* st = stages + s * C::kTileBytes;
+        for (int h = 0; h < 2; ++h) {
+          if (rows[h] < 0) continue;
+          for (int kb = 0; kb < C::kKBlocks; ++kb)
+            tc::tma_load_2d(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * 64,
+                            static_cast<int32_t>(rows[h]), &full[s]);
+        }
+        W.next(a);
+      }
+      // drain: the last load of every stage must land before the CTA exits
+      const int64_t n_issued = it;
+      for (int64_t i = n_issued > C::kNS ? n_issued - C::kNS : 0; i < n_issued; ++i)
+        tc::mbar_wait(&full[i % C::kNS], static_cast<uint32_t>((i / C::kNS) & 1), nullptr);
+    }
+  } else if (warp == kWarpMma) {
+    if (lane == 0 && plan.n_items > 0) {
+      Walker<QB> W;
+      W.start(a, plan.r_first, plan.j_first);
+      int gi = -1;
+      int qi = 0;
+      for (int64_t it = 0; it < plan.n_items; ++it) {
+        if (it == 0 || W.j == 0) {
+          ++gi;
+          qi = gi % C::kNQ;
+          if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) goto mma_fail;
+        }
+        {
+          const int s = static_cast<int>(it % C::kNS);
+          if (!tc::mbar_wait(&full[s], static_cast<uint32_t>((it / C::kNS) & 1), abort_flag)) goto mma_fail;
+          const int acc = static_cast<int>(it & 1);
+          if (!tc::mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag)) goto mma_fail;
+          tc::tc_fence_after();
+          const uint32_t d = tmem_base + acc * C::kAccCols;
+          const uint32_t a_base = tc::smem_u32(stages + s * C::kTileBytes);
+          const uint32_t b_base = tc::smem_u32(qbufs + qi * C::kQBytes);
+#pragma unroll
+          for (int kb = 0; kb < C::kKBlocks; ++kb) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad_ = tc::desc_sw128(a_base + kb * C::kKBlockBytes + k * 32);
+              const uint64_t bd_ = tc::desc_sw128(b_base + kb * C::kQKBlockBytes + k * 32);
+              if (C::kFp8) tc::mma_f8(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
+              else tc::mma_f16(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
+            }
+          }
+          tc::mma_commit(&empty[s]);
+          tc::mma_commit(&tfull[acc]);
+          const int jn = W.j + 1;
+          if (it + 1 == plan.n_items || jn >= W.g.tiles) tc::mma_commit(&qempty[qi]);
+          W.next(a);
+        }
+        continue;
+      mma_fail:
+        record_error(a.status, LSA_ERR_TIMEOUT, 0, 2);
+        *abort_flag = 1;
+        break;
+      }
+      tc::mma_commit(done);
+      tc::mbar_wait(done, 0, nullptr);
+    }
+  } else if (warp == kWarpQ) {
+    if (plan.n_items > 0) {
+      Walker<QB> W;
+      W.start(a, plan.r_first, plan.j_first);
+      int gi = -1;
+      for (int64_t it = 0; it < plan.n_items; ++it) {
+        if (it == 0 || W.j == 0) {
+          ++gi;
+          const int qi = gi % C::kNQ;
+          if (!tc::mbar_wait(&qempty[qi], static_cast<uint32_t>(((gi / C::kNQ) & 1) ^ 1), abort_flag)) {
+            if (lane == 0) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 3);
+              *abort_flag = 1;
+            }
+            break;
+          }
+          uint8_t* qb = qbufs + qi * C::kQBytes;
+          float* wb = wbufs + qi * (C::kWBytes / 4);
+          if (C::kFp8) stage_query_fp8<QB>(a, W.g, qb, wb, lane);
+          else stage_query_bf16<QB>(a, W.g, qb, wb, lane);
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&qfull[qi]);
+        }
+        W.next(a);
+      }
+    }
+  } else {
+    // epilogue: warp (3..6) % 4 selects the TMEM lane quarter = token rows of the tile
+    const int quarter = warp & 3;
+    const int t = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    if (plan.n_items > 0) {
+      Walker<QB> W;
+      W.start(a, plan.r_first, plan.j_first);
+      int gi = -1, qi = 0;
+      int64_t vis_r[QB];
+      for (int64_t it = 0; it < plan.n_items; ++it) {
+        if (it == 0 || W.j == 0) {
+          ++gi;
+          qi = gi % C::kNQ;
+          if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) {
+            if (lane == 0) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 4);
+              *abort_flag = 1;
+            }
+            break;
+          }
+#pragma unroll
+          for (int qq = 0; qq < QB; ++qq) {
+            int bb;
+            vis_r[qq] = qq < W.g.nrows ? row_visible(a, W.g.r0 + qq, &bb) : 0;
+          }
+        }
+        const int acc = static_cast<int>(it & 1);
+        if (!tc::mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1), abort_flag)) {
+          if (lane == 0) {
+            record_error(a.status, LSA_ERR_TIMEOUT, 0, 5);
+            *abort_flag = 1;
+          }
+          break;
+        }
+        tc::tc_fence_after();
+        const int64_t p = static_cast<int64_t>(W.j) * kTile + t;
+        const int64_t prow = p < W.g.vis ? ad.row(W.g.b, p) : -1;
+        float kscale = 1.f;
+        if (C::kFp8 && prow >= 0) kscale = __ldg(a.cache.idx_key_scales + prow);
+        const float* wb = wbufs + qi * (C::kWBytes / 4);
+        float sc[QB];
+#pragma unroll
+        for (int qq = 0; qq < QB; ++qq) {
+          float s = 0.f;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float v[32];
+            const uint32_t col = acc * C::kAccCols + (C::kFp8 ? qq * 2 * kHeads : qq * kHeads) + c * 32;
+            tc::tmem_ld32(tmem_base + lane_base + col, v);
+            if (C::kFp8) {
+              float u[32];
+              tc::tmem_ld32(tmem_base + lane_base + col + kHeads, u);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) s = fmaf(wb[qq * kHeads + c * 32 + i], fmaxf(v[i] + u[i], 0.f), s);
+            } else {
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) s = fmaf(wb[qq * kHeads + c * 32 + i], fmaxf(v[i], 0.f), s);
+            }
+          }
+          sc[qq] = s * kscale;
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+#pragma unroll
+        for (int qq = 0; qq < QB; ++qq) {
+          if (qq < W.g.nrows && p < a.ld) {
+            float o = -INFINITY;
+            if (p < vis_r[qq]) o = prow >= 0 ? sc[qq] : NAN;
+            a.scores[static_cast<int64_t>(W.g.r0 + qq) * a.ld + p] = o;
+          }
+        }
+        const bool last = (it + 1 == plan.n_items) || (W.j + 1 >= W.g.tiles);
+        if (last) {
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&qempty[qi]);
+        }
+        W.next(a);
+      }
+    }
+    // tails: positions past each row's group tiles are -inf (NaN for an invalid row)
+    for (int r = blockIdx.x; r < a.rows; r += gridDim.x) {
+      int r0 = r;
+      while (!is_leader<QB>(a, r0)) --r0;
+      const Group g = group_at<QB>(a, r0);
+      int b;
+      row_visible(a, r, &b);
+      const bool ok = b >= 0 && b < a.cache.batch;
+      if (ok && threadIdx.x == kWarpEpi * 32) {
+        const int L = __ldg(a.cache.seq_lens + b);
+        if (L < 0 || L > a.cache.max_len) record_error(a.status, LSA_ERR_BOUNDS, r, L);
+      } else if (!ok && threadIdx.x == kWarpEpi * 32) {
+        record_error(a.status, LSA_ERR_BOUNDS, r, b);
+      }
+      const float val = ok ? -INFINITY : NAN;
+      const int64_t start = ok ? static_cast<int64_t>(g.tiles) * kTile : 0;
+      float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+      for (int64_t p = start + (threadIdx.x - kWarpEpi * 32); p < a.ld; p += 128) row[p] = val;
+    }
+  }
+
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return kPlanSMs;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return kPlanSMs;
+  return n;
+}
+
+int64_t key_rows(const ScoresArgs& a) {
+  return a.cache.block_size > 0 ? a.cache.n_blocks * a.cache.block_size
+                                : static_cast<int64_t>(a.cache.batch) * a.cache.max_len;
+}
+
+template <int KDT, int QB>
+cudaError_t launch_t(const ScoresArgs& a, cudaStream_t s) {
+  using C = Cfg<KDT, QB>;
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap tmap;
+  const bool fp8 = KDT == LSA_FP8_E4M3;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(key_rows(a))};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDim * (fp8 ? 1 : 2))};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), static_cast<cuuint32_t>(kBoxRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(&tmap, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(a.cache.idx_keys), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  auto kern = k_scan_tc<KDT, QB>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<num_sms(), kThreads, C::kSmemBytes, s>>>(tmap, a);
+  return cudaGetLastError();
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+bool scores_tc_shape_ok(int32_t key_dtype, int32_t q_dtype, int32_t H, int32_t dI, int32_t block_size) {
+  return (key_dtype == LSA_BF16 || key_dtype == LSA_FP8_E4M3) && q_dtype == LSA_BF16 && H == kHeads &&
+         dI == kDim && (block_size == 0 || block_size % kBoxRows == 0);
+}
+
 int scores_tc_launches(bool) { return 1; }
-bool scores_tc_supported(const ScoresArgs&) { return false; }
+
+bool scores_tc_supported(const ScoresArgs& a) {
+  if (!scores_tc_shape_ok(a.key_dtype, a.q_dtype, a.H, a.dI, a.cache.block_size)) return false;
+  if (!aligned16(a.cache.idx_keys) || !aligned16(a.q_idx)) return false;
+  const int64_t kr = key_rows(a);
+  if (kr <= 0 || kr >= (1LL << 31)) return false;
+  if (a.key_dtype == LSA_FP8_E4M3 && !a.cache.idx_key_scales) return false;
+  return true;
+}
+
 size_t scores_tc_ws_bytes(int32_t, bool) { return 0; }
-cudaError_t launch_scores_tc(const ScoresArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+
+cudaError_t launch_scores_tc(const ScoresArgs& a, cudaStream_t s) {
+  const bool causal = a.row_pos != nullptr;
+  if (a.key_dtype == LSA_FP8_E4M3) return causal ? launch_t<LSA_FP8_E4M3, 2>(a, s) : launch_t<LSA_FP8_E4M3, 1>(a, s);
+  return causal ? launch_t<LSA_BF16, 4>(a, s) : launch_t<LSA_BF16, 1>(a, s);
+}
+
 }  // namespace lsa
