@@ -284,6 +284,14 @@ def run_ours(args, world, rank, local):
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
     with ClockSampler(gpu_index) as clk:
+        # keep the GPU under the same load for ~1 s before the timed steps so the
+        # clock sampler (100 ms period) sees the loaded state of this workload
+        t_soak = time.perf_counter()
+        while time.perf_counter() - t_soak < 1.0:
+            step()
+            if flush is not None:
+                flush.zero_()
+            torch.cuda.synchronize(dev)
         barrier()
         torch.cuda.synchronize(dev)
         t_start = torch.cuda.Event(enable_timing=True)
