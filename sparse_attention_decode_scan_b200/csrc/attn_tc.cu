@@ -1,9 +1,484 @@
-// placeholder: tensor-core sparse attention
+// Sparse MQA decode on the sm_100a tensor cores (tcgen05 + TMEM), gathering
+// the selected KV rows through the block table.
+//
+// The layer attends only the k tokens the lightning indexer kept (MLI abstract,
+// sentence 2): o[h] = softmax_j(scale * q[h] . KV[idx_j]) . KV[idx_j][:512]
+// over 128 query heads sharing 576-wide bf16 KV rows (value = first 512
+// columns), plus lse[h].  Sparse attention reads only the kept rows (LeanSparse
+// episode page: it reduces reads, not storage).
+//
+// Layout of the work: one CTA per (query row, half of the heads, split of the
+// index list).  64 heads make the MMA's M side (M = 64), so the fp32 output
+// accumulator O[64 x 512] takes half of the TMEM lanes: dims 0-255 at lane
+// offset 0 and dims 256-511 at lane offset 16, columns 0-255; the two score
+// buffers S[64 x 64] sit at lane offset 0, columns 256-383.  Each softmax warp
+// then holds, for its 16 heads, the scores in lanes 0-15 and both output halves
+// in lanes 0-31, so a rescale touches only output columns.
+//   warps 0-3  producer: cp.async gathers of 64 selected rows per chunk into the
+//              128-byte-swizzled operand layout (zero rows for -1 / bad entries)
+//   warp 4     MMA issuer: S = Q K^T (36 x M64N64K16), O += P V (8 x M64N256K16)
+//   warps 5-8  online softmax (base 2, lazy rescale when the max grows by > 8),
+//              P to shared memory, final normalisation and stores
+// Splits write normalised partials and lse; the shared merge kernel combines them.
+#include <math.h>
+
+#include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
+
 namespace lsa {
-bool attn_tc_shape_ok(int32_t, int32_t, int32_t, int32_t, int32_t) { return false; }
-int attn_tc_launches(int32_t, int32_t, int32_t) { return 2; }
-bool attn_tc_supported(const AttnArgs&) { return false; }
-size_t attn_tc_ws_bytes(int32_t, int32_t, int32_t, int32_t, int32_t) { return 0; }
-cudaError_t launch_attn_tc(const AttnArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kHeadsAll = 128;
+constexpr int kHeadsCta = 64;
+constexpr int kD = 576;
+constexpr int kDv = 512;
+constexpr int kChunk = 64;                 // KV rows per chunk
+constexpr int kBoxes = kD / 64;            // 9 column blocks of 64 dims
+constexpr int kBoxBytes = kChunk * 128;    // 64 rows x 128 B
+constexpr int kKvBytes = kBoxes * kBoxBytes;          // 73728
+constexpr int kQBytes = kBoxes * kHeadsCta * 128;     // 73728
+constexpr int kPBytes = kHeadsCta * 128;              // 8192
+constexpr int kThreads = 288;
+constexpr int kProdThreads = 128;
+constexpr int kWarpMma = 4;  // warps 5-8: softmax
+constexpr int kSmemBytes = kQBytes + 2 * kKvBytes + kPBytes + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 256;            // score buffers start column
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.f;        // lazy rescale threshold (factor 256)
+
+// idesc with B major = MN (bit 16)
+constexpr uint32_t kIdescQK = tc::idesc(tc::kFmtBF16, tc::kFmtBF16, 64, kChunk);
+constexpr uint32_t kIdescPV = tc::idesc(tc::kFmtBF16, tc::kFmtBF16, 64, 256) | (1u << 16);
+
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+struct TcAttnParams {
+  AttnArgs a;
+  int nsplit;
+  int split_len;  // multiple of kChunk
+  float* part_o;
+  float* part_lse;
+};
+
+// MN-major operand in the 128-byte swizzle layout: 64-element MN blocks `lbo`
+// bytes apart, 8-row K groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t addr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+struct RowCtx {
+  int b;
+  int64_t L;
+  bool ok;
+};
+
+__device__ __forceinline__ RowCtx row_ctx(const AttnArgs& a, int r) {
+  RowCtx c;
+  c.b = a.row_seq ? __ldg(a.row_seq + r) : r;
+  c.ok = c.b >= 0 && c.b < a.cache.batch;
+  c.L = c.ok ? __ldg(a.cache.seq_lens + c.b) : 0;
+  if (c.L < 0) c.L = 0;
+  if (c.L > a.cache.max_len) c.L = a.cache.max_len;
+  return c;
+}
+
+// Stored KV row of list entry j of row r, or -1 (padding, out of range, bad block).
+__device__ __forceinline__ int64_t entry_row(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r, int j,
+                                             int j1, bool report) {
+  if (j >= j1 || !rc.ok) return -1;
+  const int32_t pos = __ldg(a.idx + static_cast<int64_t>(r) * a.k + j);
+  if (pos < 0) return -1;
+  const int64_t row = pos < rc.L ? ad.row(rc.b, pos) : -1;
+  if (row < 0 && report) record_error(a.status, LSA_ERR_BOUNDS, r, pos);
+  return row;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
+  const AttnArgs& a = P.a;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* qs = smem;
+  uint8_t* kvs = qs + kQBytes;         // 2 chunk buffers
+  uint8_t* ps = kvs + 2 * kKvBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + kPBytes);
+  uint64_t* qfull = bars;
+  uint64_t* kvfull = bars + 1;    // [2]
+  uint64_t* kvempty = bars + 3;   // [2]
+  uint64_t* sfull = bars + 5;     // [2]
+  uint64_t* sempty = bars + 7;    // [2]
+  uint64_t* pfull = bars + 9;
+  uint64_t* pvdone = bars + 10;
+  uint64_t* done = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int split = blockIdx.x, half = blockIdx.y, r = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = split * P.split_len;
+  const int j1 = min(a.k, j0 + P.split_len);
+  const int nch = j1 > j0 ? (j1 - j0 + kChunk - 1) / kChunk : 0;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(qfull, kProdThreads);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&kvfull[i], kProdThreads);
+      tc::mbar_init(&kvempty[i], 1);
+      tc::mbar_init(&sfull[i], 1);
+      tc::mbar_init(&sempty[i], 4);
+    }
+    tc::mbar_init(pfull, 4);
+    tc::mbar_init(pvdone, 1);
+    tc::mbar_init(done, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tc::tmem_alloc(tmem_slot, kTmemCols);
+    tc::tc_fence_before();
+  }
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const RowCtx rc = row_ctx(a, r);
+  CacheAddr ad{a.cache.block_table, a.cache.max_blocks, a.cache.block_size, a.cache.n_blocks, a.cache.max_len};
+  if (!rc.ok && threadIdx.x == 0 && split == 0 && half == 0) record_error(a.status, LSA_ERR_BOUNDS, r, rc.b);
+
+  if (warp < 4) {
+    // ---------------------------------------------------------------- producer
+    const int t = threadIdx.x;
+    const int sub = t & 7;         // 16-byte column chunk within each 128-byte block
+    const int rbase = t >> 3;      // 0..15
+    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q) +
+                          (static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta) * kD * 2;
+    const uint32_t qs_u = tc::smem_u32(qs);
+    for (int m = 0; m < 4; ++m) {
+      const int i = rbase + 16 * m;
+      const uint8_t* src = qsrc + static_cast<int64_t>(i) * kD * 2;
+      for (int d = 0; d < kBoxes; ++d)
+        cp_async16(qs_u + d * (kHeadsCta * 128) + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
+    }
+    cp_async_arrive_noinc(qfull);
+    for (int j = 0; j < nch; ++j) {
+      const int b = j & 1;
+      if (!tc::mbar_wait(&kvempty[b], ((j >> 1) & 1) ^ 1, abort_flag)) {
+        if (t == 0) {
+          record_error(a.status, LSA_ERR_TIMEOUT, r, 10);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      const uint32_t kv_u = tc::smem_u32(kvs + b * kKvBytes);
+      bool zeroed = false;
+      for (int m = 0; m < 4; ++m) {
+        const int i = rbase + 16 * m;
+        const int64_t row = entry_row(a, ad, rc, r, j0 + j * kChunk + i, j1, sub == 0 && half == 0);
+        if (row >= 0) {
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cache.kv) + row * (kD * 2);
+          for (int d = 0; d < kBoxes; ++d) cp_async16(kv_u + d * kBoxBytes + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
+        } else {
+          for (int d = 0; d < kBoxes; ++d)
+            *reinterpret_cast<uint4*>(kvs + b * kKvBytes + d * kBoxBytes + tc::sw128_offset(i, sub)) =
+                make_uint4(0, 0, 0, 0);
+          zeroed = true;
+        }
+      }
+      if (zeroed) tc::fence_proxy_async_smem();
+      cp_async_arrive_noinc(&kvfull[b]);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == kWarpMma) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && nch > 0) {
+      const uint32_t q_u = tc::smem_u32(qs);
+      const uint32_t p_u = tc::smem_u32(ps);
+      bool ok = tc::mbar_wait(qfull, 0, abort_flag);
+      tc::fence_proxy_async_smem();
+      auto issue_pv = [&](int i) -> bool {
+        if (!tc::mbar_wait(pfull, i & 1, abort_flag)) return false;
+        tc::tc_fence_after();
+        const uint32_t kv_u = tc::smem_u32(kvs + (i & 1) * kKvBytes);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t d = tmem + (static_cast<uint32_t>(16 * c) << 16);  // dims 256c.. at lane offset 16c
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad_ = tc::desc_sw128(p_u + kk * 32);
+            const uint64_t bd_ = desc_sw128_mn(kv_u + (4 * c) * kBoxBytes + kk * 2048, kBoxBytes);
+            tc::mma_f16(d, ad_, bd_, kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc::mma_commit(pvdone);
+        tc::mma_commit(&kvempty[i & 1]);
+        return true;
+      };
+      for (int j = 0; ok && j < nch; ++j) {
+        const int b = j & 1;
+        if (!tc::mbar_wait(&kvfull[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc::fence_proxy_async_smem();
+        if (!tc::mbar_wait(&sempty[b], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint32_t kv_u = tc::smem_u32(kvs + b * kKvBytes);
+        const uint32_t d = tmem + kColS + b * kChunk;
+#pragma unroll 1
+        for (int blk = 0; blk < kBoxes; ++blk) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad_ = tc::desc_sw128(q_u + blk * (kHeadsCta * 128) + k * 32);
+            const uint64_t bd_ = tc::desc_sw128(kv_u + blk * kBoxBytes + k * 32);
+            tc::mma_f16(d, ad_, bd_, kIdescQK, (blk | k) != 0);
+          }
+        }
+        tc::mma_commit(&sfull[b]);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) ok = issue_pv(nch - 1);
+      if (!ok) {
+        record_error(a.status, LSA_ERR_TIMEOUT, r, 11);
+        *abort_flag = 1;
+      }
+      // every MMA issued must finish before TMEM is released
+      tc::mma_commit(done);
+      tc::mbar_wait(done, 0, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax / epilogue
+    const int quarter = warp & 3;                       // TMEM lanes 32q .. 32q+31
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool srow = lane < 16;                        // lanes holding a score row
+    const int head_local = quarter * 16 + (lane & 15);  // 0..63
+    const float c2 = a.scale * kLog2e;
+    float m_run = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nch; ++j) {
+      const int b = j & 1;
+      // validity of the 64 rows of this chunk (recomputed; same rule as the producer)
+      const bool v0 = entry_row(a, ad, rc, r, j0 + j * kChunk + lane, j1, false) >= 0;
+      const bool v1 = entry_row(a, ad, rc, r, j0 + j * kChunk + 32 + lane, j1, false) >= 0;
+      const uint32_t mlo = __ballot_sync(0xffffffffu, v0), mhi = __ballot_sync(0xffffffffu, v1);
+      if (!tc::mbar_wait(&sfull[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc::tc_fence_after();
+      float s[64];
+      {
+        float t0[32], t1[32];
+        tc::tmem_ld32(tmem + lane_base + kColS + b * kChunk, t0);
+        tc::tmem_ld32(tmem + lane_base + kColS + b * kChunk + 32, t1);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = t0[i];
+          s[32 + i] = t1[i];
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sempty[b]);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const bool valid = (i < 32) ? ((mlo >> i) & 1u) : ((mhi >> (i - 32)) & 1u);
+        s[i] = valid ? s[i] * c2 : -INFINITY;
+        mx = fmaxf(mx, s[i]);
+      }
+      const float m_new = fmaxf(m_run, mx);
+      // P buffer is single: PV(j-1) must be done before P(j) is written (and before any rescale)
+      if (j > 0 && !tc::mbar_wait(pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
+      const bool need = srow && (j > 0) && (m_new > m_run + kRescaleLog2);
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha_own = need ? exp2f(m_run - m_new) : 1.f;
+        const float alpha = __shfl_sync(0xffffffffu, alpha_own, lane & 15);
+        tc::tc_fence_after();
+#pragma unroll 1
+        for (int cb = 0; cb < 8; ++cb) {
+          float v[32];
+          tc::tmem_ld32(tmem + lane_base + cb * 32, v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= alpha;
+          tmem_st32(tmem + lane_base + cb * 32, v);
+        }
+        tmem_wait_st();
+        if (need) {
+          l *= alpha_own;
+          m_run = m_new;
+        }
+      }
+      if (j == 0) m_run = m_new;
+      // probabilities (base 2), bf16 P row of this head, running sum of the rounded values
+      if (srow) {
+        uint8_t* prow_base = ps;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i0 = c * 8 + 2 * u;
+            const float p0 = (m_run == -INFINITY || s[i0] == -INFINITY) ? 0.f : exp2f(s[i0] - m_run);
+            const float p1 = (m_run == -INFINITY || s[i0 + 1] == -INFINITY) ? 0.f : exp2f(s[i0 + 1] - m_run);
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            l += __low2float(pb) + __high2float(pb);
+            w[u] = *reinterpret_cast<const uint32_t*>(&pb);
+          }
+          *reinterpret_cast<uint4*>(prow_base + tc::sw128_offset(head_local, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(pfull);
+    }
+    if (!ok && lane == 0) {
+      record_error(a.status, LSA_ERR_TIMEOUT, r, 12);
+      *abort_flag = 1;
+    }
+    // final: wait for the last PV, normalise, store
+    bool fin = ok;
+    if (ok && nch > 0) fin = tc::mbar_wait(pvdone, (nch - 1) & 1, abort_flag);
+    const float l_h = __shfl_sync(0xffffffffu, l, lane & 15);
+    const float m_h = __shfl_sync(0xffffffffu, m_run, lane & 15);
+    const float inv = l_h > 0.f ? 1.f / l_h : 0.f;
+    const float lse = l_h > 0.f ? (m_h + log2f(l_h)) * kLn2 : -INFINITY;
+    const int h = half * kHeadsCta + head_local;
+    const int dim0 = lane < 16 ? 0 : 256;
+    if (fin) tc::tc_fence_after();
+#pragma unroll 1
+    for (int cb = 0; cb < 8; ++cb) {
+      float v[32];
+      if (fin && nch > 0) {
+        tc::tmem_ld32(tmem + lane_base + cb * 32, v);
+        tc::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+      if (P.nsplit == 1) {
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) +
+                           (static_cast<int64_t>(r) * kHeadsAll + h) * kDv + dim0 + cb * 32;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(v[u * 8 + 2 * e] * inv, v[u * 8 + 2 * e + 1] * inv);
+            w[e] = *reinterpret_cast<const uint32_t*>(&pb);
+          }
+          *reinterpret_cast<uint4*>(o + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      } else {
+        float* o = P.part_o + ((static_cast<int64_t>(r) * P.nsplit + split) * kHeadsAll + h) * kDv + dim0 + cb * 32;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<float4*>(o + 4 * u) =
+              make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
+      }
+    }
+    if (lane < 16) {
+      if (P.nsplit == 1) {
+        if (a.lse) a.lse[static_cast<int64_t>(r) * kHeadsAll + h] = lse;
+      } else {
+        P.part_lse[(static_cast<int64_t>(r) * P.nsplit + split) * kHeadsAll + h] = lse;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+int tc_nsplit(int32_t rows, int32_t k) {
+  const int chunks = (k + kChunk - 1) / kChunk;
+  const int64_t per = 2LL * (rows > 0 ? rows : 1);
+  int want = static_cast<int>((kPlanSMs + per - 1) / per);
+  if (want > chunks) want = chunks;
+  if (want < 1) want = 1;
+  // equalise chunks per split
+  const int cps = (chunks + want - 1) / want;
+  return (chunks + cps - 1) / cps;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+bool attn_tc_shape_ok(int32_t dtype, int32_t H, int32_t D, int32_t Dv, int32_t) {
+  return dtype == LSA_BF16 && H == kHeadsAll && D == kD && Dv == kDv;
+}
+
+int attn_tc_launches(int32_t rows, int32_t, int32_t k) { return tc_nsplit(rows, k) > 1 ? 2 : 1; }
+
+bool attn_tc_supported(const AttnArgs& a) {
+  return attn_tc_shape_ok(a.dtype, a.H, a.D, a.Dv, a.cache.block_size) && aligned16(a.cache.kv) && aligned16(a.q) &&
+         aligned16(a.out);
+}
+
+size_t attn_tc_ws_bytes(int32_t rows, int32_t H, int32_t D, int32_t Dv, int32_t k) {
+  if (H != kHeadsAll || D != kD || Dv != kDv) return 0;
+  const int ns = tc_nsplit(rows, k);
+  if (ns == 1) return 0;
+  size_t b = static_cast<size_t>(rows) * ns * H * (Dv + 1) * sizeof(float);
+  return (b + 255) / 256 * 256;
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
+  if (a.rows == 0) return cudaSuccess;
+  TcAttnParams P;
+  P.a = a;
+  P.nsplit = tc_nsplit(a.rows, a.k);
+  const int chunks = (a.k + kChunk - 1) / kChunk;
+  P.split_len = ((chunks + P.nsplit - 1) / P.nsplit) * kChunk;
+  float* ws = reinterpret_cast<float*>(a.ws);
+  P.part_o = ws;
+  P.part_lse = ws + static_cast<size_t>(a.rows) * P.nsplit * kHeadsAll * kDv;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid(P.nsplit, 2, a.rows);
+  k_attn_tc<<<grid, kThreads, kSmemBytes, s>>>(P);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || P.nsplit == 1) return e;
+  return launch_lse_merge(a, P.nsplit, P.part_o, P.part_lse, s);
+}
+
 }  // namespace lsa
