@@ -7,19 +7,23 @@
 // columns), plus lse[h].  Sparse attention reads only the kept rows (LeanSparse
 // episode page: it reduces reads, not storage).
 //
-// Layout of the work: one CTA per (query row, half of the heads, split of the
-// index list).  64 heads make the MMA's M side (M = 64), so the fp32 output
-// accumulator O[64 x 512] takes half of the TMEM lanes: dims 0-255 at lane
-// offset 0 and dims 256-511 at lane offset 16, columns 0-255; the two score
-// buffers S[64 x 64] sit at lane offset 0, columns 256-383.  Each softmax warp
-// then holds, for its 16 heads, the scores in lanes 0-15 and both output halves
-// in lanes 0-31, so a rescale touches only output columns.
-//   warps 0-3  producer: cp.async gathers of 64 selected rows per chunk into the
-//              128-byte-swizzled operand layout (zero rows for -1 / bad entries)
-//   warp 4     MMA issuer: S = Q K^T (36 x M64N64K16), O += P V (8 x M64N256K16)
+// Work: one CTA per (query row, half of the heads, split of the index list).
+// 64 heads make the MMA's M side (M = 64), so the fp32 output accumulator
+// O[64 x 512] takes half of the TMEM lanes: dims 0-255 at lane offset 0 and
+// dims 256-511 at lane offset 16, columns 0-255; the two score buffers
+// S[64 x 32] sit at lane offset 0, columns 256-319.  Each softmax warp then
+// holds, for its 16 heads, the scores in lanes 0-15 and both output halves in
+// lanes 0-31, so a rescale touches only output columns.
+//   warps 0-3  producer: cp.async gathers of 32 selected rows per chunk into the
+//              128-byte-swizzled operand layout, four chunks in flight; the
+//              block-table lookups of the next chunk are loaded one chunk ahead
+//   warp 4     MMA issuer: S = Q K^T (36 x M64N32K16), O += P V (4 x M64N256K16),
+//              V read MN-major from the same tile as K
 //   warps 5-8  online softmax (base 2, lazy rescale when the max grows by > 8),
-//              P to shared memory, final normalisation and stores
-// Splits write normalised partials and lse; the shared merge kernel combines them.
+//              P to shared memory, final normalisation
+// With several splits per row, each CTA writes a normalised partial and its
+// lse; the last CTA of a (row, half) to finish merges them (global counter,
+// no waiting), so no separate merge launch is needed.
 #include <math.h>
 
 #include "common.cuh"
@@ -33,34 +37,36 @@ constexpr int kHeadsAll = 128;
 constexpr int kHeadsCta = 64;
 constexpr int kD = 576;
 constexpr int kDv = 512;
-constexpr int kChunk = 64;                 // KV rows per chunk
+constexpr int kChunk = 32;                 // KV rows per chunk
+constexpr int kNBuf = 4;                   // chunk buffers
 constexpr int kBoxes = kD / 64;            // 9 column blocks of 64 dims
-constexpr int kBoxBytes = kChunk * 128;    // 64 rows x 128 B
-constexpr int kKvBytes = kBoxes * kBoxBytes;          // 73728
-constexpr int kQBytes = kBoxes * kHeadsCta * 128;     // 73728
-constexpr int kPBytes = kHeadsCta * 128;              // 8192
+constexpr int kBoxBytes = kChunk * 128;    // 32 rows x 128 B
+constexpr int kKvBytes = kBoxes * kBoxBytes;          // 36864
+constexpr int kQBlock = kHeadsCta * 128;              // 8192
+constexpr int kQBytes = kBoxes * kQBlock;             // 73728
+constexpr int kPBytes = kHeadsCta * 128;              // 8192 (64 B of each row used)
 constexpr int kThreads = 288;
 constexpr int kProdThreads = 128;
-constexpr int kWarpMma = 4;  // warps 5-8: softmax
-constexpr int kSmemBytes = kQBytes + 2 * kKvBytes + kPBytes + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr int kWarpMma = 4;                // warps 5-8: softmax
+constexpr int kSmemBytes = kQBytes + kNBuf * kKvBytes + kPBytes + 1024 /*barriers*/ + 1024 /*align*/;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256;            // score buffers start column
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.f;        // lazy rescale threshold (factor 256)
 
-// idesc with B major = MN (bit 16)
 constexpr uint32_t kIdescQK = tc::idesc(tc::kFmtBF16, tc::kFmtBF16, 64, kChunk);
-constexpr uint32_t kIdescPV = tc::idesc(tc::kFmtBF16, tc::kFmtBF16, 64, 256) | (1u << 16);
+constexpr uint32_t kIdescPV = tc::idesc(tc::kFmtBF16, tc::kFmtBF16, 64, 256) | (1u << 16);  // B MN-major
 
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 struct TcAttnParams {
   AttnArgs a;
   int nsplit;
-  int split_len;  // multiple of kChunk
-  float* part_o;
-  float* part_lse;
+  int split_len;   // multiple of kChunk
+  float* part_o;   // [rows][nsplit][128][512]
+  float* part_lse; // [rows][nsplit][128]
+  int* counters;   // [rows][2], zeroed before the launch
 };
 
 // MN-major operand in the 128-byte swizzle layout: 64-element MN blocks `lbo`
@@ -131,24 +137,38 @@ __device__ __forceinline__ int64_t entry_row(const AttnArgs& a, const CacheAddr&
   return row;
 }
 
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* o, const float (&v)[32], float inv) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 pb = __floats2bfloat162_rn(v[u * 8 + 2 * e] * inv, v[u * 8 + 2 * e + 1] * inv);
+      w[e] = *reinterpret_cast<const uint32_t*>(&pb);
+    }
+    *reinterpret_cast<uint4*>(o + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
   const AttnArgs& a = P.a;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qs = smem;
-  uint8_t* kvs = qs + kQBytes;         // 2 chunk buffers
-  uint8_t* ps = kvs + 2 * kKvBytes;
+  uint8_t* kvs = qs + kQBytes;         // kNBuf chunk buffers
+  uint8_t* ps = kvs + kNBuf * kKvBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ps + kPBytes);
   uint64_t* qfull = bars;
-  uint64_t* kvfull = bars + 1;    // [2]
-  uint64_t* kvempty = bars + 3;   // [2]
-  uint64_t* sfull = bars + 5;     // [2]
-  uint64_t* sempty = bars + 7;    // [2]
-  uint64_t* pfull = bars + 9;
-  uint64_t* pvdone = bars + 10;
-  uint64_t* done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* kvfull = bars + 1;            // [kNBuf]
+  uint64_t* kvempty = kvfull + kNBuf;     // [kNBuf]
+  uint64_t* sfull = kvempty + kNBuf;      // [2]
+  uint64_t* sempty = sfull + 2;           // [2]
+  uint64_t* pfull = sempty + 2;
+  uint64_t* pvdone = pfull + 1;
+  uint64_t* done = pvdone + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* last_flag = const_cast<int*>(abort_flag) + 1;
 
   const int split = blockIdx.x, half = blockIdx.y, r = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -158,9 +178,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
 
   if (threadIdx.x == 0) {
     tc::mbar_init(qfull, kProdThreads);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNBuf; ++i) {
       tc::mbar_init(&kvfull[i], kProdThreads);
       tc::mbar_init(&kvempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&sfull[i], 1);
       tc::mbar_init(&sempty[i], 4);
     }
@@ -193,30 +215,41 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       const int i = rbase + 16 * m;
       const uint8_t* src = qsrc + static_cast<int64_t>(i) * kD * 2;
       for (int d = 0; d < kBoxes; ++d)
-        cp_async16(qs_u + d * (kHeadsCta * 128) + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
+        cp_async16(qs_u + d * kQBlock + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
     }
     cp_async_arrive_noinc(qfull);
+    const bool report = sub == 0 && half == 0;
+    int64_t rn0 = entry_row(a, ad, rc, r, j0 + rbase, j1, report);
+    int64_t rn1 = entry_row(a, ad, rc, r, j0 + rbase + 16, j1, report);
     for (int j = 0; j < nch; ++j) {
-      const int b = j & 1;
-      if (!tc::mbar_wait(&kvempty[b], ((j >> 1) & 1) ^ 1, abort_flag)) {
+      const int b = j % kNBuf;
+      const int64_t rows_cur[2] = {rn0, rn1};
+      if (j + 1 < nch) {  // next chunk's lookups, in flight while this one is issued
+        rn0 = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + rbase, j1, report);
+        rn1 = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + rbase + 16, j1, report);
+      }
+      if (!tc::mbar_wait(&kvempty[b], ((j / kNBuf) & 1) ^ 1, abort_flag)) {
         if (t == 0) {
           record_error(a.status, LSA_ERR_TIMEOUT, r, 10);
           *abort_flag = 1;
         }
         break;
       }
-      const uint32_t kv_u = tc::smem_u32(kvs + b * kKvBytes);
+      uint8_t* kvb = kvs + b * kKvBytes;
+      const uint32_t kv_u = tc::smem_u32(kvb);
       bool zeroed = false;
-      for (int m = 0; m < 4; ++m) {
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
         const int i = rbase + 16 * m;
-        const int64_t row = entry_row(a, ad, rc, r, j0 + j * kChunk + i, j1, sub == 0 && half == 0);
-        if (row >= 0) {
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cache.kv) + row * (kD * 2);
-          for (int d = 0; d < kBoxes; ++d) cp_async16(kv_u + d * kBoxBytes + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
-        } else {
+        if (rows_cur[m] >= 0) {
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cache.kv) + rows_cur[m] * (kD * 2);
+#pragma unroll
           for (int d = 0; d < kBoxes; ++d)
-            *reinterpret_cast<uint4*>(kvs + b * kKvBytes + d * kBoxBytes + tc::sw128_offset(i, sub)) =
-                make_uint4(0, 0, 0, 0);
+            cp_async16(kv_u + d * kBoxBytes + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
+        } else {
+#pragma unroll
+          for (int d = 0; d < kBoxes; ++d)
+            *reinterpret_cast<uint4*>(kvb + d * kBoxBytes + tc::sw128_offset(i, sub)) = make_uint4(0, 0, 0, 0);
           zeroed = true;
         }
       }
@@ -234,39 +267,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       auto issue_pv = [&](int i) -> bool {
         if (!tc::mbar_wait(pfull, i & 1, abort_flag)) return false;
         tc::tc_fence_after();
-        const uint32_t kv_u = tc::smem_u32(kvs + (i & 1) * kKvBytes);
+        const uint32_t kv_u = tc::smem_u32(kvs + (i % kNBuf) * kKvBytes);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const uint32_t d = tmem + (static_cast<uint32_t>(16 * c) << 16);  // dims 256c.. at lane offset 16c
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < kChunk / 16; ++kk) {
             const uint64_t ad_ = tc::desc_sw128(p_u + kk * 32);
             const uint64_t bd_ = desc_sw128_mn(kv_u + (4 * c) * kBoxBytes + kk * 2048, kBoxBytes);
             tc::mma_f16(d, ad_, bd_, kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
           }
         }
         tc::mma_commit(pvdone);
-        tc::mma_commit(&kvempty[i & 1]);
+        tc::mma_commit(&kvempty[i % kNBuf]);
         return true;
       };
       for (int j = 0; ok && j < nch; ++j) {
-        const int b = j & 1;
-        if (!tc::mbar_wait(&kvfull[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+        const int b = j % kNBuf, sb = j & 1;
+        if (!tc::mbar_wait(&kvfull[b], (j / kNBuf) & 1, abort_flag)) { ok = false; break; }
         tc::fence_proxy_async_smem();
-        if (!tc::mbar_wait(&sempty[b], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&sempty[sb], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t kv_u = tc::smem_u32(kvs + b * kKvBytes);
-        const uint32_t d = tmem + kColS + b * kChunk;
+        const uint32_t d = tmem + kColS + sb * kChunk;
 #pragma unroll 1
         for (int blk = 0; blk < kBoxes; ++blk) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint64_t ad_ = tc::desc_sw128(q_u + blk * (kHeadsCta * 128) + k * 32);
+            const uint64_t ad_ = tc::desc_sw128(q_u + blk * kQBlock + k * 32);
             const uint64_t bd_ = tc::desc_sw128(kv_u + blk * kBoxBytes + k * 32);
             tc::mma_f16(d, ad_, bd_, kIdescQK, (blk | k) != 0);
           }
         }
-        tc::mma_commit(&sfull[b]);
+        tc::mma_commit(&sfull[sb]);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok) ok = issue_pv(nch - 1);
@@ -279,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       tc::mbar_wait(done, 0, nullptr);
     }
   } else {
-    // ---------------------------------------------------------------- softmax / epilogue
+    // ---------------------------------------------------------------- softmax
     const int quarter = warp & 3;                       // TMEM lanes 32q .. 32q+31
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool srow = lane < 16;                        // lanes holding a score row
@@ -287,34 +320,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     const float c2 = a.scale * kLog2e;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
+    bool vnext = nch > 0 && entry_row(a, ad, rc, r, j0 + lane, j1, false) >= 0;
     for (int j = 0; j < nch; ++j) {
-      const int b = j & 1;
-      // validity of the 64 rows of this chunk (recomputed; same rule as the producer)
-      const bool v0 = entry_row(a, ad, rc, r, j0 + j * kChunk + lane, j1, false) >= 0;
-      const bool v1 = entry_row(a, ad, rc, r, j0 + j * kChunk + 32 + lane, j1, false) >= 0;
-      const uint32_t mlo = __ballot_sync(0xffffffffu, v0), mhi = __ballot_sync(0xffffffffu, v1);
-      if (!tc::mbar_wait(&sfull[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      const int sb = j & 1;
+      const uint32_t mask = __ballot_sync(0xffffffffu, vnext);
+      if (j + 1 < nch) vnext = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + lane, j1, false) >= 0;
+      if (!tc::mbar_wait(&sfull[sb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       tc::tc_fence_after();
-      float s[64];
-      {
-        float t0[32], t1[32];
-        tc::tmem_ld32(tmem + lane_base + kColS + b * kChunk, t0);
-        tc::tmem_ld32(tmem + lane_base + kColS + b * kChunk + 32, t1);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = t0[i];
-          s[32 + i] = t1[i];
-        }
-      }
+      float s[32];
+      tc::tmem_ld32(tmem + lane_base + kColS + sb * kChunk, s);
+      tc::tmem_wait_ld();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sempty[b]);
+      if (lane == 0) tc::mbar_arrive(&sempty[sb]);
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const bool valid = (i < 32) ? ((mlo >> i) & 1u) : ((mhi >> (i - 32)) & 1u);
-        s[i] = valid ? s[i] * c2 : -INFINITY;
+      for (int i = 0; i < 32; ++i) {
+        s[i] = ((mask >> i) & 1u) ? s[i] * c2 : -INFINITY;
         mx = fmaxf(mx, s[i]);
       }
       const float m_new = fmaxf(m_run, mx);
@@ -343,9 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       if (j == 0) m_run = m_new;
       // probabilities (base 2), bf16 P row of this head, running sum of the rounded values
       if (srow) {
-        uint8_t* prow_base = ps;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -356,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
             l += __low2float(pb) + __high2float(pb);
             w[u] = *reinterpret_cast<const uint32_t*>(&pb);
           }
-          *reinterpret_cast<uint4*>(prow_base + tc::sw128_offset(head_local, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(ps + tc::sw128_offset(head_local, c)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       tc::fence_proxy_async_smem();
@@ -368,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       record_error(a.status, LSA_ERR_TIMEOUT, r, 12);
       *abort_flag = 1;
     }
-    // final: wait for the last PV, normalise, store
+    // final: wait for the last PV, normalise, store (bf16 output or fp32 partial)
     bool fin = ok;
     if (ok && nch > 0) fin = tc::mbar_wait(pvdone, (nch - 1) & 1, abort_flag);
     const float l_h = __shfl_sync(0xffffffffu, l, lane & 15);
@@ -389,18 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
         for (int i = 0; i < 32; ++i) v[i] = 0.f;
       }
       if (P.nsplit == 1) {
-        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) +
-                           (static_cast<int64_t>(r) * kHeadsAll + h) * kDv + dim0 + cb * 32;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(v[u * 8 + 2 * e] * inv, v[u * 8 + 2 * e + 1] * inv);
-            w[e] = *reinterpret_cast<const uint32_t*>(&pb);
-          }
-          *reinterpret_cast<uint4*>(o + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        store_bf16x32(reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<int64_t>(r) * kHeadsAll + h) * kDv +
+                          dim0 + cb * 32, v, inv);
       } else {
         float* o = P.part_o + ((static_cast<int64_t>(r) * P.nsplit + split) * kHeadsAll + h) * kDv + dim0 + cb * 32;
 #pragma unroll
@@ -417,6 +428,57 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       }
     }
   }
+  // ---------------------------------------------------------------- split merge by the last CTA
+  if (P.nsplit > 1) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const int prev = atomicAdd(P.counters + 2 * r + half, 1);
+      *last_flag = prev == P.nsplit - 1;
+    }
+    __syncthreads();
+    if (*last_flag) {
+      __threadfence();
+      if (threadIdx.x == 0) P.counters[2 * r + half] = 0;  // left zeroed for the next call
+      // 128 threads: head = t / 2, 256 dims each
+      if (threadIdx.x >= kWarpMma * 32 + 32) {
+        const int t = threadIdx.x - (kWarpMma * 32 + 32);
+        const int h = half * kHeadsCta + (t >> 1);
+        const int dim0 = (t & 1) * 256;
+        const float* lse_p = P.part_lse + static_cast<int64_t>(r) * P.nsplit * kHeadsAll + h;
+        float mx = -INFINITY;
+        for (int sp = 0; sp < P.nsplit; ++sp) mx = fmaxf(mx, __ldcg(lse_p + sp * kHeadsAll));
+        float den = 0.f;
+        if (mx != -INFINITY)
+          for (int sp = 0; sp < P.nsplit; ++sp) den += exp2f((__ldcg(lse_p + sp * kHeadsAll) - mx) * kLog2e);
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<int64_t>(r) * kHeadsAll + h) * kDv;
+#pragma unroll 1
+        for (int cb = 0; cb < 8; ++cb) {
+          float acc[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+          for (int sp = 0; sp < P.nsplit && mx != -INFINITY; ++sp) {
+            const float wgt = exp2f((__ldcg(lse_p + sp * kHeadsAll) - mx) * kLog2e);
+            if (!(wgt > 0.f)) continue;
+            const float4* src = reinterpret_cast<const float4*>(
+                P.part_o + ((static_cast<int64_t>(r) * P.nsplit + sp) * kHeadsAll + h) * kDv + dim0 + cb * 32);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float4 x = __ldcg(src + u);
+              acc[4 * u] = fmaf(wgt, x.x, acc[4 * u]);
+              acc[4 * u + 1] = fmaf(wgt, x.y, acc[4 * u + 1]);
+              acc[4 * u + 2] = fmaf(wgt, x.z, acc[4 * u + 2]);
+              acc[4 * u + 3] = fmaf(wgt, x.w, acc[4 * u + 3]);
+            }
+          }
+          store_bf16x32(o + dim0 + cb * 32, acc, inv);
+        }
+        if ((t & 1) == 0 && a.lse)
+          a.lse[static_cast<int64_t>(r) * kHeadsAll + h] = mx == -INFINITY ? -INFINITY : mx + logf(den);
+      }
+    }
+  }
   __syncthreads();
   if (warp == kWarpMma) {
     tc::tc_fence_after();
@@ -426,16 +488,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
 
 int tc_nsplit(int32_t rows, int32_t k) {
   const int chunks = (k + kChunk - 1) / kChunk;
-  const int64_t per = 2LL * (rows > 0 ? rows : 1);
-  int want = static_cast<int>((kPlanSMs + per - 1) / per);
+  const int64_t per = 2LL * (rows > 0 ? rows : 1);       // CTAs per split
+  int want = static_cast<int>(kPlanSMs / per);          // stay within one wave
   if (want > chunks) want = chunks;
   if (want < 1) want = 1;
-  // equalise chunks per split
-  const int cps = (chunks + want - 1) / want;
+  const int cps = (chunks + want - 1) / want;            // equal chunks per split
   return (chunks + cps - 1) / cps;
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
 }  // namespace
 
@@ -443,7 +506,7 @@ bool attn_tc_shape_ok(int32_t dtype, int32_t H, int32_t D, int32_t Dv, int32_t) 
   return dtype == LSA_BF16 && H == kHeadsAll && D == kD && Dv == kDv;
 }
 
-int attn_tc_launches(int32_t rows, int32_t, int32_t k) { return tc_nsplit(rows, k) > 1 ? 2 : 1; }
+int attn_tc_launches(int32_t, int32_t, int32_t) { return 1; }
 
 bool attn_tc_supported(const AttnArgs& a) {
   return attn_tc_shape_ok(a.dtype, a.H, a.D, a.Dv, a.cache.block_size) && aligned16(a.cache.kv) && aligned16(a.q) &&
@@ -454,8 +517,9 @@ size_t attn_tc_ws_bytes(int32_t rows, int32_t H, int32_t D, int32_t Dv, int32_t 
   if (H != kHeadsAll || D != kD || Dv != kDv) return 0;
   const int ns = tc_nsplit(rows, k);
   if (ns == 1) return 0;
-  size_t b = static_cast<size_t>(rows) * ns * H * (Dv + 1) * sizeof(float);
-  return (b + 255) / 256 * 256;
+  return align256(static_cast<size_t>(rows) * 2 * sizeof(int)) +
+         align256(static_cast<size_t>(rows) * ns * H * sizeof(float)) +
+         align256(static_cast<size_t>(rows) * ns * H * Dv * sizeof(float));
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
@@ -465,9 +529,16 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   P.nsplit = tc_nsplit(a.rows, a.k);
   const int chunks = (a.k + kChunk - 1) / kChunk;
   P.split_len = ((chunks + P.nsplit - 1) / P.nsplit) * kChunk;
-  float* ws = reinterpret_cast<float*>(a.ws);
-  P.part_o = ws;
-  P.part_lse = ws + static_cast<size_t>(a.rows) * P.nsplit * kHeadsAll * kDv;
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  const size_t cnt_b = align256(static_cast<size_t>(a.rows) * 2 * sizeof(int));
+  const size_t lse_b = align256(static_cast<size_t>(a.rows) * P.nsplit * kHeadsAll * sizeof(float));
+  P.counters = reinterpret_cast<int*>(ws);
+  P.part_lse = reinterpret_cast<float*>(ws + cnt_b);
+  P.part_o = reinterpret_cast<float*>(ws + cnt_b + lse_b);
+  if (P.nsplit > 1) {
+    cudaError_t e = cudaMemsetAsync(P.counters, 0, static_cast<size_t>(a.rows) * 2 * sizeof(int), s);
+    if (e != cudaSuccess) return e;
+  }
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
@@ -476,9 +547,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   }
   dim3 grid(P.nsplit, 2, a.rows);
   k_attn_tc<<<grid, kThreads, kSmemBytes, s>>>(P);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || P.nsplit == 1) return e;
-  return launch_lse_merge(a, P.nsplit, P.part_o, P.part_lse, s);
+  return cudaGetLastError();
 }
 
 }  // namespace lsa

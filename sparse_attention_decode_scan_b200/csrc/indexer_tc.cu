@@ -454,6 +454,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
       W.start(a, plan.r_first, plan.j_first);
       int gi = -1, qi = 0;
       int64_t vis_r[QB];
+      // The block-table lookup (and FP8 scale) of a tile is loaded one tile
+      // ahead, so its latency overlaps the wait for the accumulator.
+      int64_t prow_next, p_next;
+      float ks_next;
+      auto prefetch = [&](const Walker<QB>& w) {
+        p_next = static_cast<int64_t>(w.j) * kTile + t;
+        prow_next = p_next < w.g.vis ? ad.row(w.g.b, p_next) : -1;
+        ks_next = (C::kFp8 && prow_next >= 0) ? __ldg(a.cache.idx_key_scales + prow_next) : 1.f;
+      };
+      prefetch(W);
       for (int64_t it = 0; it < plan.n_items; ++it) {
         if (it == 0 || W.j == 0) {
           ++gi;
@@ -480,10 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
           break;
         }
         tc::tc_fence_after();
-        const int64_t p = static_cast<int64_t>(W.j) * kTile + t;
-        const int64_t prow = p < W.g.vis ? ad.row(W.g.b, p) : -1;
-        float kscale = 1.f;
-        if (C::kFp8 && prow >= 0) kscale = __ldg(a.cache.idx_key_scales + prow);
+        const int64_t p = p_next;
+        const int64_t prow = prow_next;
+        const float kscale = ks_next;
         const float* wb = wbufs + qi * (C::kWBytes / 4);
         float sc[QB];
 #pragma unroll
@@ -525,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
           if (lane == 0) tc::mbar_arrive(&qempty[qi]);
         }
         W.next(a);
+        if (it + 1 < plan.n_items) prefetch(W);
       }
     }
     // tails: positions past each row's group tiles are -inf (NaN for an invalid row)
