@@ -188,6 +188,31 @@ lsa_status lsa_decode_step(const lsa_dims* d, const lsa_cache* c, const void* q_
 lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream);
 
 /*
+ * Top-k without a workspace argument, for callers that cannot allocate device
+ * memory where they call it: a plugin host whose enqueue path forbids
+ * allocation, a runtime whose device memory is all pre-reserved by another
+ * allocator, or a latency-critical loop that cannot pay for cudaMalloc's
+ * implicit synchronisation.  (The pages describe no such entry point; it is
+ * an addition of this library.)
+ *   Same arguments, results and errors as lsa_topk, minus ws / ws_bytes.
+ *   Scratch: a 2 MiB static device array inside liblsa.so, held by every GPU
+ *   that loads the library until the process exits.  Sizes whose top-k scratch
+ *   (lsa_workspace_size(NULL, rows, n_cols, LSA_OP_TOPK)) exceeds 2 MiB return
+ *   LSA_ERR_UNSUPPORTED (about 100 rows fit, whatever their length).
+ *   Allocates nothing: no cudaMalloc / cudaFree; the histograms are cleared
+ *   with cudaMemsetAsync on `stream` at every call.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.
+ *   Every call shares the one array: calls that overlap on the GPU (different
+ *   streams, or different host threads on one device) race and give wrong
+ *   results.  Device-side error reports of this entry point are not readable
+ *   through lsa_read_device_status.
+ */
+lsa_status lsa_topk_noalloc(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len,
+                            int64_t n_cols, int32_t k, int32_t* idx, lsa_stream_t stream);
+
+/*
  * Number of kernel launches `op` enqueues for `rows` query rows with score rows
  * of `max_len` entries (`causal` != 0: prefill rows with positions), assuming
  * 16-byte aligned buffers.  A planning aid for launch accounting and graph

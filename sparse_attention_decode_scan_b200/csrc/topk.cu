@@ -13,6 +13,8 @@
 // global memory between launches, so no kernel waits on another CTA.
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -341,3 +343,70 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
 }
 
 }  // namespace lsa
+
+// ---------------------------------------------------------------------------
+// Top-k without a caller workspace.
+//
+// Some callers cannot allocate device memory where they call the top-k: a
+// plugin host whose enqueue path forbids allocation, a runtime whose device
+// memory is entirely pre-reserved by another allocator, or a latency-critical
+// loop that cannot afford cudaMalloc's implicit synchronisation.  For them the
+// scratch of the five top-k passes lives in the fixed-size array below, which
+// every GPU that loads this library holds until the process exits.
+
+namespace lsa {
+namespace {
+
+constexpr size_t kStaticScratchBytes = 2u << 20;  // 2 MiB: status word + histograms + segment counts
+
+static __device__ __align__(256) uint8_t g_topk_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_topk_scratch on the current device (the host-side name of
+// the array is only a stand-in and must never reach a kernel).  Looked up once
+// per device, with that device current.
+cudaError_t static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_topk_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace lsa
+
+extern "C" lsa_status lsa_topk_noalloc(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len,
+                                       int64_t n_cols, int32_t k, int32_t* idx, lsa_stream_t stream) {
+  using namespace lsa;
+  if (rows < 0 || k < 1 || n_cols < 0 || ld < n_cols || (ld % 4) != 0) return LSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!scores || !idx || (reinterpret_cast<uintptr_t>(scores) & 15u) != 0)) return LSA_ERR_INVALID_ARG;
+  if (n_cols > (1LL << 31) - 1) return LSA_ERR_UNSUPPORTED;
+  const size_t need = kStatusBytes + topk_ws_bytes(rows, n_cols);
+  if (need > kStaticScratchBytes) return LSA_ERR_UNSUPPORTED;  // beyond the static scratch
+  if (rows == 0) return LSA_OK;
+  void* base = nullptr;
+  if (static_scratch(&base) != cudaSuccess) return LSA_ERR_CUDA;
+  TopkArgs a;
+  a.scores = scores;
+  a.ld = ld;
+  a.rows = rows;
+  a.valid_len = valid_len;
+  a.n_cols = n_cols;
+  a.k = k;
+  a.idx = idx;
+  a.ws = static_cast<uint8_t*>(base) + kStatusBytes;  // histograms are zeroed by launch_topk
+  a.status = reinterpret_cast<DevStatus*>(base);
+  return launch_topk(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}

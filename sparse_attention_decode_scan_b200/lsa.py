@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
     L.lsa_workspace_size.restype = sz
     L.lsa_indexer_scores.argtypes = [D, C, i32, vp, vp, vp, vp, vp, i64, vp, sz, vp]
     L.lsa_topk.argtypes = [vp, i64, i32, vp, i64, i32, vp, vp, sz, vp]
+    L.lsa_topk_noalloc.argtypes = [vp, i64, i32, vp, i64, i32, vp, vp]
     L.lsa_sparse_attn_decode.argtypes = [D, C, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.lsa_decode_step.argtypes = [D, C, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
     L.lsa_read_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
@@ -70,7 +71,7 @@ def lib() -> ctypes.CDLL:
     L.lsa_version.restype = i32
     L.lsa_launch_count.argtypes = [D, i32, i64, i32, i32]
     L.lsa_launch_count.restype = i32
-    for f in ("lsa_indexer_scores", "lsa_topk", "lsa_sparse_attn_decode", "lsa_decode_step",
+    for f in ("lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode", "lsa_decode_step",
               "lsa_read_device_status"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
@@ -127,6 +128,16 @@ def topk(scores, k: int, idx, ws, valid_len=None, n_cols: Optional[int] = None, 
     return _check(lib().lsa_topk(_ptr(scores), ld, rows, _ptr(valid_len), n_cols, int(k), _ptr(idx), _ptr(ws),
                                  ws.numel() if ws is not None else 0, _stream(stream)),
                   "lsa_topk", raise_on_error)
+
+
+def topk_noalloc(scores, k: int, idx, valid_len=None, n_cols: Optional[int] = None, ld: Optional[int] = None,
+                 rows: Optional[int] = None, stream=None, raise_on_error=True) -> int:
+    """lsa_topk_noalloc: the top-k with the library's static scratch instead of a workspace."""
+    rows = int(scores.shape[0]) if rows is None else rows
+    ld = int(scores.stride(0)) if ld is None else ld
+    n_cols = int(scores.shape[1]) if n_cols is None else n_cols
+    return _check(lib().lsa_topk_noalloc(_ptr(scores), ld, rows, _ptr(valid_len), n_cols, int(k), _ptr(idx),
+                                         _stream(stream)), "lsa_topk_noalloc", raise_on_error)
 
 
 def sparse_attn_decode(dims: Dims, cache: Cache, q, idx, out, lse, ws, row_seq=None, rows: Optional[int] = None,
