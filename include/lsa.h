@@ -117,8 +117,8 @@ typedef enum {
 
 /*
  * Bytes of workspace `op` needs for `rows` query rows whose score rows hold
- * `max_len` entries (0 on invalid arguments).  For LSA_OP_TOPK, `d` is not
- * read and may be NULL (the top-k workspace does not depend on k).
+ * `max_len` entries (0 on invalid arguments).  For LSA_OP_TOPK only d->top_k
+ * is read (the k of the lsa_topk call).
  */
 size_t lsa_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t op);
 
@@ -197,8 +197,8 @@ lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream
  *   Same arguments, results and errors as lsa_topk, minus ws / ws_bytes.
  *   Scratch: a 2 MiB static device array inside liblsa.so, held by every GPU
  *   that loads the library until the process exits.  Sizes whose top-k scratch
- *   (lsa_workspace_size(NULL, rows, n_cols, LSA_OP_TOPK)) exceeds 2 MiB return
- *   LSA_ERR_UNSUPPORTED (about 100 rows fit, whatever their length).
+ *   (lsa_workspace_size with d->top_k = k, LSA_OP_TOPK) exceeds 2 MiB return
+ *   LSA_ERR_UNSUPPORTED (for k = 2048: 32 rows fit, whatever their length).
  *   Allocates nothing: no cudaMalloc / cudaFree; the histograms are cleared
  *   with cudaMemsetAsync on `stream` at every call.
  *   The first call on a device looks up the array's device address (once per

@@ -91,7 +91,7 @@ StepLayout step_layout(const lsa_dims* d, int32_t rows, int64_t max_len) {
   L.scores_off = kStatusBytes;
   L.idx_off = L.scores_off + align_up(static_cast<size_t>(rows) * score_ld(max_len) * 4);
   L.inner_off = L.idx_off + align_up(static_cast<size_t>(rows) * d->top_k * 4);
-  size_t inner = topk_ws_bytes(rows, max_len);
+  size_t inner = topk_ws_bytes(rows, max_len, d->top_k);
   size_t a = attn_ws(d, rows);
   size_t s = scores_ws(rows, false);
   if (a > inner) inner = a;
@@ -188,7 +188,8 @@ size_t lsa_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int3
       if (!valid_dims(d)) return 0;
       return kStatusBytes + scores_ws(rows, true);
     case LSA_OP_TOPK:
-      return kStatusBytes + align_up(topk_ws_bytes(rows, max_len));
+      if (!d || d->top_k < 1) return 0;
+      return kStatusBytes + align_up(topk_ws_bytes(rows, max_len, d->top_k));
     case LSA_OP_ATTN:
       if (!valid_dims(d)) return 0;
       return kStatusBytes + attn_ws(d, rows);
@@ -222,7 +223,7 @@ lsa_status lsa_topk(const float* scores, int64_t ld, int32_t rows, const int32_t
   if (rows > 0 && (!scores || !idx || !aligned16(scores))) return LSA_ERR_INVALID_ARG;
   if (rows > 65535) return LSA_ERR_UNSUPPORTED;
   if (n_cols > (1LL << 31) - 1) return LSA_ERR_UNSUPPORTED;
-  const size_t need = kStatusBytes + align_up(topk_ws_bytes(rows, n_cols));
+  const size_t need = kStatusBytes + align_up(topk_ws_bytes(rows, n_cols, k));
   lsa_status st = ws_check(ws, ws_bytes, need);
   if (st != LSA_OK) return st;
   if (rows == 0) return LSA_OK;
@@ -285,7 +286,7 @@ lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream
 
 int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t op, int32_t causal) {
   if (rows < 0 || max_len < 0) return -1;
-  if (op != LSA_OP_TOPK && !valid_dims(d)) return -1;
+  if (op == LSA_OP_TOPK ? (!d || d->top_k < 1) : !valid_dims(d)) return -1;
   if (rows == 0) return 0;
   const bool simt = force_simt();
   int scan = 1;
@@ -300,9 +301,9 @@ int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32
   }
   switch (op) {
     case LSA_OP_SCORES: return scan;
-    case LSA_OP_TOPK: return kTopkLaunches;
+    case LSA_OP_TOPK: return topk_launches(max_len);
     case LSA_OP_ATTN: return attn;
-    case LSA_OP_DECODE_STEP: return scan + kTopkLaunches + attn;
+    case LSA_OP_DECODE_STEP: return scan + topk_launches(max_len) + attn;
     default: return -1;
   }
 }

@@ -15,15 +15,16 @@
 // holds, for its 16 heads, the scores in lanes 0-15 and both output halves in
 // lanes 0-31, so a rescale touches only output columns.
 //   warps 0-3  producer: cp.async gathers of 32 selected rows per chunk into the
-//              128-byte-swizzled operand layout, four chunks in flight; the
+//              128-byte-swizzled operand layout, three chunks in flight; the
 //              block-table lookups of the next chunk are loaded one chunk ahead
 //   warp 4     MMA issuer: S = Q K^T (36 x M64N32K16), O += P V (4 x M64N256K16),
 //              V read MN-major from the same tile as K
 //   warps 5-8  online softmax (base 2, lazy rescale when the max grows by > 8),
-//              P to shared memory, final normalisation
+//              P to one of two shared-memory buffers (so the softmax of chunk j+1
+//              overlaps P V of chunk j), final normalisation
 // With several splits per row, each CTA writes a normalised partial and its
-// lse; the last CTA of a (row, half) to finish merges them (global counter,
-// no waiting), so no separate merge launch is needed.
+// lse; the last CTA of a (row, half) to finish merges them with all of its
+// threads (global counter, no waiting), so no separate merge launch is needed.
 #include <math.h>
 
 #include "common.cuh"
@@ -38,17 +39,17 @@ constexpr int kHeadsCta = 64;
 constexpr int kD = 576;
 constexpr int kDv = 512;
 constexpr int kChunk = 32;                 // KV rows per chunk
-constexpr int kNBuf = 4;                   // chunk buffers
+constexpr int kNBuf = 3;                   // chunk buffers (gathers in flight)
 constexpr int kBoxes = kD / 64;            // 9 column blocks of 64 dims
 constexpr int kBoxBytes = kChunk * 128;    // 32 rows x 128 B
 constexpr int kKvBytes = kBoxes * kBoxBytes;          // 36864
 constexpr int kQBlock = kHeadsCta * 128;              // 8192
 constexpr int kQBytes = kBoxes * kQBlock;             // 73728
-constexpr int kPBytes = kHeadsCta * 128;              // 8192 (64 B of each row used)
+constexpr int kPBytes = kHeadsCta * 128;              // 8192 per P buffer (64 B of each row used)
 constexpr int kThreads = 288;
 constexpr int kProdThreads = 128;
 constexpr int kWarpMma = 4;                // warps 5-8: softmax
-constexpr int kSmemBytes = kQBytes + kNBuf * kKvBytes + kPBytes + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr int kSmemBytes = kQBytes + kNBuf * kKvBytes + 2 * kPBytes + 1024 /*barriers*/ + 1024 /*align*/;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256;            // score buffers start column
 constexpr float kLog2e = 1.4426950408889634f;
@@ -156,16 +157,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qs = smem;
   uint8_t* kvs = qs + kQBytes;         // kNBuf chunk buffers
-  uint8_t* ps = kvs + kNBuf * kKvBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + kPBytes);
+  uint8_t* ps = kvs + kNBuf * kKvBytes;  // 2 P buffers
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + 2 * kPBytes);
   uint64_t* qfull = bars;
   uint64_t* kvfull = bars + 1;            // [kNBuf]
   uint64_t* kvempty = kvfull + kNBuf;     // [kNBuf]
   uint64_t* sfull = kvempty + kNBuf;      // [2]
   uint64_t* sempty = sfull + 2;           // [2]
-  uint64_t* pfull = sempty + 2;
-  uint64_t* pvdone = pfull + 1;
-  uint64_t* done = pvdone + 1;
+  uint64_t* pfull = sempty + 2;           // [2] per P buffer
+  uint64_t* pvdone = pfull + 2;           // [2] per P buffer
+  uint64_t* done = pvdone + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
@@ -186,8 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       tc::mbar_init(&sfull[i], 1);
       tc::mbar_init(&sempty[i], 4);
     }
-    tc::mbar_init(pfull, 4);
-    tc::mbar_init(pvdone, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&pfull[i], 4);
+      tc::mbar_init(&pvdone[i], 1);
+    }
     tc::mbar_init(done, 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
@@ -261,12 +264,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0 && nch > 0) {
       const uint32_t q_u = tc::smem_u32(qs);
-      const uint32_t p_u = tc::smem_u32(ps);
       bool ok = tc::mbar_wait(qfull, 0, abort_flag);
       tc::fence_proxy_async_smem();
       auto issue_pv = [&](int i) -> bool {
-        if (!tc::mbar_wait(pfull, i & 1, abort_flag)) return false;
+        const int pb = i & 1;
+        if (!tc::mbar_wait(&pfull[pb], (i >> 1) & 1, abort_flag)) return false;
         tc::tc_fence_after();
+        const uint32_t p_u = tc::smem_u32(ps + pb * kPBytes);
         const uint32_t kv_u = tc::smem_u32(kvs + (i % kNBuf) * kKvBytes);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -278,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
             tc::mma_f16(d, ad_, bd_, kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        tc::mma_commit(pvdone);
+        tc::mma_commit(&pvdone[pb]);
         tc::mma_commit(&kvempty[i % kNBuf]);
         return true;
       };
@@ -320,11 +324,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     const float c2 = a.scale * kLog2e;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
-    bool vnext = nch > 0 && entry_row(a, ad, rc, r, j0 + lane, j1, false) >= 0;
+    // validity of chunk rows, looked up two chunks ahead of their use
+    bool v0 = nch > 0 && entry_row(a, ad, rc, r, j0 + lane, j1, false) >= 0;
+    bool v1 = nch > 1 && entry_row(a, ad, rc, r, j0 + kChunk + lane, j1, false) >= 0;
     for (int j = 0; j < nch; ++j) {
       const int sb = j & 1;
-      const uint32_t mask = __ballot_sync(0xffffffffu, vnext);
-      if (j + 1 < nch) vnext = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + lane, j1, false) >= 0;
+      const uint32_t mask = __ballot_sync(0xffffffffu, v0);
+      v0 = v1;
+      if (j + 2 < nch) v1 = entry_row(a, ad, rc, r, j0 + (j + 2) * kChunk + lane, j1, false) >= 0;
       if (!tc::mbar_wait(&sfull[sb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       tc::tc_fence_after();
       float s[32];
@@ -340,10 +347,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
         mx = fmaxf(mx, s[i]);
       }
       const float m_new = fmaxf(m_run, mx);
-      // P buffer is single: PV(j-1) must be done before P(j) is written (and before any rescale)
-      if (j > 0 && !tc::mbar_wait(pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
       const bool need = srow && (j > 0) && (m_new > m_run + kRescaleLog2);
-      if (__any_sync(0xffffffffu, need)) {
+      const bool any_need = __any_sync(0xffffffffu, need);
+      // a rescale touches O: P V of chunk j-1 must have finished
+      if (any_need && !tc::mbar_wait(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+      // P(j) reuses the buffer of chunk j-2: its P V must have finished
+      if (j >= 2 && !tc::mbar_wait(&pvdone[j & 1], ((j - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (any_need) {
         const float alpha_own = need ? exp2f(m_run - m_new) : 1.f;
         const float alpha = __shfl_sync(0xffffffffu, alpha_own, lane & 15);
         tc::tc_fence_after();
@@ -377,13 +387,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
             l += __low2float(pb) + __high2float(pb);
             w[u] = *reinterpret_cast<const uint32_t*>(&pb);
           }
-          *reinterpret_cast<uint4*>(ps + tc::sw128_offset(head_local, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(ps + (j & 1) * kPBytes + tc::sw128_offset(head_local, c)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(pfull);
+      if (lane == 0) tc::mbar_arrive(&pfull[j & 1]);
     }
     if (!ok && lane == 0) {
       record_error(a.status, LSA_ERR_TIMEOUT, r, 12);
@@ -391,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     }
     // final: wait for the last PV, normalise, store (bf16 output or fp32 partial)
     bool fin = ok;
-    if (ok && nch > 0) fin = tc::mbar_wait(pvdone, (nch - 1) & 1, abort_flag);
+    if (ok && nch > 0) fin = tc::mbar_wait(&pvdone[(nch - 1) & 1], ((nch - 1) >> 1) & 1, abort_flag);
     const float l_h = __shfl_sync(0xffffffffu, l, lane & 15);
     const float m_h = __shfl_sync(0xffffffffu, m_run, lane & 15);
     const float inv = l_h > 0.f ? 1.f / l_h : 0.f;
@@ -440,42 +451,56 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     if (*last_flag) {
       __threadfence();
       if (threadIdx.x == 0) P.counters[2 * r + half] = 0;  // left zeroed for the next call
-      // 128 threads: head = t / 2, 256 dims each
-      if (threadIdx.x >= kWarpMma * 32 + 32) {
-        const int t = threadIdx.x - (kWarpMma * 32 + 32);
-        const int h = half * kHeadsCta + (t >> 1);
-        const int dim0 = (t & 1) * 256;
-        const float* lse_p = P.part_lse + static_cast<int64_t>(r) * P.nsplit * kHeadsAll + h;
+      // weights of every split for the 64 heads, in the (now idle) P buffers
+      float* wsm = reinterpret_cast<float*>(ps);          // [nsplit][64], nsplit <= 32
+      const int ns = P.nsplit;
+      const float* lse_p = P.part_lse + static_cast<int64_t>(r) * ns * kHeadsAll + half * kHeadsCta;
+      if (threadIdx.x < kHeadsCta) {
+        const int hl = threadIdx.x;
         float mx = -INFINITY;
-        for (int sp = 0; sp < P.nsplit; ++sp) mx = fmaxf(mx, __ldcg(lse_p + sp * kHeadsAll));
+        for (int sp = 0; sp < ns; ++sp) mx = fmaxf(mx, __ldcg(lse_p + sp * kHeadsAll + hl));
         float den = 0.f;
-        if (mx != -INFINITY)
-          for (int sp = 0; sp < P.nsplit; ++sp) den += exp2f((__ldcg(lse_p + sp * kHeadsAll) - mx) * kLog2e);
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<int64_t>(r) * kHeadsAll + h) * kDv;
-#pragma unroll 1
-        for (int cb = 0; cb < 8; ++cb) {
-          float acc[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-          for (int sp = 0; sp < P.nsplit && mx != -INFINITY; ++sp) {
-            const float wgt = exp2f((__ldcg(lse_p + sp * kHeadsAll) - mx) * kLog2e);
-            if (!(wgt > 0.f)) continue;
-            const float4* src = reinterpret_cast<const float4*>(
-                P.part_o + ((static_cast<int64_t>(r) * P.nsplit + sp) * kHeadsAll + h) * kDv + dim0 + cb * 32);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const float4 x = __ldcg(src + u);
-              acc[4 * u] = fmaf(wgt, x.x, acc[4 * u]);
-              acc[4 * u + 1] = fmaf(wgt, x.y, acc[4 * u + 1]);
-              acc[4 * u + 2] = fmaf(wgt, x.z, acc[4 * u + 2]);
-              acc[4 * u + 3] = fmaf(wgt, x.w, acc[4 * u + 3]);
-            }
-          }
-          store_bf16x32(o + dim0 + cb * 32, acc, inv);
+        for (int sp = 0; sp < ns; ++sp) {
+          const float e = mx == -INFINITY ? 0.f : exp2f((__ldcg(lse_p + sp * kHeadsAll + hl) - mx) * kLog2e);
+          wsm[sp * kHeadsCta + hl] = e;
+          den += e;
         }
-        if ((t & 1) == 0 && a.lse)
-          a.lse[static_cast<int64_t>(r) * kHeadsAll + h] = mx == -INFINITY ? -INFINITY : mx + logf(den);
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        for (int sp = 0; sp < ns; ++sp) wsm[sp * kHeadsCta + hl] *= inv;
+        if (a.lse) a.lse[static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + hl] = den > 0.f ? mx + logf(den) : -INFINITY;
+      }
+      __syncthreads();
+      // 64 heads x 128 groups of 4 dims, spread over every thread of the CTA
+      const float4* po = reinterpret_cast<const float4*>(P.part_o);
+      for (int item = threadIdx.x; item < kHeadsCta * (kDv / 4); item += kThreads) {
+        const int hl = item / (kDv / 4), c4 = item % (kDv / 4);
+        const int h = half * kHeadsCta + hl;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        int sp = 0;
+        for (; sp + 4 <= ns; sp += 4) {
+          float4 x[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            x[u] = __ldcg(po + ((static_cast<int64_t>(r) * ns + sp + u) * kHeadsAll + h) * (kDv / 4) + c4);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float wgt = wsm[(sp + u) * kHeadsCta + hl];
+            acc.x = fmaf(wgt, x[u].x, acc.x); acc.y = fmaf(wgt, x[u].y, acc.y);
+            acc.z = fmaf(wgt, x[u].z, acc.z); acc.w = fmaf(wgt, x[u].w, acc.w);
+          }
+        }
+        for (; sp < ns; ++sp) {
+          const float4 x = __ldcg(po + ((static_cast<int64_t>(r) * ns + sp) * kHeadsAll + h) * (kDv / 4) + c4);
+          const float wgt = wsm[sp * kHeadsCta + hl];
+          acc.x = fmaf(wgt, x.x, acc.x); acc.y = fmaf(wgt, x.y, acc.y);
+          acc.z = fmaf(wgt, x.z, acc.z); acc.w = fmaf(wgt, x.w, acc.w);
+        }
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                  (static_cast<int64_t>(r) * kHeadsAll + h) * kDv + c4 * 4) = pk;
       }
     }
   }
@@ -491,6 +516,7 @@ int tc_nsplit(int32_t rows, int32_t k) {
   const int64_t per = 2LL * (rows > 0 ? rows : 1);       // CTAs per split
   int want = static_cast<int>(kPlanSMs / per);          // stay within one wave
   if (want > chunks) want = chunks;
+  if (want > 32) want = 32;                              // merge weights fit one P buffer
   if (want < 1) want = 1;
   const int cps = (chunks + want - 1) / want;            // equal chunks per split
   return (chunks + cps - 1) / cps;

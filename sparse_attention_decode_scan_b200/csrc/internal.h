@@ -58,7 +58,8 @@ struct TopkPlan {
   int64_t seg_len;
 };
 TopkPlan topk_plan(int32_t rows, int64_t n_cols);
-size_t topk_ws_bytes(int32_t rows, int64_t n_cols);
+size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t k);
+int topk_launches(int64_t n_cols);
 
 struct TopkArgs {
   const float* scores;
@@ -72,7 +73,6 @@ struct TopkArgs {
   DevStatus* status;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
-constexpr int kTopkLaunches = 5;
 
 // ---- sparse attention
 struct AttnArgs {

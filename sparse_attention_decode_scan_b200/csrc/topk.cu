@@ -1,6 +1,4 @@
-// Exact top-k of fp32 score rows: three radix-histogram passes (11 + 11 + 10
-// bits of an order-preserving 32-bit key) find the k-th largest key T, then a
-// count pass and an order-preserving compaction write the positions.
+// Exact top-k of fp32 score rows on an order-preserving 32-bit key.
 //
 // Keeps the k highest-scoring tokens of each row (MLI abstract, sentence 2):
 //   * -0.0 compares equal to +0.0 (canonicalised before the key transform);
@@ -8,9 +6,17 @@
 //   * among equal scores the lower position is kept;
 //   * the output holds min(k, #selectable) positions sorted ascending, then -1.
 //
-// Each row is cut into segments so that long rows with few rows (4 x 512K)
-// still spread over every SM; segments publish histograms and counts through
-// global memory between launches, so no kernel waits on another CTA.
+// Rows of up to 2^19 entries (every decode and prefill shape here) take three
+// launches: a 12-bit histogram over segments of every row (all SMs), a collect
+// pass that appends the positions above the threshold bin ("sure") and the
+// (key, position) pairs inside it ("candidates") to per-row lists, and one CTA
+// per row that finishes the radix select on the candidates in shared memory
+// and writes the positions in order through a position bitmap.  If a
+// threshold bin holds more candidates than the list keeps, that row's CTA
+// re-reads its row instead.  Longer rows use five launches of segment-parallel
+// radix passes (11 + 11 + 10 bits) with a count pass and an ordered compaction.
+// Segments publish histograms and counts through global memory between
+// launches, so no kernel waits on another CTA.
 #include <math.h>
 
 #include <mutex>
@@ -302,6 +308,324 @@ __global__ void __launch_bounds__(kT) k_topk_write(TopkArgs a, int64_t seg_len, 
   }
 }
 
+
+// ============================================================ three-launch path
+constexpr int kB1 = 4096;          // 12-bit first digit
+constexpr int kCandCap = 4096;     // candidates kept per row
+constexpr int64_t kMaxBitmapCols = 1 << 19;
+constexpr int kFinT = 1024;        // threads of the per-row CTA
+
+struct V2Layout {
+  uint32_t* hist;   // [rows][kB1]
+  uint32_t* cnt;    // [rows][2]: sure, candidates
+  int32_t* sure;    // [rows][k]
+  uint2* cand;      // [rows][kCandCap]: (key, position)
+};
+
+__device__ __forceinline__ V2Layout v2_layout(const TopkArgs& a) {
+  V2Layout L;
+  uint8_t* b = reinterpret_cast<uint8_t*>(a.ws);
+  L.hist = reinterpret_cast<uint32_t*>(b);
+  b += static_cast<size_t>(a.rows) * kB1 * 4;
+  L.cnt = reinterpret_cast<uint32_t*>(b);
+  b += (static_cast<size_t>(a.rows) * 8 + 255) / 256 * 256;
+  L.sure = reinterpret_cast<int32_t*>(b);
+  b += (static_cast<size_t>(a.rows) * a.k * 4 + 255) / 256 * 256;
+  L.cand = reinterpret_cast<uint2*>(b);
+  return L;
+}
+
+// Launch 1: histogram of key bits [31:20] per row.
+__global__ void __launch_bounds__(kT) k_tk_hist12(TopkArgs a, int64_t seg_len) {
+  __shared__ uint32_t h[kB1];
+  const int r = blockIdx.y, seg = blockIdx.x;
+  const Row rr = row_range(a, r, seg, seg_len);
+  if (rr.s0 >= rr.s1) return;
+  for (int i = threadIdx.x; i < kB1; i += kT) h[i] = 0;
+  __syncthreads();
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  for (int64_t base = rr.s0; base < rr.s1; base += kRound) {
+    uint32_t key[4];
+    load_keys(row, base, rr.s1, key);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (key[j]) atomicAdd(&h[key[j] >> 20], 1u);
+  }
+  __syncthreads();
+  uint32_t* dst = v2_layout(a).hist + static_cast<int64_t>(r) * kB1;
+  for (int i = threadIdx.x; i < kB1; i += kT)
+    if (h[i]) atomicAdd(dst + i, h[i]);
+}
+
+// Appends `pos` (or (key,pos)) for the lanes whose flag is set, with one
+// global atomic per warp.
+__device__ __forceinline__ uint32_t warp_append_base(bool flag, uint32_t* counter, uint32_t* my_off) {
+  const uint32_t m = __ballot_sync(0xffffffffu, flag);
+  if (!m) return 0;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(m) - 1;
+  uint32_t base = 0;
+  if (lane == leader) base = atomicAdd(counter, static_cast<uint32_t>(__popc(m)));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  *my_off = base + __popc(m & ((1u << lane) - 1u));
+  return m;
+}
+
+// Launch 2: threshold bin b1 of each row, then every key above it ("sure") and
+// inside it ("candidate") is appended to the row's lists.
+__global__ void __launch_bounds__(kT) k_tk_collect(TopkArgs a, int64_t seg_len) {
+  __shared__ int sh[kT / 32];
+  const int r = blockIdx.y, seg = blockIdx.x;
+  const Row rr = row_range(a, r, seg, seg_len);
+  if (rr.s0 >= rr.s1) return;
+  const V2Layout L = v2_layout(a);
+  const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
+  Found f = find_bin<kB1>(hist, 0xffffffffu, sh);
+  const uint32_t keff = f.total < static_cast<uint32_t>(a.k) ? f.total : static_cast<uint32_t>(a.k);
+  if (keff == 0) return;
+  f = find_bin<kB1>(hist, keff, sh);
+  const uint32_t b1 = static_cast<uint32_t>(f.bin);
+  uint32_t* cnt = L.cnt + 2 * r;
+  int32_t* sure = L.sure + static_cast<int64_t>(r) * a.k;
+  uint2* cand = L.cand + static_cast<int64_t>(r) * kCandCap;
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  for (int64_t base = rr.s0; base < rr.s1; base += kRound) {
+    uint32_t key[4];
+    load_keys(row, base, rr.s1, key);
+    const int64_t p = base + threadIdx.x * 4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t bin = key[j] >> 20;
+      const bool is_sure = key[j] != 0u && bin > b1;
+      const bool is_cand = key[j] != 0u && bin == b1;
+      uint32_t off;
+      if (warp_append_base(is_sure, &cnt[0], &off) && is_sure) {
+        if (off < static_cast<uint32_t>(a.k)) sure[off] = static_cast<int32_t>(p + j);
+        else record_error(a.status, LSA_ERR_BOUNDS, r, static_cast<int>(off));  // cannot happen
+      }
+      if (warp_append_base(is_cand, &cnt[1], &off) && is_cand && off < static_cast<uint32_t>(kCandCap))
+        cand[off] = make_uint2(key[j], static_cast<uint32_t>(p + j));
+    }
+  }
+}
+
+// Block-wide (kFinT threads) exclusive scan.
+__device__ __forceinline__ int fin_excl_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const int before = warp ? warp_sums[warp - 1] : 0;
+  *total = warp_sums[kFinT / 32 - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// Bin of the rank-th largest key in a 1024-bin shared histogram (one bin per
+// thread); returns the bin and the rank inside it through shared memory.
+__device__ __forceinline__ void fin_find(const uint32_t* h, uint32_t rank, int* warp_sums, int* out_bin,
+                                         uint32_t* out_rank) {
+  const int t = threadIdx.x;
+  const uint32_t v = h[t];
+  int tot;
+  const int excl = fin_excl_scan(static_cast<int>(v), warp_sums, &tot);
+  const uint32_t above = static_cast<uint32_t>(tot - excl) - v;  // keys in higher bins
+  if (v > 0 && above < rank && rank <= above + v) {
+    *out_bin = t;
+    *out_rank = rank - above;
+  }
+  __syncthreads();
+}
+
+// keeps the n lowest set bits of x
+__device__ __forceinline__ uint32_t low_bits(uint32_t x, int n) {
+  uint32_t y = 0;
+  for (int i = 0; i < n && x; ++i) {
+    const uint32_t b = x & (0u - x);
+    y |= b;
+    x ^= b;
+  }
+  return y;
+}
+
+// Launch 3: one CTA per row.  Finishes the select on the candidates (bits
+// [19:0], in shared memory; or by re-reading the row if the list overflowed),
+// marks the chosen positions in a bitmap and writes them in position order.
+__global__ void __launch_bounds__(kFinT) k_tk_final(TopkArgs a) {
+  extern __shared__ __align__(16) uint32_t fsm[];
+  __shared__ int warp_sums[32];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_rank;
+  __shared__ uint32_t h[1024];
+  const int r = blockIdx.x;
+  const int t = threadIdx.x;
+  const int64_t nwords = (a.n_cols + 31) / 32;
+  uint32_t* bm = fsm;               // selected positions
+  uint32_t* tb = fsm + nwords;      // positions equal to the threshold key
+  uint2* cs = reinterpret_cast<uint2*>(fsm + 2 * nwords);  // candidates: 2*nwords words keep 8-byte alignment
+  const V2Layout L = v2_layout(a);
+  int32_t* out = a.idx + static_cast<int64_t>(r) * a.k;
+  int64_t n = a.n_cols;
+  if (a.valid_len) {
+    const int64_t v = __ldg(a.valid_len + r);
+    n = v < 0 ? 0 : (v < n ? v : n);
+  }
+  // keff and the threshold bin from the 12-bit histogram
+  const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
+  uint32_t tot = 0;
+  for (int i = t; i < kB1; i += kFinT) tot += __ldcg(hist + i);
+  int tt;
+  fin_excl_scan(static_cast<int>(tot), warp_sums, &tt);
+  const uint32_t keff = static_cast<uint32_t>(tt) < static_cast<uint32_t>(a.k) ? static_cast<uint32_t>(tt)
+                                                                               : static_cast<uint32_t>(a.k);
+  for (int i = static_cast<int>(keff) + t; i < a.k; i += kFinT) out[i] = -1;
+  if (keff == 0) return;
+  // bin b1 (4 bins per thread)
+  {
+    uint32_t v[4], mine = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[i] = __ldcg(hist + t * 4 + i);
+      mine += v[i];
+    }
+    int total;
+    const int excl = fin_excl_scan(static_cast<int>(mine), warp_sums, &total);
+    uint32_t cum = static_cast<uint32_t>(total - excl) - mine;
+    if (cum < keff && keff <= cum + mine) {
+      for (int i = 3; i >= 0; --i) {
+        if (cum + v[i] >= keff) {
+          s_bin = t * 4 + i;
+          s_rank = keff - cum;
+          break;
+        }
+        cum += v[i];
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t b1 = static_cast<uint32_t>(s_bin);
+  const uint32_t rank1 = s_rank;           // wanted rank inside bin b1
+  const uint32_t n_sure = keff - rank1;    // keys above bin b1
+  const uint32_t n_cand = __ldcg(L.cnt + 2 * r + 1);
+  const bool overflow = n_cand > static_cast<uint32_t>(kCandCap);
+  for (int64_t w = t; w < 2 * nwords; w += kFinT) fsm[w] = 0;
+  const int nc = overflow ? 0 : static_cast<int>(n_cand);
+  for (int c = t; c < nc; c += kFinT) cs[c] = __ldcg(L.cand + static_cast<int64_t>(r) * kCandCap + c);
+  __syncthreads();
+  const int32_t* sure = L.sure + static_cast<int64_t>(r) * a.k;
+  for (uint32_t i = t; i < n_sure; i += kFinT) {
+    const int32_t p = __ldcg(sure + i);
+    atomicOr(&bm[p >> 5], 1u << (p & 31));
+  }
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  // radix select on bits [19:10] then [9:0] among the keys of bin b1
+  uint32_t T = 0, ties = 0;
+  for (int pass = 0; pass < 2; ++pass) {
+    h[t] = 0;
+    __syncthreads();
+    const uint32_t shift = pass == 0 ? 10 : 0;
+    const uint32_t pre_shift = pass == 0 ? 20 : 10;
+    const uint32_t prefix = pass == 0 ? b1 : (T >> 10);
+    if (!overflow) {
+      for (int c = t; c < nc; c += kFinT) {
+        const uint32_t key = cs[c].x;
+        if ((key >> pre_shift) == prefix) atomicAdd(&h[(key >> shift) & 1023u], 1u);
+      }
+    } else {
+      for (int64_t base = 0; base < n; base += kFinT * 4) {
+        const int64_t p = base + t * 4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (p + j >= n) break;
+          const uint32_t key = order_key(__ldg(row + p + j));
+          if (key && (key >> pre_shift) == prefix) atomicAdd(&h[(key >> shift) & 1023u], 1u);
+        }
+      }
+    }
+    __syncthreads();
+    if (t == 0) s_bin = -1;
+    __syncthreads();
+    fin_find(h, pass == 0 ? rank1 : ties, warp_sums, &s_bin, &s_rank);
+    const uint32_t bb = static_cast<uint32_t>(s_bin);
+    if (pass == 0) {
+      T = (b1 << 20) | (bb << 10);
+      ties = s_rank;
+    } else {
+      T |= bb;
+      ties = s_rank;
+    }
+    __syncthreads();
+  }
+  // mark keys of bin b1 above T, and collect the keys equal to T
+  if (!overflow) {
+    for (int c = t; c < nc; c += kFinT) {
+      const uint2 e = cs[c];
+      if (e.x > T) atomicOr(&bm[e.y >> 5], 1u << (e.y & 31));
+      else if (e.x == T) atomicOr(&tb[e.y >> 5], 1u << (e.y & 31));
+    }
+  } else {
+    for (int64_t base = 0; base < n; base += kFinT * 4) {
+      const int64_t p = base + t * 4;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (p + j >= n) break;
+        const uint32_t key = order_key(__ldg(row + p + j));
+        if ((key >> 20) != b1) continue;
+        const uint32_t q = static_cast<uint32_t>(p + j);
+        if (key > T) atomicOr(&bm[q >> 5], 1u << (q & 31));
+        else if (key == T) atomicOr(&tb[q >> 5], 1u << (q & 31));
+      }
+    }
+  }
+  __syncthreads();
+  // ordered compaction: the lowest `ties` positions equal to T join the selection
+  const int64_t per = (nwords + kFinT - 1) / kFinT;
+  const int64_t w0 = t * per, w1 = (w0 + per < nwords) ? w0 + per : nwords;
+  int my_ties = 0;
+  for (int64_t w = w0; w < w1; ++w) my_ties += __popc(tb[w]);
+  int tie_tot;
+  int tie_before = fin_excl_scan(my_ties, warp_sums, &tie_tot);
+  int my_sel = 0;
+  for (int64_t w = w0; w < w1; ++w) {
+    const uint32_t x = tb[w];
+    const int px = __popc(x);
+    const int take = static_cast<int>(ties) - tie_before;
+    uint32_t add = 0;
+    if (take > 0) add = take >= px ? x : low_bits(x, take);
+    tie_before += px;
+    const uint32_t merged = bm[w] | add;
+    bm[w] = merged;
+    my_sel += __popc(merged);
+  }
+  int sel_tot;
+  int o = fin_excl_scan(my_sel, warp_sums, &sel_tot);
+  for (int64_t w = w0; w < w1; ++w) {
+    uint32_t x = bm[w];
+    while (x) {
+      const int b = __ffs(x) - 1;
+      x &= x - 1;
+      if (o < a.k) out[o] = static_cast<int32_t>(w * 32 + b);
+      else record_error(a.status, LSA_ERR_BOUNDS, r, o);  // cannot happen
+      ++o;
+    }
+  }
+}
+
 }  // namespace
 
 TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
@@ -321,19 +645,45 @@ TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
   return p;
 }
 
-size_t topk_ws_bytes(int32_t rows, int64_t n_cols) {
+bool topk_v2_ok(int64_t n_cols) { return n_cols <= kMaxBitmapCols; }
+
+size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t k) {
+  const size_t R = static_cast<size_t>(rows);
+  if (topk_v2_ok(n_cols)) {
+    const size_t b = R * kB1 * 4 + (R * 8 + 255) / 256 * 256 + (R * k * 4 + 255) / 256 * 256 + R * kCandCap * 8;
+    return (b + 255) / 256 * 256;
+  }
   TopkPlan p = topk_plan(rows, n_cols);
-  size_t b = static_cast<size_t>(rows) * kHistStride * 4 + static_cast<size_t>(rows) * p.nseg * 8;
+  size_t b = R * kHistStride * 4 + R * p.nseg * 8;
   return (b + 255) / 256 * 256;
 }
+
+int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 3 : 5; }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   if (a.rows == 0 || a.k == 0) return cudaSuccess;
   TopkPlan p = topk_plan(a.rows, a.n_cols);
+  dim3 grid(static_cast<unsigned>(p.nseg), static_cast<unsigned>(a.rows));
+  if (topk_v2_ok(a.n_cols)) {
+    const size_t zero = static_cast<size_t>(a.rows) * kB1 * 4 + (static_cast<size_t>(a.rows) * 8 + 255) / 256 * 256;
+    cudaError_t e = cudaMemsetAsync(a.ws, 0, zero, s);
+    if (e != cudaSuccess) return e;
+    k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
+    k_tk_collect<<<grid, kT, 0, s>>>(a, p.seg_len);
+    const int64_t nwords = (a.n_cols + 31) / 32;
+    const size_t smem = 2 * nwords * 4 + static_cast<size_t>(kCandCap) * 8;
+    static size_t smem_set = 0;
+    if (smem > 48 * 1024 && smem > smem_set) {
+      e = cudaFuncSetAttribute(k_tk_final, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      smem_set = smem;
+    }
+    k_tk_final<<<a.rows, kFinT, smem, s>>>(a);
+    return cudaGetLastError();
+  }
   size_t hist_bytes = static_cast<size_t>(a.rows) * kHistStride * 4;
   cudaError_t e = cudaMemsetAsync(a.ws, 0, hist_bytes, s);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(p.nseg), static_cast<unsigned>(a.rows));
   k_topk_hist<1><<<grid, kT, 0, s>>>(a, p.seg_len);
   k_topk_hist<2><<<grid, kT, 0, s>>>(a, p.seg_len);
   k_topk_hist<3><<<grid, kT, 0, s>>>(a, p.seg_len);
@@ -393,7 +743,7 @@ extern "C" lsa_status lsa_topk_noalloc(const float* scores, int64_t ld, int32_t 
   if (rows < 0 || k < 1 || n_cols < 0 || ld < n_cols || (ld % 4) != 0) return LSA_ERR_INVALID_ARG;
   if (rows > 0 && (!scores || !idx || (reinterpret_cast<uintptr_t>(scores) & 15u) != 0)) return LSA_ERR_INVALID_ARG;
   if (n_cols > (1LL << 31) - 1) return LSA_ERR_UNSUPPORTED;
-  const size_t need = kStatusBytes + topk_ws_bytes(rows, n_cols);
+  const size_t need = kStatusBytes + topk_ws_bytes(rows, n_cols, k);
   if (need > kStaticScratchBytes) return LSA_ERR_UNSUPPORTED;  // beyond the static scratch
   if (rows == 0) return LSA_OK;
   void* base = nullptr;

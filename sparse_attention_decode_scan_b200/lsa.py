@@ -105,6 +105,13 @@ def workspace_size(dims: Optional[Dims], rows: int, max_len: int, op: int) -> in
     return int(lib().lsa_workspace_size(ctypes.byref(dims) if dims is not None else None, rows, max_len, op))
 
 
+def topk_workspace_size(rows: int, n_cols: int, k: int) -> int:
+    """Workspace bytes of lsa_topk for these sizes (only k of the dims is read)."""
+    d = Dims()
+    d.top_k = int(k)
+    return workspace_size(d, rows, n_cols, LSA_OP_TOPK)
+
+
 def workspace(nbytes: int, device="cuda"):
     """A zero-filled, 256-byte aligned workspace tensor (torch's allocator aligns to 512 B)."""
     import torch

@@ -64,7 +64,8 @@ def test_workspace_sizes(lsa):
     # at least: status + fp32 scores + selection
     assert step >= 256 + 32 * 131072 * 4 + 32 * 2048 * 4
     assert step % 256 == 0
-    assert lsa.workspace_size(None, 4, 524288, lsa.LSA_OP_TOPK) > 0
+    assert lsa.topk_workspace_size(4, 524288, 2048) > 0
+    assert lsa.workspace_size(None, 4, 524288, lsa.LSA_OP_TOPK) == 0
     assert lsa.workspace_size(_dims(lsa, n_idx_heads=0), 1, 10, lsa.LSA_OP_DECODE_STEP) == 0
     assert lsa.workspace_size(d, -1, 10, lsa.LSA_OP_ATTN) == 0
     assert lsa.workspace_size(d, 1, 10, 99) == 0

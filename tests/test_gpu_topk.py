@@ -51,7 +51,7 @@ def test_topk_exact(kind, rows, n, k, mode):
     dev[:, :n] = torch.from_numpy(sc).cuda()
     vdev = torch.from_numpy(valid).cuda() if valid is not None else None
     idx = torch.full((rows, k), -7, dtype=torch.int32, device="cuda")
-    ws = lsa.workspace(lsa.workspace_size(None, rows, n, lsa.LSA_OP_TOPK))
+    ws = lsa.workspace(lsa.topk_workspace_size(rows, n, k))
     lsa.topk(dev, k, idx, ws, valid_len=vdev, n_cols=n, ld=ld)
     torch.cuda.synchronize()
     assert lsa.read_device_status(ws) == lsa.LSA_OK
@@ -68,7 +68,7 @@ def test_topk_repeatable_and_workspace_reuse():
     rows, n, k = 6, 50000, 2048
     sc = synth.topk_scores("ties", rows, n, 31)
     dev = torch.from_numpy(sc).cuda()
-    ws = lsa.workspace(lsa.workspace_size(None, rows, n, lsa.LSA_OP_TOPK))
+    ws = lsa.workspace(lsa.topk_workspace_size(rows, n, k))
     outs = []
     for _ in range(3):
         idx = torch.empty((rows, k), dtype=torch.int32, device="cuda")

@@ -22,7 +22,7 @@ def _both(sc: np.ndarray, k: int, valid=None):
     dev = torch.from_numpy(sc).cuda()
     vdev = torch.from_numpy(valid).cuda() if valid is not None else None
     ref = torch.full((rows, k), -7, dtype=torch.int32, device="cuda")
-    ws = lsa.workspace(lsa.workspace_size(None, rows, n, lsa.LSA_OP_TOPK))
+    ws = lsa.workspace(lsa.topk_workspace_size(rows, n, k))
     lsa.topk(dev, k, ref, ws, valid_len=vdev)
     got = torch.full((rows, k), -7, dtype=torch.int32, device="cuda")
     lsa.topk_noalloc(dev, k, got, valid_len=vdev)
