@@ -271,7 +271,19 @@ def run_ours(args, world, rank, local):
             lsa.topk(scores, s.top_k, idx, ws, valid_len=None if prefill else dc.seq_lens,
                      n_cols=L if prefill else dc.max_len, ld=ld, stream=stream)
 
+    # The decode step runs through the public one-call entry point (its scan
+    # also builds the top-k's first histogram); the profiled variant records
+    # the phase-boundary events inside it.
+    use_step_api = (not prefill) and args.op == "step"
+
     def step(ev=None):
+        if use_step_api:
+            if ev is None:
+                lsa.decode_step(dc.dims, dc.cache, dc.q_idx, dc.w, dc.q, out, lse, ws, idx_out=idx, stream=stream)
+            else:
+                lsa.decode_step_profiled(dc.dims, dc.cache, dc.q_idx, dc.w, dc.q, out, lse, ws, ev, idx_out=idx,
+                                         stream=stream)
+            return
         if ev is not None:
             ev[0].record(stream)
         if run_scan:
@@ -300,6 +312,10 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     assert lsa.read_device_status(ws) == lsa.LSA_OK
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for e4 in evs:  # create the CUDA events (torch creates them at first record)
+        for e in e4:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
     with ClockSampler(gpu_index) as clk:
@@ -393,8 +409,13 @@ def run_ours(args, world, rank, local):
         unit = "steps/s"
     step_gbs = nb["total"] / (ms_per_step / 1e3) / 1e9
     # launches of our kernels per step, as the library plans them for these sizes
-    per_step = sum(lsa.launch_count(dc.dims, R, dc.max_len, op, causal=prefill)
-                   for op in (lsa.LSA_OP_SCORES, lsa.LSA_OP_TOPK, lsa.LSA_OP_ATTN))
+    if use_step_api:
+        per_step = lsa.launch_count(dc.dims, R, dc.max_len, lsa.LSA_OP_DECODE_STEP)
+    else:
+        per_step = sum(lsa.launch_count(dc.dims, R, dc.max_len, op, causal=prefill)
+                       for op in (lsa.LSA_OP_SCORES, lsa.LSA_OP_TOPK, lsa.LSA_OP_ATTN)
+                       if (op, args.op) in ((lsa.LSA_OP_SCORES, "scan"), (lsa.LSA_OP_TOPK, "topk"),
+                                            (lsa.LSA_OP_ATTN, "attn")) or args.op == "step")
     launches = per_step * args.steps
 
     cpu = None

@@ -182,6 +182,19 @@ lsa_status lsa_decode_step(const lsa_dims* d, const lsa_cache* c, const void* q_
                            void* ws, size_t ws_bytes, lsa_stream_t stream);
 
 /*
+ * lsa_decode_step that also records CUDA events on `stream` at its phase
+ * boundaries, for profiling: events[0] before the scan, events[1] after the
+ * scan, events[2] after the top-k, events[3] after the sparse attention.
+ * `events` is an array of 4 cudaEvent_t (NULL entries are skipped) or NULL.
+ * Results, workspace and errors as lsa_decode_step (LSA_ERR_CUDA if an event
+ * record fails).
+ */
+lsa_status lsa_decode_step_profiled(const lsa_dims* d, const lsa_cache* c, const void* q_idx,
+                                    const float* w, const void* q, void* out, float* lse,
+                                    int32_t* idx_out, int32_t flags, void* ws, size_t ws_bytes,
+                                    lsa_stream_t stream, void* const* events);
+
+/*
  * Copies the workspace status word to *status (an lsa_status value), clears it,
  * and synchronises `stream`.  Returns LSA_ERR_CUDA if a CUDA call fails.
  */

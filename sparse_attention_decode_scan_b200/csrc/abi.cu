@@ -112,7 +112,8 @@ inline DevStatus* status_of(void* ws) { return reinterpret_cast<DevStatus*>(ws);
 
 lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
                      const int32_t* row_pos, const void* q_idx, const float* w, float* scores,
-                     int64_t ld, void* ws, void* inner_ws, size_t inner_bytes, cudaStream_t s) {
+                     int64_t ld, void* ws, void* inner_ws, size_t inner_bytes, cudaStream_t s,
+                     uint32_t* hist12 = nullptr, bool* hist_done = nullptr) {
   ScoresArgs a;
   a.cache = view(d, c);
   a.key_dtype = d->idx_key_dtype;
@@ -129,13 +130,24 @@ lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const 
   a.status = status_of(ws);
   a.plan_ws = inner_ws;
   a.plan_bytes = inner_bytes;
+  a.hist12 = nullptr;
+  if (hist_done) *hist_done = false;
   if (rows == 0 || ld == 0) return LSA_OK;
-  if (!force_simt() && scores_tc_supported(a)) return cuda_status(launch_scores_tc(a, s));
+  if (!force_simt() && scores_tc_supported(a)) {
+    if (hist12 && scores_tc_fused_hist_ok(a)) {
+      // the scan also counts the first top-k digit; the counters start at zero
+      cudaError_t e = cudaMemsetAsync(hist12, 0, topk_hist_zero_bytes(rows), s);
+      if (e != cudaSuccess) return LSA_ERR_CUDA;
+      a.hist12 = hist12;
+      if (hist_done) *hist_done = true;
+    }
+    return cuda_status(launch_scores_tc(a, s));
+  }
   return cuda_status(launch_scores_simt(a, s));
 }
 
 lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
-                   int32_t k, int32_t* idx, void* ws, void* inner_ws, cudaStream_t s) {
+                   int32_t k, int32_t* idx, void* ws, void* inner_ws, cudaStream_t s, bool hist_ready = false) {
   TopkArgs a;
   a.scores = scores;
   a.ld = ld;
@@ -146,6 +158,7 @@ lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t*
   a.idx = idx;
   a.ws = inner_ws;
   a.status = status_of(ws);
+  a.hist_ready = hist_ready;
   return cuda_status(launch_topk(a, s));
 }
 
@@ -246,9 +259,9 @@ lsa_status lsa_sparse_attn_decode(const lsa_dims* d, const lsa_cache* c, int32_t
                  ws_bytes - kStatusBytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
-lsa_status lsa_decode_step(const lsa_dims* d, const lsa_cache* c, const void* q_idx, const float* w,
-                           const void* q, void* out, float* lse, int32_t* idx_out, int32_t flags, void* ws,
-                           size_t ws_bytes, lsa_stream_t stream) {
+static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const void* q_idx, const float* w,
+                                   const void* q, void* out, float* lse, int32_t* idx_out, int32_t flags, void* ws,
+                                   size_t ws_bytes, lsa_stream_t stream, void* const* events) {
   if (!valid_dims(d) || !valid_cache(d, c, true, true)) return LSA_ERR_INVALID_ARG;
   if (flags != LSA_STEP_UNFUSED && flags != LSA_STEP_FUSED) return LSA_ERR_INVALID_ARG;
   const int32_t B = c->batch;
@@ -260,17 +273,43 @@ lsa_status lsa_decode_step(const lsa_dims* d, const lsa_cache* c, const void* q_
   if (st != LSA_OK) return st;
   if (B == 0) return LSA_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) -> bool {
+    if (!events || !events[i]) return true;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s) == cudaSuccess;
+  };
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* scores = reinterpret_cast<float*>(base + L.scores_off);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + L.idx_off);
   void* inner = base + L.inner_off;
   const size_t inner_bytes = L.total - L.inner_off;
   const int64_t ld = score_ld(c->max_len);
-  st = do_scores(d, c, B, nullptr, nullptr, q_idx, w, scores, ld, ws, inner, inner_bytes, s);
+  // With the tensor-core scan and the three-launch top-k, the scan writes the
+  // top-k's first histogram into the top-k workspace (which starts with it).
+  uint32_t* hist12 = (!force_simt() && topk_v2_ok(c->max_len)) ? static_cast<uint32_t*>(inner) : nullptr;
+  bool hist_done = false;
+  if (!mark(0)) return LSA_ERR_CUDA;
+  st = do_scores(d, c, B, nullptr, nullptr, q_idx, w, scores, ld, ws, inner, inner_bytes, s, hist12, &hist_done);
   if (st != LSA_OK) return st;
-  st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, s);
+  if (!mark(1)) return LSA_ERR_CUDA;
+  st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, s, hist_done);
   if (st != LSA_OK) return st;
-  return do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s);
+  if (!mark(2)) return LSA_ERR_CUDA;
+  st = do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s);
+  if (st != LSA_OK) return st;
+  if (!mark(3)) return LSA_ERR_CUDA;
+  return LSA_OK;
+}
+
+lsa_status lsa_decode_step(const lsa_dims* d, const lsa_cache* c, const void* q_idx, const float* w,
+                           const void* q, void* out, float* lse, int32_t* idx_out, int32_t flags, void* ws,
+                           size_t ws_bytes, lsa_stream_t stream) {
+  return decode_step_impl(d, c, q_idx, w, q, out, lse, idx_out, flags, ws, ws_bytes, stream, nullptr);
+}
+
+lsa_status lsa_decode_step_profiled(const lsa_dims* d, const lsa_cache* c, const void* q_idx, const float* w,
+                                    const void* q, void* out, float* lse, int32_t* idx_out, int32_t flags,
+                                    void* ws, size_t ws_bytes, lsa_stream_t stream, void* const* events) {
+  return decode_step_impl(d, c, q_idx, w, q, out, lse, idx_out, flags, ws, ws_bytes, stream, events);
 }
 
 lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream) {
@@ -303,7 +342,11 @@ int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32
     case LSA_OP_SCORES: return scan;
     case LSA_OP_TOPK: return topk_launches(max_len);
     case LSA_OP_ATTN: return attn;
-    case LSA_OP_DECODE_STEP: return scan + topk_launches(max_len) + attn;
+    case LSA_OP_DECODE_STEP: {
+      const bool fused = !simt && topk_v2_ok(max_len) &&
+                         scores_tc_shape_ok(d->idx_key_dtype, d->act_dtype, d->n_idx_heads, d->idx_dim, d->block_size);
+      return scan + topk_launches(max_len) - (fused ? 1 : 0) + attn;
+    }
     default: return -1;
   }
 }

@@ -104,6 +104,18 @@ struct CacheAddr {
   }
 };
 
+// Order-preserving 32-bit key of a score (larger score -> larger key).  -0.0
+// maps like +0.0; -inf and NaN map to 0, the key that is never selected.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (!(f == f) || f == -INFINITY) return 0u;
+  uint32_t u = __float_as_uint(f);
+  if (f == 0.f) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Bins of the first top-k digit (key bits [31:20]).
+constexpr int kTopkBins1 = 4096;
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -53,7 +53,9 @@ struct Cfg {
   static constexpr int kQBytes = kKBlocks * kQKBlockBytes;
   static constexpr int kNQ = QB == 1 ? 2 : 1;                      // query operand buffers
   static constexpr int kWBytes = QB * kHeads * 4;
-  static constexpr int kFixed = kNQ * kQBytes + kNQ * kWBytes + 1024 /*barriers, scratch*/ + 1024 /*align*/;
+  static constexpr int kHistBytes = QB == 1 ? kTopkBins1 * 4 : 0;  // fused first top-k histogram (decode)
+  static constexpr int kFixed = kNQ * kQBytes + kNQ * kWBytes + kHistBytes + 1024 /*barriers, scratch*/ +
+                                1024 /*align*/;
   static constexpr int kNSmax = (kSmemLimit - kFixed) / kTileBytes;
   static constexpr int kNS = kNSmax > 8 ? 8 : kNSmax;              // key stages
   static constexpr int kAccCols = kN;
@@ -290,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
   uint8_t* stages = smem;
   uint8_t* qbufs = stages + C::kNS * C::kTileBytes;
   float* wbufs = reinterpret_cast<float*>(qbufs + C::kNQ * C::kQBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(wbufs) + C::kNQ * C::kWBytes);
+  uint32_t* shist = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(wbufs) + C::kNQ * C::kWBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(shist) + C::kHistBytes);
   uint64_t* full = bars;
   uint64_t* empty = full + C::kNS;
   uint64_t* qfull = empty + C::kNS;
@@ -298,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
   uint64_t* tfull = qempty + C::kNQ;
   uint64_t* tempty = tfull + 2;
   uint64_t* done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* ebar = done + 1;  // epilogue warps' rendezvous around histogram flushes
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* sfound = const_cast<int*>(abort_flag) + 1;                       // 2 ints
   int64_t* sbuf = reinterpret_cast<int64_t*>(sfound + 2 + 1);           // kThreads/32 int64 (8-aligned below)
@@ -319,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
       tc::mbar_init(&tempty[s], 4);
     }
     tc::mbar_init(done, 1);
+    tc::mbar_init(ebar, 4);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -334,42 +339,73 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
   CacheAddr ad{a.cache.block_table, a.cache.max_blocks, a.cache.block_size, a.cache.n_blocks, a.cache.max_len};
 
   if (warp == kWarpProd) {
-    if (lane == 0 && plan.n_items > 0) {
-      Walker<QB> W;
-      W.start(a, plan.r_first, plan.j_first);
+    // The whole warp looks up the block-table rows of 32 tiles at a time (one
+    // tile per lane, next batch loaded while this one is issued); lane 0 issues
+    // the TMA loads.  A single thread doing the lookups serially would wait one
+    // global-load latency per tile.
+    if (plan.n_items > 0) {
+      Walker<QB> Wb;
+      Wb.start(a, plan.r_first, plan.j_first);
+      auto lookup = [&](const Walker<QB>& base, int64_t base_item, int64_t* r0, int64_t* r1) {
+        Walker<QB> w = base;
+        for (int i = 0; i < lane; ++i) w.next(a);
+        *r0 = -2;
+        *r1 = -2;  // -2: no such item
+        if (base_item + lane < plan.n_items) {
+          const int64_t p0 = static_cast<int64_t>(w.j) * kTile;
+          *r0 = p0 < w.g.vis ? ad.row(w.g.b, p0) : -3;             // -3: past the visible range
+          *r1 = p0 + kBoxRows < w.g.vis ? ad.row(w.g.b, p0 + kBoxRows) : -3;
+          if (*r0 == -1) record_error(a.status, LSA_ERR_BOUNDS, w.g.r0, static_cast<int>(p0));
+          if (*r1 == -1) record_error(a.status, LSA_ERR_BOUNDS, w.g.r0, static_cast<int>(p0 + kBoxRows));
+        }
+      };
+      int64_t cur0, cur1;
+      lookup(Wb, 0, &cur0, &cur1);
       int64_t it = 0;
-      for (; it < plan.n_items; ++it) {
-        const int s = static_cast<int>(it % C::kNS);
-        const uint32_t ph = static_cast<uint32_t>((it / C::kNS) & 1);
-        if (!tc::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
-          record_error(a.status, LSA_ERR_TIMEOUT, 0, 1);
-          *abort_flag = 1;
-          break;
-        }
-        int64_t rows[2] = {-1, -1};
-        uint32_t bytes = 0;
-        for (int h = 0; h < 2; ++h) {
-          const int64_t p = static_cast<int64_t>(W.j) * kTile + h * kBoxRows;
-          if (p < W.g.vis) {
-            rows[h] = ad.row(W.g.b, p);
-            if (rows[h] >= 0) bytes += C::kKBlocks * C::kBoxBytes;
-            else record_error(a.status, LSA_ERR_BOUNDS, W.g.r0, static_cast<int>(p));
+      bool failed = false;
+      for (int64_t base_item = 0; base_item < plan.n_items && !failed; base_item += 32) {
+        Walker<QB> Wn = Wb;
+        for (int i = 0; i < 32; ++i) Wn.next(a);
+        int64_t nxt0 = -2, nxt1 = -2;
+        if (base_item + 32 < plan.n_items) lookup(Wn, base_item + 32, &nxt0, &nxt1);
+        const int nb = static_cast<int>(plan.n_items - base_item < 32 ? plan.n_items - base_item : 32);
+        for (int i = 0; i < nb; ++i) {
+          const int64_t rows[2] = {__shfl_sync(0xffffffffu, cur0, i), __shfl_sync(0xffffffffu, cur1, i)};
+          if (lane == 0) {
+            const int s = static_cast<int>(it % C::kNS);
+            const uint32_t ph = static_cast<uint32_t>((it / C::kNS) & 1);
+            if (!tc::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 1);
+              *abort_flag = 1;
+              failed = true;
+            } else {
+              uint32_t bytes = 0;
+              for (int h = 0; h < 2; ++h)
+                if (rows[h] >= 0) bytes += C::kKBlocks * C::kBoxBytes;
+              tc::mbar_arrive_expect_tx(&full[s], bytes);
+              uint8_t* st = stages + s * C::kTileBytes;
+              for (int h = 0; h < 2; ++h) {
+                if (rows[h] < 0) continue;
+                for (int kb = 0; kb < C::kKBlocks; ++kb)
+                  tc::tma_load_2d(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * 64,
+                                  static_cast<int32_t>(rows[h]), &full[s]);
+              }
+              ++it;
+            }
           }
+          failed = __shfl_sync(0xffffffffu, failed, 0);
+          if (failed) break;
         }
-        tc::mbar_arrive_expect_tx(&full[s], bytes);
-        uint8_t* st = stages + s * C::kTileBytes;
-        for (int h = 0; h < 2; ++h) {
-          if (rows[h] < 0) continue;
-          for (int kb = 0; kb < C::kKBlocks; ++kb)
-            tc::tma_load_2d(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * 64,
-                            static_cast<int32_t>(rows[h]), &full[s]);
-        }
-        W.next(a);
+        Wb = Wn;
+        cur0 = nxt0;
+        cur1 = nxt1;
       }
       // drain: the last load of every stage must land before the CTA exits
-      const int64_t n_issued = it;
-      for (int64_t i = n_issued > C::kNS ? n_issued - C::kNS : 0; i < n_issued; ++i)
-        tc::mbar_wait(&full[i % C::kNS], static_cast<uint32_t>((i / C::kNS) & 1), nullptr);
+      if (lane == 0) {
+        const int64_t n_issued = it;
+        for (int64_t i = n_issued > C::kNS ? n_issued - C::kNS : 0; i < n_issued; ++i)
+          tc::mbar_wait(&full[i % C::kNS], static_cast<uint32_t>((i / C::kNS) & 1), nullptr);
+      }
     }
   } else if (warp == kWarpMma) {
     if (lane == 0 && plan.n_items > 0) {
@@ -449,10 +485,38 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
     const int quarter = warp & 3;
     const int t = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    // Decode with a histogram target: the epilogue also counts each score's
+    // top-k digit (key bits [31:20]) in shared memory and adds the counts of a
+    // row to hist12 when the CTA leaves that row, so the top-k skips one pass.
+    const bool use_hist = QB == 1 && a.hist12 != nullptr;
+    const int et = threadIdx.x - kWarpEpi * 32;  // 0..127
+    int ephase = 0;
+    auto epi_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(ebar);
+      const bool ok = tc::mbar_wait(ebar, static_cast<uint32_t>(ephase & 1), abort_flag);
+      ++ephase;
+      return ok;
+    };
+    auto flush_hist = [&](int row) -> bool {
+      if (!epi_sync()) return false;
+      uint32_t* dst = a.hist12 + static_cast<int64_t>(row) * kTopkBins1;
+      for (int i = et; i < kTopkBins1; i += 128) {
+        const uint32_t v = shist[i];
+        if (v) {
+          atomicAdd(dst + i, v);
+          shist[i] = 0;
+        }
+      }
+      return epi_sync();
+    };
+    if (use_hist)
+      for (int i = et; i < kTopkBins1; i += 128) shist[i] = 0;
     if (plan.n_items > 0) {
       Walker<QB> W;
       W.start(a, plan.r_first, plan.j_first);
       int gi = -1, qi = 0;
+      int hist_row = -1;
       int64_t vis_r[QB];
       // The block-table lookup (and FP8 scale) of a tile is loaded one tile
       // ahead, so its latency overlaps the wait for the accumulator.
@@ -468,11 +532,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
         if (it == 0 || W.j == 0) {
           ++gi;
           qi = gi % C::kNQ;
+          if (use_hist && hist_row >= 0 && !flush_hist(hist_row)) {
+            if (lane == 0) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 6);
+              *abort_flag = 1;
+            }
+            hist_row = -1;
+            break;
+          }
+          hist_row = W.g.r0;
           if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) {
             if (lane == 0) {
               record_error(a.status, LSA_ERR_TIMEOUT, 0, 4);
               *abort_flag = 1;
             }
+            hist_row = -1;
             break;
           }
 #pragma unroll
@@ -487,6 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
             record_error(a.status, LSA_ERR_TIMEOUT, 0, 5);
             *abort_flag = 1;
           }
+          hist_row = -1;
           break;
         }
         tc::tc_fence_after();
@@ -520,6 +595,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+        if (use_hist && p < vis_r[0] && prow >= 0) {
+          const uint32_t key = order_key(sc[0]);
+          if (key) atomicAdd(&shist[key >> 20], 1u);
+        }
 #pragma unroll
         for (int qq = 0; qq < QB; ++qq) {
           if (qq < W.g.nrows && p < a.ld) {
@@ -535,6 +614,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
         }
         W.next(a);
         if (it + 1 < plan.n_items) prefetch(W);
+      }
+      if (use_hist && hist_row >= 0 && !flush_hist(hist_row) && lane == 0) {
+        record_error(a.status, LSA_ERR_TIMEOUT, 0, 7);
+        *abort_flag = 1;
       }
     }
     // tails: positions past each row's group tiles are -inf (NaN for an invalid row)
@@ -638,6 +721,8 @@ bool scores_tc_supported(const ScoresArgs& a) {
 }
 
 size_t scores_tc_ws_bytes(int32_t, bool) { return 0; }
+
+bool scores_tc_fused_hist_ok(const ScoresArgs& a) { return a.row_pos == nullptr && scores_tc_supported(a); }
 
 cudaError_t launch_scores_tc(const ScoresArgs& a, cudaStream_t s) {
   const bool causal = a.row_pos != nullptr;

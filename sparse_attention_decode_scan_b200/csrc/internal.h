@@ -41,6 +41,8 @@ struct ScoresArgs {
   DevStatus* status;
   void* plan_ws;       // tensor-core path scratch (row groups), may be null
   size_t plan_bytes;
+  uint32_t* hist12;    // if set: per-row histogram of score-key bits [31:20] ([rows][4096],
+                       // zeroed by the caller), accumulated by the scan for the top-k
 };
 
 // ---- indexer
@@ -71,8 +73,16 @@ struct TopkArgs {
   int32_t* idx;
   void* ws;            // topk_ws_bytes bytes (256-aligned)
   DevStatus* status;
+  bool hist_ready;     // the first histogram and list counters are already in ws
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+// The three-launch top-k applies (rows up to 2^19 entries); its first
+// histogram then sits at the start of the top-k workspace, followed by the
+// list counters; topk_hist_zero_bytes of them must be zero before the scan.
+bool topk_v2_ok(int64_t n_cols);
+size_t topk_hist_zero_bytes(int32_t rows);
+// true if the scan can accumulate the top-k histogram itself
+bool scores_tc_fused_hist_ok(const ScoresArgs& a);
 
 // ---- sparse attention
 struct AttnArgs {

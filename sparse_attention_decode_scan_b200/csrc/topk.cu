@@ -32,12 +32,6 @@ constexpr int kRound = kT * 4;     // elements per round (one float4 per thread)
 constexpr int kBins1 = 2048, kBins2 = 2048, kBins3 = 1024;
 constexpr int kHistStride = kBins1 + kBins2 + kBins3;
 
-__device__ __forceinline__ uint32_t order_key(float f) {
-  if (!(f == f) || f == -INFINITY) return 0u;  // NaN, -inf: never selectable
-  uint32_t u = __float_as_uint(f);
-  if (f == 0.f) u = 0u;                          // -0.0 -> +0.0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 struct Row {
   int64_t n;       // valid entries of this row
@@ -310,7 +304,7 @@ __global__ void __launch_bounds__(kT) k_topk_write(TopkArgs a, int64_t seg_len, 
 
 
 // ============================================================ three-launch path
-constexpr int kB1 = 4096;          // 12-bit first digit
+constexpr int kB1 = kTopkBins1;     // 12-bit first digit
 constexpr int kCandCap = 4096;     // candidates kept per row
 constexpr int64_t kMaxBitmapCols = 1 << 19;
 constexpr int kFinT = 1024;        // threads of the per-row CTA
@@ -372,9 +366,13 @@ __device__ __forceinline__ uint32_t warp_append_base(bool flag, uint32_t* counte
 }
 
 // Launch 2: threshold bin b1 of each row, then every key above it ("sure") and
-// inside it ("candidate") is appended to the row's lists.
+// inside it ("candidate") is appended to the row's lists.  The segment is read
+// in batches of kCollectVec float4 per thread, all loads of a batch in flight
+// together; each batch reserves its list slots with one atomic per list.
+constexpr int kCollectVec = 8;
 __global__ void __launch_bounds__(kT) k_tk_collect(TopkArgs a, int64_t seg_len) {
   __shared__ int sh[kT / 32];
+  __shared__ uint32_t s_base[2];
   const int r = blockIdx.y, seg = blockIdx.x;
   const Row rr = row_range(a, r, seg, seg_len);
   if (rr.s0 >= rr.s1) return;
@@ -389,22 +387,47 @@ __global__ void __launch_bounds__(kT) k_tk_collect(TopkArgs a, int64_t seg_len) 
   int32_t* sure = L.sure + static_cast<int64_t>(r) * a.k;
   uint2* cand = L.cand + static_cast<int64_t>(r) * kCandCap;
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  for (int64_t base = rr.s0; base < rr.s1; base += kRound) {
-    uint32_t key[4];
-    load_keys(row, base, rr.s1, key);
-    const int64_t p = base + threadIdx.x * 4;
+  constexpr int kBatch = kRound * kCollectVec;
+  for (int64_t b0 = rr.s0; b0 < rr.s1; b0 += kBatch) {
+    uint32_t key[kCollectVec][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t bin = key[j] >> 20;
-      const bool is_sure = key[j] != 0u && bin > b1;
-      const bool is_cand = key[j] != 0u && bin == b1;
-      uint32_t off;
-      if (warp_append_base(is_sure, &cnt[0], &off) && is_sure) {
-        if (off < static_cast<uint32_t>(a.k)) sure[off] = static_cast<int32_t>(p + j);
-        else record_error(a.status, LSA_ERR_BOUNDS, r, static_cast<int>(off));  // cannot happen
+    for (int v = 0; v < kCollectVec; ++v) load_keys(row, b0 + v * kRound, rr.s1, key[v]);
+    int ns = 0, nc = 0;
+#pragma unroll
+    for (int v = 0; v < kCollectVec; ++v)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t bin = key[v][j] >> 20;
+        ns += key[v][j] != 0u && bin > b1;
+        nc += key[v][j] != 0u && bin == b1;
       }
-      if (warp_append_base(is_cand, &cnt[1], &off) && is_cand && off < static_cast<uint32_t>(kCandCap))
-        cand[off] = make_uint2(key[j], static_cast<uint32_t>(p + j));
+    int tot_s, tot_c;
+    const int off_s = block_excl_scan(ns, sh, &tot_s);
+    const int off_c = block_excl_scan(nc, sh, &tot_c);
+    if (threadIdx.x == 0) {
+      s_base[0] = tot_s ? atomicAdd(&cnt[0], static_cast<uint32_t>(tot_s)) : 0u;
+      s_base[1] = tot_c ? atomicAdd(&cnt[1], static_cast<uint32_t>(tot_c)) : 0u;
+    }
+    __syncthreads();
+    uint32_t os = s_base[0] + off_s, oc = s_base[1] + off_c;
+    __syncthreads();
+#pragma unroll
+    for (int v = 0; v < kCollectVec; ++v) {
+      const int64_t p = b0 + v * kRound + threadIdx.x * 4;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t x = key[v][j];
+        if (x == 0u) continue;
+        const uint32_t bin = x >> 20;
+        if (bin > b1) {
+          if (os < static_cast<uint32_t>(a.k)) sure[os] = static_cast<int32_t>(p + j);
+          else record_error(a.status, LSA_ERR_BOUNDS, r, static_cast<int>(os));  // cannot happen
+          ++os;
+        } else if (bin == b1) {
+          if (oc < static_cast<uint32_t>(kCandCap)) cand[oc] = make_uint2(x, static_cast<uint32_t>(p + j));
+          ++oc;
+        }
+      }
     }
   }
 }
@@ -485,6 +508,7 @@ __global__ void __launch_bounds__(kFinT) k_tk_final(TopkArgs a) {
     const int64_t v = __ldg(a.valid_len + r);
     n = v < 0 ? 0 : (v < n ? v : n);
   }
+  for (int64_t w = t; w < 2 * nwords; w += kFinT) fsm[w] = 0;
   // keff and the threshold bin from the 12-bit histogram
   const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
   uint32_t tot = 0;
@@ -523,7 +547,6 @@ __global__ void __launch_bounds__(kFinT) k_tk_final(TopkArgs a) {
   const uint32_t n_sure = keff - rank1;    // keys above bin b1
   const uint32_t n_cand = __ldcg(L.cnt + 2 * r + 1);
   const bool overflow = n_cand > static_cast<uint32_t>(kCandCap);
-  for (int64_t w = t; w < 2 * nwords; w += kFinT) fsm[w] = 0;
   const int nc = overflow ? 0 : static_cast<int>(n_cand);
   for (int c = t; c < nc; c += kFinT) cs[c] = __ldcg(L.cand + static_cast<int64_t>(r) * kCandCap + c);
   __syncthreads();
@@ -647,6 +670,10 @@ TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
 
 bool topk_v2_ok(int64_t n_cols) { return n_cols <= kMaxBitmapCols; }
 
+size_t topk_hist_zero_bytes(int32_t rows) {
+  return static_cast<size_t>(rows) * kB1 * 4 + (static_cast<size_t>(rows) * 8 + 255) / 256 * 256;
+}
+
 size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t k) {
   const size_t R = static_cast<size_t>(rows);
   if (topk_v2_ok(n_cols)) {
@@ -665,10 +692,12 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   TopkPlan p = topk_plan(a.rows, a.n_cols);
   dim3 grid(static_cast<unsigned>(p.nseg), static_cast<unsigned>(a.rows));
   if (topk_v2_ok(a.n_cols)) {
-    const size_t zero = static_cast<size_t>(a.rows) * kB1 * 4 + (static_cast<size_t>(a.rows) * 8 + 255) / 256 * 256;
-    cudaError_t e = cudaMemsetAsync(a.ws, 0, zero, s);
-    if (e != cudaSuccess) return e;
-    k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
+    cudaError_t e = cudaSuccess;
+    if (!a.hist_ready) {
+      e = cudaMemsetAsync(a.ws, 0, topk_hist_zero_bytes(a.rows), s);
+      if (e != cudaSuccess) return e;
+      k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
+    }
     k_tk_collect<<<grid, kT, 0, s>>>(a, p.seg_len);
     const int64_t nwords = (a.n_cols + 31) / 32;
     const size_t smem = 2 * nwords * 4 + static_cast<size_t>(kCandCap) * 8;
@@ -758,5 +787,6 @@ extern "C" lsa_status lsa_topk_noalloc(const float* scores, int64_t ld, int32_t 
   a.idx = idx;
   a.ws = static_cast<uint8_t*>(base) + kStatusBytes;  // histograms are zeroed by launch_topk
   a.status = reinterpret_cast<DevStatus*>(base);
+  a.hist_ready = false;
   return launch_topk(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
 }

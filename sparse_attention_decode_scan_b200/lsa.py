@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
     L.lsa_topk_noalloc.argtypes = [vp, i64, i32, vp, i64, i32, vp, vp]
     L.lsa_sparse_attn_decode.argtypes = [D, C, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.lsa_decode_step.argtypes = [D, C, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
+    L.lsa_decode_step_profiled.argtypes = [D, C, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]
     L.lsa_read_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
     L.lsa_status_string.argtypes = [ctypes.c_int]
     L.lsa_status_string.restype = ctypes.c_char_p
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
     L.lsa_launch_count.argtypes = [D, i32, i64, i32, i32]
     L.lsa_launch_count.restype = i32
     for f in ("lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode", "lsa_decode_step",
+              "lsa_decode_step_profiled",
               "lsa_read_device_status"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
@@ -162,6 +164,16 @@ def decode_step(dims: Dims, cache: Cache, q_idx, w, q, out, lse, ws, idx_out=Non
                                         _ptr(out), _ptr(lse), _ptr(idx_out), int(flags), _ptr(ws),
                                         ws.numel() if ws is not None else 0, _stream(stream)),
                   "lsa_decode_step", raise_on_error)
+
+
+def decode_step_profiled(dims: Dims, cache: Cache, q_idx, w, q, out, lse, ws, events, idx_out=None,
+                         flags: int = LSA_STEP_UNFUSED, stream=None, raise_on_error=True) -> int:
+    """lsa_decode_step recording 4 CUDA events (torch.cuda.Event, already created) at phase boundaries."""
+    ev = (ctypes.c_void_p * 4)(*[int(e.cuda_event) if e is not None else None for e in events])
+    return _check(lib().lsa_decode_step_profiled(ctypes.byref(dims), ctypes.byref(cache), _ptr(q_idx), _ptr(w),
+                                                 _ptr(q), _ptr(out), _ptr(lse), _ptr(idx_out), int(flags),
+                                                 _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream),
+                                                 ev), "lsa_decode_step_profiled", raise_on_error)
 
 
 def read_device_status(ws, stream=None) -> int:

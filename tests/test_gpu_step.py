@@ -109,3 +109,22 @@ def test_decode_step_full(cfg):
 def test_decode_step_full_fp8():
     case = cases.full(4)
     _check_step(case, [0, 3])
+
+
+@pytest.mark.parametrize("name", ["paged_B5", "fp8_L6001", "bf16_L5000"])
+def test_decode_step_selection_equals_separate_calls(name):
+    """lsa_decode_step (whose scan may also build the top-k's first histogram)
+    selects exactly what lsa_indexer_scores followed by lsa_topk selects."""
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+    dc = DeviceCase(cases.small(name))
+    _, _, idx_step = _step(dc)
+    B, k = dc.rows, dc.spec.top_k
+    ld = (dc.max_len + 3) // 4 * 4
+    scores = torch.empty((B, ld), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.workspace_size(dc.dims, B, dc.max_len, lsa.LSA_OP_DECODE_STEP))
+    lsa.indexer_scores(dc.dims, dc.cache, dc.q_idx, dc.w, scores, ld, ws)
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    lsa.topk(scores, k, idx, ws, valid_len=dc.seq_lens, n_cols=dc.max_len, ld=ld)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_step)
