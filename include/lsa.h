@@ -211,7 +211,7 @@ lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream
  *   Scratch: a 2 MiB static device array inside liblsa.so, held by every GPU
  *   that loads the library until the process exits.  Sizes whose top-k scratch
  *   (lsa_workspace_size with d->top_k = k, LSA_OP_TOPK) exceeds 2 MiB return
- *   LSA_ERR_UNSUPPORTED (for k = 2048: 32 rows fit, whatever their length).
+ *   LSA_ERR_UNSUPPORTED (about 100 rows fit).
  *   Allocates nothing: no cudaMalloc / cudaFree; the histograms are cleared
  *   with cudaMemsetAsync on `stream` at every call.
  *   The first call on a device looks up the array's device address (once per

@@ -342,11 +342,7 @@ int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32
     case LSA_OP_SCORES: return scan;
     case LSA_OP_TOPK: return topk_launches(max_len);
     case LSA_OP_ATTN: return attn;
-    case LSA_OP_DECODE_STEP: {
-      const bool fused = !simt && topk_v2_ok(max_len) &&
-                         scores_tc_shape_ok(d->idx_key_dtype, d->act_dtype, d->n_idx_heads, d->idx_dim, d->block_size);
-      return scan + topk_launches(max_len) - (fused ? 1 : 0) + attn;
-    }
+    case LSA_OP_DECODE_STEP: return scan + topk_launches(max_len) + attn;
     default: return -1;
   }
 }

@@ -11,17 +11,19 @@
 // 64 heads make the MMA's M side (M = 64), so the fp32 output accumulator
 // O[64 x 512] takes half of the TMEM lanes: dims 0-255 at lane offset 0 and
 // dims 256-511 at lane offset 16, columns 0-255; the two score buffers
-// S[64 x 32] sit at lane offset 0, columns 256-319.  Each softmax warp then
+// S[64 x 64] sit at lane offset 0, columns 256-383.  Each softmax warp then
 // holds, for its 16 heads, the scores in lanes 0-15 and both output halves in
 // lanes 0-31, so a rescale touches only output columns.
-//   warps 0-3  producer: cp.async gathers of 32 selected rows per chunk into the
-//              128-byte-swizzled operand layout, three chunks in flight; the
-//              block-table lookups of the next chunk are loaded one chunk ahead
-//   warp 4     MMA issuer: S = Q K^T (36 x M64N32K16), O += P V (4 x M64N256K16),
+//   warps 0-3  producer: cp.async gathers of 64 selected rows per chunk into the
+//              128-byte-swizzled operand layout (two chunk buffers); the rows of
+//              chunk j+2 are looked up and prefetched into L2 while chunk j is
+//              gathered, so the gathers read L2, not HBM
+//   warp 4     MMA issuer: S = Q K^T (36 x M64N64K16), O += P V (8 x M64N256K16),
 //              V read MN-major from the same tile as K
 //   warps 5-8  online softmax (base 2, lazy rescale when the max grows by > 8),
-//              P to one of two shared-memory buffers (so the softmax of chunk j+1
-//              overlaps P V of chunk j), final normalisation
+//              P to shared memory, final normalisation
+// (Below N = 64 an MMA costs as much as at N = 64 on this part, so 64-row
+// chunks halve the score MMAs per row compared with 32-row chunks.)
 // With several splits per row, each CTA writes a normalised partial and its
 // lse; the last CTA of a (row, half) to finish merges them with all of its
 // threads (global counter, no waiting), so no separate merge launch is needed.
@@ -38,18 +40,18 @@ constexpr int kHeadsAll = 128;
 constexpr int kHeadsCta = 64;
 constexpr int kD = 576;
 constexpr int kDv = 512;
-constexpr int kChunk = 32;                 // KV rows per chunk
-constexpr int kNBuf = 3;                   // chunk buffers (gathers in flight)
+constexpr int kChunk = 64;                 // KV rows per chunk
+constexpr int kNBuf = 2;                   // chunk buffers
 constexpr int kBoxes = kD / 64;            // 9 column blocks of 64 dims
-constexpr int kBoxBytes = kChunk * 128;    // 32 rows x 128 B
-constexpr int kKvBytes = kBoxes * kBoxBytes;          // 36864
+constexpr int kBoxBytes = kChunk * 128;    // 64 rows x 128 B
+constexpr int kKvBytes = kBoxes * kBoxBytes;          // 73728
 constexpr int kQBlock = kHeadsCta * 128;              // 8192
 constexpr int kQBytes = kBoxes * kQBlock;             // 73728
-constexpr int kPBytes = kHeadsCta * 128;              // 8192 per P buffer (64 B of each row used)
+constexpr int kPBytes = kHeadsCta * 128;              // 8192: P [64 heads x 64 rows] bf16
 constexpr int kThreads = 288;
 constexpr int kProdThreads = 128;
 constexpr int kWarpMma = 4;                // warps 5-8: softmax
-constexpr int kSmemBytes = kQBytes + kNBuf * kKvBytes + 2 * kPBytes + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr int kSmemBytes = kQBytes + kNBuf * kKvBytes + kPBytes + 1024 /*barriers*/ + 1024 /*align*/;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256;            // score buffers start column
 constexpr float kLog2e = 1.4426950408889634f;
@@ -157,16 +159,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qs = smem;
   uint8_t* kvs = qs + kQBytes;         // kNBuf chunk buffers
-  uint8_t* ps = kvs + kNBuf * kKvBytes;  // 2 P buffers
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + 2 * kPBytes);
+  uint8_t* ps = kvs + kNBuf * kKvBytes;  // P
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + kPBytes);
   uint64_t* qfull = bars;
   uint64_t* kvfull = bars + 1;            // [kNBuf]
   uint64_t* kvempty = kvfull + kNBuf;     // [kNBuf]
   uint64_t* sfull = kvempty + kNBuf;      // [2]
   uint64_t* sempty = sfull + 2;           // [2]
-  uint64_t* pfull = sempty + 2;           // [2] per P buffer
-  uint64_t* pvdone = pfull + 2;           // [2] per P buffer
-  uint64_t* done = pvdone + 2;
+  uint64_t* pfull = sempty + 2;
+  uint64_t* pvdone = pfull + 1;
+  uint64_t* done = pvdone + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
@@ -187,10 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       tc::mbar_init(&sfull[i], 1);
       tc::mbar_init(&sempty[i], 4);
     }
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&pfull[i], 4);
-      tc::mbar_init(&pvdone[i], 1);
-    }
+    tc::mbar_init(pfull, 4);
+    tc::mbar_init(pvdone, 1);
     tc::mbar_init(done, 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
@@ -222,15 +222,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     }
     cp_async_arrive_noinc(qfull);
     const bool report = sub == 0 && half == 0;
-    int64_t rn0 = entry_row(a, ad, rc, r, j0 + rbase, j1, report);
-    int64_t rn1 = entry_row(a, ad, rc, r, j0 + rbase + 16, j1, report);
+    // rows of this thread (4 per chunk) for chunks j, j+1 and j+2
+    int64_t rc_[4], rn_[4], rn2_[4];
+    auto lookup = [&](int jj, int64_t (&dst)[4]) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        dst[m] = jj < nch ? entry_row(a, ad, rc, r, j0 + jj * kChunk + rbase + 16 * m, j1, report) : -1;
+    };
+    auto prefetch_l2 = [&](const int64_t (&rows)[4]) {
+      if (sub != 0) return;
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        if (rows[m] >= 0)
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                           reinterpret_cast<const uint8_t*>(a.cache.kv) + rows[m] * (kD * 2)),
+                       "r"(kD * 2)
+                       : "memory");
+    };
+    lookup(0, rc_);
+    lookup(1, rn_);
+    prefetch_l2(rc_);
+    prefetch_l2(rn_);
+    lookup(2, rn2_);
     for (int j = 0; j < nch; ++j) {
       const int b = j % kNBuf;
-      const int64_t rows_cur[2] = {rn0, rn1};
-      if (j + 1 < nch) {  // next chunk's lookups, in flight while this one is issued
-        rn0 = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + rbase, j1, report);
-        rn1 = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + rbase + 16, j1, report);
-      }
+      prefetch_l2(rn2_);  // chunk j+2 (looked up during the previous iteration)
       if (!tc::mbar_wait(&kvempty[b], ((j / kNBuf) & 1) ^ 1, abort_flag)) {
         if (t == 0) {
           record_error(a.status, LSA_ERR_TIMEOUT, r, 10);
@@ -242,10 +258,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       const uint32_t kv_u = tc::smem_u32(kvb);
       bool zeroed = false;
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
+      for (int m = 0; m < 4; ++m) {
         const int i = rbase + 16 * m;
-        if (rows_cur[m] >= 0) {
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cache.kv) + rows_cur[m] * (kD * 2);
+        if (rc_[m] >= 0) {
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cache.kv) + rc_[m] * (kD * 2);
 #pragma unroll
           for (int d = 0; d < kBoxes; ++d)
             cp_async16(kv_u + d * kBoxBytes + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
@@ -258,6 +274,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       }
       if (zeroed) tc::fence_proxy_async_smem();
       cp_async_arrive_noinc(&kvfull[b]);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        rc_[m] = rn_[m];
+        rn_[m] = rn2_[m];
+      }
+      lookup(j + 3, rn2_);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kWarpMma) {
@@ -266,11 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       const uint32_t q_u = tc::smem_u32(qs);
       bool ok = tc::mbar_wait(qfull, 0, abort_flag);
       tc::fence_proxy_async_smem();
+      const uint32_t p_u = tc::smem_u32(ps);
       auto issue_pv = [&](int i) -> bool {
-        const int pb = i & 1;
-        if (!tc::mbar_wait(&pfull[pb], (i >> 1) & 1, abort_flag)) return false;
+        if (!tc::mbar_wait(pfull, i & 1, abort_flag)) return false;
         tc::tc_fence_after();
-        const uint32_t p_u = tc::smem_u32(ps + pb * kPBytes);
         const uint32_t kv_u = tc::smem_u32(kvs + (i % kNBuf) * kKvBytes);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -282,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
             tc::mma_f16(d, ad_, bd_, kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        tc::mma_commit(&pvdone[pb]);
+        tc::mma_commit(pvdone);
         tc::mma_commit(&kvempty[i % kNBuf]);
         return true;
       };
@@ -324,36 +345,46 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     const float c2 = a.scale * kLog2e;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
-    // validity of chunk rows, looked up two chunks ahead of their use
-    bool v0 = nch > 0 && entry_row(a, ad, rc, r, j0 + lane, j1, false) >= 0;
-    bool v1 = nch > 1 && entry_row(a, ad, rc, r, j0 + kChunk + lane, j1, false) >= 0;
+    // validity of the chunk's rows (lane and lane + 32), looked up one chunk ahead
+    bool va = nch > 0 && entry_row(a, ad, rc, r, j0 + lane, j1, false) >= 0;
+    bool vb = nch > 0 && entry_row(a, ad, rc, r, j0 + 32 + lane, j1, false) >= 0;
     for (int j = 0; j < nch; ++j) {
       const int sb = j & 1;
-      const uint32_t mask = __ballot_sync(0xffffffffu, v0);
-      v0 = v1;
-      if (j + 2 < nch) v1 = entry_row(a, ad, rc, r, j0 + (j + 2) * kChunk + lane, j1, false) >= 0;
+      const uint32_t mlo = __ballot_sync(0xffffffffu, va), mhi = __ballot_sync(0xffffffffu, vb);
+      if (j + 1 < nch) {
+        va = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + lane, j1, false) >= 0;
+        vb = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + 32 + lane, j1, false) >= 0;
+      }
       if (!tc::mbar_wait(&sfull[sb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       tc::tc_fence_after();
-      float s[32];
-      tc::tmem_ld32(tmem + lane_base + kColS + sb * kChunk, s);
-      tc::tmem_wait_ld();
+      float s[64];
+      {
+        float t0[32], t1[32];
+        tc::tmem_ld32(tmem + lane_base + kColS + sb * kChunk, t0);
+        tc::tmem_ld32(tmem + lane_base + kColS + sb * kChunk + 32, t1);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = t0[i];
+          s[32 + i] = t1[i];
+        }
+      }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sempty[sb]);
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        s[i] = ((mask >> i) & 1u) ? s[i] * c2 : -INFINITY;
+      for (int i = 0; i < 64; ++i) {
+        const bool valid = (i < 32) ? ((mlo >> i) & 1u) : ((mhi >> (i - 32)) & 1u);
+        s[i] = valid ? s[i] * c2 : -INFINITY;
         mx = fmaxf(mx, s[i]);
       }
       const float m_new = fmaxf(m_run, mx);
+      // P is single-buffered: P V of chunk j-1 must be done before P(j) is written
+      // (which also makes a rescale of O safe)
+      if (j > 0 && !tc::mbar_wait(pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
       const bool need = srow && (j > 0) && (m_new > m_run + kRescaleLog2);
-      const bool any_need = __any_sync(0xffffffffu, need);
-      // a rescale touches O: P V of chunk j-1 must have finished
-      if (any_need && !tc::mbar_wait(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
-      // P(j) reuses the buffer of chunk j-2: its P V must have finished
-      if (j >= 2 && !tc::mbar_wait(&pvdone[j & 1], ((j - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
-      if (any_need) {
+      if (__any_sync(0xffffffffu, need)) {
         const float alpha_own = need ? exp2f(m_run - m_new) : 1.f;
         const float alpha = __shfl_sync(0xffffffffu, alpha_own, lane & 15);
         tc::tc_fence_after();
@@ -376,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       // probabilities (base 2), bf16 P row of this head, running sum of the rounded values
       if (srow) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -387,14 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
             l += __low2float(pb) + __high2float(pb);
             w[u] = *reinterpret_cast<const uint32_t*>(&pb);
           }
-          *reinterpret_cast<uint4*>(ps + (j & 1) * kPBytes + tc::sw128_offset(head_local, c)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(ps + tc::sw128_offset(head_local, c)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&pfull[j & 1]);
+      if (lane == 0) tc::mbar_arrive(pfull);
     }
     if (!ok && lane == 0) {
       record_error(a.status, LSA_ERR_TIMEOUT, r, 12);
@@ -402,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     }
     // final: wait for the last PV, normalise, store (bf16 output or fp32 partial)
     bool fin = ok;
-    if (ok && nch > 0) fin = tc::mbar_wait(&pvdone[(nch - 1) & 1], ((nch - 1) >> 1) & 1, abort_flag);
+    if (ok && nch > 0) fin = tc::mbar_wait(pvdone, (nch - 1) & 1, abort_flag);
     const float l_h = __shfl_sync(0xffffffffu, l, lane & 15);
     const float m_h = __shfl_sync(0xffffffffu, m_run, lane & 15);
     const float inv = l_h > 0.f ? 1.f / l_h : 0.f;
@@ -452,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       __threadfence();
       if (threadIdx.x == 0) P.counters[2 * r + half] = 0;  // left zeroed for the next call
       // weights of every split for the 64 heads, in the (now idle) P buffers
-      float* wsm = reinterpret_cast<float*>(ps);          // [nsplit][64], nsplit <= 32
+      float* wsm = reinterpret_cast<float*>(ps);          // [nsplit][64] in the idle P buffer, nsplit <= 32
       const int ns = P.nsplit;
       const float* lse_p = P.part_lse + static_cast<int64_t>(r) * ns * kHeadsAll + half * kHeadsCta;
       if (threadIdx.x < kHeadsCta) {

@@ -303,133 +303,17 @@ __global__ void __launch_bounds__(kT) k_topk_write(TopkArgs a, int64_t seg_len, 
 }
 
 
-// ============================================================ three-launch path
+// ============================================================ per-row path
 constexpr int kB1 = kTopkBins1;     // 12-bit first digit
-constexpr int kCandCap = 4096;     // candidates kept per row
+constexpr int kCandCap = 8192;     // candidates kept per row (in shared memory)
 constexpr int64_t kMaxBitmapCols = 1 << 19;
 constexpr int kFinT = 1024;        // threads of the per-row CTA
+constexpr int kRowVec = 8;         // float4 loads in flight per thread
 
-struct V2Layout {
-  uint32_t* hist;   // [rows][kB1]
-  uint32_t* cnt;    // [rows][2]: sure, candidates
-  int32_t* sure;    // [rows][k]
-  uint2* cand;      // [rows][kCandCap]: (key, position)
-};
-
-__device__ __forceinline__ V2Layout v2_layout(const TopkArgs& a) {
-  V2Layout L;
-  uint8_t* b = reinterpret_cast<uint8_t*>(a.ws);
-  L.hist = reinterpret_cast<uint32_t*>(b);
-  b += static_cast<size_t>(a.rows) * kB1 * 4;
-  L.cnt = reinterpret_cast<uint32_t*>(b);
-  b += (static_cast<size_t>(a.rows) * 8 + 255) / 256 * 256;
-  L.sure = reinterpret_cast<int32_t*>(b);
-  b += (static_cast<size_t>(a.rows) * a.k * 4 + 255) / 256 * 256;
-  L.cand = reinterpret_cast<uint2*>(b);
-  return L;
-}
-
-// Launch 1: histogram of key bits [31:20] per row.
-__global__ void __launch_bounds__(kT) k_tk_hist12(TopkArgs a, int64_t seg_len) {
-  __shared__ uint32_t h[kB1];
-  const int r = blockIdx.y, seg = blockIdx.x;
-  const Row rr = row_range(a, r, seg, seg_len);
-  if (rr.s0 >= rr.s1) return;
-  for (int i = threadIdx.x; i < kB1; i += kT) h[i] = 0;
-  __syncthreads();
-  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  for (int64_t base = rr.s0; base < rr.s1; base += kRound) {
-    uint32_t key[4];
-    load_keys(row, base, rr.s1, key);
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (key[j]) atomicAdd(&h[key[j] >> 20], 1u);
-  }
-  __syncthreads();
-  uint32_t* dst = v2_layout(a).hist + static_cast<int64_t>(r) * kB1;
-  for (int i = threadIdx.x; i < kB1; i += kT)
-    if (h[i]) atomicAdd(dst + i, h[i]);
-}
-
-// Appends `pos` (or (key,pos)) for the lanes whose flag is set, with one
-// global atomic per warp.
-__device__ __forceinline__ uint32_t warp_append_base(bool flag, uint32_t* counter, uint32_t* my_off) {
-  const uint32_t m = __ballot_sync(0xffffffffu, flag);
-  if (!m) return 0;
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(m) - 1;
-  uint32_t base = 0;
-  if (lane == leader) base = atomicAdd(counter, static_cast<uint32_t>(__popc(m)));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  *my_off = base + __popc(m & ((1u << lane) - 1u));
-  return m;
-}
-
-// Launch 2: threshold bin b1 of each row, then every key above it ("sure") and
-// inside it ("candidate") is appended to the row's lists.  The segment is read
-// in batches of kCollectVec float4 per thread, all loads of a batch in flight
-// together; each batch reserves its list slots with one atomic per list.
-constexpr int kCollectVec = 8;
-__global__ void __launch_bounds__(kT) k_tk_collect(TopkArgs a, int64_t seg_len) {
-  __shared__ int sh[kT / 32];
-  __shared__ uint32_t s_base[2];
-  const int r = blockIdx.y, seg = blockIdx.x;
-  const Row rr = row_range(a, r, seg, seg_len);
-  if (rr.s0 >= rr.s1) return;
-  const V2Layout L = v2_layout(a);
-  const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
-  Found f = find_bin<kB1>(hist, 0xffffffffu, sh);
-  const uint32_t keff = f.total < static_cast<uint32_t>(a.k) ? f.total : static_cast<uint32_t>(a.k);
-  if (keff == 0) return;
-  f = find_bin<kB1>(hist, keff, sh);
-  const uint32_t b1 = static_cast<uint32_t>(f.bin);
-  uint32_t* cnt = L.cnt + 2 * r;
-  int32_t* sure = L.sure + static_cast<int64_t>(r) * a.k;
-  uint2* cand = L.cand + static_cast<int64_t>(r) * kCandCap;
-  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  constexpr int kBatch = kRound * kCollectVec;
-  for (int64_t b0 = rr.s0; b0 < rr.s1; b0 += kBatch) {
-    uint32_t key[kCollectVec][4];
-#pragma unroll
-    for (int v = 0; v < kCollectVec; ++v) load_keys(row, b0 + v * kRound, rr.s1, key[v]);
-    int ns = 0, nc = 0;
-#pragma unroll
-    for (int v = 0; v < kCollectVec; ++v)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t bin = key[v][j] >> 20;
-        ns += key[v][j] != 0u && bin > b1;
-        nc += key[v][j] != 0u && bin == b1;
-      }
-    int tot_s, tot_c;
-    const int off_s = block_excl_scan(ns, sh, &tot_s);
-    const int off_c = block_excl_scan(nc, sh, &tot_c);
-    if (threadIdx.x == 0) {
-      s_base[0] = tot_s ? atomicAdd(&cnt[0], static_cast<uint32_t>(tot_s)) : 0u;
-      s_base[1] = tot_c ? atomicAdd(&cnt[1], static_cast<uint32_t>(tot_c)) : 0u;
-    }
-    __syncthreads();
-    uint32_t os = s_base[0] + off_s, oc = s_base[1] + off_c;
-    __syncthreads();
-#pragma unroll
-    for (int v = 0; v < kCollectVec; ++v) {
-      const int64_t p = b0 + v * kRound + threadIdx.x * 4;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t x = key[v][j];
-        if (x == 0u) continue;
-        const uint32_t bin = x >> 20;
-        if (bin > b1) {
-          if (os < static_cast<uint32_t>(a.k)) sure[os] = static_cast<int32_t>(p + j);
-          else record_error(a.status, LSA_ERR_BOUNDS, r, static_cast<int>(os));  // cannot happen
-          ++os;
-        } else if (bin == b1) {
-          if (oc < static_cast<uint32_t>(kCandCap)) cand[oc] = make_uint2(x, static_cast<uint32_t>(p + j));
-          ++oc;
-        }
-      }
-    }
-  }
+// Workspace of the per-row path: the first-digit histograms [rows][4096],
+// written by the decode scan when it runs first (hist_ready); otherwise unused.
+__device__ __forceinline__ const uint32_t* v2_hist(const TopkArgs& a) {
+  return reinterpret_cast<const uint32_t*>(a.ws);
 }
 
 // Block-wide (kFinT threads) exclusive scan.
@@ -486,51 +370,68 @@ __device__ __forceinline__ uint32_t low_bits(uint32_t x, int n) {
   return y;
 }
 
-// Launch 3: one CTA per row.  Finishes the select on the candidates (bits
-// [19:0], in shared memory; or by re-reading the row if the list overflowed),
-// marks the chosen positions in a bitmap and writes them in position order.
-__global__ void __launch_bounds__(kFinT) k_tk_final(TopkArgs a) {
+// One CTA per row: the first-digit histogram (from the scan, or one pass over
+// the row here), the threshold bin b1, one pass that marks every key above b1
+// in a position bitmap and keeps the keys inside b1 as candidates, a radix
+// select on the candidates' low 20 bits (or, if they overflow the list, on
+// the row again), and an ordered compaction of the bitmap.
+__global__ void __launch_bounds__(kFinT) k_tk_row(TopkArgs a) {
   extern __shared__ __align__(16) uint32_t fsm[];
   __shared__ int warp_sums[32];
   __shared__ int s_bin;
   __shared__ uint32_t s_rank;
+  __shared__ uint32_t s_nc;
   __shared__ uint32_t h[1024];
+  __shared__ uint32_t h12[kB1];
   const int r = blockIdx.x;
   const int t = threadIdx.x;
   const int64_t nwords = (a.n_cols + 31) / 32;
   uint32_t* bm = fsm;               // selected positions
   uint32_t* tb = fsm + nwords;      // positions equal to the threshold key
   uint2* cs = reinterpret_cast<uint2*>(fsm + 2 * nwords);  // candidates: 2*nwords words keep 8-byte alignment
-  const V2Layout L = v2_layout(a);
   int32_t* out = a.idx + static_cast<int64_t>(r) * a.k;
   int64_t n = a.n_cols;
   if (a.valid_len) {
     const int64_t v = __ldg(a.valid_len + r);
     n = v < 0 ? 0 : (v < n ? v : n);
   }
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
   for (int64_t w = t; w < 2 * nwords; w += kFinT) fsm[w] = 0;
-  // keff and the threshold bin from the 12-bit histogram
-  const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
-  uint32_t tot = 0;
-  for (int i = t; i < kB1; i += kFinT) tot += __ldcg(hist + i);
-  int tt;
-  fin_excl_scan(static_cast<int>(tot), warp_sums, &tt);
-  const uint32_t keff = static_cast<uint32_t>(tt) < static_cast<uint32_t>(a.k) ? static_cast<uint32_t>(tt)
-                                                                               : static_cast<uint32_t>(a.k);
-  for (int i = static_cast<int>(keff) + t; i < a.k; i += kFinT) out[i] = -1;
-  if (keff == 0) return;
-  // bin b1 (4 bins per thread)
+  if (t == 0) s_nc = 0;
+  // first-digit histogram
+  if (a.hist_ready) {
+    const uint32_t* g = v2_hist(a) + static_cast<int64_t>(r) * kB1;
+    for (int i = t; i < kB1; i += kFinT) h12[i] = __ldcg(g + i);
+  } else {
+    for (int i = t; i < kB1; i += kFinT) h12[i] = 0;
+    __syncthreads();
+    for (int64_t base = 0; base < n; base += kFinT * 4 * kRowVec) {
+      uint32_t key[kRowVec][4];
+#pragma unroll
+      for (int v = 0; v < kRowVec; ++v) load_keys(row, base + v * kFinT * 4, n, key[v]);
+#pragma unroll
+      for (int v = 0; v < kRowVec; ++v)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (key[v][j]) atomicAdd(&h12[key[v][j] >> 20], 1u);
+    }
+  }
+  __syncthreads();
+  // keff and the threshold bin (4 bins per thread)
+  uint32_t keff, b1, rank1;
   {
     uint32_t v[4], mine = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      v[i] = __ldcg(hist + t * 4 + i);
+      v[i] = h12[t * 4 + i];
       mine += v[i];
     }
     int total;
     const int excl = fin_excl_scan(static_cast<int>(mine), warp_sums, &total);
+    keff = static_cast<uint32_t>(total) < static_cast<uint32_t>(a.k) ? static_cast<uint32_t>(total)
+                                                                     : static_cast<uint32_t>(a.k);
     uint32_t cum = static_cast<uint32_t>(total - excl) - mine;
-    if (cum < keff && keff <= cum + mine) {
+    if (keff > 0 && cum < keff && keff <= cum + mine) {
       for (int i = 3; i >= 0; --i) {
         if (cum + v[i] >= keff) {
           s_bin = t * 4 + i;
@@ -541,21 +442,42 @@ __global__ void __launch_bounds__(kFinT) k_tk_final(TopkArgs a) {
       }
     }
     __syncthreads();
+    b1 = static_cast<uint32_t>(s_bin);
+    rank1 = s_rank;  // wanted rank inside bin b1
   }
-  const uint32_t b1 = static_cast<uint32_t>(s_bin);
-  const uint32_t rank1 = s_rank;           // wanted rank inside bin b1
-  const uint32_t n_sure = keff - rank1;    // keys above bin b1
-  const uint32_t n_cand = __ldcg(L.cnt + 2 * r + 1);
+  for (int i = static_cast<int>(keff) + t; i < a.k; i += kFinT) out[i] = -1;
+  if (keff == 0) return;
+  // one pass: keys above b1 -> bitmap, keys in b1 -> candidates
+  for (int64_t base = 0; base < n; base += kFinT * 4 * kRowVec) {
+    uint32_t key[kRowVec][4];
+#pragma unroll
+    for (int v = 0; v < kRowVec; ++v) load_keys(row, base + v * kFinT * 4, n, key[v]);
+#pragma unroll
+    for (int v = 0; v < kRowVec; ++v) {
+      const uint32_t p0 = static_cast<uint32_t>(base + v * kFinT * 4 + t * 4);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t x = key[v][j];
+        const uint32_t bin = x >> 20;
+        const bool is_cand = x != 0u && bin == b1;
+        if (x != 0u && bin > b1) atomicOr(&bm[(p0 + j) >> 5], 1u << ((p0 + j) & 31));
+        const uint32_t m = __ballot_sync(0xffffffffu, is_cand);
+        if (m) {
+          const int lane = t & 31;
+          const int leader = __ffs(m) - 1;
+          uint32_t boff = 0;
+          if (lane == leader) boff = atomicAdd(&s_nc, static_cast<uint32_t>(__popc(m)));
+          boff = __shfl_sync(0xffffffffu, boff, leader);
+          const uint32_t off = boff + __popc(m & ((1u << lane) - 1u));
+          if (is_cand && off < static_cast<uint32_t>(kCandCap)) cs[off] = make_uint2(x, p0 + j);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t n_cand = s_nc;
   const bool overflow = n_cand > static_cast<uint32_t>(kCandCap);
   const int nc = overflow ? 0 : static_cast<int>(n_cand);
-  for (int c = t; c < nc; c += kFinT) cs[c] = __ldcg(L.cand + static_cast<int64_t>(r) * kCandCap + c);
-  __syncthreads();
-  const int32_t* sure = L.sure + static_cast<int64_t>(r) * a.k;
-  for (uint32_t i = t; i < n_sure; i += kFinT) {
-    const int32_t p = __ldcg(sure + i);
-    atomicOr(&bm[p >> 5], 1u << (p & 31));
-  }
-  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
   // radix select on bits [19:10] then [9:0] among the keys of bin b1
   uint32_t T = 0, ties = 0;
   for (int pass = 0; pass < 2; ++pass) {
@@ -670,44 +592,32 @@ TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
 
 bool topk_v2_ok(int64_t n_cols) { return n_cols <= kMaxBitmapCols; }
 
-size_t topk_hist_zero_bytes(int32_t rows) {
-  return static_cast<size_t>(rows) * kB1 * 4 + (static_cast<size_t>(rows) * 8 + 255) / 256 * 256;
-}
+size_t topk_hist_zero_bytes(int32_t rows) { return static_cast<size_t>(rows) * kB1 * 4; }
 
-size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t k) {
+size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t) {
   const size_t R = static_cast<size_t>(rows);
-  if (topk_v2_ok(n_cols)) {
-    const size_t b = R * kB1 * 4 + (R * 8 + 255) / 256 * 256 + (R * k * 4 + 255) / 256 * 256 + R * kCandCap * 8;
-    return (b + 255) / 256 * 256;
-  }
+  if (topk_v2_ok(n_cols)) return (R * kB1 * 4 + 255) / 256 * 256;
   TopkPlan p = topk_plan(rows, n_cols);
   size_t b = R * kHistStride * 4 + R * p.nseg * 8;
   return (b + 255) / 256 * 256;
 }
 
-int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 3 : 5; }
+int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 1 : 5; }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   if (a.rows == 0 || a.k == 0) return cudaSuccess;
   TopkPlan p = topk_plan(a.rows, a.n_cols);
   dim3 grid(static_cast<unsigned>(p.nseg), static_cast<unsigned>(a.rows));
   if (topk_v2_ok(a.n_cols)) {
-    cudaError_t e = cudaSuccess;
-    if (!a.hist_ready) {
-      e = cudaMemsetAsync(a.ws, 0, topk_hist_zero_bytes(a.rows), s);
-      if (e != cudaSuccess) return e;
-      k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
-    }
-    k_tk_collect<<<grid, kT, 0, s>>>(a, p.seg_len);
     const int64_t nwords = (a.n_cols + 31) / 32;
     const size_t smem = 2 * nwords * 4 + static_cast<size_t>(kCandCap) * 8;
     static size_t smem_set = 0;
     if (smem > 48 * 1024 && smem > smem_set) {
-      e = cudaFuncSetAttribute(k_tk_final, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      cudaError_t e = cudaFuncSetAttribute(k_tk_row, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return e;
       smem_set = smem;
     }
-    k_tk_final<<<a.rows, kFinT, smem, s>>>(a);
+    k_tk_row<<<a.rows, kFinT, smem, s>>>(a);
     return cudaGetLastError();
   }
   size_t hist_bytes = static_cast<size_t>(a.rows) * kHistStride * 4;
