@@ -208,10 +208,10 @@ lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream
  * implicit synchronisation.  (The pages describe no such entry point; it is
  * an addition of this library.)
  *   Same arguments, results and errors as lsa_topk, minus ws / ws_bytes.
- *   Scratch: a 2 MiB static device array inside liblsa.so, held by every GPU
+ *   Scratch: a 4 MiB static device array inside liblsa.so, held by every GPU
  *   that loads the library until the process exits.  Sizes whose top-k scratch
- *   (lsa_workspace_size with d->top_k = k, LSA_OP_TOPK) exceeds 2 MiB return
- *   LSA_ERR_UNSUPPORTED (about 100 rows fit).
+ *   (lsa_workspace_size with d->top_k = k, LSA_OP_TOPK) exceeds 4 MiB less
+ *   256 bytes return LSA_ERR_UNSUPPORTED (about 40 rows of 128K scores fit).
  *   Allocates nothing: no cudaMalloc / cudaFree; the histograms are cleared
  *   with cudaMemsetAsync on `stream` at every call.
  *   The first call on a device looks up the array's device address (once per

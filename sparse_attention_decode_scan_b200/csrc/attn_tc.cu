@@ -111,6 +111,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 
+// 2^x on the special-function unit (ex2.approx.ftz); 2^-inf = +0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 struct RowCtx {
@@ -211,16 +218,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     const int t = threadIdx.x;
     const int sub = t & 7;         // 16-byte column chunk within each 128-byte block
     const int rbase = t >> 3;      // 0..15
-    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q) +
-                          (static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta) * kD * 2;
-    const uint32_t qs_u = tc::smem_u32(qs);
-    for (int m = 0; m < 4; ++m) {
-      const int i = rbase + 16 * m;
-      const uint8_t* src = qsrc + static_cast<int64_t>(i) * kD * 2;
-      for (int d = 0; d < kBoxes; ++d)
-        cp_async16(qs_u + d * kQBlock + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
-    }
-    cp_async_arrive_noinc(qfull);
     const bool report = sub == 0 && half == 0;
     // rows of this thread (4 per chunk) for chunks j, j+1 and j+2
     int64_t rc_[4], rn_[4], rn2_[4];
@@ -239,11 +236,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
                        "r"(kD * 2)
                        : "memory");
     };
+    // the first three chunks' lookups go out before the query copy, so their
+    // latency overlaps it
     lookup(0, rc_);
     lookup(1, rn_);
+    lookup(2, rn2_);
+    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q) +
+                          (static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta) * kD * 2;
+    const uint32_t qs_u = tc::smem_u32(qs);
+    for (int m = 0; m < 4; ++m) {
+      const int i = rbase + 16 * m;
+      const uint8_t* src = qsrc + static_cast<int64_t>(i) * kD * 2;
+      for (int d = 0; d < kBoxes; ++d)
+        cp_async16(qs_u + d * kQBlock + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
+    }
+    cp_async_arrive_noinc(qfull);
     prefetch_l2(rc_);
     prefetch_l2(rn_);
-    lookup(2, rn2_);
     for (int j = 0; j < nch; ++j) {
       const int b = j % kNBuf;
       prefetch_l2(rn2_);  // chunk j+2 (looked up during the previous iteration)
@@ -385,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       if (j > 0 && !tc::mbar_wait(pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
       const bool need = srow && (j > 0) && (m_new > m_run + kRescaleLog2);
       if (__any_sync(0xffffffffu, need)) {
-        const float alpha_own = need ? exp2f(m_run - m_new) : 1.f;
+        const float alpha_own = need ? ex2(m_run - m_new) : 1.f;
         const float alpha = __shfl_sync(0xffffffffu, alpha_own, lane & 15);
         tc::tc_fence_after();
 #pragma unroll 1
@@ -404,22 +413,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
         }
       }
       if (j == 0) m_run = m_new;
-      // probabilities (base 2), bf16 P row of this head, running sum of the rounded values
+      // probabilities (base 2): masked entries are -inf and give 2^-inf = 0; a
+      // head with no valid entry yet (m_run = -inf) gives 0 everywhere.  P is
+      // stored in bf16 and the row sum adds the rounded values.
       if (srow) {
+        const float mref = m_run == -INFINITY ? INFINITY : m_run;
+        float lsum[2] = {0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int i0 = c * 8 + 2 * u;
-            const float p0 = (m_run == -INFINITY || s[i0] == -INFINITY) ? 0.f : exp2f(s[i0] - m_run);
-            const float p1 = (m_run == -INFINITY || s[i0 + 1] == -INFINITY) ? 0.f : exp2f(s[i0 + 1] - m_run);
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            l += __low2float(pb) + __high2float(pb);
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(ex2(s[i0] - mref), ex2(s[i0 + 1] - mref));
+            const float2 pf = __bfloat1622float2(pb);
+            lsum[u & 1] += pf.x + pf.y;
             w[u] = *reinterpret_cast<const uint32_t*>(&pb);
           }
           *reinterpret_cast<uint4*>(ps + tc::sw128_offset(head_local, c)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        l += lsum[0] + lsum[1];
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
@@ -500,30 +513,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
         if (a.lse) a.lse[static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + hl] = den > 0.f ? mx + logf(den) : -INFINITY;
       }
       __syncthreads();
-      // 64 heads x 128 groups of 4 dims, spread over every thread of the CTA
+      // 64 heads x 128 groups of 4 dims, spread over every thread of the CTA;
+      // the loads of up to 4 splits are issued before they are used
       const float4* po = reinterpret_cast<const float4*>(P.part_o);
       for (int item = threadIdx.x; item < kHeadsCta * (kDv / 4); item += kThreads) {
         const int hl = item / (kDv / 4), c4 = item % (kDv / 4);
         const int h = half * kHeadsCta + hl;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        int sp = 0;
-        for (; sp + 4 <= ns; sp += 4) {
+        for (int sp0 = 0; sp0 < ns; sp0 += 4) {
           float4 x[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u)
-            x[u] = __ldcg(po + ((static_cast<int64_t>(r) * ns + sp + u) * kHeadsAll + h) * (kDv / 4) + c4);
+            x[u] = sp0 + u < ns ? __ldcg(po + ((static_cast<int64_t>(r) * ns + sp0 + u) * kHeadsAll + h) * (kDv / 4) + c4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float wgt = wsm[(sp + u) * kHeadsCta + hl];
+            const float wgt = sp0 + u < ns ? wsm[(sp0 + u) * kHeadsCta + hl] : 0.f;
             acc.x = fmaf(wgt, x[u].x, acc.x); acc.y = fmaf(wgt, x[u].y, acc.y);
             acc.z = fmaf(wgt, x[u].z, acc.z); acc.w = fmaf(wgt, x[u].w, acc.w);
           }
-        }
-        for (; sp < ns; ++sp) {
-          const float4 x = __ldcg(po + ((static_cast<int64_t>(r) * ns + sp) * kHeadsAll + h) * (kDv / 4) + c4);
-          const float wgt = wsm[sp * kHeadsCta + hl];
-          acc.x = fmaf(wgt, x.x, acc.x); acc.y = fmaf(wgt, x.y, acc.y);
-          acc.z = fmaf(wgt, x.z, acc.z); acc.w = fmaf(wgt, x.w, acc.w);
         }
         const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
         uint2 pk;

@@ -303,17 +303,132 @@ __global__ void __launch_bounds__(kT) k_topk_write(TopkArgs a, int64_t seg_len, 
 }
 
 
-// ============================================================ per-row path
+// ============================================================ three-kernel path
 constexpr int kB1 = kTopkBins1;     // 12-bit first digit
-constexpr int kCandCap = 8192;     // candidates kept per row (in shared memory)
+constexpr int kCandCap = 8192;     // candidates kept per row
 constexpr int64_t kMaxBitmapCols = 1 << 19;
 constexpr int kFinT = 1024;        // threads of the per-row CTA
-constexpr int kRowVec = 8;         // float4 loads in flight per thread
+constexpr int kWordElems = 32;     // positions per bitmap word (one thread's share of a round)
+constexpr int kColRound = kT * kWordElems;  // positions per collect round (8192)
 
-// Workspace of the per-row path: the first-digit histograms [rows][4096],
-// written by the decode scan when it runs first (hist_ready); otherwise unused.
-__device__ __forceinline__ const uint32_t* v2_hist(const TopkArgs& a) {
-  return reinterpret_cast<const uint32_t*>(a.ws);
+// Workspace: [rows][4096] first-digit histograms | [rows][words] bitmaps of the
+// keys above the threshold bin | [rows] candidate counts | [rows][kCandCap]
+// candidates (key, position).
+struct TkLayout {
+  uint32_t* hist;
+  uint32_t* bitmap;
+  uint32_t* ncand;
+  uint2* cand;
+  int64_t words;
+};
+
+__host__ __device__ inline size_t al256(size_t b) { return (b + 255) / 256 * 256; }
+
+__host__ __device__ inline TkLayout tk_layout(void* ws, int32_t rows, int64_t n_cols) {
+  TkLayout L;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  L.words = (n_cols + 31) / 32;
+  L.hist = reinterpret_cast<uint32_t*>(b);
+  b += al256(static_cast<size_t>(rows) * kB1 * 4);
+  L.ncand = reinterpret_cast<uint32_t*>(b);
+  b += al256(static_cast<size_t>(rows) * 4);
+  L.bitmap = reinterpret_cast<uint32_t*>(b);
+  b += al256(static_cast<size_t>(rows) * L.words * 4);
+  L.cand = reinterpret_cast<uint2*>(b);
+  return L;
+}
+
+// Histogram of key bits [31:20] per row (when the scan did not build it).
+__global__ void __launch_bounds__(kT) k_tk_hist12(TopkArgs a, int64_t seg_len) {
+  __shared__ uint32_t h[kB1];
+  const int r = blockIdx.y, seg = blockIdx.x;
+  const Row rr = row_range(a, r, seg, seg_len);
+  if (rr.s0 >= rr.s1) return;
+  for (int i = threadIdx.x; i < kB1; i += kT) h[i] = 0;
+  __syncthreads();
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  for (int64_t base = rr.s0; base < rr.s1; base += kRound) {
+    uint32_t key[4];
+    load_keys(row, base, rr.s1, key);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (key[j]) atomicAdd(&h[key[j] >> 20], 1u);
+  }
+  __syncthreads();
+  uint32_t* dst = tk_layout(a.ws, a.rows, a.n_cols).hist + static_cast<int64_t>(r) * kB1;
+  for (int i = threadIdx.x; i < kB1; i += kT)
+    if (h[i]) atomicAdd(dst + i, h[i]);
+}
+
+// Threshold bin b1 of each row, then each thread takes 32 consecutive
+// positions per round: the keys above b1 become one bitmap word (written once,
+// no atomics) and the keys inside b1 are appended to the row's candidates
+// (one atomic per CTA and round).  Segments are multiples of 8192 positions
+// and cover [0, n_cols), so every bitmap word is written.
+__global__ void __launch_bounds__(kT) k_tk_collect(TopkArgs a, int64_t seg_len) {
+  __shared__ int sh[kT / 32];
+  __shared__ uint32_t s_base;
+  const int r = blockIdx.y, seg = blockIdx.x;
+  int64_t n = a.n_cols;
+  if (a.valid_len) {
+    const int64_t v = __ldg(a.valid_len + r);
+    n = v < 0 ? 0 : (v < n ? v : n);
+  }
+  const int64_t s0 = static_cast<int64_t>(seg) * seg_len;
+  const int64_t s1 = s0 + seg_len < a.n_cols ? s0 + seg_len : a.n_cols;
+  if (s0 >= s1) return;
+  const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
+  const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
+  Found f = find_bin<kB1>(hist, 0xffffffffu, sh);
+  const uint32_t keff = f.total < static_cast<uint32_t>(a.k) ? f.total : static_cast<uint32_t>(a.k);
+  uint32_t b1 = 0xffffffffu;  // no selection: no bin qualifies
+  if (keff > 0) {
+    f = find_bin<kB1>(hist, keff, sh);
+    b1 = static_cast<uint32_t>(f.bin);
+  }
+  uint32_t* bitmap = L.bitmap + static_cast<int64_t>(r) * L.words;
+  uint2* cand = L.cand + static_cast<int64_t>(r) * kCandCap;
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  for (int64_t base = s0; base < s1; base += kColRound) {
+    const int64_t p0 = base + static_cast<int64_t>(threadIdx.x) * kWordElems;
+    uint32_t key[kWordElems];
+    if (p0 + kWordElems <= n) {
+      const float4* src = reinterpret_cast<const float4*>(row + p0);
+#pragma unroll
+      for (int v = 0; v < kWordElems / 4; ++v) {
+        const float4 x = __ldg(src + v);
+        key[4 * v] = order_key(x.x); key[4 * v + 1] = order_key(x.y);
+        key[4 * v + 2] = order_key(x.z); key[4 * v + 3] = order_key(x.w);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kWordElems; ++e) key[e] = p0 + e < n ? order_key(__ldg(row + p0 + e)) : 0u;
+    }
+    uint32_t word = 0;
+    int nc = 0;
+#pragma unroll
+    for (int e = 0; e < kWordElems; ++e) {
+      const uint32_t bin = key[e] ? (key[e] >> 20) : 0xffffffffu;
+      if (keff > 0 && key[e] && bin > b1) word |= 1u << e;
+      nc += (keff > 0 && key[e] && bin == b1);
+    }
+    if (p0 < a.n_cols) bitmap[p0 / kWordElems] = word;
+    int tot;
+    const int off = block_excl_scan(nc, sh, &tot);
+    if (threadIdx.x == 0) s_base = tot ? atomicAdd(L.ncand + r, static_cast<uint32_t>(tot)) : 0u;
+    __syncthreads();
+    uint32_t o = s_base + static_cast<uint32_t>(off);
+    __syncthreads();
+    if (nc) {
+#pragma unroll
+      for (int e = 0; e < kWordElems; ++e) {
+        if (keff > 0 && key[e] && (key[e] >> 20) == b1) {
+          if (o < static_cast<uint32_t>(kCandCap)) cand[o] = make_uint2(key[e], static_cast<uint32_t>(p0 + e));
+          ++o;
+        }
+      }
+    }
+  }
 }
 
 // Block-wide (kFinT threads) exclusive scan.
@@ -370,22 +485,20 @@ __device__ __forceinline__ uint32_t low_bits(uint32_t x, int n) {
   return y;
 }
 
-// One CTA per row: the first-digit histogram (from the scan, or one pass over
-// the row here), the threshold bin b1, one pass that marks every key above b1
-// in a position bitmap and keeps the keys inside b1 as candidates, a radix
-// select on the candidates' low 20 bits (or, if they overflow the list, on
-// the row again), and an ordered compaction of the bitmap.
-__global__ void __launch_bounds__(kFinT) k_tk_row(TopkArgs a) {
+// One CTA per row: keff and b1 from the histogram, the bitmap of the keys
+// above b1 and the candidates in shared memory, a radix select on the
+// candidates' low 20 bits (or, if they overflowed the list, on the row again),
+// and an ordered compaction of the bitmap.
+__global__ void __launch_bounds__(kFinT) k_tk_final(TopkArgs a) {
   extern __shared__ __align__(16) uint32_t fsm[];
   __shared__ int warp_sums[32];
   __shared__ int s_bin;
   __shared__ uint32_t s_rank;
-  __shared__ uint32_t s_nc;
   __shared__ uint32_t h[1024];
-  __shared__ uint32_t h12[kB1];
   const int r = blockIdx.x;
   const int t = threadIdx.x;
-  const int64_t nwords = (a.n_cols + 31) / 32;
+  const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
+  const int64_t nwords = L.words;
   uint32_t* bm = fsm;               // selected positions
   uint32_t* tb = fsm + nwords;      // positions equal to the threshold key
   uint2* cs = reinterpret_cast<uint2*>(fsm + 2 * nwords);  // candidates: 2*nwords words keep 8-byte alignment
@@ -396,36 +509,24 @@ __global__ void __launch_bounds__(kFinT) k_tk_row(TopkArgs a) {
     n = v < 0 ? 0 : (v < n ? v : n);
   }
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  for (int64_t w = t; w < 2 * nwords; w += kFinT) fsm[w] = 0;
-  if (t == 0) s_nc = 0;
-  // first-digit histogram
-  if (a.hist_ready) {
-    const uint32_t* g = v2_hist(a) + static_cast<int64_t>(r) * kB1;
-    for (int i = t; i < kB1; i += kFinT) h12[i] = __ldcg(g + i);
-  } else {
-    for (int i = t; i < kB1; i += kFinT) h12[i] = 0;
-    __syncthreads();
-    for (int64_t base = 0; base < n; base += kFinT * 4 * kRowVec) {
-      uint32_t key[kRowVec][4];
+  // issue every independent load first
+  const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
+  uint32_t hv[4];
 #pragma unroll
-      for (int v = 0; v < kRowVec; ++v) load_keys(row, base + v * kFinT * 4, n, key[v]);
-#pragma unroll
-      for (int v = 0; v < kRowVec; ++v)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (key[v][j]) atomicAdd(&h12[key[v][j] >> 20], 1u);
-    }
+  for (int i = 0; i < 4; ++i) hv[i] = __ldcg(hist + t * 4 + i);
+  const uint32_t n_cand = __ldcg(L.ncand + r);
+  const uint32_t* gbm = L.bitmap + static_cast<int64_t>(r) * nwords;
+  for (int64_t w = t; w < nwords; w += kFinT) {
+    bm[w] = __ldcg(gbm + w);
+    tb[w] = 0;
   }
-  __syncthreads();
+  const bool overflow = n_cand > static_cast<uint32_t>(kCandCap);
+  const int nc = overflow ? 0 : static_cast<int>(n_cand);
+  for (int c = t; c < nc; c += kFinT) cs[c] = __ldcg(L.cand + static_cast<int64_t>(r) * kCandCap + c);
   // keff and the threshold bin (4 bins per thread)
   uint32_t keff, b1, rank1;
   {
-    uint32_t v[4], mine = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[i] = h12[t * 4 + i];
-      mine += v[i];
-    }
+    const uint32_t mine = hv[0] + hv[1] + hv[2] + hv[3];
     int total;
     const int excl = fin_excl_scan(static_cast<int>(mine), warp_sums, &total);
     keff = static_cast<uint32_t>(total) < static_cast<uint32_t>(a.k) ? static_cast<uint32_t>(total)
@@ -433,12 +534,12 @@ __global__ void __launch_bounds__(kFinT) k_tk_row(TopkArgs a) {
     uint32_t cum = static_cast<uint32_t>(total - excl) - mine;
     if (keff > 0 && cum < keff && keff <= cum + mine) {
       for (int i = 3; i >= 0; --i) {
-        if (cum + v[i] >= keff) {
+        if (cum + hv[i] >= keff) {
           s_bin = t * 4 + i;
           s_rank = keff - cum;
           break;
         }
-        cum += v[i];
+        cum += hv[i];
       }
     }
     __syncthreads();
@@ -447,37 +548,6 @@ __global__ void __launch_bounds__(kFinT) k_tk_row(TopkArgs a) {
   }
   for (int i = static_cast<int>(keff) + t; i < a.k; i += kFinT) out[i] = -1;
   if (keff == 0) return;
-  // one pass: keys above b1 -> bitmap, keys in b1 -> candidates
-  for (int64_t base = 0; base < n; base += kFinT * 4 * kRowVec) {
-    uint32_t key[kRowVec][4];
-#pragma unroll
-    for (int v = 0; v < kRowVec; ++v) load_keys(row, base + v * kFinT * 4, n, key[v]);
-#pragma unroll
-    for (int v = 0; v < kRowVec; ++v) {
-      const uint32_t p0 = static_cast<uint32_t>(base + v * kFinT * 4 + t * 4);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t x = key[v][j];
-        const uint32_t bin = x >> 20;
-        const bool is_cand = x != 0u && bin == b1;
-        if (x != 0u && bin > b1) atomicOr(&bm[(p0 + j) >> 5], 1u << ((p0 + j) & 31));
-        const uint32_t m = __ballot_sync(0xffffffffu, is_cand);
-        if (m) {
-          const int lane = t & 31;
-          const int leader = __ffs(m) - 1;
-          uint32_t boff = 0;
-          if (lane == leader) boff = atomicAdd(&s_nc, static_cast<uint32_t>(__popc(m)));
-          boff = __shfl_sync(0xffffffffu, boff, leader);
-          const uint32_t off = boff + __popc(m & ((1u << lane) - 1u));
-          if (is_cand && off < static_cast<uint32_t>(kCandCap)) cs[off] = make_uint2(x, p0 + j);
-        }
-      }
-    }
-  }
-  __syncthreads();
-  const uint32_t n_cand = s_nc;
-  const bool overflow = n_cand > static_cast<uint32_t>(kCandCap);
-  const int nc = overflow ? 0 : static_cast<int>(n_cand);
   // radix select on bits [19:10] then [9:0] among the keys of bin b1
   uint32_t T = 0, ties = 0;
   for (int pass = 0; pass < 2; ++pass) {
@@ -592,32 +662,58 @@ TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
 
 bool topk_v2_ok(int64_t n_cols) { return n_cols <= kMaxBitmapCols; }
 
-size_t topk_hist_zero_bytes(int32_t rows) { return static_cast<size_t>(rows) * kB1 * 4; }
+size_t topk_hist_zero_bytes(int32_t rows) {
+  return al256(static_cast<size_t>(rows) * kB1 * 4) + al256(static_cast<size_t>(rows) * 4);
+}
 
 size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t) {
   const size_t R = static_cast<size_t>(rows);
-  if (topk_v2_ok(n_cols)) return (R * kB1 * 4 + 255) / 256 * 256;
+  if (topk_v2_ok(n_cols))
+    return topk_hist_zero_bytes(rows) + al256(R * ((n_cols + 31) / 32) * 4) + al256(R * kCandCap * 8);
   TopkPlan p = topk_plan(rows, n_cols);
   size_t b = R * kHistStride * 4 + R * p.nseg * 8;
   return (b + 255) / 256 * 256;
 }
 
-int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 1 : 5; }
+int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 3 : 5; }
+
+// Segments of the collect pass: multiples of 8192 positions, about two CTAs
+// per SM in total.
+TopkPlan collect_plan(int32_t rows, int64_t n_cols) {
+  TopkPlan p;
+  const int64_t rounds = (n_cols + kColRound - 1) / kColRound;
+  int64_t want = (2LL * kPlanSMs + rows - 1) / (rows > 0 ? rows : 1);
+  if (want > rounds) want = rounds;
+  if (want < 1) want = 1;
+  const int64_t per = (rounds + want - 1) / want;
+  p.seg_len = per * kColRound;
+  p.nseg = static_cast<int32_t>((rounds + per - 1) / per);
+  if (p.nseg < 1) p.nseg = 1;
+  return p;
+}
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   if (a.rows == 0 || a.k == 0) return cudaSuccess;
   TopkPlan p = topk_plan(a.rows, a.n_cols);
   dim3 grid(static_cast<unsigned>(p.nseg), static_cast<unsigned>(a.rows));
   if (topk_v2_ok(a.n_cols)) {
+    cudaError_t e;
+    if (!a.hist_ready) {
+      e = cudaMemsetAsync(a.ws, 0, topk_hist_zero_bytes(a.rows), s);
+      if (e != cudaSuccess) return e;
+      k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
+    }
+    const TopkPlan cp = collect_plan(a.rows, a.n_cols);
+    k_tk_collect<<<dim3(static_cast<unsigned>(cp.nseg), static_cast<unsigned>(a.rows)), kT, 0, s>>>(a, cp.seg_len);
     const int64_t nwords = (a.n_cols + 31) / 32;
     const size_t smem = 2 * nwords * 4 + static_cast<size_t>(kCandCap) * 8;
     static size_t smem_set = 0;
     if (smem > 48 * 1024 && smem > smem_set) {
-      cudaError_t e = cudaFuncSetAttribute(k_tk_row, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      e = cudaFuncSetAttribute(k_tk_final, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return e;
       smem_set = smem;
     }
-    k_tk_row<<<a.rows, kFinT, smem, s>>>(a);
+    k_tk_final<<<a.rows, kFinT, smem, s>>>(a);
     return cudaGetLastError();
   }
   size_t hist_bytes = static_cast<size_t>(a.rows) * kHistStride * 4;
@@ -646,7 +742,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
 namespace lsa {
 namespace {
 
-constexpr size_t kStaticScratchBytes = 2u << 20;  // 2 MiB: status word + histograms + segment counts
+constexpr size_t kStaticScratchBytes = 4u << 20;  // 4 MiB: status word + histograms, bitmaps, candidates
 
 static __device__ __align__(256) uint8_t g_topk_scratch[kStaticScratchBytes];
 

@@ -43,7 +43,7 @@ def test_noalloc_matches_workspace_topk_twice():
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     from sparse_attention_decode_scan_b200 import lsa
-    rows, n = 200, 4096  # 200 rows of histograms exceed the 2 MiB scratch
+    rows, n = 200, 4096  # 200 rows of top-k scratch exceed the 4 MiB array
     dev = torch.zeros((rows, n), dtype=torch.float32, device="cuda")
     idx = torch.empty((rows, 8), dtype=torch.int32, device="cuda")
     assert lsa.topk_noalloc(dev, 8, idx, raise_on_error=False) == lsa.LSA_ERR_UNSUPPORTED
