@@ -21,7 +21,9 @@
 //   warp 4     MMA issuer: S = Q K^T (36 x M64N64K16), O += P V (8 x M64N256K16),
 //              V read MN-major from the same tile as K
 //   warps 5-8  online softmax (base 2, lazy rescale when the max grows by > 8),
-//              P to shared memory, final normalisation
+//              P[64 heads x 64 rows] written over the chunk's rope block (dims
+//              512-575, dead once S is computed), so P is double-buffered with
+//              the chunks and the softmax of chunk j+1 overlaps P V of chunk j
 // (Below N = 64 an MMA costs as much as at N = 64 on this part, so 64-row
 // chunks halve the score MMAs per row compared with 32-row chunks.)
 // With several splits per row, each CTA writes a normalised partial and its
@@ -47,11 +49,11 @@ constexpr int kBoxBytes = kChunk * 128;    // 64 rows x 128 B
 constexpr int kKvBytes = kBoxes * kBoxBytes;          // 73728
 constexpr int kQBlock = kHeadsCta * 128;              // 8192
 constexpr int kQBytes = kBoxes * kQBlock;             // 73728
-constexpr int kPBytes = kHeadsCta * 128;              // 8192: P [64 heads x 64 rows] bf16
+constexpr int kRopeBox = kBoxes - 1;                  // column block of dims 512-575; holds P after S
 constexpr int kThreads = 288;
 constexpr int kProdThreads = 128;
 constexpr int kWarpMma = 4;                // warps 5-8: softmax
-constexpr int kSmemBytes = kQBytes + kNBuf * kKvBytes + kPBytes + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr int kSmemBytes = kQBytes + kNBuf * kKvBytes + 1024 /*barriers*/ + 1024 /*align*/;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256;            // score buffers start column
 constexpr float kLog2e = 1.4426950408889634f;
@@ -136,15 +138,36 @@ __device__ __forceinline__ RowCtx row_ctx(const AttnArgs& a, int r) {
   return c;
 }
 
-// Stored KV row of list entry j of row r, or -1 (padding, out of range, bad block).
-__device__ __forceinline__ int64_t entry_row(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r, int j,
-                                             int j1, bool report) {
-  if (j >= j1 || !rc.ok) return -1;
-  const int32_t pos = __ldg(a.idx + static_cast<int64_t>(r) * a.k + j);
-  if (pos < 0) return -1;
-  const int64_t row = pos < rc.L ? ad.row(rc.b, pos) : -1;
-  if (row < 0 && report) record_error(a.status, LSA_ERR_BOUNDS, r, pos);
-  return row;
+// Stored rows of list entries j[0..N) of row r (-1: padding, out of range or
+// bad block).  All index loads are issued before the block-table loads.
+template <int N>
+__device__ __forceinline__ void entry_rows(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r,
+                                           const int (&j)[N], int j1, bool report, int64_t (&out)[N]) {
+  int32_t pos[N];
+#pragma unroll
+  for (int m = 0; m < N; ++m)
+    pos[m] = (j[m] < j1 && rc.ok) ? __ldg(a.idx + static_cast<int64_t>(r) * a.k + j[m]) : -1;
+  if (ad.block_size == 0) {
+#pragma unroll
+    for (int m = 0; m < N; ++m) out[m] = (pos[m] >= 0 && pos[m] < rc.L) ? static_cast<int64_t>(rc.b) * ad.max_len + pos[m] : -1;
+  } else {
+    int32_t blk[N];
+#pragma unroll
+    for (int m = 0; m < N; ++m) {
+      const int64_t lb = pos[m] / ad.block_size;
+      blk[m] = (pos[m] >= 0 && pos[m] < rc.L && lb < ad.max_blocks)
+                   ? __ldg(ad.block_table + static_cast<int64_t>(rc.b) * ad.max_blocks + lb) : -1;
+    }
+#pragma unroll
+    for (int m = 0; m < N; ++m)
+      out[m] = (blk[m] >= 0 && blk[m] < ad.n_blocks)
+                   ? static_cast<int64_t>(blk[m]) * ad.block_size + (pos[m] % ad.block_size) : -1;
+  }
+  if (report) {
+#pragma unroll
+    for (int m = 0; m < N; ++m)
+      if (pos[m] >= 0 && out[m] < 0) record_error(a.status, LSA_ERR_BOUNDS, r, pos[m]);
+  }
 }
 
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* o, const float (&v)[32], float inv) {
@@ -166,8 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qs = smem;
   uint8_t* kvs = qs + kQBytes;         // kNBuf chunk buffers
-  uint8_t* ps = kvs + kNBuf * kKvBytes;  // P
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + kPBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kvs + kNBuf * kKvBytes);
   uint64_t* qfull = bars;
   uint64_t* kvfull = bars + 1;            // [kNBuf]
   uint64_t* kvempty = kvfull + kNBuf;     // [kNBuf]
@@ -222,9 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     // rows of this thread (4 per chunk) for chunks j, j+1 and j+2
     int64_t rc_[4], rn_[4], rn2_[4];
     auto lookup = [&](int jj, int64_t (&dst)[4]) {
+      int jl[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-        dst[m] = jj < nch ? entry_row(a, ad, rc, r, j0 + jj * kChunk + rbase + 16 * m, j1, report) : -1;
+      for (int m = 0; m < 4; ++m) jl[m] = jj < nch ? j0 + jj * kChunk + rbase + 16 * m : j1;
+      entry_rows<4>(a, ad, rc, r, jl, j1, report, dst);
     };
     auto prefetch_l2 = [&](const int64_t (&rows)[4]) {
       if (sub != 0) return;
@@ -297,20 +320,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
       const uint32_t q_u = tc::smem_u32(qs);
       bool ok = tc::mbar_wait(qfull, 0, abort_flag);
       tc::fence_proxy_async_smem();
-      const uint32_t p_u = tc::smem_u32(ps);
       auto issue_pv = [&](int i) -> bool {
         if (!tc::mbar_wait(pfull, i & 1, abort_flag)) return false;
         tc::tc_fence_after();
         const uint32_t kv_u = tc::smem_u32(kvs + (i % kNBuf) * kKvBytes);
+        const uint32_t p_u = kv_u + kRopeBox * kBoxBytes;  // P(i) sits in chunk i's rope block
+        const uint64_t pa0 = tc::desc_sw128(p_u), vb0 = desc_sw128_mn(kv_u, kBoxBytes);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const uint32_t d = tmem + (static_cast<uint32_t>(16 * c) << 16);  // dims 256c.. at lane offset 16c
 #pragma unroll
-          for (int kk = 0; kk < kChunk / 16; ++kk) {
-            const uint64_t ad_ = tc::desc_sw128(p_u + kk * 32);
-            const uint64_t bd_ = desc_sw128_mn(kv_u + (4 * c) * kBoxBytes + kk * 2048, kBoxBytes);
-            tc::mma_f16(d, ad_, bd_, kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kChunk / 16; ++kk)
+            tc::mma_f16(d, pa0 + static_cast<uint64_t>((kk * 32) >> 4),
+                        vb0 + static_cast<uint64_t>(((4 * c) * kBoxBytes + kk * 2048) >> 4), kIdescPV,
+                        (i > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(pvdone);
         tc::mma_commit(&kvempty[i % kNBuf]);
@@ -324,14 +347,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
         tc::tc_fence_after();
         const uint32_t kv_u = tc::smem_u32(kvs + b * kKvBytes);
         const uint32_t d = tmem + kColS + sb * kChunk;
-#pragma unroll 1
+        // descriptors of the 36 K-steps differ only in the start-address field
+        // (addresses stay below 256 KB, so the 14-bit field never carries)
+        const uint64_t a0 = tc::desc_sw128(q_u), b0 = tc::desc_sw128(kv_u);
+#pragma unroll
         for (int blk = 0; blk < kBoxes; ++blk) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad_ = tc::desc_sw128(q_u + blk * kQBlock + k * 32);
-            const uint64_t bd_ = tc::desc_sw128(kv_u + blk * kBoxBytes + k * 32);
-            tc::mma_f16(d, ad_, bd_, kIdescQK, (blk | k) != 0);
-          }
+          for (int k = 0; k < 4; ++k)
+            tc::mma_f16(d, a0 + static_cast<uint64_t>((blk * kQBlock + k * 32) >> 4),
+                        b0 + static_cast<uint64_t>((blk * kBoxBytes + k * 32) >> 4), kIdescQK, (blk | k) != 0);
         }
         tc::mma_commit(&sfull[sb]);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
@@ -355,15 +379,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
     // validity of the chunk's rows (lane and lane + 32), looked up one chunk ahead
-    bool va = nch > 0 && entry_row(a, ad, rc, r, j0 + lane, j1, false) >= 0;
-    bool vb = nch > 0 && entry_row(a, ad, rc, r, j0 + 32 + lane, j1, false) >= 0;
+    auto valid2 = [&](int jj, bool* x, bool* y) {
+      const int jl[2] = {jj < nch ? j0 + jj * kChunk + lane : j1, jj < nch ? j0 + jj * kChunk + 32 + lane : j1};
+      int64_t rr[2];
+      entry_rows<2>(a, ad, rc, r, jl, j1, false, rr);
+      *x = rr[0] >= 0;
+      *y = rr[1] >= 0;
+    };
+    bool va, vb;
+    valid2(0, &va, &vb);
     for (int j = 0; j < nch; ++j) {
       const int sb = j & 1;
       const uint32_t mlo = __ballot_sync(0xffffffffu, va), mhi = __ballot_sync(0xffffffffu, vb);
-      if (j + 1 < nch) {
-        va = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + lane, j1, false) >= 0;
-        vb = entry_row(a, ad, rc, r, j0 + (j + 1) * kChunk + 32 + lane, j1, false) >= 0;
-      }
+      if (j + 1 < nch) valid2(j + 1, &va, &vb);
       if (!tc::mbar_wait(&sfull[sb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       tc::tc_fence_after();
       float s[64];
@@ -389,11 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
         mx = fmaxf(mx, s[i]);
       }
       const float m_new = fmaxf(m_run, mx);
-      // P is single-buffered: P V of chunk j-1 must be done before P(j) is written
-      // (which also makes a rescale of O safe)
-      if (j > 0 && !tc::mbar_wait(pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
       const bool need = srow && (j > 0) && (m_new > m_run + kRescaleLog2);
       if (__any_sync(0xffffffffu, need)) {
+        // a rescale touches O: P V of chunk j-1 must have finished
+        if (!tc::mbar_wait(pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
         const float alpha_own = need ? ex2(m_run - m_new) : 1.f;
         const float alpha = __shfl_sync(0xffffffffu, alpha_own, lane & 15);
         tc::tc_fence_after();
@@ -430,7 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
             lsum[u & 1] += pf.x + pf.y;
             w[u] = *reinterpret_cast<const uint32_t*>(&pb);
           }
-          *reinterpret_cast<uint4*>(ps + tc::sw128_offset(head_local, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(kvs + (j % kNBuf) * kKvBytes + kRopeBox * kBoxBytes +
+                                    tc::sw128_offset(head_local, c)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         l += lsum[0] + lsum[1];
       }
@@ -494,8 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
     if (*last_flag) {
       __threadfence();
       if (threadIdx.x == 0) P.counters[2 * r + half] = 0;  // left zeroed for the next call
-      // weights of every split for the 64 heads, in the (now idle) P buffers
-      float* wsm = reinterpret_cast<float*>(ps);          // [nsplit][64] in the idle P buffer, nsplit <= 32
+      // weights of every split for the 64 heads
+      float* wsm = reinterpret_cast<float*>(kvs);         // [nsplit][64] in the idle chunk buffer, nsplit <= 32
       const int ns = P.nsplit;
       const float* lse_p = P.part_lse + static_cast<int64_t>(r) * ns * kHeadsAll + half * kHeadsCta;
       if (threadIdx.x < kHeadsCta) {
@@ -513,32 +541,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
         if (a.lse) a.lse[static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + hl] = den > 0.f ? mx + logf(den) : -INFINITY;
       }
       __syncthreads();
-      // 64 heads x 128 groups of 4 dims, spread over every thread of the CTA;
-      // the loads of up to 4 splits are issued before they are used
+      // 64 heads x 128 groups of 4 dims over every thread of the CTA, eight
+      // groups per pass with the loads of two splits in flight together
       const float4* po = reinterpret_cast<const float4*>(P.part_o);
-      for (int item = threadIdx.x; item < kHeadsCta * (kDv / 4); item += kThreads) {
-        const int hl = item / (kDv / 4), c4 = item % (kDv / 4);
-        const int h = half * kHeadsCta + hl;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp0 = 0; sp0 < ns; sp0 += 4) {
-          float4 x[4];
+      constexpr int kItems = kHeadsCta * (kDv / 4);
+      for (int it0 = threadIdx.x; it0 < kItems; it0 += 8 * kThreads) {
+        float4 acc[8];
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            x[u] = sp0 + u < ns ? __ldcg(po + ((static_cast<int64_t>(r) * ns + sp0 + u) * kHeadsAll + h) * (kDv / 4) + c4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp0 = 0; sp0 < ns; sp0 += 2) {
+          float4 x[8][2];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float wgt = sp0 + u < ns ? wsm[(sp0 + u) * kHeadsCta + hl] : 0.f;
-            acc.x = fmaf(wgt, x[u].x, acc.x); acc.y = fmaf(wgt, x[u].y, acc.y);
-            acc.z = fmaf(wgt, x[u].z, acc.z); acc.w = fmaf(wgt, x[u].w, acc.w);
+          for (int u = 0; u < 8; ++u) {
+            const int item = it0 + u * kThreads;
+            const int hl = item / (kDv / 4), c4 = item % (kDv / 4);
+            const int h = half * kHeadsCta + hl;
+#pragma unroll
+            for (int v = 0; v < 2; ++v)
+              x[u][v] = (item < kItems && sp0 + v < ns)
+                            ? __ldcg(po + ((static_cast<int64_t>(r) * ns + sp0 + v) * kHeadsAll + h) * (kDv / 4) + c4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int item = it0 + u * kThreads;
+            const int hl = (item < kItems ? item : 0) / (kDv / 4);
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              const float wgt = sp0 + v < ns ? wsm[(sp0 + v) * kHeadsCta + hl] : 0.f;
+              acc[u].x = fmaf(wgt, x[u][v].x, acc[u].x); acc[u].y = fmaf(wgt, x[u][v].y, acc[u].y);
+              acc[u].z = fmaf(wgt, x[u][v].z, acc[u].z); acc[u].w = fmaf(wgt, x[u][v].w, acc[u].w);
+            }
           }
         }
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
-                                  (static_cast<int64_t>(r) * kHeadsAll + h) * kDv + c4 * 4) = pk;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int item = it0 + u * kThreads;
+          if (item >= kItems) continue;
+          const int hl = item / (kDv / 4), c4 = item % (kDv / 4);
+          const int h = half * kHeadsCta + hl;
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[u].x, acc[u].y), hi = __floats2bfloat162_rn(acc[u].z, acc[u].w);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                    (static_cast<int64_t>(r) * kHeadsAll + h) * kDv + c4 * 4) = pk;
+        }
       }
     }
   }
