@@ -147,7 +147,8 @@ def source_hash(paths) -> str:
 
 SCAN_SOURCES = ["sparse_attention_decode_scan_b200/csrc/indexer_tc.cu",
                 "sparse_attention_decode_scan_b200/csrc/indexer_simt.cu",
-                "sparse_attention_decode_scan_b200/csrc/common.cuh"]
+                "sparse_attention_decode_scan_b200/csrc/common.cuh",
+                "sparse_attention_decode_scan_b200/csrc/tc.cuh"]
 
 
 def scan_traffic(workload: str):
