@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -37,6 +38,9 @@ constexpr int kHeads = 64;       // indexer heads
 constexpr int kDim = 128;        // indexer head dim
 constexpr int kTile = 128;       // tokens per tile (MMA M, TMEM lanes)
 constexpr int kBoxRows = 64;     // rows per TMA box (one 64-token page or half tile)
+constexpr int kBoxX = 32;        // 4-byte TMA elements per 128-byte K block
+constexpr int kScaleBox = 68;    // FP8 scales per box load: 64 + up to 3 for the 16-byte aligned start
+constexpr int kScaleSlot = 96;   // floats per scale slot: a TMA destination starts on a 128-byte boundary
 constexpr int kThreads = 224;    // 7 warps
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpQ = 2, kWarpEpi = 3;
 constexpr int kSmemLimit = 232448;
@@ -51,23 +55,32 @@ struct Cfg {
   static constexpr int kBoxBytes = kBoxRows * 128;
   static constexpr int kQKBlockBytes = kN * 128;                   // B: N rows x 128 B per K block
   static constexpr int kQBytes = kKBlocks * kQKBlockBytes;
-  static constexpr int kNQ = QB == 1 ? 2 : 1;                      // query operand buffers
+  static constexpr int kNQ = (QB == 1 && kFp8) ? 2 : 1;            // query operand buffers
   static constexpr int kWBytes = QB * kHeads * 4;
   static constexpr int kHistBytes = QB == 1 ? kTopkBins1 * 4 : 0;  // fused first top-k histogram (decode)
-  static constexpr int kFixed = kNQ * kQBytes + kNQ * kWBytes + kHistBytes + 1024 /*barriers, scratch*/ +
+  // Per stage besides the keys: the key rows of its two boxes (written by the
+  // producer for the epilogue) and, for FP8, the two boxes' scales (TMA).
+  static constexpr int kMetaBytes = 2 * 4 + (kFp8 ? 2 * kScaleSlot * 4 : 0);
+  static constexpr int kRawBytes = kFp8 ? QB * kHeads * kDim * 2 : 0;  // FP8: bf16 query rows before the split
+  static constexpr int kFixed = kNQ * kQBytes + kNQ * kWBytes + kRawBytes + kHistBytes + 512 /*barriers, scratch*/ +
                                 1024 /*align*/;
-  static constexpr int kNSmax = (kSmemLimit - kFixed) / kTileBytes;
-  static constexpr int kNS = kNSmax > 8 ? 8 : kNSmax;              // key stages
+  static constexpr int kNSmax = (kSmemLimit - kFixed) / (kTileBytes + kMetaBytes);
+  static constexpr int kNS = kNSmax > 12 ? 12 : kNSmax;            // key stages
   static constexpr int kAccCols = kN;
   static constexpr int kTmemCols = 2 * kN <= 32 ? 32 : 2 * kN <= 64 ? 64 : 2 * kN <= 128 ? 128
                                    : 2 * kN <= 256 ? 256 : 512;
-  static constexpr int kSmemBytes = kNS * kTileBytes + kFixed;
+  static constexpr int kSmemBytes = kNS * (kTileBytes + kMetaBytes) + kFixed;
   static constexpr uint32_t kIdesc = tc::idesc(kFp8 ? tc::kFmtE4M3 : tc::kFmtBF16,
                                                kFp8 ? tc::kFmtE4M3 : tc::kFmtBF16, kTile, kN);
   static_assert(kNS >= 3, "too few key stages");
   static_assert(2 * kN <= 512, "accumulators exceed TMEM");
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
+
+// Stages of the configurations that run: decode 6 (bf16) and 9 (FP8) tiles in
+// flight, the causal prefill 5 (bf16, 4 rows per tile) and 9 (FP8, 2 rows).
+static_assert(Cfg<LSA_BF16, 1>::kNS == 6 && Cfg<LSA_FP8_E4M3, 1>::kNS == 9, "decode stages");
+static_assert(Cfg<LSA_BF16, 4>::kNS == 5 && Cfg<LSA_FP8_E4M3, 2>::kNS == 9, "prefill stages");
 
 // ---------------------------------------------------------------- work items
 
@@ -177,6 +190,28 @@ struct Plan {
 // group holding its first tile.
 template <int QB>
 __device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
+  Plan p;
+  p.r_first = 0;
+  p.j_first = 0;
+  if (a.rows <= kThreads) {  // one row per thread: a single block scan
+    const int r = threadIdx.x;
+    int64_t t = 0;
+    if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
+    int64_t incl, tot;
+    block_sum_i64_scan(t, sbuf, &incl, &tot);
+    const int64_t t0 = tot * blockIdx.x / gridDim.x;
+    p.n_items = tot * (blockIdx.x + 1) / gridDim.x - t0;
+    if (p.n_items <= 0) return p;
+    const int64_t start = incl - t;
+    if (t > 0 && start <= t0 && t0 < start + t) {  // exactly one thread holds tile t0
+      sfound[0] = r;
+      sfound[1] = static_cast<int>(t0 - start);
+    }
+    __syncthreads();
+    p.r_first = sfound[0];
+    p.j_first = sfound[1];
+    return p;
+  }
   int64_t total = 0;
   for (int base = 0; base < a.rows; base += kThreads) {
     const int r = base + threadIdx.x;
@@ -186,12 +221,9 @@ __device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
     block_sum_i64_scan(t, sbuf, &incl, &tot);
     total += tot;
   }
-  Plan p;
   const int64_t t0 = total * blockIdx.x / gridDim.x;
   const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
   p.n_items = t1 - t0;
-  p.r_first = 0;
-  p.j_first = 0;
   if (p.n_items <= 0) return p;
   if (threadIdx.x == 0) sfound[0] = -1;
   __syncthreads();
@@ -219,22 +251,27 @@ __device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
 // ---------------------------------------------------------------- query staging
 
 // bf16: B row n = qq * 64 + h holds q[row r0+qq][h][:] in two 128-byte K blocks.
+// Every 16-byte piece (and the weights) is a cp.async issued at once, so the
+// staging costs one memory round trip even while the key loads crowd the
+// memory system; rows of absent queries are zero-filled.
 template <int QB>
 __device__ void stage_query_bf16(const ScoresArgs& a, const Group& g, uint8_t* qbuf, float* wbuf, int lane) {
   constexpr int N = kHeads * QB;
-  const uint4* src = reinterpret_cast<const uint4*>(a.q_idx);
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q_idx);
   for (int idx = lane; idx < N * (kDim / 8); idx += 32) {
     const int n = idx >> 4, c = idx & 15;
     const int qq = n / kHeads, h = n % kHeads;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (qq < g.nrows) v = __ldg(src + ((static_cast<int64_t>(g.r0 + qq) * kHeads + h) * kDim) / 8 + c);
-    const int kb = c >> 3, cc = c & 7;
-    *reinterpret_cast<uint4*>(qbuf + kb * (N * 128) + tc::sw128_offset(n, cc)) = v;
+    const bool live = qq < g.nrows;
+    const uint8_t* p = src + ((static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + h) * kDim) * 2 + c * 16;
+    tc::cp_async16_zfill(qbuf + (c >> 3) * (N * 128) + tc::sw128_offset(n, c & 7), p, live ? 16u : 0u);
   }
-  for (int i = lane; i < QB * kHeads; i += 32) {
-    const int qq = i / kHeads;
-    wbuf[i] = qq < g.nrows ? __ldg(a.w + static_cast<int64_t>(g.r0 + qq) * kHeads + (i % kHeads)) : 0.f;
+  for (int i = lane; i < QB * (kHeads / 4); i += 32) {
+    const int qq = i / (kHeads / 4), c = i % (kHeads / 4);
+    const bool live = qq < g.nrows;
+    tc::cp_async16_zfill(wbuf + qq * kHeads + c * 4, a.w + static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + c * 4,
+                         live ? 16u : 0u);
   }
+  tc::cp_async_wait_all();
 }
 
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
@@ -247,52 +284,91 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 // q*s = hi + lo with hi = e4m3(q*s), lo = e4m3(q*s - hi), exact for bf16 q
 // (4 + 4 significant bits) outside the e4m3 subnormal range.  B row
 // qq*128 + h holds hi, qq*128 + 64 + h holds lo; w' = w / s.
+// The raw rows and the weights arrive by cp.async in one round trip; half a
+// warp then converts one head (8 dims per lane) from shared memory.
 template <int QB>
-__device__ void stage_query_fp8(const ScoresArgs& a, const Group& g, uint8_t* qbuf, float* wbuf, int lane) {
-  const uint16_t* q = reinterpret_cast<const uint16_t*>(a.q_idx);
-  for (int n = lane; n < QB * kHeads; n += 32) {
+__device__ void stage_query_fp8(const ScoresArgs& a, const Group& g, uint8_t* qbuf, float* wbuf, uint8_t* raw,
+                                int lane) {
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q_idx);
+  for (int idx = lane; idx < QB * kHeads * (kDim / 8); idx += 32) {
+    const int n = idx >> 4, c = idx & 15;
     const int qq = n / kHeads, h = n % kHeads;
     const bool live = qq < g.nrows;
-    const uint16_t* src = q + (static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + h) * kDim;
+    const uint8_t* p = src + ((static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + h) * kDim) * 2 + c * 16;
+    tc::cp_async16_zfill(raw + n * (kDim * 2) + c * 16, p, live ? 16u : 0u);
+  }
+  for (int i = lane; i < QB * (kHeads / 4); i += 32) {
+    const int qq = i / (kHeads / 4), c = i % (kHeads / 4);
+    const bool live = qq < g.nrows;
+    tc::cp_async16_zfill(wbuf + qq * kHeads + c * 4, a.w + static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + c * 4,
+                         live ? 16u : 0u);
+  }
+  tc::cp_async_wait_all();
+  __syncwarp();
+  const int half = lane >> 4, seg = lane & 15;  // seg: dims [8 seg, 8 seg + 8)
+#pragma unroll 2
+  for (int n0 = 0; n0 < QB * kHeads; n0 += 2) {
+    const int n = n0 + half;
+    const int qq = n / kHeads, h = n % kHeads;
+    const uint4 v = *reinterpret_cast<const uint4*>(raw + n * (kDim * 2) + seg * 16);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    float x[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      x[2 * j] = __uint_as_float(wv[j] << 16);
+      x[2 * j + 1] = __uint_as_float(wv[j] & 0xffff0000u);
+    }
     float mx = 0.f;
-    for (int d = 0; d < kDim; ++d) mx = fmaxf(mx, fabsf(bf16_bits_to_float(__ldg(src + d))));
-    float s = 1.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(x[j]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    // Largest power of two s = 2^k with mx * s <= 448 = 1.75 * 2^8: for
+    // mx = m * 2^E (1 <= m < 2), k = 8 - E if m <= 1.75, else 7 - E.
+    int k = 0;
     if (mx > 0.f) {
-      int e;
-      frexpf(448.f / mx, &e);  // 448/mx = f * 2^e, f in [0.5, 1)
-      s = ldexpf(1.f, e - 1);  // largest power of two <= 448 / mx
+      const uint32_t mb = __float_as_uint(mx);
+      const int E = static_cast<int>(mb >> 23) - 127;
+      k = (mb & 0x7fffffu) <= 0x600000u ? 8 - E : 7 - E;
+      k = k < -126 ? -126 : (k > 126 ? 126 : k);
+    }
+    const float sc = __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+    const float inv = __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
+    uint32_t hw[2], lw[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float xs[4], lv[4];
+#pragma unroll
+      for (int e4 = 0; e4 < 4; ++e4) xs[e4] = x[4 * u + e4] * sc;
+      hw[u] = pack_e4m3x4(xs[0], xs[1], xs[2], xs[3]);
+#pragma unroll
+      for (int e4 = 0; e4 < 4; ++e4) lv[e4] = xs[e4] - e4m3_to_float(static_cast<uint8_t>(hw[u] >> (8 * e4)));
+      lw[u] = pack_e4m3x4(lv[0], lv[1], lv[2], lv[3]);
     }
     const int row_hi = qq * 2 * kHeads + h, row_lo = row_hi + kHeads;
-    for (int c = 0; c < 8; ++c) {  // 16-byte chunks of 16 dims
-      uint32_t hw[4], lw[4];
-      for (int u = 0; u < 4; ++u) {
-        float x[4], hv[4], lv[4];
-        for (int e4 = 0; e4 < 4; ++e4) x[e4] = live ? bf16_bits_to_float(__ldg(src + c * 16 + u * 4 + e4)) * s : 0.f;
-        hw[u] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
-        for (int e4 = 0; e4 < 4; ++e4) {
-          hv[e4] = e4m3_to_float(static_cast<uint8_t>(hw[u] >> (8 * e4)));
-          lv[e4] = x[e4] - hv[e4];
-        }
-        lw[u] = pack_e4m3x4(lv[0], lv[1], lv[2], lv[3]);
-      }
-      *reinterpret_cast<uint4*>(qbuf + tc::sw128_offset(row_hi, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(qbuf + tc::sw128_offset(row_lo, c)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-    wbuf[n] = live ? __ldg(a.w + static_cast<int64_t>(g.r0 + qq) * kHeads + h) / s : 0.f;
+    const uint32_t off = (seg & 1) * 8;
+    *reinterpret_cast<uint2*>(qbuf + tc::sw128_offset(row_hi, seg >> 1) + off) = make_uint2(hw[0], hw[1]);
+    *reinterpret_cast<uint2*>(qbuf + tc::sw128_offset(row_lo, seg >> 1) + off) = make_uint2(lw[0], lw[1]);
+    if (seg == 0) wbuf[n] *= inv;  // w / s, exact for a power of two
   }
 }
 
 // ---------------------------------------------------------------- the kernel
 
 template <int KDT, int QB>
-__global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmap, const ScoresArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmap,
+                                                         const __grid_constant__ CUtensorMap smap, const ScoresArgs a) {
   using C = Cfg<KDT, QB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* qbufs = stages + C::kNS * C::kTileBytes;
+  // Offsets keep every TMA destination 128-byte and every cp.async one 16-byte aligned.
+  uint8_t* qbufs = stages + C::kNS * C::kTileBytes;                                  // 1024-aligned operands
   float* wbufs = reinterpret_cast<float*>(qbufs + C::kNQ * C::kQBytes);
-  uint32_t* shist = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(wbufs) + C::kNQ * C::kWBytes);
+  uint8_t* qraw = reinterpret_cast<uint8_t*>(wbufs) + C::kNQ * C::kWBytes;          // FP8: raw query rows
+  float* sscale = reinterpret_cast<float*>(qraw + C::kRawBytes);                     // FP8: [kNS][2][kScaleSlot]
+  int32_t* smeta = reinterpret_cast<int32_t*>(sscale + (C::kFp8 ? C::kNS * 2 * kScaleSlot : 0));  // [kNS][2]
+  uint32_t* shist = reinterpret_cast<uint32_t*>(smeta + 2 * C::kNS);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(shist) + C::kHistBytes);
   uint64_t* full = bars;
   uint64_t* empty = full + C::kNS;
@@ -309,10 +385,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
   sbuf = reinterpret_cast<int64_t*>((reinterpret_cast<uintptr_t>(sbuf) + 7) & ~uintptr_t(7));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The epilogue reads a stage's key rows (paged cache) and scales (FP8); a
+  // contiguous bf16 cache needs neither, and its stages free at MMA completion.
+  const bool stage_meta = C::kFp8 || a.cache.block_size > 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kNS; ++s) {
       tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], 1);
+      tc::mbar_init(&empty[s], stage_meta ? 1 + 4 : 1);  // MMA commit (+ 4 epilogue warps done with the stage)
     }
     for (int s = 0; s < C::kNQ; ++s) {
       tc::mbar_init(&qfull[s], 1);
@@ -327,7 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == kWarpProd && lane == 0) tc::prefetch_tmap(&tmap);
+  if (warp == kWarpProd && lane == 0) {
+    tc::prefetch_tmap(&tmap);
+    if (C::kFp8) tc::prefetch_tmap(&smap);
+  }
   if (warp == kWarpMma) {
     tc::tmem_alloc(tmem_slot, C::kTmemCols);
     tc::tc_fence_before();
@@ -339,38 +421,80 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
   CacheAddr ad{a.cache.block_table, a.cache.max_blocks, a.cache.block_size, a.cache.n_blocks, a.cache.max_len};
 
   if (warp == kWarpProd) {
-    // The whole warp looks up the block-table rows of 32 tiles at a time (one
-    // tile per lane, next batch loaded while this one is issued); lane 0 issues
-    // the TMA loads.  A single thread doing the lookups serially would wait one
-    // global-load latency per tile.
+    // The whole warp looks up the block-table entries of 32 tiles at a time
+    // (one tile per lane) and lane 0 issues their TMA loads.  The next batch's
+    // entries are loaded before the current batch is issued and only read
+    // after it, so their latency hides behind the 32 issues; a single thread
+    // doing the lookups serially would wait one load latency per tile.
     if (plan.n_items > 0) {
-      Walker<QB> Wb;
-      Wb.start(a, plan.r_first, plan.j_first);
-      auto lookup = [&](const Walker<QB>& base, int64_t base_item, int64_t* r0, int64_t* r1) {
+      struct Look {
+        int64_t p0, vis;  // first position of the tile; visible positions of its group
+        int b, r0;
+        int32_t blk[2];   // block-table entries of the tile's two boxes (paged cache)
+        bool live;
+      };
+      auto look = [&](const Walker<QB>& base, int64_t base_item) -> Look {
         Walker<QB> w = base;
-        for (int i = 0; i < lane; ++i) w.next(a);
-        *r0 = -2;
-        *r1 = -2;  // -2: no such item
-        if (base_item + lane < plan.n_items) {
-          const int64_t p0 = static_cast<int64_t>(w.j) * kTile;
-          *r0 = p0 < w.g.vis ? ad.row(w.g.b, p0) : -3;             // -3: past the visible range
-          *r1 = p0 + kBoxRows < w.g.vis ? ad.row(w.g.b, p0 + kBoxRows) : -3;
-          if (*r0 == -1) record_error(a.status, LSA_ERR_BOUNDS, w.g.r0, static_cast<int>(p0));
-          if (*r1 == -1) record_error(a.status, LSA_ERR_BOUNDS, w.g.r0, static_cast<int>(p0 + kBoxRows));
+        if (w.j + lane < w.g.tiles) w.j += lane;  // same group: no walk
+        else
+          for (int i = 0; i < lane; ++i) w.next(a);
+        Look L;
+        L.live = base_item + lane < plan.n_items;
+        L.p0 = static_cast<int64_t>(w.j) * kTile;
+        L.vis = w.g.vis;
+        L.b = w.g.b;
+        L.r0 = w.g.r0;
+        L.blk[0] = L.blk[1] = -1;
+        if (L.live && ad.block_size > 0) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int64_t p = L.p0 + h * kBoxRows;
+            const int64_t lb = p / ad.block_size;
+            if (p < L.vis && lb < ad.max_blocks)
+              L.blk[h] = __ldg(ad.block_table + static_cast<int64_t>(L.b) * ad.max_blocks + lb);
+          }
+        }
+        return L;
+      };
+      // Key rows of the two boxes: >= 0 a row, -3 past the visible range, -2 no such item.
+      auto resolve = [&](const Look& L, int64_t* rows) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t p = L.p0 + h * kBoxRows;
+          int64_t r = -2;
+          if (L.live) {
+            if (p >= L.vis) {
+              r = -3;
+            } else if (ad.block_size == 0) {
+              r = static_cast<int64_t>(L.b) * ad.max_len + p;
+            } else {
+              const int64_t lb = p / ad.block_size;
+              const int32_t blk = L.blk[h];
+              r = (lb < ad.max_blocks && blk >= 0 && blk < ad.n_blocks)
+                      ? static_cast<int64_t>(blk) * ad.block_size + (p - lb * ad.block_size)
+                      : -1;
+              if (r == -1) record_error(a.status, LSA_ERR_BOUNDS, L.r0, static_cast<int>(p));
+            }
+          }
+          rows[h] = r;
         }
       };
-      int64_t cur0, cur1;
-      lookup(Wb, 0, &cur0, &cur1);
+      Walker<QB> Wb;
+      Wb.start(a, plan.r_first, plan.j_first);
+      Look cur = look(Wb, 0);
       int64_t it = 0;
       bool failed = false;
       for (int64_t base_item = 0; base_item < plan.n_items && !failed; base_item += 32) {
+        int64_t cur_rows[2];
+        resolve(cur, cur_rows);
         Walker<QB> Wn = Wb;
-        for (int i = 0; i < 32; ++i) Wn.next(a);
-        int64_t nxt0 = -2, nxt1 = -2;
-        if (base_item + 32 < plan.n_items) lookup(Wn, base_item + 32, &nxt0, &nxt1);
+        if (Wn.j + 32 < Wn.g.tiles) Wn.j += 32;
+        else
+          for (int i = 0; i < 32; ++i) Wn.next(a);
+        const Look nxt = look(Wn, base_item + 32);  // loads stay in flight during the issues below
         const int nb = static_cast<int>(plan.n_items - base_item < 32 ? plan.n_items - base_item : 32);
         for (int i = 0; i < nb; ++i) {
-          const int64_t rows[2] = {__shfl_sync(0xffffffffu, cur0, i), __shfl_sync(0xffffffffu, cur1, i)};
+          const int64_t rows[2] = {__shfl_sync(0xffffffffu, cur_rows[0], i), __shfl_sync(0xffffffffu, cur_rows[1], i)};
           if (lane == 0) {
             const int s = static_cast<int>(it % C::kNS);
             const uint32_t ph = static_cast<uint32_t>((it / C::kNS) & 1);
@@ -381,14 +505,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
             } else {
               uint32_t bytes = 0;
               for (int h = 0; h < 2; ++h)
-                if (rows[h] >= 0) bytes += C::kKBlocks * C::kBoxBytes;
+                if (rows[h] >= 0) bytes += C::kKBlocks * C::kBoxBytes + (C::kFp8 ? kScaleBox * 4 : 0);
+              smeta[2 * s] = static_cast<int32_t>(rows[0]);  // published to the epilogue by full[s]
+              smeta[2 * s + 1] = static_cast<int32_t>(rows[1]);
               tc::mbar_arrive_expect_tx(&full[s], bytes);
               uint8_t* st = stages + s * C::kTileBytes;
               for (int h = 0; h < 2; ++h) {
                 if (rows[h] < 0) continue;
                 for (int kb = 0; kb < C::kKBlocks; ++kb)
-                  tc::tma_load_2d(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * 64,
+                  tc::tma_load_2d(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * kBoxX,
                                   static_cast<int32_t>(rows[h]), &full[s]);
+                // the box's 64 scales, from the 16-byte aligned row at or below its first
+                if (C::kFp8)
+                  tc::tma_load_1d(sscale + (2 * s + h) * kScaleSlot, &smap, static_cast<int32_t>(rows[h] & ~int64_t(3)),
+                                  &full[s]);
               }
               ++it;
             }
@@ -397,8 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
           if (failed) break;
         }
         Wb = Wn;
-        cur0 = nxt0;
-        cur1 = nxt1;
+        cur = nxt;
       }
       // drain: the last load of every stage must land before the CTA exits
       if (lane == 0) {
@@ -471,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
           }
           uint8_t* qb = qbufs + qi * C::kQBytes;
           float* wb = wbufs + qi * (C::kWBytes / 4);
-          if (C::kFp8) stage_query_fp8<QB>(a, W.g, qb, wb, lane);
+          if (C::kFp8) stage_query_fp8<QB>(a, W.g, qb, wb, qraw, lane);
           else stage_query_bf16<QB>(a, W.g, qb, wb, lane);
           tc::fence_proxy_async_smem();
           __syncwarp();
@@ -512,22 +641,41 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
     };
     if (use_hist)
       for (int i = et; i < kTopkBins1; i += 128) shist[i] = 0;
+    // Tails first (the epilogue warps wait for their first accumulator
+    // anyway): positions past each row's group tiles are -inf, the whole row
+    // NaN for an invalid row.  No tile writes there, so the order is free.
+    for (int r = blockIdx.x; r < a.rows; r += gridDim.x) {
+      int r0 = r;
+      while (!is_leader<QB>(a, r0)) --r0;
+      const Group g = group_at<QB>(a, r0);
+      int b;
+      row_visible(a, r, &b);
+      const bool ok = b >= 0 && b < a.cache.batch;
+      if (ok && et == 0) {
+        const int L = __ldg(a.cache.seq_lens + b);
+        if (L < 0 || L > a.cache.max_len) record_error(a.status, LSA_ERR_BOUNDS, r, L);
+      } else if (!ok && et == 0) {
+        record_error(a.status, LSA_ERR_BOUNDS, r, b);
+      }
+      const float val = ok ? -INFINITY : NAN;
+      int64_t start = ok ? static_cast<int64_t>(g.tiles) * kTile : 0;
+      start = start < a.ld ? start : a.ld;
+      float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+      const int64_t mis = (reinterpret_cast<uintptr_t>(row + start) >> 2) & 3;  // floats to 16-byte alignment
+      int64_t head = start + ((4 - mis) & 3);
+      head = head < a.ld ? head : a.ld;
+      for (int64_t p = start + et; p < head; p += 128) row[p] = val;
+      const int64_t nvec = (a.ld - head) >> 2;
+      float4* v4 = reinterpret_cast<float4*>(row + head);
+      for (int64_t i = et; i < nvec; i += 128) v4[i] = make_float4(val, val, val, val);
+      for (int64_t p = head + nvec * 4 + et; p < a.ld; p += 128) row[p] = val;
+    }
     if (plan.n_items > 0) {
       Walker<QB> W;
       W.start(a, plan.r_first, plan.j_first);
       int gi = -1, qi = 0;
       int hist_row = -1;
       int64_t vis_r[QB];
-      // The block-table lookup (and FP8 scale) of a tile is loaded one tile
-      // ahead, so its latency overlaps the wait for the accumulator.
-      int64_t prow_next, p_next;
-      float ks_next;
-      auto prefetch = [&](const Walker<QB>& w) {
-        p_next = static_cast<int64_t>(w.j) * kTile + t;
-        prow_next = p_next < w.g.vis ? ad.row(w.g.b, p_next) : -1;
-        ks_next = (C::kFp8 && prow_next >= 0) ? __ldg(a.cache.idx_key_scales + prow_next) : 1.f;
-      };
-      prefetch(W);
       for (int64_t it = 0; it < plan.n_items; ++it) {
         if (it == 0 || W.j == 0) {
           ++gi;
@@ -565,9 +713,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
           break;
         }
         tc::tc_fence_after();
-        const int64_t p = p_next;
-        const int64_t prow = prow_next;
-        const float kscale = ks_next;
+        // The tile's key rows (and FP8 scales) come from the producer through
+        // the stage; the stage is released once all four warps have read them.
+        int32_t mrow = 0;  // contiguous bf16: every visible position has a key row
+        float kscale = 1.f;
+        if (stage_meta) {
+          const int stg = static_cast<int>(it % C::kNS);
+          if (!tc::mbar_wait(&full[stg], static_cast<uint32_t>((it / C::kNS) & 1), abort_flag)) {
+            if (lane == 0) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 8);
+              *abort_flag = 1;
+            }
+            hist_row = -1;
+            break;
+          }
+          const int box = 2 * stg + (t >> 6);
+          mrow = smeta[box];
+          if (C::kFp8 && mrow >= 0) kscale = sscale[box * kScaleSlot + (mrow & 3) + (t & 63)];
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&empty[stg]);
+        }
+        const int64_t p = static_cast<int64_t>(W.j) * kTile + t;
+        const int64_t prow = mrow >= 0 ? static_cast<int64_t>(mrow) + (t & 63) : -1;
         const float* wb = wbufs + qi * (C::kWBytes / 4);
         float sc[QB];
 #pragma unroll
@@ -613,34 +780,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__
           if (lane == 0) tc::mbar_arrive(&qempty[qi]);
         }
         W.next(a);
-        if (it + 1 < plan.n_items) prefetch(W);
       }
       if (use_hist && hist_row >= 0 && !flush_hist(hist_row) && lane == 0) {
         record_error(a.status, LSA_ERR_TIMEOUT, 0, 7);
         *abort_flag = 1;
       }
     }
-    // tails: positions past each row's group tiles are -inf (NaN for an invalid row)
-    for (int r = blockIdx.x; r < a.rows; r += gridDim.x) {
-      int r0 = r;
-      while (!is_leader<QB>(a, r0)) --r0;
-      const Group g = group_at<QB>(a, r0);
-      int b;
-      row_visible(a, r, &b);
-      const bool ok = b >= 0 && b < a.cache.batch;
-      if (ok && threadIdx.x == kWarpEpi * 32) {
-        const int L = __ldg(a.cache.seq_lens + b);
-        if (L < 0 || L > a.cache.max_len) record_error(a.status, LSA_ERR_BOUNDS, r, L);
-      } else if (!ok && threadIdx.x == kWarpEpi * 32) {
-        record_error(a.status, LSA_ERR_BOUNDS, r, b);
-      }
-      const float val = ok ? -INFINITY : NAN;
-      const int64_t start = ok ? static_cast<int64_t>(g.tiles) * kTile : 0;
-      float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-      for (int64_t p = start + (threadIdx.x - kWarpEpi * 32); p < a.ld; p += 128) row[p] = val;
-    }
   }
-
   __syncthreads();
   if (warp == kWarpMma) {
     tc::tc_fence_after();
@@ -681,14 +827,30 @@ cudaError_t launch_t(const ScoresArgs& a, cudaStream_t s) {
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tmap;
   const bool fp8 = KDT == LSA_FP8_E4M3;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(key_rows(a))};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDim * (fp8 ? 1 : 2))};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), static_cast<cuuint32_t>(kBoxRows)};
+  // The key rows are moved as opaque 4-byte elements (the 128-byte swizzle
+  // works on bytes, so the shared-memory image is the same for bf16 and e4m3);
+  // wider elements make fewer TMA element steps per byte.
+  const int row_bytes = kDim * (fp8 ? 1 : 2);
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes / 4), static_cast<cuuint64_t>(key_rows(a))};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBoxX), static_cast<cuuint32_t>(kBoxRows)};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(&tmap, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  CUresult r = fn(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2,
                   const_cast<void*>(a.cache.idx_keys), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  CUtensorMap smap;
+  memset(&smap, 0, sizeof(smap));
+  if (fp8) {  // FP8 key scales as a 1-D tensor over the same flat key rows
+    const cuuint64_t sdims[1] = {static_cast<cuuint64_t>(key_rows(a))};
+    const cuuint64_t sstrides[1] = {4};  // unused for rank 1
+    const cuuint32_t sbox[1] = {static_cast<cuuint32_t>(kScaleBox)};
+    const cuuint32_t sestr[1] = {1};
+    r = fn(&smap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<float*>(a.cache.idx_key_scales), sdims, sstrides,
+           sbox, sestr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
   auto kern = k_scan_tc<KDT, QB>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -696,7 +858,7 @@ cudaError_t launch_t(const ScoresArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<num_sms(), kThreads, C::kSmemBytes, s>>>(tmap, a);
+  kern<<<num_sms(), kThreads, C::kSmemBytes, s>>>(tmap, smap, a);
   return cudaGetLastError();
 }
 
@@ -713,10 +875,10 @@ int scores_tc_launches(bool) { return 1; }
 
 bool scores_tc_supported(const ScoresArgs& a) {
   if (!scores_tc_shape_ok(a.key_dtype, a.q_dtype, a.H, a.dI, a.cache.block_size)) return false;
-  if (!aligned16(a.cache.idx_keys) || !aligned16(a.q_idx)) return false;
+  if (!aligned16(a.cache.idx_keys) || !aligned16(a.q_idx) || !aligned16(a.w)) return false;
   const int64_t kr = key_rows(a);
   if (kr <= 0 || kr >= (1LL << 31)) return false;
-  if (a.key_dtype == LSA_FP8_E4M3 && !a.cache.idx_key_scales) return false;
+  if (a.key_dtype == LSA_FP8_E4M3 && (!a.cache.idx_key_scales || !aligned16(a.cache.idx_key_scales))) return false;
   return true;
 }
 
