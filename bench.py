@@ -276,14 +276,16 @@ def run_ours(args, world, rank, local):
     # also builds the top-k's first histogram); the profiled variant records
     # the phase-boundary events inside it.
     use_step_api = (not prefill) and args.op == "step"
+    step_flags = lsa.LSA_STEP_FUSED if args.fused else lsa.LSA_STEP_UNFUSED
 
     def step(ev=None):
         if use_step_api:
             if ev is None:
-                lsa.decode_step(dc.dims, dc.cache, dc.q_idx, dc.w, dc.q, out, lse, ws, idx_out=idx, stream=stream)
+                lsa.decode_step(dc.dims, dc.cache, dc.q_idx, dc.w, dc.q, out, lse, ws, idx_out=idx, flags=step_flags,
+                                stream=stream)
             else:
                 lsa.decode_step_profiled(dc.dims, dc.cache, dc.q_idx, dc.w, dc.q, out, lse, ws, ev, idx_out=idx,
-                                         stream=stream)
+                                         flags=step_flags, stream=stream)
             return
         if ev is not None:
             ev[0].record(stream)
@@ -365,7 +367,7 @@ def run_ours(args, world, rank, local):
             d_qidx.copy_(h_qidx, non_blocking=True)
             d_w.copy_(h_w, non_blocking=True)
             d_q.copy_(h_q, non_blocking=True)
-            lsa.decode_step(dc.dims, dc.cache, d_qidx, d_w, d_q, out, lse, ws, stream=stream)
+            lsa.decode_step(dc.dims, dc.cache, d_qidx, d_w, d_q, out, lse, ws, flags=step_flags, stream=stream)
             h_out.copy_(out, non_blocking=True)
             h_lse.copy_(lse, non_blocking=True)
 
@@ -391,6 +393,10 @@ def run_ours(args, world, rank, local):
     ms_per_step = timed_ms / args.steps
     value = world * args.steps / (timed_ms / 1e3)
     scan_avg = statistics.mean(scan_ms)
+    # with the fused flag the step is one launch (when it applies): the first
+    # phase-event window then holds the whole step
+    fused = use_step_api and args.fused and \
+        lsa.launch_count(dc.dims, R, dc.max_len, lsa.LSA_OP_DECODE_STEP_FUSED) == 1
     if prefill:
         fl = synth.flops_prefill_scan(case)
         achieved = fl / (scan_avg / 1e3) / 1e12
@@ -400,6 +406,14 @@ def run_ours(args, world, rank, local):
                 "peak_source": f"{peak_src} bf16_tflops (burst)"}
         unit = "chunk rows/s"
         value = world * args.steps * R / (timed_ms / 1e3)
+    elif fused:
+        # the one launch is the whole step: its algorithmic bytes are the step's
+        achieved = nb["total"] / (scan_avg / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None, "kernel": "fused decode step (scan + top-k + sparse attn, one launch)",
+                "algorithmic_bytes_per_launch": nb["total"], "peak_source": f"{peak_src} hbm_gbs"}
+        unit = "steps/s"
     else:
         scan_bytes = nb["keys"] + nb["scales"] + nb["block_table"] + nb["q_idx_w"] + nb["scores_fp32"]
         achieved = scan_bytes / (scan_avg / 1e3) / 1e9
@@ -411,7 +425,8 @@ def run_ours(args, world, rank, local):
     step_gbs = nb["total"] / (ms_per_step / 1e3) / 1e9
     # launches of our kernels per step, as the library plans them for these sizes
     if use_step_api:
-        per_step = lsa.launch_count(dc.dims, R, dc.max_len, lsa.LSA_OP_DECODE_STEP)
+        per_step = lsa.launch_count(dc.dims, R, dc.max_len,
+                                    lsa.LSA_OP_DECODE_STEP_FUSED if args.fused else lsa.LSA_OP_DECODE_STEP)
     else:
         per_step = sum(lsa.launch_count(dc.dims, R, dc.max_len, op, causal=prefill)
                        for op in (lsa.LSA_OP_SCORES, lsa.LSA_OP_TOPK, lsa.LSA_OP_ATTN)
@@ -437,11 +452,14 @@ def run_ours(args, world, rank, local):
             "value": value, "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": s.act_dtype if s.idx_key_dtype != "fp8" else "bf16+fp8",
-            "data": "synthetic (seeded, generated on host)", "config": workload_config(cfg, case),
+            "data": "synthetic (seeded, generated on host)",
+            "config": dict(workload_config(cfg, case),
+                           step="one cooperative launch (LSA_STEP_FUSED)" if fused else "separate launches"),
             "tokens_per_s": value * R if not prefill else None,
             "step_hbm_gbs": step_gbs, "step_hbm_frac": step_gbs / peaks["hbm_gbs"],
             "step_algorithmic_bytes": nb["total"],
-            "kernel_ms": {"scan": scan_avg, "topk": statistics.mean(topk_ms), "attn": statistics.mean(attn_ms)},
+            "kernel_ms": ({"fused_step": scan_avg} if fused else
+                          {"scan": scan_avg, "topk": statistics.mean(topk_ms), "attn": statistics.mean(attn_ms)}),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -460,6 +478,8 @@ def main(argv=None):
     ap.add_argument("--op", default="step", choices=["step", "scan", "topk", "attn"],
                     help="time one stage only (profiling); the bench line is for 'step'")
     ap.add_argument("--no-soak", action="store_true", help="skip the 1 s clock-sampling soak (profiling)")
+    ap.add_argument("--fused", action="store_true",
+                    help="decode step as one cooperative launch (LSA_STEP_FUSED) instead of separate launches")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

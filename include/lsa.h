@@ -108,12 +108,13 @@ typedef enum {
   LSA_OP_SCORES = 0,
   LSA_OP_TOPK = 1,
   LSA_OP_ATTN = 2,
-  LSA_OP_DECODE_STEP = 3
+  LSA_OP_DECODE_STEP = 3,
+  LSA_OP_DECODE_STEP_FUSED = 4 /* lsa_launch_count only: lsa_decode_step with LSA_STEP_FUSED */
 } lsa_op;
 
 /* Flags of lsa_decode_step. */
 #define LSA_STEP_UNFUSED 0 /* scan, top-k, attention as separate launches     */
-#define LSA_STEP_FUSED 1   /* reserved for the single-launch step; see below  */
+#define LSA_STEP_FUSED 1   /* the whole step in one cooperative launch        */
 
 /*
  * Bytes of workspace `op` needs for `rows` query rows whose score rows hold
@@ -173,8 +174,19 @@ lsa_status lsa_sparse_attn_decode(const lsa_dims* d, const lsa_cache* c, int32_t
  *   q_idx [B, H_I, d_I], w [B, H_I] fp32, q [B, H, D]: device inputs.
  *   out [B, H, D_v], lse [B, H] (or NULL): device outputs.
  *   idx_out [B, k] device int32 or NULL: the selection, if wanted.
- *   flags: LSA_STEP_UNFUSED (LSA_STEP_FUSED currently runs the same launches).
- * Workspace: lsa_workspace_size(d, B, c->max_len, LSA_OP_DECODE_STEP).
+ *   flags: LSA_STEP_UNFUSED: the scan, the top-k and the attention are
+ *            separate launches (3-5 kernels, see lsa_launch_count).
+ *          LSA_STEP_FUSED: the same three stages in ONE cooperative launch of
+ *            one CTA per SM, with grid-wide barriers (bounded waits) between
+ *            them (the optional fused decode kernel of the MLI page, a
+ *            single persistent launch here).  It runs the same CTA code as the
+ *            separate launches, so its results are bitwise those of
+ *            LSA_STEP_UNFUSED.  It applies when the tensor-core scan, the
+ *            three-pass top-k (c->max_len <= 2^19) and the tensor-core
+ *            attention all apply and every CTA of the grid fits on the device
+ *            at once; otherwise the step silently takes the separate launches.
+ *            A barrier that times out records LSA_ERR_TIMEOUT in the status word.
+ * Workspace: lsa_workspace_size(d, B, c->max_len, LSA_OP_DECODE_STEP) (either flag).
  */
 lsa_status lsa_decode_step(const lsa_dims* d, const lsa_cache* c, const void* q_idx,
                            const float* w, const void* q, void* out, float* lse,
@@ -229,7 +241,10 @@ lsa_status lsa_topk_noalloc(const float* scores, int64_t ld, int32_t rows, const
  * Number of kernel launches `op` enqueues for `rows` query rows with score rows
  * of `max_len` entries (`causal` != 0: prefill rows with positions), assuming
  * 16-byte aligned buffers.  A planning aid for launch accounting and graph
- * capture; runtime memsets are not counted.  -1 on invalid arguments.
+ * capture; runtime memsets are not counted.  LSA_OP_DECODE_STEP_FUSED gives
+ * 1 when the fused step applies to these shapes, else the separate launches'
+ * count (the device can still refuse the cooperative launch at run time, in
+ * which case the step falls back to them).  -1 on invalid arguments.
  */
 int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t op, int32_t causal);
 

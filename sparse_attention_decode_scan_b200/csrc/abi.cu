@@ -92,6 +92,10 @@ StepLayout step_layout(const lsa_dims* d, int32_t rows, int64_t max_len) {
   L.idx_off = L.scores_off + align_up(static_cast<size_t>(rows) * score_ld(max_len) * 4);
   L.inner_off = L.idx_off + align_up(static_cast<size_t>(rows) * d->top_k * 4);
   size_t inner = topk_ws_bytes(rows, max_len, d->top_k);
+  if (topk_v2_ok(max_len)) {  // the fused step keeps the top-k head and the attention partials together
+    const size_t f = step_fused_ws_bytes(rows, max_len, d->top_k);
+    if (f > inner) inner = f;
+  }
   size_t a = attn_ws(d, rows);
   size_t s = scores_ws(rows, false);
   if (a > inner) inner = a;
@@ -110,10 +114,9 @@ inline lsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LSA_OK 
 
 inline DevStatus* status_of(void* ws) { return reinterpret_cast<DevStatus*>(ws); }
 
-lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
-                     const int32_t* row_pos, const void* q_idx, const float* w, float* scores,
-                     int64_t ld, void* ws, void* inner_ws, size_t inner_bytes, cudaStream_t s,
-                     uint32_t* hist12 = nullptr, bool* hist_done = nullptr) {
+ScoresArgs scores_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
+                       const int32_t* row_pos, const void* q_idx, const float* w, float* scores, int64_t ld,
+                       void* ws, void* inner_ws, size_t inner_bytes) {
   ScoresArgs a;
   a.cache = view(d, c);
   a.key_dtype = d->idx_key_dtype;
@@ -131,6 +134,14 @@ lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const 
   a.plan_ws = inner_ws;
   a.plan_bytes = inner_bytes;
   a.hist12 = nullptr;
+  return a;
+}
+
+lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
+                     const int32_t* row_pos, const void* q_idx, const float* w, float* scores,
+                     int64_t ld, void* ws, void* inner_ws, size_t inner_bytes, cudaStream_t s,
+                     uint32_t* hist12 = nullptr, bool* hist_done = nullptr) {
+  ScoresArgs a = scores_args(d, c, rows, row_seq, row_pos, q_idx, w, scores, ld, ws, inner_ws, inner_bytes);
   if (hist_done) *hist_done = false;
   if (rows == 0 || ld == 0) return LSA_OK;
   if (!force_simt() && scores_tc_supported(a)) {
@@ -146,8 +157,8 @@ lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const 
   return cuda_status(launch_scores_simt(a, s));
 }
 
-lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
-                   int32_t k, int32_t* idx, void* ws, void* inner_ws, cudaStream_t s, bool hist_ready = false) {
+TopkArgs topk_args(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
+                   int32_t k, int32_t* idx, void* ws, void* inner_ws, bool hist_ready) {
   TopkArgs a;
   a.scores = scores;
   a.ld = ld;
@@ -159,12 +170,17 @@ lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t*
   a.ws = inner_ws;
   a.status = status_of(ws);
   a.hist_ready = hist_ready;
+  return a;
+}
+
+lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
+                   int32_t k, int32_t* idx, void* ws, void* inner_ws, cudaStream_t s, bool hist_ready = false) {
+  const TopkArgs a = topk_args(scores, ld, rows, valid_len, n_cols, k, idx, ws, inner_ws, hist_ready);
   return cuda_status(launch_topk(a, s));
 }
 
-lsa_status do_attn(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq, const void* q,
-                   const int32_t* idx, void* out, float* lse, void* ws, void* inner_ws, size_t inner_bytes,
-                   cudaStream_t s) {
+AttnArgs attn_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq, const void* q,
+                   const int32_t* idx, void* out, float* lse, void* ws, void* inner_ws, size_t inner_bytes) {
   AttnArgs a;
   a.cache = view(d, c);
   a.dtype = d->act_dtype;
@@ -182,6 +198,13 @@ lsa_status do_attn(const lsa_dims* d, const lsa_cache* c, int32_t rows, const in
   a.ws = inner_ws;
   a.ws_bytes = inner_bytes;
   a.status = status_of(ws);
+  return a;
+}
+
+lsa_status do_attn(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq, const void* q,
+                   const int32_t* idx, void* out, float* lse, void* ws, void* inner_ws, size_t inner_bytes,
+                   cudaStream_t s) {
+  const AttnArgs a = attn_args(d, c, rows, row_seq, q, idx, out, lse, ws, inner_ws, inner_bytes);
   if (rows == 0) return LSA_OK;
   if (!force_simt() && attn_tc_supported(a)) return cuda_status(launch_attn_tc(a, s));
   return cuda_status(launch_attn_simt(a, s));
@@ -285,9 +308,26 @@ static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const 
   const int64_t ld = score_ld(c->max_len);
   // With the tensor-core scan and the three-launch top-k, the scan writes the
   // top-k's first histogram into the top-k workspace (which starts with it).
+  if (!mark(0)) return LSA_ERR_CUDA;
+  if (flags == LSA_STEP_FUSED && !force_simt()) {
+    // one cooperative launch when every stage has its tensor-core / three-pass
+    // form and all CTAs fit at once; otherwise the separate launches below
+    const ScoresArgs sa = scores_args(d, c, B, nullptr, nullptr, q_idx, w, scores, ld, ws, inner, inner_bytes);
+    const TopkArgs ta = topk_args(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, true);
+    const AttnArgs aa = attn_args(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes);
+    if (step_fused_supported(sa, aa, c->max_len)) {
+      const cudaError_t e = launch_step_fused(sa, ta, aa, s);
+      if (e == cudaSuccess) {
+        for (int i = 1; i < 4; ++i)
+          if (!mark(i)) return LSA_ERR_CUDA;
+        return LSA_OK;
+      }
+      if (e != cudaErrorCooperativeLaunchTooLarge) return LSA_ERR_CUDA;
+      (void)cudaGetLastError();  // not co-resident on this device: fall back
+    }
+  }
   uint32_t* hist12 = (!force_simt() && topk_v2_ok(c->max_len)) ? static_cast<uint32_t*>(inner) : nullptr;
   bool hist_done = false;
-  if (!mark(0)) return LSA_ERR_CUDA;
   st = do_scores(d, c, B, nullptr, nullptr, q_idx, w, scores, ld, ws, inner, inner_bytes, s, hist12, &hist_done);
   if (st != LSA_OK) return st;
   if (!mark(1)) return LSA_ERR_CUDA;
@@ -343,6 +383,13 @@ int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32
     case LSA_OP_TOPK: return topk_launches(max_len);
     case LSA_OP_ATTN: return attn;
     case LSA_OP_DECODE_STEP: return scan + topk_launches(max_len) + attn;
+    case LSA_OP_DECODE_STEP_FUSED: {
+      const bool fused = !simt && causal == 0 && topk_v2_ok(max_len) &&
+                         scores_tc_shape_ok(d->idx_key_dtype, d->act_dtype, d->n_idx_heads, d->idx_dim,
+                                            d->block_size) &&
+                         attn_tc_shape_ok(d->act_dtype, d->n_heads, d->qk_dim, d->v_dim, d->block_size);
+      return fused ? 1 : scan + topk_launches(max_len) + attn;
+    }
     default: return -1;
   }
 }

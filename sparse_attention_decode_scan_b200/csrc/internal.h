@@ -1,6 +1,7 @@
 // Internal launch interface between the C-ABI layer (abi.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -83,6 +84,10 @@ bool topk_v2_ok(int64_t n_cols);
 size_t topk_hist_zero_bytes(int32_t rows);
 // true if the scan can accumulate the top-k histogram itself
 bool scores_tc_fused_hist_ok(const ScoresArgs& a);
+// segments of the top-k collect pass
+TopkPlan topk_collect_plan(int32_t rows, int64_t n_cols);
+// tensor maps of the tensor-core scan (keys; FP8 scales)
+cudaError_t scan_tc_maps(const ScoresArgs& a, CUtensorMap* tmap, CUtensorMap* smap);
 
 // ---- sparse attention
 struct AttnArgs {
@@ -112,5 +117,14 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);
 // exact merge of per-split softmax partials (shared by both attention paths)
 cudaError_t launch_lse_merge(const AttnArgs& a, int nsplit, const float* part_o, const float* part_lse,
                              cudaStream_t s);
+
+// ---- fused decode step: scan -> top-k -> attention in one cooperative launch
+// (one CTA per SM, grid-wide barriers between the phases).  Applies when the
+// tensor-core scan with its histogram, the three-launch top-k and the
+// tensor-core attention all apply.  Workspace: the top-k workspace `topk.ws`,
+// of step_fused_ws_bytes bytes.
+bool step_fused_supported(const ScoresArgs& sa, const AttnArgs& aa, int64_t n_cols);
+size_t step_fused_ws_bytes(int32_t rows, int64_t n_cols, int32_t k);
+cudaError_t launch_step_fused(const ScoresArgs& sa, const TopkArgs& ta, const AttnArgs& aa, cudaStream_t s);
 
 }  // namespace lsa

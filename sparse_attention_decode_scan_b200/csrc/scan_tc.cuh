@@ -1,0 +1,814 @@
+#pragma once
+// Lightning-indexer scan on the sm_100a tensor cores: the device code of one
+// CTA, shared by the standalone scan kernel and the fused decode step.
+//
+// Before each DSA layer the lightning indexer scores every cached token of the
+// sequence, and at long context this scan is where decode time goes (MLI
+// "Multi-layer Indexer" abstract, sentences 2-3).  Score of token s for a query
+// row: I(s) = sum_h w[h] * ReLU(q[h] . K[s]) over 64 indexer heads of dim 128
+// (DSA lightning indexer, DeepSeek-V3.2-Exp report); FP8 keys carry a per-token
+// scale (the compact indexer keys of the LeanSparse episode page).
+//
+// Mapping: keys are the MMA's M side (128 tokens per tile, one TMEM lane per
+// token) and the query heads its N side, so after the MMA every epilogue thread
+// owns one token with all of its head dot products in TMEM; the ReLU-weighted
+// head reduction then runs in registers.  Decode groups one query row per tile
+// (N = 64); the causal prefill groups 4 rows of one sequence (N = 256), reusing
+// each key tile 4 times.  FP8 keys go straight to kind::f8f6f4 MMAs: the bf16
+// query is split exactly into two e4m3 terms (hi + lo, per-head power-of-two
+// scale folded into w), so N doubles and no key conversion is needed.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0  TMA producer: 64-row boxes of the key cache (block-table gather)
+//   warp 1  MMA issuer (one thread) + TMEM owner
+//   warp 2  query staging: query rows -> swizzled smem operand, weights
+//   warps 3-6 epilogue: TMEM -> registers, ReLU-weighted sum, score stores
+// Every wait is bounded; a timeout records LSA_ERR_TIMEOUT and unwinds.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace lsa {
+namespace scan {
+
+constexpr int kHeads = 64;       // indexer heads
+constexpr int kDim = 128;        // indexer head dim
+constexpr int kTile = 128;       // tokens per tile (MMA M, TMEM lanes)
+constexpr int kBoxRows = 64;     // rows per TMA box (one 64-token page or half tile)
+constexpr int kBoxX = 32;        // 4-byte TMA elements per 128-byte K block
+constexpr int kScaleBox = 68;    // FP8 scales per box load: 64 + up to 3 for the 16-byte aligned start
+constexpr int kScaleSlot = 96;   // floats per scale slot: a TMA destination starts on a 128-byte boundary
+constexpr int kThreads = 224;    // 7 warps
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpQ = 2, kWarpEpi = 3;
+constexpr int kSmemLimit = 232448;
+constexpr int kBarrierId = 1;    // named barrier of the scan's threads (a fused block holds more threads)
+
+__device__ __forceinline__ void scan_sync() {
+  asm volatile("bar.sync %0, %1;" ::"n"(kBarrierId), "n"(kThreads) : "memory");
+}
+
+template <int KDT, int QB>
+struct Cfg {
+  static constexpr bool kFp8 = KDT == LSA_FP8_E4M3;
+  static constexpr int kN = (kFp8 ? 2 * kHeads : kHeads) * QB;    // MMA N (columns per accumulator)
+  static constexpr int kKBlocks = kFp8 ? 1 : 2;                    // 128-byte K blocks per row
+  static constexpr int kKBlockBytes = kTile * 128;                 // A: 128 rows x 128 B
+  static constexpr int kTileBytes = kKBlocks * kKBlockBytes;
+  static constexpr int kBoxBytes = kBoxRows * 128;
+  static constexpr int kQKBlockBytes = kN * 128;                   // B: N rows x 128 B per K block
+  static constexpr int kQBytes = kKBlocks * kQKBlockBytes;
+  static constexpr int kNQ = (QB == 1 && kFp8) ? 2 : 1;            // query operand buffers
+  static constexpr int kWBytes = QB * kHeads * 4;
+  static constexpr int kHistBytes = QB == 1 ? kTopkBins1 * 4 : 0;  // fused first top-k histogram (decode)
+  // Per stage besides the keys: the key rows of its two boxes (written by the
+  // producer for the epilogue) and, for FP8, the two boxes' scales (TMA).
+  static constexpr int kMetaBytes = 2 * 4 + (kFp8 ? 2 * kScaleSlot * 4 : 0);
+  static constexpr int kRawBytes = kFp8 ? QB * kHeads * kDim * 2 : 0;  // FP8: bf16 query rows before the split
+  static constexpr int kFixed = kNQ * kQBytes + kNQ * kWBytes + kRawBytes + kHistBytes + 512 /*barriers, scratch*/ +
+                                1024 /*align*/;
+  static constexpr int kNSmax = (kSmemLimit - kFixed) / (kTileBytes + kMetaBytes);
+  static constexpr int kNS = kNSmax > 12 ? 12 : kNSmax;            // key stages
+  static constexpr int kAccCols = kN;
+  static constexpr int kTmemCols = 2 * kN <= 32 ? 32 : 2 * kN <= 64 ? 64 : 2 * kN <= 128 ? 128
+                                   : 2 * kN <= 256 ? 256 : 512;
+  static constexpr int kSmemBytes = kNS * (kTileBytes + kMetaBytes) + kFixed;
+  static constexpr uint32_t kIdesc = tc::idesc(kFp8 ? tc::kFmtE4M3 : tc::kFmtBF16,
+                                               kFp8 ? tc::kFmtE4M3 : tc::kFmtBF16, kTile, kN);
+  static_assert(kNS >= 3, "too few key stages");
+  static_assert(2 * kN <= 512, "accumulators exceed TMEM");
+  static_assert(kSmemBytes <= kSmemLimit, "shared memory");
+};
+
+// Stages of the configurations that run: decode 6 (bf16) and 9 (FP8) tiles in
+// flight, the causal prefill 5 (bf16, 4 rows per tile) and 9 (FP8, 2 rows).
+static_assert(Cfg<LSA_BF16, 1>::kNS == 6 && Cfg<LSA_FP8_E4M3, 1>::kNS == 9, "decode stages");
+static_assert(Cfg<LSA_BF16, 4>::kNS == 5 && Cfg<LSA_FP8_E4M3, 2>::kNS == 9, "prefill stages");
+
+// ---------------------------------------------------------------- work items
+
+__device__ __forceinline__ int seq_of(const ScoresArgs& a, int r) { return a.row_seq ? __ldg(a.row_seq + r) : r; }
+
+// Visible positions of query row r (0 for an invalid row).
+__device__ __forceinline__ int64_t row_visible(const ScoresArgs& a, int r, int* b_out) {
+  const int b = seq_of(a, r);
+  *b_out = b;
+  if (b < 0 || b >= a.cache.batch) return 0;
+  int64_t L = __ldg(a.cache.seq_lens + b);
+  L = L < 0 ? 0 : (L > a.cache.max_len ? a.cache.max_len : L);
+  if (a.row_pos) {
+    int64_t p = static_cast<int64_t>(__ldg(a.row_pos + r)) + 1;
+    p = p < 0 ? 0 : p;
+    L = p < L ? p : L;
+  }
+  return L;
+}
+
+// A group is a run of up to QB consecutive query rows of one sequence that
+// does not cross a multiple of QB; its rows share every key tile.
+template <int QB>
+__device__ __forceinline__ bool is_leader(const ScoresArgs& a, int r) {
+  if (QB == 1 || r % QB == 0) return true;
+  return seq_of(a, r) != seq_of(a, r - 1);
+}
+
+struct Group {
+  int r0, nrows, b, tiles;
+  int64_t vis;  // max visible positions over the group's rows
+};
+
+template <int QB>
+__device__ Group group_at(const ScoresArgs& a, int r0) {
+  Group g;
+  g.r0 = r0;
+  int b;
+  int64_t vis = row_visible(a, r0, &b);
+  g.b = b;
+  int n = 1;
+  if (QB > 1) {
+    while (n < QB && r0 + n < a.rows && ((r0 + n) % QB) != 0 && seq_of(a, r0 + n) == b) {
+      int bb;
+      int64_t v = row_visible(a, r0 + n, &bb);
+      vis = v > vis ? v : vis;
+      ++n;
+    }
+  }
+  g.nrows = n;
+  g.vis = vis;
+  g.tiles = static_cast<int>((vis + kTile - 1) / kTile);
+  return g;
+}
+
+// Walks the CTA's items (group, tile) in global order, skipping empty groups.
+template <int QB>
+struct Walker {
+  Group g;
+  int j;
+  __device__ void start(const ScoresArgs& a, int r0, int j0) {
+    g = group_at<QB>(a, r0);
+    j = j0;
+  }
+  __device__ void next(const ScoresArgs& a) {
+    if (++j < g.tiles) return;
+    j = 0;
+    int r = g.r0 + g.nrows;
+    while (r < a.rows) {
+      g = group_at<QB>(a, r);
+      if (g.tiles > 0) return;
+      r += g.nrows;
+    }
+    g.tiles = 0;  // past the end
+  }
+};
+
+__device__ __forceinline__ int block_sum_i64_scan(int64_t v, int64_t* warp_buf, int64_t* incl, int64_t* total) {
+  // inclusive scan over the block (kThreads threads), returns nothing; used by the planner
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_buf[warp] = x;
+  scan_sync();
+  int64_t before = 0, tot = 0;
+  for (int w = 0; w < kThreads / 32; ++w) {
+    if (w < warp) before += warp_buf[w];
+    tot += warp_buf[w];
+  }
+  *incl = before + x;
+  *total = tot;
+  scan_sync();
+  return 0;
+}
+
+struct Plan {
+  int r_first;  // leader row of the CTA's first item
+  int j_first;
+  int64_t n_items;
+};
+
+// Every thread of the CTA takes part: total tiles, this CTA's share, and the
+// group holding its first tile.
+template <int QB>
+__device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
+  Plan p;
+  p.r_first = 0;
+  p.j_first = 0;
+  if (a.rows <= kThreads) {  // one row per thread: a single block scan
+    const int r = threadIdx.x;
+    int64_t t = 0;
+    if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
+    int64_t incl, tot;
+    block_sum_i64_scan(t, sbuf, &incl, &tot);
+    const int64_t t0 = tot * blockIdx.x / gridDim.x;
+    p.n_items = tot * (blockIdx.x + 1) / gridDim.x - t0;
+    if (p.n_items <= 0) return p;
+    const int64_t start = incl - t;
+    if (t > 0 && start <= t0 && t0 < start + t) {  // exactly one thread holds tile t0
+      sfound[0] = r;
+      sfound[1] = static_cast<int>(t0 - start);
+    }
+    scan_sync();
+    p.r_first = sfound[0];
+    p.j_first = sfound[1];
+    return p;
+  }
+  int64_t total = 0;
+  for (int base = 0; base < a.rows; base += kThreads) {
+    const int r = base + threadIdx.x;
+    int64_t t = 0;
+    if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
+    int64_t incl, tot;
+    block_sum_i64_scan(t, sbuf, &incl, &tot);
+    total += tot;
+  }
+  const int64_t t0 = total * blockIdx.x / gridDim.x;
+  const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
+  p.n_items = t1 - t0;
+  if (p.n_items <= 0) return p;
+  if (threadIdx.x == 0) sfound[0] = -1;
+  scan_sync();
+  int64_t acc = 0;
+  for (int base = 0; base < a.rows; base += kThreads) {
+    const int r = base + threadIdx.x;
+    int64_t t = 0;
+    if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
+    int64_t incl, tot;
+    block_sum_i64_scan(t, sbuf, &incl, &tot);
+    const int64_t start = acc + incl - t;
+    if (t > 0 && start <= t0 && t0 < start + t) {
+      sfound[0] = r;
+      sfound[1] = static_cast<int>(t0 - start);
+    }
+    acc += tot;
+    scan_sync();
+    if (sfound[0] >= 0) break;
+  }
+  p.r_first = sfound[0];
+  p.j_first = sfound[1];
+  return p;
+}
+
+// ---------------------------------------------------------------- query staging
+
+// bf16: B row n = qq * 64 + h holds q[row r0+qq][h][:] in two 128-byte K blocks.
+// Every 16-byte piece (and the weights) is a cp.async issued at once, so the
+// staging costs one memory round trip even while the key loads crowd the
+// memory system; rows of absent queries are zero-filled.
+template <int QB>
+__device__ void stage_query_bf16(const ScoresArgs& a, const Group& g, uint8_t* qbuf, float* wbuf, int lane) {
+  constexpr int N = kHeads * QB;
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q_idx);
+  for (int idx = lane; idx < N * (kDim / 8); idx += 32) {
+    const int n = idx >> 4, c = idx & 15;
+    const int qq = n / kHeads, h = n % kHeads;
+    const bool live = qq < g.nrows;
+    const uint8_t* p = src + ((static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + h) * kDim) * 2 + c * 16;
+    tc::cp_async16_zfill(qbuf + (c >> 3) * (N * 128) + tc::sw128_offset(n, c & 7), p, live ? 16u : 0u);
+  }
+  for (int i = lane; i < QB * (kHeads / 4); i += 32) {
+    const int qq = i / (kHeads / 4), c = i % (kHeads / 4);
+    const bool live = qq < g.nrows;
+    tc::cp_async16_zfill(wbuf + qq * kHeads + c * 4, a.w + static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + c * 4,
+                         live ? 16u : 0u);
+  }
+  tc::cp_async_wait_all();
+}
+
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// fp8: per (query, head) a power-of-two scale s puts max|q| into [224, 448];
+// q*s = hi + lo with hi = e4m3(q*s), lo = e4m3(q*s - hi), exact for bf16 q
+// (4 + 4 significant bits) outside the e4m3 subnormal range.  B row
+// qq*128 + h holds hi, qq*128 + 64 + h holds lo; w' = w / s.
+// The raw rows and the weights arrive by cp.async in one round trip; half a
+// warp then converts one head (8 dims per lane) from shared memory.
+template <int QB>
+__device__ void stage_query_fp8(const ScoresArgs& a, const Group& g, uint8_t* qbuf, float* wbuf, uint8_t* raw,
+                                int lane) {
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q_idx);
+  for (int idx = lane; idx < QB * kHeads * (kDim / 8); idx += 32) {
+    const int n = idx >> 4, c = idx & 15;
+    const int qq = n / kHeads, h = n % kHeads;
+    const bool live = qq < g.nrows;
+    const uint8_t* p = src + ((static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + h) * kDim) * 2 + c * 16;
+    tc::cp_async16_zfill(raw + n * (kDim * 2) + c * 16, p, live ? 16u : 0u);
+  }
+  for (int i = lane; i < QB * (kHeads / 4); i += 32) {
+    const int qq = i / (kHeads / 4), c = i % (kHeads / 4);
+    const bool live = qq < g.nrows;
+    tc::cp_async16_zfill(wbuf + qq * kHeads + c * 4, a.w + static_cast<int64_t>(live ? g.r0 + qq : g.r0) * kHeads + c * 4,
+                         live ? 16u : 0u);
+  }
+  tc::cp_async_wait_all();
+  __syncwarp();
+  const int half = lane >> 4, seg = lane & 15;  // seg: dims [8 seg, 8 seg + 8)
+#pragma unroll 2
+  for (int n0 = 0; n0 < QB * kHeads; n0 += 2) {
+    const int n = n0 + half;
+    const int qq = n / kHeads, h = n % kHeads;
+    const uint4 v = *reinterpret_cast<const uint4*>(raw + n * (kDim * 2) + seg * 16);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    float x[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      x[2 * j] = __uint_as_float(wv[j] << 16);
+      x[2 * j + 1] = __uint_as_float(wv[j] & 0xffff0000u);
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(x[j]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    // Largest power of two s = 2^k with mx * s <= 448 = 1.75 * 2^8: for
+    // mx = m * 2^E (1 <= m < 2), k = 8 - E if m <= 1.75, else 7 - E.
+    int k = 0;
+    if (mx > 0.f) {
+      const uint32_t mb = __float_as_uint(mx);
+      const int E = static_cast<int>(mb >> 23) - 127;
+      k = (mb & 0x7fffffu) <= 0x600000u ? 8 - E : 7 - E;
+      k = k < -126 ? -126 : (k > 126 ? 126 : k);
+    }
+    const float sc = __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+    const float inv = __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
+    uint32_t hw[2], lw[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float xs[4], lv[4];
+#pragma unroll
+      for (int e4 = 0; e4 < 4; ++e4) xs[e4] = x[4 * u + e4] * sc;
+      hw[u] = pack_e4m3x4(xs[0], xs[1], xs[2], xs[3]);
+#pragma unroll
+      for (int e4 = 0; e4 < 4; ++e4) lv[e4] = xs[e4] - e4m3_to_float(static_cast<uint8_t>(hw[u] >> (8 * e4)));
+      lw[u] = pack_e4m3x4(lv[0], lv[1], lv[2], lv[3]);
+    }
+    const int row_hi = qq * 2 * kHeads + h, row_lo = row_hi + kHeads;
+    const uint32_t off = (seg & 1) * 8;
+    *reinterpret_cast<uint2*>(qbuf + tc::sw128_offset(row_hi, seg >> 1) + off) = make_uint2(hw[0], hw[1]);
+    *reinterpret_cast<uint2*>(qbuf + tc::sw128_offset(row_lo, seg >> 1) + off) = make_uint2(lw[0], lw[1]);
+    if (seg == 0) wbuf[n] *= inv;  // w / s, exact for a power of two
+  }
+}
+
+// ---------------------------------------------------------------- the kernel
+
+// One CTA's share of the scan, run by threads [0, kThreads) of the block
+// (the only threads that take part in its barriers).  `tmem_slot` holds (or,
+// once the first barrier of the plan has passed, will hold) the base of at
+// least Cfg::kTmemCols allocated TMEM columns.  Every mbarrier it used is
+// invalidated before it returns, so the caller may reuse the shared memory.
+template <int KDT, int QB>
+__device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtensorMap* smap_p, const ScoresArgs& a,
+                                         uint8_t* smem_raw, const volatile uint32_t* tmem_slot) {
+  using C = Cfg<KDT, QB>;
+  const CUtensorMap& tmap = *tmap_p;
+  const CUtensorMap& smap = *smap_p;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  // Offsets keep every TMA destination 128-byte and every cp.async one 16-byte aligned.
+  uint8_t* qbufs = stages + C::kNS * C::kTileBytes;                                  // 1024-aligned operands
+  float* wbufs = reinterpret_cast<float*>(qbufs + C::kNQ * C::kQBytes);
+  uint8_t* qraw = reinterpret_cast<uint8_t*>(wbufs) + C::kNQ * C::kWBytes;          // FP8: raw query rows
+  float* sscale = reinterpret_cast<float*>(qraw + C::kRawBytes);                     // FP8: [kNS][2][kScaleSlot]
+  int32_t* smeta = reinterpret_cast<int32_t*>(sscale + (C::kFp8 ? C::kNS * 2 * kScaleSlot : 0));  // [kNS][2]
+  uint32_t* shist = reinterpret_cast<uint32_t*>(smeta + 2 * C::kNS);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(shist) + C::kHistBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = full + C::kNS;
+  uint64_t* qfull = empty + C::kNS;
+  uint64_t* qempty = qfull + C::kNQ;
+  uint64_t* tfull = qempty + C::kNQ;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint64_t* ebar = done + 1;  // epilogue warps' rendezvous around histogram flushes
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ebar + 1);
+  int* sfound = const_cast<int*>(abort_flag) + 1;                       // 2 ints
+  int64_t* sbuf = reinterpret_cast<int64_t*>(sfound + 2 + 1);           // kThreads/32 int64 (8-aligned below)
+  sbuf = reinterpret_cast<int64_t*>((reinterpret_cast<uintptr_t>(sbuf) + 7) & ~uintptr_t(7));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The epilogue reads a stage's key rows (paged cache) and scales (FP8); a
+  // contiguous bf16 cache needs neither, and its stages free at MMA completion.
+  const bool stage_meta = C::kFp8 || a.cache.block_size > 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kNS; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], stage_meta ? 1 + 4 : 1);  // MMA commit (+ 4 epilogue warps done with the stage)
+    }
+    for (int s = 0; s < C::kNQ; ++s) {
+      tc::mbar_init(&qfull[s], 1);
+      tc::mbar_init(&qempty[s], 1 + 4);  // MMA commit + 4 epilogue warps
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&tfull[s], 1);
+      tc::mbar_init(&tempty[s], 4);
+    }
+    tc::mbar_init(done, 1);
+    tc::mbar_init(ebar, 4);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == kWarpProd && lane == 0) {
+    tc::prefetch_tmap(&tmap);
+    if (C::kFp8) tc::prefetch_tmap(&smap);
+  }
+  const Plan plan = plan_work<QB>(a, sbuf, sfound);
+  scan_sync();
+  tc::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  CacheAddr ad{a.cache.block_table, a.cache.max_blocks, a.cache.block_size, a.cache.n_blocks, a.cache.max_len};
+
+  if (warp == kWarpProd) {
+    // The whole warp looks up the block-table entries of 32 tiles at a time
+    // (one tile per lane) and lane 0 issues their TMA loads.  The next batch's
+    // entries are loaded before the current batch is issued and only read
+    // after it, so their latency hides behind the 32 issues; a single thread
+    // doing the lookups serially would wait one load latency per tile.
+    if (plan.n_items > 0) {
+      struct Look {
+        int64_t p0, vis;  // first position of the tile; visible positions of its group
+        int b, r0;
+        int32_t blk[2];   // block-table entries of the tile's two boxes (paged cache)
+        bool live;
+      };
+      auto look = [&](const Walker<QB>& base, int64_t base_item) -> Look {
+        Walker<QB> w = base;
+        if (w.j + lane < w.g.tiles) w.j += lane;  // same group: no walk
+        else
+          for (int i = 0; i < lane; ++i) w.next(a);
+        Look L;
+        L.live = base_item + lane < plan.n_items;
+        L.p0 = static_cast<int64_t>(w.j) * kTile;
+        L.vis = w.g.vis;
+        L.b = w.g.b;
+        L.r0 = w.g.r0;
+        L.blk[0] = L.blk[1] = -1;
+        if (L.live && ad.block_size > 0) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int64_t p = L.p0 + h * kBoxRows;
+            const int64_t lb = p / ad.block_size;
+            if (p < L.vis && lb < ad.max_blocks)
+              L.blk[h] = __ldg(ad.block_table + static_cast<int64_t>(L.b) * ad.max_blocks + lb);
+          }
+        }
+        return L;
+      };
+      // Key rows of the two boxes: >= 0 a row, -3 past the visible range, -2 no such item.
+      auto resolve = [&](const Look& L, int64_t* rows) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t p = L.p0 + h * kBoxRows;
+          int64_t r = -2;
+          if (L.live) {
+            if (p >= L.vis) {
+              r = -3;
+            } else if (ad.block_size == 0) {
+              r = static_cast<int64_t>(L.b) * ad.max_len + p;
+            } else {
+              const int64_t lb = p / ad.block_size;
+              const int32_t blk = L.blk[h];
+              r = (lb < ad.max_blocks && blk >= 0 && blk < ad.n_blocks)
+                      ? static_cast<int64_t>(blk) * ad.block_size + (p - lb * ad.block_size)
+                      : -1;
+              if (r == -1) record_error(a.status, LSA_ERR_BOUNDS, L.r0, static_cast<int>(p));
+            }
+          }
+          rows[h] = r;
+        }
+      };
+      Walker<QB> Wb;
+      Wb.start(a, plan.r_first, plan.j_first);
+      Look cur = look(Wb, 0);
+      int64_t it = 0;
+      bool failed = false;
+      for (int64_t base_item = 0; base_item < plan.n_items && !failed; base_item += 32) {
+        int64_t cur_rows[2];
+        resolve(cur, cur_rows);
+        Walker<QB> Wn = Wb;
+        if (Wn.j + 32 < Wn.g.tiles) Wn.j += 32;
+        else
+          for (int i = 0; i < 32; ++i) Wn.next(a);
+        const Look nxt = look(Wn, base_item + 32);  // loads stay in flight during the issues below
+        const int nb = static_cast<int>(plan.n_items - base_item < 32 ? plan.n_items - base_item : 32);
+        for (int i = 0; i < nb; ++i) {
+          const int64_t rows[2] = {__shfl_sync(0xffffffffu, cur_rows[0], i), __shfl_sync(0xffffffffu, cur_rows[1], i)};
+          if (lane == 0) {
+            const int s = static_cast<int>(it % C::kNS);
+            const uint32_t ph = static_cast<uint32_t>((it / C::kNS) & 1);
+            if (!tc::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 1);
+              *abort_flag = 1;
+              failed = true;
+            } else {
+              uint32_t bytes = 0;
+              for (int h = 0; h < 2; ++h)
+                if (rows[h] >= 0) bytes += C::kKBlocks * C::kBoxBytes + (C::kFp8 ? kScaleBox * 4 : 0);
+              smeta[2 * s] = static_cast<int32_t>(rows[0]);  // published to the epilogue by full[s]
+              smeta[2 * s + 1] = static_cast<int32_t>(rows[1]);
+              tc::mbar_arrive_expect_tx(&full[s], bytes);
+              uint8_t* st = stages + s * C::kTileBytes;
+              for (int h = 0; h < 2; ++h) {
+                if (rows[h] < 0) continue;
+                for (int kb = 0; kb < C::kKBlocks; ++kb)
+                  tc::tma_load_2d(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * kBoxX,
+                                  static_cast<int32_t>(rows[h]), &full[s]);
+                // the box's 64 scales, from the 16-byte aligned row at or below its first
+                if (C::kFp8)
+                  tc::tma_load_1d(sscale + (2 * s + h) * kScaleSlot, &smap, static_cast<int32_t>(rows[h] & ~int64_t(3)),
+                                  &full[s]);
+              }
+              ++it;
+            }
+          }
+          failed = __shfl_sync(0xffffffffu, failed, 0);
+          if (failed) break;
+        }
+        Wb = Wn;
+        cur = nxt;
+      }
+      // drain: the last load of every stage must land before the CTA exits
+      if (lane == 0) {
+        const int64_t n_issued = it;
+        for (int64_t i = n_issued > C::kNS ? n_issued - C::kNS : 0; i < n_issued; ++i)
+          tc::mbar_wait(&full[i % C::kNS], static_cast<uint32_t>((i / C::kNS) & 1), nullptr);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    if (lane == 0 && plan.n_items > 0) {
+      Walker<QB> W;
+      W.start(a, plan.r_first, plan.j_first);
+      int gi = -1;
+      int qi = 0;
+      for (int64_t it = 0; it < plan.n_items; ++it) {
+        if (it == 0 || W.j == 0) {
+          ++gi;
+          qi = gi % C::kNQ;
+          if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) goto mma_fail;
+        }
+        {
+          const int s = static_cast<int>(it % C::kNS);
+          if (!tc::mbar_wait(&full[s], static_cast<uint32_t>((it / C::kNS) & 1), abort_flag)) goto mma_fail;
+          const int acc = static_cast<int>(it & 1);
+          if (!tc::mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag)) goto mma_fail;
+          tc::tc_fence_after();
+          const uint32_t d = tmem_base + acc * C::kAccCols;
+          const uint32_t a_base = tc::smem_u32(stages + s * C::kTileBytes);
+          const uint32_t b_base = tc::smem_u32(qbufs + qi * C::kQBytes);
+#pragma unroll
+          for (int kb = 0; kb < C::kKBlocks; ++kb) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad_ = tc::desc_sw128(a_base + kb * C::kKBlockBytes + k * 32);
+              const uint64_t bd_ = tc::desc_sw128(b_base + kb * C::kQKBlockBytes + k * 32);
+              if (C::kFp8) tc::mma_f8(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
+              else tc::mma_f16(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
+            }
+          }
+          tc::mma_commit(&empty[s]);
+          tc::mma_commit(&tfull[acc]);
+          const int jn = W.j + 1;
+          if (it + 1 == plan.n_items || jn >= W.g.tiles) tc::mma_commit(&qempty[qi]);
+          W.next(a);
+        }
+        continue;
+      mma_fail:
+        record_error(a.status, LSA_ERR_TIMEOUT, 0, 2);
+        *abort_flag = 1;
+        break;
+      }
+      tc::mma_commit(done);
+      tc::mbar_wait(done, 0, nullptr);
+      // The releases of the last stages and query buffer arrive asynchronously
+      // too; they must land before the barriers are invalidated.
+      if (!*abort_flag) {
+        const int64_t n = plan.n_items;
+        for (int64_t i = n > C::kNS ? n - C::kNS : 0; i < n; ++i)
+          tc::mbar_wait(&empty[i % C::kNS], static_cast<uint32_t>((i / C::kNS) & 1), abort_flag);
+        if (gi >= 0) tc::mbar_wait(&qempty[gi % C::kNQ], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag);
+      }
+    }
+  } else if (warp == kWarpQ) {
+    if (plan.n_items > 0) {
+      Walker<QB> W;
+      W.start(a, plan.r_first, plan.j_first);
+      int gi = -1;
+      for (int64_t it = 0; it < plan.n_items; ++it) {
+        if (it == 0 || W.j == 0) {
+          ++gi;
+          const int qi = gi % C::kNQ;
+          if (!tc::mbar_wait(&qempty[qi], static_cast<uint32_t>(((gi / C::kNQ) & 1) ^ 1), abort_flag)) {
+            if (lane == 0) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 3);
+              *abort_flag = 1;
+            }
+            break;
+          }
+          uint8_t* qb = qbufs + qi * C::kQBytes;
+          float* wb = wbufs + qi * (C::kWBytes / 4);
+          if (C::kFp8) stage_query_fp8<QB>(a, W.g, qb, wb, qraw, lane);
+          else stage_query_bf16<QB>(a, W.g, qb, wb, lane);
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&qfull[qi]);
+        }
+        W.next(a);
+      }
+    }
+  } else {
+    // epilogue: warp (3..6) % 4 selects the TMEM lane quarter = token rows of the tile
+    const int quarter = warp & 3;
+    const int t = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    // Decode with a histogram target: the epilogue also counts each score's
+    // top-k digit (key bits [31:20]) in shared memory and adds the counts of a
+    // row to hist12 when the CTA leaves that row, so the top-k skips one pass.
+    const bool use_hist = QB == 1 && a.hist12 != nullptr;
+    const int et = threadIdx.x - kWarpEpi * 32;  // 0..127
+    int ephase = 0;
+    auto epi_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(ebar);
+      const bool ok = tc::mbar_wait(ebar, static_cast<uint32_t>(ephase & 1), abort_flag);
+      ++ephase;
+      return ok;
+    };
+    auto flush_hist = [&](int row) -> bool {
+      if (!epi_sync()) return false;
+      uint32_t* dst = a.hist12 + static_cast<int64_t>(row) * kTopkBins1;
+      for (int i = et; i < kTopkBins1; i += 128) {
+        const uint32_t v = shist[i];
+        if (v) {
+          atomicAdd(dst + i, v);
+          shist[i] = 0;
+        }
+      }
+      return epi_sync();
+    };
+    if (use_hist)
+      for (int i = et; i < kTopkBins1; i += 128) shist[i] = 0;
+    // Tails first (the epilogue warps wait for their first accumulator
+    // anyway): positions past each row's group tiles are -inf, the whole row
+    // NaN for an invalid row.  No tile writes there, so the order is free.
+    for (int r = blockIdx.x; r < a.rows; r += gridDim.x) {
+      int r0 = r;
+      while (!is_leader<QB>(a, r0)) --r0;
+      const Group g = group_at<QB>(a, r0);
+      int b;
+      row_visible(a, r, &b);
+      const bool ok = b >= 0 && b < a.cache.batch;
+      if (ok && et == 0) {
+        const int L = __ldg(a.cache.seq_lens + b);
+        if (L < 0 || L > a.cache.max_len) record_error(a.status, LSA_ERR_BOUNDS, r, L);
+      } else if (!ok && et == 0) {
+        record_error(a.status, LSA_ERR_BOUNDS, r, b);
+      }
+      const float val = ok ? -INFINITY : NAN;
+      int64_t start = ok ? static_cast<int64_t>(g.tiles) * kTile : 0;
+      start = start < a.ld ? start : a.ld;
+      float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+      const int64_t mis = (reinterpret_cast<uintptr_t>(row + start) >> 2) & 3;  // floats to 16-byte alignment
+      int64_t head = start + ((4 - mis) & 3);
+      head = head < a.ld ? head : a.ld;
+      for (int64_t p = start + et; p < head; p += 128) row[p] = val;
+      const int64_t nvec = (a.ld - head) >> 2;
+      float4* v4 = reinterpret_cast<float4*>(row + head);
+      for (int64_t i = et; i < nvec; i += 128) v4[i] = make_float4(val, val, val, val);
+      for (int64_t p = head + nvec * 4 + et; p < a.ld; p += 128) row[p] = val;
+    }
+    if (plan.n_items > 0) {
+      Walker<QB> W;
+      W.start(a, plan.r_first, plan.j_first);
+      int gi = -1, qi = 0;
+      int hist_row = -1;
+      int64_t vis_r[QB];
+      for (int64_t it = 0; it < plan.n_items; ++it) {
+        if (it == 0 || W.j == 0) {
+          ++gi;
+          qi = gi % C::kNQ;
+          if (use_hist && hist_row >= 0 && !flush_hist(hist_row)) {
+            if (lane == 0) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 6);
+              *abort_flag = 1;
+            }
+            hist_row = -1;
+            break;
+          }
+          hist_row = W.g.r0;
+          if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) {
+            if (lane == 0) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 4);
+              *abort_flag = 1;
+            }
+            hist_row = -1;
+            break;
+          }
+#pragma unroll
+          for (int qq = 0; qq < QB; ++qq) {
+            int bb;
+            vis_r[qq] = qq < W.g.nrows ? row_visible(a, W.g.r0 + qq, &bb) : 0;
+          }
+        }
+        const int acc = static_cast<int>(it & 1);
+        if (!tc::mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1), abort_flag)) {
+          if (lane == 0) {
+            record_error(a.status, LSA_ERR_TIMEOUT, 0, 5);
+            *abort_flag = 1;
+          }
+          hist_row = -1;
+          break;
+        }
+        tc::tc_fence_after();
+        // The tile's key rows (and FP8 scales) come from the producer through
+        // the stage; the stage is released once all four warps have read them.
+        int32_t mrow = 0;  // contiguous bf16: every visible position has a key row
+        float kscale = 1.f;
+        if (stage_meta) {
+          const int stg = static_cast<int>(it % C::kNS);
+          if (!tc::mbar_wait(&full[stg], static_cast<uint32_t>((it / C::kNS) & 1), abort_flag)) {
+            if (lane == 0) {
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 8);
+              *abort_flag = 1;
+            }
+            hist_row = -1;
+            break;
+          }
+          const int box = 2 * stg + (t >> 6);
+          mrow = smeta[box];
+          if (C::kFp8 && mrow >= 0) kscale = sscale[box * kScaleSlot + (mrow & 3) + (t & 63)];
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&empty[stg]);
+        }
+        const int64_t p = static_cast<int64_t>(W.j) * kTile + t;
+        const int64_t prow = mrow >= 0 ? static_cast<int64_t>(mrow) + (t & 63) : -1;
+        const float* wb = wbufs + qi * (C::kWBytes / 4);
+        float sc[QB];
+#pragma unroll
+        for (int qq = 0; qq < QB; ++qq) {
+          float s = 0.f;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float v[32];
+            const uint32_t col = acc * C::kAccCols + (C::kFp8 ? qq * 2 * kHeads : qq * kHeads) + c * 32;
+            tc::tmem_ld32(tmem_base + lane_base + col, v);
+            if (C::kFp8) {
+              float u[32];
+              tc::tmem_ld32(tmem_base + lane_base + col + kHeads, u);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) s = fmaf(wb[qq * kHeads + c * 32 + i], fmaxf(v[i] + u[i], 0.f), s);
+            } else {
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) s = fmaf(wb[qq * kHeads + c * 32 + i], fmaxf(v[i], 0.f), s);
+            }
+          }
+          sc[qq] = s * kscale;
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+        if (use_hist && p < vis_r[0] && prow >= 0) {
+          const uint32_t key = order_key(sc[0]);
+          if (key) atomicAdd(&shist[key >> 20], 1u);
+        }
+#pragma unroll
+        for (int qq = 0; qq < QB; ++qq) {
+          if (qq < W.g.nrows && p < a.ld) {
+            float o = -INFINITY;
+            if (p < vis_r[qq]) o = prow >= 0 ? sc[qq] : NAN;
+            a.scores[static_cast<int64_t>(W.g.r0 + qq) * a.ld + p] = o;
+          }
+        }
+        const bool last = (it + 1 == plan.n_items) || (W.j + 1 >= W.g.tiles);
+        if (last) {
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&qempty[qi]);
+        }
+        W.next(a);
+      }
+      if (use_hist && hist_row >= 0 && !flush_hist(hist_row) && lane == 0) {
+        record_error(a.status, LSA_ERR_TIMEOUT, 0, 7);
+        *abort_flag = 1;
+      }
+    }
+  }
+  tc::tc_fence_before();
+  scan_sync();
+  if (threadIdx.x == 0) {
+    for (uint64_t* b = bars; b <= ebar; ++b) tc::mbar_inval(b);
+  }
+  scan_sync();
+}
+
+}  // namespace scan
+}  // namespace lsa

@@ -23,6 +23,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "topk_sel.cuh"
 
 namespace lsa {
 namespace {
@@ -304,39 +305,11 @@ __global__ void __launch_bounds__(kT) k_topk_write(TopkArgs a, int64_t seg_len, 
 
 
 // ============================================================ three-kernel path
-constexpr int kB1 = kTopkBins1;     // 12-bit first digit
-constexpr int kCandCap = 8192;     // candidates kept per row
-constexpr int64_t kMaxBitmapCols = 1 << 19;
-constexpr int kFinT = 1024;        // threads of the per-row CTA
-constexpr int kWordElems = 32;     // positions per bitmap word (one thread's share of a round)
-constexpr int kColRound = kT * kWordElems;  // positions per collect round (8192)
-
-// Workspace: [rows][4096] first-digit histograms | [rows][words] bitmaps of the
-// keys above the threshold bin | [rows] candidate counts | [rows][kCandCap]
-// candidates (key, position).
-struct TkLayout {
-  uint32_t* hist;
-  uint32_t* bitmap;
-  uint32_t* ncand;
-  uint2* cand;
-  int64_t words;
-};
-
-__host__ __device__ inline size_t al256(size_t b) { return (b + 255) / 256 * 256; }
-
-__host__ __device__ inline TkLayout tk_layout(void* ws, int32_t rows, int64_t n_cols) {
-  TkLayout L;
-  uint8_t* b = static_cast<uint8_t*>(ws);
-  L.words = (n_cols + 31) / 32;
-  L.hist = reinterpret_cast<uint32_t*>(b);
-  b += al256(static_cast<size_t>(rows) * kB1 * 4);
-  L.ncand = reinterpret_cast<uint32_t*>(b);
-  b += al256(static_cast<size_t>(rows) * 4);
-  L.bitmap = reinterpret_cast<uint32_t*>(b);
-  b += al256(static_cast<size_t>(rows) * L.words * 4);
-  L.cand = reinterpret_cast<uint2*>(b);
-  return L;
-}
+using tk::kB1;
+using tk::kCandCap;
+using tk::TkLayout;
+using tk::tk_layout;
+constexpr int kFinT = 1024;  // threads of the per-row select CTA
 
 // Histogram of key bits [31:20] per row (when the scan did not build it).
 __global__ void __launch_bounds__(kT) k_tk_hist12(TopkArgs a, int64_t seg_len) {
@@ -360,285 +333,15 @@ __global__ void __launch_bounds__(kT) k_tk_hist12(TopkArgs a, int64_t seg_len) {
     if (h[i]) atomicAdd(dst + i, h[i]);
 }
 
-// Threshold bin b1 of each row, then each thread takes 32 consecutive
-// positions per round: the keys above b1 become one bitmap word (written once,
-// no atomics) and the keys inside b1 are appended to the row's candidates
-// (one atomic per CTA and round).  Segments are multiples of 8192 positions
-// and cover [0, n_cols), so every bitmap word is written.
-__global__ void __launch_bounds__(kT) k_tk_collect(TopkArgs a, int64_t seg_len) {
-  __shared__ int sh[kT / 32];
-  __shared__ uint32_t s_base;
-  const int r = blockIdx.y, seg = blockIdx.x;
-  int64_t n = a.n_cols;
-  if (a.valid_len) {
-    const int64_t v = __ldg(a.valid_len + r);
-    n = v < 0 ? 0 : (v < n ? v : n);
-  }
-  const int64_t s0 = static_cast<int64_t>(seg) * seg_len;
-  const int64_t s1 = s0 + seg_len < a.n_cols ? s0 + seg_len : a.n_cols;
-  if (s0 >= s1) return;
-  const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
-  const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
-  Found f = find_bin<kB1>(hist, 0xffffffffu, sh);
-  const uint32_t keff = f.total < static_cast<uint32_t>(a.k) ? f.total : static_cast<uint32_t>(a.k);
-  uint32_t b1 = 0xffffffffu;  // no selection: no bin qualifies
-  if (keff > 0) {
-    f = find_bin<kB1>(hist, keff, sh);
-    b1 = static_cast<uint32_t>(f.bin);
-  }
-  uint32_t* bitmap = L.bitmap + static_cast<int64_t>(r) * L.words;
-  uint2* cand = L.cand + static_cast<int64_t>(r) * kCandCap;
-  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  for (int64_t base = s0; base < s1; base += kColRound) {
-    const int64_t p0 = base + static_cast<int64_t>(threadIdx.x) * kWordElems;
-    uint32_t key[kWordElems];
-    if (p0 + kWordElems <= n) {
-      const float4* src = reinterpret_cast<const float4*>(row + p0);
-#pragma unroll
-      for (int v = 0; v < kWordElems / 4; ++v) {
-        const float4 x = __ldg(src + v);
-        key[4 * v] = order_key(x.x); key[4 * v + 1] = order_key(x.y);
-        key[4 * v + 2] = order_key(x.z); key[4 * v + 3] = order_key(x.w);
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < kWordElems; ++e) key[e] = p0 + e < n ? order_key(__ldg(row + p0 + e)) : 0u;
-    }
-    uint32_t word = 0;
-    int nc = 0;
-#pragma unroll
-    for (int e = 0; e < kWordElems; ++e) {
-      const uint32_t bin = key[e] ? (key[e] >> 20) : 0xffffffffu;
-      if (keff > 0 && key[e] && bin > b1) word |= 1u << e;
-      nc += (keff > 0 && key[e] && bin == b1);
-    }
-    if (p0 < a.n_cols) bitmap[p0 / kWordElems] = word;
-    int tot;
-    const int off = block_excl_scan(nc, sh, &tot);
-    if (threadIdx.x == 0) s_base = tot ? atomicAdd(L.ncand + r, static_cast<uint32_t>(tot)) : 0u;
-    __syncthreads();
-    uint32_t o = s_base + static_cast<uint32_t>(off);
-    __syncthreads();
-    if (nc) {
-#pragma unroll
-      for (int e = 0; e < kWordElems; ++e) {
-        if (keff > 0 && key[e] && (key[e] >> 20) == b1) {
-          if (o < static_cast<uint32_t>(kCandCap)) cand[o] = make_uint2(key[e], static_cast<uint32_t>(p0 + e));
-          ++o;
-        }
-      }
-    }
-  }
+__global__ void __launch_bounds__(tk::kCollectThreads) k_tk_collect(TopkArgs a, int64_t seg_len) {
+  __shared__ tk::TkScratch S;
+  tk::tk_collect_cta<2>(a, seg_len, blockIdx.x, blockIdx.y, S);
 }
 
-// Block-wide (kFinT threads) exclusive scan.
-__device__ __forceinline__ int fin_excl_scan(int v, int* warp_sums, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_sums[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = warp_sums[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    warp_sums[lane] = w;
-  }
-  __syncthreads();
-  const int before = warp ? warp_sums[warp - 1] : 0;
-  *total = warp_sums[kFinT / 32 - 1];
-  __syncthreads();
-  return before + x - v;
-}
-
-// Bin of the rank-th largest key in a 1024-bin shared histogram (one bin per
-// thread); returns the bin and the rank inside it through shared memory.
-__device__ __forceinline__ void fin_find(const uint32_t* h, uint32_t rank, int* warp_sums, int* out_bin,
-                                         uint32_t* out_rank) {
-  const int t = threadIdx.x;
-  const uint32_t v = h[t];
-  int tot;
-  const int excl = fin_excl_scan(static_cast<int>(v), warp_sums, &tot);
-  const uint32_t above = static_cast<uint32_t>(tot - excl) - v;  // keys in higher bins
-  if (v > 0 && above < rank && rank <= above + v) {
-    *out_bin = t;
-    *out_rank = rank - above;
-  }
-  __syncthreads();
-}
-
-// keeps the n lowest set bits of x
-__device__ __forceinline__ uint32_t low_bits(uint32_t x, int n) {
-  uint32_t y = 0;
-  for (int i = 0; i < n && x; ++i) {
-    const uint32_t b = x & (0u - x);
-    y |= b;
-    x ^= b;
-  }
-  return y;
-}
-
-// One CTA per row: keff and b1 from the histogram, the bitmap of the keys
-// above b1 and the candidates in shared memory, a radix select on the
-// candidates' low 20 bits (or, if they overflowed the list, on the row again),
-// and an ordered compaction of the bitmap.
 __global__ void __launch_bounds__(kFinT) k_tk_final(TopkArgs a) {
   extern __shared__ __align__(16) uint32_t fsm[];
-  __shared__ int warp_sums[32];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_rank;
-  __shared__ uint32_t h[1024];
-  const int r = blockIdx.x;
-  const int t = threadIdx.x;
-  const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
-  const int64_t nwords = L.words;
-  uint32_t* bm = fsm;               // selected positions
-  uint32_t* tb = fsm + nwords;      // positions equal to the threshold key
-  uint2* cs = reinterpret_cast<uint2*>(fsm + 2 * nwords);  // candidates: 2*nwords words keep 8-byte alignment
-  int32_t* out = a.idx + static_cast<int64_t>(r) * a.k;
-  int64_t n = a.n_cols;
-  if (a.valid_len) {
-    const int64_t v = __ldg(a.valid_len + r);
-    n = v < 0 ? 0 : (v < n ? v : n);
-  }
-  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  // issue every independent load first
-  const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
-  uint32_t hv[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) hv[i] = __ldcg(hist + t * 4 + i);
-  const uint32_t n_cand = __ldcg(L.ncand + r);
-  const uint32_t* gbm = L.bitmap + static_cast<int64_t>(r) * nwords;
-  for (int64_t w = t; w < nwords; w += kFinT) {
-    bm[w] = __ldcg(gbm + w);
-    tb[w] = 0;
-  }
-  const bool overflow = n_cand > static_cast<uint32_t>(kCandCap);
-  const int nc = overflow ? 0 : static_cast<int>(n_cand);
-  for (int c = t; c < nc; c += kFinT) cs[c] = __ldcg(L.cand + static_cast<int64_t>(r) * kCandCap + c);
-  // keff and the threshold bin (4 bins per thread)
-  uint32_t keff, b1, rank1;
-  {
-    const uint32_t mine = hv[0] + hv[1] + hv[2] + hv[3];
-    int total;
-    const int excl = fin_excl_scan(static_cast<int>(mine), warp_sums, &total);
-    keff = static_cast<uint32_t>(total) < static_cast<uint32_t>(a.k) ? static_cast<uint32_t>(total)
-                                                                     : static_cast<uint32_t>(a.k);
-    uint32_t cum = static_cast<uint32_t>(total - excl) - mine;
-    if (keff > 0 && cum < keff && keff <= cum + mine) {
-      for (int i = 3; i >= 0; --i) {
-        if (cum + hv[i] >= keff) {
-          s_bin = t * 4 + i;
-          s_rank = keff - cum;
-          break;
-        }
-        cum += hv[i];
-      }
-    }
-    __syncthreads();
-    b1 = static_cast<uint32_t>(s_bin);
-    rank1 = s_rank;  // wanted rank inside bin b1
-  }
-  for (int i = static_cast<int>(keff) + t; i < a.k; i += kFinT) out[i] = -1;
-  if (keff == 0) return;
-  // radix select on bits [19:10] then [9:0] among the keys of bin b1
-  uint32_t T = 0, ties = 0;
-  for (int pass = 0; pass < 2; ++pass) {
-    h[t] = 0;
-    __syncthreads();
-    const uint32_t shift = pass == 0 ? 10 : 0;
-    const uint32_t pre_shift = pass == 0 ? 20 : 10;
-    const uint32_t prefix = pass == 0 ? b1 : (T >> 10);
-    if (!overflow) {
-      for (int c = t; c < nc; c += kFinT) {
-        const uint32_t key = cs[c].x;
-        if ((key >> pre_shift) == prefix) atomicAdd(&h[(key >> shift) & 1023u], 1u);
-      }
-    } else {
-      for (int64_t base = 0; base < n; base += kFinT * 4) {
-        const int64_t p = base + t * 4;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (p + j >= n) break;
-          const uint32_t key = order_key(__ldg(row + p + j));
-          if (key && (key >> pre_shift) == prefix) atomicAdd(&h[(key >> shift) & 1023u], 1u);
-        }
-      }
-    }
-    __syncthreads();
-    if (t == 0) s_bin = -1;
-    __syncthreads();
-    fin_find(h, pass == 0 ? rank1 : ties, warp_sums, &s_bin, &s_rank);
-    const uint32_t bb = static_cast<uint32_t>(s_bin);
-    if (pass == 0) {
-      T = (b1 << 20) | (bb << 10);
-      ties = s_rank;
-    } else {
-      T |= bb;
-      ties = s_rank;
-    }
-    __syncthreads();
-  }
-  // mark keys of bin b1 above T, and collect the keys equal to T
-  if (!overflow) {
-    for (int c = t; c < nc; c += kFinT) {
-      const uint2 e = cs[c];
-      if (e.x > T) atomicOr(&bm[e.y >> 5], 1u << (e.y & 31));
-      else if (e.x == T) atomicOr(&tb[e.y >> 5], 1u << (e.y & 31));
-    }
-  } else {
-    for (int64_t base = 0; base < n; base += kFinT * 4) {
-      const int64_t p = base + t * 4;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (p + j >= n) break;
-        const uint32_t key = order_key(__ldg(row + p + j));
-        if ((key >> 20) != b1) continue;
-        const uint32_t q = static_cast<uint32_t>(p + j);
-        if (key > T) atomicOr(&bm[q >> 5], 1u << (q & 31));
-        else if (key == T) atomicOr(&tb[q >> 5], 1u << (q & 31));
-      }
-    }
-  }
-  __syncthreads();
-  // ordered compaction: the lowest `ties` positions equal to T join the selection
-  const int64_t per = (nwords + kFinT - 1) / kFinT;
-  const int64_t w0 = t * per, w1 = (w0 + per < nwords) ? w0 + per : nwords;
-  int my_ties = 0;
-  for (int64_t w = w0; w < w1; ++w) my_ties += __popc(tb[w]);
-  int tie_tot;
-  int tie_before = fin_excl_scan(my_ties, warp_sums, &tie_tot);
-  int my_sel = 0;
-  for (int64_t w = w0; w < w1; ++w) {
-    const uint32_t x = tb[w];
-    const int px = __popc(x);
-    const int take = static_cast<int>(ties) - tie_before;
-    uint32_t add = 0;
-    if (take > 0) add = take >= px ? x : low_bits(x, take);
-    tie_before += px;
-    const uint32_t merged = bm[w] | add;
-    bm[w] = merged;
-    my_sel += __popc(merged);
-  }
-  int sel_tot;
-  int o = fin_excl_scan(my_sel, warp_sums, &sel_tot);
-  for (int64_t w = w0; w < w1; ++w) {
-    uint32_t x = bm[w];
-    while (x) {
-      const int b = __ffs(x) - 1;
-      x &= x - 1;
-      if (o < a.k) out[o] = static_cast<int32_t>(w * 32 + b);
-      else record_error(a.status, LSA_ERR_BOUNDS, r, o);  // cannot happen
-      ++o;
-    }
-  }
+  __shared__ tk::TkScratch S;
+  tk::tk_final_cta<kFinT, 3>(a, blockIdx.x, fsm, S);
 }
 
 }  // namespace
@@ -660,16 +363,13 @@ TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
   return p;
 }
 
-bool topk_v2_ok(int64_t n_cols) { return n_cols <= kMaxBitmapCols; }
+bool topk_v2_ok(int64_t n_cols) { return n_cols <= tk::kMaxBitmapCols; }
 
-size_t topk_hist_zero_bytes(int32_t rows) {
-  return al256(static_cast<size_t>(rows) * kB1 * 4) + al256(static_cast<size_t>(rows) * 4);
-}
+size_t topk_hist_zero_bytes(int32_t rows) { return tk::tk_zero_bytes(rows); }
 
 size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t) {
   const size_t R = static_cast<size_t>(rows);
-  if (topk_v2_ok(n_cols))
-    return topk_hist_zero_bytes(rows) + al256(R * ((n_cols + 31) / 32) * 4) + al256(R * kCandCap * 8);
+  if (topk_v2_ok(n_cols)) return tk::tk_ws_bytes(rows, n_cols);
   TopkPlan p = topk_plan(rows, n_cols);
   size_t b = R * kHistStride * 4 + R * p.nseg * 8;
   return (b + 255) / 256 * 256;
@@ -679,14 +379,14 @@ int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 3 : 5; }
 
 // Segments of the collect pass: multiples of 8192 positions, about two CTAs
 // per SM in total.
-TopkPlan collect_plan(int32_t rows, int64_t n_cols) {
+TopkPlan topk_collect_plan(int32_t rows, int64_t n_cols) {
   TopkPlan p;
-  const int64_t rounds = (n_cols + kColRound - 1) / kColRound;
+  const int64_t rounds = (n_cols + tk::kColRound - 1) / tk::kColRound;
   int64_t want = (2LL * kPlanSMs + rows - 1) / (rows > 0 ? rows : 1);
   if (want > rounds) want = rounds;
   if (want < 1) want = 1;
   const int64_t per = (rounds + want - 1) / want;
-  p.seg_len = per * kColRound;
+  p.seg_len = per * tk::kColRound;
   p.nseg = static_cast<int32_t>((rounds + per - 1) / per);
   if (p.nseg < 1) p.nseg = 1;
   return p;
@@ -703,10 +403,10 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
       if (e != cudaSuccess) return e;
       k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
     }
-    const TopkPlan cp = collect_plan(a.rows, a.n_cols);
-    k_tk_collect<<<dim3(static_cast<unsigned>(cp.nseg), static_cast<unsigned>(a.rows)), kT, 0, s>>>(a, cp.seg_len);
-    const int64_t nwords = (a.n_cols + 31) / 32;
-    const size_t smem = 2 * nwords * 4 + static_cast<size_t>(kCandCap) * 8;
+    const TopkPlan cp = topk_collect_plan(a.rows, a.n_cols);
+    k_tk_collect<<<dim3(static_cast<unsigned>(cp.nseg), static_cast<unsigned>(a.rows)), tk::kCollectThreads, 0, s>>>(
+        a, cp.seg_len);
+    const size_t smem = tk::tk_final_smem(a.n_cols);
     static size_t smem_set = 0;
     if (smem > 48 * 1024 && smem > smem_set) {
       e = cudaFuncSetAttribute(k_tk_final, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "liblsa.so")
 LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_TIMEOUT, \
     LSA_ERR_BOUNDS = range(7)
 LSA_F32, LSA_BF16, LSA_FP8_E4M3 = 0, 1, 2
-LSA_OP_SCORES, LSA_OP_TOPK, LSA_OP_ATTN, LSA_OP_DECODE_STEP = 0, 1, 2, 3
+LSA_OP_SCORES, LSA_OP_TOPK, LSA_OP_ATTN, LSA_OP_DECODE_STEP, LSA_OP_DECODE_STEP_FUSED = 0, 1, 2, 3, 4
 LSA_STEP_UNFUSED, LSA_STEP_FUSED = 0, 1
 
 DTYPE_CODE = {"f32": LSA_F32, "bf16": LSA_BF16, "fp8": LSA_FP8_E4M3}

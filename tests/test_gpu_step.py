@@ -65,13 +65,57 @@ def test_decode_step_small(name):
     _check_step(case, list(range(case.rows)))
 
 
-def test_decode_step_fused_flag_matches_unfused():
+@pytest.mark.parametrize("name", ["tiny_fp32", "bf16_L5000", "paged_B5", "fp8_L6001", "len1"])
+def test_decode_step_fused_bitwise_equals_unfused(name):
+    """The fused step runs the CTA code of the separate launches with the same
+    plans, so selection, output and lse agree bit for bit (tiny_fp32 takes the
+    separate CUDA-core launches under either flag)."""
     from sparse_attention_decode_scan_b200.device import DeviceCase
-    dc = DeviceCase(cases.small("paged_B5"))
+    dc = DeviceCase(cases.small(name))
     o1, l1, i1 = _step(dc, 0)
     o2, l2, i2 = _step(dc, 1)
     assert torch.equal(i1, i2)
-    assert (o1.float() - o2.float()).abs().max().item() <= 1e-2
+    assert torch.equal(o1, o2)
+    assert torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("name", ["bf16_L5000", "paged_B5", "fp8_L6001", "len1"])
+def test_decode_step_fused_vs_oracle(name):
+    case = cases.small(name)
+    _check_step(case, list(range(case.rows)), flags=1)
+
+
+def _phase_ms(dc, flags):
+    from sparse_attention_decode_scan_b200 import lsa
+    s = dc.spec
+    B = dc.rows
+    out = torch.empty((B, s.n_heads, s.v_dim), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, s.n_heads), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.workspace_size(dc.dims, B, dc.max_len, lsa.LSA_OP_DECODE_STEP))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in ev:  # torch creates (and marks recorded) an event at its first record
+        e.record()
+    for _ in range(2):
+        lsa.decode_step_profiled(dc.dims, dc.cache, dc.q_idx, dc.w, dc.q, out, lse, ws, ev, flags=flags)
+    torch.cuda.synchronize()
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    return [ev[i].elapsed_time(ev[i + 1]) for i in range(3)]
+
+
+@pytest.mark.parametrize("name", ["paged_B5", "fp8_L6001"])
+def test_fused_step_is_one_launch(name):
+    """With LSA_STEP_FUSED the whole step is the one launch between the first
+    two phase events (the later events follow it immediately)."""
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+    dc = DeviceCase(cases.small(name))
+    assert lsa.launch_count(dc.dims, dc.rows, dc.max_len, lsa.LSA_OP_DECODE_STEP_FUSED) == 1
+    assert lsa.launch_count(dc.dims, dc.rows, dc.max_len, lsa.LSA_OP_DECODE_STEP) >= 3
+    fused = _phase_ms(dc, 1)
+    unfused = _phase_ms(dc, 0)
+    assert fused[0] > 0.0
+    assert fused[1] < 0.01 and fused[2] < 0.01, fused      # nothing runs after the single launch
+    assert unfused[1] > 0.002 and unfused[2] > 0.002, unfused  # top-k and attention launches
 
 
 def test_prefill_chain_small():
@@ -109,6 +153,25 @@ def test_decode_step_full(cfg):
 def test_decode_step_full_fp8():
     case = cases.full(4)
     _check_step(case, [0, 3])
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [2, 3, 4])
+def test_decode_step_full_fused_bitwise_equals_unfused(cfg):
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+    dc = DeviceCase(cases.full(cfg))
+    o1, l1, i1 = _step(dc, 0)
+    o2, l2, i2 = _step(dc, 1)
+    assert torch.equal(i1, i2)
+    assert torch.equal(o1, o2)
+    assert torch.equal(l1, l2)
+
+
+@pytest.mark.slow
+def test_decode_step_full_fused_vs_oracle():
+    case = cases.full(3)
+    rows = sorted({0, case.rows - 1, case.rows // 2})
+    _check_step(case, rows, flags=1)
 
 
 @pytest.mark.parametrize("name", ["paged_B5", "fp8_L6001", "bf16_L5000"])
