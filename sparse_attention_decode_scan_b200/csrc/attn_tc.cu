@@ -7,6 +7,8 @@
 #include "internal.h"
 #include "tc.cuh"
 
+#include <string.h>
+
 #include "attn_tc.cuh"
 
 namespace lsa {
@@ -68,19 +70,44 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   P.counters = reinterpret_cast<int*>(ws);
   P.part_lse = reinterpret_cast<float*>(ws + cnt_b);
   P.part_o = reinterpret_cast<float*>(ws + cnt_b + lse_b);
-  if (P.nsplit > 1) {
-    cudaError_t e = cudaMemsetAsync(P.counters, 0, static_cast<size_t>(a.rows) * 2 * sizeof(int), s);
-    if (e != cudaSuccess) return e;
-  }
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid(P.nsplit, 2, a.rows);
+  const dim3 grid(P.nsplit, 2, a.rows);
+  if (P.nsplit == 1) {
+    P.merge = kMergeSeparate;  // nothing to merge
+    k_attn_tc<<<grid, kThreads, kSmemBytes, s>>>(P);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaMemsetAsync(P.counters, 0, static_cast<size_t>(a.rows) * 2 * sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  // The split CTAs of a row meet in the kernel, which needs them all resident:
+  // a cooperative launch guarantees that or refuses.  Refused (fewer SMs than
+  // the one-wave plan assumes), the partials are merged by a second launch.
+  P.merge = kMergeInKernel;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr_c[1];
+  attr_c[0].id = cudaLaunchAttributeCooperative;
+  attr_c[0].val.cooperative = 1;
+  cfg.attrs = attr_c;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_attn_tc, P);
+  if (e == cudaSuccess) return cudaSuccess;
+  if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+  (void)cudaGetLastError();
+  P.merge = kMergeSeparate;
   k_attn_tc<<<grid, kThreads, kSmemBytes, s>>>(P);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_lse_merge(a, P.nsplit, P.part_o, P.part_lse, s);
 }
 
 }  // namespace lsa

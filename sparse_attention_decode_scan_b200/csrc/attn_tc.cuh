@@ -66,6 +66,11 @@ constexpr uint32_t kIdescPV = tc::idesc(tc::kFmtBF16, tc::kFmtBF16, 64, 256) | (
 
 static_assert(kSmemBytes <= 232448, "shared memory");
 
+// How the split partials of a (row, 64 heads) are combined.
+constexpr int kMergeSeparate = 0;  // partials only; a separate merge launch follows
+constexpr int kMergeInKernel = 1;  // the split CTAs meet, then each merges a slice
+                                   // (needs every CTA resident at once)
+
 struct TcAttnParams {
   AttnArgs a;
   int nsplit;
@@ -73,6 +78,7 @@ struct TcAttnParams {
   float* part_o;   // [rows][nsplit][128][512]
   float* part_lse; // [rows][nsplit][128]
   int* counters;   // [rows][2], zeroed before the launch
+  int merge;       // kMergeSeparate or kMergeInKernel
 };
 
 // MN-major operand in the 128-byte swizzle layout: 64-element MN blocks `lbo`
@@ -140,36 +146,55 @@ __device__ __forceinline__ RowCtx row_ctx(const AttnArgs& a, int r) {
 }
 
 // Stored rows of list entries j[0..N) of row r (-1: padding, out of range or
-// bad block).  All index loads are issued before the block-table loads.
+// bad block), in three steps that a caller may spread out so that each step's
+// loads have time to land: the positions (list loads), the block-table
+// entries of a paged cache (loads indexed by the positions), the rows.
 template <int N>
-__device__ __forceinline__ void entry_rows(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r,
-                                           const int (&j)[N], int j1, bool report, int64_t (&out)[N]) {
-  int32_t pos[N];
+__device__ __forceinline__ void ent_pos(const AttnArgs& a, const RowCtx& rc, int r, const int (&j)[N], int j1,
+                                        int32_t (&pos)[N]) {
 #pragma unroll
   for (int m = 0; m < N; ++m)
     // L2-coherent load: in the fused step the selection is written earlier in the same launch
     pos[m] = (j[m] < j1 && rc.ok) ? __ldcg(a.idx + static_cast<int64_t>(r) * a.k + j[m]) : -1;
-  if (ad.block_size == 0) {
+}
+
+template <int N>
+__device__ __forceinline__ void ent_blk(const CacheAddr& ad, const RowCtx& rc, const int32_t (&pos)[N],
+                                        int32_t (&blk)[N]) {
 #pragma unroll
-    for (int m = 0; m < N; ++m) out[m] = (pos[m] >= 0 && pos[m] < rc.L) ? static_cast<int64_t>(rc.b) * ad.max_len + pos[m] : -1;
-  } else {
-    int32_t blk[N];
-#pragma unroll
-    for (int m = 0; m < N; ++m) {
+  for (int m = 0; m < N; ++m) {
+    blk[m] = -1;
+    if (ad.block_size > 0) {
       const int64_t lb = pos[m] / ad.block_size;
-      blk[m] = (pos[m] >= 0 && pos[m] < rc.L && lb < ad.max_blocks)
-                   ? __ldg(ad.block_table + static_cast<int64_t>(rc.b) * ad.max_blocks + lb) : -1;
+      if (pos[m] >= 0 && pos[m] < rc.L && lb < ad.max_blocks)
+        blk[m] = __ldg(ad.block_table + static_cast<int64_t>(rc.b) * ad.max_blocks + lb);
     }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void ent_rows(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r,
+                                         const int32_t (&pos)[N], const int32_t (&blk)[N], bool report,
+                                         int64_t (&out)[N]) {
 #pragma unroll
-    for (int m = 0; m < N; ++m)
+  for (int m = 0; m < N; ++m) {
+    if (ad.block_size == 0)
+      out[m] = (pos[m] >= 0 && pos[m] < rc.L) ? static_cast<int64_t>(rc.b) * ad.max_len + pos[m] : -1;
+    else
       out[m] = (blk[m] >= 0 && blk[m] < ad.n_blocks)
                    ? static_cast<int64_t>(blk[m]) * ad.block_size + (pos[m] % ad.block_size) : -1;
+    if (report && pos[m] >= 0 && out[m] < 0) record_error(a.status, LSA_ERR_BOUNDS, r, pos[m]);
   }
-  if (report) {
-#pragma unroll
-    for (int m = 0; m < N; ++m)
-      if (pos[m] >= 0 && out[m] < 0) record_error(a.status, LSA_ERR_BOUNDS, r, pos[m]);
-  }
+}
+
+// The three steps back to back.
+template <int N>
+__device__ __forceinline__ void entry_rows(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r,
+                                           const int (&j)[N], int j1, bool report, int64_t (&out)[N]) {
+  int32_t pos[N], blk[N];
+  ent_pos<N>(a, rc, r, j, j1, pos);
+  ent_blk<N>(ad, rc, pos, blk);
+  ent_rows<N>(a, ad, rc, r, pos, blk, report, out);
 }
 
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* o, const float (&v)[32], float inv) {
@@ -182,6 +207,60 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* o, const float (&v)
       w[e] = *reinterpret_cast<const uint32_t*>(&pb);
     }
     *reinterpret_cast<uint4*>(o + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// out[r][half*64 + g/128][4(g%128) .. +3] = sum_s w[s][head] * part_o[r][s][..]
+// for the groups g in [i0, i1) of one (row, half), U groups per thread and
+// pass with the loads of V splits in flight together; w in shared memory
+// ([nsplit][64], normalised), splits summed in ascending order.
+template <int U, int V>
+__device__ __forceinline__ void merge_slice(const TcAttnParams& P, int r, int half, int i0, int i1,
+                                            const float* wsm) {
+  const int ns = P.nsplit;
+  const float4* po = reinterpret_cast<const float4*>(P.part_o);
+  for (int it0 = i0 + threadIdx.x; it0 < i1; it0 += U * kThreads) {
+    float4 acc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp0 = 0; sp0 < ns; sp0 += V) {
+      float4 x[U][V];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int item = it0 + u * kThreads;
+        const int hl = item / (kDv / 4), c4 = item % (kDv / 4);
+        const int h = half * kHeadsCta + hl;
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+          x[u][v] = (item < i1 && sp0 + v < ns)
+                        ? __ldcg(po + ((static_cast<int64_t>(r) * ns + sp0 + v) * kHeadsAll + h) * (kDv / 4) + c4)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int item = it0 + u * kThreads;
+        const int hl = (item < i1 ? item : i0) / (kDv / 4);
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+          const float wgt = sp0 + v < ns ? wsm[(sp0 + v) * kHeadsCta + hl] : 0.f;
+          acc[u].x = fmaf(wgt, x[u][v].x, acc[u].x); acc[u].y = fmaf(wgt, x[u][v].y, acc[u].y);
+          acc[u].z = fmaf(wgt, x[u][v].z, acc[u].z); acc[u].w = fmaf(wgt, x[u][v].w, acc[u].w);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int item = it0 + u * kThreads;
+      if (item >= i1) continue;
+      const int hl = item / (kDv / 4), c4 = item % (kDv / 4);
+      const int h = half * kHeadsCta + hl;
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[u].x, acc[u].y), hi = __floats2bfloat162_rn(acc[u].z, acc[u].w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(P.a.out) +
+                                (static_cast<int64_t>(r) * kHeadsAll + h) * kDv + c4 * 4) = pk;
+    }
   }
 }
 
@@ -242,13 +321,16 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     const int sub = t & 7;         // 16-byte column chunk within each 128-byte block
     const int rbase = t >> 3;      // 0..15
     const bool report = sub == 0 && half == 0;
-    // rows of this thread (4 per chunk) for chunks j, j+1 and j+2
-    int64_t rc_[4], rn_[4], rn2_[4];
-    auto lookup = [&](int jj, int64_t (&dst)[4]) {
-      int jl[4];
+    // This thread's 4 rows of each chunk go through three steps one chunk
+    // apart, so no step waits on the loads of the one before: at chunk j the
+    // rows of chunk j (formed two chunks earlier) are gathered, then the rows
+    // of chunk j+2 are formed (and prefetched into L2), the block-table
+    // entries of chunk j+3 and the list entries of chunk j+4 are loaded.  The
+    // lookups follow the gather, so each load has the next wait for a free
+    // buffer to land in.
+    auto jl_of = [&](int jj, int (&jl)[4]) {
 #pragma unroll
       for (int m = 0; m < 4; ++m) jl[m] = jj < nch ? j0 + jj * kChunk + rbase + 16 * m : j1;
-      entry_rows<4>(a, ad, rc, r, jl, j1, report, dst);
     };
     auto prefetch_l2 = [&](const int64_t (&rows)[4]) {
       if (sub != 0) return;
@@ -260,26 +342,36 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
                        "r"(kD * 2)
                        : "memory");
     };
-    // the first three chunks' lookups go out before the query copy, so their
-    // latency overlaps it
-    lookup(0, rc_);
-    lookup(1, rn_);
-    lookup(2, rn2_);
-    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q) +
-                          (static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta) * kD * 2;
-    const uint32_t qs_u = tc::smem_u32(qs);
-    for (int m = 0; m < 4; ++m) {
-      const int i = rbase + 16 * m;
-      const uint8_t* src = qsrc + static_cast<int64_t>(i) * kD * 2;
-      for (int d = 0; d < kBoxes; ++d)
-        cp_async16(qs_u + d * kQBlock + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
+    int64_t R0[4], R1[4];        // rows of chunks j, j+1
+    int32_t P2[4], B2[4], P3[4];  // positions and block entries of chunk j+2; positions of chunk j+3
+    {
+      int jl[4];
+      int32_t p0[4], p1[4], b0[4], b1[4];
+      jl_of(0, jl); ent_pos<4>(a, rc, r, jl, j1, p0);
+      jl_of(1, jl); ent_pos<4>(a, rc, r, jl, j1, p1);
+      jl_of(2, jl); ent_pos<4>(a, rc, r, jl, j1, P2);
+      jl_of(3, jl); ent_pos<4>(a, rc, r, jl, j1, P3);
+      ent_blk<4>(ad, rc, p0, b0);
+      ent_blk<4>(ad, rc, p1, b1);
+      ent_blk<4>(ad, rc, P2, B2);
+      // the query copy goes out while those loads are in flight
+      const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q) +
+                            (static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta) * kD * 2;
+      const uint32_t qs_u = tc::smem_u32(qs);
+      for (int m = 0; m < 4; ++m) {
+        const int i = rbase + 16 * m;
+        const uint8_t* src = qsrc + static_cast<int64_t>(i) * kD * 2;
+        for (int d = 0; d < kBoxes; ++d)
+          cp_async16(qs_u + d * kQBlock + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
+      }
+      cp_async_arrive_noinc(qfull);
+      ent_rows<4>(a, ad, rc, r, p0, b0, report, R0);
+      ent_rows<4>(a, ad, rc, r, p1, b1, report, R1);
+      prefetch_l2(R0);
+      prefetch_l2(R1);
     }
-    cp_async_arrive_noinc(qfull);
-    prefetch_l2(rc_);
-    prefetch_l2(rn_);
     for (int j = 0; j < nch; ++j) {
       const int b = j % kNBuf;
-      prefetch_l2(rn2_);  // chunk j+2 (looked up during the previous iteration)
       if (!tc::mbar_wait(&kvempty[b], ((j / kNBuf) & 1) ^ 1, abort_flag)) {
         if (t == 0) {
           record_error(a.status, LSA_ERR_TIMEOUT, r, 10);
@@ -293,8 +385,8 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int i = rbase + 16 * m;
-        if (rc_[m] >= 0) {
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cache.kv) + rc_[m] * (kD * 2);
+        if (R0[m] >= 0) {
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cache.kv) + R0[m] * (kD * 2);
 #pragma unroll
           for (int d = 0; d < kBoxes; ++d)
             cp_async16(kv_u + d * kBoxBytes + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
@@ -307,12 +399,22 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       }
       if (zeroed) tc::fence_proxy_async_smem();
       cp_async_arrive_noinc(&kvfull[b]);
+      int64_t R2[4];
+      ent_rows<4>(a, ad, rc, r, P2, B2, report, R2);  // chunk j+2
+      prefetch_l2(R2);
+      int32_t B3[4], P4[4];
+      int jl[4];
+      ent_blk<4>(ad, rc, P3, B3);  // chunk j+3
+      jl_of(j + 4, jl);
+      ent_pos<4>(a, rc, r, jl, j1, P4);  // chunk j+4
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        rc_[m] = rn_[m];
-        rn_[m] = rn2_[m];
+        R0[m] = R1[m];
+        R1[m] = R2[m];
+        P2[m] = P3[m];
+        B2[m] = B3[m];
+        P3[m] = P4[m];
       }
-      lookup(j + 3, rn2_);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kWarpMma) {
@@ -321,47 +423,66 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       const uint32_t q_u = tc::smem_u32(qs);
       bool ok = tc::mbar_wait(qfull, 0, abort_flag);
       tc::fence_proxy_async_smem();
-      auto issue_pv = [&](int i) -> bool {
-        if (!tc::mbar_wait(pfull, i & 1, abort_flag)) return false;
-        tc::tc_fence_after();
-        const uint32_t kv_u = tc::smem_u32(kvs + (i % kNBuf) * kKvBytes);
-        const uint32_t p_u = kv_u + kRopeBox * kBoxBytes;  // P(i) sits in chunk i's rope block
-        const uint64_t pa0 = tc::desc_sw128(p_u), vb0 = desc_sw128_mn(kv_u, kBoxBytes);
+      // Two event streams, served as they become ready: S(j) = Q K(j)^T once
+      // chunk j has landed and its score buffer is free, and P V(i) once P(i)
+      // is written.  P V(i) goes out as soon as it can (not after S(i+1)), so
+      // chunk i's buffer is released while chunk i+1 is still arriving and two
+      // gathers overlap.  S(j) waits until P V(j-2) has been issued: its commit
+      // then covers P V(j-2), which the softmax's parity wait on P V(j-1) needs.
+      int next_s = 0, next_pv = 0;
+      uint64_t t_last = tc::globaltimer_ns();
+      uint32_t spin = 0;
+      while (ok && next_pv < nch) {
+        bool progressed = false;
+        if (next_pv < next_s && tc::mbar_test(pfull, static_cast<uint32_t>(next_pv & 1))) {
+          const int i = next_pv;
+          tc::tc_fence_after();
+          const uint32_t kv_u = tc::smem_u32(kvs + (i % kNBuf) * kKvBytes);
+          const uint32_t p_u = kv_u + kRopeBox * kBoxBytes;  // P(i) sits in chunk i's rope block
+          const uint64_t pa0 = tc::desc_sw128(p_u), vb0 = desc_sw128_mn(kv_u, kBoxBytes);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t d = tmem + (static_cast<uint32_t>(16 * c) << 16);  // dims 256c.. at lane offset 16c
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t d = tmem + (static_cast<uint32_t>(16 * c) << 16);  // dims 256c.. at lane offset 16c
 #pragma unroll
-          for (int kk = 0; kk < kChunk / 16; ++kk)
-            tc::mma_f16(d, pa0 + static_cast<uint64_t>((kk * 32) >> 4),
-                        vb0 + static_cast<uint64_t>(((4 * c) * kBoxBytes + kk * 2048) >> 4), kIdescPV,
-                        (i > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kChunk / 16; ++kk)
+              tc::mma_f16(d, pa0 + static_cast<uint64_t>((kk * 32) >> 4),
+                          vb0 + static_cast<uint64_t>(((4 * c) * kBoxBytes + kk * 2048) >> 4), kIdescPV,
+                          (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::mma_commit(pvdone);
+          tc::mma_commit(&kvempty[i % kNBuf]);
+          ++next_pv;
+          progressed = true;
         }
-        tc::mma_commit(pvdone);
-        tc::mma_commit(&kvempty[i % kNBuf]);
-        return true;
-      };
-      for (int j = 0; ok && j < nch; ++j) {
-        const int b = j % kNBuf, sb = j & 1;
-        if (!tc::mbar_wait(&kvfull[b], (j / kNBuf) & 1, abort_flag)) { ok = false; break; }
-        tc::fence_proxy_async_smem();
-        if (!tc::mbar_wait(&sempty[sb], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        tc::tc_fence_after();
-        const uint32_t kv_u = tc::smem_u32(kvs + b * kKvBytes);
-        const uint32_t d = tmem + kColS + sb * kChunk;
-        // descriptors of the 36 K-steps differ only in the start-address field
-        // (addresses stay below 256 KB, so the 14-bit field never carries)
-        const uint64_t a0 = tc::desc_sw128(q_u), b0 = tc::desc_sw128(kv_u);
+        if (next_s < nch && next_s <= next_pv + 1) {
+          const int j = next_s;
+          const int b = j % kNBuf, sb = j & 1;
+          if (tc::mbar_test(&kvfull[b], static_cast<uint32_t>((j / kNBuf) & 1)) &&
+              tc::mbar_test(&sempty[sb], static_cast<uint32_t>(((j >> 1) & 1) ^ 1))) {
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_after();
+            const uint32_t d = tmem + kColS + sb * kChunk;
+            // descriptors of the 36 K-steps differ only in the start-address field
+            // (addresses stay below 256 KB, so the 14-bit field never carries)
+            const uint64_t a0 = tc::desc_sw128(q_u), b0 = tc::desc_sw128(tc::smem_u32(kvs + b * kKvBytes));
 #pragma unroll
-        for (int blk = 0; blk < kBoxes; ++blk) {
+            for (int blk = 0; blk < kBoxes; ++blk) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc::mma_f16(d, a0 + static_cast<uint64_t>((blk * kQBlock + k * 32) >> 4),
-                        b0 + static_cast<uint64_t>((blk * kBoxBytes + k * 32) >> 4), kIdescQK, (blk | k) != 0);
+              for (int k = 0; k < 4; ++k)
+                tc::mma_f16(d, a0 + static_cast<uint64_t>((blk * kQBlock + k * 32) >> 4),
+                            b0 + static_cast<uint64_t>((blk * kBoxBytes + k * 32) >> 4), kIdescQK, (blk | k) != 0);
+            }
+            tc::mma_commit(&sfull[sb]);
+            ++next_s;
+            progressed = true;
+          }
         }
-        tc::mma_commit(&sfull[sb]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        if (progressed) {
+          t_last = tc::globaltimer_ns();
+        } else if ((++spin & 63u) == 0) {
+          if (*abort_flag || tc::globaltimer_ns() - t_last > tc::kWaitLimitNs) ok = false;
+        }
       }
-      if (ok) ok = issue_pv(nch - 1);
       if (!ok) {
         record_error(a.status, LSA_ERR_TIMEOUT, r, 11);
         *abort_flag = 1;
@@ -385,19 +506,41 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
     // validity of the chunk's rows (lane and lane + 32), looked up one chunk ahead
-    auto valid2 = [&](int jj, bool* x, bool* y) {
-      const int jl[2] = {jj < nch ? j0 + jj * kChunk + lane : j1, jj < nch ? j0 + jj * kChunk + 32 + lane : j1};
-      int64_t rr[2];
-      entry_rows<2>(a, ad, rc, r, jl, j1, false, rr);
-      *x = rr[0] >= 0;
-      *y = rr[1] >= 0;
+    // Validity of this lane's two rows of each chunk (entries lane and lane+32),
+    // in the same three steps as the producer's lookups, one chunk apart:
+    // list entries two chunks ahead, block-table entries one ahead, so no
+    // load is read in the iteration that issues it.
+    auto jl_of = [&](int jj, int (&jl)[2]) {
+      jl[0] = jj < nch ? j0 + jj * kChunk + lane : j1;
+      jl[1] = jj < nch ? j0 + jj * kChunk + 32 + lane : j1;
     };
-    bool va, vb;
-    valid2(0, &va, &vb);
+    int32_t pA[2], bA[2], pB[2];  // chunk j: entries + block entries; chunk j+1: entries
+    {
+      int jl[2];
+      jl_of(0, jl);
+      ent_pos<2>(a, rc, r, jl, j1, pA);
+      jl_of(1, jl);
+      ent_pos<2>(a, rc, r, jl, j1, pB);
+      ent_blk<2>(ad, rc, pA, bA);
+    }
     for (int j = 0; j < nch; ++j) {
       const int sb = j & 1;
-      const uint32_t mlo = __ballot_sync(0xffffffffu, va), mhi = __ballot_sync(0xffffffffu, vb);
-      if (j + 1 < nch) valid2(j + 1, &va, &vb);
+      int64_t rr[2];
+      ent_rows<2>(a, ad, rc, r, pA, bA, false, rr);
+      const uint32_t mlo = __ballot_sync(0xffffffffu, rr[0] >= 0), mhi = __ballot_sync(0xffffffffu, rr[1] >= 0);
+      {
+        int32_t bB[2], pC[2];
+        int jl[2];
+        ent_blk<2>(ad, rc, pB, bB);  // chunk j+1
+        jl_of(j + 2, jl);
+        ent_pos<2>(a, rc, r, jl, j1, pC);  // chunk j+2
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          pA[m] = pB[m];
+          bA[m] = bB[m];
+          pB[m] = pC[m];
+        }
+      }
       if (!tc::mbar_wait(&sfull[sb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       tc::tc_fence_after();
       float s[64];
@@ -505,10 +648,14 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
         store_bf16x32(reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<int64_t>(r) * kHeadsAll + h) * kDv +
                           dim0 + cb * 32, v, inv);
       } else {
-        float* o = P.part_o + ((static_cast<int64_t>(r) * P.nsplit + split) * kHeadsAll + h) * kDv + dim0 + cb * 32;
+        // Staged in the idle chunk buffers as [64 heads][512], the 16-byte
+        // pieces of each 128-byte segment rotated by (head & 7) so that the
+        // warp's rows spread over the banks; written out coalesced below.
+        float* stg = reinterpret_cast<float*>(kvs);
+        const int seg = (dim0 + cb * 32) >> 5;
 #pragma unroll
         for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<float4*>(o + 4 * u) =
+          *reinterpret_cast<float4*>(stg + head_local * kDv + seg * 32 + ((u ^ (head_local & 7)) << 2)) =
               make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
       }
     }
@@ -520,84 +667,81 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       }
     }
   }
-  // ---------------------------------------------------------------- split merge by the last CTA
+  // ---------------------------------------------------------------- split partials out
+  // The CTA's partial O block [64 heads][512] is contiguous in part_o: every
+  // thread copies 16-byte pieces from the staging area, consecutive threads to
+  // consecutive addresses (full-line writes that drain quickly).
   if (P.nsplit > 1) {
+    __syncthreads();
+    const float4* stg4 = reinterpret_cast<const float4*>(kvs);
+    float4* dst = reinterpret_cast<float4*>(
+        P.part_o + ((static_cast<int64_t>(r) * P.nsplit + split) * kHeadsAll + half * kHeadsCta) * kDv);
+    for (int i = threadIdx.x; i < kHeadsCta * (kDv / 4); i += kThreads) {
+      const int hl = i >> 7, d4 = i & 127;
+      dst[i] = stg4[hl * (kDv / 4) + (d4 & ~7) + ((d4 & 7) ^ (hl & 7))];
+    }
+  }
+  // ---------------------------------------------------------------- split merge
+  // Every split CTA of (row, half) publishes its partials and counts itself;
+  // once all have (a bounded wait: the CTAs are co-resident), each merges its
+  // own slice of the 64 heads x 128 groups of 4 dims, so the merge reads run
+  // on all split CTAs at once.
+  if (P.nsplit > 1 && P.merge == kMergeInKernel) {
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
-      const int prev = atomicAdd(P.counters + 2 * r + half, 1);
-      *last_flag = prev == P.nsplit - 1;
+      int* ctr = P.counters + 2 * r + half;
+      atomicAdd(ctr, 1);
+      int go = 1;
+      const uint64_t t0 = tc::globaltimer_ns();
+      for (;;) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= P.nsplit) break;
+        if (tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) {
+          go = 0;
+          record_error(a.status, LSA_ERR_TIMEOUT, r, 13);
+          break;
+        }
+        __nanosleep(32);
+      }
+      *last_flag = go;
     }
     __syncthreads();
     if (*last_flag) {
-      __threadfence();
-      if (threadIdx.x == 0) P.counters[2 * r + half] = 0;  // left zeroed for the next call
-      // weights of every split for the 64 heads
-      float* wsm = reinterpret_cast<float*>(kvs);         // [nsplit][64] in the idle chunk buffer, nsplit <= 32
       const int ns = P.nsplit;
+      constexpr int kItems = kHeadsCta * (kDv / 4);
+      const int per = (kItems + ns - 1) / ns;
+      const int i0 = split * per;
+      const int i1 = i0 + per < kItems ? i0 + per : kItems;
+      // weights of every split for the heads this slice touches
+      float* wsm = reinterpret_cast<float*>(kvs);  // [nsplit][64] in the idle chunk buffer, nsplit <= 32
       const float* lse_p = P.part_lse + static_cast<int64_t>(r) * ns * kHeadsAll + half * kHeadsCta;
-      if (threadIdx.x < kHeadsCta) {
-        const int hl = threadIdx.x;
-        float mx = -INFINITY;
-        for (int sp = 0; sp < ns; ++sp) mx = fmaxf(mx, __ldcg(lse_p + sp * kHeadsAll + hl));
-        float den = 0.f;
-        for (int sp = 0; sp < ns; ++sp) {
-          const float e = mx == -INFINITY ? 0.f : exp2f((__ldcg(lse_p + sp * kHeadsAll + hl) - mx) * kLog2e);
-          wsm[sp * kHeadsCta + hl] = e;
-          den += e;
-        }
+      const int hl0 = i0 / (kDv / 4), hl1 = i1 > i0 ? (i1 - 1) / (kDv / 4) + 1 : hl0;
+      // one warp per head, one lane per split (nsplit <= 32): all lse loads at once
+      for (int x = warp; x < hl1 - hl0; x += kThreads / 32) {
+        const int hl = hl0 + x;
+        const float lv = lane < ns ? __ldcg(lse_p + lane * kHeadsAll + hl) : -INFINITY;
+        float mx = lv;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float e = (lane < ns && mx != -INFINITY) ? exp2f((lv - mx) * kLog2e) : 0.f;
+        float den = e;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
         const float inv = den > 0.f ? 1.f / den : 0.f;
-        for (int sp = 0; sp < ns; ++sp) wsm[sp * kHeadsCta + hl] *= inv;
-        if (a.lse) a.lse[static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + hl] = den > 0.f ? mx + logf(den) : -INFINITY;
+        if (lane < ns) wsm[lane * kHeadsCta + hl] = e * inv;
+        // the slice holding a head's first group writes its lse
+        if (lane == 0 && a.lse && hl * (kDv / 4) >= i0)
+          a.lse[static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + hl] = den > 0.f ? mx + logf(den) : -INFINITY;
       }
       __syncthreads();
-      // 64 heads x 128 groups of 4 dims over every thread of the CTA, eight
-      // groups per pass with the loads of two splits in flight together
-      const float4* po = reinterpret_cast<const float4*>(P.part_o);
-      constexpr int kItems = kHeadsCta * (kDv / 4);
-      for (int it0 = threadIdx.x; it0 < kItems; it0 += 8 * kThreads) {
-        float4 acc[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp0 = 0; sp0 < ns; sp0 += 2) {
-          float4 x[8][2];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int item = it0 + u * kThreads;
-            const int hl = item / (kDv / 4), c4 = item % (kDv / 4);
-            const int h = half * kHeadsCta + hl;
-#pragma unroll
-            for (int v = 0; v < 2; ++v)
-              x[u][v] = (item < kItems && sp0 + v < ns)
-                            ? __ldcg(po + ((static_cast<int64_t>(r) * ns + sp0 + v) * kHeadsAll + h) * (kDv / 4) + c4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int item = it0 + u * kThreads;
-            const int hl = (item < kItems ? item : 0) / (kDv / 4);
-#pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              const float wgt = sp0 + v < ns ? wsm[(sp0 + v) * kHeadsCta + hl] : 0.f;
-              acc[u].x = fmaf(wgt, x[u][v].x, acc[u].x); acc[u].y = fmaf(wgt, x[u][v].y, acc[u].y);
-              acc[u].z = fmaf(wgt, x[u][v].z, acc[u].z); acc[u].w = fmaf(wgt, x[u][v].w, acc[u].w);
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int item = it0 + u * kThreads;
-          if (item >= kItems) continue;
-          const int hl = item / (kDv / 4), c4 = item % (kDv / 4);
-          const int h = half * kHeadsCta + hl;
-          const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[u].x, acc[u].y), hi = __floats2bfloat162_rn(acc[u].z, acc[u].w);
-          uint2 pk;
-          pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-          pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-          *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
-                                    (static_cast<int64_t>(r) * kHeadsAll + h) * kDv + c4 * 4) = pk;
-        }
-      }
+      // About 16 loads in flight per thread: 8 groups x 2 splits when the slice
+      // is large (few splits), 1 group x 16 splits when it is small (many)
+      if (i1 - i0 >= 4 * kThreads)
+        merge_slice<8, 2>(P, r, half, i0, i1, wsm);
+      else
+        merge_slice<1, 16>(P, r, half, i0, i1, wsm);
     }
   }
   tc::tc_fence_before();

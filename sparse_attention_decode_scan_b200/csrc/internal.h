@@ -84,8 +84,8 @@ bool topk_v2_ok(int64_t n_cols);
 size_t topk_hist_zero_bytes(int32_t rows);
 // true if the scan can accumulate the top-k histogram itself
 bool scores_tc_fused_hist_ok(const ScoresArgs& a);
-// segments of the top-k collect pass
-TopkPlan topk_collect_plan(int32_t rows, int64_t n_cols);
+// segments of the top-k collect pass, about target_ctas CTAs in total
+TopkPlan topk_collect_plan(int32_t rows, int64_t n_cols, int32_t target_ctas);
 // tensor maps of the tensor-core scan (keys; FP8 scales)
 cudaError_t scan_tc_maps(const ScoresArgs& a, CUtensorMap* tmap, CUtensorMap* smap);
 

@@ -211,7 +211,10 @@ cudaError_t launch_step_fused(const ScoresArgs& sa, const TopkArgs& ta, const At
   F.attn.counters = reinterpret_cast<int*>(L.ctrl + tk::kCtrlInts);
   F.attn.part_lse = reinterpret_cast<float*>(part);
   F.attn.part_o = reinterpret_cast<float*>(part + lse_bytes);
-  const TopkPlan cp = topk_collect_plan(rows, ta.n_cols);
+  F.attn.merge = attn::kMergeInKernel;
+  // the split CTAs of a row meet inside the attention phase: each must be a CTA of its own
+  if (F.attn.nsplit > 1 && F.attn.nsplit * 2 * rows > num_sms()) return cudaErrorCooperativeLaunchTooLarge;
+  const TopkPlan cp = topk_collect_plan(rows, ta.n_cols, num_sms());  // one segment per CTA
   F.collect_nseg = cp.nseg;
   F.collect_seg_len = cp.seg_len;
   F.bar = L.ctrl;

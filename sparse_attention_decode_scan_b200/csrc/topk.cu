@@ -377,12 +377,13 @@ size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t) {
 
 int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 3 : 5; }
 
-// Segments of the collect pass: multiples of 8192 positions, about two CTAs
-// per SM in total.
-TopkPlan topk_collect_plan(int32_t rows, int64_t n_cols) {
+// Segments of the collect pass: multiples of 8192 positions, about
+// `target_ctas` CTAs in total (two per SM for the standalone launch, where two
+// latency-bound CTAs share an SM; one per CTA of the fused step).
+TopkPlan topk_collect_plan(int32_t rows, int64_t n_cols, int32_t target_ctas) {
   TopkPlan p;
   const int64_t rounds = (n_cols + tk::kColRound - 1) / tk::kColRound;
-  int64_t want = (2LL * kPlanSMs + rows - 1) / (rows > 0 ? rows : 1);
+  int64_t want = (static_cast<int64_t>(target_ctas) + rows - 1) / (rows > 0 ? rows : 1);
   if (want > rounds) want = rounds;
   if (want < 1) want = 1;
   const int64_t per = (rounds + want - 1) / want;
@@ -403,7 +404,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
       if (e != cudaSuccess) return e;
       k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
     }
-    const TopkPlan cp = topk_collect_plan(a.rows, a.n_cols);
+    const TopkPlan cp = topk_collect_plan(a.rows, a.n_cols, 2 * kPlanSMs);
     k_tk_collect<<<dim3(static_cast<unsigned>(cp.nseg), static_cast<unsigned>(a.rows)), tk::kCollectThreads, 0, s>>>(
         a, cp.seg_len);
     const size_t smem = tk::tk_final_smem(a.n_cols);
