@@ -17,8 +17,8 @@
  *      LeanSparse episode page).
  *   2. Top-k: the k highest scores of each row; equal scores go to the lower
  *      position; -inf and NaN are never selected.
- *   3. Sparse MQA over the selected rows only ("reduces reads but not storage",
- *      LeanSparse episode page): for every head h,
+ *   3. Sparse MQA over the selected rows only (what is read shrinks, what is
+ *      stored does not: LeanSparse episode page): for every head h,
  *          o[h] = sum_j softmax_j(scale * q[h] . KV[idx_j]) * KV[idx_j][0:D_v]
  *      and lse[h] = log sum_j exp(scale * q[h] . KV[idx_j]).
  *   Prefill: a chunk of query rows at positions p_i scores the cache under a

@@ -15,11 +15,11 @@ It is a plain, slow, fp64 restatement of what the step computes:
      (DeepSeek-V3.2-Exp technical report, the DSA source listed on the
      LeanSparse episode page).  FP8 keys carry a per-token scale:
      k_s = scale_s * e4m3(k_s).
-  2. Top-k.  Keep the k highest-scoring tokens; equal scores go to the lower
+  2. Top-k.  Keep the k tokens with the largest scores; equal scores go to the lower
      position; -inf (masked) and NaN are never kept; the kept positions are
      returned sorted ascending and padded with -1.
-  3. Sparse attention over the kept rows only (the "reduces reads but not
-     storage" point of the LeanSparse episode page): softmax(scale * q . K_sel)
+  3. Sparse attention over the kept rows only (the LeanSparse episode page's
+     point that sparse attention cuts what is read, not what is stored): softmax(scale * q . K_sel)
      weighted sum of V_sel, V being the first v_dim columns of the KV row, plus
      the log-sum-exp of the scaled logits.
   Prefill variant: a chunk of query rows at positions p_i scores the cache

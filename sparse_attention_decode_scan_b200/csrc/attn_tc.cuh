@@ -5,8 +5,8 @@
 // The layer attends only the k tokens the lightning indexer kept (MLI abstract,
 // sentence 2): o[h] = softmax_j(scale * q[h] . KV[idx_j]) . KV[idx_j][:512]
 // over 128 query heads sharing 576-wide bf16 KV rows (value = first 512
-// columns), plus lse[h].  Sparse attention reads only the kept rows (LeanSparse
-// episode page: it reduces reads, not storage).
+// columns), plus lse[h].  Only the kept rows are read (the LeanSparse episode
+// page: sparsity saves bytes read, the cache itself stays whole).
 //
 // Work: one CTA per (query row, half of the heads, split of the index list).
 // 64 heads make the MMA's M side (M = 64), so the fp32 output accumulator

@@ -1,8 +1,8 @@
 // Lightning-indexer scores on CUDA cores (any H_I <= 64, d_I multiple of 8).
 //
 // I(s) = sum_h w[h] * ReLU(scale_s * q_idx[h] . K[s])   (DSA lightning indexer,
-// DeepSeek-V3.2-Exp report; the scan that scores the whole cache before each
-// layer, MLI abstract sentence 2).  One thread per cached position; the query
+// DeepSeek-V3.2-Exp report; the pass over every cached token that precedes
+// each layer, MLI abstract sentence 2).  One thread per cached position; the query
 // row's H_I x d_I block and weights sit in shared memory as fp32.  This is the
 // general-shape path (the tiny fp32 workload, odd head counts); the tensor-core
 // kernel in indexer_tc.cu takes the 64 x 128 production shape.

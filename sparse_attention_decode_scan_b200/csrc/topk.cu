@@ -1,6 +1,6 @@
 // Exact top-k of fp32 score rows on an order-preserving 32-bit key.
 //
-// Keeps the k highest-scoring tokens of each row (MLI abstract, sentence 2):
+// Keeps the k tokens with the largest scores in each row (MLI abstract, sentence 2):
 //   * -0.0 compares equal to +0.0 (canonicalised before the key transform);
 //   * -inf and NaN are never selected (they map to key 0, which is skipped);
 //   * among equal scores the lower position is kept;

@@ -4,7 +4,7 @@
 // named barrier, so a block may hold more threads than take part.
 //
 // Exact top-k on an order-preserving 32-bit key (MLI abstract, sentence 2:
-// the k highest-scoring tokens are kept): -0.0 equals +0.0, -inf and NaN are
+// the k best-scored tokens are kept): -0.0 equals +0.0, -inf and NaN are
 // never selected, among equal scores the lower position wins, and a row's
 // output is its min(k, #selectable) positions in ascending order, then -1.
 #pragma once
