@@ -145,7 +145,8 @@ def source_hash(paths) -> str:
     return h.hexdigest()[:16]
 
 
-SCAN_SOURCES = ["sparse_attention_decode_scan_b200/csrc/indexer_tc.cu",
+SCAN_SOURCES = ["sparse_attention_decode_scan_b200/csrc/scan_tc.cuh",
+                "sparse_attention_decode_scan_b200/csrc/indexer_tc.cu",
                 "sparse_attention_decode_scan_b200/csrc/indexer_simt.cu",
                 "sparse_attention_decode_scan_b200/csrc/common.cuh",
                 "sparse_attention_decode_scan_b200/csrc/tc.cuh"]
