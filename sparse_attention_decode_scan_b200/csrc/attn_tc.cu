@@ -44,8 +44,11 @@ bool attn_tc_shape_ok(int32_t dtype, int32_t H, int32_t D, int32_t Dv, int32_t) 
 int attn_tc_launches(int32_t, int32_t, int32_t) { return 1; }
 
 bool attn_tc_supported(const AttnArgs& a) {
+  // KV rows are kept as 32-bit indices
+  const int64_t kv_rows = a.cache.block_size > 0 ? a.cache.n_blocks * a.cache.block_size
+                                                 : static_cast<int64_t>(a.cache.batch) * a.cache.max_len;
   return attn_tc_shape_ok(a.dtype, a.H, a.D, a.Dv, a.cache.block_size) && aligned16(a.cache.kv) && aligned16(a.q) &&
-         aligned16(a.out);
+         aligned16(a.out) && kv_rows < (1LL << 31);
 }
 
 size_t attn_tc_ws_bytes(int32_t rows, int32_t H, int32_t D, int32_t Dv, int32_t k) {

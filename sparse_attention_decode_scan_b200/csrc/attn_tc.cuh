@@ -44,19 +44,28 @@ constexpr int kHeadsCta = 64;
 constexpr int kD = 576;
 constexpr int kDv = 512;
 constexpr int kChunk = 64;                 // KV rows per chunk
-constexpr int kNBuf = 2;                   // chunk buffers
+constexpr int kNBuf = 3;                   // chunk buffers
 constexpr int kBoxes = kD / 64;            // 9 column blocks of 64 dims
 constexpr int kBoxBytes = kChunk * 128;    // 64 rows x 128 B
 constexpr int kKvBytes = kBoxes * kBoxBytes;          // 73728
-constexpr int kQBlock = kHeadsCta * 128;              // 8192
-constexpr int kQBytes = kBoxes * kQBlock;             // 73728
+constexpr int kRowTab = 2048;                         // KV rows of up to 2048 list entries, resolved ahead in smem
 constexpr int kRopeBox = kBoxes - 1;                  // column block of dims 512-575; holds P after S
 constexpr int kThreads = 288;
 constexpr int kProdThreads = 128;
 constexpr int kWarpMma = 4;                // warps 5-8: softmax
-constexpr int kSmemBytes = kQBytes + kNBuf * kKvBytes + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr int kSmemBytes = kNBuf * kKvBytes + kRowTab * 4 + 1024 /*barriers*/ + 1024 /*align*/;
+// TMEM (512 columns x 128 lanes; an M = 64 tile uses lanes 0-15 or 16-31 of
+// each 32-lane quarter):
+//   lanes 0-15:  Q, dims 0-575 as bf16 pairs, the QK MMA's A operand (columns
+//                0-287) | S (columns 288-351)
+//   lanes 16-31: O, dims 0-511 (columns 0-511)
+// An A operand in TMEM must start at lane 0 and its accumulator must sit on
+// the same lanes, so Q and S share lanes 0-15.  Shared memory then holds three
+// chunk buffers and a table of the split's KV rows.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 256;            // score buffers start column
+constexpr uint32_t kColQ = 0;              // Q dims 0-575 (lane offset 0)
+constexpr uint32_t kColS = 288;            // S (lane offset 0)
+constexpr uint32_t kLaneHi = 16u << 16;    // TMEM address offset of lane 16 (O)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.f;        // lazy rescale threshold (factor 256)
@@ -91,6 +100,29 @@ __device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t addr, uint32_t lbo) {
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (A read from tensor memory).
+__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+      "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+      "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -172,6 +204,22 @@ __device__ __forceinline__ void ent_blk(const CacheAddr& ad, const RowCtx& rc, c
   }
 }
 
+// Block-table entries from the row's table cached in shared memory (sbt), or
+// from global memory when it is not cached.
+template <int N>
+__device__ __forceinline__ void ent_blk_s(const CacheAddr& ad, const RowCtx& rc, const int32_t* sbt, bool cached,
+                                          const int32_t (&pos)[N], int32_t (&blk)[N]) {
+  if (!cached) {
+    ent_blk<N>(ad, rc, pos, blk);
+    return;
+  }
+#pragma unroll
+  for (int m = 0; m < N; ++m) {
+    const int64_t lb = pos[m] / ad.block_size;
+    blk[m] = (pos[m] >= 0 && pos[m] < rc.L && lb < ad.max_blocks) ? sbt[lb] : -1;
+  }
+}
+
 template <int N>
 __device__ __forceinline__ void ent_rows(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r,
                                          const int32_t (&pos)[N], const int32_t (&blk)[N], bool report,
@@ -195,6 +243,27 @@ __device__ __forceinline__ void entry_rows(const AttnArgs& a, const CacheAddr& a
   ent_pos<N>(a, rc, r, j, j1, pos);
   ent_blk<N>(ad, rc, pos, blk);
   ent_rows<N>(a, ad, rc, r, pos, blk, report, out);
+}
+
+// KV rows of the list entries at offsets [lo, hi) from j0 (at most kRowTab
+// past the table's base offset `base`) into rtab, by n threads (tid): per
+// pass 8 list loads in flight, then their 8 block-table loads.
+__device__ __forceinline__ void fill_rows(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r, int j0,
+                                          int j1, int base, int lo, int hi, int tid, int n, bool report,
+                                          int32_t* rtab) {
+  for (int e = lo + tid; e < hi; e += 8 * n) {
+    int jl[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) jl[u] = e + u * n < hi ? j0 + e + u * n : j1;
+    int32_t pos[8], blk[8];
+    int64_t rows[8];
+    ent_pos<8>(a, rc, r, jl, j1, pos);
+    ent_blk<8>(ad, rc, pos, blk);
+    ent_rows<8>(a, ad, rc, r, pos, blk, report, rows);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (e + u * n < hi) rtab[e + u * n - base] = static_cast<int32_t>(rows[u]);
+  }
 }
 
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* o, const float (&v)[32], float inv) {
@@ -273,19 +342,22 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
                                          const volatile uint32_t* tmem_slot) {
   const AttnArgs& a = P.a;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qs = smem;
-  uint8_t* kvs = qs + kQBytes;         // kNBuf chunk buffers
-  uint64_t* bars = reinterpret_cast<uint64_t*>(kvs + kNBuf * kKvBytes);
+  uint8_t* kvs = smem;                                                  // kNBuf chunk buffers
+  int32_t* rtab = reinterpret_cast<int32_t*>(kvs + kNBuf * kKvBytes);   // KV rows of the split's entries (-1: none)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rtab + kRowTab);
   uint64_t* qfull = bars;
   uint64_t* kvfull = bars + 1;            // [kNBuf]
   uint64_t* kvempty = kvfull + kNBuf;     // [kNBuf]
-  uint64_t* sfull = kvempty + kNBuf;      // [2]
-  uint64_t* sempty = sfull + 2;           // [2]
-  uint64_t* pfull = sempty + 2;
+  uint64_t* sfull = kvempty + kNBuf;      // S(j) computed
+  uint64_t* rdone = sfull + 1;            // S(j) read and O rescaled: S(j+1) may be computed
+  uint64_t* pfull = rdone + 1;
   uint64_t* pvdone = pfull + 1;
   uint64_t* done = pvdone + 1;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 1);
+  uint64_t* vfull = done + 1;             // [kNBuf] the chunk's row validity is written
+  uint64_t* tfull = vfull + kNBuf;        // the softmax warps resolved the table's tail
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tfull + 1);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
+  uint8_t* vrow = reinterpret_cast<uint8_t*>(last_flag + 1);  // [kNBuf][kChunk]: 1 = the row has a KV row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j0 = split * P.split_len;
@@ -293,18 +365,18 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
   const int nch = j1 > j0 ? (j1 - j0 + kChunk - 1) / kChunk : 0;
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(qfull, kProdThreads);
+    tc::mbar_init(qfull, 4);  // the softmax warps' TMEM stores of Q
     for (int i = 0; i < kNBuf; ++i) {
       tc::mbar_init(&kvfull[i], kProdThreads);
       tc::mbar_init(&kvempty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&sfull[i], 1);
-      tc::mbar_init(&sempty[i], 4);
-    }
+    tc::mbar_init(sfull, 1);
+    tc::mbar_init(rdone, 4);
     tc::mbar_init(pfull, 4);
     tc::mbar_init(pvdone, 1);
     tc::mbar_init(done, 1);
+    for (int i = 0; i < kNBuf; ++i) tc::mbar_init(&vfull[i], 4);  // one arrival per producer warp
+    tc::mbar_init(tfull, 4);                                        // one arrival per softmax warp
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -321,57 +393,62 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     const int sub = t & 7;         // 16-byte column chunk within each 128-byte block
     const int rbase = t >> 3;      // 0..15
     const bool report = sub == 0 && half == 0;
-    // This thread's 4 rows of each chunk go through three steps one chunk
-    // apart, so no step waits on the loads of the one before: at chunk j the
-    // rows of chunk j (formed two chunks earlier) are gathered, then the rows
-    // of chunk j+2 are formed (and prefetched into L2), the block-table
-    // entries of chunk j+3 and the list entries of chunk j+4 are loaded.  The
-    // lookups follow the gather, so each load has the next wait for a free
-    // buffer to land in.
-    auto jl_of = [&](int jj, int (&jl)[4]) {
-#pragma unroll
-      for (int m = 0; m < 4; ++m) jl[m] = jj < nch ? j0 + jj * kChunk + rbase + 16 * m : j1;
+    // The KV rows of the split's list entries are resolved ahead into a table
+    // in shared memory (up to kRowTab entries at a time), so the gather loop
+    // issues no dependent global load of its own.  The first kHeadRows rows are
+    // resolved here; the softmax warps, idle until the first scores, resolve the
+    // rest of the first kRowTab and signal tfull.
+    constexpr int kHeadRows = 4 * kChunk;
+    const int n_ent = j1 - j0;
+    const int first_hi = n_ent < kRowTab ? n_ent : kRowTab;
+    auto fill_table = [&](int e0) {  // a later part: entries [e0, e0 + kRowTab), all by the producer
+      const int hi = n_ent - e0 < kRowTab ? n_ent : e0 + kRowTab;
+      fill_rows(a, ad, rc, r, j0, j1, e0, e0, hi, t, kProdThreads, half == 0, rtab);
+      asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");  // the producer warps
     };
-    auto prefetch_l2 = [&](const int64_t (&rows)[4]) {
-      if (sub != 0) return;
+    auto row_of = [&](int jj, int m) -> int64_t {  // chunk jj, this thread's m-th row
+      const int e = jj * kChunk + rbase + 16 * m;  // entry offset in the split
+      return jj < nch ? static_cast<int64_t>(rtab[e % kRowTab]) : -1;
+    };
+    auto prefetch_l2 = [&](int jj, int j_now) {
+      // only chunks whose rows are in the table now
+      if (sub != 0 || jj >= nch || (jj * kChunk) / kRowTab != (j_now * kChunk) / kRowTab) return;
+      if (jj * kChunk >= kHeadRows && j_now * kChunk < kHeadRows) return;  // the table's tail may not be there yet
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-        if (rows[m] >= 0)
+      for (int m = 0; m < 4; ++m) {
+        const int64_t row = row_of(jj, m);
+        if (row >= 0)
           asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                           reinterpret_cast<const uint8_t*>(a.cache.kv) + rows[m] * (kD * 2)),
+                           reinterpret_cast<const uint8_t*>(a.cache.kv) + row * (kD * 2)),
                        "r"(kD * 2)
                        : "memory");
-    };
-    int64_t R0[4], R1[4];        // rows of chunks j, j+1
-    int32_t P2[4], B2[4], P3[4];  // positions and block entries of chunk j+2; positions of chunk j+3
-    {
-      int jl[4];
-      int32_t p0[4], p1[4], b0[4], b1[4];
-      jl_of(0, jl); ent_pos<4>(a, rc, r, jl, j1, p0);
-      jl_of(1, jl); ent_pos<4>(a, rc, r, jl, j1, p1);
-      jl_of(2, jl); ent_pos<4>(a, rc, r, jl, j1, P2);
-      jl_of(3, jl); ent_pos<4>(a, rc, r, jl, j1, P3);
-      ent_blk<4>(ad, rc, p0, b0);
-      ent_blk<4>(ad, rc, p1, b1);
-      ent_blk<4>(ad, rc, P2, B2);
-      // the query copy goes out while those loads are in flight
-      const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q) +
-                            (static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta) * kD * 2;
-      const uint32_t qs_u = tc::smem_u32(qs);
-      for (int m = 0; m < 4; ++m) {
-        const int i = rbase + 16 * m;
-        const uint8_t* src = qsrc + static_cast<int64_t>(i) * kD * 2;
-        for (int d = 0; d < kBoxes; ++d)
-          cp_async16(qs_u + d * kQBlock + tc::sw128_offset(i, sub), src + d * 128 + sub * 16);
       }
-      cp_async_arrive_noinc(qfull);
-      ent_rows<4>(a, ad, rc, r, p0, b0, report, R0);
-      ent_rows<4>(a, ad, rc, r, p1, b1, report, R1);
-      prefetch_l2(R0);
-      prefetch_l2(R1);
-    }
+    };
+    (void)report;
+    fill_rows(a, ad, rc, r, j0, j1, 0, 0, first_hi < kHeadRows ? first_hi : kHeadRows, t, kProdThreads, half == 0,
+              rtab);
+    asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");  // the producer warps
+    prefetch_l2(0, 0);
+    prefetch_l2(1, 0);
+#pragma unroll 1
     for (int j = 0; j < nch; ++j) {
       const int b = j % kNBuf;
+      if (j > 0 && (j * kChunk) % kRowTab == 0) {  // the next kRowTab entries (splits longer than the table)
+        // every producer thread has read its rows of the previous part
+        asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");
+        fill_table(j * kChunk);
+        prefetch_l2(j, j);
+        prefetch_l2(j + 1, j);
+      }
+      if (j * kChunk == kHeadRows && first_hi > kHeadRows) {  // the rest of the first part, from the softmax warps
+        if (!tc::mbar_wait(tfull, 0, abort_flag)) {
+          if (t == 0) {
+            record_error(a.status, LSA_ERR_TIMEOUT, r, 14);
+            *abort_flag = 1;
+          }
+          break;
+        }
+      }
       if (!tc::mbar_wait(&kvempty[b], ((j / kNBuf) & 1) ^ 1, abort_flag)) {
         if (t == 0) {
           record_error(a.status, LSA_ERR_TIMEOUT, r, 10);
@@ -382,9 +459,11 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       uint8_t* kvb = kvs + b * kKvBytes;
       const uint32_t kv_u = tc::smem_u32(kvb);
       bool zeroed = false;
+      int64_t R0[4];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int i = rbase + 16 * m;
+        R0[m] = row_of(j, m);
         if (R0[m] >= 0) {
           const uint8_t* src = reinterpret_cast<const uint8_t*>(a.cache.kv) + R0[m] * (kD * 2);
 #pragma unroll
@@ -399,30 +478,22 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       }
       if (zeroed) tc::fence_proxy_async_smem();
       cp_async_arrive_noinc(&kvfull[b]);
-      int64_t R2[4];
-      ent_rows<4>(a, ad, rc, r, P2, B2, report, R2);  // chunk j+2
-      prefetch_l2(R2);
-      int32_t B3[4], P4[4];
-      int jl[4];
-      ent_blk<4>(ad, rc, P3, B3);  // chunk j+3
-      jl_of(j + 4, jl);
-      ent_pos<4>(a, rc, r, jl, j1, P4);  // chunk j+4
+      // the softmax masks the rows without a KV row
+      if (sub == 0) {
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        R0[m] = R1[m];
-        R1[m] = R2[m];
-        P2[m] = P3[m];
-        B2[m] = B3[m];
-        P3[m] = P4[m];
+        for (int m = 0; m < 4; ++m) vrow[b * kChunk + rbase + 16 * m] = R0[m] >= 0 ? 1 : 0;
       }
+      __syncwarp();
+      if ((t & 31) == 0) tc::mbar_arrive(&vfull[b]);
+      prefetch_l2(j + 2, j);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0 && nch > 0) {
-      const uint32_t q_u = tc::smem_u32(qs);
       bool ok = tc::mbar_wait(qfull, 0, abort_flag);
       tc::fence_proxy_async_smem();
+      tc::tc_fence_after();  // Q's TMEM part was stored by the softmax warps
       // Two event streams, served as they become ready: S(j) = Q K(j)^T once
       // chunk j has landed and its score buffer is free, and P V(i) once P(i)
       // is written.  P V(i) goes out as soon as it can (not after S(i+1)), so
@@ -442,7 +513,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
           const uint64_t pa0 = tc::desc_sw128(p_u), vb0 = desc_sw128_mn(kv_u, kBoxBytes);
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            const uint32_t d = tmem + (static_cast<uint32_t>(16 * c) << 16);  // dims 256c.. at lane offset 16c
+            const uint32_t d = tmem + kLaneHi + 256u * c;  // O dims 256c.. at columns 256c..
 #pragma unroll
             for (int kk = 0; kk < kChunk / 16; ++kk)
               tc::mma_f16(d, pa0 + static_cast<uint64_t>((kk * 32) >> 4),
@@ -454,25 +525,29 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
           ++next_pv;
           progressed = true;
         }
+        // S(j) also waits until the softmax has read S(j-1) (one S buffer) and
+        // finished any rescale of O, which rewrites the Q and S lanes as well:
+        // no MMA may touch TMEM meanwhile.
         if (next_s < nch && next_s <= next_pv + 1) {
           const int j = next_s;
-          const int b = j % kNBuf, sb = j & 1;
+          const int b = j % kNBuf;
           if (tc::mbar_test(&kvfull[b], static_cast<uint32_t>((j / kNBuf) & 1)) &&
-              tc::mbar_test(&sempty[sb], static_cast<uint32_t>(((j >> 1) & 1) ^ 1))) {
+              (j == 0 || tc::mbar_test(rdone, static_cast<uint32_t>((j - 1) & 1)))) {
             tc::fence_proxy_async_smem();
             tc::tc_fence_after();
-            const uint32_t d = tmem + kColS + sb * kChunk;
+            const uint32_t d = tmem + kColS;
             // descriptors of the 36 K-steps differ only in the start-address field
             // (addresses stay below 256 KB, so the 14-bit field never carries)
-            const uint64_t a0 = tc::desc_sw128(q_u), b0 = tc::desc_sw128(tc::smem_u32(kvs + b * kKvBytes));
+            const uint64_t b0 = tc::desc_sw128(tc::smem_u32(kvs + b * kKvBytes));
+            // Q from TMEM, 16 dims = 8 columns per K-step
 #pragma unroll
             for (int blk = 0; blk < kBoxes; ++blk) {
 #pragma unroll
               for (int k = 0; k < 4; ++k)
-                tc::mma_f16(d, a0 + static_cast<uint64_t>((blk * kQBlock + k * 32) >> 4),
-                            b0 + static_cast<uint64_t>((blk * kBoxBytes + k * 32) >> 4), kIdescQK, (blk | k) != 0);
+                mma_f16_ta(d, tmem + kColQ + static_cast<uint32_t>((blk * 4 + k) * 8),
+                           b0 + static_cast<uint64_t>((blk * kBoxBytes + k * 32) >> 4), kIdescQK, (blk | k) != 0);
             }
-            tc::mma_commit(&sfull[sb]);
+            tc::mma_commit(sfull);
             ++next_s;
             progressed = true;
           }
@@ -500,54 +575,61 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     // ---------------------------------------------------------------- softmax
     const int quarter = warp & 3;                       // TMEM lanes 32q .. 32q+31
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const bool srow = lane < 16;                        // lanes holding a score row
+    const bool srow = lane < 16;                        // lanes holding a score row; lanes 16-31 hold O rows
     const int head_local = quarter * 16 + (lane & 15);  // 0..63
+    const int sl = lane & 15;                           // the score lane of this lane's head
+    // Q (576 dims) of the heads of this quarter into TMEM lanes 0-15, columns
+    // 0-287 (lanes 16-31 of those columns, O's, get zeros: the first P V
+    // overwrites them)
+    {
+      const uint4* qsrc = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint8_t*>(a.q) +
+          ((static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + head_local) * kD) * 2);
+#pragma unroll 1
+      for (int g = 0; g < kBoxes; g += 3) {  // 64 dims = 32 columns per group, three groups of loads in flight
+        uint4 x[24];
+#pragma unroll
+        for (int i = 0; i < 24; ++i) x[i] = lane < 16 ? __ldg(qsrc + g * 8 + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int gg = 0; gg < 3; ++gg) {
+          uint32_t v[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[4 * i] = x[gg * 8 + i].x; v[4 * i + 1] = x[gg * 8 + i].y;
+            v[4 * i + 2] = x[gg * 8 + i].z; v[4 * i + 3] = x[gg * 8 + i].w;
+          }
+          tmem_st32u(tmem + lane_base + kColQ + (g + gg) * 32, v);
+        }
+      }
+      tmem_wait_st();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(qfull);
+      // the rest of the first part of the row table (see the producer)
+      const int n_ent = j1 - j0;
+      const int first_hi = n_ent < kRowTab ? n_ent : kRowTab;
+      if (first_hi > 4 * kChunk)
+        fill_rows(a, ad, rc, r, j0, j1, 0, 4 * kChunk, first_hi, threadIdx.x - (kWarpMma + 1) * 32, 128, half == 0,
+                  rtab);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(tfull);
+    }
     const float c2 = a.scale * kLog2e;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
-    // validity of the chunk's rows (lane and lane + 32), looked up one chunk ahead
-    // Validity of this lane's two rows of each chunk (entries lane and lane+32),
-    // in the same three steps as the producer's lookups, one chunk apart:
-    // list entries two chunks ahead, block-table entries one ahead, so no
-    // load is read in the iteration that issues it.
-    auto jl_of = [&](int jj, int (&jl)[2]) {
-      jl[0] = jj < nch ? j0 + jj * kChunk + lane : j1;
-      jl[1] = jj < nch ? j0 + jj * kChunk + 32 + lane : j1;
-    };
-    int32_t pA[2], bA[2], pB[2];  // chunk j: entries + block entries; chunk j+1: entries
-    {
-      int jl[2];
-      jl_of(0, jl);
-      ent_pos<2>(a, rc, r, jl, j1, pA);
-      jl_of(1, jl);
-      ent_pos<2>(a, rc, r, jl, j1, pB);
-      ent_blk<2>(ad, rc, pA, bA);
-    }
     for (int j = 0; j < nch; ++j) {
-      const int sb = j & 1;
-      int64_t rr[2];
-      ent_rows<2>(a, ad, rc, r, pA, bA, false, rr);
-      const uint32_t mlo = __ballot_sync(0xffffffffu, rr[0] >= 0), mhi = __ballot_sync(0xffffffffu, rr[1] >= 0);
-      {
-        int32_t bB[2], pC[2];
-        int jl[2];
-        ent_blk<2>(ad, rc, pB, bB);  // chunk j+1
-        jl_of(j + 2, jl);
-        ent_pos<2>(a, rc, r, jl, j1, pC);  // chunk j+2
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          pA[m] = pB[m];
-          bA[m] = bB[m];
-          pB[m] = pC[m];
-        }
-      }
-      if (!tc::mbar_wait(&sfull[sb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      // validity of the chunk's rows lane and lane + 32, from the producer
+      const int b = j % kNBuf;
+      if (!tc::mbar_wait(&vfull[b], (j / kNBuf) & 1, abort_flag)) { ok = false; break; }
+      const uint32_t mlo = __ballot_sync(0xffffffffu, vrow[b * kChunk + lane] != 0);
+      const uint32_t mhi = __ballot_sync(0xffffffffu, vrow[b * kChunk + 32 + lane] != 0);
+      if (!tc::mbar_wait(sfull, j & 1, abort_flag)) { ok = false; break; }
       tc::tc_fence_after();
       float s[64];
       {
         float t0[32], t1[32];
-        tc::tmem_ld32(tmem + lane_base + kColS + sb * kChunk, t0);
-        tc::tmem_ld32(tmem + lane_base + kColS + sb * kChunk + 32, t1);
+        tc::tmem_ld32(tmem + lane_base + kColS, t0);       // lanes 0-15: S rows
+        tc::tmem_ld32(tmem + lane_base + kColS + 32, t1);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -555,9 +637,6 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
           s[32 + i] = t1[i];
         }
       }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sempty[sb]);
       float mx = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
@@ -568,18 +647,22 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       const float m_new = fmaxf(m_run, mx);
       const bool need = srow && (j > 0) && (m_new > m_run + kRescaleLog2);
       if (__any_sync(0xffffffffu, need)) {
-        // a rescale touches O: P V of chunk j-1 must have finished
+        // a rescale touches O: P V of chunk j-1 must have finished.  The 32-lane
+        // accesses also cover lanes 0-15 (Q, S), whose bits are written back
+        // untouched; no MMA runs meanwhile (S(j+1) waits for rdone).
         if (!tc::mbar_wait(pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
         const float alpha_own = need ? ex2(m_run - m_new) : 1.f;
-        const float alpha = __shfl_sync(0xffffffffu, alpha_own, lane & 15);
+        const float alpha = __shfl_sync(0xffffffffu, alpha_own, sl);
         tc::tc_fence_after();
 #pragma unroll 1
-        for (int cb = 0; cb < 8; ++cb) {
+        for (int cb = 0; cb < 16; ++cb) {
           float v[32];
           tc::tmem_ld32(tmem + lane_base + cb * 32, v);
           tc::tmem_wait_ld();
+          if (!srow) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;
+            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+          }
           tmem_st32(tmem + lane_base + cb * 32, v);
         }
         tmem_wait_st();
@@ -588,6 +671,10 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
           m_run = m_new;
         }
       }
+      // S(j) has been read and O rescaled: S(j+1) may be computed
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(rdone);
       if (j == 0) m_run = m_new;
       // probabilities (base 2): masked entries are -inf and give 2^-inf = 0; a
       // head with no valid entry yet (m_run = -inf) gives 0 everywhere.  P is
@@ -627,15 +714,15 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     bool fin = ok;
     if (ok && nch > 1) fin = tc::mbar_wait(pvdone, (nch - 2) & 1, abort_flag);
     if (fin && nch > 0) fin = tc::mbar_wait(pvdone, (nch - 1) & 1, abort_flag);
-    const float l_h = __shfl_sync(0xffffffffu, l, lane & 15);
-    const float m_h = __shfl_sync(0xffffffffu, m_run, lane & 15);
+    const float l_h = __shfl_sync(0xffffffffu, l, sl);
+    const float m_h = __shfl_sync(0xffffffffu, m_run, sl);
     const float inv = l_h > 0.f ? 1.f / l_h : 0.f;
     const float lse = l_h > 0.f ? (m_h + log2f(l_h)) * kLn2 : -INFINITY;
     const int h = half * kHeadsCta + head_local;
-    const int dim0 = lane < 16 ? 0 : 256;
     if (fin) tc::tc_fence_after();
+    // lanes 16-31 hold the O rows: dims 32 cb .. 32 cb + 31 in columns 32 cb ..
 #pragma unroll 1
-    for (int cb = 0; cb < 8; ++cb) {
+    for (int cb = 0; cb < 16; ++cb) {
       float v[32];
       if (fin && nch > 0) {
         tc::tmem_ld32(tmem + lane_base + cb * 32, v);
@@ -644,18 +731,19 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0.f;
       }
-      if (P.nsplit == 1) {
+      if (srow) {
+        // lanes 0-15 hold Q and S here
+      } else if (P.nsplit == 1) {
         store_bf16x32(reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<int64_t>(r) * kHeadsAll + h) * kDv +
-                          dim0 + cb * 32, v, inv);
+                          cb * 32, v, inv);
       } else {
         // Staged in the idle chunk buffers as [64 heads][512], the 16-byte
         // pieces of each 128-byte segment rotated by (head & 7) so that the
         // warp's rows spread over the banks; written out coalesced below.
         float* stg = reinterpret_cast<float*>(kvs);
-        const int seg = (dim0 + cb * 32) >> 5;
 #pragma unroll
         for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<float4*>(stg + head_local * kDv + seg * 32 + ((u ^ (head_local & 7)) << 2)) =
+          *reinterpret_cast<float4*>(stg + head_local * kDv + cb * 32 + ((u ^ (head_local & 7)) << 2)) =
               make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
       }
     }
@@ -747,7 +835,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
   tc::tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (uint64_t* b = bars; b <= done; ++b) tc::mbar_inval(b);
+    for (uint64_t* b = bars; b <= tfull; ++b) tc::mbar_inval(b);
   }
   __syncthreads();
 }
