@@ -174,8 +174,10 @@ TopkArgs topk_args(const float* scores, int64_t ld, int32_t rows, const int32_t*
 }
 
 lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
-                   int32_t k, int32_t* idx, void* ws, void* inner_ws, cudaStream_t s, bool hist_ready = false) {
-  const TopkArgs a = topk_args(scores, ld, rows, valid_len, n_cols, k, idx, ws, inner_ws, hist_ready);
+                   int32_t k, int32_t* idx, void* ws, void* inner_ws, cudaStream_t s, bool hist_ready = false,
+                   bool pdl = false) {
+  TopkArgs a = topk_args(scores, ld, rows, valid_len, n_cols, k, idx, ws, inner_ws, hist_ready);
+  a.pdl = pdl;
   return cuda_status(launch_topk(a, s));
 }
 
@@ -203,8 +205,11 @@ AttnArgs attn_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, const in
 
 lsa_status do_attn(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq, const void* q,
                    const int32_t* idx, void* out, float* lse, void* ws, void* inner_ws, size_t inner_bytes,
-                   cudaStream_t s) {
-  const AttnArgs a = attn_args(d, c, rows, row_seq, q, idx, out, lse, ws, inner_ws, inner_bytes);
+                   cudaStream_t s, bool pdl = false) {
+  AttnArgs a = attn_args(d, c, rows, row_seq, q, idx, out, lse, ws, inner_ws, inner_bytes);
+  // in a decode step the kernel before is the step's top-k, which does not write q
+  a.pdl = pdl;
+  a.q_early = pdl;
   if (rows == 0) return LSA_OK;
   if (!force_simt() && attn_tc_supported(a)) return cuda_status(launch_attn_tc(a, s));
   return cuda_status(launch_attn_simt(a, s));
@@ -331,10 +336,13 @@ static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const 
   st = do_scores(d, c, B, nullptr, nullptr, q_idx, w, scores, ld, ws, inner, inner_bytes, s, hist12, &hist_done);
   if (st != LSA_OK) return st;
   if (!mark(1)) return LSA_ERR_CUDA;
-  st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, s, hist_done);
+  // The top-k and the attention are launched as programmatic dependents of the
+  // kernel before them: their CTAs may be scheduled while it finishes, and
+  // they wait for it (griddepcontrol.wait) before reading what it wrote.
+  st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, s, hist_done, true);
   if (st != LSA_OK) return st;
   if (!mark(2)) return LSA_ERR_CUDA;
-  st = do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s);
+  st = do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s, true);
   if (st != LSA_OK) return st;
   if (!mark(3)) return LSA_ERR_CUDA;
   return LSA_OK;
@@ -370,9 +378,10 @@ int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32
   const bool simt = force_simt();
   int scan = 1;
   int attn = 0;
+  bool tc_scan = false;
   if (op != LSA_OP_TOPK) {
-    if (!simt && scores_tc_shape_ok(d->idx_key_dtype, d->act_dtype, d->n_idx_heads, d->idx_dim, d->block_size))
-      scan = scores_tc_launches(causal != 0);
+    tc_scan = !simt && scores_tc_shape_ok(d->idx_key_dtype, d->act_dtype, d->n_idx_heads, d->idx_dim, d->block_size);
+    if (tc_scan) scan = scores_tc_launches(causal != 0);
     if (!simt && attn_tc_shape_ok(d->act_dtype, d->n_heads, d->qk_dim, d->v_dim, d->block_size))
       attn = attn_tc_launches(rows, d->n_heads, d->top_k);
     else
@@ -382,13 +391,18 @@ int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32
     case LSA_OP_SCORES: return scan;
     case LSA_OP_TOPK: return topk_launches(max_len);
     case LSA_OP_ATTN: return attn;
-    case LSA_OP_DECODE_STEP: return scan + topk_launches(max_len) + attn;
+    case LSA_OP_DECODE_STEP: {
+      // the tensor-core scan of a decode step also builds the top-k's first histogram
+      const int topk = topk_launches(max_len) - (tc_scan && causal == 0 && topk_v2_ok(max_len) ? 1 : 0);
+      return scan + topk + attn;
+    }
     case LSA_OP_DECODE_STEP_FUSED: {
       const bool fused = !simt && causal == 0 && topk_v2_ok(max_len) &&
                          scores_tc_shape_ok(d->idx_key_dtype, d->act_dtype, d->n_idx_heads, d->idx_dim,
                                             d->block_size) &&
                          attn_tc_shape_ok(d->act_dtype, d->n_heads, d->qk_dim, d->v_dim, d->block_size);
-      return fused ? 1 : scan + topk_launches(max_len) + attn;
+      const int topk = topk_launches(max_len) - (tc_scan && causal == 0 && topk_v2_ok(max_len) ? 1 : 0);
+      return fused ? 1 : scan + topk + attn;
     }
     default: return -1;
   }

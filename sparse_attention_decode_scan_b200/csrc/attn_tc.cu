@@ -33,6 +33,41 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Clusters of `n` attention CTAs the device keeps resident at once (queried
+// once per n; 0 when clusters of that size are refused).  The cluster merge is
+// used only when all of a launch's clusters fit in one wave, as the split plan
+// assumes.
+int resident_clusters(int n) {
+  static int cached[17] = {-1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1};
+  if (n < 2 || n > 16) return 0;
+  if (cached[n] >= 0) return cached[n];
+  cached[n] = 0;
+  if (cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
+      (n > 8 && cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(n), 1, 1);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(n);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int c = 0;
+  if (cudaOccupancyMaxActiveClusters(&c, k_attn_tc, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    c = 0;
+  }
+  cached[n] = c;
+  return c;
+}
+
 size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
 }  // namespace
@@ -80,10 +115,37 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
     attr = true;
   }
   const dim3 grid(P.nsplit, 2, a.rows);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr_c[2];
+  attr_c[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_c[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr_c;
   if (P.nsplit == 1) {
     P.merge = kMergeSeparate;  // nothing to merge
-    k_attn_tc<<<grid, kThreads, kSmemBytes, s>>>(P);
-    return cudaGetLastError();
+    cfg.attrs = attr_c + 1;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_attn_tc, P);
+  }
+  cfg.numAttrs = 1;
+  // The split CTAs of a (row, half) as one thread-block cluster merge through
+  // distributed shared memory; the hardware schedules a cluster's CTAs
+  // together, so no counters, global partials or cooperative launch are needed.
+  if (resident_clusters(P.nsplit) >= 2 * a.rows) {
+    P.merge = kMergeCluster;
+    attr_c[0].id = cudaLaunchAttributeClusterDimension;
+    attr_c[0].val.clusterDim.x = static_cast<unsigned>(P.nsplit);
+    attr_c[0].val.clusterDim.y = 1;
+    attr_c[0].val.clusterDim.z = 1;
+    cfg.numAttrs = a.pdl ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_attn_tc, P);
+    cfg.numAttrs = 1;
+    if (e == cudaSuccess) return cudaSuccess;
+    (void)cudaGetLastError();  // refused: the merge below
   }
   cudaError_t e = cudaMemsetAsync(P.counters, 0, static_cast<size_t>(a.rows) * 2 * sizeof(int), s);
   if (e != cudaSuccess) return e;
@@ -91,17 +153,8 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   // a cooperative launch guarantees that or refuses.  Refused (fewer SMs than
   // the one-wave plan assumes), the partials are merged by a second launch.
   P.merge = kMergeInKernel;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr_c[1];
   attr_c[0].id = cudaLaunchAttributeCooperative;
   attr_c[0].val.cooperative = 1;
-  cfg.attrs = attr_c;
-  cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, k_attn_tc, P);
   if (e == cudaSuccess) return cudaSuccess;
   if (e != cudaErrorCooperativeLaunchTooLarge) return e;

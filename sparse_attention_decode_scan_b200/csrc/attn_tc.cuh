@@ -9,27 +9,26 @@
 // page: sparsity saves bytes read, the cache itself stays whole).
 //
 // Work: one CTA per (query row, half of the heads, split of the index list).
-// 64 heads make the MMA's M side (M = 64), so the fp32 output accumulator
-// O[64 x 512] takes half of the TMEM lanes: dims 0-255 at lane offset 0 and
-// dims 256-511 at lane offset 16, columns 0-255; the two score buffers
-// S[64 x 64] sit at lane offset 0, columns 256-383.  Each softmax warp then
-// holds, for its 16 heads, the scores in lanes 0-15 and both output halves in
-// lanes 0-31, so a rescale touches only output columns.
-//   warps 0-3  producer: cp.async gathers of 64 selected rows per chunk into the
-//              128-byte-swizzled operand layout (two chunk buffers); the rows of
-//              chunk j+2 are looked up and prefetched into L2 while chunk j is
-//              gathered, so the gathers read L2, not HBM
-//   warp 4     MMA issuer: S = Q K^T (36 x M64N64K16), O += P V (8 x M64N256K16),
-//              V read MN-major from the same tile as K
-//   warps 5-8  online softmax (base 2, lazy rescale when the max grows by > 8),
-//              P[64 heads x 64 rows] written over the chunk's rope block (dims
-//              512-575, dead once S is computed), so P is double-buffered with
-//              the chunks and the softmax of chunk j+1 overlaps P V of chunk j
+// 64 heads make the MMA's M side (M = 64), which uses lanes 0-15 or 16-31 of
+// each 32-lane TMEM quarter: the query Q[64 x 576] (the score MMA's A operand,
+// read from TMEM) and the scores S[64 x 64] sit on lanes 0-15, the fp32 output
+// accumulator O[64 x 512] on lanes 16-31.
+//   warps 0-3  producer: resolves the KV rows of the split's list entries into
+//              a shared-memory table before the first gather, then gathers 64
+//              rows per chunk with cp.async into the 128-byte-swizzled operand
+//              layout (three chunk buffers; the chunk two ahead is prefetched
+//              into L2) and publishes which rows exist
+//   warp 4     MMA issuer: S = Q K^T (36 x M64N64K16, A from TMEM), O += P V
+//              (8 x M64N256K16, V read MN-major from the same tile as K)
+//   warps 5-8  load Q into TMEM, then the online softmax (base 2, lazy rescale
+//              when the max grows by > 8): P[64 heads x 64 rows] is written
+//              over the chunk's rope block (dims 512-575, dead once S is
+//              computed), so P is buffered with the chunks
 // (Below N = 64 an MMA costs as much as at N = 64 on this part, so 64-row
 // chunks halve the score MMAs per row compared with 32-row chunks.)
 // With several splits per row, each CTA writes a normalised partial and its
-// lse; the last CTA of a (row, half) to finish merges them with all of its
-// threads (global counter, no waiting), so no separate merge launch is needed.
+// lse; the split CTAs of a (row, half) then meet (co-resident by a cooperative
+// launch) and each merges one slice, or a separate merge launch follows.
 #include <math.h>
 
 #include "common.cuh"
@@ -78,6 +77,7 @@ static_assert(kSmemBytes <= 232448, "shared memory");
 // How the split partials of a (row, 64 heads) are combined.
 constexpr int kMergeSeparate = 0;  // partials only; a separate merge launch follows
 constexpr int kMergeInKernel = 1;  // the split CTAs meet, then each merges a slice
+constexpr int kMergeCluster = 2;   // the split CTAs of a (row, half) form a cluster and merge through DSMEM
                                    // (needs every CTA resident at once)
 
 struct TcAttnParams {
@@ -86,8 +86,8 @@ struct TcAttnParams {
   int split_len;   // multiple of kChunk
   float* part_o;   // [rows][nsplit][128][512]
   float* part_lse; // [rows][nsplit][128]
-  int* counters;   // [rows][2], zeroed before the launch
-  int merge;       // kMergeSeparate or kMergeInKernel
+  int* counters;   // [rows][2], zeroed before the launch (kMergeInKernel)
+  int merge;       // kMergeSeparate, kMergeInKernel or kMergeCluster
 };
 
 // MN-major operand in the 128-byte swizzle layout: 64-element MN blocks `lbo`
@@ -177,92 +177,49 @@ __device__ __forceinline__ RowCtx row_ctx(const AttnArgs& a, int r) {
   return c;
 }
 
-// Stored rows of list entries j[0..N) of row r (-1: padding, out of range or
-// bad block), in three steps that a caller may spread out so that each step's
-// loads have time to land: the positions (list loads), the block-table
-// entries of a paged cache (loads indexed by the positions), the rows.
-template <int N>
-__device__ __forceinline__ void ent_pos(const AttnArgs& a, const RowCtx& rc, int r, const int (&j)[N], int j1,
-                                        int32_t (&pos)[N]) {
-#pragma unroll
-  for (int m = 0; m < N; ++m)
-    // L2-coherent load: in the fused step the selection is written earlier in the same launch
-    pos[m] = (j[m] < j1 && rc.ok) ? __ldcg(a.idx + static_cast<int64_t>(r) * a.k + j[m]) : -1;
-}
-
-template <int N>
-__device__ __forceinline__ void ent_blk(const CacheAddr& ad, const RowCtx& rc, const int32_t (&pos)[N],
-                                        int32_t (&blk)[N]) {
-#pragma unroll
-  for (int m = 0; m < N; ++m) {
-    blk[m] = -1;
-    if (ad.block_size > 0) {
-      const int64_t lb = pos[m] / ad.block_size;
-      if (pos[m] >= 0 && pos[m] < rc.L && lb < ad.max_blocks)
-        blk[m] = __ldg(ad.block_table + static_cast<int64_t>(rc.b) * ad.max_blocks + lb);
-    }
-  }
-}
-
-// Block-table entries from the row's table cached in shared memory (sbt), or
-// from global memory when it is not cached.
-template <int N>
-__device__ __forceinline__ void ent_blk_s(const CacheAddr& ad, const RowCtx& rc, const int32_t* sbt, bool cached,
-                                          const int32_t (&pos)[N], int32_t (&blk)[N]) {
-  if (!cached) {
-    ent_blk<N>(ad, rc, pos, blk);
-    return;
-  }
-#pragma unroll
-  for (int m = 0; m < N; ++m) {
-    const int64_t lb = pos[m] / ad.block_size;
-    blk[m] = (pos[m] >= 0 && pos[m] < rc.L && lb < ad.max_blocks) ? sbt[lb] : -1;
-  }
-}
-
-template <int N>
-__device__ __forceinline__ void ent_rows(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r,
-                                         const int32_t (&pos)[N], const int32_t (&blk)[N], bool report,
-                                         int64_t (&out)[N]) {
-#pragma unroll
-  for (int m = 0; m < N; ++m) {
-    if (ad.block_size == 0)
-      out[m] = (pos[m] >= 0 && pos[m] < rc.L) ? static_cast<int64_t>(rc.b) * ad.max_len + pos[m] : -1;
-    else
-      out[m] = (blk[m] >= 0 && blk[m] < ad.n_blocks)
-                   ? static_cast<int64_t>(blk[m]) * ad.block_size + (pos[m] % ad.block_size) : -1;
-    if (report && pos[m] >= 0 && out[m] < 0) record_error(a.status, LSA_ERR_BOUNDS, r, pos[m]);
-  }
-}
-
-// The three steps back to back.
-template <int N>
-__device__ __forceinline__ void entry_rows(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r,
-                                           const int (&j)[N], int j1, bool report, int64_t (&out)[N]) {
-  int32_t pos[N], blk[N];
-  ent_pos<N>(a, rc, r, j, j1, pos);
-  ent_blk<N>(ad, rc, pos, blk);
-  ent_rows<N>(a, ad, rc, r, pos, blk, report, out);
-}
-
-// KV rows of the list entries at offsets [lo, hi) from j0 (at most kRowTab
-// past the table's base offset `base`) into rtab, by n threads (tid): per
-// pass 8 list loads in flight, then their 8 block-table loads.
-__device__ __forceinline__ void fill_rows(const AttnArgs& a, const CacheAddr& ad, const RowCtx& rc, int r, int j0,
-                                          int j1, int base, int lo, int hi, int tid, int n, bool report,
-                                          int32_t* rtab) {
+// KV rows of the list entries at offsets [lo, hi) of the split (list = the
+// row's selection from the split's first entry) into rtab[e - base], by n
+// threads (tid): per pass 8 list loads in flight, then their 8 block-table
+// loads.  -1 marks padding, positions out of range and bad blocks (reported
+// when `report`).  Out of line: it runs once per table part, and one compact
+// copy is cheaper to fetch than inlined ones.
+static __device__ __noinline__ void fill_rows(const int32_t* list, const int32_t* bt, int32_t max_blocks, int32_t block_size,
+                                              int64_t n_blocks, int64_t row_base, int64_t L, bool ok, DevStatus* status,
+                                              int r, int base, int lo, int hi, int tid, int n, bool report,
+                                              int32_t* rtab) {
+  const bool paged = block_size > 0;
+  const DivU32 bs = make_divu32(paged ? static_cast<uint32_t>(block_size) : 1u);
   for (int e = lo + tid; e < hi; e += 8 * n) {
-    int jl[8];
+    int32_t pos[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) jl[u] = e + u * n < hi ? j0 + e + u * n : j1;
-    int32_t pos[8], blk[8];
-    int64_t rows[8];
-    ent_pos<8>(a, rc, r, jl, j1, pos);
-    ent_blk<8>(ad, rc, pos, blk);
-    ent_rows<8>(a, ad, rc, r, pos, blk, report, rows);
+    for (int u = 0; u < 8; ++u) {
+      const int eu = e + u * n;
+      // L2-coherent load: in the fused step the selection is written earlier in the same launch
+      pos[u] = (eu < hi && ok) ? __ldcg(list + eu) : -1;
+    }
+    int32_t blk[8];
+    uint32_t lb[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (e + u * n < hi) rtab[e + u * n - base] = static_cast<int32_t>(rows[u]);
+    for (int u = 0; u < 8; ++u) {
+      blk[u] = -1;
+      lb[u] = 0;
+      if (paged && pos[u] >= 0 && pos[u] < L) {
+        lb[u] = divu32(bs, static_cast<uint32_t>(pos[u]));
+        if (lb[u] < static_cast<uint32_t>(max_blocks)) blk[u] = __ldg(bt + lb[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int eu = e + u * n;
+      int64_t row = -1;
+      if (!paged) {
+        if (pos[u] >= 0 && pos[u] < L) row = row_base + pos[u];
+      } else if (blk[u] >= 0 && blk[u] < n_blocks) {
+        row = static_cast<int64_t>(blk[u]) * block_size + (pos[u] - static_cast<int32_t>(lb[u] * bs.d));
+      }
+      if (report && pos[u] >= 0 && row < 0) record_error(status, LSA_ERR_BOUNDS, r, pos[u]);
+      if (eu < hi) rtab[eu - base] = static_cast<int32_t>(row);
+    }
   }
 }
 
@@ -354,10 +311,14 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
   uint64_t* pvdone = pfull + 1;
   uint64_t* done = pvdone + 1;
   uint64_t* vfull = done + 1;             // [kNBuf] the chunk's row validity is written
-  uint64_t* tfull = vfull + kNBuf;        // the softmax warps resolved the table's tail
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tfull + 1);
+  uint64_t* mready = vfull + kNBuf;       // cluster merge: every split CTA has staged its partial
+  uint64_t* mdone = mready + 1;           // cluster merge: every split CTA has read the others' partials
+  uint64_t* bars_end = mdone + 1;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars_end);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
   uint8_t* vrow = reinterpret_cast<uint8_t*>(last_flag + 1);  // [kNBuf][kChunk]: 1 = the row has a KV row
+  float* slse = reinterpret_cast<float*>(vrow + kNBuf * kChunk);  // [64] cluster merge: the partial's lse
+  const bool cmerge = P.nsplit > 1 && P.merge == kMergeCluster;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j0 = split * P.split_len;
@@ -376,11 +337,13 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     tc::mbar_init(pvdone, 1);
     tc::mbar_init(done, 1);
     for (int i = 0; i < kNBuf; ++i) tc::mbar_init(&vfull[i], 4);  // one arrival per producer warp
-    tc::mbar_init(tfull, 4);                                        // one arrival per softmax warp
+    tc::mbar_init(mready, cmerge ? P.nsplit : 1);                   // one arrival per split CTA
+    tc::mbar_init(mdone, cmerge ? P.nsplit : 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
   __syncthreads();
+  if (cmerge) tc::cluster_arrive_relaxed();  // waited for before the first remote arrival
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const RowCtx rc = row_ctx(a, r);
@@ -392,18 +355,19 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     const int t = threadIdx.x;
     const int sub = t & 7;         // 16-byte column chunk within each 128-byte block
     const int rbase = t >> 3;      // 0..15
-    const bool report = sub == 0 && half == 0;
     // The KV rows of the split's list entries are resolved ahead into a table
     // in shared memory (up to kRowTab entries at a time), so the gather loop
-    // issues no dependent global load of its own.  The first kHeadRows rows are
-    // resolved here; the softmax warps, idle until the first scores, resolve the
-    // rest of the first kRowTab and signal tfull.
-    constexpr int kHeadRows = 4 * kChunk;
+    // issues no dependent global load of its own.  The first part is resolved
+    // before the first gather: its two dependent rounds of loads (list, then
+    // block table) cost about the same for 64 entries as for 2048, and HBM is
+    // still idle then.
     const int n_ent = j1 - j0;
-    const int first_hi = n_ent < kRowTab ? n_ent : kRowTab;
-    auto fill_table = [&](int e0) {  // a later part: entries [e0, e0 + kRowTab), all by the producer
+    const int32_t* bt = ad.block_size > 0 ? ad.block_table + static_cast<int64_t>(rc.b) * ad.max_blocks : nullptr;
+    auto fill_table = [&](int e0) {  // entries [e0, e0 + kRowTab)
       const int hi = n_ent - e0 < kRowTab ? n_ent : e0 + kRowTab;
-      fill_rows(a, ad, rc, r, j0, j1, e0, e0, hi, t, kProdThreads, half == 0, rtab);
+      fill_rows(a.idx + static_cast<int64_t>(r) * a.k + j0, bt, ad.max_blocks, ad.block_size, ad.n_blocks,
+                static_cast<int64_t>(rc.b) * ad.max_len, rc.L, rc.ok, a.status, r, e0, e0, hi, t, kProdThreads,
+                half == 0, rtab);
       asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");  // the producer warps
     };
     auto row_of = [&](int jj, int m) -> int64_t {  // chunk jj, this thread's m-th row
@@ -413,7 +377,6 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     auto prefetch_l2 = [&](int jj, int j_now) {
       // only chunks whose rows are in the table now
       if (sub != 0 || jj >= nch || (jj * kChunk) / kRowTab != (j_now * kChunk) / kRowTab) return;
-      if (jj * kChunk >= kHeadRows && j_now * kChunk < kHeadRows) return;  // the table's tail may not be there yet
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int64_t row = row_of(jj, m);
@@ -424,10 +387,8 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
                        : "memory");
       }
     };
-    (void)report;
-    fill_rows(a, ad, rc, r, j0, j1, 0, 0, first_hi < kHeadRows ? first_hi : kHeadRows, t, kProdThreads, half == 0,
-              rtab);
-    asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");  // the producer warps
+    tc::griddep_wait();  // launched early in a decode step: the selection is complete from here on
+    fill_table(0);
     prefetch_l2(0, 0);
     prefetch_l2(1, 0);
 #pragma unroll 1
@@ -439,15 +400,6 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
         fill_table(j * kChunk);
         prefetch_l2(j, j);
         prefetch_l2(j + 1, j);
-      }
-      if (j * kChunk == kHeadRows && first_hi > kHeadRows) {  // the rest of the first part, from the softmax warps
-        if (!tc::mbar_wait(tfull, 0, abort_flag)) {
-          if (t == 0) {
-            record_error(a.status, LSA_ERR_TIMEOUT, r, 14);
-            *abort_flag = 1;
-          }
-          break;
-        }
       }
       if (!tc::mbar_wait(&kvempty[b], ((j / kNBuf) & 1) ^ 1, abort_flag)) {
         if (t == 0) {
@@ -490,6 +442,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA issuer
+    tc::griddep_wait();
     if (lane == 0 && nch > 0) {
       bool ok = tc::mbar_wait(qfull, 0, abort_flag);
       tc::fence_proxy_async_smem();
@@ -580,7 +533,9 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     const int sl = lane & 15;                           // the score lane of this lane's head
     // Q (576 dims) of the heads of this quarter into TMEM lanes 0-15, columns
     // 0-287 (lanes 16-31 of those columns, O's, get zeros: the first P V
-    // overwrites them)
+    // overwrites them).  In a decode step q is an input of the step, so it is
+    // loaded while the top-k may still run.
+    if (!a.q_early) tc::griddep_wait();
     {
       const uint4* qsrc = reinterpret_cast<const uint4*>(
           reinterpret_cast<const uint8_t*>(a.q) +
@@ -605,15 +560,8 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qfull);
-      // the rest of the first part of the row table (see the producer)
-      const int n_ent = j1 - j0;
-      const int first_hi = n_ent < kRowTab ? n_ent : kRowTab;
-      if (first_hi > 4 * kChunk)
-        fill_rows(a, ad, rc, r, j0, j1, 0, 4 * kChunk, first_hi, threadIdx.x - (kWarpMma + 1) * 32, 128, half == 0,
-                  rtab);
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(tfull);
     }
+    if (a.q_early) tc::griddep_wait();
     const float c2 = a.scale * kLog2e;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
@@ -750,6 +698,8 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     if (lane < 16) {
       if (P.nsplit == 1) {
         if (a.lse) a.lse[static_cast<int64_t>(r) * kHeadsAll + h] = lse;
+      } else if (cmerge) {
+        slse[head_local] = lse;
       } else {
         P.part_lse[(static_cast<int64_t>(r) * P.nsplit + split) * kHeadsAll + h] = lse;
       }
@@ -759,7 +709,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
   // The CTA's partial O block [64 heads][512] is contiguous in part_o: every
   // thread copies 16-byte pieces from the staging area, consecutive threads to
   // consecutive addresses (full-line writes that drain quickly).
-  if (P.nsplit > 1) {
+  if (P.nsplit > 1 && !cmerge) {
     __syncthreads();
     const float4* stg4 = reinterpret_cast<const float4*>(kvs);
     float4* dst = reinterpret_cast<float4*>(
@@ -806,14 +756,23 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       float* wsm = reinterpret_cast<float*>(kvs);  // [nsplit][64] in the idle chunk buffer, nsplit <= 32
       const float* lse_p = P.part_lse + static_cast<int64_t>(r) * ns * kHeadsAll + half * kHeadsCta;
       const int hl0 = i0 / (kDv / 4), hl1 = i1 > i0 ? (i1 - 1) / (kDv / 4) + 1 : hl0;
-      // one warp per head, one lane per split (nsplit <= 32): all lse loads at once
-      for (int x = warp; x < hl1 - hl0; x += kThreads / 32) {
-        const int hl = hl0 + x;
-        const float lv = lane < ns ? __ldcg(lse_p + lane * kHeadsAll + hl) : -INFINITY;
-        float mx = lv;
+      // one warp per head, one lane per split (nsplit <= 32); a warp's heads'
+      // lse loads are all issued before the first is used
+      constexpr int kHeadsPerWarp = (kHeadsCta + kThreads / 32 - 1) / (kThreads / 32);
+      float lv[kHeadsPerWarp];
+#pragma unroll
+      for (int x = 0; x < kHeadsPerWarp; ++x) {
+        const int hl = hl0 + warp + x * (kThreads / 32);
+        lv[x] = (hl < hl1 && lane < ns) ? __ldcg(lse_p + lane * kHeadsAll + hl) : -INFINITY;
+      }
+#pragma unroll
+      for (int x = 0; x < kHeadsPerWarp; ++x) {
+        const int hl = hl0 + warp + x * (kThreads / 32);
+        if (hl >= hl1) break;
+        float mx = lv[x];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float e = (lane < ns && mx != -INFINITY) ? exp2f((lv - mx) * kLog2e) : 0.f;
+        const float e = (lane < ns && mx != -INFINITY) ? exp2f((lv[x] - mx) * kLog2e) : 0.f;
         float den = e;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
@@ -832,10 +791,131 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
         merge_slice<1, 16>(P, r, half, i0, i1, wsm);
     }
   }
+  // ---------------------------------------------------------------- cluster merge
+  // The split CTAs of a (row, half) are one cluster (CTA rank = split).  Each
+  // staged its normalised partial O [64 heads][512] (rotated pieces, as above)
+  // and lse in its own shared memory; once all have (remote arrivals on every
+  // CTA's mready), each merges its slice of the 64 heads x 128 groups of 4
+  // dims reading the partials through DSMEM, and keeps its shared memory until
+  // every CTA has finished reading (mdone).
+  if (cmerge) {
+    __syncthreads();
+    tc::cluster_wait();  // every CTA of the cluster has initialised its barriers
+    const int ns = P.nsplit;
+    if (threadIdx.x == 0) {
+      tc::fence_acq_rel_cluster();
+      const uint32_t mr = tc::smem_u32(mready);
+      for (int s2 = 0; s2 < ns; ++s2) tc::mbar_arrive_cluster(tc::cluster_map(mr, static_cast<uint32_t>(s2)));
+    }
+    if (tc::mbar_wait_cluster(mready, 0)) {
+      constexpr int kItems = kHeadsCta * (kDv / 4);
+      const int per = (kItems + ns - 1) / ns;
+      const int i0 = split * per;
+      const int i1 = i0 + per < kItems ? i0 + per : kItems;
+      // weights [nsplit][64] past the staged partial (which peers read)
+      float* wsm = reinterpret_cast<float*>(kvs + kHeadsCta * kDv * 4);
+      const int hl0 = i0 / (kDv / 4), hl1 = i1 > i0 ? (i1 - 1) / (kDv / 4) + 1 : hl0;
+      const uint32_t slse_u = tc::smem_u32(slse);
+      // one warp per head, one lane per split (nsplit <= 32); a warp's lse
+      // loads are all issued before the first is used
+      constexpr int kHeadsPerWarp = (kHeadsCta + kThreads / 32 - 1) / (kThreads / 32);
+      float lv[kHeadsPerWarp];
+      const uint32_t peer_lse = lane < ns ? tc::cluster_map(slse_u, static_cast<uint32_t>(lane)) : 0u;
+#pragma unroll
+      for (int x = 0; x < kHeadsPerWarp; ++x) {
+        const int hl = hl0 + warp + x * (kThreads / 32);
+        lv[x] = (hl < hl1 && lane < ns) ? tc::ld_cluster_f32(peer_lse + hl * 4) : -INFINITY;
+      }
+#pragma unroll
+      for (int x = 0; x < kHeadsPerWarp; ++x) {
+        const int hl = hl0 + warp + x * (kThreads / 32);
+        if (hl >= hl1) break;
+        float mx = lv[x];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float e = (lane < ns && mx != -INFINITY) ? exp2f((lv[x] - mx) * kLog2e) : 0.f;
+        float den = e;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        if (lane < ns) wsm[lane * kHeadsCta + hl] = e * inv;
+        // the slice holding a head's first group writes its lse
+        if (lane == 0 && a.lse && hl * (kDv / 4) >= i0)
+          a.lse[static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + hl] = den > 0.f ? mx + logf(den) : -INFINITY;
+      }
+      __syncthreads();
+      const uint32_t stg_u = tc::smem_u32(kvs);
+      constexpr int U = 8;  // groups per thread and pass, loads in flight together
+#pragma unroll 1
+      for (int it0 = i0 + threadIdx.x; it0 < i1; it0 += U * kThreads) {
+        float4 acc[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        uint32_t off[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int item = it0 + u * kThreads;
+          const int hl = item >> 7, c4 = item & 127;
+          off[u] = static_cast<uint32_t>(hl * (kDv / 4) + (c4 & ~7) + ((c4 & 7) ^ (hl & 7))) * 16u;
+        }
+        // two splits per step: 2U loads in flight; the splits are summed in ascending order
+#pragma unroll 1
+        for (int s2 = 0; s2 < ns; s2 += 2) {
+          // this CTA's own partial is read from its shared memory directly
+          const int s3 = s2 + 1 < ns ? s2 + 1 : s2;
+          const uint32_t pb0 = s2 == split ? stg_u : tc::cluster_map(stg_u, static_cast<uint32_t>(s2));
+          const uint32_t pb1 = s3 == split ? stg_u : tc::cluster_map(stg_u, static_cast<uint32_t>(s3));
+          float4 x0[U], x1[U];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const bool in = it0 + u * kThreads < i1;
+            x0[u] = !in ? make_float4(0.f, 0.f, 0.f, 0.f)
+                        : (s2 == split ? tc::ld_shared_f4(pb0 + off[u]) : tc::ld_cluster_f4(pb0 + off[u]));
+            x1[u] = !(in && s2 + 1 < ns) ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                         : (s3 == split ? tc::ld_shared_f4(pb1 + off[u]) : tc::ld_cluster_f4(pb1 + off[u]));
+          }
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int item = it0 + u * kThreads;
+            const int hl = (item < i1 ? item : i0) >> 7;
+            const float w0 = wsm[s2 * kHeadsCta + hl];
+            acc[u].x = fmaf(w0, x0[u].x, acc[u].x); acc[u].y = fmaf(w0, x0[u].y, acc[u].y);
+            acc[u].z = fmaf(w0, x0[u].z, acc[u].z); acc[u].w = fmaf(w0, x0[u].w, acc[u].w);
+            if (s2 + 1 < ns) {
+              const float w1 = wsm[(s2 + 1) * kHeadsCta + hl];
+              acc[u].x = fmaf(w1, x1[u].x, acc[u].x); acc[u].y = fmaf(w1, x1[u].y, acc[u].y);
+              acc[u].z = fmaf(w1, x1[u].z, acc[u].z); acc[u].w = fmaf(w1, x1[u].w, acc[u].w);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int item = it0 + u * kThreads;
+          if (item >= i1) continue;
+          const int hl = item >> 7, c4 = item & 127;
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[u].x, acc[u].y);
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[u].z, acc[u].w);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                    (static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + hl) * kDv + c4 * 4) = pk;
+        }
+      }
+    } else if (threadIdx.x == 0) {
+      record_error(a.status, LSA_ERR_TIMEOUT, r, 15);
+    }
+    __syncthreads();  // this CTA's reads of the others' partials have completed
+    if (threadIdx.x == 0) {
+      const uint32_t md = tc::smem_u32(mdone);
+      for (int s2 = 0; s2 < ns; ++s2) tc::mbar_arrive_cluster(tc::cluster_map(md, static_cast<uint32_t>(s2)));
+    }
+    if (!tc::mbar_wait_cluster(mdone, 0) && threadIdx.x == 0) record_error(a.status, LSA_ERR_TIMEOUT, r, 16);
+  }
   tc::tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (uint64_t* b = bars; b <= tfull; ++b) tc::mbar_inval(b);
+    for (uint64_t* b = bars; b < bars_end; ++b) tc::mbar_inval(b);
   }
   __syncthreads();
 }

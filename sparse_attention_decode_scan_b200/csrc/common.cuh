@@ -21,7 +21,10 @@ struct DevStatus {
   int32_t count;     // number of recorded errors
 };
 
-__device__ __forceinline__ void record_error(DevStatus* st, int code, int d0, int d1) {
+// Kept out of line: it is on error paths only, and inlining its atomics at
+// every call site would grow the kernels' code (cold code is fetched from
+// memory at each launch).
+static __device__ __noinline__ void record_error(DevStatus* st, int code, int d0, int d1) {
   if (st == nullptr) return;
   if (atomicCAS(&st->code, 0, code) == 0) {
     st->detail0 = d0;
@@ -29,6 +32,27 @@ __device__ __forceinline__ void record_error(DevStatus* st, int code, int d0, in
   }
   atomicAdd(&st->count, 1);
 }
+
+// Unsigned division by an invariant d >= 1 as a multiply-high, an add and a
+// shift (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994, the round-up multiplier m' = floor(2^(32+l)/d)+1
+// with l = ceil(log2 d), stored as m' - 2^32); exact for n < 2^31.
+struct DivU32 {
+  uint32_t d, m;
+  int l;
+};
+
+__host__ __device__ inline DivU32 make_divu32(uint32_t d) {
+  DivU32 v;
+  v.d = d;
+  int l = 0;
+  while ((1ull << l) < d) ++l;
+  v.l = l;
+  v.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+  return v;
+}
+
+__device__ __forceinline__ uint32_t divu32(const DivU32& v, uint32_t n) { return (__umulhi(n, v.m) + n) >> v.l; }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);

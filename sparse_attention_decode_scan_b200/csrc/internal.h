@@ -75,6 +75,7 @@ struct TopkArgs {
   void* ws;            // topk_ws_bytes bytes (256-aligned)
   DevStatus* status;
   bool hist_ready;     // the first histogram and list counters are already in ws
+  bool pdl = false;    // launched as a programmatic dependent of the kernel before it (decode step)
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 // The three-launch top-k applies (rows up to 2^19 entries); its first
@@ -105,6 +106,8 @@ struct AttnArgs {
   void* ws;
   size_t ws_bytes;
   DevStatus* status;
+  bool pdl = false;      // launched as a programmatic dependent of the kernel before it (decode step)
+  bool q_early = false;  // with pdl: q may be read before the kernel before it completes
 };
 size_t attn_simt_ws_bytes(int32_t rows, int32_t H, int32_t Dv, int32_t k);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);

@@ -396,6 +396,9 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   sbuf = reinterpret_cast<int64_t*>((reinterpret_cast<uintptr_t>(sbuf) + 7) & ~uintptr_t(7));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // a decode step's top-k may be scheduled onto SMs this launch frees (it
+  // waits for the scan to complete before reading anything)
+  tc::griddep_launch_dependents();
   // The epilogue reads a stage's key rows (paged cache) and scales (FP8); a
   // contiguous bf16 cache needs neither, and its stages free at MMA completion.
   const bool stage_meta = C::kFp8 || a.cache.block_size > 0;
@@ -486,6 +489,8 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
           rows[h] = r;
         }
       };
+      // the keys are streamed once per step: evict them from L2 first
+      const uint64_t l2_policy = tc::l2_evict_first_policy();
       Walker<QB> Wb;
       Wb.start(a, plan.r_first, plan.j_first);
       Look cur = look(Wb, 0);
@@ -520,8 +525,8 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
               for (int h = 0; h < 2; ++h) {
                 if (rows[h] < 0) continue;
                 for (int kb = 0; kb < C::kKBlocks; ++kb)
-                  tc::tma_load_2d(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * kBoxX,
-                                  static_cast<int32_t>(rows[h]), &full[s]);
+                  tc::tma_load_2d_hint(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * kBoxX,
+                                       static_cast<int32_t>(rows[h]), &full[s], l2_policy);
                 // the box's 64 scales, from the 16-byte aligned row at or below its first
                 if (C::kFp8)
                   tc::tma_load_1d(sscale + (2 * s + h) * kScaleSlot, &smap, static_cast<int32_t>(rows[h] & ~int64_t(3)),

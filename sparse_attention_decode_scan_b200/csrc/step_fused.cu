@@ -127,7 +127,7 @@ template <int KDT>
 size_t fused_smem(int64_t n_cols) {
   size_t b = scan::Cfg<KDT, 1>::kSmemBytes;
   if (static_cast<size_t>(attn::kSmemBytes) > b) b = attn::kSmemBytes;
-  const size_t t = 1024 + kScratchBytes + tk::tk_final_smem(n_cols);
+  const size_t t = 1024 + kScratchBytes + tk::tk_final_smem(n_cols, kSelThreads);
   return t > b ? t : b;
 }
 

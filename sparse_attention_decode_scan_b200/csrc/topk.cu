@@ -21,8 +21,11 @@
 
 #include <mutex>
 
+#include <string.h>
+
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 #include "topk_sel.cuh"
 
 namespace lsa {
@@ -309,7 +312,6 @@ using tk::kB1;
 using tk::kCandCap;
 using tk::TkLayout;
 using tk::tk_layout;
-constexpr int kFinT = 1024;  // threads of the per-row select CTA
 
 // Histogram of key bits [31:20] per row (when the scan did not build it).
 __global__ void __launch_bounds__(kT) k_tk_hist12(TopkArgs a, int64_t seg_len) {
@@ -333,15 +335,47 @@ __global__ void __launch_bounds__(kT) k_tk_hist12(TopkArgs a, int64_t seg_len) {
     if (h[i]) atomicAdd(dst + i, h[i]);
 }
 
-__global__ void __launch_bounds__(tk::kCollectThreads) k_tk_collect(TopkArgs a, int64_t seg_len) {
-  __shared__ tk::TkScratch S;
-  tk::tk_collect_cta<2>(a, seg_len, blockIdx.x, blockIdx.y, S);
-}
-
-__global__ void __launch_bounds__(kFinT) k_tk_final(TopkArgs a) {
+// Collect pass of segment blockIdx.x of row blockIdx.y; the row's last CTA to
+// finish its segment then selects the row's k (a grid-wide order is not
+// needed: each row waits only for its own segments, and no CTA waits at all).
+__global__ void __launch_bounds__(tk::kCollectThreads, 2) k_tk_rows(TopkArgs a, int64_t seg_len, int nseg) {
   extern __shared__ __align__(16) uint32_t fsm[];
   __shared__ tk::TkScratch S;
-  tk::tk_final_cta<kFinT, 3>(a, blockIdx.x, fsm, S);
+  __shared__ int s_last;
+  const int r = blockIdx.y;
+  tc::griddep_wait();  // launched early in a decode step: the scores are complete from here on
+  tc::griddep_launch_dependents();
+  tk::tk_collect_cta<2>(a, seg_len, blockIdx.x, r, S);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's bitmap words and candidates before its count
+    const uint32_t done = atomicAdd(tk::tk_layout(a.ws, a.rows, a.n_cols).row_done + r, 1u);
+    s_last = done == static_cast<uint32_t>(nseg - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();  // the other segments' writes, read through L2 by the select
+  tk::tk_final_cta<tk::kCollectThreads, 3>(a, r, fsm, S);
+}
+
+// SMs of the current device (the plan's CTA target).
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return kPlanSMs;
+  }
+  return n;
+}
+
+// Collect CTAs resident per SM with the select's shared memory (at most 2).
+int rows_ctas_per_sm(size_t smem) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_tk_rows, tk::kCollectThreads, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 1;
+  }
+  return n < 1 ? 1 : (n > 2 ? 2 : n);
 }
 
 }  // namespace
@@ -375,7 +409,7 @@ size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t) {
   return (b + 255) / 256 * 256;
 }
 
-int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 3 : 5; }
+int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 2 : 5; }
 
 // Segments of the collect pass: multiples of 8192 positions, about
 // `target_ctas` CTAs in total (two per SM for the standalone launch, where two
@@ -404,18 +438,26 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
       if (e != cudaSuccess) return e;
       k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
     }
-    const TopkPlan cp = topk_collect_plan(a.rows, a.n_cols, 2 * kPlanSMs);
-    k_tk_collect<<<dim3(static_cast<unsigned>(cp.nseg), static_cast<unsigned>(a.rows)), tk::kCollectThreads, 0, s>>>(
-        a, cp.seg_len);
-    const size_t smem = tk::tk_final_smem(a.n_cols);
+    const size_t smem = tk::tk_final_smem(a.n_cols, tk::kCollectThreads);
     static size_t smem_set = 0;
     if (smem > 48 * 1024 && smem > smem_set) {
-      e = cudaFuncSetAttribute(k_tk_final, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      e = cudaFuncSetAttribute(k_tk_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return e;
       smem_set = smem;
     }
-    k_tk_final<<<a.rows, kFinT, smem, s>>>(a);
-    return cudaGetLastError();
+    const TopkPlan cp = topk_collect_plan(a.rows, a.n_cols, rows_ctas_per_sm(smem) * device_sms());
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(cp.nseg), static_cast<unsigned>(a.rows));
+    cfg.blockDim = dim3(tk::kCollectThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_tk_rows, a, cp.seg_len, static_cast<int>(cp.nseg));
   }
   size_t hist_bytes = static_cast<size_t>(a.rows) * kHistStride * 4;
   cudaError_t e = cudaMemsetAsync(a.ws, 0, hist_bytes, s);

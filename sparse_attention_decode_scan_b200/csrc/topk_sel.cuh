@@ -26,20 +26,22 @@ constexpr int kCtrlInts = 64;            // control words of the fused step (gri
 __host__ __device__ inline size_t al256(size_t b) { return (b + 255) / 256 * 256; }
 
 // Workspace: [rows][4096] first-digit histograms | [rows] candidate counts |
-// control block (fused step: grid-barrier word, attention split counters) |
+// control block (fused step: grid-barrier word, attention split counters;
+// per-row counts of finished collect CTAs) |
 // [rows][words] bitmaps of the keys above the threshold bin | [rows][kCandCap]
 // candidates (key, position).  The first three are zeroed before each use.
 struct TkLayout {
   uint32_t* hist;
   uint32_t* ncand;
   uint32_t* ctrl;
+  uint32_t* row_done;  // per row: collect CTAs finished (the last one selects)
   uint32_t* bitmap;
   uint2* cand;
   int64_t words;
 };
 
 __host__ __device__ inline size_t tk_ctrl_bytes(int32_t rows) {
-  return al256((static_cast<size_t>(kCtrlInts) + 2 * static_cast<size_t>(rows)) * 4);
+  return al256((static_cast<size_t>(kCtrlInts) + 3 * static_cast<size_t>(rows)) * 4);
 }
 
 __host__ __device__ inline size_t tk_zero_bytes(int32_t rows) {
@@ -55,6 +57,7 @@ __host__ __device__ inline TkLayout tk_layout(void* ws, int32_t rows, int64_t n_
   L.ncand = reinterpret_cast<uint32_t*>(b);
   b += al256(static_cast<size_t>(rows) * 4);
   L.ctrl = reinterpret_cast<uint32_t*>(b);
+  L.row_done = L.ctrl + kCtrlInts + 2 * rows;
   b += tk_ctrl_bytes(rows);
   L.bitmap = reinterpret_cast<uint32_t*>(b);
   b += al256(static_cast<size_t>(rows) * L.words * 4);
@@ -139,58 +142,120 @@ __device__ __forceinline__ uint32_t tk_find(const uint32_t (&v)[NB / NT], uint32
   return static_cast<uint32_t>(tot);
 }
 
+// The NB/NT consecutive bins of thread t from a row's histogram (16-byte
+// aligned), as 16-byte loads: scalar loads NB/NT words apart would touch one
+// cache line per thread and instruction.
+template <int NT, int NB>
+__device__ __forceinline__ void tk_load_bins(const uint32_t* hist, int t, uint32_t (&v)[NB / NT]) {
+  constexpr int PER = NB / NT;
+  static_assert(PER % 4 == 0, "bins per thread");
+  const uint4* src = reinterpret_cast<const uint4*>(hist + t * PER);
+#pragma unroll
+  for (int q = 0; q < PER / 4; ++q) {
+    const uint4 x = __ldcg(src + q);
+    v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+  }
+}
+
+// Bit j of the low byte of x moved to bit 4j.
+__device__ __forceinline__ uint32_t spread8(uint32_t x) {
+  x &= 0xffu;
+  x = (x | (x << 12)) & 0x000f000fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  x = (x | (x << 3)) & 0x11111111u;
+  return x;
+}
+
+// One round's scores of a thread: warp w covers the 1024 positions from
+// base + 1024 w, lane l and step v the four at base + 1024 w + 128 v + 4 l, so
+// every load instruction of the warp reads 512 consecutive bytes.  Only the
+// 16-byte groups holding a position below `lim` (the row's length rounded up
+// to 4, at most ld, so inside the row) are read; positions at or past the
+// row's length are masked when the keys are formed.
+struct ColRound {
+  float4 x[8];
+};
+
+__device__ __forceinline__ void tk_round_load(const float* row, int base, int lim, ColRound& R) {
+  const int p0 = base + (threadIdx.x >> 5) * 1024 + (threadIdx.x & 31) * 4;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    const int p = p0 + v * 128;
+    // coherent: the fused step writes the scores in the same launch
+    R.x[v] = p < lim ? __ldcg(reinterpret_cast<const float4*>(row + p))
+                     : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+  }
+}
+
 // The collect pass for segment `seg` of row r: threshold bin b1 of the row from
-// its first-digit histogram, then each thread takes 32 consecutive positions
-// per round: the keys above b1 become one bitmap word (written once, no
-// atomics) and the keys inside b1 are appended to the row's candidates (one
-// atomic per CTA and round).  Segments are multiples of kColRound positions and
-// cover [0, n_cols), so every bitmap word is written.
+// its first-digit histogram, then per round of kColRound positions the keys
+// above b1 become bitmap words (built from warp ballots, one coalesced store per
+// warp) and the keys inside b1 are appended to the row's candidates (one atomic
+// per CTA and round).  The first round's scores are requested before the
+// histogram is read, and each next round's before this round's atomic.
+// Segments are multiples of kColRound positions and cover [0, n_cols), so every
+// bitmap word is written.
 template <int ID>
 __device__ void tk_collect_cta(const TopkArgs& a, int64_t seg_len, int seg, int r, TkScratch& S) {
   constexpr int NT = kCollectThreads;
-  int64_t n = a.n_cols;
+  static_assert(NT * kWordElems == kColRound && kColRound == (NT / 32) * 1024, "collect round shape");
+  static_assert(kMaxBitmapCols <= (1 << 30), "positions fit 32 bits");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int n = static_cast<int>(a.n_cols);
   if (a.valid_len) {
     const int64_t v = __ldg(a.valid_len + r);
-    n = v < 0 ? 0 : (v < n ? v : n);
+    n = v < 0 ? 0 : (v < n ? static_cast<int>(v) : n);
   }
-  const int64_t s0 = static_cast<int64_t>(seg) * seg_len;
-  const int64_t s1 = s0 + seg_len < a.n_cols ? s0 + seg_len : a.n_cols;
+  const int s0 = seg * static_cast<int>(seg_len);
+  const int s1 = s0 + static_cast<int>(seg_len) < static_cast<int>(a.n_cols) ? s0 + static_cast<int>(seg_len)
+                                                                              : static_cast<int>(a.n_cols);
   if (s0 >= s1) return;
+  const int lim = ((n + 3) & ~3) < a.ld ? ((n + 3) & ~3) : static_cast<int>(a.ld);
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  ColRound cur;
+  tk_round_load(row, s0, lim, cur);
   const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
   const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
   uint32_t hv[kB1 / NT];
-#pragma unroll
-  for (int i = 0; i < kB1 / NT; ++i) hv[i] = __ldcg(hist + threadIdx.x * (kB1 / NT) + i);
+  tk_load_bins<NT, kB1>(hist, threadIdx.x, hv);
   const uint32_t total = tk_find<NT, ID, kB1>(hv, static_cast<uint32_t>(a.k), S, true);
   const uint32_t keff = total < static_cast<uint32_t>(a.k) ? total : static_cast<uint32_t>(a.k);
   const uint32_t b1 = keff > 0 ? static_cast<uint32_t>(S.s_bin) : 0xffffffffu;  // none: no bin qualifies
   uint32_t* bitmap = L.bitmap + static_cast<int64_t>(r) * L.words;
   uint2* cand = L.cand + static_cast<int64_t>(r) * kCandCap;
-  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  for (int64_t base = s0; base < s1; base += kColRound) {
-    const int64_t p0 = base + static_cast<int64_t>(threadIdx.x) * kWordElems;
-    uint32_t key[kWordElems];
-    if (p0 + kWordElems <= n) {
-      const float4* src = reinterpret_cast<const float4*>(row + p0);
+#pragma unroll 1
+  for (int base = s0; base < s1; base += kColRound) {
+    const int p0 = base + warp * 1024 + lane * 4;
+    uint32_t key[8][4];
 #pragma unroll
-      for (int v = 0; v < kWordElems / 4; ++v) {
-        const float4 x = __ldcg(src + v);  // coherent: the fused step writes the scores in the same launch
-        key[4 * v] = order_key(x.x); key[4 * v + 1] = order_key(x.y);
-        key[4 * v + 2] = order_key(x.z); key[4 * v + 3] = order_key(x.w);
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < kWordElems; ++e) key[e] = p0 + e < n ? order_key(__ldcg(row + p0 + e)) : 0u;
+    for (int v = 0; v < 8; ++v) {
+      const int p = p0 + v * 128;
+      key[v][0] = p < n ? order_key(cur.x[v].x) : 0u;
+      key[v][1] = p + 1 < n ? order_key(cur.x[v].y) : 0u;
+      key[v][2] = p + 2 < n ? order_key(cur.x[v].z) : 0u;
+      key[v][3] = p + 3 < n ? order_key(cur.x[v].w) : 0u;
     }
-    uint32_t word = 0;
+    if (base + kColRound < s1) tk_round_load(row, base + kColRound, lim, cur);
+    // bitmap word of lane l: positions 32 l .. 32 l + 31 of the warp's 1024,
+    // i.e. step v = l / 4, lanes 8 (l % 4) .. 8 (l % 4) + 7
+    uint32_t bal[4] = {0u, 0u, 0u, 0u};  // the ballots of step lane / 4
     int nc = 0;
 #pragma unroll
-    for (int e = 0; e < kWordElems; ++e) {
-      const uint32_t bin = key[e] ? (key[e] >> 20) : 0xffffffffu;
-      if (keff > 0 && key[e] && bin > b1) word |= 1u << e;
-      nc += (keff > 0 && key[e] && bin == b1);
+    for (int v = 0; v < 8; ++v) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t k = key[v][c];
+        const uint32_t bin = k >> 20;
+        const uint32_t b = __ballot_sync(0xffffffffu, k != 0u && bin > b1);
+        bal[c] = (lane >> 2) == v ? b : bal[c];
+        nc += (k != 0u && bin == b1) ? 1 : 0;
+      }
     }
-    if (p0 < a.n_cols) bitmap[p0 / kWordElems] = word;
+    const int sh = 8 * (lane & 3);
+    const uint32_t word = spread8(bal[0] >> sh) | (spread8(bal[1] >> sh) << 1) | (spread8(bal[2] >> sh) << 2) |
+                          (spread8(bal[3] >> sh) << 3);
+    const int wi = (base + warp * 1024) / kWordElems + lane;
+    if (wi < L.words) bitmap[wi] = word;
     int tot;
     const int off = tk_excl_scan<NT, ID>(nc, S.warp_sums, &tot);
     if (threadIdx.x == 0) S.s_base = tot ? atomicAdd(L.ncand + r, static_cast<uint32_t>(tot)) : 0u;
@@ -199,10 +264,15 @@ __device__ void tk_collect_cta(const TopkArgs& a, int64_t seg_len, int seg, int 
     tk_sync<NT, ID>();
     if (nc) {
 #pragma unroll
-      for (int e = 0; e < kWordElems; ++e) {
-        if (keff > 0 && key[e] && (key[e] >> 20) == b1) {
-          if (o < static_cast<uint32_t>(kCandCap)) cand[o] = make_uint2(key[e], static_cast<uint32_t>(p0 + e));
-          ++o;
+      for (int v = 0; v < 8; ++v) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t k = key[v][c];
+          if (k != 0u && (k >> 20) == b1) {
+            if (o < static_cast<uint32_t>(kCandCap))
+              cand[o] = make_uint2(k, static_cast<uint32_t>(p0 + v * 128 + c));
+            ++o;
+          }
         }
       }
     }
@@ -220,9 +290,27 @@ __device__ __forceinline__ uint32_t low_bits(uint32_t x, int n) {
   return y;
 }
 
-// Shared memory of the select body besides TkScratch: two bitmaps and the candidates.
-__host__ __device__ inline size_t tk_final_smem(int64_t n_cols) {
-  return 2 * static_cast<size_t>((n_cols + 31) / 32) * 4 + static_cast<size_t>(kCandCap) * 8;
+// Bitmaps of the select body in shared memory: thread t owns the `per`
+// consecutive words from t * per and keeps them at t * stride, stride = per | 1
+// (odd), so the threads' walks over their own words hit distinct banks.
+struct TkPad {
+  int per, stride;
+};
+
+__host__ __device__ inline TkPad tk_pad(int64_t n_cols, int nt) {
+  TkPad p;
+  const int64_t words = (n_cols + 31) / 32;
+  p.per = static_cast<int>((words + nt - 1) / nt);
+  p.stride = p.per | 1;
+  return p;
+}
+
+// Shared memory of the select body besides TkScratch: two padded bitmaps and
+// the candidates.
+__host__ __device__ inline size_t tk_final_smem(int64_t n_cols, int nt) {
+  const TkPad p = tk_pad(n_cols, nt);
+  const size_t bm_words = static_cast<size_t>(nt) * p.stride;
+  return 2 * ((bm_words + 1) / 2 * 2) * 4 + static_cast<size_t>(kCandCap) * 8;
 }
 
 // The select of row r: keff and b1 from the histogram, the bitmap of the keys
@@ -234,9 +322,16 @@ __device__ void tk_final_cta(const TopkArgs& a, int r, uint32_t* fsm, TkScratch&
   const int t = threadIdx.x;
   const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
   const int64_t nwords = L.words;
-  uint32_t* bm = fsm;               // selected positions
-  uint32_t* tb = fsm + nwords;      // positions equal to the threshold key
-  uint2* cs = reinterpret_cast<uint2*>(fsm + 2 * nwords);  // 2*nwords words keep 8-byte alignment
+  const TkPad pad = tk_pad(a.n_cols, NT);
+  const int bm_words = (NT * pad.stride + 1) / 2 * 2;  // even: keeps cs 8-byte aligned
+  uint32_t* bm = fsm;                // selected positions (padded)
+  uint32_t* tb = fsm + bm_words;     // positions equal to the threshold key (padded)
+  uint2* cs = reinterpret_cast<uint2*>(fsm + 2 * bm_words);
+  const DivU32 dper = make_divu32(static_cast<uint32_t>(pad.per));
+  auto pw = [&](uint32_t w) -> int {  // padded index of word w
+    const uint32_t q = divu32(dper, w);
+    return static_cast<int>(q * pad.stride + (w - q * pad.per));
+  };
   int32_t* out = a.idx + static_cast<int64_t>(r) * a.k;
   int64_t n = a.n_cols;
   if (a.valid_len) {
@@ -248,17 +343,33 @@ __device__ void tk_final_cta(const TopkArgs& a, int r, uint32_t* fsm, TkScratch&
   const uint32_t* hist = L.hist + static_cast<int64_t>(r) * kB1;
   constexpr int HB = kB1 / NT;
   uint32_t hv[HB];
-#pragma unroll
-  for (int i = 0; i < HB; ++i) hv[i] = __ldcg(hist + t * HB + i);
+  tk_load_bins<NT, kB1>(hist, t, hv);
   const uint32_t n_cand = __ldcg(L.ncand + r);
   const uint32_t* gbm = L.bitmap + static_cast<int64_t>(r) * nwords;
-  for (int64_t w = t; w < nwords; w += NT) {
-    bm[w] = __ldcg(gbm + w);
-    tb[w] = 0;
+  // eight loads in flight per thread and pass, stored once they have landed
+  for (int w0 = t; w0 < nwords; w0 += 8 * NT) {
+    uint32_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = w0 + u * NT < nwords ? __ldcg(gbm + w0 + u * NT) : 0u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (w0 + u * NT >= nwords) break;
+      const int pi = pw(static_cast<uint32_t>(w0 + u * NT));
+      bm[pi] = v[u];
+      tb[pi] = 0;
+    }
   }
   const bool overflow = n_cand > static_cast<uint32_t>(kCandCap);
   const int nc = overflow ? 0 : static_cast<int>(n_cand);
-  for (int c = t; c < nc; c += NT) cs[c] = __ldcg(L.cand + static_cast<int64_t>(r) * kCandCap + c);
+  for (int c0 = t; c0 < nc; c0 += 4 * NT) {
+    uint2 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      v[u] = c0 + u * NT < nc ? __ldcg(L.cand + static_cast<int64_t>(r) * kCandCap + c0 + u * NT) : make_uint2(0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (c0 + u * NT < nc) cs[c0 + u * NT] = v[u];
+  }
   // keff and the threshold bin
   const uint32_t total = tk_find<NT, ID, kB1>(hv, static_cast<uint32_t>(a.k), S, true);
   const uint32_t keff = total < static_cast<uint32_t>(a.k) ? total : static_cast<uint32_t>(a.k);
@@ -309,8 +420,8 @@ __device__ void tk_final_cta(const TopkArgs& a, int r, uint32_t* fsm, TkScratch&
   if (!overflow) {
     for (int c = t; c < nc; c += NT) {
       const uint2 e = cs[c];
-      if (e.x > T) atomicOr(&bm[e.y >> 5], 1u << (e.y & 31));
-      else if (e.x == T) atomicOr(&tb[e.y >> 5], 1u << (e.y & 31));
+      if (e.x > T) atomicOr(&bm[pw(e.y >> 5)], 1u << (e.y & 31));
+      else if (e.x == T) atomicOr(&tb[pw(e.y >> 5)], 1u << (e.y & 31));
     }
   } else {
     for (int64_t base = 0; base < n; base += NT * 4) {
@@ -321,42 +432,59 @@ __device__ void tk_final_cta(const TopkArgs& a, int r, uint32_t* fsm, TkScratch&
         const uint32_t key = order_key(__ldcg(row + p + j));
         if ((key >> 20) != b1) continue;
         const uint32_t q = static_cast<uint32_t>(p + j);
-        if (key > T) atomicOr(&bm[q >> 5], 1u << (q & 31));
-        else if (key == T) atomicOr(&tb[q >> 5], 1u << (q & 31));
+        if (key > T) atomicOr(&bm[pw(q >> 5)], 1u << (q & 31));
+        else if (key == T) atomicOr(&tb[pw(q >> 5)], 1u << (q & 31));
       }
     }
   }
   tk_sync<NT, ID>();
-  // ordered compaction: the lowest `ties` positions equal to T join the selection
-  const int64_t per = (nwords + NT - 1) / NT;
-  const int64_t w0 = t * per, w1 = (w0 + per < nwords) ? w0 + per : nwords;
+  // ordered compaction: the lowest `ties` positions equal to T join the
+  // selection, then the selected positions are written in ascending order;
+  // thread t walks its own words (padded: no bank conflicts).
+  const int w0 = t * pad.per;
+  const int nmine = static_cast<int>(nwords) - w0 < pad.per ? static_cast<int>(nwords) - w0 : pad.per;
+  const int pb = t * pad.stride;
   int my_ties = 0;
-  for (int64_t w = w0; w < w1; ++w) my_ties += __popc(tb[w]);
+  for (int i = 0; i < nmine; ++i) my_ties += __popc(tb[pb + i]);
   int tie_tot;
   int tie_before = tk_excl_scan<NT, ID>(my_ties, S.warp_sums, &tie_tot);
   int my_sel = 0;
-  for (int64_t w = w0; w < w1; ++w) {
-    const uint32_t x = tb[w];
+  for (int i = 0; i < nmine; ++i) {
+    const uint32_t x = tb[pb + i];
     const int px = __popc(x);
     const int take = static_cast<int>(ties) - tie_before;
     uint32_t add = 0;
     if (take > 0) add = take >= px ? x : low_bits(x, take);
     tie_before += px;
-    const uint32_t merged = bm[w] | add;
-    bm[w] = merged;
+    const uint32_t merged = bm[pb + i] | add;
+    bm[pb + i] = merged;
     my_sel += __popc(merged);
   }
   int sel_tot;
   int o = tk_excl_scan<NT, ID>(my_sel, S.warp_sums, &sel_tot);
-  for (int64_t w = w0; w < w1; ++w) {
-    uint32_t x = bm[w];
+  // The positions are gathered in shared memory (the candidates' space, free
+  // now) and written out coalesced: written straight from the walk, every
+  // store instruction of a warp would touch up to 32 lines.
+  int32_t* os = reinterpret_cast<int32_t*>(cs);
+  const bool staged = a.k <= 2 * kCandCap;
+  for (int i = 0; i < nmine; ++i) {
+    uint32_t x = bm[pb + i];
     while (x) {
       const int b = __ffs(x) - 1;
       x &= x - 1;
-      if (o < a.k) out[o] = static_cast<int32_t>(w * 32 + b);
-      else record_error(a.status, LSA_ERR_BOUNDS, r, o);  // cannot happen
+      if (o < a.k) {
+        if (staged) os[o] = (w0 + i) * 32 + b;
+        else out[o] = (w0 + i) * 32 + b;
+      } else {
+        record_error(a.status, LSA_ERR_BOUNDS, r, o);  // cannot happen
+      }
       ++o;
     }
+  }
+  if (staged) {
+    tk_sync<NT, ID>();
+    const int n_out = static_cast<int>(keff);
+    for (int i = t; i < n_out; i += NT) out[i] = os[i];
   }
   tk_sync<NT, ID>();  // shared memory free for the caller's next use
 }

@@ -19,6 +19,9 @@ SMALL = {
     "prefill_3000x256": synth.scaled(C[5], len_lo=3000, len_hi=3000, chunk=256, top_k=512),
     # single short sequence (length 1) and contiguous bf16
     "len1": synth.scaled(C[2], batch=3, len_lo=1, len_hi=300, top_k=64),
+    # pages of 48 tokens (not a power of two; the tensor-core scan takes multiples of 64, so its
+    # scan runs on the CUDA cores)
+    "paged48_B3": synth.scaled(C[3], batch=3, len_lo=300, len_hi=2500, top_k=256, block_size=48),
 }
 
 SEEDS = {name: 5000 + i for i, name in enumerate(SMALL)}

@@ -33,7 +33,7 @@ def _visible(case):
 
 
 @pytest.mark.parametrize("path", ["default", "simt"])
-@pytest.mark.parametrize("name", ["tiny_fp32", "bf16_L5000", "paged_B5", "prefill_3000x256", "len1"])
+@pytest.mark.parametrize("name", ["tiny_fp32", "bf16_L5000", "paged_B5", "prefill_3000x256", "len1", "paged48_B3"])
 def test_attention_on_given_indices(name, path, monkeypatch):
     if path == "simt":
         monkeypatch.setenv("LSA_FORCE_SIMT", "1")
