@@ -140,7 +140,7 @@ ScoresArgs scores_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, cons
 lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
                      const int32_t* row_pos, const void* q_idx, const float* w, float* scores,
                      int64_t ld, void* ws, void* inner_ws, size_t inner_bytes, cudaStream_t s,
-                     uint32_t* hist12 = nullptr, bool* hist_done = nullptr) {
+                     uint32_t* hist12 = nullptr, bool* hist_done = nullptr, uint32_t* done_ctr = nullptr) {
   ScoresArgs a = scores_args(d, c, rows, row_seq, row_pos, q_idx, w, scores, ld, ws, inner_ws, inner_bytes);
   if (hist_done) *hist_done = false;
   if (rows == 0 || ld == 0) return LSA_OK;
@@ -150,6 +150,7 @@ lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const 
       cudaError_t e = cudaMemsetAsync(hist12, 0, topk_hist_zero_bytes(rows), s);
       if (e != cudaSuccess) return LSA_ERR_CUDA;
       a.hist12 = hist12;
+      a.done_ctr = done_ctr;  // zeroed with the histograms
       if (hist_done) *hist_done = true;
     }
     return cuda_status(launch_scores_tc(a, s));
@@ -175,9 +176,11 @@ TopkArgs topk_args(const float* scores, int64_t ld, int32_t rows, const int32_t*
 
 lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
                    int32_t k, int32_t* idx, void* ws, void* inner_ws, cudaStream_t s, bool hist_ready = false,
-                   bool pdl = false) {
+                   bool pdl = false, const uint32_t* wait_ctr = nullptr, uint32_t wait_target = 0) {
   TopkArgs a = topk_args(scores, ld, rows, valid_len, n_cols, k, idx, ws, inner_ws, hist_ready);
   a.pdl = pdl;
+  a.wait_ctr = wait_ctr;
+  a.wait_target = wait_target;
   return cuda_status(launch_topk(a, s));
 }
 
@@ -205,11 +208,12 @@ AttnArgs attn_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, const in
 
 lsa_status do_attn(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq, const void* q,
                    const int32_t* idx, void* out, float* lse, void* ws, void* inner_ws, size_t inner_bytes,
-                   cudaStream_t s, bool pdl = false) {
+                   cudaStream_t s, bool pdl = false, const uint32_t* row_ready = nullptr) {
   AttnArgs a = attn_args(d, c, rows, row_seq, q, idx, out, lse, ws, inner_ws, inner_bytes);
   // in a decode step the kernel before is the step's top-k, which does not write q
   a.pdl = pdl;
   a.q_early = pdl;
+  a.row_ready = row_ready;
   if (rows == 0) return LSA_OK;
   if (!force_simt() && attn_tc_supported(a)) return cuda_status(launch_attn_tc(a, s));
   return cuda_status(launch_attn_simt(a, s));
@@ -333,16 +337,24 @@ static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const 
   }
   uint32_t* hist12 = (!force_simt() && topk_v2_ok(c->max_len)) ? static_cast<uint32_t*>(inner) : nullptr;
   bool hist_done = false;
-  st = do_scores(d, c, B, nullptr, nullptr, q_idx, w, scores, ld, ws, inner, inner_bytes, s, hist12, &hist_done);
+  // With the histogram built by the scan, the kernels hand over through words
+  // zeroed with it: the top-k starts once every scan CTA has counted itself,
+  // the attention of a row once that row's selection is written.
+  uint32_t *scan_done = nullptr, *sel_done = nullptr;
+  if (hist12) topk_step_flags(inner, B, c->max_len, &scan_done, &sel_done);
+  st = do_scores(d, c, B, nullptr, nullptr, q_idx, w, scores, ld, ws, inner, inner_bytes, s, hist12, &hist_done,
+                 scan_done);
   if (st != LSA_OK) return st;
   if (!mark(1)) return LSA_ERR_CUDA;
   // The top-k and the attention are launched as programmatic dependents of the
   // kernel before them: their CTAs may be scheduled while it finishes, and
   // they wait for it (griddepcontrol.wait) before reading what it wrote.
-  st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, s, hist_done, true);
+  const bool handoff = hist_done && !events;  // events between the kernels would serialise them anyway
+  st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, s, hist_done, true,
+               handoff ? scan_done : nullptr, handoff ? static_cast<uint32_t>(scan_tc_grid()) : 0u);
   if (st != LSA_OK) return st;
   if (!mark(2)) return LSA_ERR_CUDA;
-  st = do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s, true);
+  st = do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s, true, handoff ? sel_done : nullptr);
   if (st != LSA_OK) return st;
   if (!mark(3)) return LSA_ERR_CUDA;
   return LSA_OK;

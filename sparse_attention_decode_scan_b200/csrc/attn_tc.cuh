@@ -290,6 +290,18 @@ __device__ __forceinline__ void merge_slice(const TcAttnParams& P, int r, int ha
   }
 }
 
+// Bounded wait (acquire) until *flag != 0; false after tc::kWaitLimitNs.
+__device__ __forceinline__ bool wait_flag(const uint32_t* flag) {
+  const uint64_t t0 = tc::globaltimer_ns();
+  for (;;) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v != 0) return true;
+    if (tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) return false;
+    __nanosleep(64);
+  }
+}
+
 // One CTA of the sparse attention: 64 heads (`half`) of query row r over the
 // split-th range of its selection.  `tmem_slot` holds (or, once the first block
 // barrier has passed, will hold) the base of kTmemCols allocated TMEM columns.
@@ -387,7 +399,16 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
                        : "memory");
       }
     };
-    tc::griddep_wait();  // launched early in a decode step: the selection is complete from here on
+    if (a.row_ready) {
+      // decode step, launched early: wait for this row's selection only
+      if (t == 0 && !wait_flag(a.row_ready + r)) {
+        record_error(a.status, LSA_ERR_TIMEOUT, r, 21);
+        *abort_flag = 1;
+      }
+      asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");  // the producer warps
+    } else {
+      tc::griddep_wait();  // launched early in a decode step: the selection is complete from here on
+    }
     fill_table(0);
     prefetch_l2(0, 0);
     prefetch_l2(1, 0);
@@ -442,7 +463,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA issuer
-    tc::griddep_wait();
+    if (!a.row_ready) tc::griddep_wait();
     if (lane == 0 && nch > 0) {
       bool ok = tc::mbar_wait(qfull, 0, abort_flag);
       tc::fence_proxy_async_smem();
@@ -535,7 +556,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     // 0-287 (lanes 16-31 of those columns, O's, get zeros: the first P V
     // overwrites them).  In a decode step q is an input of the step, so it is
     // loaded while the top-k may still run.
-    if (!a.q_early) tc::griddep_wait();
+    if (!a.q_early && !a.row_ready) tc::griddep_wait();
     {
       const uint4* qsrc = reinterpret_cast<const uint4*>(
           reinterpret_cast<const uint8_t*>(a.q) +
@@ -561,7 +582,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qfull);
     }
-    if (a.q_early) tc::griddep_wait();
+    if (a.q_early && !a.row_ready) tc::griddep_wait();
     const float c2 = a.scale * kLog2e;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;

@@ -136,6 +136,8 @@ bool scores_tc_fused_hist_ok(const ScoresArgs& a) { return a.row_pos == nullptr 
 
 cudaError_t scan_tc_maps(const ScoresArgs& a, CUtensorMap* tmap, CUtensorMap* smap) { return make_maps(a, tmap, smap); }
 
+int scan_tc_grid() { return num_sms(); }
+
 cudaError_t launch_scores_tc(const ScoresArgs& a, cudaStream_t s) {
   const bool causal = a.row_pos != nullptr;
   if (a.key_dtype == LSA_FP8_E4M3) return causal ? launch_t<LSA_FP8_E4M3, 2>(a, s) : launch_t<LSA_FP8_E4M3, 1>(a, s);

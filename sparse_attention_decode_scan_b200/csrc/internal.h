@@ -44,6 +44,8 @@ struct ScoresArgs {
   size_t plan_bytes;
   uint32_t* hist12;    // if set: per-row histogram of score-key bits [31:20] ([rows][4096],
                        // zeroed by the caller), accumulated by the scan for the top-k
+  uint32_t* done_ctr = nullptr;  // if set (zeroed by the caller): every CTA adds 1 once its
+                                 // scores and histogram counts are written and fenced
 };
 
 // ---- indexer
@@ -76,8 +78,16 @@ struct TopkArgs {
   DevStatus* status;
   bool hist_ready;     // the first histogram and list counters are already in ws
   bool pdl = false;    // launched as a programmatic dependent of the kernel before it (decode step)
+  // Decode step: instead of waiting for the scan grid to complete, wait until
+  // *wait_ctr reaches wait_target (the scan's CTAs, each after its writes);
+  // each row's selection then raises its flag in the layout's sel_done.
+  const uint32_t* wait_ctr = nullptr;
+  uint32_t wait_target = 0;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+// The decode step's handoff words inside the top-k workspace (zeroed with its
+// head): the count of finished scan CTAs and the per-row selection flags.
+void topk_step_flags(void* ws, int32_t rows, int64_t n_cols, uint32_t** scan_done, uint32_t** sel_done);
 // The three-launch top-k applies (rows up to 2^19 entries); its first
 // histogram then sits at the start of the top-k workspace, followed by the
 // list counters; topk_hist_zero_bytes of them must be zero before the scan.
@@ -89,6 +99,8 @@ bool scores_tc_fused_hist_ok(const ScoresArgs& a);
 TopkPlan topk_collect_plan(int32_t rows, int64_t n_cols, int32_t target_ctas);
 // tensor maps of the tensor-core scan (keys; FP8 scales)
 cudaError_t scan_tc_maps(const ScoresArgs& a, CUtensorMap* tmap, CUtensorMap* smap);
+// CTAs of a tensor-core scan launch (one per SM).
+int scan_tc_grid();
 
 // ---- sparse attention
 struct AttnArgs {
@@ -108,6 +120,9 @@ struct AttnArgs {
   DevStatus* status;
   bool pdl = false;      // launched as a programmatic dependent of the kernel before it (decode step)
   bool q_early = false;  // with pdl: q may be read before the kernel before it completes
+  // Decode step: the selection of row r may be read once row_ready[r] != 0
+  // (raised by the top-k after writing it); null: wait for the kernel before.
+  const uint32_t* row_ready = nullptr;
 };
 size_t attn_simt_ws_bytes(int32_t rows, int32_t H, int32_t Dv, int32_t k);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);

@@ -813,6 +813,12 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     for (uint64_t* b = bars; b <= ebar; ++b) tc::mbar_inval(b);
   }
   scan_sync();
+  if (a.done_ctr) {
+    // decode step: the top-k starts on this count instead of the grid's completion
+    __threadfence();  // this thread's score stores and histogram adds
+    scan_sync();
+    if (threadIdx.x == 0) atomicAdd(a.done_ctr, 1u);
+  }
 }
 
 }  // namespace scan

@@ -343,19 +343,48 @@ __global__ void __launch_bounds__(tk::kCollectThreads, 2) k_tk_rows(TopkArgs a, 
   __shared__ tk::TkScratch S;
   __shared__ int s_last;
   const int r = blockIdx.y;
-  tc::griddep_wait();  // launched early in a decode step: the scores are complete from here on
+  const tk::TkLayout L = tk::tk_layout(a.ws, a.rows, a.n_cols);
+  if (a.wait_ctr) {
+    // decode step, launched early: wait until every scan CTA has counted
+    // itself (its scores and histogram counts written and fenced)
+    if (threadIdx.x == 0) {
+      s_last = 1;
+      const uint64_t t0 = tc::globaltimer_ns();
+      for (;;) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.wait_ctr) : "memory");
+        if (v >= a.wait_target) break;
+        if (tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) {
+          record_error(a.status, LSA_ERR_TIMEOUT, r, 20);
+          s_last = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __syncthreads();
+    if (!s_last) return;
+  } else {
+    tc::griddep_wait();  // launched early in a decode step: the scores are complete from here on
+  }
   tc::griddep_launch_dependents();
   tk::tk_collect_cta<2>(a, seg_len, blockIdx.x, r, S);
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();  // this CTA's bitmap words and candidates before its count
-    const uint32_t done = atomicAdd(tk::tk_layout(a.ws, a.rows, a.n_cols).row_done + r, 1u);
+    const uint32_t done = atomicAdd(L.row_done + r, 1u);
     s_last = done == static_cast<uint32_t>(nseg - 1);
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();  // the other segments' writes, read through L2 by the select
   tk::tk_final_cta<tk::kCollectThreads, 3>(a, r, fsm, S);
+  if (a.wait_ctr) {
+    // decode step: the attention of row r may read its selection from now on
+    __threadfence();  // this thread's selection writes
+    __syncthreads();
+    if (threadIdx.x == 0) asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(L.sel_done + r), "r"(1u) : "memory");
+  }
 }
 
 // SMs of the current device (the plan's CTA target).
@@ -400,6 +429,12 @@ TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
 bool topk_v2_ok(int64_t n_cols) { return n_cols <= tk::kMaxBitmapCols; }
 
 size_t topk_hist_zero_bytes(int32_t rows) { return tk::tk_zero_bytes(rows); }
+
+void topk_step_flags(void* ws, int32_t rows, int64_t n_cols, uint32_t** scan_done, uint32_t** sel_done) {
+  const tk::TkLayout L = tk::tk_layout(ws, rows, n_cols);
+  *scan_done = L.scan_done;
+  *sel_done = L.sel_done;
+}
 
 size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t) {
   const size_t R = static_cast<size_t>(rows);

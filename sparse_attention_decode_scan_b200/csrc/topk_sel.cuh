@@ -26,8 +26,9 @@ constexpr int kCtrlInts = 64;            // control words of the fused step (gri
 __host__ __device__ inline size_t al256(size_t b) { return (b + 255) / 256 * 256; }
 
 // Workspace: [rows][4096] first-digit histograms | [rows] candidate counts |
-// control block (fused step: grid-barrier word, attention split counters;
-// per-row counts of finished collect CTAs) |
+// control block (fused step: grid-barrier word; scan CTAs finished; attention
+// split counters; per-row counts of finished collect CTAs; per-row selection
+// flags) |
 // [rows][words] bitmaps of the keys above the threshold bin | [rows][kCandCap]
 // candidates (key, position).  The first three are zeroed before each use.
 struct TkLayout {
@@ -35,13 +36,15 @@ struct TkLayout {
   uint32_t* ncand;
   uint32_t* ctrl;
   uint32_t* row_done;  // per row: collect CTAs finished (the last one selects)
+  uint32_t* sel_done;  // per row: 1 once the row's selection is written (decode step)
+  uint32_t* scan_done; // scan CTAs finished (decode step)
   uint32_t* bitmap;
   uint2* cand;
   int64_t words;
 };
 
 __host__ __device__ inline size_t tk_ctrl_bytes(int32_t rows) {
-  return al256((static_cast<size_t>(kCtrlInts) + 3 * static_cast<size_t>(rows)) * 4);
+  return al256((static_cast<size_t>(kCtrlInts) + 4 * static_cast<size_t>(rows)) * 4);
 }
 
 __host__ __device__ inline size_t tk_zero_bytes(int32_t rows) {
@@ -58,6 +61,8 @@ __host__ __device__ inline TkLayout tk_layout(void* ws, int32_t rows, int64_t n_
   b += al256(static_cast<size_t>(rows) * 4);
   L.ctrl = reinterpret_cast<uint32_t*>(b);
   L.row_done = L.ctrl + kCtrlInts + 2 * rows;
+  L.sel_done = L.ctrl + kCtrlInts + 3 * rows;
+  L.scan_done = L.ctrl + 1;
   b += tk_ctrl_bytes(rows);
   L.bitmap = reinterpret_cast<uint32_t*>(b);
   b += al256(static_cast<size_t>(rows) * L.words * 4);
