@@ -176,11 +176,13 @@ TopkArgs topk_args(const float* scores, int64_t ld, int32_t rows, const int32_t*
 
 lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
                    int32_t k, int32_t* idx, void* ws, void* inner_ws, cudaStream_t s, bool hist_ready = false,
-                   bool pdl = false, const uint32_t* wait_ctr = nullptr, uint32_t wait_target = 0) {
+                   bool pdl = false, const uint32_t* wait_ctr = nullptr, uint32_t wait_target = 0,
+                   bool split_select = false) {
   TopkArgs a = topk_args(scores, ld, rows, valid_len, n_cols, k, idx, ws, inner_ws, hist_ready);
   a.pdl = pdl;
   a.wait_ctr = wait_ctr;
   a.wait_target = wait_target;
+  a.split_select = split_select;
   return cuda_status(launch_topk(a, s));
 }
 
@@ -208,12 +210,21 @@ AttnArgs attn_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, const in
 
 lsa_status do_attn(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq, const void* q,
                    const int32_t* idx, void* out, float* lse, void* ws, void* inner_ws, size_t inner_bytes,
-                   cudaStream_t s, bool pdl = false, const uint32_t* row_ready = nullptr) {
+                   cudaStream_t s, bool pdl = false, const uint32_t* row_ready = nullptr,
+                   const AttnArgs* split = nullptr) {
   AttnArgs a = attn_args(d, c, rows, row_seq, q, idx, out, lse, ws, inner_ws, inner_bytes);
   // in a decode step the kernel before is the step's top-k, which does not write q
   a.pdl = pdl;
   a.q_early = pdl;
   a.row_ready = row_ready;
+  if (split) {
+    a.split_sel = true;
+    a.tk_ws = split->tk_ws;
+    a.tk_ncols = split->tk_ncols;
+    a.tk_nseg = split->tk_nseg;
+    a.tk_seg_len = split->tk_seg_len;
+    a.idx_w = split->idx_w;
+  }
   if (rows == 0) return LSA_OK;
   if (!force_simt() && attn_tc_supported(a)) return cuda_status(launch_attn_tc(a, s));
   return cuda_status(launch_attn_simt(a, s));
@@ -291,6 +302,15 @@ lsa_status lsa_sparse_attn_decode(const lsa_dims* d, const lsa_cache* c, int32_t
                  ws_bytes - kStatusBytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Rows at least this long take the split select in a decode step (the
+// environment variable LSA_SPLIT_SELECT_MIN_COLS overrides it, for tests).
+constexpr int64_t kSplitSelectMinCols = int64_t(1) << 18;
+
+int64_t split_select_min_cols() {
+  const char* e = getenv("LSA_SPLIT_SELECT_MIN_COLS");
+  return e && e[0] ? strtoll(e, nullptr, 10) : kSplitSelectMinCols;
+}
+
 static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const void* q_idx, const float* w,
                                    const void* q, void* out, float* lse, int32_t* idx_out, int32_t flags, void* ws,
                                    size_t ws_bytes, lsa_stream_t stream, void* const* events) {
@@ -350,11 +370,30 @@ static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const 
   // kernel before them: their CTAs may be scheduled while it finishes, and
   // they wait for it (griddepcontrol.wait) before reading what it wrote.
   const bool handoff = hist_done && !events;  // events between the kernels would serialise them anyway
+  // With the handoffs and the tensor-core attention, the row's last top-k CTA
+  // only makes the row's bitmap exact and stores per-segment offsets; each
+  // attention CTA compacts its own entries from the segments holding them
+  // (and writes them to idx only if the caller asked for the selection).
+  // It pays for long rows (the full select walks the whole row's bitmap in one
+  // CTA: about 27 us at 512K positions, against a few microseconds of
+  // compaction per attention CTA); for rows up to about 128K the full select
+  // is as fast or faster (measured at 32K and 128K).
+  AttnArgs split;
+  bool split_sel = false;
+  if (handoff && !force_simt() && c->max_len >= split_select_min_cols() && attn_tc_split_fits(B, d->top_k) &&
+      attn_tc_supported(attn_args(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes)) &&
+      topk_rows_plan(B, c->max_len, &split.tk_nseg, &split.tk_seg_len)) {
+    split_sel = true;
+    split.tk_ws = inner;
+    split.tk_ncols = c->max_len;
+    split.idx_w = idx_out;
+  }
   st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, s, hist_done, true,
-               handoff ? scan_done : nullptr, handoff ? static_cast<uint32_t>(scan_tc_grid()) : 0u);
+               handoff ? scan_done : nullptr, handoff ? static_cast<uint32_t>(scan_tc_grid()) : 0u, split_sel);
   if (st != LSA_OK) return st;
   if (!mark(2)) return LSA_ERR_CUDA;
-  st = do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s, true, handoff ? sel_done : nullptr);
+  st = do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s, true,
+               handoff && !split_sel ? sel_done : nullptr, split_sel ? &split : nullptr);
   if (st != LSA_OK) return st;
   if (!mark(3)) return LSA_ERR_CUDA;
   return LSA_OK;

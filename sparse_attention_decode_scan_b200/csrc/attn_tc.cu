@@ -78,6 +78,12 @@ bool attn_tc_shape_ok(int32_t dtype, int32_t H, int32_t D, int32_t Dv, int32_t) 
 
 int attn_tc_launches(int32_t, int32_t, int32_t) { return 1; }
 
+bool attn_tc_split_fits(int32_t rows, int32_t k) {
+  const int ns = tc_nsplit(rows, k);
+  const int chunks = (k + kChunk - 1) / kChunk;
+  return ((chunks + ns - 1) / ns) * kChunk <= kRowTab;
+}
+
 bool attn_tc_supported(const AttnArgs& a) {
   // KV rows are kept as 32-bit indices
   const int64_t kv_rows = a.cache.block_size > 0 ? a.cache.n_blocks * a.cache.block_size

@@ -34,6 +34,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
+#include "topk_sel.cuh"
 
 namespace lsa {
 namespace attn {
@@ -178,15 +179,16 @@ __device__ __forceinline__ RowCtx row_ctx(const AttnArgs& a, int r) {
 }
 
 // KV rows of the list entries at offsets [lo, hi) of the split (list = the
-// row's selection from the split's first entry) into rtab[e - base], by n
-// threads (tid): per pass 8 list loads in flight, then their 8 block-table
-// loads.  -1 marks padding, positions out of range and bad blocks (reported
+// row's selection from the split's first entry, in global memory, or in shared
+// memory with list_shared, where it may be rtab itself) into rtab[e - base],
+// by n threads (tid): per pass 8 list loads in flight, then their 8
+// block-table loads.  -1 marks padding, positions out of range and bad blocks (reported
 // when `report`).  Out of line: it runs once per table part, and one compact
 // copy is cheaper to fetch than inlined ones.
 static __device__ __noinline__ void fill_rows(const int32_t* list, const int32_t* bt, int32_t max_blocks, int32_t block_size,
                                               int64_t n_blocks, int64_t row_base, int64_t L, bool ok, DevStatus* status,
                                               int r, int base, int lo, int hi, int tid, int n, bool report,
-                                              int32_t* rtab) {
+                                              int32_t* rtab, bool list_shared = false) {
   const bool paged = block_size > 0;
   const DivU32 bs = make_divu32(paged ? static_cast<uint32_t>(block_size) : 1u);
   for (int e = lo + tid; e < hi; e += 8 * n) {
@@ -195,7 +197,7 @@ static __device__ __noinline__ void fill_rows(const int32_t* list, const int32_t
     for (int u = 0; u < 8; ++u) {
       const int eu = e + u * n;
       // L2-coherent load: in the fused step the selection is written earlier in the same launch
-      pos[u] = (eu < hi && ok) ? __ldcg(list + eu) : -1;
+      pos[u] = (eu < hi && ok) ? (list_shared ? list[eu] : __ldcg(list + eu)) : -1;
     }
     int32_t blk[8];
     uint32_t lb[8];
@@ -290,6 +292,88 @@ __device__ __forceinline__ void merge_slice(const TcAttnParams& P, int r, int ha
   }
 }
 
+// Bounded wait (acquire) until *flag != 0; its value, or 0 after tc::kWaitLimitNs.
+__device__ __forceinline__ uint32_t wait_value(const uint32_t* flag) {
+  const uint64_t t0 = tc::globaltimer_ns();
+  for (;;) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v != 0) return v;
+    if (tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) return 0;
+    __nanosleep(64);
+  }
+}
+
+// Entries [j0, j1) of a row's ordered selection (ascending positions) from the
+// top-k's exact bitmap of the row and its per-segment first entries (segoff,
+// keff at [nseg]), as positions (-1 past keff) into rtab[0, j1 - j0): only the
+// segments holding those entries are compacted.  By the 128 producer threads
+// (named barrier 4); scratch: 1 KB plus the staged words (padded per thread)
+// at `scratch` + 1024.
+static __device__ __noinline__ void split_entries(const uint32_t* segoff, const uint32_t* bitmap, int64_t nwords,
+                                                  int nseg, int64_t seg_len, int j0, int j1, int32_t* rtab,
+                                                  uint8_t* scratch, int t) {
+  constexpr int NT = kProdThreads;
+  int* warp_sums = reinterpret_cast<int*>(scratch);
+  uint32_t* so = reinterpret_cast<uint32_t*>(scratch + 128);  // [nseg + 1]
+  uint32_t* st = reinterpret_cast<uint32_t*>(scratch + 1024);
+  for (int i = t; i <= nseg; i += NT) so[i] = __ldcg(segoff + i);
+  asm volatile("bar.sync 4, %0;" ::"n"(NT) : "memory");
+  const int keff = static_cast<int>(so[nseg]);
+  const int n_ent = j1 - j0;
+  const int e_hi = keff < j1 ? keff : j1;
+  for (int e = (keff > j0 ? keff : j0) - j0 + t; e < n_ent; e += NT) rtab[e] = -1;
+  if (j0 < e_hi) {
+    // the segments holding entries j0 and e_hi - 1
+    int s_lo = 0, s_hi = 0;
+    for (int s2 = 0; s2 < nseg; ++s2) {
+      if (static_cast<int>(so[s2]) <= j0) s_lo = s2;
+      if (static_cast<int>(so[s2]) <= e_hi - 1) s_hi = s2;
+    }
+    const int64_t wps = seg_len / 32;
+    const int64_t w_lo = s_lo * wps;
+    const int64_t w_hi = (s_hi + 1) * wps < nwords ? (s_hi + 1) * wps : nwords;
+    const int W = static_cast<int>(w_hi - w_lo);
+    const int per = (W + NT - 1) / NT, stride = per | 1;
+    const DivU32 dper = make_divu32(static_cast<uint32_t>(per));
+    for (int w0 = t; w0 < W; w0 += 8 * NT) {
+      uint32_t v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = w0 + u * NT < W ? __ldcg(bitmap + w_lo + w0 + u * NT) : 0u;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t w = static_cast<uint32_t>(w0 + u * NT);
+        if (w0 + u * NT < W) {
+          const uint32_t q = divu32(dper, w);
+          st[q * stride + (w - q * per)] = v[u];
+        }
+      }
+    }
+    asm volatile("bar.sync 4, %0;" ::"n"(NT) : "memory");
+    const int wa = t * per;
+    const int nm = W - wa < per ? (W - wa > 0 ? W - wa : 0) : per;
+    int cnt = 0;
+    for (int i = 0; i < nm; ++i) cnt += __popc(st[t * stride + i]);
+    int tot;
+    int o = static_cast<int>(so[s_lo]) + tk::tk_excl_scan<NT, 4>(cnt, warp_sums, &tot);
+    for (int i = 0; i < nm && o < e_hi; ++i) {
+      uint32_t x = st[t * stride + i];
+      const int px = __popc(x);
+      if (o + px <= j0) {
+        o += px;
+        continue;
+      }
+      while (x) {
+        const int b = __ffs(x) - 1;
+        x &= x - 1;
+        if (o >= j0 && o < e_hi) rtab[o - j0] = static_cast<int32_t>((w_lo + wa + i) * 32 + b);
+        ++o;
+      }
+    }
+  }
+  asm volatile("bar.sync 4, %0;" ::"n"(NT) : "memory");
+}
+
 // Bounded wait (acquire) until *flag != 0; false after tc::kWaitLimitNs.
 __device__ __forceinline__ bool wait_flag(const uint32_t* flag) {
   const uint64_t t0 = tc::globaltimer_ns();
@@ -331,6 +415,8 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
   uint8_t* vrow = reinterpret_cast<uint8_t*>(last_flag + 1);  // [kNBuf][kChunk]: 1 = the row has a KV row
   float* slse = reinterpret_cast<float*>(vrow + kNBuf * kChunk);  // [64] cluster merge: the partial's lse
   const bool cmerge = P.nsplit > 1 && P.merge == kMergeCluster;
+  // the producer waits for this row's data itself (no wait for the kernel before)
+  const bool handoff = a.row_ready != nullptr || a.split_sel;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j0 = split * P.split_len;
@@ -399,7 +485,37 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
                        : "memory");
       }
     };
-    if (a.row_ready) {
+    uint32_t sel_state = 2;  // 2: the row's selection is in a.idx
+    if (a.split_sel) {
+      // decode step, launched early: wait for the top-k's split select of this
+      // row (1: exact bitmap and segment offsets, 2: the full selection in idx)
+      const tk::TkLayout TL = tk::tk_layout(a.tk_ws, a.rows, a.tk_ncols);
+      if (t == 0) {
+        const uint32_t v = wait_value(TL.selready + r);
+        if (v == 0) {
+          record_error(a.status, LSA_ERR_TIMEOUT, r, 22);
+          *abort_flag = 1;
+        }
+        *last_flag = static_cast<int>(v);
+      }
+      asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");  // the producer warps
+      sel_state = static_cast<uint32_t>(*last_flag);
+      if (sel_state == 1) {
+        // this split's entries, compacted from the segments that hold them
+        // (the chunk buffers are idle until the first gather)
+        split_entries(TL.segoff + static_cast<int64_t>(r) * (tk::kMaxSeg + 1),
+                      TL.bitmap + static_cast<int64_t>(r) * TL.words, TL.words, a.tk_nseg, a.tk_seg_len, j0, j1, rtab,
+                      kvs, t);
+        if (a.idx_w && half == 0)
+          for (int e = t; e < n_ent; e += kProdThreads) a.idx_w[static_cast<int64_t>(r) * a.k + j0 + e] = rtab[e];
+        fill_rows(rtab, bt, ad.max_blocks, ad.block_size, ad.n_blocks, static_cast<int64_t>(rc.b) * ad.max_len, rc.L,
+                  rc.ok, a.status, r, 0, 0, n_ent, t, kProdThreads, half == 0, rtab, true);
+        asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");  // the producer warps
+      } else if (sel_state == 0) {
+        for (int e = t; e < kRowTab; e += kProdThreads) rtab[e] = -1;
+        asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");  // the producer warps
+      }
+    } else if (a.row_ready) {
       // decode step, launched early: wait for this row's selection only
       if (t == 0 && !wait_flag(a.row_ready + r)) {
         record_error(a.status, LSA_ERR_TIMEOUT, r, 21);
@@ -409,7 +525,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     } else {
       tc::griddep_wait();  // launched early in a decode step: the selection is complete from here on
     }
-    fill_table(0);
+    if (sel_state == 2) fill_table(0);
     prefetch_l2(0, 0);
     prefetch_l2(1, 0);
 #pragma unroll 1
@@ -463,7 +579,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA issuer
-    if (!a.row_ready) tc::griddep_wait();
+    if (!handoff) tc::griddep_wait();
     if (lane == 0 && nch > 0) {
       bool ok = tc::mbar_wait(qfull, 0, abort_flag);
       tc::fence_proxy_async_smem();
@@ -556,7 +672,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
     // 0-287 (lanes 16-31 of those columns, O's, get zeros: the first P V
     // overwrites them).  In a decode step q is an input of the step, so it is
     // loaded while the top-k may still run.
-    if (!a.q_early && !a.row_ready) tc::griddep_wait();
+    if (!a.q_early && !handoff) tc::griddep_wait();
     {
       const uint4* qsrc = reinterpret_cast<const uint4*>(
           reinterpret_cast<const uint8_t*>(a.q) +
@@ -582,7 +698,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qfull);
     }
-    if (a.q_early && !a.row_ready) tc::griddep_wait();
+    if (a.q_early && !handoff) tc::griddep_wait();
     const float c2 = a.scale * kLog2e;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;

@@ -83,11 +83,18 @@ struct TopkArgs {
   // each row's selection then raises its flag in the layout's sel_done.
   const uint32_t* wait_ctr = nullptr;
   uint32_t wait_target = 0;
+  // Decode step: the row's last collect CTA runs the split select (exact
+  // bitmap and per-segment offsets, flag selready = 1) instead of writing idx
+  // (or, when the split select cannot, the full select, flag 2).
+  bool split_select = false;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 // The decode step's handoff words inside the top-k workspace (zeroed with its
 // head): the count of finished scan CTAs and the per-row selection flags.
 void topk_step_flags(void* ws, int32_t rows, int64_t n_cols, uint32_t** scan_done, uint32_t** sel_done);
+// Collect segments per row and their length of the one-launch top-k for these
+// sizes; false on a CUDA error.
+bool topk_rows_plan(int32_t rows, int64_t n_cols, int* nseg, int64_t* seg_len);
 // The three-launch top-k applies (rows up to 2^19 entries); its first
 // histogram then sits at the start of the top-k workspace, followed by the
 // list counters; topk_hist_zero_bytes of them must be zero before the scan.
@@ -123,6 +130,16 @@ struct AttnArgs {
   // Decode step: the selection of row r may be read once row_ready[r] != 0
   // (raised by the top-k after writing it); null: wait for the kernel before.
   const uint32_t* row_ready = nullptr;
+  // Decode step with the top-k's split select: each CTA compacts its split's
+  // entries from the exact bitmap itself (top-k workspace tk_ws, n_cols score
+  // columns per row in tk_nseg segments of tk_seg_len); idx_w (or null):
+  // where CTAs of the first head half store them.
+  bool split_sel = false;
+  void* tk_ws = nullptr;
+  int64_t tk_ncols = 0;
+  int tk_nseg = 0;
+  int64_t tk_seg_len = 0;
+  int32_t* idx_w = nullptr;
 };
 size_t attn_simt_ws_bytes(int32_t rows, int32_t H, int32_t Dv, int32_t k);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
@@ -130,6 +147,9 @@ int attn_simt_launches(int32_t rows, int32_t H, int32_t k);
 bool attn_tc_shape_ok(int32_t dtype, int32_t H, int32_t D, int32_t Dv, int32_t block_size);
 int attn_tc_launches(int32_t rows, int32_t H, int32_t k);
 bool attn_tc_supported(const AttnArgs& a);
+// Whether each split of the tensor-core attention holds at most one row table
+// of entries (needed for it to compact its entries itself).
+bool attn_tc_split_fits(int32_t rows, int32_t k);
 size_t attn_tc_ws_bytes(int32_t rows, int32_t H, int32_t D, int32_t Dv, int32_t k);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);
 // exact merge of per-split softmax partials (shared by both attention paths)

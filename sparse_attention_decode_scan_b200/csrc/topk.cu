@@ -368,7 +368,9 @@ __global__ void __launch_bounds__(tk::kCollectThreads, 2) k_tk_rows(TopkArgs a, 
     tc::griddep_wait();  // launched early in a decode step: the scores are complete from here on
   }
   tc::griddep_launch_dependents();
-  tk::tk_collect_cta<2>(a, seg_len, blockIdx.x, r, S);
+  if (threadIdx.x == 0) S.s_keff = 0;  // what an empty segment leaves (the row's last CTA may be one)
+  __syncthreads();
+  const bool collected = tk::tk_collect_cta<2>(a, seg_len, blockIdx.x, r, S, a.split_select);
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();  // this CTA's bitmap words and candidates before its count
@@ -378,6 +380,19 @@ __global__ void __launch_bounds__(tk::kCollectThreads, 2) k_tk_rows(TopkArgs a, 
   __syncthreads();
   if (!s_last) return;
   __threadfence();  // the other segments' writes, read through L2 by the select
+  if (a.split_select) {
+    // decode step: exact bitmap and segment offsets for the attention's own
+    // compaction, or (when that cannot be done) the full select into idx
+    // (its keff, threshold bin and rank are this CTA's own, from its collect)
+    const bool split = collected && tk::tk_split_select<tk::kCollectThreads, 3>(
+                                        a, r, nseg, seg_len, S.s_keff, static_cast<uint32_t>(S.s_bin), S.s_rank, fsm, S);
+    if (!split) tk::tk_final_cta<tk::kCollectThreads, 3>(a, r, fsm, S);
+    __threadfence();  // this thread's marks, offsets or selection writes
+    __syncthreads();
+    if (threadIdx.x == 0)
+      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(L.selready + r), "r"(split ? 1u : 2u) : "memory");
+    return;
+  }
   tk::tk_final_cta<tk::kCollectThreads, 3>(a, r, fsm, S);
   if (a.wait_ctr) {
     // decode step: the attention of row r may read its selection from now on
@@ -430,6 +445,35 @@ bool topk_v2_ok(int64_t n_cols) { return n_cols <= tk::kMaxBitmapCols; }
 
 size_t topk_hist_zero_bytes(int32_t rows) { return tk::tk_zero_bytes(rows); }
 
+// Shared memory of a k_tk_rows launch (raising the kernel's limit once) and
+// its segment plan.
+cudaError_t rows_plan(int32_t rows, int64_t n_cols, size_t* smem_out, TopkPlan* plan) {
+  size_t smem = tk::tk_final_smem(n_cols, tk::kCollectThreads);
+  if (tk::tk_split_smem() > smem) smem = tk::tk_split_smem();
+  static size_t smem_set = 0;
+  if (smem > 48 * 1024 && smem > smem_set) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k_tk_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    smem_set = smem;
+  }
+  *smem_out = smem;
+  *plan = topk_collect_plan(rows, n_cols, rows_ctas_per_sm(smem) * device_sms());
+  return cudaSuccess;
+}
+
+bool topk_rows_plan(int32_t rows, int64_t n_cols, int* nseg, int64_t* seg_len) {
+  size_t smem;
+  TopkPlan p;
+  if (rows_plan(rows, n_cols, &smem, &p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  *nseg = p.nseg;
+  *seg_len = p.seg_len;
+  return true;
+}
+
 void topk_step_flags(void* ws, int32_t rows, int64_t n_cols, uint32_t** scan_done, uint32_t** sel_done) {
   const tk::TkLayout L = tk::tk_layout(ws, rows, n_cols);
   *scan_done = L.scan_done;
@@ -473,14 +517,10 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
       if (e != cudaSuccess) return e;
       k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
     }
-    const size_t smem = tk::tk_final_smem(a.n_cols, tk::kCollectThreads);
-    static size_t smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
-      e = cudaFuncSetAttribute(k_tk_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      smem_set = smem;
-    }
-    const TopkPlan cp = topk_collect_plan(a.rows, a.n_cols, rows_ctas_per_sm(smem) * device_sms());
+    size_t smem;
+    TopkPlan cp;
+    e = rows_plan(a.rows, a.n_cols, &smem, &cp);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(cp.nseg), static_cast<unsigned>(a.rows));

@@ -22,6 +22,8 @@ constexpr int kWordElems = 32;           // positions per bitmap word (one threa
 constexpr int kCollectThreads = 256;
 constexpr int kColRound = kCollectThreads * kWordElems;  // positions per collect round (8192)
 constexpr int kCtrlInts = 64;            // control words of the fused step (grid barrier) before the counters
+constexpr int kMaxSeg = static_cast<int>(kMaxBitmapCols / kColRound);  // collect segments per row at most
+constexpr int kTieCap = 256;             // keys equal to the threshold a split select ranks itself
 
 __host__ __device__ inline size_t al256(size_t b) { return (b + 255) / 256 * 256; }
 
@@ -30,7 +32,8 @@ __host__ __device__ inline size_t al256(size_t b) { return (b + 255) / 256 * 256
 // split counters; per-row counts of finished collect CTAs; per-row selection
 // flags) |
 // [rows][words] bitmaps of the keys above the threshold bin | [rows][kCandCap]
-// candidates (key, position).  The first three are zeroed before each use.
+// candidates (key, position) | per-segment counts and selection offsets.  The
+// first three are zeroed before each use.
 struct TkLayout {
   uint32_t* hist;
   uint32_t* ncand;
@@ -38,13 +41,16 @@ struct TkLayout {
   uint32_t* row_done;  // per row: collect CTAs finished (the last one selects)
   uint32_t* sel_done;  // per row: 1 once the row's selection is written (decode step)
   uint32_t* scan_done; // scan CTAs finished (decode step)
+  uint32_t* selready;  // per row: 1 once segoff and the marked bitmap are final, 2 once idx is (decode step)
   uint32_t* bitmap;
   uint2* cand;
+  uint32_t* segcnt;    // [rows][kMaxSeg]: keys above the threshold bin per collect segment
+  uint32_t* segoff;    // [rows][kMaxSeg + 1]: first selection entry of each segment, then keff
   int64_t words;
 };
 
 __host__ __device__ inline size_t tk_ctrl_bytes(int32_t rows) {
-  return al256((static_cast<size_t>(kCtrlInts) + 4 * static_cast<size_t>(rows)) * 4);
+  return al256((static_cast<size_t>(kCtrlInts) + 5 * static_cast<size_t>(rows)) * 4);
 }
 
 __host__ __device__ inline size_t tk_zero_bytes(int32_t rows) {
@@ -63,16 +69,22 @@ __host__ __device__ inline TkLayout tk_layout(void* ws, int32_t rows, int64_t n_
   L.row_done = L.ctrl + kCtrlInts + 2 * rows;
   L.sel_done = L.ctrl + kCtrlInts + 3 * rows;
   L.scan_done = L.ctrl + 1;
+  L.selready = L.ctrl + kCtrlInts + 4 * rows;
   b += tk_ctrl_bytes(rows);
   L.bitmap = reinterpret_cast<uint32_t*>(b);
   b += al256(static_cast<size_t>(rows) * L.words * 4);
   L.cand = reinterpret_cast<uint2*>(b);
+  b += al256(static_cast<size_t>(rows) * kCandCap * 8);
+  L.segcnt = reinterpret_cast<uint32_t*>(b);
+  b += al256(static_cast<size_t>(rows) * kMaxSeg * 4);
+  L.segoff = reinterpret_cast<uint32_t*>(b);
   return L;
 }
 
 __host__ __device__ inline size_t tk_ws_bytes(int32_t rows, int64_t n_cols) {
   const size_t R = static_cast<size_t>(rows);
-  return tk_zero_bytes(rows) + al256(R * ((n_cols + 31) / 32) * 4) + al256(R * kCandCap * 8);
+  return tk_zero_bytes(rows) + al256(R * ((n_cols + 31) / 32) * 4) + al256(R * kCandCap * 8) +
+         al256(R * kMaxSeg * 4) + al256(R * (kMaxSeg + 1) * 4);
 }
 
 // Shared scratch of the bodies (static in the standalone kernels, carved from
@@ -82,6 +94,7 @@ struct TkScratch {
   int s_bin;
   uint32_t s_rank;
   uint32_t s_base;
+  uint32_t s_keff;
   uint32_t h[1024];
 };
 
@@ -199,9 +212,13 @@ __device__ __forceinline__ void tk_round_load(const float* row, int base, int li
 // per CTA and round).  The first round's scores are requested before the
 // histogram is read, and each next round's before this round's atomic.
 // Segments are multiples of kColRound positions and cover [0, n_cols), so every
-// bitmap word is written.
+// bitmap word is written.  With count_above, the segment's count of keys above
+// b1 goes to segcnt (a split select's offsets); S keeps keff, b1 and the rank
+// wanted in b1.  Returns false for an
+// empty segment (S then holds nothing of the row).
 template <int ID>
-__device__ void tk_collect_cta(const TopkArgs& a, int64_t seg_len, int seg, int r, TkScratch& S) {
+__device__ bool tk_collect_cta(const TopkArgs& a, int64_t seg_len, int seg, int r, TkScratch& S,
+                               bool count_above = false) {
   constexpr int NT = kCollectThreads;
   static_assert(NT * kWordElems == kColRound && kColRound == (NT / 32) * 1024, "collect round shape");
   static_assert(kMaxBitmapCols <= (1 << 30), "positions fit 32 bits");
@@ -214,7 +231,10 @@ __device__ void tk_collect_cta(const TopkArgs& a, int64_t seg_len, int seg, int 
   const int s0 = seg * static_cast<int>(seg_len);
   const int s1 = s0 + static_cast<int>(seg_len) < static_cast<int>(a.n_cols) ? s0 + static_cast<int>(seg_len)
                                                                               : static_cast<int>(a.n_cols);
-  if (s0 >= s1) return;
+  if (s0 >= s1) {
+    if (threadIdx.x == 0 && seg < kMaxSeg) tk_layout(a.ws, a.rows, a.n_cols).segcnt[r * kMaxSeg + seg] = 0;
+    return false;
+  }
   const int lim = ((n + 3) & ~3) < a.ld ? ((n + 3) & ~3) : static_cast<int>(a.ld);
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
   ColRound cur;
@@ -226,8 +246,10 @@ __device__ void tk_collect_cta(const TopkArgs& a, int64_t seg_len, int seg, int 
   const uint32_t total = tk_find<NT, ID, kB1>(hv, static_cast<uint32_t>(a.k), S, true);
   const uint32_t keff = total < static_cast<uint32_t>(a.k) ? total : static_cast<uint32_t>(a.k);
   const uint32_t b1 = keff > 0 ? static_cast<uint32_t>(S.s_bin) : 0xffffffffu;  // none: no bin qualifies
+  if (threadIdx.x == 0) S.s_keff = keff;  // with S.s_bin and S.s_rank: the row's threshold bin and rank in it
   uint32_t* bitmap = L.bitmap + static_cast<int64_t>(r) * L.words;
   uint2* cand = L.cand + static_cast<int64_t>(r) * kCandCap;
+  int above = 0;  // this thread's keys above the threshold bin
 #pragma unroll 1
   for (int base = s0; base < s1; base += kColRound) {
     const int p0 = base + warp * 1024 + lane * 4;
@@ -261,6 +283,7 @@ __device__ void tk_collect_cta(const TopkArgs& a, int64_t seg_len, int seg, int 
                           (spread8(bal[3] >> sh) << 3);
     const int wi = (base + warp * 1024) / kWordElems + lane;
     if (wi < L.words) bitmap[wi] = word;
+    above += __popc(word);
     int tot;
     const int off = tk_excl_scan<NT, ID>(nc, S.warp_sums, &tot);
     if (threadIdx.x == 0) S.s_base = tot ? atomicAdd(L.ncand + r, static_cast<uint32_t>(tot)) : 0u;
@@ -282,6 +305,12 @@ __device__ void tk_collect_cta(const TopkArgs& a, int64_t seg_len, int seg, int 
       }
     }
   }
+  if (count_above) {  // the segment's keys above the threshold bin
+    int above_tot;
+    tk_excl_scan<NT, ID>(above, S.warp_sums, &above_tot);
+    if (threadIdx.x == 0 && seg < kMaxSeg) L.segcnt[r * kMaxSeg + seg] = static_cast<uint32_t>(above_tot);
+  }
+  return true;
 }
 
 // keeps the n lowest set bits of x
@@ -316,6 +345,56 @@ __host__ __device__ inline size_t tk_final_smem(int64_t n_cols, int nt) {
   const TkPad p = tk_pad(n_cols, nt);
   const size_t bm_words = static_cast<size_t>(nt) * p.stride;
   return 2 * ((bm_words + 1) / 2 * 2) * 4 + static_cast<size_t>(kCandCap) * 8;
+}
+
+// Radix select on key bits [19:10] then [9:0] among the keys of bin b1: the
+// key T of the rank1-th largest key of the bin, and how many keys equal to T
+// (`ties`, the lowest positions first) are still wanted.  The keys are the
+// candidates cs[0, nc), or with `overflow` the row's scores (n of them).
+template <int NT, int ID>
+__device__ void tk_radix_T(const uint2* cs, int nc, bool overflow, const float* row, int64_t n, uint32_t b1,
+                           uint32_t rank1, TkScratch& S, uint32_t* T_out, uint32_t* ties_out) {
+  const int t = threadIdx.x % NT;
+  uint32_t T = 0, ties = 0;
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int i = t; i < 1024; i += NT) S.h[i] = 0;
+    tk_sync<NT, ID>();
+    const uint32_t shift = pass == 0 ? 10 : 0;
+    const uint32_t pre_shift = pass == 0 ? 20 : 10;
+    const uint32_t prefix = pass == 0 ? b1 : (T >> 10);
+    if (!overflow) {
+      for (int c = t; c < nc; c += NT) {
+        const uint32_t key = cs[c].x;
+        if ((key >> pre_shift) == prefix) atomicAdd(&S.h[(key >> shift) & 1023u], 1u);
+      }
+    } else {
+      for (int64_t base = 0; base < n; base += NT * 4) {
+        const int64_t p = base + t * 4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (p + j >= n) break;
+          const uint32_t key = order_key(__ldcg(row + p + j));
+          if (key && (key >> pre_shift) == prefix) atomicAdd(&S.h[(key >> shift) & 1023u], 1u);
+        }
+      }
+    }
+    tk_sync<NT, ID>();
+    uint32_t hl[1024 / NT];
+#pragma unroll
+    for (int i = 0; i < 1024 / NT; ++i) hl[i] = S.h[t * (1024 / NT) + i];
+    tk_find<NT, ID, 1024>(hl, pass == 0 ? rank1 : ties, S, false);
+    const uint32_t bb = static_cast<uint32_t>(S.s_bin);
+    if (pass == 0) {
+      T = (b1 << 20) | (bb << 10);
+      ties = S.s_rank;
+    } else {
+      T |= bb;
+      ties = S.s_rank;
+    }
+    tk_sync<NT, ID>();
+  }
+  *T_out = T;
+  *ties_out = ties;
 }
 
 // The select of row r: keff and b1 from the histogram, the bitmap of the keys
@@ -384,43 +463,7 @@ __device__ void tk_final_cta(const TopkArgs& a, int r, uint32_t* fsm, TkScratch&
   if (keff == 0) return;
   // radix select on bits [19:10] then [9:0] among the keys of bin b1
   uint32_t T = 0, ties = 0;
-  for (int pass = 0; pass < 2; ++pass) {
-    for (int i = t; i < 1024; i += NT) S.h[i] = 0;
-    tk_sync<NT, ID>();
-    const uint32_t shift = pass == 0 ? 10 : 0;
-    const uint32_t pre_shift = pass == 0 ? 20 : 10;
-    const uint32_t prefix = pass == 0 ? b1 : (T >> 10);
-    if (!overflow) {
-      for (int c = t; c < nc; c += NT) {
-        const uint32_t key = cs[c].x;
-        if ((key >> pre_shift) == prefix) atomicAdd(&S.h[(key >> shift) & 1023u], 1u);
-      }
-    } else {
-      for (int64_t base = 0; base < n; base += NT * 4) {
-        const int64_t p = base + t * 4;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (p + j >= n) break;
-          const uint32_t key = order_key(__ldcg(row + p + j));
-          if (key && (key >> pre_shift) == prefix) atomicAdd(&S.h[(key >> shift) & 1023u], 1u);
-        }
-      }
-    }
-    tk_sync<NT, ID>();
-    uint32_t hl[1024 / NT];
-#pragma unroll
-    for (int i = 0; i < 1024 / NT; ++i) hl[i] = S.h[t * (1024 / NT) + i];
-    tk_find<NT, ID, 1024>(hl, pass == 0 ? rank1 : ties, S, false);
-    const uint32_t bb = static_cast<uint32_t>(S.s_bin);
-    if (pass == 0) {
-      T = (b1 << 20) | (bb << 10);
-      ties = S.s_rank;
-    } else {
-      T |= bb;
-      ties = S.s_rank;
-    }
-    tk_sync<NT, ID>();
-  }
+  tk_radix_T<NT, ID>(cs, nc, overflow, row, n, b1, rank1, S, &T, &ties);
   // mark keys of bin b1 above T, and collect the keys equal to T
   if (!overflow) {
     for (int c = t; c < nc; c += NT) {
@@ -492,6 +535,88 @@ __device__ void tk_final_cta(const TopkArgs& a, int r, uint32_t* fsm, TkScratch&
     for (int i = t; i < n_out; i += NT) out[i] = os[i];
   }
   tk_sync<NT, ID>();  // shared memory free for the caller's next use
+}
+
+// Split select of row r, run by the row's last collect CTA in a decode step
+// (NT threads; fsm: shared memory of at least tk_split_smem() bytes, 8-byte
+// aligned).  Instead of compacting the row's selection it makes the row's
+// bitmap exact (marks the threshold bin's keys above T and the `ties` lowest
+// positions equal to T) and stores, per collect segment, the first selection
+// entry it holds (segoff[r][s], then keff at [nseg]): a consumer of entries
+// [e0, e1) then compacts only the segments those entries fall in.  Returns
+// false, having changed nothing a full select relies on, when the candidates
+// overflowed their list or more than kTieCap keys equal T; the caller then
+// runs the full select.
+__host__ __device__ inline size_t tk_split_smem() {
+  return (static_cast<size_t>(kMaxSeg) + kTieCap + 8) * 4 + static_cast<size_t>(kCandCap) * 8;
+}
+
+template <int NT, int ID>
+__device__ bool tk_split_select(const TopkArgs& a, int r, int nseg, int64_t seg_len, uint32_t keff, uint32_t b1,
+                                uint32_t rank1, uint32_t* fsm, TkScratch& S) {
+  const int t = threadIdx.x % NT;
+  const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
+  uint32_t* seg_add = fsm;                              // [kMaxSeg]
+  uint32_t* eqpos = fsm + kMaxSeg;                      // [kTieCap]
+  uint32_t* s_eq = fsm + kMaxSeg + kTieCap;             // count of keys equal to T
+  uint2* cs = reinterpret_cast<uint2*>(fsm + kMaxSeg + kTieCap + 8);
+  uint32_t* segoff = L.segoff + static_cast<int64_t>(r) * (kMaxSeg + 1);
+  if (keff == 0) {
+    for (int i = t; i <= nseg; i += NT) segoff[i] = 0;
+    return true;
+  }
+  const uint32_t n_cand = __ldcg(L.ncand + r);
+  if (n_cand > static_cast<uint32_t>(kCandCap)) return false;
+  const int nc = static_cast<int>(n_cand);
+  for (int c0 = t; c0 < nc; c0 += 4 * NT) {
+    uint2 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      v[u] = c0 + u * NT < nc ? __ldcg(L.cand + static_cast<int64_t>(r) * kCandCap + c0 + u * NT) : make_uint2(0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (c0 + u * NT < nc) cs[c0 + u * NT] = v[u];
+  }
+  for (int i = t; i < kMaxSeg; i += NT) seg_add[i] = 0;
+  if (t == 0) *s_eq = 0;
+  uint32_t T, ties;
+  tk_radix_T<NT, ID>(cs, nc, false, nullptr, 0, b1, rank1, S, &T, &ties);  // its barriers publish the above
+  // keys equal to T: their positions, to rank (ties are broken by lowest position)
+  for (int c = t; c < nc; c += NT) {
+    if (cs[c].x == T) {
+      const uint32_t i = atomicAdd(s_eq, 1u);
+      if (i < static_cast<uint32_t>(kTieCap)) eqpos[i] = cs[c].y;
+    }
+  }
+  tk_sync<NT, ID>();
+  const int n_eq = static_cast<int>(*s_eq);
+  if (n_eq > kTieCap) return false;  // nothing marked yet
+  uint32_t* bitmap = L.bitmap + static_cast<int64_t>(r) * L.words;
+  for (int c = t; c < nc; c += NT) {
+    const uint2 e = cs[c];
+    if (e.x > T) {
+      atomicOr(bitmap + (e.y >> 5), 1u << (e.y & 31));
+      atomicAdd(seg_add + e.y / static_cast<uint32_t>(seg_len), 1u);
+    }
+  }
+  for (int i = t; i < n_eq; i += NT) {
+    const uint32_t p = eqpos[i];
+    int rank = 0;
+    for (int j = 0; j < n_eq; ++j) rank += eqpos[j] < p ? 1 : 0;
+    if (rank < static_cast<int>(ties)) {
+      atomicOr(bitmap + (p >> 5), 1u << (p & 31));
+      atomicAdd(seg_add + p / static_cast<uint32_t>(seg_len), 1u);
+    }
+  }
+  tk_sync<NT, ID>();
+  // first entry of each segment: keys above the bin plus the marked ones, scanned
+  const uint32_t mine = t < nseg ? __ldcg(L.segcnt + r * kMaxSeg + t) + seg_add[t] : 0u;
+  int total;
+  const int before = tk_excl_scan<NT, ID>(static_cast<int>(mine), S.warp_sums, &total);
+  if (t < nseg) segoff[t] = static_cast<uint32_t>(before);
+  if (t == 0) segoff[nseg] = static_cast<uint32_t>(total);
+  if (t == 0 && total != static_cast<int>(keff)) record_error(a.status, LSA_ERR_BOUNDS, r, total);  // cannot happen
+  return true;
 }
 
 }  // namespace tk

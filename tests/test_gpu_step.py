@@ -191,3 +191,52 @@ def test_decode_step_selection_equals_separate_calls(name):
     lsa.topk(scores, k, idx, ws, valid_len=dc.seq_lens, n_cols=dc.max_len, ld=ld)
     torch.cuda.synchronize()
     assert torch.equal(idx, idx_step)
+
+
+def _split_case():
+    """Decode case for the split select: 4 sequences of 5000-6000 tokens (k = 512)
+    where sequence 0 is cut to 200 tokens whose keys are all one key (every
+    score equal: 200 ties at the threshold, ranked by the split select itself)
+    and sequence 1 keeps its length with all keys equal too (more ties than the
+    split select ranks: the row falls back to the full select)."""
+    from sparse_attention_decode_scan_b200 import synth
+    spec = synth.scaled(cases.C[3], batch=4, len_lo=5000, len_hi=6000, top_k=512)
+    case = synth.make_case(spec, 7101)
+    bs = spec.block_size
+    case.seq_lens[0] = 200
+    for b in (0, 1):
+        first = case.block_table[b][0]
+        key = case.idx_keys[first, 0].copy()
+        for p in range(int(case.seq_lens[b])):
+            case.idx_keys[case.block_table[b][p // bs], p % bs] = key
+    return case
+
+
+@pytest.mark.parametrize("min_cols", ["0", "100000000"])
+def test_decode_step_split_select(min_cols, monkeypatch):
+    """With the split select forced on (rows of any length) or off, the decode
+    step selects what lsa_indexer_scores + lsa_topk select, ties and the
+    fallback row included, and its outputs match the oracle."""
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+    monkeypatch.setenv("LSA_SPLIT_SELECT_MIN_COLS", min_cols)
+    case = _split_case()
+    dc = DeviceCase(case)
+    _, _, idx_step = _step(dc)
+    B, k = dc.rows, dc.spec.top_k
+    ld = (dc.max_len + 3) // 4 * 4
+    scores = torch.empty((B, ld), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.workspace_size(dc.dims, B, dc.max_len, lsa.LSA_OP_DECODE_STEP))
+    lsa.indexer_scores(dc.dims, dc.cache, dc.q_idx, dc.w, scores, ld, ws)
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    lsa.topk(scores, k, idx, ws, valid_len=dc.seq_lens, n_cols=dc.max_len, ld=ld)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_step)
+    # all-equal rows keep the lowest positions
+    assert (idx_step[0, :200].cpu().numpy() == np.arange(200)).all() and (idx_step[0, 200:] == -1).all()
+    assert (idx_step[1].cpu().numpy() == np.arange(k)).all()
+    _check_step(case, list(range(B)))
+    # unfused and fused agree bit for bit (the fused step never splits)
+    o1, l1, i1 = _step(dc, 0)
+    o2, l2, i2 = _step(dc, 1)
+    assert torch.equal(i1, i2) and torch.equal(o1, o2) and torch.equal(l1, l2)
