@@ -238,6 +238,40 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* o, const float (&v)
   }
 }
 
+// Merge weights of the heads [hl0, hl1) of one (row, half): the ns split lse
+// values (load(s, hl)) are gathered into wsm[s][hl] by one thread per pair,
+// then one thread per head turns them into w[s][hl] = exp(lse_s - m) /
+// sum_s' exp(lse_s' - m), m the largest, the sum taken in ascending split
+// order; the slice that holds a head's first group (hl * 128 >= i0) also
+// writes the head's merged lse to lse_row[hl].  The loops are kept rolled:
+// this code runs once per CTA, on a cold instruction cache.
+template <class Load>
+__device__ __forceinline__ void merge_weights(int ns, int hl0, int hl1, int i0, Load load, float* wsm,
+                                              float* lse_row) {
+  const int nh = hl1 - hl0;
+  for (int i = static_cast<int>(threadIdx.x); i < ns * nh; i += kThreads) {
+    const int s = i / nh, hl = hl0 + i % nh;
+    wsm[s * kHeadsCta + hl] = load(s, hl);
+  }
+  __syncthreads();
+  for (int hl = hl0 + static_cast<int>(threadIdx.x); hl < hl1; hl += kThreads) {
+    float mx = -INFINITY;
+#pragma unroll 1
+    for (int s = 0; s < ns; ++s) mx = fmaxf(mx, wsm[s * kHeadsCta + hl]);
+    float den = 0.f;
+#pragma unroll 1
+    for (int s = 0; s < ns; ++s) {
+      const float e = mx != -INFINITY ? exp2f((wsm[s * kHeadsCta + hl] - mx) * kLog2e) : 0.f;
+      wsm[s * kHeadsCta + hl] = e;
+      den += e;
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll 1
+    for (int s = 0; s < ns; ++s) wsm[s * kHeadsCta + hl] *= inv;
+    if (lse_row && hl * (kDv / 4) >= i0) lse_row[hl] = den > 0.f ? mx + logf(den) : -INFINITY;
+  }
+}
+
 // out[r][half*64 + g/128][4(g%128) .. +3] = sum_s w[s][head] * part_o[r][s][..]
 // for the groups g in [i0, i1) of one (row, half), U groups per thread and
 // pass with the loads of V splits in flight together; w in shared memory
@@ -893,32 +927,9 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       float* wsm = reinterpret_cast<float*>(kvs);  // [nsplit][64] in the idle chunk buffer, nsplit <= 32
       const float* lse_p = P.part_lse + static_cast<int64_t>(r) * ns * kHeadsAll + half * kHeadsCta;
       const int hl0 = i0 / (kDv / 4), hl1 = i1 > i0 ? (i1 - 1) / (kDv / 4) + 1 : hl0;
-      // one warp per head, one lane per split (nsplit <= 32); a warp's heads'
-      // lse loads are all issued before the first is used
-      constexpr int kHeadsPerWarp = (kHeadsCta + kThreads / 32 - 1) / (kThreads / 32);
-      float lv[kHeadsPerWarp];
-#pragma unroll
-      for (int x = 0; x < kHeadsPerWarp; ++x) {
-        const int hl = hl0 + warp + x * (kThreads / 32);
-        lv[x] = (hl < hl1 && lane < ns) ? __ldcg(lse_p + lane * kHeadsAll + hl) : -INFINITY;
-      }
-#pragma unroll
-      for (int x = 0; x < kHeadsPerWarp; ++x) {
-        const int hl = hl0 + warp + x * (kThreads / 32);
-        if (hl >= hl1) break;
-        float mx = lv[x];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float e = (lane < ns && mx != -INFINITY) ? exp2f((lv[x] - mx) * kLog2e) : 0.f;
-        float den = e;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        if (lane < ns) wsm[lane * kHeadsCta + hl] = e * inv;
-        // the slice holding a head's first group writes its lse
-        if (lane == 0 && a.lse && hl * (kDv / 4) >= i0)
-          a.lse[static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + hl] = den > 0.f ? mx + logf(den) : -INFINITY;
-      }
+      merge_weights(
+          ns, hl0, hl1, i0, [&](int s2, int hl) { return __ldcg(lse_p + s2 * kHeadsAll + hl); }, wsm,
+          a.lse ? a.lse + static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta : nullptr);
       __syncthreads();
       // About 16 loads in flight per thread: 8 groups x 2 splits when the slice
       // is large (few splits), 1 group x 16 splits when it is small (many)
@@ -953,36 +964,15 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
       float* wsm = reinterpret_cast<float*>(kvs + kHeadsCta * kDv * 4);
       const int hl0 = i0 / (kDv / 4), hl1 = i1 > i0 ? (i1 - 1) / (kDv / 4) + 1 : hl0;
       const uint32_t slse_u = tc::smem_u32(slse);
-      // one warp per head, one lane per split (nsplit <= 32); a warp's lse
-      // loads are all issued before the first is used
-      constexpr int kHeadsPerWarp = (kHeadsCta + kThreads / 32 - 1) / (kThreads / 32);
-      float lv[kHeadsPerWarp];
-      const uint32_t peer_lse = lane < ns ? tc::cluster_map(slse_u, static_cast<uint32_t>(lane)) : 0u;
-#pragma unroll
-      for (int x = 0; x < kHeadsPerWarp; ++x) {
-        const int hl = hl0 + warp + x * (kThreads / 32);
-        lv[x] = (hl < hl1 && lane < ns) ? tc::ld_cluster_f32(peer_lse + hl * 4) : -INFINITY;
-      }
-#pragma unroll
-      for (int x = 0; x < kHeadsPerWarp; ++x) {
-        const int hl = hl0 + warp + x * (kThreads / 32);
-        if (hl >= hl1) break;
-        float mx = lv[x];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float e = (lane < ns && mx != -INFINITY) ? exp2f((lv[x] - mx) * kLog2e) : 0.f;
-        float den = e;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        if (lane < ns) wsm[lane * kHeadsCta + hl] = e * inv;
-        // the slice holding a head's first group writes its lse
-        if (lane == 0 && a.lse && hl * (kDv / 4) >= i0)
-          a.lse[static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta + hl] = den > 0.f ? mx + logf(den) : -INFINITY;
-      }
+      merge_weights(
+          ns, hl0, hl1, i0,
+          [&](int s2, int hl) {
+            return tc::ld_cluster_f32(tc::cluster_map(slse_u, static_cast<uint32_t>(s2)) + static_cast<uint32_t>(hl) * 4u);
+          },
+          wsm, a.lse ? a.lse + static_cast<int64_t>(r) * kHeadsAll + half * kHeadsCta : nullptr);
       __syncthreads();
       const uint32_t stg_u = tc::smem_u32(kvs);
-      constexpr int U = 8;  // groups per thread and pass, loads in flight together
+      constexpr int U = 4;  // groups per thread and pass, loads in flight together (more: longer cold code)
 #pragma unroll 1
       for (int it0 = i0 + threadIdx.x; it0 < i1; it0 += U * kThreads) {
         float4 acc[U];
