@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of one DSA decode step (indexer scan -> top-k -> sparse MQA) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 Default workload: batched paged decode, B=32 sequences with lengths drawn
 uniformly in [65536, 131072], 64-token blocks under a random block permutation,
@@ -48,9 +48,9 @@ def dist_env():
     return ws, rank, local
 
 
-def rank_seed(cfg: int, rank: int) -> int:
+def rank_seed(spec, rank: int) -> int:
     """Each rank draws its own batch (independent units, weak scaling)."""
-    return synth.seed_of(cfg) + 7919 * rank
+    return synth.seed_of(spec) + 7919 * rank
 
 
 def reduce_max(x: float, group=None) -> float:
@@ -194,8 +194,8 @@ def cpu_oracle_rate(case, rows, repeats: int = 1):
 def run_reference(args, ws_, rank):
     if rank != 0:
         return
-    cfg = args.config
-    case = synth.make_case(synth.CONFIGS[cfg], rank_seed(cfg, 0))
+    spec = synth.workload(args.workload)
+    case = synth.make_case(spec, rank_seed(spec, 0))
     B = case.rows
     per = []
     for i in range(args.warmup + args.steps):
@@ -210,7 +210,7 @@ def run_reference(args, ws_, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec_per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(cfg, case),
+            "data": "synthetic", "config": workload_config(case),
             "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -219,14 +219,14 @@ def run_reference(args, ws_, rank):
 
 # --------------------------------------------------------------------------- our arm
 
-def workload_config(cfg, case):
+def workload_config(case):
     s = case.spec
     c = {"workload": s.name, "batch": case.rows, "seq_len_min": int(case.seq_lens.min()),
          "seq_len_max": int(case.seq_lens.max()), "seq_len_mean": float(case.seq_lens.mean()),
          "block_size": s.block_size, "idx_heads": s.n_idx_heads, "idx_dim": s.idx_dim,
          "idx_key_dtype": s.idx_key_dtype, "top_k": s.top_k, "heads": s.n_heads, "kv_width": s.qk_dim,
          "v_dim": s.v_dim, "parallelism": "replicas (independent batch per GPU)",
-         "l2": "inputs larger than L2 (indexer keys streamed from HBM every step)" if cfg in (3, 4)
+         "l2": "inputs larger than L2 (indexer keys streamed from HBM every step)" if s.streams_past_l2
          else "L2 flushed between steps (256 MB write, outside the kernels' event windows)"}
     return c
 
@@ -239,13 +239,13 @@ def run_ours(args, world, rank, local):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    cfg = args.config
-    spec = synth.CONFIGS[cfg]
+    base = synth.workload(args.workload)
+    spec = base
     if args.batch:
         spec = synth.scaled(spec, batch=args.batch)
     if args.op == "scan":
         spec = synth.scaled(spec, with_kv=False)
-    case = synth.make_case(spec, rank_seed(cfg, rank))
+    case = synth.make_case(spec, rank_seed(base, rank))
     dc = DeviceCase(case, device=dev)
     s = case.spec
     R = dc.rows
@@ -260,7 +260,7 @@ def run_ours(args, world, rank, local):
                    (lsa.LSA_OP_SCORES, lsa.LSA_OP_TOPK, lsa.LSA_OP_ATTN, lsa.LSA_OP_DECODE_STEP))
     ws = lsa.workspace(ws_bytes, device=dev)
     stream = torch.cuda.current_stream(dev)
-    flush = None if cfg in (3, 4) else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = None if base.streams_past_l2 else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     L = int(case.seq_lens[0])
 
     run_scan = args.op in ("step", "scan")
@@ -474,7 +474,7 @@ def run_ours(args, world, rank, local):
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": s.act_dtype if s.idx_key_dtype != "fp8" else "bf16+fp8",
             "data": "synthetic (seeded, generated on host)",
-            "config": dict(workload_config(cfg, case),
+            "config": dict(workload_config(case),
                            step="one cooperative launch (LSA_STEP_FUSED)" if fused else "separate launches"),
             "tokens_per_s": value * R if not prefill else None,
             "step_hbm_gbs": step_gbs, "step_hbm_frac": step_gbs / peaks["hbm_gbs"],
@@ -493,7 +493,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", type=int, default=3, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--workload", default=synth.DECODE_B32,
+                    help="workload name (or a unique prefix of one): " + ", ".join(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     # profiling aids: a smaller batch of the same workload, one stage only, no clock soak

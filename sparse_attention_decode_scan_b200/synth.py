@@ -128,6 +128,16 @@ class Spec:
     chunk: int = 0                 # prefill chunk rows (0 = decode)
     max_len: int = 0               # contiguous row stride; 0 -> len_hi
     with_kv: bool = True
+    seed: int = 0                  # seed of the workload's data
+
+    @property
+    def streams_past_l2(self) -> bool:
+        """The indexer keys of one step (bytes read by the scan) exceed twice
+        the 126 MB L2, so consecutive steps need no L2 flush between them."""
+        per_tok = {"f32": 4, "bf16": 2, "fp8": 1}[self.idx_key_dtype] * self.idx_dim + (
+            4 if self.idx_key_dtype == "fp8" else 0)
+        mean_len = (self.len_lo + self.len_hi) / 2
+        return not self.causal and self.batch * mean_len * per_tok >= 2 * 126e6
 
     @property
     def causal(self) -> bool:
@@ -138,26 +148,44 @@ class Spec:
         return self.max_len or self.len_hi
 
 
-CONFIGS: Dict[int, Spec] = {
-    1: Spec("tiny_fp32_L4096", batch=1, len_lo=4096, len_hi=4096, n_idx_heads=4, idx_dim=64,
-            n_heads=8, qk_dim=64, v_dim=64, top_k=256, act_dtype="f32", idx_key_dtype="f32",
-            w_std=0.5, softmax_scale=1.0 / 8.0),
-    2: Spec("decode_B1_L32K_bf16", batch=1, len_lo=32768, len_hi=32768, n_idx_heads=64,
-            idx_dim=128, n_heads=128, qk_dim=576, v_dim=512, top_k=2048),
-    3: Spec("decode_B32_L64K-128K_paged64_bf16", batch=32, len_lo=65536, len_hi=131072,
-            n_idx_heads=64, idx_dim=128, n_heads=128, qk_dim=576, v_dim=512, top_k=2048,
-            block_size=64),
-    4: Spec("decode_B4_L512K_fp8keys", batch=4, len_lo=524288, len_hi=524288, n_idx_heads=64,
-            idx_dim=128, n_heads=128, qk_dim=576, v_dim=512, top_k=2048, idx_key_dtype="fp8",
-            heavy_frac=0.1, heavy_offset=3.0),
-    5: Spec("prefill_8192x139264_causal_bf16", batch=1, len_lo=139264, len_hi=139264,
-            n_idx_heads=64, idx_dim=128, n_heads=128, qk_dim=576, v_dim=512, top_k=2048,
-            chunk=8192),
-}
+# The benchmark workloads, by name.  Each carries the seed its data is drawn
+# with (every rank adds its own offset).
+TINY = "tiny_fp32_L4096"
+DECODE_B1 = "decode_B1_L32K_bf16"
+DECODE_B32 = "decode_B32_L64K-128K_paged64_bf16"
+DECODE_B4_FP8 = "decode_B4_L512K_fp8keys"
+PREFILL = "prefill_8192x139264_causal_bf16"
+
+WORKLOADS: Dict[str, Spec] = {s.name: s for s in [
+    Spec(TINY, batch=1, len_lo=4096, len_hi=4096, n_idx_heads=4, idx_dim=64,
+         n_heads=8, qk_dim=64, v_dim=64, top_k=256, act_dtype="f32", idx_key_dtype="f32",
+         w_std=0.5, softmax_scale=1.0 / 8.0, seed=1001),
+    Spec(DECODE_B1, batch=1, len_lo=32768, len_hi=32768, n_idx_heads=64,
+         idx_dim=128, n_heads=128, qk_dim=576, v_dim=512, top_k=2048, seed=1002),
+    Spec(DECODE_B32, batch=32, len_lo=65536, len_hi=131072,
+         n_idx_heads=64, idx_dim=128, n_heads=128, qk_dim=576, v_dim=512, top_k=2048,
+         block_size=64, seed=1003),
+    Spec(DECODE_B4_FP8, batch=4, len_lo=524288, len_hi=524288, n_idx_heads=64,
+         idx_dim=128, n_heads=128, qk_dim=576, v_dim=512, top_k=2048, idx_key_dtype="fp8",
+         heavy_frac=0.1, heavy_offset=3.0, seed=1004),
+    Spec(PREFILL, batch=1, len_lo=139264, len_hi=139264,
+         n_idx_heads=64, idx_dim=128, n_heads=128, qk_dim=576, v_dim=512, top_k=2048,
+         chunk=8192, seed=1005),
+]}
 
 
-def seed_of(cfg: int) -> int:
-    return 1000 + cfg
+def workload(name: str) -> Spec:
+    """The workload called `name`, or the only one whose name starts with it."""
+    if name in WORKLOADS:
+        return WORKLOADS[name]
+    hits = [k for k in WORKLOADS if k.startswith(name)]
+    if len(hits) != 1:
+        raise KeyError(f"workload {name!r}: {'ambiguous' if hits else 'unknown'} (one of {sorted(WORKLOADS)})")
+    return WORKLOADS[hits[0]]
+
+
+def seed_of(spec: Spec) -> int:
+    return spec.seed
 
 
 @dataclass
@@ -315,6 +343,7 @@ def flops_prefill_scan(case: Case) -> int:
     return int(2 * s.n_idx_heads * s.idx_dim * int(vis.sum()))
 
 
-__all__ = ["Spec", "Case", "CONFIGS", "make_case", "scaled", "seed_of", "normal", "rng",
+__all__ = ["Spec", "Case", "WORKLOADS", "workload", "TINY", "DECODE_B1", "DECODE_B32", "DECODE_B4_FP8",
+           "PREFILL", "make_case", "scaled", "seed_of", "normal", "rng",
            "to_bf16_bits", "to_e4m3_bits", "topk_scores", "index_lists",
            "nbytes_decode_step", "flops_prefill_scan"]

@@ -52,7 +52,7 @@ def test_version_and_status_strings(lsa):
 def _dims(lsa, **kw):
     from sparse_attention_decode_scan_b200 import synth
     from sparse_attention_decode_scan_b200.device import make_dims
-    d = make_dims(synth.CONFIGS[3])
+    d = make_dims(synth.WORKLOADS[synth.DECODE_B32])
     for k, v in kw.items():
         setattr(d, k, v)
     return d

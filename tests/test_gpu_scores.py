@@ -3,6 +3,7 @@ import numpy as np
 import pytest
 
 from oracle import lsa_oracle as O
+from sparse_attention_decode_scan_b200 import synth
 from tests import cases
 from tests.helpers import SCORE_TOL, check_scores
 
@@ -45,9 +46,9 @@ def test_scores_small(name, path, monkeypatch):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("cfg", [2, 3, 4])
-def test_scores_full_decode(cfg):
-    case = cases.full(cfg, with_kv=False)
+@pytest.mark.parametrize("name", [synth.DECODE_B1, synth.DECODE_B32, synth.DECODE_B4_FP8])
+def test_scores_full_decode(name):
+    case = cases.full(name, with_kv=False)
     scores = _run_scores(case)
     rows = sorted({0, case.rows - 1, case.rows // 2})
     _check_rows(case, scores, rows)
@@ -59,7 +60,7 @@ def test_scores_full_decode(cfg):
 
 @pytest.mark.slow
 def test_scores_full_prefill():
-    case = cases.full(5, with_kv=False)
+    case = cases.full(synth.PREFILL, with_kv=False)
     scores = _run_scores(case)
     g = np.random.default_rng(77)
     rows = sorted({0, 1, case.rows - 2, case.rows - 1, *g.integers(0, case.rows, 4).tolist()})

@@ -3,6 +3,7 @@ import numpy as np
 import pytest
 
 from oracle import lsa_oracle as O
+from sparse_attention_decode_scan_b200 import synth
 from tests import cases
 from tests.helpers import check_attention, check_selection
 
@@ -142,24 +143,24 @@ def test_prefill_chain_small():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("cfg", [2, 3])
-def test_decode_step_full(cfg):
-    case = cases.full(cfg)
+@pytest.mark.parametrize("name", [synth.DECODE_B1, synth.DECODE_B32])
+def test_decode_step_full(name):
+    case = cases.full(name)
     rows = sorted({0, case.rows - 1, case.rows // 2})
     _check_step(case, rows)
 
 
 @pytest.mark.slow
 def test_decode_step_full_fp8():
-    case = cases.full(4)
+    case = cases.full(synth.DECODE_B4_FP8)
     _check_step(case, [0, 3])
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("cfg", [2, 3, 4])
-def test_decode_step_full_fused_bitwise_equals_unfused(cfg):
+@pytest.mark.parametrize("name", [synth.DECODE_B1, synth.DECODE_B32, synth.DECODE_B4_FP8])
+def test_decode_step_full_fused_bitwise_equals_unfused(name):
     from sparse_attention_decode_scan_b200.device import DeviceCase
-    dc = DeviceCase(cases.full(cfg))
+    dc = DeviceCase(cases.full(name))
     o1, l1, i1 = _step(dc, 0)
     o2, l2, i2 = _step(dc, 1)
     assert torch.equal(i1, i2)
@@ -169,7 +170,7 @@ def test_decode_step_full_fused_bitwise_equals_unfused(cfg):
 
 @pytest.mark.slow
 def test_decode_step_full_fused_vs_oracle():
-    case = cases.full(3)
+    case = cases.full(synth.DECODE_B32)
     rows = sorted({0, case.rows - 1, case.rows // 2})
     _check_step(case, rows, flags=1)
 

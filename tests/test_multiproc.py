@@ -31,7 +31,7 @@ def _worker(rank, world, port, q):
         elapsed = 10.0 + 5.0 * rank       # rank 1 is the slow one
         m = bench.reduce_max(elapsed)
         ws, rk, lr = bench.dist_env()
-        q.put((rank, m, bench.rank_seed(3, rank), ws, rk))
+        q.put((rank, m, bench.rank_seed(bench.synth.WORKLOADS[bench.synth.DECODE_B32], rank), ws, rk))
         bench.barrier()
     finally:
         dist.destroy_process_group()
@@ -57,7 +57,7 @@ def test_reference_arm_prints_on_rank0_only(capsys):
     import argparse
 
     import bench
-    args = argparse.Namespace(config=1, steps=1, warmup=3, gpus=2)
+    args = argparse.Namespace(workload=bench.synth.TINY, steps=1, warmup=3, gpus=2)
     bench.run_reference(args, 2, 1)                     # rank 1: no work, no output
     assert capsys.readouterr().out == ""
 

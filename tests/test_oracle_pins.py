@@ -118,7 +118,7 @@ def test_paged_addressing_hand_example():
 
 
 def test_paged_equals_contiguous_on_synthetic_case():
-    spec = synth.scaled(synth.CONFIGS[3], batch=2, len_lo=150, len_hi=300, n_idx_heads=4,
+    spec = synth.scaled(synth.WORKLOADS[synth.DECODE_B32], batch=2, len_lo=150, len_hi=300, n_idx_heads=4,
                         idx_dim=16, n_heads=4, qk_dim=24, v_dim=16, top_k=32, block_size=16)
     case = synth.make_case(spec, 11)
     # rebuild the same logical cache contiguously
@@ -219,7 +219,7 @@ def test_attention_matches_torch_sdpa():
 
 
 def test_sparse_with_k_at_least_L_equals_dense():
-    spec = synth.scaled(synth.CONFIGS[2], len_lo=200, len_hi=200, n_idx_heads=4, idx_dim=16,
+    spec = synth.scaled(synth.WORKLOADS[synth.DECODE_B1], len_lo=200, len_hi=200, n_idx_heads=4, idx_dim=16,
                         n_heads=6, qk_dim=40, v_dim=32, top_k=256)
     case = synth.make_case(spec, 12)
     _, sel, o, lse = O.row_step(case, 0)
@@ -253,7 +253,7 @@ def test_attention_invariants():
 # --------------------------------------------------------------------------- whole step invariants
 
 def test_prefill_rows_are_causal():
-    spec = synth.scaled(synth.CONFIGS[5], len_lo=300, len_hi=300, chunk=40, n_idx_heads=4, idx_dim=16,
+    spec = synth.scaled(synth.WORKLOADS[synth.PREFILL], len_lo=300, len_hi=300, chunk=40, n_idx_heads=4, idx_dim=16,
                         n_heads=4, qk_dim=24, v_dim=16, top_k=64)
     case = synth.make_case(spec, 13)
     for r in [0, 17, 39]:
@@ -266,7 +266,7 @@ def test_prefill_rows_are_causal():
 
 
 def test_selection_size_and_distinctness():
-    spec = synth.scaled(synth.CONFIGS[3], batch=3, len_lo=40, len_hi=300, n_idx_heads=4, idx_dim=16,
+    spec = synth.scaled(synth.WORKLOADS[synth.DECODE_B32], batch=3, len_lo=40, len_hi=300, n_idx_heads=4, idx_dim=16,
                         n_heads=4, qk_dim=24, v_dim=16, top_k=100, block_size=16)
     case = synth.make_case(spec, 14)
     for r in range(3):
