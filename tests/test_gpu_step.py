@@ -201,7 +201,7 @@ def _split_case():
     and sequence 1 keeps its length with all keys equal too (more ties than the
     split select ranks: the row falls back to the full select)."""
     from sparse_attention_decode_scan_b200 import synth
-    spec = synth.scaled(cases.C[3], batch=4, len_lo=5000, len_hi=6000, top_k=512)
+    spec = synth.scaled(synth.WORKLOADS[synth.DECODE_B32], batch=4, len_lo=5000, len_hi=6000, top_k=512)
     case = synth.make_case(spec, 7101)
     bs = spec.block_size
     case.seq_lens[0] = 200
