@@ -226,3 +226,53 @@ def decode_step(case, rows=None, threads: int = 1):
     else:
         res = [row_step(case, r) for r in rows]
     return rows, res
+
+
+# --------------------------------------------------------------------------- several layers
+# A decode step runs one DSA layer after another.  The MLI page ("Multi-layer
+# Indexer" abstract, zhuanzhiai.com) fixes two routings of the selections:
+#  - IndexCache (sentences 8-9): only a fraction 1/r of the layers (the
+#    retention) keep an indexer; a layer without one reuses the selection of
+#    the latest layer that has one.  With r = 1 every layer attends its own
+#    selection: plain DSA.
+#  - MLI (sentences 4-5): a layer attends the selection of the previous indexer
+#    layer instead of its own, so its indexer no longer gates its attention.
+# Readings where the page is silent: the layers that keep an indexer are 0, r,
+# 2r, ...; layer 0 has no earlier indexer layer and attends its own selection.
+
+ROUTE_OWN = 0   # IndexCache (DSA at r = 1): the latest indexer layer i <= l
+ROUTE_PREV = 1  # MLI: the latest indexer layer i < l (layer 0: its own)
+
+
+def indexer_layers(n_layers: int, retention: int) -> list:
+    """Layers that keep an indexer at retention 1/retention."""
+    return [l for l in range(n_layers) if l % retention == 0]
+
+
+def selection_source(n_layers: int, retention: int, route: int) -> list:
+    """For every layer, the layer whose indexer selection it attends."""
+    keep = indexer_layers(n_layers, retention)
+    src = []
+    for l in range(n_layers):
+        before = [i for i in keep if (i <= l if route == ROUTE_OWN else i < l)]
+        src.append(before[-1] if before else 0)
+    return src
+
+
+def decode_layers(layers, retention: int, route: int):
+    """Several layers of one decode batch (a list of cases sharing the
+    sequence lengths and block table).  Each layer attends, with its own query
+    and KV cache, the selection its route names; an indexer layer's selection
+    is the top-k of its own scores.  Returns the source table and per layer
+    (selection attended [rows, k], o [rows, H, D_v], lse [rows, H])."""
+    src = selection_source(len(layers), retention, route)
+    sel = {}
+    for i in sorted(set(src)):
+        c = layers[i]
+        sel[i] = np.stack([topk(row_scores(c, r), row_visible(c, r), c.spec.top_k) for r in range(c.rows)])
+    res = []
+    for l, c in enumerate(layers):
+        idx = sel[src[l]]
+        att = [row_attention(c, r, idx[r]) for r in range(c.rows)]
+        res.append((idx, np.stack([a[0] for a in att]), np.stack([a[1] for a in att])))
+    return src, res

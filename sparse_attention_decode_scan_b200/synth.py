@@ -29,7 +29,7 @@ import os
 import zlib
 from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field, replace
-from typing import Dict, Optional
+from typing import Dict, List, Optional
 
 import numpy as np
 
@@ -214,8 +214,12 @@ class Case:
         return 0 if self.block_table is None else int(self.block_table.shape[1])
 
 
-def make_case(spec: Spec, seed: int) -> Case:
+def make_case(spec: Spec, seed: int, layer: int = 0) -> Case:
+    """Host arrays of one workload.  `layer` > 0 draws another DSA layer of the
+    same batch: the same sequence lengths and block table, its own cache
+    contents and queries (layer 0 is the plain single-layer workload)."""
     s = spec
+    tag = (lambda name: name) if layer == 0 else (lambda name: f"{name}@layer{layer}")
     r = rng(seed, "lengths")
     if s.causal:
         assert s.batch == 1 and s.len_lo == s.len_hi
@@ -238,19 +242,19 @@ def make_case(spec: Spec, seed: int) -> Case:
         bt = None
         lead = (s.batch, s.stride)
     ntok = int(np.prod(lead))
-    keys_f = normal(lead + (d_key,), seed, "idx_keys")
+    keys_f = normal(lead + (d_key,), seed, tag("idx_keys"))
     scales = None
     if key_dt == "fp8":
         if s.heavy_frac > 0:
-            heavy = rng(seed, "heavy").random(ntok, dtype=np.float64) < s.heavy_frac
+            heavy = rng(seed, tag("heavy")).random(ntok, dtype=np.float64) < s.heavy_frac
             keys_f.reshape(ntok, d_key)[heavy, 0] += np.float32(s.heavy_offset)
-        scales = rng(seed, "idx_scales").uniform(s.scale_lo, s.scale_hi, size=ntok).astype(np.float32)
+        scales = rng(seed, tag("idx_scales")).uniform(s.scale_lo, s.scale_hi, size=ntok).astype(np.float32)
         scales = scales.reshape(lead)
     idx_keys = encode(keys_f, key_dt)
     del keys_f
     kv = None
     if s.with_kv:
-        kv = encode(normal(lead + (s.qk_dim,), seed, "kv"), s.act_dtype)
+        kv = encode(normal(lead + (s.qk_dim,), seed, tag("kv")), s.act_dtype)
     if s.causal:
         R = s.chunk
         row_seq = np.zeros(R, np.int32)
@@ -259,10 +263,15 @@ def make_case(spec: Spec, seed: int) -> Case:
         R = s.batch
         row_seq = np.arange(R, dtype=np.int32)
         row_pos = None
-    q_idx = encode(normal((R, s.n_idx_heads, s.idx_dim), seed, "q_idx"), s.act_dtype)
-    w = normal((R, s.n_idx_heads), seed, "w", std=s.w_std)
-    q = encode(normal((R, s.n_heads, s.qk_dim), seed, "q"), s.act_dtype) if s.with_kv else None
+    q_idx = encode(normal((R, s.n_idx_heads, s.idx_dim), seed, tag("q_idx")), s.act_dtype)
+    w = normal((R, s.n_idx_heads), seed, tag("w"), std=s.w_std)
+    q = encode(normal((R, s.n_heads, s.qk_dim), seed, tag("q")), s.act_dtype) if s.with_kv else None
     return Case(s, seed, seq_lens, bt, idx_keys, scales, kv, row_seq, row_pos, q_idx, w, q)
+
+
+def make_layers(spec: Spec, seed: int, n_layers: int) -> List[Case]:
+    """n_layers DSA layers of one decode batch (make_case with layer = 0..n-1)."""
+    return [make_case(spec, seed, layer=l) for l in range(n_layers)]
 
 
 def scaled(spec: Spec, **kw) -> Spec:
@@ -344,6 +353,6 @@ def flops_prefill_scan(case: Case) -> int:
 
 
 __all__ = ["Spec", "Case", "WORKLOADS", "workload", "TINY", "DECODE_B1", "DECODE_B32", "DECODE_B4_FP8",
-           "PREFILL", "make_case", "scaled", "seed_of", "normal", "rng",
+           "PREFILL", "make_case", "make_layers", "scaled", "seed_of", "normal", "rng",
            "to_bf16_bits", "to_e4m3_bits", "topk_scores", "index_lists",
            "nbytes_decode_step", "flops_prefill_scan"]
