@@ -109,7 +109,8 @@ typedef enum {
   LSA_OP_TOPK = 1,
   LSA_OP_ATTN = 2,
   LSA_OP_DECODE_STEP = 3,
-  LSA_OP_DECODE_STEP_FUSED = 4 /* lsa_launch_count only: lsa_decode_step with LSA_STEP_FUSED */
+  LSA_OP_DECODE_STEP_FUSED = 4, /* lsa_launch_count only: lsa_decode_step with LSA_STEP_FUSED */
+  LSA_OP_DECODE_LAYERS = 5      /* lsa_decode_layers (workspace size only) */
 } lsa_op;
 
 /* Flags of lsa_decode_step. */
@@ -205,6 +206,47 @@ lsa_status lsa_decode_step_profiled(const lsa_dims* d, const lsa_cache* c, const
                                     const float* w, const void* q, void* out, float* lse,
                                     int32_t* idx_out, int32_t flags, void* ws, size_t ws_bytes,
                                     lsa_stream_t stream, void* const* events);
+
+/* Routes of lsa_decode_layers: which indexer layer's selection a layer attends. */
+#define LSA_ROUTE_OWN 0  /* the latest indexer layer at or before it (IndexCache; DSA at retention 1) */
+#define LSA_ROUTE_PREV 1 /* the latest indexer layer before it (Multi-layer Indexer); layer 0: its own */
+
+/*
+ * Several DSA layers of one decode step ("Multi-layer Indexer" abstract,
+ * zhuanzhiai.com, sentences 4-5 and 8-9: IndexCache keeps an indexer on a
+ * fraction 1/r of the layers and the others reuse the latest selection; MLI
+ * lets a layer attend the previous indexer layer's selection, so its own
+ * indexer runs alongside its attention).
+ *   n_layers >= 1 layers; every array argument is a HOST array of n_layers
+ *   entries holding device pointers:
+ *     caches[l]  layer l's cache: the same batch B, max_len, seq_lens, block
+ *                table and block size for every layer, its own idx_keys,
+ *                idx_key_scales (FP8) and kv.
+ *     q_idx[l] [B, H_I, d_I], w[l] [B, H_I] fp32: read only for the layers
+ *                that keep an indexer.
+ *     q[l] [B, H, D]: layer l's attention query.
+ *     out[l] [B, H, D_v], lse[l] [B, H] fp32 (lse may be NULL, or lse[l] NULL).
+ *   retention r >= 1: layers 0, r, 2r, ... keep an indexer.
+ *   route: LSA_ROUTE_OWN or LSA_ROUTE_PREV (above).
+ *   idx_out: NULL or device int32 [n_layers, B, k]: the selection each layer
+ *            attended (sorted ascending, -1 padded, as lsa_topk).
+ * Order on `stream`: layer l+1 starts after layer l's attention has finished
+ * (a layer's queries depend on the previous layer's output).  Within a layer
+ * that keeps an indexer, LSA_ROUTE_OWN runs scan -> top-k -> attention as
+ * lsa_decode_step does; LSA_ROUTE_PREV launches the attention (on the earlier
+ * selection) as a programmatic dependent of the layer's top-k that does not
+ * wait for it, so the two overlap and the attention starts as the scan ends.
+ * Results per layer equal lsa_decode_step / lsa_sparse_attn_decode on the
+ * routed selection.
+ * Workspace: lsa_workspace_size(d, B, max_len, LSA_OP_DECODE_LAYERS).
+ * Errors: LSA_ERR_INVALID_ARG for n_layers < 1, retention < 1, an unknown
+ * route, layers whose batch, max_len, seq_lens or block table differ from
+ * layer 0's, or a missing or misaligned pointer; nothing is launched then.
+ */
+lsa_status lsa_decode_layers(const lsa_dims* d, int32_t n_layers, const lsa_cache* caches,
+                             const void* const* q_idx, const float* const* w, const void* const* q,
+                             void* const* out, float* const* lse, int32_t retention, int32_t route,
+                             int32_t* idx_out, void* ws, size_t ws_bytes, lsa_stream_t stream);
 
 /*
  * Copies the workspace status word to *status (an lsa_status value), clears it,

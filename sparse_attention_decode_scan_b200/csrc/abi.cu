@@ -104,6 +104,30 @@ StepLayout step_layout(const lsa_dims* d, int32_t rows, int64_t max_len) {
   return L;
 }
 
+// Several layers (lsa_decode_layers): the scores, two selection buffers (the
+// latest indexer selection and the one being made), the scan / top-k scratch
+// and, apart from it, the attention's (the two run at once under the MLI route).
+struct LayersLayout {
+  size_t scores_off, sel_off[2], tk_off, tk_bytes, at_off, at_bytes, total;
+};
+
+LayersLayout layers_layout(const lsa_dims* d, int32_t rows, int64_t max_len) {
+  LayersLayout L;
+  const size_t sel = align_up(static_cast<size_t>(rows) * d->top_k * 4);
+  L.scores_off = kStatusBytes;
+  L.sel_off[0] = L.scores_off + align_up(static_cast<size_t>(rows) * score_ld(max_len) * 4);
+  L.sel_off[1] = L.sel_off[0] + sel;
+  L.tk_off = L.sel_off[1] + sel;
+  size_t tk = topk_ws_bytes(rows, max_len, d->top_k);
+  const size_t sc = scores_ws(rows, false);
+  if (sc > tk) tk = sc;
+  L.tk_bytes = align_up(tk);
+  L.at_off = L.tk_off + L.tk_bytes;
+  L.at_bytes = attn_ws(d, rows);
+  L.total = L.at_off + L.at_bytes;
+  return L;
+}
+
 lsa_status ws_check(void* ws, size_t have, size_t need) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LSA_ERR_WORKSPACE;
   if (have < need) return LSA_ERR_WORKSPACE;
@@ -211,12 +235,13 @@ AttnArgs attn_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, const in
 lsa_status do_attn(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq, const void* q,
                    const int32_t* idx, void* out, float* lse, void* ws, void* inner_ws, size_t inner_bytes,
                    cudaStream_t s, bool pdl = false, const uint32_t* row_ready = nullptr,
-                   const AttnArgs* split = nullptr) {
+                   const AttnArgs* split = nullptr, bool inputs_ready = false) {
   AttnArgs a = attn_args(d, c, rows, row_seq, q, idx, out, lse, ws, inner_ws, inner_bytes);
   // in a decode step the kernel before is the step's top-k, which does not write q
   a.pdl = pdl;
   a.q_early = pdl;
   a.row_ready = row_ready;
+  a.inputs_ready = inputs_ready;
   if (split) {
     a.split_sel = true;
     a.tk_ws = split->tk_ws;
@@ -252,6 +277,9 @@ size_t lsa_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int3
     case LSA_OP_DECODE_STEP:
       if (!valid_dims(d)) return 0;
       return step_layout(d, rows, max_len).total;
+    case LSA_OP_DECODE_LAYERS:
+      if (!valid_dims(d)) return 0;
+      return layers_layout(d, rows, max_len).total;
     default:
       return 0;
   }
@@ -409,6 +437,82 @@ lsa_status lsa_decode_step_profiled(const lsa_dims* d, const lsa_cache* c, const
                                     const void* q, void* out, float* lse, int32_t* idx_out, int32_t flags,
                                     void* ws, size_t ws_bytes, lsa_stream_t stream, void* const* events) {
   return decode_step_impl(d, c, q_idx, w, q, out, lse, idx_out, flags, ws, ws_bytes, stream, events);
+}
+
+lsa_status lsa_decode_layers(const lsa_dims* d, int32_t n_layers, const lsa_cache* caches,
+                             const void* const* q_idx, const float* const* w, const void* const* q,
+                             void* const* out, float* const* lse, int32_t retention, int32_t route,
+                             int32_t* idx_out, void* ws, size_t ws_bytes, lsa_stream_t stream) {
+  if (!valid_dims(d) || n_layers < 1 || retention < 1 || !caches || !q || !out) return LSA_ERR_INVALID_ARG;
+  if (route != LSA_ROUTE_OWN && route != LSA_ROUTE_PREV) return LSA_ERR_INVALID_ARG;
+  const lsa_cache& c0 = caches[0];
+  const int32_t B = c0.batch;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const lsa_cache& c = caches[l];
+    const bool keeps = l % retention == 0;
+    if (!valid_cache(d, &c, keeps, true)) return LSA_ERR_INVALID_ARG;
+    if (c.batch != B || c.max_len != c0.max_len || c.seq_lens != c0.seq_lens || c.block_table != c0.block_table ||
+        c.max_blocks_per_seq != c0.max_blocks_per_seq)
+      return LSA_ERR_INVALID_ARG;
+    if (B > 0) {
+      if (!q[l] || !out[l] || !aligned16(q[l]) || !aligned16(out[l])) return LSA_ERR_INVALID_ARG;
+      if (keeps && (!q_idx || !w || !q_idx[l] || !w[l] || !aligned16(q_idx[l]))) return LSA_ERR_INVALID_ARG;
+    }
+  }
+  if (B > 65535) return LSA_ERR_UNSUPPORTED;
+  const LayersLayout L = layers_layout(d, B, c0.max_len);
+  lsa_status st = ws_check(ws, ws_bytes, L.total);
+  if (st != LSA_OK) return st;
+  if (B == 0) return LSA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* scores = reinterpret_cast<float*>(base + L.scores_off);
+  int32_t* sel[2] = {reinterpret_cast<int32_t*>(base + L.sel_off[0]), reinterpret_cast<int32_t*>(base + L.sel_off[1])};
+  void* tk = base + L.tk_off;
+  void* at = base + L.at_off;
+  const int64_t ld = score_ld(c0.max_len);
+  const size_t sel_bytes = static_cast<size_t>(B) * d->top_k * 4;
+  int cur = 0;  // the buffer holding the latest indexer layer's selection
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const lsa_cache* c = &caches[l];
+    float* lse_l = lse ? lse[l] : nullptr;
+    const int32_t* attended = sel[cur];
+    if (l % retention == 0) {
+      // MLI: from the second indexer layer on, the attention takes the
+      // selection already made and the top-k writes the other buffer
+      const bool overlap = route == LSA_ROUTE_PREV && l > 0;
+      const int nxt = overlap ? 1 - cur : cur;
+      uint32_t* hist12 = (!force_simt() && topk_v2_ok(c->max_len)) ? static_cast<uint32_t*>(tk) : nullptr;
+      bool hist_done = false;
+      uint32_t *scan_done = nullptr, *sel_done = nullptr;
+      if (hist12) topk_step_flags(tk, B, c->max_len, &scan_done, &sel_done);
+      st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
+                     &hist_done, scan_done);
+      if (st != LSA_OK) return st;
+      st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, sel[nxt], ws, tk, s, hist_done, true,
+                   hist_done ? scan_done : nullptr, hist_done ? static_cast<uint32_t>(scan_tc_grid()) : 0u);
+      if (st != LSA_OK) return st;
+      if (overlap) {
+        // launched as the top-k's dependent and waiting for nothing: its
+        // inputs were complete before this layer's scan started
+        st = do_attn(d, c, B, nullptr, q[l], sel[cur], out[l], lse_l, ws, at, L.at_bytes, s, true, nullptr,
+                     nullptr, true);
+      } else {
+        st = do_attn(d, c, B, nullptr, q[l], sel[nxt], out[l], lse_l, ws, at, L.at_bytes, s, true,
+                     hist_done ? sel_done : nullptr);
+        attended = sel[nxt];
+      }
+      if (st != LSA_OK) return st;
+      cur = nxt;
+    } else {
+      st = do_attn(d, c, B, nullptr, q[l], attended, out[l], lse_l, ws, at, L.at_bytes, s);
+      if (st != LSA_OK) return st;
+    }
+    if (idx_out && cudaMemcpyAsync(idx_out + static_cast<int64_t>(l) * B * d->top_k, attended, sel_bytes,
+                                   cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return LSA_ERR_CUDA;
+  }
+  return LSA_OK;
 }
 
 lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream) {

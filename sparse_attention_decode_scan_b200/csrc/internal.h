@@ -127,6 +127,9 @@ struct AttnArgs {
   DevStatus* status;
   bool pdl = false;      // launched as a programmatic dependent of the kernel before it (decode step)
   bool q_early = false;  // with pdl: q may be read before the kernel before it completes
+  // with pdl: nothing the kernel reads is written by the kernels before it
+  // still running (several layers, MLI route): no wait at all
+  bool inputs_ready = false;
   // Decode step: the selection of row r may be read once row_ready[r] != 0
   // (raised by the top-k after writing it); null: wait for the kernel before.
   const uint32_t* row_ready = nullptr;

@@ -24,14 +24,20 @@ def to_device(arr: np.ndarray, dtype: str, device="cuda", pin: bool = False):
 class DeviceCase:
     """A synth.Case on the GPU plus its lsa Dims / Cache structs."""
 
-    def __init__(self, case, device="cuda", top_k=None):
+    def __init__(self, case, device="cuda", top_k=None, share: "DeviceCase" = None):
+        """`share`: another layer of the same batch whose lengths, block table
+        and row map (the same arrays) this layer's cache struct points at."""
         import torch
         s = case.spec
         self.case = case
         self.spec = s
         self.device = device
-        self.seq_lens = torch.from_numpy(case.seq_lens).to(device)
-        self.block_table = torch.from_numpy(case.block_table).to(device) if case.block_table is not None else None
+        if share is not None:
+            assert np.array_equal(case.seq_lens, share.case.seq_lens)
+            self.seq_lens, self.block_table = share.seq_lens, share.block_table
+        else:
+            self.seq_lens = torch.from_numpy(case.seq_lens).to(device)
+            self.block_table = torch.from_numpy(case.block_table).to(device) if case.block_table is not None else None
         self.idx_keys = to_device(case.idx_keys, s.idx_key_dtype, device)
         self.idx_scales = torch.from_numpy(case.idx_scales).to(device) if case.idx_scales is not None else None
         self.kv = to_device(case.kv, s.act_dtype, device) if case.kv is not None else None
@@ -76,3 +82,9 @@ def make_dims(s, top_k=None) -> lsa.Dims:
     d.act_dtype = lsa.DTYPE_CODE[s.act_dtype]
     d.idx_key_dtype = lsa.DTYPE_CODE[s.idx_key_dtype]
     return d
+
+
+def device_layers(cases, device="cuda"):
+    """DeviceCases of the layers of one batch, sharing layer 0's lengths and block table."""
+    first = DeviceCase(cases[0], device=device)
+    return [first] + [DeviceCase(c, device=device, share=first) for c in cases[1:]]

@@ -17,8 +17,10 @@ LIB_PATH = os.path.join(_HERE, "liblsa.so")
 LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_TIMEOUT, \
     LSA_ERR_BOUNDS = range(7)
 LSA_F32, LSA_BF16, LSA_FP8_E4M3 = 0, 1, 2
-LSA_OP_SCORES, LSA_OP_TOPK, LSA_OP_ATTN, LSA_OP_DECODE_STEP, LSA_OP_DECODE_STEP_FUSED = 0, 1, 2, 3, 4
+LSA_OP_SCORES, LSA_OP_TOPK, LSA_OP_ATTN, LSA_OP_DECODE_STEP, LSA_OP_DECODE_STEP_FUSED, LSA_OP_DECODE_LAYERS = \
+    0, 1, 2, 3, 4, 5
 LSA_STEP_UNFUSED, LSA_STEP_FUSED = 0, 1
+LSA_ROUTE_OWN, LSA_ROUTE_PREV = 0, 1
 
 DTYPE_CODE = {"f32": LSA_F32, "bf16": LSA_BF16, "fp8": LSA_FP8_E4M3}
 
@@ -66,6 +68,8 @@ def lib() -> ctypes.CDLL:
     L.lsa_sparse_attn_decode.argtypes = [D, C, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.lsa_decode_step.argtypes = [D, C, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
     L.lsa_decode_step_profiled.argtypes = [D, C, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]
+    PV = ctypes.POINTER(vp)
+    L.lsa_decode_layers.argtypes = [D, C, i32, PV, PV, PV, PV, PV, i32, i32, vp, vp, sz, vp]
     L.lsa_read_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
     L.lsa_status_string.argtypes = [ctypes.c_int]
     L.lsa_status_string.restype = ctypes.c_char_p
@@ -73,7 +77,7 @@ def lib() -> ctypes.CDLL:
     L.lsa_launch_count.argtypes = [D, i32, i64, i32, i32]
     L.lsa_launch_count.restype = i32
     for f in ("lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode", "lsa_decode_step",
-              "lsa_decode_step_profiled",
+              "lsa_decode_step_profiled", "lsa_decode_layers",
               "lsa_read_device_status"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
@@ -174,6 +178,22 @@ def decode_step_profiled(dims: Dims, cache: Cache, q_idx, w, q, out, lse, ws, ev
                                                  _ptr(q), _ptr(out), _ptr(lse), _ptr(idx_out), int(flags),
                                                  _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream),
                                                  ev), "lsa_decode_step_profiled", raise_on_error)
+
+
+def decode_layers(dims: Dims, caches, q_idx, w, q, out, lse, ws, retention: int = 1, route: int = LSA_ROUTE_OWN,
+                  idx_out=None, stream=None, raise_on_error=True) -> int:
+    """lsa_decode_layers: per-layer lists of Cache structs and tensors (q_idx / w entries may be None for
+    layers without an indexer, lse may be None)."""
+    n = len(caches)
+    arr = (Cache * n)(*caches)
+
+    def ptrs(ts):
+        return (ctypes.c_void_p * n)(*[_ptr(t) for t in ts]) if ts is not None else None
+
+    return _check(lib().lsa_decode_layers(ctypes.byref(dims), arr, n, ptrs(q_idx), ptrs(w), ptrs(q), ptrs(out),
+                                          ptrs(lse), int(retention), int(route), _ptr(idx_out), _ptr(ws),
+                                          ws.numel() if ws is not None else 0, _stream(stream)),
+                  "lsa_decode_layers", raise_on_error)
 
 
 def read_device_status(ws, stream=None) -> int:
