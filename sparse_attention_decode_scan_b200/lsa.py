@@ -69,7 +69,7 @@ def lib() -> ctypes.CDLL:
     L.lsa_decode_step.argtypes = [D, C, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
     L.lsa_decode_step_profiled.argtypes = [D, C, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]
     PV = ctypes.POINTER(vp)
-    L.lsa_decode_layers.argtypes = [D, C, i32, PV, PV, PV, PV, PV, i32, i32, vp, vp, sz, vp]
+    L.lsa_decode_layers.argtypes = [D, i32, C, PV, PV, PV, PV, PV, i32, i32, vp, vp, sz, vp]
     L.lsa_read_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
     L.lsa_status_string.argtypes = [ctypes.c_int]
     L.lsa_status_string.restype = ctypes.c_char_p
@@ -190,7 +190,7 @@ def decode_layers(dims: Dims, caches, q_idx, w, q, out, lse, ws, retention: int 
     def ptrs(ts):
         return (ctypes.c_void_p * n)(*[_ptr(t) for t in ts]) if ts is not None else None
 
-    return _check(lib().lsa_decode_layers(ctypes.byref(dims), arr, n, ptrs(q_idx), ptrs(w), ptrs(q), ptrs(out),
+    return _check(lib().lsa_decode_layers(ctypes.byref(dims), n, arr, ptrs(q_idx), ptrs(w), ptrs(q), ptrs(out),
                                           ptrs(lse), int(retention), int(route), _ptr(idx_out), _ptr(ws),
                                           ws.numel() if ws is not None else 0, _stream(stream)),
                   "lsa_decode_layers", raise_on_error)
