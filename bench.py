@@ -488,6 +488,102 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_layers(args, world, rank, local):
+    """Several DSA layers per decode step (lsa_decode_layers): the IndexCache
+    route (DSA at retention 1) or the MLI route.  Every layer has its own cache
+    memory (layer 0's host-drawn cache copied into distinct device buffers, so
+    no layer finds another's rows in L2) and its own queries drawn on the host;
+    layer l+1 starts after layer l's attention."""
+    import torch
+
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase, to_device
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = synth.workload(args.workload)
+    spec = synth.scaled(base, batch=args.batch) if args.batch else base
+    assert not spec.causal, "layers: decode workloads only"
+    case = synth.make_case(spec, rank_seed(base, rank))
+    dc0 = DeviceCase(case, device=dev)
+    s = case.spec
+    B, n = dc0.rows, args.layers
+    route = lsa.LSA_ROUTE_PREV if args.route == "prev" else lsa.LSA_ROUTE_OWN
+    caches, q_idx, w, q = [], [], [], []
+    keep = []  # device buffers of the layers
+    for l in range(n):
+        qi, wl, ql = synth.queries(s, rank_seed(base, rank), B, layer=l)
+        q_idx.append(to_device(qi, s.act_dtype, dev))
+        w.append(torch.from_numpy(wl).to(dev))
+        q.append(to_device(ql, s.act_dtype, dev))
+        if l == 0:
+            caches.append(dc0.cache)
+            continue
+        keys = dc0.idx_keys.clone()
+        scales = dc0.idx_scales.clone() if dc0.idx_scales is not None else None
+        kv = dc0.kv.clone()
+        keep += [keys, scales, kv]
+        c = dc0.make_cache()
+        c.idx_keys = keys.data_ptr()
+        c.idx_key_scales = scales.data_ptr() if scales is not None else None
+        c.kv = kv.data_ptr()
+        caches.append(c)
+    out = [torch.empty((B, s.n_heads, s.v_dim), dtype=torch.bfloat16, device=dev) for _ in range(n)]
+    lse = [torch.empty((B, s.n_heads), dtype=torch.float32, device=dev) for _ in range(n)]
+    ws = lsa.workspace(lsa.workspace_size(dc0.dims, B, dc0.max_len, lsa.LSA_OP_DECODE_LAYERS), device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lsa.decode_layers(dc0.dims, caches, q_idx, w, q, out, lse, ws, retention=args.retention, route=route,
+                          stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    with ClockSampler(gpu_index) as clk:
+        t_soak = time.perf_counter()
+        while not args.no_soak and time.perf_counter() - t_soak < 1.0:
+            step()
+            torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    timed_ms = reduce_max(a.elapsed_time(b))
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    peaks, peak_src = load_peaks()
+    nb = synth.nbytes_decode_step(case)
+    n_ind = len(range(0, n, args.retention))
+    # algorithmic bytes: every indexer layer's keys and queries, every layer's gathered rows, query and output
+    step_bytes = n_ind * (nb["keys"] + nb["scales"] + nb["block_table"] + nb["q_idx_w"]) + \
+        n * (nb["kv_gather"] + nb["q"] + nb["out"])
+    ms_per_step = timed_ms / args.steps
+    gbs = step_bytes / (ms_per_step / 1e3) / 1e9
+    route_name = "MLI (previous indexer layer)" if route == lsa.LSA_ROUTE_PREV else \
+        ("DSA (own selection)" if args.retention == 1 else "IndexCache (latest indexer layer)")
+    line = {"metric": f"decode steps/s over {n} layers, {route_name}, retention 1/{args.retention}",
+            "value": world * args.steps / (timed_ms / 1e3), "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "ms_per_layer": ms_per_step / n, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": s.act_dtype if s.idx_key_dtype != "fp8" else "bf16+fp8",
+            "data": "synthetic (seeded, generated on host; layer caches are copies of layer 0's in distinct "
+                    "device memory, queries drawn per layer)",
+            "config": dict(workload_config(case), layers=n, retention=args.retention, route=args.route,
+                           indexer_layers=n_ind),
+            "step_hbm_gbs": gbs, "step_hbm_frac": gbs / peaks["hbm_gbs"], "step_algorithmic_bytes": step_bytes,
+            "peak_source": peak_src, "gpu_launches": None, "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -502,6 +598,11 @@ def main(argv=None):
     ap.add_argument("--op", default="step", choices=["step", "scan", "topk", "attn"],
                     help="time one stage only (profiling); the bench line is for 'step'")
     ap.add_argument("--no-soak", action="store_true", help="skip the 1 s clock-sampling soak (profiling)")
+    ap.add_argument("--layers", type=int, default=1,
+                    help="DSA layers per decode step (lsa_decode_layers); 1 = the single-layer step")
+    ap.add_argument("--route", default="own", choices=["own", "prev"],
+                    help="layers: attend the latest indexer layer at or before (own) or before (prev, MLI) a layer")
+    ap.add_argument("--retention", type=int, default=1, help="layers: every retention-th layer keeps an indexer")
     ap.add_argument("--fused", action="store_true",
                     help="decode step as one cooperative launch (LSA_STEP_FUSED) instead of separate launches")
     args = ap.parse_args(argv)
@@ -521,7 +622,10 @@ def main(argv=None):
         if args.impl == "reference":
             run_reference(args, world, rank)
         else:
-            run_ours(args, world, rank, local)
+            if args.layers > 1:
+                run_layers(args, world, rank, local)
+            else:
+                run_ours(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -263,10 +263,20 @@ def make_case(spec: Spec, seed: int, layer: int = 0) -> Case:
         R = s.batch
         row_seq = np.arange(R, dtype=np.int32)
         row_pos = None
-    q_idx = encode(normal((R, s.n_idx_heads, s.idx_dim), seed, tag("q_idx")), s.act_dtype)
-    w = normal((R, s.n_idx_heads), seed, tag("w"), std=s.w_std)
-    q = encode(normal((R, s.n_heads, s.qk_dim), seed, tag("q")), s.act_dtype) if s.with_kv else None
+    q_idx, w, q = queries(s, seed, R, layer)
     return Case(s, seed, seq_lens, bt, idx_keys, scales, kv, row_seq, row_pos, q_idx, w, q)
+
+
+def queries(spec: Spec, seed: int, rows: int, layer: int = 0):
+    """The query rows of one layer (as make_case draws them): indexer queries
+    q_idx [rows, H_I, d_I], weights w [rows, H_I] and attention queries q
+    [rows, H, D] (None without a KV cache)."""
+    s = spec
+    tag = (lambda name: name) if layer == 0 else (lambda name: f"{name}@layer{layer}")
+    q_idx = encode(normal((rows, s.n_idx_heads, s.idx_dim), seed, tag("q_idx")), s.act_dtype)
+    w = normal((rows, s.n_idx_heads), seed, tag("w"), std=s.w_std)
+    q = encode(normal((rows, s.n_heads, s.qk_dim), seed, tag("q")), s.act_dtype) if s.with_kv else None
+    return q_idx, w, q
 
 
 def make_layers(spec: Spec, seed: int, n_layers: int) -> List[Case]:
@@ -353,6 +363,6 @@ def flops_prefill_scan(case: Case) -> int:
 
 
 __all__ = ["Spec", "Case", "WORKLOADS", "workload", "TINY", "DECODE_B1", "DECODE_B32", "DECODE_B4_FP8",
-           "PREFILL", "make_case", "make_layers", "scaled", "seed_of", "normal", "rng",
+           "PREFILL", "make_case", "make_layers", "queries", "scaled", "seed_of", "normal", "rng",
            "to_bf16_bits", "to_e4m3_bits", "topk_scores", "index_lists",
            "nbytes_decode_step", "flops_prefill_scan"]
