@@ -164,24 +164,14 @@ ScoresArgs scores_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, cons
 lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
                      const int32_t* row_pos, const void* q_idx, const float* w, float* scores,
                      int64_t ld, void* ws, void* inner_ws, size_t inner_bytes, cudaStream_t s,
-                     uint32_t* hist12 = nullptr, bool* hist_done = nullptr, uint32_t* done_ctr = nullptr,
-                     bool zeroed = false, bool pdl = false, const ScoresArgs* split = nullptr) {
+                     uint32_t* hist12 = nullptr, bool* hist_done = nullptr, uint32_t* done_ctr = nullptr) {
   ScoresArgs a = scores_args(d, c, rows, row_seq, row_pos, q_idx, w, scores, ld, ws, inner_ws, inner_bytes);
   if (hist_done) *hist_done = false;
   if (rows == 0 || ld == 0) return LSA_OK;
   if (!force_simt() && scores_tc_supported(a)) {
-    a.pdl = pdl;
-    if (split) {
-      a.grid = split->grid;
-      a.split_part = split->split_part;
-      a.split_free = split->split_free;
-      a.split_busy_us = split->split_busy_us;
-      a.split_tile_us = split->split_tile_us;
-    }
     if (hist12 && scores_tc_fused_hist_ok(a)) {
-      // the scan also counts the first top-k digit; the counters start at
-      // zero (cleared here unless the caller already did)
-      cudaError_t e = zeroed ? cudaSuccess : cudaMemsetAsync(hist12, 0, topk_hist_zero_bytes(rows), s);
+      // the scan also counts the first top-k digit; the counters start at zero
+      cudaError_t e = cudaMemsetAsync(hist12, 0, topk_hist_zero_bytes(rows), s);
       if (e != cudaSuccess) return LSA_ERR_CUDA;
       a.hist12 = hist12;
       a.done_ctr = done_ctr;  // zeroed with the histograms
@@ -245,13 +235,12 @@ AttnArgs attn_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, const in
 lsa_status do_attn(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq, const void* q,
                    const int32_t* idx, void* out, float* lse, void* ws, void* inner_ws, size_t inner_bytes,
                    cudaStream_t s, bool pdl = false, const uint32_t* row_ready = nullptr,
-                   const AttnArgs* split = nullptr, bool inputs_ready = false) {
+                   const AttnArgs* split = nullptr) {
   AttnArgs a = attn_args(d, c, rows, row_seq, q, idx, out, lse, ws, inner_ws, inner_bytes);
   // in a decode step the kernel before is the step's top-k, which does not write q
   a.pdl = pdl;
   a.q_early = pdl;
   a.row_ready = row_ready;
-  a.inputs_ready = inputs_ready;
   if (split) {
     a.split_sel = true;
     a.tk_ws = split->tk_ws;
@@ -339,13 +328,6 @@ lsa_status lsa_sparse_attn_decode(const lsa_dims* d, const lsa_cache* c, int32_t
   return do_attn(d, c, rows, row_seq, q, idx, out, lse, ws, static_cast<uint8_t*>(ws) + kStatusBytes,
                  ws_bytes - kStatusBytes, reinterpret_cast<cudaStream_t>(stream));
 }
-
-// Timing model of the MLI layer's scan split (measured on B200 at 1965 MHz): a
-// tensor-core attention CTA takes about kAttnFixedUs plus kAttnChunkUs per
-// 64-entry chunk, and a scan CTA streams one 128-token tile per kScanTileUs.
-constexpr double kAttnFixedUs = 21.0;
-constexpr double kAttnChunkUs = 2.2;
-constexpr double kScanTileUs = 0.72;
 
 // Rows at least this long take the split select in a decode step (the
 // environment variable LSA_SPLIT_SELECT_MIN_COLS overrides it, for tests).
@@ -504,51 +486,15 @@ lsa_status lsa_decode_layers(const lsa_dims* d, int32_t n_layers, const lsa_cach
       uint32_t *scan_done = nullptr, *sel_done = nullptr;
       if (hist12) topk_step_flags(tk, B, c->max_len, &scan_done, &sel_done);
       if (overlap) {
-        // The attention on the selection already made goes first.  The scan
-        // follows as its programmatic dependent (it reads nothing the
-        // attention writes) and takes every SM the attention leaves; the
-        // top-k follows the scan.  The counters they share are cleared before
-        // the attention, so no copy-engine step separates the kernels.
-        const ScoresArgs sa =
-            scores_args(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes);
-        const bool fused_hist = hist12 && !force_simt() && scores_tc_supported(sa) && scores_tc_fused_hist_ok(sa);
-        if (fused_hist && cudaMemsetAsync(hist12, 0, topk_hist_zero_bytes(B), s) != cudaSuccess) return LSA_ERR_CUDA;
+        // The attention on the selection already made, then this layer's
+        // scan and top-k (which writes the other buffer), in stream order.
         st = do_attn(d, c, B, nullptr, q[l], sel[cur], out[l], lse_l, ws, at, L.at_bytes, s);
         if (st != LSA_OK) return st;
-        // The attention's CTAs (one per SM) leave some SMs free: a first scan
-        // launch of one CTA per free SM takes the tiles those SMs stream while
-        // the attention runs, a second (one CTA per SM) the rest as the
-        // attention's CTAs end (each CTA has a static share, so a single
-        // launch would end with its last-started CTAs).
-        const int sms = scan_tc_grid();
-        int cps = 0;
-        const bool tc_attn =
-            !force_simt() && attn_tc_supported(attn_args(d, c, B, nullptr, q[l], sel[cur], out[l], lse_l, ws, at,
-                                                         L.at_bytes));
-        const int free_sms = tc_attn ? sms - attn_tc_ctas(B, d->top_k, &cps) : 0;
-        uint32_t target = static_cast<uint32_t>(sms);
-        if (fused_hist && free_sms > 0) {
-          ScoresArgs sp;
-          sp.split_free = free_sms;
-          sp.split_busy_us = static_cast<float>(kAttnFixedUs + kAttnChunkUs * cps);
-          sp.split_tile_us = static_cast<float>(kScanTileUs);
-          sp.grid = free_sms;
-          sp.split_part = 1;
-          st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
-                         &hist_done, scan_done, true, true, &sp);
-          if (st != LSA_OK) return st;
-          sp.grid = sms;
-          sp.split_part = 2;
-          st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
-                         &hist_done, scan_done, true, true, &sp);
-          target = static_cast<uint32_t>(sms + free_sms);
-        } else {
-          st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s,
-                         fused_hist ? hist12 : nullptr, &hist_done, scan_done, true, true);
-        }
+        st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
+                       &hist_done, scan_done);
         if (st != LSA_OK) return st;
         st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, sel[nxt], ws, tk, s, hist_done, true,
-                     hist_done ? scan_done : nullptr, hist_done ? target : 0u);
+                     hist_done ? scan_done : nullptr, hist_done ? static_cast<uint32_t>(scan_tc_grid()) : 0u);
       } else {
         st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
                        &hist_done, scan_done);

@@ -450,7 +450,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
   float* slse = reinterpret_cast<float*>(vrow + kNBuf * kChunk);  // [64] cluster merge: the partial's lse
   const bool cmerge = P.nsplit > 1 && P.merge == kMergeCluster;
   // the producer waits for this row's data itself (no wait for the kernel before)
-  const bool handoff = a.row_ready != nullptr || a.split_sel || a.inputs_ready;
+  const bool handoff = a.row_ready != nullptr || a.split_sel;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j0 = split * P.split_len;
@@ -556,7 +556,7 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
         *abort_flag = 1;
       }
       asm volatile("bar.sync 4, %0;" ::"n"(kProdThreads) : "memory");  // the producer warps
-    } else if (!a.inputs_ready) {
+    } else {
       tc::griddep_wait();  // launched early in a decode step: the selection is complete from here on
     }
     if (sel_state == 2) fill_table(0);

@@ -106,21 +106,7 @@ cudaError_t launch_t(const ScoresArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  if (a.pdl) {
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(a.grid > 0 ? a.grid : num_sms());
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr.val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tmap, smap, a);
-  }
-  kern<<<a.grid > 0 ? a.grid : num_sms(), kThreads, C::kSmemBytes, s>>>(tmap, smap, a);
+  kern<<<num_sms(), kThreads, C::kSmemBytes, s>>>(tmap, smap, a);
   return cudaGetLastError();
 }
 

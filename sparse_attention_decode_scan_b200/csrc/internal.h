@@ -46,16 +46,6 @@ struct ScoresArgs {
                        // zeroed by the caller), accumulated by the scan for the top-k
   uint32_t* done_ctr = nullptr;  // if set (zeroed by the caller): every CTA adds 1 once its
                                  // scores and histogram counts are written and fenced
-  bool pdl = false;  // tensor-core scan: launched as a programmatic dependent of the kernel
-                     // before it, which writes nothing the scan reads (the scan never waits)
-  // tensor-core scan: `grid` CTAs (0: one per SM).  split_part 1 or 2: the
-  // launch covers the first or the second part of the rows' tiles: the first
-  // is what split_free CTAs stream in split_busy_us (the other SMs being held
-  // by another kernel meanwhile), one tile taking split_tile_us; 0: all tiles.
-  int grid = 0;
-  int split_part = 0;
-  int split_free = 0;
-  float split_busy_us = 0.f, split_tile_us = 1.f;
 };
 
 // ---- indexer
@@ -66,10 +56,6 @@ int scores_tc_launches(bool causal);
 bool scores_tc_supported(const ScoresArgs& a);
 size_t scores_tc_ws_bytes(int32_t rows, bool causal);
 cudaError_t launch_scores_tc(const ScoresArgs& a, cudaStream_t s);
-
-// CTAs of the tensor-core attention's launch for `rows` rows and k entries
-// (and the 64-entry chunks each CTA works through).
-int attn_tc_ctas(int32_t rows, int32_t k, int* chunks_per_cta);
 
 // ---- top-k
 struct TopkPlan {
@@ -141,9 +127,6 @@ struct AttnArgs {
   DevStatus* status;
   bool pdl = false;      // launched as a programmatic dependent of the kernel before it (decode step)
   bool q_early = false;  // with pdl: q may be read before the kernel before it completes
-  // with pdl: nothing the kernel reads is written by the kernels before it
-  // still running (several layers, MLI route): no wait at all
-  bool inputs_ready = false;
   // Decode step: the selection of row r may be read once row_ready[r] != 0
   // (raised by the top-k after writing it); null: wait for the kernel before.
   const uint32_t* row_ready = nullptr;
