@@ -2,6 +2,7 @@
 """Benchmark of one DSA decode step (indexer scan -> top-k -> sparse MQA) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py --layers 8 --route own|prev --retention R   (several DSA layers per step)
 
 Default workload: batched paged decode, B=32 sequences with lengths drawn
 uniformly in [65536, 131072], 64-token blocks under a random block permutation,
