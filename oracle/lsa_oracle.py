@@ -276,3 +276,37 @@ def decode_layers(layers, retention: int, route: int):
         att = [row_attention(c, r, idx[r]) for r in range(c.rows)]
         res.append((idx, np.stack([a[0] for a in att]), np.stack([a[1] for a in att])))
     return src, res
+
+
+# --------------------------------------------------------------------------- two-stage indexer
+# The LeanSparse episode page (summary paragraph) proposes, for decode, to
+# search compact indexer keys and fetch only a short list of the original keys
+# to rank exactly.  Readings where the page is silent: the compact keys are
+# e4m3 with one fp32 scale per token (the FP8 indexer-key form); the short
+# list is the n_cand best tokens by their compact scores (ties to the lower
+# position, as the top-k); the exact ranking is the top-k of those candidates
+# by their scores with the original keys.
+
+def compact_row_scores(case, compact_bits: np.ndarray, compact_scales: np.ndarray, r: int) -> np.ndarray:
+    """Scores of row r over its sequence with the compact keys (fp64)."""
+    s = case.spec
+    b = int(case.row_seq[r])
+    L = int(case.seq_lens[b])
+    pos = np.arange(L)
+    keys = e4m3_to_f64(cache_rows(compact_bits, b, pos, case.block_table, s.block_size, s.stride))
+    scales = cache_rows(compact_scales, b, pos, case.block_table, s.block_size, s.stride).astype(np.float64)
+    qi = decode(case.q_idx[r], s.act_dtype)
+    return indexer_scores(qi, case.w[r].astype(np.float64), keys, scales, None)
+
+
+def two_stage_select(case, compact_bits: np.ndarray, compact_scales: np.ndarray, r: int, k: int,
+                     n_cand: int) -> np.ndarray:
+    """Row r's selection by the two-stage search: the n_cand candidates of the
+    compact scores, ranked by their exact scores (the case's own keys); k
+    positions sorted ascending, -1 padded."""
+    L = row_visible(case, r)
+    cand = topk(compact_row_scores(case, compact_bits, compact_scales, r), L, n_cand)
+    cand = cand[cand >= 0]
+    exact = np.full(L, -np.inf)
+    exact[cand] = row_scores(case, r)[cand]
+    return topk(exact, L, k)

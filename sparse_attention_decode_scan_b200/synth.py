@@ -267,6 +267,18 @@ def make_case(spec: Spec, seed: int, layer: int = 0) -> Case:
     return Case(s, seed, seq_lens, bt, idx_keys, scales, kv, row_seq, row_pos, q_idx, w, q)
 
 
+def compact_keys(idx_keys_bf16: np.ndarray):
+    """A compact copy of bf16 indexer keys, as a cache would store it next to
+    the originals: e4m3 bits of key / scale with one fp32 scale per token
+    (its largest magnitude over 448; 1 for an all-zero key).  Returns (bits,
+    scales) with the keys' leading shape."""
+    import torch
+    k = torch.from_numpy(np.ascontiguousarray(idx_keys_bf16).view(np.int16)).view(torch.bfloat16).float().numpy()
+    amax = np.abs(k).max(axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    return to_e4m3_bits(k / scale[..., None]), scale
+
+
 def queries(spec: Spec, seed: int, rows: int, layer: int = 0):
     """The query rows of one layer (as make_case draws them): indexer queries
     q_idx [rows, H_I, d_I], weights w [rows, H_I] and attention queries q
@@ -363,6 +375,6 @@ def flops_prefill_scan(case: Case) -> int:
 
 
 __all__ = ["Spec", "Case", "WORKLOADS", "workload", "TINY", "DECODE_B1", "DECODE_B32", "DECODE_B4_FP8",
-           "PREFILL", "make_case", "make_layers", "queries", "scaled", "seed_of", "normal", "rng",
+           "PREFILL", "make_case", "make_layers", "queries", "compact_keys", "scaled", "seed_of", "normal", "rng",
            "to_bf16_bits", "to_e4m3_bits", "topk_scores", "index_lists",
            "nbytes_decode_step", "flops_prefill_scan"]
