@@ -110,7 +110,7 @@ typedef enum {
   LSA_OP_ATTN = 2,
   LSA_OP_DECODE_STEP = 3,
   LSA_OP_DECODE_STEP_FUSED = 4, /* lsa_launch_count only: lsa_decode_step with LSA_STEP_FUSED */
-  LSA_OP_DECODE_LAYERS = 5      /* lsa_decode_layers (workspace size only) */
+  LSA_OP_DECODE_LAYERS = 5      /* lsa_decode_layers (lsa_workspace_size; see lsa_launch_count) */
 } lsa_op;
 
 /* Flags of lsa_decode_step. */
@@ -286,7 +286,10 @@ lsa_status lsa_topk_noalloc(const float* scores, int64_t ld, int32_t rows, const
  * capture; runtime memsets are not counted.  LSA_OP_DECODE_STEP_FUSED gives
  * 1 when the fused step applies to these shapes, else the separate launches'
  * count (the device can still refuse the cooperative launch at run time, in
- * which case the step falls back to them).  -1 on invalid arguments.
+ * which case the step falls back to them).  LSA_OP_DECODE_LAYERS gives -1:
+ * lsa_decode_layers enqueues, per layer, the launches of LSA_OP_DECODE_STEP
+ * for a layer that keeps an indexer and of LSA_OP_ATTN for the others.  -1 on
+ * invalid arguments.
  */
 int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t op, int32_t causal);
 
