@@ -568,6 +568,9 @@ def run_layers(args, world, rank, local):
         n * (nb["kv_gather"] + nb["q"] + nb["out"])
     ms_per_step = timed_ms / args.steps
     gbs = step_bytes / (ms_per_step / 1e3) / 1e9
+    # kernels of the timed steps: a layer with an indexer launches a decode step's, the others an attention's
+    launches = args.steps * (n_ind * lsa.launch_count(dc0.dims, B, dc0.max_len, lsa.LSA_OP_DECODE_STEP) +
+                             (n - n_ind) * lsa.launch_count(dc0.dims, B, dc0.max_len, lsa.LSA_OP_ATTN))
     route_name = "MLI (previous indexer layer)" if route == lsa.LSA_ROUTE_PREV else \
         ("DSA (own selection)" if args.retention == 1 else "IndexCache (latest indexer layer)")
     line = {"metric": f"decode steps/s over {n} layers, {route_name}, retention 1/{args.retention}",
@@ -580,7 +583,7 @@ def run_layers(args, world, rank, local):
             "config": dict(workload_config(case), layers=n, retention=args.retention, route=args.route,
                            indexer_layers=n_ind),
             "step_hbm_gbs": gbs, "step_hbm_frac": gbs / peaks["hbm_gbs"], "step_algorithmic_bytes": step_bytes,
-            "peak_source": peak_src, "gpu_launches": None, "clocks": clk.summary()}
+            "peak_source": peak_src, "gpu_launches": launches, "clocks": clk.summary()}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
