@@ -338,6 +338,15 @@ int64_t split_select_min_cols() {
   return e && e[0] ? strtoll(e, nullptr, 10) : kSplitSelectMinCols;
 }
 
+// LSA_TEST_SCAN_WAIT_EXTRA=n (tests only) raises the count of scan CTAs the
+// decode step's top-k waits for by n: that count is never reached, so the
+// top-k's and then the attention's bounded waits run out and record
+// LSA_ERR_TIMEOUT, without any fault.
+uint32_t test_scan_wait_extra() {
+  const char* e = getenv("LSA_TEST_SCAN_WAIT_EXTRA");
+  return e && e[0] ? static_cast<uint32_t>(strtoul(e, nullptr, 10)) : 0u;
+}
+
 static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const void* q_idx, const float* w,
                                    const void* q, void* out, float* lse, int32_t* idx_out, int32_t flags, void* ws,
                                    size_t ws_bytes, lsa_stream_t stream, void* const* events) {
@@ -416,7 +425,8 @@ static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const 
     split.idx_w = idx_out;
   }
   st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, idx, ws, inner, s, hist_done, true,
-               handoff ? scan_done : nullptr, handoff ? static_cast<uint32_t>(scan_tc_grid()) : 0u, split_sel);
+               handoff ? scan_done : nullptr,
+               handoff ? static_cast<uint32_t>(scan_tc_grid()) + test_scan_wait_extra() : 0u, split_sel);
   if (st != LSA_OK) return st;
   if (!mark(2)) return LSA_ERR_CUDA;
   st = do_attn(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes, s, true,
