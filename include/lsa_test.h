@@ -1,0 +1,43 @@
+/*
+ * lsa_test.h -- test-only switches of liblsa_test.so.
+ *
+ * liblsa_test.so is built from the same sources as liblsa.so, with one extra
+ * entry point.  The product library liblsa.so does not export it and has no
+ * switch of any kind (no environment variable is read): a serving process
+ * cannot change its kernel path or break its handoffs by accident.  Tests load
+ * liblsa_test.so when they need one of the switches below, and liblsa.so
+ * otherwise.  The paper has no counterpart of this file.
+ */
+#ifndef LSA_TEST_H_
+#define LSA_TEST_H_
+
+#include "lsa.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * Sets the switches for every later call into liblsa_test.so in this process
+ * (process-wide, not thread-safe: set them before the calls they affect).
+ *   force_simt_path        != 0: every call runs the CUDA-core kernels instead
+ *                          of the tensor-core ones (to compare the two GPU
+ *                          paths on the same inputs); 0: the normal choice.
+ *   split_select_min_cols  rows of at least this many positions take the split
+ *                          select inside lsa_decode_step; < 0: the library's
+ *                          default (2^18).
+ *   scan_wait_extra        added to the count of scan CTAs that the decode
+ *                          step's top-k waits for.  Any value > 0 makes that
+ *                          count unreachable, so the top-k's bounded wait and
+ *                          then the attention's run out after about a second
+ *                          each and record LSA_ERR_TIMEOUT in the status word
+ *                          (the failure path of the handoff, without a fault).
+ * Returns LSA_OK.
+ */
+lsa_status lsa_test_set_hooks(int32_t force_simt_path, int64_t split_select_min_cols, uint32_t scan_wait_extra);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_TEST_H_ */

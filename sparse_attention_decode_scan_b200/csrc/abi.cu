@@ -9,6 +9,9 @@
 #include "common.cuh"
 #include "internal.h"
 #include "lsa.h"
+#ifdef LSA_TEST_HOOKS
+#include "lsa_test.h"
+#endif
 
 namespace lsa {
 namespace {
@@ -19,13 +22,28 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// LSA_FORCE_SIMT=1 routes every call to the CUDA-core kernels (a debugging aid
-// for comparing the two GPU paths); default is the tensor-core path wherever
-// its shape is supported.
-bool force_simt() {
-  const char* e = getenv("LSA_FORCE_SIMT");
-  return e && e[0] == '1';
-}
+// Rows at least this long take the split select in a decode step.
+constexpr int64_t kSplitSelectMinCols = int64_t(1) << 18;
+
+#ifdef LSA_TEST_HOOKS
+// Test build only (liblsa_test.so, include/lsa_test.h): switches that tests
+// set through lsa_test_set_hooks.  The product library has none of them, so
+// nothing in a serving process (no environment variable, no call) can change
+// its path or break its handoffs.
+struct TestHooks {
+  bool force_simt = false;                         // every call on the CUDA-core kernels
+  int64_t split_select_min_cols = kSplitSelectMinCols;
+  uint32_t scan_wait_extra = 0;                    // raises the decode step's scan-CTA count
+};
+TestHooks g_hooks;
+bool force_simt() { return g_hooks.force_simt; }
+int64_t split_select_min_cols() { return g_hooks.split_select_min_cols; }
+uint32_t test_scan_wait_extra() { return g_hooks.scan_wait_extra; }
+#else
+constexpr bool force_simt() { return false; }
+constexpr int64_t split_select_min_cols() { return kSplitSelectMinCols; }
+constexpr uint32_t test_scan_wait_extra() { return 0u; }
+#endif
 
 bool valid_dims(const lsa_dims* d) {
   if (!d) return false;
@@ -269,7 +287,7 @@ size_t lsa_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int3
       return kStatusBytes + scores_ws(rows, true);
     case LSA_OP_TOPK:
       if (!d || d->top_k < 1) return 0;
-      return kStatusBytes + align_up(topk_ws_bytes(rows, max_len, d->top_k));
+      return topk_call_bytes(rows, max_len, d->top_k);
     case LSA_OP_ATTN:
       if (!valid_dims(d)) return 0;
       return kStatusBytes + attn_ws(d, rows);
@@ -302,12 +320,9 @@ lsa_status lsa_indexer_scores(const lsa_dims* d, const lsa_cache* c, int32_t row
 
 lsa_status lsa_topk(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
                     int32_t k, int32_t* idx, void* ws, size_t ws_bytes, lsa_stream_t stream) {
-  if (rows < 0 || k < 1 || n_cols < 0 || ld < n_cols || (ld % 4) != 0) return LSA_ERR_INVALID_ARG;
-  if (rows > 0 && (!scores || !idx || !aligned16(scores))) return LSA_ERR_INVALID_ARG;
-  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
-  if (n_cols > (1LL << 31) - 1) return LSA_ERR_UNSUPPORTED;
-  const size_t need = kStatusBytes + align_up(topk_ws_bytes(rows, n_cols, k));
-  lsa_status st = ws_check(ws, ws_bytes, need);
+  lsa_status st = topk_check_args(scores, ld, rows, n_cols, k, idx);
+  if (st != LSA_OK) return st;
+  st = ws_check(ws, ws_bytes, topk_call_bytes(rows, n_cols, k));
   if (st != LSA_OK) return st;
   if (rows == 0) return LSA_OK;
   return do_topk(scores, ld, rows, valid_len, n_cols, k, idx, ws, static_cast<uint8_t*>(ws) + kStatusBytes,
@@ -327,24 +342,6 @@ lsa_status lsa_sparse_attn_decode(const lsa_dims* d, const lsa_cache* c, int32_t
   if (st != LSA_OK) return st;
   return do_attn(d, c, rows, row_seq, q, idx, out, lse, ws, static_cast<uint8_t*>(ws) + kStatusBytes,
                  ws_bytes - kStatusBytes, reinterpret_cast<cudaStream_t>(stream));
-}
-
-// Rows at least this long take the split select in a decode step (the
-// environment variable LSA_SPLIT_SELECT_MIN_COLS overrides it, for tests).
-constexpr int64_t kSplitSelectMinCols = int64_t(1) << 18;
-
-int64_t split_select_min_cols() {
-  const char* e = getenv("LSA_SPLIT_SELECT_MIN_COLS");
-  return e && e[0] ? strtoll(e, nullptr, 10) : kSplitSelectMinCols;
-}
-
-// LSA_TEST_SCAN_WAIT_EXTRA=n (tests only) raises the count of scan CTAs the
-// decode step's top-k waits for by n: that count is never reached, so the
-// top-k's and then the attention's bounded waits run out and record
-// LSA_ERR_TIMEOUT, without any fault.
-uint32_t test_scan_wait_extra() {
-  const char* e = getenv("LSA_TEST_SCAN_WAIT_EXTRA");
-  return e && e[0] ? static_cast<uint32_t>(strtoul(e, nullptr, 10)) : 0u;
 }
 
 static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const void* q_idx, const float* w,
@@ -591,5 +588,14 @@ const char* lsa_status_string(lsa_status s) {
 }
 
 int32_t lsa_version(void) { return LSA_VERSION; }
+
+#ifdef LSA_TEST_HOOKS
+lsa_status lsa_test_set_hooks(int32_t force_simt_path, int64_t split_select_min_cols_, uint32_t scan_wait_extra) {
+  g_hooks.force_simt = force_simt_path != 0;
+  g_hooks.split_select_min_cols = split_select_min_cols_ < 0 ? kSplitSelectMinCols : split_select_min_cols_;
+  g_hooks.scan_wait_extra = scan_wait_extra;
+  return LSA_OK;
+}
+#endif
 
 }  // extern "C"

@@ -4,6 +4,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "host_util.h"
 #include "internal.h"
 #include "tc.cuh"
 
@@ -33,16 +34,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Clusters of `n` attention CTAs the device keeps resident at once (queried
-// once per n; 0 when clusters of that size are refused).  The cluster merge is
-// used only when all of a launch's clusters fit in one wave, as the split plan
-// assumes.
+// Clusters of `n` attention CTAs the current device keeps resident at once
+// (queried once per device and n, under a lock; 0 when clusters of that size
+// are refused).  The cluster merge is used only when all of a launch's
+// clusters fit in one wave, as the split plan assumes.
 int resident_clusters(int n) {
-  static int cached[17] = {-1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1};
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static int cached[kMaxDev][17];
+  static bool init = false;
   if (n < 2 || n > 16) return 0;
-  if (cached[n] >= 0) return cached[n];
-  cached[n] = 0;
-  if (cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!init) {
+    for (auto& row : cached)
+      for (int& v : row) v = -1;
+    init = true;
+  }
+  if (cached[dev][n] >= 0) return cached[dev][n];
+  cached[dev][n] = 0;
+  if (ensure_dyn_smem(k_attn_tc, kSmemBytes) != cudaSuccess ||
       (n > 8 && cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {
     (void)cudaGetLastError();
     return 0;
@@ -64,7 +79,7 @@ int resident_clusters(int n) {
     (void)cudaGetLastError();
     c = 0;
   }
-  cached[n] = c;
+  cached[dev][n] = c;
   return c;
 }
 
@@ -114,11 +129,9 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   P.counters = reinterpret_cast<int*>(ws);
   P.part_lse = reinterpret_cast<float*>(ws + cnt_b);
   P.part_o = reinterpret_cast<float*>(ws + cnt_b + lse_b);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  {
+    cudaError_t e = ensure_dyn_smem(k_attn_tc, kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const dim3 grid(P.nsplit, 2, a.rows);
   cudaLaunchConfig_t cfg;

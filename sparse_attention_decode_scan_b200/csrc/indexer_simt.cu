@@ -9,6 +9,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "host_util.h"
 #include "internal.h"
 
 namespace lsa {
@@ -95,7 +96,7 @@ cudaError_t launch_t(const ScoresArgs& a, cudaStream_t s) {
   size_t smem = (static_cast<size_t>(MAXH) * a.dI + MAXH) * sizeof(float);
   auto fn = k_scores_simt<KDT, QDT, MAXH>;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = ensure_dyn_smem(fn, smem);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(static_cast<unsigned>((a.ld + kThreads - 1) / kThreads), static_cast<unsigned>(a.rows));

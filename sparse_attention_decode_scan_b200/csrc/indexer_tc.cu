@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include "common.cuh"
+#include "host_util.h"
 #include "internal.h"
 #include "tc.cuh"
 
@@ -100,12 +101,8 @@ cudaError_t launch_t(const ScoresArgs& a, cudaStream_t s) {
   cudaError_t me = make_maps(a, &tmap, &smap);
   if (me != cudaSuccess) return me;
   auto kern = k_scan_tc<KDT, QB>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_dyn_smem(kern, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   kern<<<num_sms(), kThreads, C::kSmemBytes, s>>>(tmap, smap, a);
   return cudaGetLastError();
 }

@@ -64,6 +64,11 @@ struct TopkPlan {
 };
 TopkPlan topk_plan(int32_t rows, int64_t n_cols);
 size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t k);
+// Argument checks of the top-k entry points (lsa_topk, lsa_topk_noalloc), and
+// the bytes either needs: status word plus the 256-aligned top-k scratch.
+lsa_status topk_check_args(const float* scores, int64_t ld, int32_t rows, int64_t n_cols, int32_t k,
+                           const int32_t* idx);
+size_t topk_call_bytes(int32_t rows, int64_t n_cols, int32_t k);
 int topk_launches(int64_t n_cols);
 
 struct TopkArgs {

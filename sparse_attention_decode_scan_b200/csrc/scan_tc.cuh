@@ -15,8 +15,9 @@
 // head reduction then runs in registers.  Decode groups one query row per tile
 // (N = 64); the causal prefill groups 4 rows of one sequence (N = 256), reusing
 // each key tile 4 times.  FP8 keys go straight to kind::f8f6f4 MMAs: the bf16
-// query is split exactly into two e4m3 terms (hi + lo, per-head power-of-two
-// scale folded into w), so N doubles and no key conversion is needed.
+// query is split into two e4m3 terms (hi + lo, per-head power-of-two scale
+// folded into w; exact for entries within 2^10 of the head's largest, see
+// stage_query_fp8), so N doubles and no key conversion is needed.
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0  TMA producer: 64-row boxes of the key cache (block-table gather)
@@ -287,8 +288,13 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 }
 
 // fp8: per (query, head) a power-of-two scale s puts max|q| into [224, 448];
-// q*s = hi + lo with hi = e4m3(q*s), lo = e4m3(q*s - hi), exact for bf16 q
-// (4 + 4 significant bits) outside the e4m3 subnormal range.  B row
+// q*s ~ hi + lo with hi = e4m3(q*s), lo = e4m3(q*s - hi).  A bf16 entry has 8
+// significant bits and each e4m3 term 4, so the split is exact while both
+// terms are normal e4m3 numbers (magnitude >= 2^-6), which holds for
+// |q*s| >= 2^-2, i.e. entries at least 2^-10 of the head's largest.  Smaller
+// entries are not exact: a term in e4m3's subnormal range is rounded to its
+// step 2^-9, an absolute error of at most 2^-10 in scaled units (below 5e-6 of
+// the head's largest entry), well inside the 2e-2 score tolerance.  B row
 // qq*128 + h holds hi, qq*128 + 64 + h holds lo; w' = w / s.
 // The raw rows and the weights arrive by cp.async in one round trip; half a
 // warp then converts one head (8 dims per lane) from shared memory.

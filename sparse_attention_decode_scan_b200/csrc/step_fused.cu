@@ -21,6 +21,7 @@
 
 #include "attn_tc.cuh"
 #include "common.cuh"
+#include "host_util.h"
 #include "internal.h"
 #include "scan_tc.cuh"
 #include "tc.cuh"
@@ -142,11 +143,9 @@ template <int KDT>
 cudaError_t launch_t(const FusedParams& F, const CUtensorMap& tmap, const CUtensorMap& smap, cudaStream_t s) {
   const size_t smem = fused_smem<KDT>(F.topk.n_cols);
   auto kern = k_step_fused<KDT>;
-  static size_t smem_set = 0;
-  if (smem > smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  {
+    cudaError_t e = ensure_dyn_smem(kern, smem);
     if (e != cudaSuccess) return e;
-    smem_set = smem;
   }
   // every CTA must be resident at once (the grid barriers wait for all of them)
   int per_sm = 0;

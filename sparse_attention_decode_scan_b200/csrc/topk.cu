@@ -24,6 +24,7 @@
 #include <string.h>
 
 #include "common.cuh"
+#include "host_util.h"
 #include "internal.h"
 #include "tc.cuh"
 #include "topk_sel.cuh"
@@ -450,13 +451,8 @@ size_t topk_hist_zero_bytes(int32_t rows) { return tk::tk_zero_bytes(rows); }
 cudaError_t rows_plan(int32_t rows, int64_t n_cols, size_t* smem_out, TopkPlan* plan) {
   size_t smem = tk::tk_final_smem(n_cols, tk::kCollectThreads);
   if (tk::tk_split_smem() > smem) smem = tk::tk_split_smem();
-  static size_t smem_set = 0;
-  if (smem > 48 * 1024 && smem > smem_set) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(k_tk_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    smem_set = smem;
-  }
+  const cudaError_t e = ensure_dyn_smem(k_tk_rows, smem);
+  if (e != cudaSuccess) return e;
   *smem_out = smem;
   *plan = topk_collect_plan(rows, n_cols, rows_ctas_per_sm(smem) * device_sms());
   return cudaSuccess;
@@ -486,6 +482,19 @@ size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t) {
   TopkPlan p = topk_plan(rows, n_cols);
   size_t b = R * kHistStride * 4 + R * p.nseg * 8;
   return (b + 255) / 256 * 256;
+}
+
+lsa_status topk_check_args(const float* scores, int64_t ld, int32_t rows, int64_t n_cols, int32_t k,
+                           const int32_t* idx) {
+  if (rows < 0 || k < 1 || n_cols < 0 || ld < n_cols || (ld % 4) != 0) return LSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!scores || !idx || (reinterpret_cast<uintptr_t>(scores) & 15u) != 0)) return LSA_ERR_INVALID_ARG;
+  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
+  if (n_cols > (1LL << 31) - 1) return LSA_ERR_UNSUPPORTED;
+  return LSA_OK;
+}
+
+size_t topk_call_bytes(int32_t rows, int64_t n_cols, int32_t k) {
+  return kStatusBytes + (topk_ws_bytes(rows, n_cols, k) + 255) / 256 * 256;
 }
 
 int topk_launches(int64_t n_cols) { return topk_v2_ok(n_cols) ? 2 : 5; }
@@ -593,11 +602,9 @@ cudaError_t static_scratch(void** out) {
 extern "C" lsa_status lsa_topk_noalloc(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len,
                                        int64_t n_cols, int32_t k, int32_t* idx, lsa_stream_t stream) {
   using namespace lsa;
-  if (rows < 0 || k < 1 || n_cols < 0 || ld < n_cols || (ld % 4) != 0) return LSA_ERR_INVALID_ARG;
-  if (rows > 0 && (!scores || !idx || (reinterpret_cast<uintptr_t>(scores) & 15u) != 0)) return LSA_ERR_INVALID_ARG;
-  if (n_cols > (1LL << 31) - 1) return LSA_ERR_UNSUPPORTED;
-  const size_t need = kStatusBytes + topk_ws_bytes(rows, n_cols, k);
-  if (need > kStaticScratchBytes) return LSA_ERR_UNSUPPORTED;  // beyond the static scratch
+  const lsa_status st = topk_check_args(scores, ld, rows, n_cols, k, idx);
+  if (st != LSA_OK) return st;
+  if (topk_call_bytes(rows, n_cols, k) > kStaticScratchBytes) return LSA_ERR_UNSUPPORTED;  // beyond the static scratch
   if (rows == 0) return LSA_OK;
   void* base = nullptr;
   if (static_scratch(&base) != cudaSuccess) return LSA_ERR_CUDA;

@@ -13,6 +13,8 @@ from typing import Optional
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblsa.so")
+# Test build (include/lsa_test.h): the same kernels plus lsa_test_set_hooks.
+TEST_LIB_PATH = os.path.join(_HERE, "liblsa_test.so")
 
 LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_TIMEOUT, \
     LSA_ERR_BOUNDS = range(7)
@@ -46,18 +48,35 @@ class Cache(ctypes.Structure):
                 ("max_len", ctypes.c_int64), ("seq_lens", ctypes.c_void_p), ("batch", ctypes.c_int32)]
 
 
-_lib = None
+_libs = {}
+_use_test = False
+
+
+def use_test_library(on: bool = True) -> None:
+    """Routes every later call of this binding to liblsa_test.so (on) or back to liblsa.so.
+    Only tests do this, to reach lsa_test_set_hooks."""
+    global _use_test
+    _use_test = bool(on)
+
+
+def set_test_hooks(force_simt: bool = False, split_select_min_cols: int = -1, scan_wait_extra: int = 0) -> None:
+    """lsa_test_set_hooks of liblsa_test.so (include/lsa_test.h); needs use_test_library()."""
+    if not _use_test:
+        raise RuntimeError("test hooks exist only in liblsa_test.so: call use_test_library() first")
+    _check(lib().lsa_test_set_hooks(1 if force_simt else 0, int(split_select_min_cols), int(scan_wait_extra)),
+           "lsa_test_set_hooks")
 
 
 def lib() -> ctypes.CDLL:
-    """Loads liblsa.so once; raises if it is absent (no fallback path exists)."""
-    global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"liblsa.so not built at {LIB_PATH}; run "
+    """Loads liblsa.so (or, after use_test_library(), liblsa_test.so) once; raises if it is absent
+    (no fallback path exists)."""
+    path = TEST_LIB_PATH if _use_test else LIB_PATH
+    if path in _libs:
+        return _libs[path]
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} not built at {path}; run "
                           "`python -m sparse_attention_decode_scan_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     D, C = ctypes.POINTER(Dims), ctypes.POINTER(Cache)
     L.lsa_workspace_size.argtypes = [D, i32, i64, i32]
@@ -76,11 +95,14 @@ def lib() -> ctypes.CDLL:
     L.lsa_version.restype = i32
     L.lsa_launch_count.argtypes = [D, i32, i64, i32, i32]
     L.lsa_launch_count.restype = i32
-    for f in ("lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode", "lsa_decode_step",
-              "lsa_decode_step_profiled", "lsa_decode_layers",
-              "lsa_read_device_status"):
+    names = ["lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode", "lsa_decode_step",
+             "lsa_decode_step_profiled", "lsa_decode_layers", "lsa_read_device_status"]
+    if path == TEST_LIB_PATH:
+        L.lsa_test_set_hooks.argtypes = [i32, i64, ctypes.c_uint32]
+        names.append("lsa_test_set_hooks")
+    for f in names:
         getattr(L, f).restype = ctypes.c_int
-    _lib = L
+    _libs[path] = L
     return L
 
 

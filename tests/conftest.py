@@ -25,3 +25,16 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture
+def test_hooks():
+    """Routes the binding to liblsa_test.so (the product library has no switches) and yields its
+    hook setter; restores the defaults and the product library afterwards."""
+    from sparse_attention_decode_scan_b200 import lsa
+    lsa.use_test_library(True)
+    try:
+        yield lsa.set_test_hooks
+    finally:
+        lsa.set_test_hooks()
+        lsa.use_test_library(False)

@@ -12,6 +12,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "lsa.h")
+TEST_HEADER = os.path.join(ROOT, "include", "lsa_test.h")
 
 
 @pytest.fixture(scope="module")
@@ -23,8 +24,8 @@ def lsa():
     return binding
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(lsa_[a-z_]+)\s*\(", text)))
 
@@ -40,6 +41,26 @@ def test_every_declared_symbol_is_exported(lsa):
     lib = lsa.lib()
     for n in declared_functions():
         assert hasattr(lib, n), f"{n} declared in lsa.h but not exported"
+
+
+def test_test_library_exports_both_headers_and_the_product_no_switch(lsa):
+    """liblsa_test.so exports lsa.h and lsa_test.h; liblsa.so exports nothing of lsa_test.h."""
+    import ctypes as C
+    test_only = declared_functions(TEST_HEADER)
+    assert test_only == ["lsa_test_set_hooks"]
+    prod = C.CDLL(lsa.LIB_PATH)
+    for n in test_only:
+        assert not hasattr(prod, n), f"{n} must exist only in the test build"
+    test_lib = C.CDLL(lsa.TEST_LIB_PATH)
+    for n in declared_functions() + test_only:
+        assert hasattr(test_lib, n), f"{n} not exported by liblsa_test.so"
+
+
+def test_product_library_reads_no_environment():
+    """The product path has no environment switch: no source of the library calls getenv."""
+    import glob
+    for f in glob.glob(os.path.join(ROOT, "sparse_attention_decode_scan_b200", "csrc", "*")):
+        assert "getenv" not in open(f).read(), f"{os.path.basename(f)} reads the environment"
 
 
 def test_version_and_status_strings(lsa):

@@ -34,9 +34,9 @@ def _visible(case):
 
 @pytest.mark.parametrize("path", ["default", "simt"])
 @pytest.mark.parametrize("name", ["tiny_fp32", "bf16_L5000", "paged_B5", "prefill_3000x256", "len1", "paged48_B3"])
-def test_attention_on_given_indices(name, path, monkeypatch):
+def test_attention_on_given_indices(name, path, request):
     if path == "simt":
-        monkeypatch.setenv("LSA_FORCE_SIMT", "1")
+        request.getfixturevalue("test_hooks")(force_simt=True)
     case = cases.small(name)
     k = case.spec.top_k
     idx = synth.index_lists(case.rows, k, _visible(case), 600 + k)

@@ -54,9 +54,9 @@ def test_host_argument_errors():
 
 
 @pytest.mark.parametrize("path", ["default", "simt"])
-def test_block_id_out_of_pool_is_reported(path, monkeypatch):
+def test_block_id_out_of_pool_is_reported(path, request):
     if path == "simt":
-        monkeypatch.setenv("LSA_FORCE_SIMT", "1")
+        request.getfixturevalue("test_hooks")(force_simt=True)
     from sparse_attention_decode_scan_b200 import lsa
     dc = _dc()
     bt = dc.block_table.clone()

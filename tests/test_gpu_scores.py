@@ -37,9 +37,9 @@ def _check_rows(case, scores, rows):
 
 @pytest.mark.parametrize("path", ["default", "simt"])
 @pytest.mark.parametrize("name", list(cases.SMALL))
-def test_scores_small(name, path, monkeypatch):
+def test_scores_small(name, path, request):
     if path == "simt":
-        monkeypatch.setenv("LSA_FORCE_SIMT", "1")
+        request.getfixturevalue("test_hooks")(force_simt=True)
     case = cases.small(name)
     scores = _run_scores(case)
     _check_rows(case, scores, range(case.rows))

@@ -143,6 +143,51 @@ def test_prefill_chain_small():
 
 
 @pytest.mark.slow
+def test_prefill_chain_full():
+    """The full prefill workload (8192 chunk rows at positions 131072..139263
+    over 139264 tokens, causal): lsa_indexer_scores with the rows' positions,
+    lsa_topk over every row, lsa_sparse_attn_decode for every row, in the
+    launch configuration the benchmark times.  Checked on sampled rows (first,
+    last and random): the selection against the oracle's top-k of the oracle's
+    scores, and the attention run on the oracle's selection against the
+    oracle's attention."""
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+    case = cases.full(synth.PREFILL)
+    dc = DeviceCase(case)
+    R, k = dc.rows, case.spec.top_k
+    L = int(case.seq_lens[0])
+    ld = (dc.max_len + 3) // 4 * 4
+    scores = torch.empty((R, ld), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(max(lsa.workspace_size(dc.dims, R, dc.max_len, op) for op in range(3)))
+    lsa.indexer_scores(dc.dims, dc.cache, dc.q_idx, dc.w, scores, ld, ws, row_seq=dc.row_seq, row_pos=dc.row_pos)
+    idx = torch.empty((R, k), dtype=torch.int32, device="cuda")
+    lsa.topk(scores, k, idx, ws, n_cols=L, ld=ld)
+    out = torch.empty((R, case.spec.n_heads, case.spec.v_dim), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((R, case.spec.n_heads), dtype=torch.float32, device="cuda")
+    lsa.sparse_attn_decode(dc.dims, dc.cache, dc.q, idx, out, lse, ws, row_seq=dc.row_seq)
+    torch.cuda.synchronize()
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    idx_h = idx.cpu().numpy()
+    out_h = out.float().cpu().numpy()
+    lse_h = lse.cpu().numpy()
+    g = np.random.default_rng(8192)
+    rows = sorted({0, 1, R - 1, *g.integers(2, R - 1, 5).tolist()})
+    ref_sel = np.full((R, k), -1, np.int32)
+    for r in rows:
+        sc = O.row_scores(case, r)
+        ref_sel[r] = O.topk(sc, L, k)
+        check_selection(idx_h[r], ref_sel[r], sc, what=f"prefill row {r}")
+        assert (idx_h[r][idx_h[r] >= 0] <= case.row_pos[r]).all()
+    o_on_ref, l_on_ref = _attn_on(dc, ref_sel)
+    for r in rows:
+        o_ref, l_ref = O.row_attention(case, r, ref_sel[r])
+        check_attention(o_on_ref[r], o_ref, l_on_ref[r], l_ref, what=f"prefill attention row {r}")
+        if np.array_equal(idx_h[r], ref_sel[r]):
+            check_attention(out_h[r], o_ref, lse_h[r], l_ref, what=f"prefill chain row {r}")
+
+
+@pytest.mark.slow
 @pytest.mark.parametrize("name", [synth.DECODE_B1, synth.DECODE_B32])
 def test_decode_step_full(name):
     case = cases.full(name)
@@ -213,14 +258,14 @@ def _split_case():
     return case
 
 
-@pytest.mark.parametrize("min_cols", ["0", "100000000"])
-def test_decode_step_split_select(min_cols, monkeypatch):
+@pytest.mark.parametrize("min_cols", [0, 100000000])
+def test_decode_step_split_select(min_cols, test_hooks):
     """With the split select forced on (rows of any length) or off, the decode
     step selects what lsa_indexer_scores + lsa_topk select, ties and the
     fallback row included, and its outputs match the oracle."""
     from sparse_attention_decode_scan_b200 import lsa
     from sparse_attention_decode_scan_b200.device import DeviceCase
-    monkeypatch.setenv("LSA_SPLIT_SELECT_MIN_COLS", min_cols)
+    test_hooks(split_select_min_cols=min_cols)
     case = _split_case()
     dc = DeviceCase(case)
     _, _, idx_step = _step(dc)

@@ -24,6 +24,10 @@ CASES = [
     ("normal", 4, 3000, 64, "with_zero"),      # a row with no valid entry
     ("ties", 40, 139264, 2048, "ragged"),      # many rows
     ("equal", 1, 200000, 2048, "full"),        # one tie class spread over many segments
+    # rows longer than 2^19 positions take the general five-launch path
+    ("normal", 2, 600000, 2048, "full"),
+    ("ties", 2, 600000, 2048, "ragged"),
+    ("heavy", 1, 1 << 20, 4096, "full"),
 ]
 
 
