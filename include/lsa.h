@@ -249,6 +249,58 @@ lsa_status lsa_decode_layers(const lsa_dims* d, int32_t n_layers, const lsa_cach
                              int32_t* idx_out, void* ws, size_t ws_bytes, lsa_stream_t stream);
 
 /*
+ * Exact indexer scores of given candidate positions (the second stage of the
+ * two-stage search below): for row r and entry j < n_cand,
+ *   scores[r][j] = I(cand[r][j]) over the cache's own (original) keys,
+ * the score of step 1 at that position.
+ *   row_seq, row_pos, q_idx, w: as lsa_indexer_scores.
+ *   cand   [rows, n_cand] device int32: positions (any order, -1 = none).
+ *   scores [rows, ld] device fp32 out, ld >= n_cand: -inf for -1 entries and
+ *          for [n_cand, ld); NaN (and LSA_ERR_BOUNDS in the status word) for a
+ *          position outside the row's visible range or a bad block.
+ * Supported: bf16 keys and queries, 64 x 128 indexer heads (else
+ * LSA_ERR_UNSUPPORTED); any block size.  Workspace: 256 bytes (status word).
+ */
+lsa_status lsa_candidate_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows,
+                                const int32_t* row_seq, const int32_t* row_pos,
+                                const void* q_idx, const float* w, const int32_t* cand,
+                                int32_t n_cand, float* scores, int64_t ld,
+                                void* ws, size_t ws_bytes, lsa_stream_t stream);
+
+/*
+ * Two-stage selection (LeanSparse episode page, summary: during decode, search
+ * compact indexer keys and fetch only a short list of the originals to rank
+ * exactly).  For each query row:
+ *   1. compact scores: step 1 over the compact keys, e4m3 with one fp32 scale
+ *      per token (K ~ scale * e4m3, the FP8 key form);
+ *   2. the short list: the n_cand positions with the highest compact scores
+ *      (ties to the lower position);
+ *   3. their exact scores over the original bf16 keys of `c`;
+ *   4. the k = d->top_k best of the list by exact score (ties to the lower
+ *      position), sorted ascending, -1 padded -> idx [rows, k].
+ * The original keys are read only at the n_cand listed positions: per row the
+ * bytes of the scan drop from L * 256 to L * 132 + n_cand * 256.
+ *   c               the cache with its original bf16 keys (d->idx_key_dtype =
+ *                   LSA_BF16); kv is not read.
+ *   compact_keys    e4m3 bytes in the layout of c->idx_keys (1 byte per dim).
+ *   compact_scales  fp32, one per token, in the layout of FP8 key scales.
+ *   n_cand          >= k; with n_cand >= the row's length the result is the
+ *                   exact top-k of step 2.
+ * Workspace: lsa_two_stage_workspace_size(d, rows, c->max_len, n_cand).
+ * Errors: LSA_ERR_INVALID_ARG (n_cand < k, missing or misaligned pointers),
+ * LSA_ERR_UNSUPPORTED (other than bf16 keys and queries with 64 x 128 indexer
+ * heads and block sizes that are multiples of 64), LSA_ERR_WORKSPACE,
+ * LSA_ERR_CUDA.  Launches: scan, top-k (2), candidate scores, top-k (2), and
+ * one kernel that maps list entries to positions.
+ */
+size_t lsa_two_stage_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t n_cand);
+lsa_status lsa_two_stage_select(const lsa_dims* d, const lsa_cache* c, const void* compact_keys,
+                                const float* compact_scales, int32_t rows, const int32_t* row_seq,
+                                const int32_t* row_pos, const void* q_idx, const float* w,
+                                int32_t n_cand, int32_t* idx, void* ws, size_t ws_bytes,
+                                lsa_stream_t stream);
+
+/*
  * Copies the workspace status word to *status (an lsa_status value), clears it,
  * and synchronises `stream`.  Returns LSA_ERR_CUDA if a CUDA call fails.
  */

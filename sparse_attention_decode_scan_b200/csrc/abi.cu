@@ -146,6 +146,34 @@ LayersLayout layers_layout(const lsa_dims* d, int32_t rows, int64_t max_len) {
   return L;
 }
 
+// The two-stage search (lsa_two_stage_select): the compact scores, the
+// candidate list, the candidates' exact scores, the chosen candidate entries,
+// and the scratch of the scans and the two top-k calls.
+struct TwoStageLayout {
+  size_t cscores_off, cand_off, exact_off, slot_off, inner_off, inner_bytes, total;
+  int64_t ld_c, ld_x;
+};
+
+TwoStageLayout two_stage_layout(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t n_cand) {
+  TwoStageLayout L;
+  const size_t R = static_cast<size_t>(rows);
+  L.ld_c = score_ld(max_len);
+  L.ld_x = score_ld(n_cand);
+  L.cscores_off = kStatusBytes;
+  L.cand_off = L.cscores_off + align_up(R * L.ld_c * 4);
+  L.exact_off = L.cand_off + align_up(R * static_cast<size_t>(n_cand) * 4);
+  L.slot_off = L.exact_off + align_up(R * L.ld_x * 4);
+  L.inner_off = L.slot_off + align_up(R * static_cast<size_t>(d->top_k) * 4);
+  size_t inner = topk_ws_bytes(rows, max_len, n_cand);
+  const size_t t2 = topk_ws_bytes(rows, n_cand, d->top_k);
+  const size_t sc = scores_ws(rows, true);
+  if (t2 > inner) inner = t2;
+  if (sc > inner) inner = sc;
+  L.inner_bytes = align_up(inner);
+  L.total = L.inner_off + L.inner_bytes;
+  return L;
+}
+
 lsa_status ws_check(void* ws, size_t have, size_t need) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LSA_ERR_WORKSPACE;
   if (have < need) return LSA_ERR_WORKSPACE;
@@ -524,6 +552,82 @@ lsa_status lsa_decode_layers(const lsa_dims* d, int32_t n_layers, const lsa_cach
       return LSA_ERR_CUDA;
   }
   return LSA_OK;
+}
+
+lsa_status lsa_candidate_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
+                                const int32_t* row_pos, const void* q_idx, const float* w, const int32_t* cand,
+                                int32_t n_cand, float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                                lsa_stream_t stream) {
+  if (!valid_dims(d) || !valid_cache(d, c, true, false)) return LSA_ERR_INVALID_ARG;
+  if (rows < 0 || n_cand < 0 || ld < n_cand) return LSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!q_idx || !w || !scores || !aligned16(q_idx) || (n_cand > 0 && !cand)))
+    return LSA_ERR_INVALID_ARG;
+  if (!row_seq && rows > c->batch) return LSA_ERR_INVALID_ARG;
+  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
+  lsa_status st = ws_check(ws, ws_bytes, kStatusBytes);
+  if (st != LSA_OK) return st;
+  if (rows == 0 || ld == 0) return LSA_OK;
+  ScoresArgs a = scores_args(d, c, rows, row_seq, row_pos, q_idx, w, scores, ld, ws, nullptr, 0);
+  a.cand = cand;
+  a.cand_ld = n_cand;
+  if (!candidate_scores_tc_supported(a)) return LSA_ERR_UNSUPPORTED;
+  return cuda_status(launch_candidate_scores_tc(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t lsa_two_stage_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t n_cand) {
+  if (!valid_dims(d) || rows < 0 || max_len < 0 || n_cand < d->top_k) return 0;
+  return two_stage_layout(d, rows, max_len, n_cand).total;
+}
+
+lsa_status lsa_two_stage_select(const lsa_dims* d, const lsa_cache* c, const void* compact_keys,
+                                const float* compact_scales, int32_t rows, const int32_t* row_seq,
+                                const int32_t* row_pos, const void* q_idx, const float* w, int32_t n_cand,
+                                int32_t* idx, void* ws, size_t ws_bytes, lsa_stream_t stream) {
+  if (!valid_dims(d) || !valid_cache(d, c, true, false)) return LSA_ERR_INVALID_ARG;
+  if (rows < 0 || n_cand < d->top_k) return LSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!q_idx || !w || !idx || !aligned16(q_idx) || !compact_keys || !compact_scales ||
+                   !aligned16(compact_keys) || !aligned16(compact_scales)))
+    return LSA_ERR_INVALID_ARG;
+  if (!row_seq && rows > c->batch) return LSA_ERR_INVALID_ARG;
+  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
+  if (d->idx_key_dtype != LSA_BF16 || d->act_dtype != LSA_BF16) return LSA_ERR_UNSUPPORTED;
+  const TwoStageLayout L = two_stage_layout(d, rows, c->max_len, n_cand);
+  lsa_status st = ws_check(ws, ws_bytes, L.total);
+  if (st != LSA_OK) return st;
+  if (rows == 0) return LSA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* cscores = reinterpret_cast<float*>(base + L.cscores_off);
+  int32_t* cand = reinterpret_cast<int32_t*>(base + L.cand_off);
+  float* exact = reinterpret_cast<float*>(base + L.exact_off);
+  int32_t* slot = reinterpret_cast<int32_t*>(base + L.slot_off);
+  void* inner = base + L.inner_off;
+  // 1. the compact keys: e4m3 with a per-token scale, the FP8 scan
+  lsa_dims d8 = *d;
+  d8.idx_key_dtype = LSA_FP8_E4M3;
+  lsa_cache c8 = *c;
+  c8.idx_keys = compact_keys;
+  c8.idx_key_scales = compact_scales;
+  ScoresArgs sa = scores_args(&d8, &c8, rows, row_seq, row_pos, q_idx, w, cscores, L.ld_c, ws, inner, L.inner_bytes);
+  if (!scores_tc_supported(sa)) return LSA_ERR_UNSUPPORTED;
+  st = do_scores(&d8, &c8, rows, row_seq, row_pos, q_idx, w, cscores, L.ld_c, ws, inner, L.inner_bytes, s);
+  if (st != LSA_OK) return st;
+  // 2. the short list: the n_cand best by compact score (positions past a
+  // row's visible range are -inf and never taken)
+  const bool by_seq = row_seq == nullptr && row_pos == nullptr;
+  st = do_topk(cscores, L.ld_c, rows, by_seq ? c->seq_lens : nullptr, c->max_len, n_cand, cand, ws, inner, s);
+  if (st != LSA_OK) return st;
+  // 3. the candidates' exact scores from the original keys
+  ScoresArgs xa = scores_args(d, c, rows, row_seq, row_pos, q_idx, w, exact, L.ld_x, ws, nullptr, 0);
+  xa.cand = cand;
+  xa.cand_ld = n_cand;
+  if (!candidate_scores_tc_supported(xa)) return LSA_ERR_UNSUPPORTED;
+  st = cuda_status(launch_candidate_scores_tc(xa, s));
+  if (st != LSA_OK) return st;
+  // 4. the k best candidates, ties to the lower entry (= the lower position)
+  st = do_topk(exact, L.ld_x, rows, nullptr, n_cand, d->top_k, slot, ws, inner, s);
+  if (st != LSA_OK) return st;
+  return cuda_status(launch_cand_positions(slot, cand, rows, d->top_k, n_cand, idx, s));
 }
 
 lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream) {

@@ -18,19 +18,19 @@ namespace {
 
 using namespace scan;
 
-template <int KDT, int QB>
+template <int KDT, int QB, bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmap,
                                                          const __grid_constant__ CUtensorMap smap, const ScoresArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   if ((threadIdx.x >> 5) == kWarpMma) {
-    tc::tmem_alloc(&tmem_slot, Cfg<KDT, QB>::kTmemCols);
+    tc::tmem_alloc(&tmem_slot, Cfg<KDT, QB, GATHER>::kTmemCols);
     tc::tc_fence_before();
   }
-  scan_cta<KDT, QB>(&tmap, &smap, a, smem_raw, &tmem_slot);
+  scan_cta<KDT, QB, GATHER>(&tmap, &smap, a, smem_raw, &tmem_slot);
   if ((threadIdx.x >> 5) == kWarpMma) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem_slot, Cfg<KDT, QB>::kTmemCols);
+    tc::tmem_dealloc(tmem_slot, Cfg<KDT, QB, GATHER>::kTmemCols);
   }
 }
 
@@ -134,6 +134,27 @@ bool scores_tc_fused_hist_ok(const ScoresArgs& a) { return a.row_pos == nullptr 
 cudaError_t scan_tc_maps(const ScoresArgs& a, CUtensorMap* tmap, CUtensorMap* smap) { return make_maps(a, tmap, smap); }
 
 int scan_tc_grid() { return num_sms(); }
+
+bool candidate_scores_tc_supported(const ScoresArgs& a) {
+  if (!a.cand || a.cand_ld < 0) return false;
+  if (a.key_dtype != LSA_BF16 || a.q_dtype != LSA_BF16 || a.H != kHeads || a.dI != kDim) return false;
+  if (!aligned16(a.cache.idx_keys) || !aligned16(a.q_idx) || !aligned16(a.w)) return false;
+  const int64_t kr = key_rows(a);
+  return kr > 0 && kr < (1LL << 31);
+}
+
+// Candidate re-scoring: the scan's CTA body with the gathering producer (no
+// tensor maps: the rows are copied by cp.async).
+cudaError_t launch_candidate_scores_tc(const ScoresArgs& a, cudaStream_t s) {
+  using C = Cfg<LSA_BF16, 1, true>;
+  auto kern = k_scan_tc<LSA_BF16, 1, true>;
+  cudaError_t e = ensure_dyn_smem(kern, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  CUtensorMap none;
+  memset(&none, 0, sizeof(none));
+  kern<<<num_sms(), kThreads, C::kSmemBytes, s>>>(none, none, a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_scores_tc(const ScoresArgs& a, cudaStream_t s) {
   const bool causal = a.row_pos != nullptr;

@@ -46,6 +46,13 @@ struct ScoresArgs {
                        // zeroed by the caller), accumulated by the scan for the top-k
   uint32_t* done_ctr = nullptr;  // if set (zeroed by the caller): every CTA adds 1 once its
                                  // scores and histogram counts are written and fenced
+  // Candidate re-scoring (the second stage of the two-stage search): if set,
+  // row r scores only the positions cand[r * cand_ld + j], j < cand_ld
+  // (ascending, -1 = no candidate), and scores[r][j] is the score of entry j
+  // (-inf for -1; NaN and LSA_ERR_BOUNDS for a position outside the row's
+  // visible range or a bad block).  bf16 keys only.
+  const int32_t* cand = nullptr;
+  int32_t cand_ld = 0;
 };
 
 // ---- indexer
@@ -56,6 +63,13 @@ int scores_tc_launches(bool causal);
 bool scores_tc_supported(const ScoresArgs& a);
 size_t scores_tc_ws_bytes(int32_t rows, bool causal);
 cudaError_t launch_scores_tc(const ScoresArgs& a, cudaStream_t s);
+// Candidate re-scoring on the tensor cores (a.cand set): shape and alignment
+// test, and the launch.
+bool candidate_scores_tc_supported(const ScoresArgs& a);
+cudaError_t launch_candidate_scores_tc(const ScoresArgs& a, cudaStream_t s);
+// idx[r][j] = cand[r][slot[r][j]] (-1 for slot -1): candidate entries -> positions.
+cudaError_t launch_cand_positions(const int32_t* slot, const int32_t* cand, int32_t rows, int32_t k, int32_t n_cand,
+                                  int32_t* idx, cudaStream_t s);
 
 // ---- top-k
 struct TopkPlan {

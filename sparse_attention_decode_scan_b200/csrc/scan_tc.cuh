@@ -52,7 +52,7 @@ __device__ __forceinline__ void scan_sync() {
   asm volatile("bar.sync %0, %1;" ::"n"(kBarrierId), "n"(kThreads) : "memory");
 }
 
-template <int KDT, int QB>
+template <int KDT, int QB, bool GATHER = false>
 struct Cfg {
   static constexpr bool kFp8 = KDT == LSA_FP8_E4M3;
   static constexpr int kN = (kFp8 ? 2 * kHeads : kHeads) * QB;    // MMA N (columns per accumulator)
@@ -67,7 +67,9 @@ struct Cfg {
   static constexpr int kHistBytes = QB == 1 ? kTopkBins1 * 4 : 0;  // fused first top-k histogram (decode)
   // Per stage besides the keys: the key rows of its two boxes (written by the
   // producer for the epilogue) and, for FP8, the two boxes' scales (TMA).
-  static constexpr int kMetaBytes = 2 * 4 + (kFp8 ? 2 * kScaleSlot * 4 : 0);
+  // Gathered candidates: the stage's masks of rows with a key (4 words) and of
+  // rows whose position or block was out of range (4 words).
+  static constexpr int kMetaBytes = 2 * 4 + (kFp8 ? 2 * kScaleSlot * 4 : 0) + (GATHER ? 8 * 4 : 0);
   static constexpr int kRawBytes = kFp8 ? QB * kHeads * kDim * 2 : 0;  // FP8: bf16 query rows before the split
   static constexpr int kFixed = kNQ * kQBytes + kNQ * kWBytes + kRawBytes + kHistBytes + 512 /*barriers, scratch*/ +
                                 1024 /*align*/;
@@ -82,6 +84,7 @@ struct Cfg {
   static_assert(kNS >= 3, "too few key stages");
   static_assert(2 * kN <= 512, "accumulators exceed TMEM");
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
+  static_assert(!GATHER || (KDT == LSA_BF16 && QB == 1), "candidate gather: bf16 keys, one row per tile");
 };
 
 // Stages of the configurations that run: decode 6 (bf16) and 9 (FP8) tiles in
@@ -97,6 +100,22 @@ __device__ __forceinline__ int seq_of(const ScoresArgs& a, int r) { return a.row
 __device__ __forceinline__ int64_t row_visible(const ScoresArgs& a, int r, int* b_out) {
   const int b = seq_of(a, r);
   *b_out = b;
+  if (b < 0 || b >= a.cache.batch) return 0;
+  int64_t L = __ldg(a.cache.seq_lens + b);
+  L = L < 0 ? 0 : (L > a.cache.max_len ? a.cache.max_len : L);
+  if (a.row_pos) {
+    int64_t p = static_cast<int64_t>(__ldg(a.row_pos + r)) + 1;
+    p = p < 0 ? 0 : p;
+    L = p < L ? p : L;
+  }
+  // candidate re-scoring: the row's "positions" are its candidate entries
+  if (a.cand) L = L < a.cand_ld ? L : a.cand_ld;
+  return L;
+}
+
+// Positions of query row r a candidate may name: [0, cap) (the row's visible
+// range, before the candidate list shortens it).
+__device__ __forceinline__ int64_t row_cap(const ScoresArgs& a, int r, int b) {
   if (b < 0 || b >= a.cache.batch) return 0;
   int64_t L = __ldg(a.cache.seq_lens + b);
   L = L < 0 ? 0 : (L > a.cache.max_len ? a.cache.max_len : L);
@@ -365,6 +384,145 @@ __device__ void stage_query_fp8(const ScoresArgs& a, const Group& g, uint8_t* qb
   }
 }
 
+// ---------------------------------------------------------------- candidate gather
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
+}
+
+// Producer warp of the candidate re-scoring: each tile's 128 key rows (the
+// row's candidate entries j*128 .. j*128+127) are copied with cp.async into
+// the stage in the image the TMA boxes give (two 128-byte K blocks, 128-byte
+// swizzle); rows without a key are zero-filled.  Each half-warp copies one
+// 256-byte row per instruction (coalesced).  The rows of kBatch tiles are
+// resolved ahead (candidate entry, then block table) with all of their loads
+// in flight, so those latencies are paid once per batch.  A stage is full once
+// every lane's copies have landed (one cp.async arrival per lane) and lane 0
+// has published the stage's masks: rows with a key, and rows whose position
+// or block was out of range (their scores become NaN; the first is reported).
+template <class C>
+__device__ void gather_producer(const ScoresArgs& a, const Plan& plan, const CacheAddr& ad, uint8_t* stages,
+                                uint32_t* smask, uint64_t* full, uint64_t* empty, volatile int* abort_flag,
+                                int lane) {
+  if (plan.n_items <= 0) return;
+  constexpr int kBatch = 4;
+  constexpr int kRowBytes = kDim * 2;
+  const uint8_t* keys = static_cast<const uint8_t*>(a.cache.idx_keys);
+  Walker<1> W;
+  W.start(a, plan.r_first, plan.j_first);
+  int64_t it = 0;
+  bool failed = false;
+  while (it < plan.n_items && !failed) {
+    const int nb = plan.n_items - it < kBatch ? static_cast<int>(plan.n_items - it) : kBatch;
+    int32_t pos[kBatch][4];
+    int rb[kBatch], rr[kBatch];
+    int64_t cap[kBatch];
+    {
+      Walker<1> Wu = W;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        rb[u] = -1;
+        rr[u] = 0;
+        cap[u] = 0;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) pos[u][m] = -1;
+        if (u < nb) {
+          rr[u] = Wu.g.r0;
+          rb[u] = Wu.g.b;
+          cap[u] = row_cap(a, Wu.g.r0, Wu.g.b);
+          const int32_t* cl = a.cand + static_cast<int64_t>(Wu.g.r0) * a.cand_ld;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int64_t slot = static_cast<int64_t>(Wu.j) * kTile + lane + 32 * m;
+            if (slot < Wu.g.vis) pos[u][m] = __ldg(cl + slot);
+          }
+          Wu.next(a);
+        }
+      }
+      W = Wu;
+    }
+    // key rows: >= 0 a row, -3 no candidate (padding), -1 out of range
+    int32_t row[kBatch][4];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int32_t p = pos[u][m];
+        int32_t rw = -3;
+        if (p >= 0) {
+          rw = -1;
+          if (p < cap[u]) {
+            if (ad.block_size == 0) {
+              rw = static_cast<int32_t>(static_cast<int64_t>(rb[u]) * ad.max_len + p);
+            } else {
+              const int64_t lb = p / ad.block_size;
+              if (lb < ad.max_blocks) {
+                const int32_t blk = __ldg(ad.block_table + static_cast<int64_t>(rb[u]) * ad.max_blocks + lb);
+                if (blk >= 0 && blk < ad.n_blocks)
+                  rw = static_cast<int32_t>(static_cast<int64_t>(blk) * ad.block_size + (p - lb * ad.block_size));
+              }
+            }
+          }
+          if (rw == -1) record_error(a.status, LSA_ERR_BOUNDS, rr[u], p);
+        }
+        row[u][m] = rw;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (u >= nb) break;
+      const int s = static_cast<int>(it % C::kNS);
+      const uint32_t ph = static_cast<uint32_t>((it / C::kNS) & 1);
+      // lane 0 waits for the stage; the verdict is broadcast so the warp stays converged
+      bool ok = true;
+      if (lane == 0) ok = tc::mbar_wait(&empty[s], ph ^ 1, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) {
+          record_error(a.status, LSA_ERR_TIMEOUT, 0, 9);
+          *abort_flag = 1;
+        }
+        failed = true;
+        break;
+      }
+      __syncwarp();
+      uint32_t have[4], bad[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        have[m] = __ballot_sync(0xffffffffu, row[u][m] >= 0);
+        bad[m] = __ballot_sync(0xffffffffu, row[u][m] == -1);
+      }
+      uint8_t* st = stages + s * C::kTileBytes;
+      const int c = lane & 15;  // 16-byte chunk of the row (K block c >> 3)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+#pragma unroll 4
+        for (int i2 = 0; i2 < 16; ++i2) {
+          const int src = 2 * i2 + (lane >> 4);
+          const int32_t rv = __shfl_sync(0xffffffffu, row[u][m], src);
+          const uint32_t ri = static_cast<uint32_t>(32 * m + src);
+          const uint8_t* g = keys + static_cast<int64_t>(rv >= 0 ? rv : 0) * kRowBytes + c * 16;
+          tc::cp_async16_zfill(st + (c >> 3) * C::kKBlockBytes + tc::sw128_offset(ri, static_cast<uint32_t>(c & 7)), g,
+                               rv >= 0 ? 16u : 0u);
+        }
+      }
+      cp_async_arrive_noinc(&full[s]);
+      if (lane == 0) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          smask[8 * s + m] = have[m];
+          smask[8 * s + 4 + m] = bad[m];
+        }
+        tc::mbar_arrive(&full[s]);  // release: the masks are visible to the epilogue's acquire
+      }
+      ++it;
+    }
+    failed = __shfl_sync(0xffffffffu, failed || *abort_flag, 0);
+  }
+  // every copy must land before the CTA's shared memory is released
+  tc::cp_async_wait_all();
+}
+
 // ---------------------------------------------------------------- the kernel
 
 // One CTA's share of the scan, run by threads [0, kThreads) of the block
@@ -372,10 +530,10 @@ __device__ void stage_query_fp8(const ScoresArgs& a, const Group& g, uint8_t* qb
 // once the first barrier of the plan has passed, will hold) the base of at
 // least Cfg::kTmemCols allocated TMEM columns.  Every mbarrier it used is
 // invalidated before it returns, so the caller may reuse the shared memory.
-template <int KDT, int QB>
+template <int KDT, int QB, bool GATHER = false>
 __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtensorMap* smap_p, const ScoresArgs& a,
                                          uint8_t* smem_raw, const volatile uint32_t* tmem_slot) {
-  using C = Cfg<KDT, QB>;
+  using C = Cfg<KDT, QB, GATHER>;
   const CUtensorMap& tmap = *tmap_p;
   const CUtensorMap& smap = *smap_p;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -386,7 +544,8 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   uint8_t* qraw = reinterpret_cast<uint8_t*>(wbufs) + C::kNQ * C::kWBytes;          // FP8: raw query rows
   float* sscale = reinterpret_cast<float*>(qraw + C::kRawBytes);                     // FP8: [kNS][2][kScaleSlot]
   int32_t* smeta = reinterpret_cast<int32_t*>(sscale + (C::kFp8 ? C::kNS * 2 * kScaleSlot : 0));  // [kNS][2]
-  uint32_t* shist = reinterpret_cast<uint32_t*>(smeta + 2 * C::kNS);
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smeta + 2 * C::kNS);  // gather: [kNS][8]
+  uint32_t* shist = smask + (GATHER ? 8 * C::kNS : 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(shist) + C::kHistBytes);
   uint64_t* full = bars;
   uint64_t* empty = full + C::kNS;
@@ -407,10 +566,11 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   tc::griddep_launch_dependents();
   // The epilogue reads a stage's key rows (paged cache) and scales (FP8); a
   // contiguous bf16 cache needs neither, and its stages free at MMA completion.
-  const bool stage_meta = C::kFp8 || a.cache.block_size > 0;
+  const bool stage_meta = C::kFp8 || a.cache.block_size > 0 || GATHER;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kNS; ++s) {
-      tc::mbar_init(&full[s], 1);
+      // gather: one cp.async completion per producer lane, plus lane 0's masks
+      tc::mbar_init(&full[s], GATHER ? 32 + 1 : 1);
       tc::mbar_init(&empty[s], stage_meta ? 1 + 4 : 1);  // MMA commit (+ 4 epilogue warps done with the stage)
     }
     for (int s = 0; s < C::kNQ; ++s) {
@@ -426,7 +586,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == kWarpProd && lane == 0) {
+  if (!GATHER && warp == kWarpProd && lane == 0) {
     tc::prefetch_tmap(&tmap);
     if (C::kFp8) tc::prefetch_tmap(&smap);
   }
@@ -436,7 +596,9 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   const uint32_t tmem_base = *tmem_slot;
   CacheAddr ad{a.cache.block_table, a.cache.max_blocks, a.cache.block_size, a.cache.n_blocks, a.cache.max_len};
 
-  if (warp == kWarpProd) {
+  if (GATHER && warp == kWarpProd) {
+    gather_producer<C>(a, plan, ad, stages, smask, full, empty, abort_flag, lane);
+  } else if (warp == kWarpProd) {
     // The whole warp looks up the block-table entries of 32 tiles at a time
     // (one tile per lane) and lane 0 issues their TMA loads.  The next batch's
     // entries are loaded before the current batch is issued and only read
@@ -569,6 +731,8 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
         {
           const int s = static_cast<int>(it % C::kNS);
           if (!tc::mbar_wait(&full[s], static_cast<uint32_t>((it / C::kNS) & 1), abort_flag)) goto mma_fail;
+          // gathered rows were written by cp.async (generic proxy); the MMA reads them through the async proxy
+          if (GATHER) tc::fence_proxy_async_smem();
           const int acc = static_cast<int>(it & 1);
           if (!tc::mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag)) goto mma_fail;
           tc::tc_fence_after();
@@ -753,14 +917,20 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
             hist_row = -1;
             break;
           }
-          const int box = 2 * stg + (t >> 6);
-          mrow = smeta[box];
-          if (C::kFp8 && mrow >= 0) kscale = sscale[box * kScaleSlot + (mrow & 3) + (t & 63)];
+          if (GATHER) {
+            // row t has a key (0), is a padding entry (-3: -inf) or an out-of-range one (-1: NaN)
+            const uint32_t* mk = smask + 8 * stg;
+            mrow = ((mk[t >> 5] >> (t & 31)) & 1u) ? 0 : (((mk[4 + (t >> 5)] >> (t & 31)) & 1u) ? -1 : -3);
+          } else {
+            const int box = 2 * stg + (t >> 6);
+            mrow = smeta[box];
+            if (C::kFp8 && mrow >= 0) kscale = sscale[box * kScaleSlot + (mrow & 3) + (t & 63)];
+          }
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&empty[stg]);
         }
         const int64_t p = static_cast<int64_t>(W.j) * kTile + t;
-        const int64_t prow = mrow >= 0 ? static_cast<int64_t>(mrow) + (t & 63) : -1;
+        const int64_t prow = mrow >= 0 ? static_cast<int64_t>(mrow) + (t & 63) : (GATHER && mrow == -3 ? -3 : -1);
         const float* wb = wbufs + qi * (C::kWBytes / 4);
         float sc[QB];
 #pragma unroll
@@ -796,7 +966,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
         for (int qq = 0; qq < QB; ++qq) {
           if (qq < W.g.nrows && p < a.ld) {
             float o = -INFINITY;
-            if (p < vis_r[qq]) o = prow >= 0 ? sc[qq] : NAN;
+            if (p < vis_r[qq]) o = prow >= 0 ? sc[qq] : (prow == -3 ? -INFINITY : NAN);
             a.scores[static_cast<int64_t>(W.g.r0 + qq) * a.ld + p] = o;
           }
         }

@@ -95,8 +95,13 @@ def lib() -> ctypes.CDLL:
     L.lsa_version.restype = i32
     L.lsa_launch_count.argtypes = [D, i32, i64, i32, i32]
     L.lsa_launch_count.restype = i32
+    L.lsa_candidate_scores.argtypes = [D, C, i32, vp, vp, vp, vp, vp, i32, vp, i64, vp, sz, vp]
+    L.lsa_two_stage_workspace_size.argtypes = [D, i32, i64, i32]
+    L.lsa_two_stage_workspace_size.restype = sz
+    L.lsa_two_stage_select.argtypes = [D, C, vp, vp, i32, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     names = ["lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode", "lsa_decode_step",
-             "lsa_decode_step_profiled", "lsa_decode_layers", "lsa_read_device_status"]
+             "lsa_decode_step_profiled", "lsa_decode_layers", "lsa_read_device_status", "lsa_candidate_scores",
+             "lsa_two_stage_select"]
     if path == TEST_LIB_PATH:
         L.lsa_test_set_hooks.argtypes = [i32, i64, ctypes.c_uint32]
         names.append("lsa_test_set_hooks")
@@ -216,6 +221,33 @@ def decode_layers(dims: Dims, caches, q_idx, w, q, out, lse, ws, retention: int 
                                           ptrs(lse), int(retention), int(route), _ptr(idx_out), _ptr(ws),
                                           ws.numel() if ws is not None else 0, _stream(stream)),
                   "lsa_decode_layers", raise_on_error)
+
+
+def candidate_scores(dims: Dims, cache: Cache, q_idx, w, cand, scores, ld: int, ws, row_seq=None, row_pos=None,
+                     rows: Optional[int] = None, stream=None, raise_on_error=True) -> int:
+    """lsa_candidate_scores: exact scores of the positions cand [rows, n_cand] into scores [rows, ld]."""
+    rows = int(q_idx.shape[0]) if rows is None else rows
+    n_cand = int(cand.shape[1])
+    return _check(lib().lsa_candidate_scores(ctypes.byref(dims), ctypes.byref(cache), rows, _ptr(row_seq),
+                                             _ptr(row_pos), _ptr(q_idx), _ptr(w), _ptr(cand), n_cand, _ptr(scores),
+                                             int(ld), _ptr(ws), ws.numel() if ws is not None else 0,
+                                             _stream(stream)), "lsa_candidate_scores", raise_on_error)
+
+
+def two_stage_workspace_size(dims: Dims, rows: int, max_len: int, n_cand: int) -> int:
+    return int(lib().lsa_two_stage_workspace_size(ctypes.byref(dims), rows, max_len, n_cand))
+
+
+def two_stage_select(dims: Dims, cache: Cache, compact_keys, compact_scales, q_idx, w, n_cand: int, idx, ws,
+                     row_seq=None, row_pos=None, rows: Optional[int] = None, stream=None,
+                     raise_on_error=True) -> int:
+    """lsa_two_stage_select: the k = dims.top_k selection of each row by the two-stage search."""
+    rows = int(q_idx.shape[0]) if rows is None else rows
+    return _check(lib().lsa_two_stage_select(ctypes.byref(dims), ctypes.byref(cache), _ptr(compact_keys),
+                                             _ptr(compact_scales), rows, _ptr(row_seq), _ptr(row_pos), _ptr(q_idx),
+                                             _ptr(w), int(n_cand), _ptr(idx), _ptr(ws),
+                                             ws.numel() if ws is not None else 0, _stream(stream)),
+                  "lsa_two_stage_select", raise_on_error)
 
 
 def read_device_status(ws, stream=None) -> int:
