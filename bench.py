@@ -640,6 +640,105 @@ def run_layers(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_two_stage(args, world, rank, local):
+    """Decode steps whose selection comes from the two-stage search
+    (lsa_two_stage_select: FP8 scan of compact keys, top-n_cand, exact re-score
+    of the list with the original keys, top-k) followed by the sparse
+    attention.  Reports the selection's bytes and time next to the attention."""
+    import torch
+
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = synth.workload(args.workload)
+    spec = synth.scaled(base, batch=args.batch) if args.batch else base
+    assert not spec.causal and spec.idx_key_dtype == "bf16", "two-stage: bf16 decode workloads"
+    case = synth.make_case(spec, rank_seed(base, rank))
+    dc = DeviceCase(case, device=dev)
+    bits, scales = synth.compact_keys(case.idx_keys)
+    d_bits = torch.from_numpy(np.ascontiguousarray(bits)).to(dev)
+    d_scales = torch.from_numpy(scales).to(dev)
+    s = case.spec
+    B, k, n_cand = dc.rows, s.top_k, args.two_stage
+    idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+    out = torch.empty((B, s.n_heads, s.v_dim), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, s.n_heads), dtype=torch.float32, device=dev)
+    ws = lsa.workspace(max(lsa.two_stage_workspace_size(dc.dims, B, dc.max_len, n_cand),
+                           lsa.workspace_size(dc.dims, B, dc.max_len, lsa.LSA_OP_ATTN)), device=dev)
+    stream = torch.cuda.current_stream(dev)
+    qsets = [(dc.q_idx, dc.w, dc.q)]
+    for j in range(1, QUERY_SETS):
+        qi, wj, qj = synth.queries(s, rank_seed(base, rank) + 104729 * j, B)
+        qsets.append((to_dev(qi, s.act_dtype, dev), torch.from_numpy(wj).to(dev), to_dev(qj, s.act_dtype, dev)))
+
+    def step(i, ev=None):
+        qi, wj, qj = qsets[i % len(qsets)]
+        if ev is not None:
+            ev[0].record(stream)
+        lsa.two_stage_select(dc.dims, dc.cache, d_bits, d_scales, qi, wj, n_cand, idx, ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        lsa.sparse_attn_decode(dc.dims, dc.cache, qj, idx, out, lse, ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    with ClockSampler(gpu_index) as clk:
+        t_soak = time.perf_counter()
+        while not args.no_soak and time.perf_counter() - t_soak < 1.0:
+            step(0)
+            torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(args.steps):
+            step(i)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        for i in range(args.steps):
+            step(i, evs[i])
+        torch.cuda.synchronize(dev)
+    timed_ms = reduce_max(a.elapsed_time(b_))
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    peaks, peak_src = load_peaks()
+    nb = synth.nbytes_decode_step(case)
+    L = case.seq_lens.astype(np.int64)
+    cand_rows = np.minimum(L, n_cand)
+    sel_bytes = int(L.sum() * (s.idx_dim + 4) + cand_rows.sum() * s.idx_dim * 2 + nb["block_table"] +
+                    nb["q_idx_w"])
+    one_stage = int(nb["keys"] + nb["block_table"] + nb["q_idx_w"])
+    ms_per_step = timed_ms / args.steps
+    line = {"metric": f"decode steps/s with the two-stage selection (list of {n_cand}) + sparse attn",
+            "value": world * args.steps / (timed_ms / 1e3), "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16+fp8", "data": "synthetic (seeded)",
+            "config": dict(workload_config(case), n_cand=n_cand),
+            "kernel_ms": {"two_stage_select": sel_ms, "attn": attn_ms},
+            "selection_algorithmic_bytes": sel_bytes, "one_stage_scan_bytes": one_stage,
+            "selection_bytes_ratio": sel_bytes / one_stage,
+            "selection_hbm_frac": sel_bytes / (sel_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "peak_source": peak_src, "gpu_launches": args.steps * 8, "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def to_dev(arr, dtype, dev):
+    from sparse_attention_decode_scan_b200.device import to_device
+    return to_device(arr, dtype, dev)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -659,6 +758,8 @@ def main(argv=None):
     ap.add_argument("--route", default="own", choices=["own", "prev"],
                     help="layers: attend the latest indexer layer at or before (own) or before (prev, MLI) a layer")
     ap.add_argument("--retention", type=int, default=1, help="layers: every retention-th layer keeps an indexer")
+    ap.add_argument("--two-stage", type=int, default=0, metavar="N_CAND",
+                    help="decode steps whose selection is the two-stage search with a list of N_CAND")
     ap.add_argument("--fused", action="store_true",
                     help="decode step as one cooperative launch (LSA_STEP_FUSED) instead of separate launches")
     args = ap.parse_args(argv)
@@ -678,7 +779,9 @@ def main(argv=None):
         if args.impl == "reference":
             run_reference(args, world, rank)
         else:
-            if args.layers > 1:
+            if args.two_stage:
+                run_two_stage(args, world, rank, local)
+            elif args.layers > 1:
                 run_layers(args, world, rank, local)
             else:
                 run_ours(args, world, rank, local)

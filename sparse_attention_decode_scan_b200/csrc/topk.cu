@@ -27,6 +27,7 @@
 #include "host_util.h"
 #include "internal.h"
 #include "tc.cuh"
+#include "topk_cluster.cuh"
 #include "topk_sel.cuh"
 
 namespace lsa {
@@ -403,6 +404,42 @@ __global__ void __launch_bounds__(tk::kCollectThreads, 2) k_tk_rows(TopkArgs a, 
   }
 }
 
+// One row per thread-block cluster (rows up to tk::kClMaxCols positions): CTA
+// blockIdx.x of the cluster collects segment blockIdx.x of row blockIdx.y and
+// the cluster selects the row together (topk_cluster.cuh).
+__global__ void __launch_bounds__(tk::kClThreads, 2) k_tk_cluster(TopkArgs a, int64_t seg_len, int nseg) {
+  extern __shared__ __align__(16) uint8_t csm[];
+  __shared__ tk::TkScratch S;
+  __shared__ int s_live;
+  const int r = blockIdx.y;
+  if (a.wait_ctr) {
+    // decode step, launched early: wait until every scan CTA has counted
+    // itself (its scores and histogram counts written and fenced)
+    if (threadIdx.x == 0) {
+      s_live = 1;
+      const uint64_t t0 = tc::globaltimer_ns();
+      for (;;) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.wait_ctr) : "memory");
+        if (v >= a.wait_target) break;
+        if (tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) {
+          record_error(a.status, LSA_ERR_TIMEOUT, r, 20);
+          s_live = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+  } else {
+    tc::griddep_wait();  // launched early in a decode step: the scores are complete from here on
+    if (threadIdx.x == 0) s_live = 1;
+  }
+  __syncthreads();
+  tc::griddep_launch_dependents();
+  // every CTA of the cluster reaches the cluster barriers, live or not
+  tk::tk_cluster_row<2>(a, r, static_cast<int>(tc::cluster_ctarank()), nseg, seg_len, csm, S, s_live != 0);
+}
+
 // SMs of the current device (the plan's CTA target).
 int device_sms() {
   int dev = 0, n = 0;
@@ -443,6 +480,8 @@ TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
 }
 
 bool topk_v2_ok(int64_t n_cols) { return n_cols <= tk::kMaxBitmapCols; }
+
+bool topk_cluster_ok(int64_t n_cols) { return n_cols <= tk::kClMaxCols; }
 
 size_t topk_hist_zero_bytes(int32_t rows) { return tk::tk_zero_bytes(rows); }
 
@@ -525,6 +564,29 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
       e = cudaMemsetAsync(a.ws, 0, topk_hist_zero_bytes(a.rows), s);
       if (e != cudaSuccess) return e;
       k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
+    }
+    if (topk_cluster_ok(a.n_cols) && !a.split_select) {
+      // one cluster of up to 8 CTAs per row
+      const tk::ClPlan cp = tk::cl_plan(a.n_cols);
+      const size_t smem = tk::cl_smem(cp.seg_len);
+      e = ensure_dyn_smem(k_tk_cluster, smem);
+      if (e != cudaSuccess) return e;
+      cudaLaunchConfig_t cfg;
+      memset(&cfg, 0, sizeof(cfg));
+      cfg.gridDim = dim3(static_cast<unsigned>(cp.nseg), static_cast<unsigned>(a.rows));
+      cfg.blockDim = dim3(tk::kClThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = static_cast<unsigned>(cp.nseg);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = a.pdl ? 2 : 1;
+      return cudaLaunchKernelEx(&cfg, k_tk_cluster, a, cp.seg_len, cp.nseg);
     }
     size_t smem;
     TopkPlan cp;

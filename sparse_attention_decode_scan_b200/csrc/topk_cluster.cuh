@@ -1,0 +1,303 @@
+#pragma once
+// Top-k of one row by one thread-block cluster (rows of up to kClMaxCols
+// positions): the same exact selection as the collect + select bodies of
+// topk_sel.cuh (the k best-scored tokens, MLI abstract, sentence 2; ties to
+// the lower position, -inf and NaN never taken, positions ascending, then -1),
+// with the row's work spread over the cluster's CTAs instead of ending in one.
+//
+// CTA s of the cluster owns segment s of the row.  It reads the row's
+// first-digit histogram (key bits [31:20]) and finds the threshold bin b1,
+// then collects its segment: keys above b1 become a bitmap in its own shared
+// memory, keys inside b1 a local candidate list.  After a cluster barrier
+// every CTA runs the radix select of the threshold key T on bits [19:0] over
+// all CTAs' candidates, read through distributed shared memory (the lists are
+// short: a bin holds a few hundred keys at these sizes), marks its own
+// candidates above T into its bitmap and those equal to T into a tie bitmap,
+// and publishes two counts.  After a second barrier each CTA knows the
+// selection entries before its segment and the ties left to it (the lowest
+// positions equal to T are taken first), and compacts its own segment into
+// the output.  If any CTA's candidates overflow its list, T is found from the
+// whole row and each segment is re-read to mark.
+#include "topk_sel.cuh"
+
+namespace lsa {
+namespace tk {
+
+constexpr int kClThreads = kCollectThreads;        // the round shape of tk_round_load
+constexpr int kClMaxSeg = 8;                       // CTAs per cluster (portable cluster size)
+constexpr int64_t kClMaxCols = int64_t(1) << 18;   // longer rows take the collect + select bodies
+constexpr int kClCandCap = 2048;                   // threshold-bin keys a CTA keeps
+
+struct ClHdr {
+  uint32_t nc;  // keys of the threshold bin in the segment (> kClCandCap: the list overflowed)
+  uint32_t gt;  // selected keys above T in the segment
+  uint32_t eq;  // keys equal to T in the segment
+  uint32_t pad;
+};
+
+struct ClPlan {
+  int nseg;
+  int64_t seg_len;  // multiple of kColRound
+};
+
+__host__ __device__ inline ClPlan cl_plan(int64_t n_cols) {
+  ClPlan p;
+  int64_t rounds = (n_cols + kColRound - 1) / kColRound;
+  if (rounds < 1) rounds = 1;
+  const int64_t ns = rounds < kClMaxSeg ? rounds : kClMaxSeg;
+  const int64_t per = (rounds + ns - 1) / ns;
+  p.seg_len = per * kColRound;
+  p.nseg = static_cast<int>((rounds + per - 1) / per);
+  return p;
+}
+
+// Shared memory of the body: header | bitmap of the segment | tie bitmap |
+// candidates.  The bitmaps are padded per thread (tk_pad) so the ordered walk
+// over each thread's own words hits distinct banks.
+__host__ __device__ inline int cl_bm_words(int64_t seg_len) {
+  const TkPad p = tk_pad(seg_len, kClThreads);
+  return (kClThreads * p.stride + 3) / 4 * 4;
+}
+
+__host__ __device__ inline size_t cl_smem(int64_t seg_len) {
+  return sizeof(ClHdr) + 2 * static_cast<size_t>(cl_bm_words(seg_len)) * 4 + static_cast<size_t>(kClCandCap) * 8;
+}
+
+// Row r, segment s of ns (CTA rank s of the row's cluster).  `live` false (a
+// wait before it ran out): the CTA does no work but still takes part in the
+// cluster barriers.  ID: named barrier of the CTA's threads.
+template <int ID>
+__device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t seg_len, uint8_t* dsm, TkScratch& S,
+                               bool live) {
+  constexpr int NT = kClThreads;
+  const int t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5;
+  const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
+  const TkPad pad = tk_pad(seg_len, NT);
+  const int bm_words = cl_bm_words(seg_len);
+  ClHdr* hdr = reinterpret_cast<ClHdr*>(dsm);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(dsm + sizeof(ClHdr));
+  uint32_t* tb = bm + bm_words;
+  uint2* cs = reinterpret_cast<uint2*>(tb + bm_words);
+  const DivU32 dper = make_divu32(static_cast<uint32_t>(pad.per));
+  auto pw = [&](uint32_t w) -> int {  // padded index of segment word w
+    const uint32_t q = divu32(dper, w);
+    return static_cast<int>(q * pad.stride + (w - q * pad.per));
+  };
+  int n = static_cast<int>(a.n_cols);
+  if (a.valid_len) {
+    const int64_t v = __ldg(a.valid_len + r);
+    n = v < 0 ? 0 : (v < n ? static_cast<int>(v) : n);
+  }
+  const int s0 = s * static_cast<int>(seg_len);
+  const int s1 = s0 + static_cast<int>(seg_len) < static_cast<int>(a.n_cols) ? s0 + static_cast<int>(seg_len)
+                                                                              : static_cast<int>(a.n_cols);
+  const int nw_seg = s1 > s0 ? (s1 - s0 + 31) / 32 : 0;
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  const int lim = ((n + 3) & ~3) < a.ld ? ((n + 3) & ~3) : static_cast<int>(a.ld);
+  for (int i = t; i < bm_words; i += NT) tb[i] = 0;
+  // ---------------------------------------------------------------- collect
+  uint32_t keff = 0, b1 = 0xffffffffu, rank1 = 0;
+  int nc = 0, above = 0;
+  if (live) {
+    ColRound cur;
+    if (s0 < s1) tk_round_load(row, s0, lim, cur);
+    uint32_t hv[kB1 / NT];
+    tk_load_bins<NT, kB1>(L.hist + static_cast<int64_t>(r) * kB1, t, hv);
+    const uint32_t total = tk_find<NT, ID, kB1>(hv, static_cast<uint32_t>(a.k), S, true);
+    keff = total < static_cast<uint32_t>(a.k) ? total : static_cast<uint32_t>(a.k);
+    if (keff > 0) {
+      b1 = static_cast<uint32_t>(S.s_bin);
+      rank1 = S.s_rank;
+    }
+#pragma unroll 1
+    for (int base = s0; keff > 0 && base < s1; base += kColRound) {
+      const int p0 = base + warp * 1024 + lane * 4;
+      uint32_t key[8][4];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const int p = p0 + v * 128;
+        key[v][0] = p < n ? order_key(cur.x[v].x) : 0u;
+        key[v][1] = p + 1 < n ? order_key(cur.x[v].y) : 0u;
+        key[v][2] = p + 2 < n ? order_key(cur.x[v].z) : 0u;
+        key[v][3] = p + 3 < n ? order_key(cur.x[v].w) : 0u;
+      }
+      if (base + kColRound < s1) tk_round_load(row, base + kColRound, lim, cur);
+      // bitmap word of lane l: positions 32 l .. 32 l + 31 of the warp's 1024
+      uint32_t bal[4] = {0u, 0u, 0u, 0u};
+      int ncl = 0;
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t k = key[v][c];
+          const uint32_t bb = __ballot_sync(0xffffffffu, k != 0u && (k >> 20) > b1);
+          bal[c] = (lane >> 2) == v ? bb : bal[c];
+          ncl += (k != 0u && (k >> 20) == b1) ? 1 : 0;
+        }
+      }
+      const int sh = 8 * (lane & 3);
+      const uint32_t word = spread8(bal[0] >> sh) | (spread8(bal[1] >> sh) << 1) | (spread8(bal[2] >> sh) << 2) |
+                            (spread8(bal[3] >> sh) << 3);
+      const int wi = (base - s0) / kWordElems + warp * 32 + lane;
+      if (wi < nw_seg) bm[pw(static_cast<uint32_t>(wi))] = word;
+      above += __popc(word);
+      int tot;
+      const int off = tk_excl_scan<NT, ID>(ncl, S.warp_sums, &tot);
+      int o = nc + off;
+      if (ncl) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t k = key[v][c];
+            if (k != 0u && (k >> 20) == b1) {
+              if (o < kClCandCap) cs[o] = make_uint2(k, static_cast<uint32_t>(p0 + v * 128 + c));
+              ++o;
+            }
+          }
+        }
+      }
+      nc += tot;
+    }
+  }
+  // words of the bitmap the rounds did not write (a segment without a selectable key)
+  if (!live || keff == 0)
+    for (int i = t; i < bm_words; i += NT) bm[i] = 0;
+  if (t == 0) hdr->nc = static_cast<uint32_t>(nc);
+  tc::cluster_sync();  // ---- every segment collected
+  // ---------------------------------------------------------------- threshold key T
+  bool ovf = false;
+  const uint32_t hdr_u = tc::smem_u32(hdr), cs_u = tc::smem_u32(cs);
+#pragma unroll 1
+  for (int q = 0; q < ns; ++q)
+    ovf |= tc::ld_cluster_u32(tc::cluster_map(hdr_u, static_cast<uint32_t>(q))) > static_cast<uint32_t>(kClCandCap);
+  uint32_t T = 0, ties = 0;
+  if (live && keff > 0) {
+    if (!ovf) {
+      for (int pass = 0; pass < 2; ++pass) {
+        for (int i = t; i < 1024; i += NT) S.h[i] = 0;
+        tk_sync<NT, ID>();
+        const uint32_t shift = pass == 0 ? 10 : 0;
+        const uint32_t pre_shift = pass == 0 ? 20 : 10;
+        const uint32_t prefix = pass == 0 ? b1 : (T >> 10);
+#pragma unroll 1
+        for (int q = 0; q < ns; ++q) {
+          const uint32_t base_q = tc::cluster_map(cs_u, static_cast<uint32_t>(q));
+          const int nc_q = static_cast<int>(tc::ld_cluster_u32(tc::cluster_map(hdr_u, static_cast<uint32_t>(q))));
+          for (int c = t; c < nc_q; c += NT) {
+            const uint32_t key = tc::ld_cluster_u32(base_q + static_cast<uint32_t>(c) * 8u);
+            if ((key >> pre_shift) == prefix) atomicAdd(&S.h[(key >> shift) & 1023u], 1u);
+          }
+        }
+        tk_sync<NT, ID>();
+        uint32_t hl[1024 / NT];
+#pragma unroll
+        for (int i = 0; i < 1024 / NT; ++i) hl[i] = S.h[t * (1024 / NT) + i];
+        tk_find<NT, ID, 1024>(hl, pass == 0 ? rank1 : ties, S, false);
+        const uint32_t bb = static_cast<uint32_t>(S.s_bin);
+        T = pass == 0 ? ((b1 << 20) | (bb << 10)) : (T | bb);
+        ties = S.s_rank;
+        tk_sync<NT, ID>();
+      }
+    } else {
+      tk_radix_T<NT, ID>(cs, 0, true, row, n, b1, rank1, S, &T, &ties);
+    }
+    // this segment's keys of bin b1: above T into the bitmap, equal to T into the tie bitmap
+    if (!ovf) {
+      for (int c = t; c < nc; c += NT) {
+        const uint2 e = cs[c];
+        const uint32_t w = (e.y - static_cast<uint32_t>(s0)) >> 5;
+        if (e.x > T) atomicOr(&bm[pw(w)], 1u << (e.y & 31));
+        else if (e.x == T) atomicOr(&tb[pw(w)], 1u << (e.y & 31));
+      }
+    } else {
+      for (int p = s0 + t; p < s1 && p < n; p += NT) {
+        const uint32_t key = order_key(__ldcg(row + p));
+        if ((key >> 20) != b1) continue;
+        const uint32_t w = static_cast<uint32_t>(p - s0) >> 5;
+        if (key > T) atomicOr(&bm[pw(w)], 1u << (p & 31));
+        else if (key == T) atomicOr(&tb[pw(w)], 1u << (p & 31));
+      }
+    }
+  }
+  tk_sync<NT, ID>();
+  // ---------------------------------------------------------------- counts
+  const int w0 = t * pad.per;
+  const int nmine = nw_seg - w0 < pad.per ? (nw_seg - w0 > 0 ? nw_seg - w0 : 0) : pad.per;
+  const int pb = t * pad.stride;
+  int my_gt = 0, my_eq = 0;
+  for (int i = 0; i < nmine; ++i) {
+    my_gt += __popc(bm[pb + i]);
+    my_eq += __popc(tb[pb + i]);
+  }
+  int gt_tot, eq_tot;
+  tk_excl_scan<NT, ID>(my_gt, S.warp_sums, &gt_tot);
+  int eq_before = tk_excl_scan<NT, ID>(my_eq, S.warp_sums, &eq_tot);
+  if (t == 0) {
+    hdr->gt = static_cast<uint32_t>(gt_tot);
+    hdr->eq = static_cast<uint32_t>(eq_tot);
+  }
+  tc::cluster_sync();  // ---- every segment's counts published
+  // entries before this segment and the ties left to it (lowest positions first)
+  uint32_t off = 0, ties_mine = 0, eq_seen = 0;
+#pragma unroll 1
+  for (int q = 0; q < ns; ++q) {
+    const uint32_t gt_q = tc::ld_cluster_u32(tc::cluster_map(hdr_u + 4u, static_cast<uint32_t>(q)));
+    const uint32_t eq_q = tc::ld_cluster_u32(tc::cluster_map(hdr_u + 8u, static_cast<uint32_t>(q)));
+    const uint32_t left = ties > eq_seen ? ties - eq_seen : 0u;
+    const uint32_t take = left < eq_q ? left : eq_q;
+    if (q < s) off += gt_q + take;
+    if (q == s) ties_mine = take;
+    eq_seen += eq_q;
+  }
+  // no CTA reads another's shared memory past this point: the arrival lets
+  // the others leave once they are done; this CTA waits before it leaves
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  // ---------------------------------------------------------------- compaction
+  int32_t* out = a.idx + static_cast<int64_t>(r) * a.k;
+  if (live) {
+    int my_sel = 0;
+    for (int i = 0; i < nmine; ++i) {
+      const uint32_t x = tb[pb + i];
+      const int px = __popc(x);
+      const int take = static_cast<int>(ties_mine) - eq_before;
+      uint32_t add = 0;
+      if (take > 0) add = take >= px ? x : low_bits(x, take);
+      eq_before += px;
+      const uint32_t merged = bm[pb + i] | add;
+      bm[pb + i] = merged;
+      my_sel += __popc(merged);
+    }
+    int sel_tot;
+    int o = static_cast<int>(off) + tk_excl_scan<NT, ID>(my_sel, S.warp_sums, &sel_tot);
+    for (int i = 0; i < nmine; ++i) {
+      uint32_t x = bm[pb + i];
+      while (x) {
+        const int b = __ffs(x) - 1;
+        x &= x - 1;
+        if (o < a.k) out[o] = s0 + (w0 + i) * 32 + b;
+        else record_error(a.status, LSA_ERR_BOUNDS, r, o);  // cannot happen if the counts agree
+        ++o;
+      }
+    }
+    for (int i = static_cast<int>(keff) + s * NT + t; i < a.k; i += ns * NT) out[i] = -1;
+    if (a.wait_ctr) {
+      // decode step: the last CTA of the row to finish raises the row's flag
+      // (the attention of row r may read its selection from then on)
+      __threadfence();
+      tk_sync<NT, ID>();
+      if (t == 0) {
+        const uint32_t done = atomicAdd(L.row_done + r, 1u);
+        if (done == static_cast<uint32_t>(ns - 1)) {
+          __threadfence();
+          asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(L.sel_done + r), "r"(1u) : "memory");
+        }
+      }
+    }
+  }
+  tc::cluster_wait();  // ---- the others have read this CTA's shared memory
+}
+
+}  // namespace tk
+}  // namespace lsa
