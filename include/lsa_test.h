@@ -32,9 +32,13 @@ extern "C" {
  *                          then the attention's run out after about a second
  *                          each and record LSA_ERR_TIMEOUT in the status word
  *                          (the failure path of the handoff, without a fault).
+ *   no_cluster_topk        != 0: rows of up to 2^18 positions take the collect
+ *                          + per-row select top-k instead of the
+ *                          one-cluster-per-row kernel (to compare the two).
  * Returns LSA_OK.
  */
-lsa_status lsa_test_set_hooks(int32_t force_simt_path, int64_t split_select_min_cols, uint32_t scan_wait_extra);
+lsa_status lsa_test_set_hooks(int32_t force_simt_path, int64_t split_select_min_cols, uint32_t scan_wait_extra,
+                              int32_t no_cluster_topk);
 
 #ifdef __cplusplus
 }

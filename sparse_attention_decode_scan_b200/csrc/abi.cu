@@ -34,15 +34,18 @@ struct TestHooks {
   bool force_simt = false;                         // every call on the CUDA-core kernels
   int64_t split_select_min_cols = kSplitSelectMinCols;
   uint32_t scan_wait_extra = 0;                    // raises the decode step's scan-CTA count
+  bool no_cluster_topk = false;                    // the collect + select top-k for every row length
 };
 TestHooks g_hooks;
 bool force_simt() { return g_hooks.force_simt; }
 int64_t split_select_min_cols() { return g_hooks.split_select_min_cols; }
 uint32_t test_scan_wait_extra() { return g_hooks.scan_wait_extra; }
+bool allow_cluster_topk() { return !g_hooks.no_cluster_topk; }
 #else
 constexpr bool force_simt() { return false; }
 constexpr int64_t split_select_min_cols() { return kSplitSelectMinCols; }
 constexpr uint32_t test_scan_wait_extra() { return 0u; }
+constexpr bool allow_cluster_topk() { return true; }
 #endif
 
 bool valid_dims(const lsa_dims* d) {
@@ -249,6 +252,7 @@ lsa_status do_topk(const float* scores, int64_t ld, int32_t rows, const int32_t*
                    bool pdl = false, const uint32_t* wait_ctr = nullptr, uint32_t wait_target = 0,
                    bool split_select = false) {
   TopkArgs a = topk_args(scores, ld, rows, valid_len, n_cols, k, idx, ws, inner_ws, hist_ready);
+  a.allow_cluster = allow_cluster_topk();
   a.pdl = pdl;
   a.wait_ctr = wait_ctr;
   a.wait_target = wait_target;
@@ -694,7 +698,9 @@ const char* lsa_status_string(lsa_status s) {
 int32_t lsa_version(void) { return LSA_VERSION; }
 
 #ifdef LSA_TEST_HOOKS
-lsa_status lsa_test_set_hooks(int32_t force_simt_path, int64_t split_select_min_cols_, uint32_t scan_wait_extra) {
+lsa_status lsa_test_set_hooks(int32_t force_simt_path, int64_t split_select_min_cols_, uint32_t scan_wait_extra,
+                              int32_t no_cluster_topk) {
+  g_hooks.no_cluster_topk = no_cluster_topk != 0;
   g_hooks.force_simt = force_simt_path != 0;
   g_hooks.split_select_min_cols = split_select_min_cols_ < 0 ? kSplitSelectMinCols : split_select_min_cols_;
   g_hooks.scan_wait_extra = scan_wait_extra;

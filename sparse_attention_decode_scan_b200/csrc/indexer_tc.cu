@@ -18,16 +18,17 @@ namespace {
 
 using namespace scan;
 
-template <int KDT, int QB, bool GATHER = false>
-__global__ void __launch_bounds__(kThreads, 1) k_scan_tc(const __grid_constant__ CUtensorMap tmap,
-                                                         const __grid_constant__ CUtensorMap smap, const ScoresArgs a) {
+template <int KDT, int QB, bool GATHER = false, int EG = 1>
+__global__ void __launch_bounds__(scan_threads<EG>(), 1) k_scan_tc(const __grid_constant__ CUtensorMap tmap,
+                                                                   const __grid_constant__ CUtensorMap smap,
+                                                                   const ScoresArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   if ((threadIdx.x >> 5) == kWarpMma) {
     tc::tmem_alloc(&tmem_slot, Cfg<KDT, QB, GATHER>::kTmemCols);
     tc::tc_fence_before();
   }
-  scan_cta<KDT, QB, GATHER>(&tmap, &smap, a, smem_raw, &tmem_slot);
+  scan_cta<KDT, QB, GATHER, EG>(&tmap, &smap, a, smem_raw, &tmem_slot);
   if ((threadIdx.x >> 5) == kWarpMma) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem_slot, Cfg<KDT, QB, GATHER>::kTmemCols);
@@ -94,16 +95,25 @@ cudaError_t make_maps(const ScoresArgs& a, CUtensorMap* tmap_out, CUtensorMap* s
   return cudaSuccess;
 }
 
+// Epilogue groups: the per-tile epilogue (TMEM loads and the ReLU-weighted
+// head sums) of the FP8 decode scan and of the prefill scans is twice (FP8:
+// hi and lo terms) or four times (4 query rows) the bf16 decode scan's, so two
+// groups of epilogue warps take alternate tiles there; the bf16 decode scan
+// streams keys at the copy rate with one.
+template <int KDT, int QB>
+constexpr int epi_groups() { return (KDT == LSA_FP8_E4M3 || QB > 1) ? 2 : 1; }
+
 template <int KDT, int QB>
 cudaError_t launch_t(const ScoresArgs& a, cudaStream_t s) {
   using C = Cfg<KDT, QB>;
+  constexpr int EG = epi_groups<KDT, QB>();
   CUtensorMap tmap, smap;
   cudaError_t me = make_maps(a, &tmap, &smap);
   if (me != cudaSuccess) return me;
-  auto kern = k_scan_tc<KDT, QB>;
+  auto kern = k_scan_tc<KDT, QB, false, EG>;
   cudaError_t e = ensure_dyn_smem(kern, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<num_sms(), kThreads, C::kSmemBytes, s>>>(tmap, smap, a);
+  kern<<<num_sms(), scan_threads<EG>(), C::kSmemBytes, s>>>(tmap, smap, a);
   return cudaGetLastError();
 }
 
@@ -147,7 +157,7 @@ bool candidate_scores_tc_supported(const ScoresArgs& a) {
 // tensor maps: the rows are copied by cp.async).
 cudaError_t launch_candidate_scores_tc(const ScoresArgs& a, cudaStream_t s) {
   using C = Cfg<LSA_BF16, 1, true>;
-  auto kern = k_scan_tc<LSA_BF16, 1, true>;
+  auto kern = k_scan_tc<LSA_BF16, 1, true, 1>;
   cudaError_t e = ensure_dyn_smem(kern, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   CUtensorMap none;

@@ -106,6 +106,9 @@ struct TopkArgs {
   // bitmap and per-segment offsets, flag selready = 1) instead of writing idx
   // (or, when the split select cannot, the full select, flag 2).
   bool split_select = false;
+  // rows up to tk::kClMaxCols take the one-cluster-per-row kernel (the test
+  // build can turn it off to compare the two paths)
+  bool allow_cluster = true;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 // The decode step's handoff words inside the top-k workspace (zeroed with its

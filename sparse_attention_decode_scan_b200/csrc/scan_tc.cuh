@@ -43,13 +43,18 @@ constexpr int kBoxRows = 64;     // rows per TMA box (one 64-token page or half 
 constexpr int kBoxX = 32;        // 4-byte TMA elements per 128-byte K block
 constexpr int kScaleBox = 68;    // FP8 scales per box load: 64 + up to 3 for the 16-byte aligned start
 constexpr int kScaleSlot = 96;   // floats per scale slot: a TMA destination starts on a 128-byte boundary
-constexpr int kThreads = 224;    // 7 warps
+constexpr int kThreads = 224;    // 7 warps (one epilogue group)
+// Threads of a scan CTA with EG epilogue groups of 4 warps (warps 3.., the
+// groups taking alternate tiles, i.e. one accumulator buffer each).
+template <int EG>
+constexpr int scan_threads() { return kThreads + (EG - 1) * 128; }
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpQ = 2, kWarpEpi = 3;
 constexpr int kSmemLimit = 232448;
 constexpr int kBarrierId = 1;    // named barrier of the scan's threads (a fused block holds more threads)
 
+template <int NTH = kThreads>
 __device__ __forceinline__ void scan_sync() {
-  asm volatile("bar.sync %0, %1;" ::"n"(kBarrierId), "n"(kThreads) : "memory");
+  asm volatile("bar.sync %0, %1;" ::"n"(kBarrierId), "n"(NTH) : "memory");
 }
 
 template <int KDT, int QB, bool GATHER = false>
@@ -184,8 +189,9 @@ struct Walker {
   }
 };
 
+template <int NTH>
 __device__ __forceinline__ int block_sum_i64_scan(int64_t v, int64_t* warp_buf, int64_t* incl, int64_t* total) {
-  // inclusive scan over the block (kThreads threads), returns nothing; used by the planner
+  // inclusive scan over the block (NTH threads), returns nothing; used by the planner
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int64_t x = v;
 #pragma unroll
@@ -194,15 +200,15 @@ __device__ __forceinline__ int block_sum_i64_scan(int64_t v, int64_t* warp_buf, 
     if (lane >= o) x += y;
   }
   if (lane == 31) warp_buf[warp] = x;
-  scan_sync();
+  scan_sync<NTH>();
   int64_t before = 0, tot = 0;
-  for (int w = 0; w < kThreads / 32; ++w) {
+  for (int w = 0; w < NTH / 32; ++w) {
     if (w < warp) before += warp_buf[w];
     tot += warp_buf[w];
   }
   *incl = before + x;
   *total = tot;
-  scan_sync();
+  scan_sync<NTH>();
   return 0;
 }
 
@@ -214,17 +220,17 @@ struct Plan {
 
 // Every thread of the CTA takes part: total tiles, this CTA's share, and the
 // group holding its first tile.
-template <int QB>
+template <int QB, int NTH = kThreads>
 __device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
   Plan p;
   p.r_first = 0;
   p.j_first = 0;
-  if (a.rows <= kThreads) {  // one row per thread: a single block scan
+  if (a.rows <= NTH) {  // one row per thread: a single block scan
     const int r = threadIdx.x;
     int64_t t = 0;
     if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
     int64_t incl, tot;
-    block_sum_i64_scan(t, sbuf, &incl, &tot);
+    block_sum_i64_scan<NTH>(t, sbuf, &incl, &tot);
     const int64_t t0 = tot * blockIdx.x / gridDim.x;
     p.n_items = tot * (blockIdx.x + 1) / gridDim.x - t0;
     if (p.n_items <= 0) return p;
@@ -233,18 +239,18 @@ __device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
       sfound[0] = r;
       sfound[1] = static_cast<int>(t0 - start);
     }
-    scan_sync();
+    scan_sync<NTH>();
     p.r_first = sfound[0];
     p.j_first = sfound[1];
     return p;
   }
   int64_t total = 0;
-  for (int base = 0; base < a.rows; base += kThreads) {
+  for (int base = 0; base < a.rows; base += NTH) {
     const int r = base + threadIdx.x;
     int64_t t = 0;
     if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
     int64_t incl, tot;
-    block_sum_i64_scan(t, sbuf, &incl, &tot);
+    block_sum_i64_scan<NTH>(t, sbuf, &incl, &tot);
     total += tot;
   }
   const int64_t t0 = total * blockIdx.x / gridDim.x;
@@ -252,21 +258,21 @@ __device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
   p.n_items = t1 - t0;
   if (p.n_items <= 0) return p;
   if (threadIdx.x == 0) sfound[0] = -1;
-  scan_sync();
+  scan_sync<NTH>();
   int64_t acc = 0;
-  for (int base = 0; base < a.rows; base += kThreads) {
+  for (int base = 0; base < a.rows; base += NTH) {
     const int r = base + threadIdx.x;
     int64_t t = 0;
     if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
     int64_t incl, tot;
-    block_sum_i64_scan(t, sbuf, &incl, &tot);
+    block_sum_i64_scan<NTH>(t, sbuf, &incl, &tot);
     const int64_t start = acc + incl - t;
     if (t > 0 && start <= t0 && t0 < start + t) {
       sfound[0] = r;
       sfound[1] = static_cast<int>(t0 - start);
     }
     acc += tot;
-    scan_sync();
+    scan_sync<NTH>();
     if (sfound[0] >= 0) break;
   }
   p.r_first = sfound[0];
@@ -530,10 +536,12 @@ __device__ void gather_producer(const ScoresArgs& a, const Plan& plan, const Cac
 // once the first barrier of the plan has passed, will hold) the base of at
 // least Cfg::kTmemCols allocated TMEM columns.  Every mbarrier it used is
 // invalidated before it returns, so the caller may reuse the shared memory.
-template <int KDT, int QB, bool GATHER = false>
+template <int KDT, int QB, bool GATHER = false, int EG = 1>
 __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtensorMap* smap_p, const ScoresArgs& a,
                                          uint8_t* smem_raw, const volatile uint32_t* tmem_slot) {
   using C = Cfg<KDT, QB, GATHER>;
+  constexpr int NTH = scan_threads<EG>();
+  static_assert(EG == 1 || EG == 2, "one or two epilogue groups");
   const CUtensorMap& tmap = *tmap_p;
   const CUtensorMap& smap = *smap_p;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -575,14 +583,14 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     }
     for (int s = 0; s < C::kNQ; ++s) {
       tc::mbar_init(&qfull[s], 1);
-      tc::mbar_init(&qempty[s], 1 + 4);  // MMA commit + 4 epilogue warps
+      tc::mbar_init(&qempty[s], 1 + 4 * EG);  // MMA commit + every epilogue warp
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&tfull[s], 1);
       tc::mbar_init(&tempty[s], 4);
     }
     tc::mbar_init(done, 1);
-    tc::mbar_init(ebar, 4);
+    tc::mbar_init(ebar, 4 * EG);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -590,8 +598,8 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     tc::prefetch_tmap(&tmap);
     if (C::kFp8) tc::prefetch_tmap(&smap);
   }
-  const Plan plan = plan_work<QB>(a, sbuf, sfound);
-  scan_sync();
+  const Plan plan = plan_work<QB, NTH>(a, sbuf, sfound);
+  scan_sync<NTH>();
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   CacheAddr ad{a.cache.block_table, a.cache.max_blocks, a.cache.block_size, a.cache.n_blocks, a.cache.max_len};
@@ -800,15 +808,17 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       }
     }
   } else {
-    // epilogue: warp (3..6) % 4 selects the TMEM lane quarter = token rows of the tile
+    // epilogue: warp % 4 selects the TMEM lane quarter = token rows of the
+    // tile; group eg (warps 3 + 4 eg ..) takes the tiles it with it % EG == eg
     const int quarter = warp & 3;
+    const int eg = (warp - kWarpEpi) / 4;
     const int t = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     // Decode with a histogram target: the epilogue also counts each score's
     // top-k digit (key bits [31:20]) in shared memory and adds the counts of a
     // row to hist12 when the CTA leaves that row, so the top-k skips one pass.
     const bool use_hist = QB == 1 && a.hist12 != nullptr;
-    const int et = threadIdx.x - kWarpEpi * 32;  // 0..127
+    const int et = threadIdx.x - kWarpEpi * 32;  // 0 .. 128 EG - 1
     int ephase = 0;
     auto epi_sync = [&]() -> bool {
       __syncwarp();
@@ -820,7 +830,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     auto flush_hist = [&](int row) -> bool {
       if (!epi_sync()) return false;
       uint32_t* dst = a.hist12 + static_cast<int64_t>(row) * kTopkBins1;
-      for (int i = et; i < kTopkBins1; i += 128) {
+      for (int i = et; i < kTopkBins1; i += 128 * EG) {
         const uint32_t v = shist[i];
         if (v) {
           atomicAdd(dst + i, v);
@@ -830,7 +840,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       return epi_sync();
     };
     if (use_hist)
-      for (int i = et; i < kTopkBins1; i += 128) shist[i] = 0;
+      for (int i = et; i < kTopkBins1; i += 128 * EG) shist[i] = 0;
     // Tails first (the epilogue warps wait for their first accumulator
     // anyway): positions past each row's group tiles are -inf, the whole row
     // NaN for an invalid row.  No tile writes there, so the order is free.
@@ -854,11 +864,11 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       const int64_t mis = (reinterpret_cast<uintptr_t>(row + start) >> 2) & 3;  // floats to 16-byte alignment
       int64_t head = start + ((4 - mis) & 3);
       head = head < a.ld ? head : a.ld;
-      for (int64_t p = start + et; p < head; p += 128) row[p] = val;
+      for (int64_t p = start + et; p < head; p += 128 * EG) row[p] = val;
       const int64_t nvec = (a.ld - head) >> 2;
       float4* v4 = reinterpret_cast<float4*>(row + head);
-      for (int64_t i = et; i < nvec; i += 128) v4[i] = make_float4(val, val, val, val);
-      for (int64_t p = head + nvec * 4 + et; p < a.ld; p += 128) row[p] = val;
+      for (int64_t i = et; i < nvec; i += 128 * EG) v4[i] = make_float4(val, val, val, val);
+      for (int64_t p = head + nvec * 4 + et; p < a.ld; p += 128 * EG) row[p] = val;
     }
     if (plan.n_items > 0) {
       Walker<QB> W;
@@ -893,81 +903,99 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
             vis_r[qq] = qq < W.g.nrows ? row_visible(a, W.g.r0 + qq, &bb) : 0;
           }
         }
-        const int acc = static_cast<int>(it & 1);
-        if (!tc::mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1), abort_flag)) {
-          if (lane == 0) {
-            record_error(a.status, LSA_ERR_TIMEOUT, 0, 5);
-            *abort_flag = 1;
-          }
-          hist_row = -1;
-          break;
-        }
-        tc::tc_fence_after();
-        // The tile's key rows (and FP8 scales) come from the producer through
-        // the stage; the stage is released once all four warps have read them.
-        int32_t mrow = 0;  // contiguous bf16: every visible position has a key row
-        float kscale = 1.f;
-        if (stage_meta) {
-          const int stg = static_cast<int>(it % C::kNS);
-          if (!tc::mbar_wait(&full[stg], static_cast<uint32_t>((it / C::kNS) & 1), abort_flag)) {
+        // the other group's tiles are only walked past (both groups release
+        // every query buffer: the weights are read by either)
+        const bool mine = EG == 1 || static_cast<int>(it % EG) == eg;
+        if (mine) {
+          const int acc = static_cast<int>(it & 1);
+          if (!tc::mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1), abort_flag)) {
             if (lane == 0) {
-              record_error(a.status, LSA_ERR_TIMEOUT, 0, 8);
+              record_error(a.status, LSA_ERR_TIMEOUT, 0, 5);
               *abort_flag = 1;
             }
             hist_row = -1;
             break;
           }
-          if (GATHER) {
-            // row t has a key (0), is a padding entry (-3: -inf) or an out-of-range one (-1: NaN)
-            const uint32_t* mk = smask + 8 * stg;
-            mrow = ((mk[t >> 5] >> (t & 31)) & 1u) ? 0 : (((mk[4 + (t >> 5)] >> (t & 31)) & 1u) ? -1 : -3);
-          } else {
-            const int box = 2 * stg + (t >> 6);
-            mrow = smeta[box];
-            if (C::kFp8 && mrow >= 0) kscale = sscale[box * kScaleSlot + (mrow & 3) + (t & 63)];
-          }
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&empty[stg]);
-        }
-        const int64_t p = static_cast<int64_t>(W.j) * kTile + t;
-        const int64_t prow = mrow >= 0 ? static_cast<int64_t>(mrow) + (t & 63) : (GATHER && mrow == -3 ? -3 : -1);
-        const float* wb = wbufs + qi * (C::kWBytes / 4);
-        float sc[QB];
-#pragma unroll
-        for (int qq = 0; qq < QB; ++qq) {
-          float s = 0.f;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            float v[32];
-            const uint32_t col = acc * C::kAccCols + (C::kFp8 ? qq * 2 * kHeads : qq * kHeads) + c * 32;
-            tc::tmem_ld32(tmem_base + lane_base + col, v);
-            if (C::kFp8) {
-              float u[32];
-              tc::tmem_ld32(tmem_base + lane_base + col + kHeads, u);
-              tc::tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) s = fmaf(wb[qq * kHeads + c * 32 + i], fmaxf(v[i] + u[i], 0.f), s);
-            } else {
-              tc::tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) s = fmaf(wb[qq * kHeads + c * 32 + i], fmaxf(v[i], 0.f), s);
+          tc::tc_fence_after();
+          // The tile's key rows (and FP8 scales) come from the producer through
+          // the stage; the stage is released once all four warps have read them.
+          int32_t mrow = 0;  // contiguous bf16: every visible position has a key row
+          float kscale = 1.f;
+          if (stage_meta) {
+            const int stg = static_cast<int>(it % C::kNS);
+            if (!tc::mbar_wait(&full[stg], static_cast<uint32_t>((it / C::kNS) & 1), abort_flag)) {
+              if (lane == 0) {
+                record_error(a.status, LSA_ERR_TIMEOUT, 0, 8);
+                *abort_flag = 1;
+              }
+              hist_row = -1;
+              break;
             }
+            if (GATHER) {
+              // row t has a key (0), is a padding entry (-3: -inf) or an out-of-range one (-1: NaN)
+              const uint32_t* mk = smask + 8 * stg;
+              mrow = ((mk[t >> 5] >> (t & 31)) & 1u) ? 0 : (((mk[4 + (t >> 5)] >> (t & 31)) & 1u) ? -1 : -3);
+            } else {
+              const int box = 2 * stg + (t >> 6);
+              mrow = smeta[box];
+              if (C::kFp8 && mrow >= 0) kscale = sscale[box * kScaleSlot + (mrow & 3) + (t & 63)];
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&empty[stg]);
           }
-          sc[qq] = s * kscale;
-        }
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&tempty[acc]);
-        if (use_hist && p < vis_r[0] && prow >= 0) {
-          const uint32_t key = order_key(sc[0]);
-          if (key) atomicAdd(&shist[key >> 20], 1u);
-        }
-#pragma unroll
-        for (int qq = 0; qq < QB; ++qq) {
-          if (qq < W.g.nrows && p < a.ld) {
-            float o = -INFINITY;
-            if (p < vis_r[qq]) o = prow >= 0 ? sc[qq] : (prow == -3 ? -INFINITY : NAN);
-            a.scores[static_cast<int64_t>(W.g.r0 + qq) * a.ld + p] = o;
+          const int64_t p = static_cast<int64_t>(W.j) * kTile + t;
+          const int64_t prow = mrow >= 0 ? static_cast<int64_t>(mrow) + (t & 63) : (GATHER && mrow == -3 ? -3 : -1);
+          const float* wb = wbufs + qi * (C::kWBytes / 4);
+          float sc[QB];
+  #pragma unroll
+          for (int qq = 0; qq < QB; ++qq) {
+            float s = 0.f;
+  #pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              float v[32];
+              const uint32_t col = acc * C::kAccCols + (C::kFp8 ? qq * 2 * kHeads : qq * kHeads) + c * 32;
+              tc::tmem_ld32(tmem_base + lane_base + col, v);
+              const float4* w4 = reinterpret_cast<const float4*>(wb + qq * kHeads + c * 32);
+              if (C::kFp8) {
+                float u[32];
+                tc::tmem_ld32(tmem_base + lane_base + col + kHeads, u);
+                tc::tmem_wait_ld();
+  #pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 w = w4[i];
+                  s = fmaf(w.x, fmaxf(v[4 * i] + u[4 * i], 0.f), s);
+                  s = fmaf(w.y, fmaxf(v[4 * i + 1] + u[4 * i + 1], 0.f), s);
+                  s = fmaf(w.z, fmaxf(v[4 * i + 2] + u[4 * i + 2], 0.f), s);
+                  s = fmaf(w.w, fmaxf(v[4 * i + 3] + u[4 * i + 3], 0.f), s);
+                }
+              } else {
+                tc::tmem_wait_ld();
+  #pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 w = w4[i];
+                  s = fmaf(w.x, fmaxf(v[4 * i], 0.f), s);
+                  s = fmaf(w.y, fmaxf(v[4 * i + 1], 0.f), s);
+                  s = fmaf(w.z, fmaxf(v[4 * i + 2], 0.f), s);
+                  s = fmaf(w.w, fmaxf(v[4 * i + 3], 0.f), s);
+                }
+              }
+            }
+            sc[qq] = s * kscale;
+          }
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+          if (use_hist && p < vis_r[0] && prow >= 0) {
+            const uint32_t key = order_key(sc[0]);
+            if (key) atomicAdd(&shist[key >> 20], 1u);
+          }
+  #pragma unroll
+          for (int qq = 0; qq < QB; ++qq) {
+            if (qq < W.g.nrows && p < a.ld) {
+              float o = -INFINITY;
+              if (p < vis_r[qq]) o = prow >= 0 ? sc[qq] : (prow == -3 ? -INFINITY : NAN);
+              a.scores[static_cast<int64_t>(W.g.r0 + qq) * a.ld + p] = o;
+            }
           }
         }
         const bool last = (it + 1 == plan.n_items) || (W.j + 1 >= W.g.tiles);
@@ -984,16 +1012,17 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     }
   }
   tc::tc_fence_before();
-  scan_sync();
+  scan_sync<NTH>();
   if (threadIdx.x == 0) {
     for (uint64_t* b = bars; b <= ebar; ++b) tc::mbar_inval(b);
   }
-  scan_sync();
+  scan_sync<NTH>();
   if (a.done_ctr) {
-    // decode step: the top-k starts on this count instead of the grid's completion
-    __threadfence();  // this thread's score stores and histogram adds
-    scan_sync();
-    if (threadIdx.x == 0) atomicAdd(a.done_ctr, 1u);
+    // decode step: the top-k starts on this count instead of the grid's
+    // completion; the barrier orders every thread's score stores and histogram
+    // adds before thread 0's release
+    scan_sync<NTH>();
+    if (threadIdx.x == 0) tc::red_release_gpu_add(a.done_ctr, 1u);
   }
 }
 

@@ -162,6 +162,26 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 
 __device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 
+// Publishing a CTA's global writes to other CTAs: after a CTA-wide barrier
+// (which orders every thread's writes before it), ONE thread adds to a counter
+// with release semantics at GPU scope; a thread that acquires the counter's
+// new value then sees all of those writes (causality through the barrier).
+// This replaces a fence in every thread, which waits for the whole memory
+// system, by one release.
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Add with acquire and release at GPU scope: publishes like red_release_gpu_add
+// and returns the old value, having acquired what earlier adders published.
+__device__ __forceinline__ uint32_t atom_acq_rel_gpu_add(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Split cluster barrier: every thread of every CTA of the cluster arrives
 // (relaxed) and later waits; used once, right after the mbarriers are
 // initialised, so that no CTA arrives remotely on a barrier not yet set up.

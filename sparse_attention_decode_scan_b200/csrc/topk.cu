@@ -565,7 +565,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
       if (e != cudaSuccess) return e;
       k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
     }
-    if (topk_cluster_ok(a.n_cols) && !a.split_select) {
+    if (topk_cluster_ok(a.n_cols) && !a.split_select && a.allow_cluster) {
       // one cluster of up to 8 CTAs per row
       const tk::ClPlan cp = tk::cl_plan(a.n_cols);
       const size_t smem = tk::cl_smem(cp.seg_len);

@@ -18,6 +18,7 @@
 // positions equal to T are taken first), and compacts its own segment into
 // the output.  If any CTA's candidates overflow its list, T is found from the
 // whole row and each segment is re-read to mark.
+#include "tc.cuh"
 #include "topk_sel.cuh"
 
 namespace lsa {
@@ -284,15 +285,13 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
     for (int i = static_cast<int>(keff) + s * NT + t; i < a.k; i += ns * NT) out[i] = -1;
     if (a.wait_ctr) {
       // decode step: the last CTA of the row to finish raises the row's flag
-      // (the attention of row r may read its selection from then on)
-      __threadfence();
+      // (the attention of row r may read its selection from then on).  The
+      // barrier orders this CTA's output writes before thread 0's release;
+      // the last adder has acquired the others' and releases all of them.
       tk_sync<NT, ID>();
       if (t == 0) {
-        const uint32_t done = atomicAdd(L.row_done + r, 1u);
-        if (done == static_cast<uint32_t>(ns - 1)) {
-          __threadfence();
-          asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(L.sel_done + r), "r"(1u) : "memory");
-        }
+        const uint32_t done = tc::atom_acq_rel_gpu_add(L.row_done + r, 1u);
+        if (done == static_cast<uint32_t>(ns - 1)) tc::st_release_gpu(L.sel_done + r, 1u);
       }
     }
   }

@@ -59,12 +59,13 @@ def use_test_library(on: bool = True) -> None:
     _use_test = bool(on)
 
 
-def set_test_hooks(force_simt: bool = False, split_select_min_cols: int = -1, scan_wait_extra: int = 0) -> None:
+def set_test_hooks(force_simt: bool = False, split_select_min_cols: int = -1, scan_wait_extra: int = 0,
+                   no_cluster_topk: bool = False) -> None:
     """lsa_test_set_hooks of liblsa_test.so (include/lsa_test.h); needs use_test_library()."""
     if not _use_test:
         raise RuntimeError("test hooks exist only in liblsa_test.so: call use_test_library() first")
-    _check(lib().lsa_test_set_hooks(1 if force_simt else 0, int(split_select_min_cols), int(scan_wait_extra)),
-           "lsa_test_set_hooks")
+    _check(lib().lsa_test_set_hooks(1 if force_simt else 0, int(split_select_min_cols), int(scan_wait_extra),
+                                    1 if no_cluster_topk else 0), "lsa_test_set_hooks")
 
 
 def lib() -> ctypes.CDLL:
@@ -103,7 +104,7 @@ def lib() -> ctypes.CDLL:
              "lsa_decode_step_profiled", "lsa_decode_layers", "lsa_read_device_status", "lsa_candidate_scores",
              "lsa_two_stage_select"]
     if path == TEST_LIB_PATH:
-        L.lsa_test_set_hooks.argtypes = [i32, i64, ctypes.c_uint32]
+        L.lsa_test_set_hooks.argtypes = [i32, i64, ctypes.c_uint32, i32]
         names.append("lsa_test_set_hooks")
     for f in names:
         getattr(L, f).restype = ctypes.c_int

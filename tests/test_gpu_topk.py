@@ -67,6 +67,32 @@ def test_topk_exact(kind, rows, n, k, mode):
         assert np.array_equal(got[r], want), f"row {r}: first mismatch at {int(np.argmax(got[r] != want))}"
 
 
+@pytest.mark.parametrize("kind,rows,n,k,mode", [c for c in CASES if c[2] <= (1 << 18)][:10],
+                         ids=[f"{c[0]}-{c[1]}x{c[2]}-k{c[3]}-{c[4]}" for c in CASES if c[2] <= (1 << 18)][:10])
+def test_topk_collect_select_path_equals_cluster_path(kind, rows, n, k, mode, test_hooks):
+    """Rows of up to 2^18 positions take the one-cluster-per-row kernel; the
+    collect + per-row select kernel (the path of longer rows, forced here by
+    the test build) gives the same index arrays."""
+    from sparse_attention_decode_scan_b200 import lsa
+    seed = 900 + rows + n % 97 + k
+    sc = synth.topk_scores(kind, rows, n, seed)
+    valid = _valid(mode, rows, n, seed)
+    ld = (n + 3) // 4 * 4
+    dev = torch.full((rows, ld), float("nan"), dtype=torch.float32, device="cuda")
+    dev[:, :n] = torch.from_numpy(sc).cuda()
+    vdev = torch.from_numpy(valid).cuda() if valid is not None else None
+    got = []
+    for no_cluster in (False, True):
+        test_hooks(no_cluster_topk=no_cluster)
+        idx = torch.full((rows, k), -7, dtype=torch.int32, device="cuda")
+        ws = lsa.workspace(lsa.topk_workspace_size(rows, n, k))
+        lsa.topk(dev, k, idx, ws, valid_len=vdev, n_cols=n, ld=ld)
+        torch.cuda.synchronize()
+        assert lsa.read_device_status(ws) == lsa.LSA_OK
+        got.append(idx.cpu().numpy())
+    assert np.array_equal(got[0], got[1])
+
+
 def test_topk_repeatable_and_workspace_reuse():
     from sparse_attention_decode_scan_b200 import lsa
     rows, n, k = 6, 50000, 2048
