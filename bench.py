@@ -246,6 +246,8 @@ def run_ours(args, world, rank, local):
     spec = base
     if args.batch:
         spec = synth.scaled(spec, batch=args.batch)
+    if args.chunk and spec.causal:
+        spec = synth.scaled(spec, chunk=args.chunk)
     if args.op == "scan":
         spec = synth.scaled(spec, with_kv=False)
     case = synth.make_case(spec, rank_seed(base, rank))
@@ -750,6 +752,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     # profiling aids: a smaller batch of the same workload, one stage only, no clock soak
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
+    ap.add_argument("--chunk", type=int, default=0,
+                    help="prefill: the last CHUNK rows of the workload's chunk only (profiling)")
     ap.add_argument("--op", default="step", choices=["step", "scan", "topk", "attn"],
                     help="time one stage only (profiling); the bench line is for 'step'")
     ap.add_argument("--no-soak", action="store_true", help="skip the 1 s clock-sampling soak (profiling)")
