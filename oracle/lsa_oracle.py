@@ -310,3 +310,56 @@ def two_stage_select(case, compact_bits: np.ndarray, compact_scales: np.ndarray,
     exact = np.full(L, -np.inf)
     exact[cand] = row_scores(case, r)[cand]
     return topk(exact, L, k)
+
+
+# --------------------------------------------------------------------------- block selection
+# The SparDA abstract (page 4 of the sources) has the selector pick the KV
+# *blocks* a layer needs, and a forecast of the next layer's blocks lets their
+# host-to-device copy run while the current layer computes.  Readings where
+# the page is silent: a block is one cache page (block_size consecutive
+# positions); a block's score is the largest indexer score of its visible
+# tokens (the trained Forecast projection is out of scope, so the indexer's
+# own token scores stand in for the selector's); the kept blocks are the
+# n_blocks best by block score with ties to the lower block, ascending, -1
+# padded; the layer then attends every visible token of its kept blocks.
+
+def block_scores(scores: np.ndarray, valid_len: int, block_size: int) -> np.ndarray:
+    """Per block of block_size positions: the largest score among its positions
+    below valid_len (-inf for a block with none, NaN ignored)."""
+    s = np.asarray(scores, np.float64)[:int(valid_len)]
+    nb = (s.shape[0] + block_size - 1) // block_size
+    out = np.full(nb, -np.inf)
+    for blk in range(nb):
+        vals = s[blk * block_size:(blk + 1) * block_size]
+        vals = vals[~np.isnan(vals)]
+        if vals.size:
+            out[blk] = vals.max()
+    return out
+
+
+def block_select(scores: np.ndarray, valid_len: int, block_size: int, n_blocks: int) -> np.ndarray:
+    """The n_blocks best blocks by block score (ties to the lower block),
+    ascending, padded with -1."""
+    bs = block_scores(scores, valid_len, block_size)
+    return topk(bs, bs.shape[0], n_blocks)
+
+
+def block_positions(blocks: np.ndarray, block_size: int, valid_len: int) -> np.ndarray:
+    """Every position below valid_len inside the given blocks (-1 skipped), ascending."""
+    pos = [b * block_size + t for b in np.asarray(blocks) if b >= 0 for t in range(block_size)
+           if b * block_size + t < valid_len]
+    return np.array(sorted(pos), np.int64)
+
+
+def row_block_step(case, r: int, n_blocks: int, q_row=None):
+    """Row r of a case: its kept blocks (by its indexer scores), the positions
+    they cover, and the attention of q_row (default the row's own attention
+    query, decoded) over those positions."""
+    s = case.spec
+    L = row_visible(case, r)
+    blocks = block_select(row_scores(case, r), L, s.block_size, n_blocks)
+    pos = block_positions(blocks, s.block_size, L)
+    q = decode(case.q[r], s.act_dtype) if q_row is None else q_row
+    o, lse = sparse_attention(q, case.kv, int(case.row_seq[r]), pos, case.block_table, s.block_size, s.stride,
+                              s.act_dtype, s.v_dim, s.softmax_scale)
+    return blocks, pos, o, lse

@@ -665,8 +665,9 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
           rows[h] = r;
         }
       };
-      // the keys are streamed once per step: evict them from L2 first
-      const uint64_t l2_policy = tc::l2_evict_first_policy();
+      // decode streams each key once per step: evict it first; the causal
+      // prefill reads every key once per group of query rows: keep it
+      const uint64_t l2_policy = a.row_pos ? tc::l2_evict_last_policy() : tc::l2_evict_first_policy();
       Walker<QB> Wb;
       Wb.start(a, plan.r_first, plan.j_first);
       Look cur = look(Wb, 0);

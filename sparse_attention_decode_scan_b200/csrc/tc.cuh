@@ -235,6 +235,15 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // L2 policy for data read once: its lines are the first to be evicted, so a
 // long stream does not push out what the next kernels reuse (their code,
 // histograms, selections, block tables).
+// L2 policy for data every CTA reads again and again (the causal prefill's
+// keys): its lines are the last to be evicted, so the stream of score stores
+// does not push them out.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -19,7 +19,9 @@
 // launches, so no kernel waits on another CTA.
 #include <math.h>
 
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include <string.h>
 
@@ -440,6 +442,58 @@ __global__ void __launch_bounds__(tk::kClThreads, 2) k_tk_cluster(TopkArgs a, in
   tk::tk_cluster_row<2>(a, r, static_cast<int>(tc::cluster_ctarank()), nseg, seg_len, csm, S, s_live != 0);
 }
 
+// Clusters of `nseg` k_tk_cluster CTAs (with `smem` bytes each) the current
+// device keeps resident at once; queried once per (device, nseg, smem).
+int cluster_capacity(int nseg, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, size_t>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(dev, nseg, smem);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (ensure_dyn_smem(k_tk_cluster, smem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(nseg), 1, 1);
+    cfg.blockDim = dim3(tk::kClThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(nseg);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, k_tk_cluster, &cfg) != cudaSuccess) n = 0;
+  }
+  (void)cudaGetLastError();
+  cache[key] = n;
+  return n;
+}
+
+// The cluster plan of the one-cluster-per-row top-k for these sizes: the
+// largest cluster (8, 4, 2 CTAs, or 1) whose clusters for every row fit on the
+// device at once (a cluster that waits for a second wave costs a whole row's
+// time again).  nseg = 0: too many rows for one wave; the collect + select
+// kernel takes them.
+tk::ClPlan cluster_plan(int32_t rows, int64_t n_cols) {
+  for (int cap = tk::kClMaxSeg; cap >= 1; cap /= 2) {
+    const tk::ClPlan p = tk::cl_plan(n_cols, cap);
+    if (p.nseg < cap && cap > 1) continue;  // the row is too short for this many segments
+    if (static_cast<int64_t>(rows) <= cluster_capacity(p.nseg, tk::cl_smem(p.seg_len))) return p;
+  }
+  tk::ClPlan none;
+  none.nseg = 0;
+  none.seg_len = 0;
+  return none;
+}
+
 // SMs of the current device (the plan's CTA target).
 int device_sms() {
   int dev = 0, n = 0;
@@ -565,9 +619,11 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
       if (e != cudaSuccess) return e;
       k_tk_hist12<<<grid, kT, 0, s>>>(a, p.seg_len);
     }
-    if (topk_cluster_ok(a.n_cols) && !a.split_select && a.allow_cluster) {
+    const tk::ClPlan clp = (topk_cluster_ok(a.n_cols) && !a.split_select && a.allow_cluster)
+                               ? cluster_plan(a.rows, a.n_cols) : tk::ClPlan{0, 0};
+    if (clp.nseg > 0) {
+      const tk::ClPlan& cp = clp;
       // one cluster of up to 8 CTAs per row
-      const tk::ClPlan cp = tk::cl_plan(a.n_cols);
       const size_t smem = tk::cl_smem(cp.seg_len);
       e = ensure_dyn_smem(k_tk_cluster, smem);
       if (e != cudaSuccess) return e;

@@ -27,7 +27,7 @@ namespace tk {
 constexpr int kClThreads = kCollectThreads;        // the round shape of tk_round_load
 constexpr int kClMaxSeg = 8;                       // CTAs per cluster (portable cluster size)
 constexpr int64_t kClMaxCols = int64_t(1) << 18;   // longer rows take the collect + select bodies
-constexpr int kClCandCap = 2048;                   // threshold-bin keys a CTA keeps
+constexpr int kClCandCap = 1024;                   // threshold-bin keys a CTA keeps
 
 struct ClHdr {
   uint32_t nc;  // keys of the threshold bin in the segment (> kClCandCap: the list overflowed)
@@ -41,11 +41,14 @@ struct ClPlan {
   int64_t seg_len;  // multiple of kColRound
 };
 
-__host__ __device__ inline ClPlan cl_plan(int64_t n_cols) {
+// Segments of a row: up to max_seg CTAs (at most kClMaxSeg), at least one
+// collect round (kColRound positions) each.
+__host__ __device__ inline ClPlan cl_plan(int64_t n_cols, int max_seg = kClMaxSeg) {
   ClPlan p;
   int64_t rounds = (n_cols + kColRound - 1) / kColRound;
   if (rounds < 1) rounds = 1;
-  const int64_t ns = rounds < kClMaxSeg ? rounds : kClMaxSeg;
+  const int64_t cap = max_seg < kClMaxSeg ? (max_seg < 1 ? 1 : max_seg) : kClMaxSeg;
+  const int64_t ns = rounds < cap ? rounds : cap;
   const int64_t per = (rounds + ns - 1) / ns;
   p.seg_len = per * kColRound;
   p.nseg = static_cast<int>((rounds + per - 1) / per);
@@ -53,15 +56,17 @@ __host__ __device__ inline ClPlan cl_plan(int64_t n_cols) {
 }
 
 // Shared memory of the body: header | bitmap of the segment | tie bitmap |
-// candidates.  The bitmaps are padded per thread (tk_pad) so the ordered walk
-// over each thread's own words hits distinct banks.
+// candidates | every CTA's candidate keys, gathered.  The bitmaps are padded
+// per thread (tk_pad) so the ordered walk over each thread's own words hits
+// distinct banks.
 __host__ __device__ inline int cl_bm_words(int64_t seg_len) {
   const TkPad p = tk_pad(seg_len, kClThreads);
   return (kClThreads * p.stride + 3) / 4 * 4;
 }
 
 __host__ __device__ inline size_t cl_smem(int64_t seg_len) {
-  return sizeof(ClHdr) + 2 * static_cast<size_t>(cl_bm_words(seg_len)) * 4 + static_cast<size_t>(kClCandCap) * 8;
+  return sizeof(ClHdr) + 2 * static_cast<size_t>(cl_bm_words(seg_len)) * 4 + static_cast<size_t>(kClCandCap) * 8 +
+         static_cast<size_t>(kClMaxSeg) * kClCandCap * 4;
 }
 
 // Row r, segment s of ns (CTA rank s of the row's cluster).  `live` false (a
@@ -80,6 +85,7 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
   uint32_t* bm = reinterpret_cast<uint32_t*>(dsm + sizeof(ClHdr));
   uint32_t* tb = bm + bm_words;
   uint2* cs = reinterpret_cast<uint2*>(tb + bm_words);
+  uint32_t* allk = reinterpret_cast<uint32_t*>(cs + kClCandCap);  // [kClMaxSeg * kClCandCap]
   const DivU32 dper = make_divu32(static_cast<uint32_t>(pad.per));
   auto pw = [&](uint32_t w) -> int {  // padded index of segment word w
     const uint32_t q = divu32(dper, w);
@@ -168,28 +174,56 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
   if (t == 0) hdr->nc = static_cast<uint32_t>(nc);
   tc::cluster_sync();  // ---- every segment collected
   // ---------------------------------------------------------------- threshold key T
-  bool ovf = false;
+  // every CTA's candidate count and keys, copied into this CTA's shared
+  // memory with all of the remote loads in flight at once (a remote load is a
+  // round trip; one after another they would cost a round trip each)
   const uint32_t hdr_u = tc::smem_u32(hdr), cs_u = tc::smem_u32(cs);
-#pragma unroll 1
-  for (int q = 0; q < ns; ++q)
-    ovf |= tc::ld_cluster_u32(tc::cluster_map(hdr_u, static_cast<uint32_t>(q))) > static_cast<uint32_t>(kClCandCap);
+  uint32_t ncq[kClMaxSeg];
+#pragma unroll
+  for (int q = 0; q < kClMaxSeg; ++q)
+    ncq[q] = q < ns ? tc::ld_cluster_u32(tc::cluster_map(hdr_u, static_cast<uint32_t>(q))) : 0u;
+  bool ovf = false;
+  int n_all = 0;
+  uint32_t offq[kClMaxSeg];
+#pragma unroll
+  for (int q = 0; q < kClMaxSeg; ++q) {
+    ovf |= ncq[q] > static_cast<uint32_t>(kClCandCap);
+    offq[q] = static_cast<uint32_t>(n_all);
+    n_all += static_cast<int>(ncq[q]);
+  }
+  if (live && keff > 0 && !ovf) {
+    constexpr int U = kClCandCap / NT;
+    uint32_t kv[kClMaxSeg][U];
+#pragma unroll
+    for (int q = 0; q < kClMaxSeg; ++q) {
+      const uint32_t base_q = tc::cluster_map(cs_u, static_cast<uint32_t>(q < ns ? q : 0));
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t c = static_cast<uint32_t>(t + u * NT);
+        kv[q][u] = c < ncq[q] ? tc::ld_cluster_u32(base_q + c * 8u) : 0u;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kClMaxSeg; ++q) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t c = static_cast<uint32_t>(t + u * NT);
+        if (c < ncq[q]) allk[offq[q] + c] = kv[q][u];
+      }
+    }
+  }
   uint32_t T = 0, ties = 0;
   if (live && keff > 0) {
     if (!ovf) {
       for (int pass = 0; pass < 2; ++pass) {
         for (int i = t; i < 1024; i += NT) S.h[i] = 0;
-        tk_sync<NT, ID>();
+        tk_sync<NT, ID>();  // also: the gathered keys are complete
         const uint32_t shift = pass == 0 ? 10 : 0;
         const uint32_t pre_shift = pass == 0 ? 20 : 10;
         const uint32_t prefix = pass == 0 ? b1 : (T >> 10);
-#pragma unroll 1
-        for (int q = 0; q < ns; ++q) {
-          const uint32_t base_q = tc::cluster_map(cs_u, static_cast<uint32_t>(q));
-          const int nc_q = static_cast<int>(tc::ld_cluster_u32(tc::cluster_map(hdr_u, static_cast<uint32_t>(q))));
-          for (int c = t; c < nc_q; c += NT) {
-            const uint32_t key = tc::ld_cluster_u32(base_q + static_cast<uint32_t>(c) * 8u);
-            if ((key >> pre_shift) == prefix) atomicAdd(&S.h[(key >> shift) & 1023u], 1u);
-          }
+        for (int c = t; c < n_all; c += NT) {
+          const uint32_t key = allk[c];
+          if ((key >> pre_shift) == prefix) atomicAdd(&S.h[(key >> shift) & 1023u], 1u);
         }
         tk_sync<NT, ID>();
         uint32_t hl[1024 / NT];
@@ -240,12 +274,18 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
     hdr->eq = static_cast<uint32_t>(eq_tot);
   }
   tc::cluster_sync();  // ---- every segment's counts published
-  // entries before this segment and the ties left to it (lowest positions first)
+  // entries before this segment and the ties left to it (lowest positions
+  // first); the remote counts are loaded together
+  uint32_t gtq[kClMaxSeg], eqq[kClMaxSeg];
+#pragma unroll
+  for (int q = 0; q < kClMaxSeg; ++q) {
+    gtq[q] = q < ns ? tc::ld_cluster_u32(tc::cluster_map(hdr_u + 4u, static_cast<uint32_t>(q))) : 0u;
+    eqq[q] = q < ns ? tc::ld_cluster_u32(tc::cluster_map(hdr_u + 8u, static_cast<uint32_t>(q))) : 0u;
+  }
   uint32_t off = 0, ties_mine = 0, eq_seen = 0;
-#pragma unroll 1
-  for (int q = 0; q < ns; ++q) {
-    const uint32_t gt_q = tc::ld_cluster_u32(tc::cluster_map(hdr_u + 4u, static_cast<uint32_t>(q)));
-    const uint32_t eq_q = tc::ld_cluster_u32(tc::cluster_map(hdr_u + 8u, static_cast<uint32_t>(q)));
+#pragma unroll
+  for (int q = 0; q < kClMaxSeg; ++q) {
+    const uint32_t gt_q = gtq[q], eq_q = eqq[q];
     const uint32_t left = ties > eq_seen ? ties - eq_seen : 0u;
     const uint32_t take = left < eq_q ? left : eq_q;
     if (q < s) off += gt_q + take;
