@@ -301,6 +301,57 @@ lsa_status lsa_two_stage_select(const lsa_dims* d, const lsa_cache* c, const voi
                                 lsa_stream_t stream);
 
 /*
+ * Block-level selection (SparDA abstract, page 4 of the sources: the selector
+ * picks the KV blocks a layer needs, and a forecast of the next layer's blocks
+ * lets their host-to-device copy overlap the current layer's work).
+ *
+ * lsa_block_select: for each row, the score of every block of block_size
+ * consecutive positions is the largest score among its positions below
+ * valid_len[r] (or n_cols; NaN ignored, -inf for a block with none); the
+ * n_sel best blocks (ties to the lower block; blocks scoring -inf never) go
+ * to kept [rows, n_sel] device int32, ascending, -1 padded.
+ *   scores [rows, ld] device fp32 (e.g. lsa_indexer_scores' output).
+ * Workspace: lsa_block_select_workspace_size(rows, n_cols, block_size, n_sel).
+ * Launches: the block maximum, then the top-k's (2).
+ */
+size_t lsa_block_select_workspace_size(int32_t rows, int64_t n_cols, int32_t block_size, int32_t n_sel);
+lsa_status lsa_block_select(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len,
+                            int64_t n_cols, int32_t block_size, int32_t n_sel, int32_t* kept,
+                            void* ws, size_t ws_bytes, lsa_stream_t stream);
+
+/*
+ * lsa_stage_blocks: copies every row's kept blocks from the cache's KV into a
+ * staging pool, one launch of one CTA per (row, kept block):
+ *   c->kv may be device memory or page-locked host memory the device can map
+ *     (an offloaded cache: the copy then reads it across the host link; issue
+ *     the call on a copy-side stream to overlap it with other work).  Other
+ *     host memory returns LSA_ERR_INVALID_ARG.
+ *   row_seq, row_pos: as lsa_indexer_scores (a causal row keeps the positions
+ *     up to its own).
+ *   kept [rows, n_sel] device: block ids as lsa_block_select gives them.
+ *   block_size: positions per block; for a paged cache it must equal
+ *     d->block_size (a kept block is one page).
+ *   staged_kv [rows * n_sel, block_size, D] device, act_dtype out: staged block
+ *     r * n_sel + i holds kept block i of row r (rows past the sequence zero).
+ *   staged_table [rows, n_sel] device int32 out: r * n_sel + i, or -1 where
+ *     nothing was kept.
+ *   staged_idx [rows, n_sel * block_size] device int32 out: the positions of the
+ *     staged sequence the row attends: i * block_size + t for every kept
+ *     position, -1 elsewhere.
+ * The row then attends its kept blocks with lsa_sparse_attn_decode on a cache
+ * over the staging pool (kv = staged_kv, block_table = staged_table,
+ * block_size = block_size, max_blocks_per_seq = n_sel, n_blocks = rows *
+ * n_sel, max_len = n_sel * block_size, seq_lens = that length per row, batch
+ * = rows), d->top_k = n_sel * block_size, and idx = staged_idx.
+ * Workspace: 256 bytes (the status word; a block id outside the pool records
+ * LSA_ERR_BOUNDS).
+ */
+lsa_status lsa_stage_blocks(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
+                            const int32_t* row_pos, const int32_t* kept, int32_t n_sel, int32_t block_size, void* staged_kv,
+                            int32_t* staged_table, int32_t* staged_idx, void* ws, size_t ws_bytes,
+                            lsa_stream_t stream);
+
+/*
  * Copies the workspace status word to *status (an lsa_status value), clears it,
  * and synchronises `stream`.  Returns LSA_ERR_CUDA if a CUDA call fails.
  */

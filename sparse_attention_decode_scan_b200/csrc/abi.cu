@@ -634,6 +634,73 @@ lsa_status lsa_two_stage_select(const lsa_dims* d, const lsa_cache* c, const voi
   return cuda_status(launch_cand_positions(slot, cand, rows, d->top_k, n_cand, idx, s));
 }
 
+size_t lsa_block_select_workspace_size(int32_t rows, int64_t n_cols, int32_t block_size, int32_t n_sel) {
+  if (rows < 0 || n_cols < 0 || block_size < 1 || n_sel < 1) return 0;
+  const int64_t nb = (n_cols + block_size - 1) / block_size;
+  const int64_t nb_ld = score_ld(nb);
+  return kStatusBytes + align_up(static_cast<size_t>(rows) * nb_ld * 4) + align_up(topk_ws_bytes(rows, nb, n_sel));
+}
+
+lsa_status lsa_block_select(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
+                            int32_t block_size, int32_t n_sel, int32_t* kept, void* ws, size_t ws_bytes,
+                            lsa_stream_t stream) {
+  if (rows < 0 || n_cols < 0 || ld < n_cols || block_size < 1 || n_sel < 1) return LSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!scores || !kept)) return LSA_ERR_INVALID_ARG;
+  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
+  const int64_t nb = (n_cols + block_size - 1) / block_size;
+  const int64_t nb_ld = score_ld(nb);
+  lsa_status st = ws_check(ws, ws_bytes, lsa_block_select_workspace_size(rows, n_cols, block_size, n_sel));
+  if (st != LSA_OK) return st;
+  if (rows == 0) return LSA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* bscores = reinterpret_cast<float*>(base + kStatusBytes);
+  void* inner = base + kStatusBytes + align_up(static_cast<size_t>(rows) * nb_ld * 4);
+  if (launch_block_max(scores, ld, rows, valid_len, n_cols, block_size, nb_ld, bscores, s) != cudaSuccess)
+    return LSA_ERR_CUDA;
+  // every block past a row's visible range scores -inf and is never kept
+  return do_topk(bscores, nb_ld, rows, nullptr, nb, n_sel, kept, ws, inner, s);
+}
+
+lsa_status lsa_stage_blocks(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
+                            const int32_t* row_pos, const int32_t* kept, int32_t n_sel, int32_t block_size, void* staged_kv,
+                            int32_t* staged_table, int32_t* staged_idx, void* ws, size_t ws_bytes,
+                            lsa_stream_t stream) {
+  if (!valid_dims(d) || !c || !c->seq_lens || c->batch < 0 || c->max_len < 0 || !c->kv) return LSA_ERR_INVALID_ARG;
+  if (rows < 0 || n_sel < 1 || block_size < 1) return LSA_ERR_INVALID_ARG;
+  if (d->block_size > 0) {  // a kept block of a paged cache is one page
+    if (block_size != d->block_size || !c->block_table || c->max_blocks_per_seq < 1 || c->n_blocks < 1)
+      return LSA_ERR_INVALID_ARG;
+  }
+  if (!row_seq && rows > c->batch) return LSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!kept || !staged_kv || !staged_table || !staged_idx || !aligned16(staged_kv)))
+    return LSA_ERR_INVALID_ARG;
+  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
+  const int64_t row_bytes = static_cast<int64_t>(d->qk_dim) * (d->act_dtype == LSA_F32 ? 4 : 2);
+  if (row_bytes % 16) return LSA_ERR_UNSUPPORTED;
+  lsa_status st = ws_check(ws, ws_bytes, kStatusBytes);
+  if (st != LSA_OK) return st;
+  if (rows == 0) return LSA_OK;
+  // the source may be host memory the device maps (an offloaded cache): the
+  // kernel then reads it through its device address
+  CacheView v = view(d, c);
+  cudaPointerAttributes pa;
+  if (cudaPointerGetAttributes(&pa, c->kv) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return LSA_ERR_INVALID_ARG;
+  }
+  if (pa.type == cudaMemoryTypeHost) {
+    if (!pa.devicePointer) return LSA_ERR_INVALID_ARG;
+    v.kv = pa.devicePointer;
+  } else if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged) {
+    return LSA_ERR_INVALID_ARG;  // unregistered host memory: the device cannot read it
+  }
+  if (!aligned16(v.kv)) return LSA_ERR_INVALID_ARG;
+  return cuda_status(launch_stage_blocks(v, rows, row_seq, row_pos, kept, n_sel, block_size, row_bytes, staged_kv,
+                                         staged_table, staged_idx, status_of(ws),
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream) {
   if (!ws || !status) return LSA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

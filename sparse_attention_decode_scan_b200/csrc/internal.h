@@ -67,6 +67,14 @@ cudaError_t launch_scores_tc(const ScoresArgs& a, cudaStream_t s);
 // test, and the launch.
 bool candidate_scores_tc_supported(const ScoresArgs& a);
 cudaError_t launch_candidate_scores_tc(const ScoresArgs& a, cudaStream_t s);
+// Block selection (blocks.cu): block scores [rows, nb_ld] = the largest visible
+// token score per block; the kept blocks' KV rows copied into a staging pool
+// (staged block r * n_sel + i), its block table and the staged positions.
+cudaError_t launch_block_max(const float* scores, int64_t ld, int32_t rows, const int32_t* valid_len, int64_t n_cols,
+                             int32_t block_size, int64_t nb_ld, float* out, cudaStream_t s);
+cudaError_t launch_stage_blocks(const CacheView& c, int32_t rows, const int32_t* row_seq, const int32_t* row_pos,
+                                const int32_t* kept, int32_t n_sel, int32_t sel_bs, int64_t row_bytes, void* staged,
+                                int32_t* staged_table, int32_t* staged_idx, DevStatus* status, cudaStream_t s);
 // idx[r][j] = cand[r][slot[r][j]] (-1 for slot -1): candidate entries -> positions.
 cudaError_t launch_cand_positions(const int32_t* slot, const int32_t* cand, int32_t rows, int32_t k, int32_t n_cand,
                                   int32_t* idx, cudaStream_t s);

@@ -100,9 +100,13 @@ def lib() -> ctypes.CDLL:
     L.lsa_two_stage_workspace_size.argtypes = [D, i32, i64, i32]
     L.lsa_two_stage_workspace_size.restype = sz
     L.lsa_two_stage_select.argtypes = [D, C, vp, vp, i32, vp, vp, vp, vp, i32, vp, vp, sz, vp]
+    L.lsa_block_select_workspace_size.argtypes = [i32, i64, i32, i32]
+    L.lsa_block_select_workspace_size.restype = sz
+    L.lsa_block_select.argtypes = [vp, i64, i32, vp, i64, i32, i32, vp, vp, sz, vp]
+    L.lsa_stage_blocks.argtypes = [D, C, i32, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]
     names = ["lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode", "lsa_decode_step",
              "lsa_decode_step_profiled", "lsa_decode_layers", "lsa_read_device_status", "lsa_candidate_scores",
-             "lsa_two_stage_select"]
+             "lsa_two_stage_select", "lsa_block_select", "lsa_stage_blocks"]
     if path == TEST_LIB_PATH:
         L.lsa_test_set_hooks.argtypes = [i32, i64, ctypes.c_uint32, i32]
         names.append("lsa_test_set_hooks")
@@ -249,6 +253,47 @@ def two_stage_select(dims: Dims, cache: Cache, compact_keys, compact_scales, q_i
                                              _ptr(w), int(n_cand), _ptr(idx), _ptr(ws),
                                              ws.numel() if ws is not None else 0, _stream(stream)),
                   "lsa_two_stage_select", raise_on_error)
+
+
+def block_select_workspace_size(rows: int, n_cols: int, block_size: int, n_sel: int) -> int:
+    return int(lib().lsa_block_select_workspace_size(rows, n_cols, block_size, n_sel))
+
+
+def block_select(scores, block_size: int, n_sel: int, kept, ws, valid_len=None, n_cols: Optional[int] = None,
+                 ld: Optional[int] = None, rows: Optional[int] = None, stream=None, raise_on_error=True) -> int:
+    """lsa_block_select: kept [rows, n_sel] block ids from scores [rows, ld]."""
+    rows = int(scores.shape[0]) if rows is None else rows
+    ld = int(scores.stride(0)) if ld is None else ld
+    n_cols = int(scores.shape[1]) if n_cols is None else n_cols
+    return _check(lib().lsa_block_select(_ptr(scores), ld, rows, _ptr(valid_len), n_cols, int(block_size),
+                                         int(n_sel), _ptr(kept), _ptr(ws), ws.numel() if ws is not None else 0,
+                                         _stream(stream)), "lsa_block_select", raise_on_error)
+
+
+def stage_blocks(dims: Dims, cache: Cache, kept, block_size: int, staged_kv, staged_table, staged_idx, ws,
+                 row_seq=None, row_pos=None, rows: Optional[int] = None, stream=None, raise_on_error=True) -> int:
+    """lsa_stage_blocks: the kept blocks' KV rows into the staging pool (cache.kv may be pinned host memory)."""
+    rows = int(kept.shape[0]) if rows is None else rows
+    return _check(lib().lsa_stage_blocks(ctypes.byref(dims), ctypes.byref(cache), rows, _ptr(row_seq), _ptr(row_pos),
+                                         _ptr(kept),
+                                         int(kept.shape[1]), int(block_size), _ptr(staged_kv), _ptr(staged_table),
+                                         _ptr(staged_idx), _ptr(ws), ws.numel() if ws is not None else 0,
+                                         _stream(stream)), "lsa_stage_blocks", raise_on_error)
+
+
+def staged_cache(staged_kv, staged_table, staged_lens, n_sel: int, block_size: int) -> Cache:
+    """The lsa_cache over a staging pool that lsa_sparse_attn_decode reads after lsa_stage_blocks."""
+    c = Cache()
+    c.idx_keys = None
+    c.idx_key_scales = None
+    c.kv = staged_kv.data_ptr()
+    c.block_table = staged_table.data_ptr()
+    c.max_blocks_per_seq = int(n_sel)
+    c.n_blocks = int(staged_table.numel())
+    c.max_len = int(n_sel * block_size)
+    c.seq_lens = staged_lens.data_ptr()
+    c.batch = int(staged_table.shape[0])
+    return c
 
 
 def read_device_status(ws, stream=None) -> int:
