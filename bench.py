@@ -736,6 +736,131 @@ def run_two_stage(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_blocks(args, world, rank, local):
+    """Layers that attend whole KV blocks picked a layer ahead, with the KV cache
+    offloaded to page-locked host memory (SparDA abstract: a forecast of the
+    next layer's blocks lets their host-to-device copy overlap the current
+    layer).  Per layer l, on the compute stream: the next layer's indexer scan
+    and block selection (lsa_block_select), then layer l's sparse attention
+    over its staged blocks; on a copy stream, concurrently: the next layer's
+    kept blocks copied from host memory into the other staging buffer
+    (lsa_stage_blocks).  The forecast query of layer l+1 is that layer's own
+    indexer query (the trained Forecast projection is out of scope).  Also
+    times the same layers with the copy in line (no overlap)."""
+    import torch
+
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase, make_dims
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = synth.workload(args.workload)
+    spec = synth.scaled(base, batch=args.batch) if args.batch else base
+    assert not spec.causal and spec.block_size > 0, "blocks: paged decode workloads"
+    case = synth.make_case(spec, rank_seed(base, rank))
+    dc = DeviceCase(case, device=dev)
+    s = case.spec
+    B, bs, n_sel = dc.rows, s.block_size, args.blocks
+    n_layers = args.layers if args.layers > 1 else 4
+    host_kv = dc.kv.cpu().pin_memory()  # the offloaded KV cache (one copy serves every layer)
+    hcache = dc.make_cache()
+    hcache.kv = host_kv.data_ptr()
+    qs = []
+    for l in range(n_layers + 1):
+        qi, wl, ql = synth.queries(s, rank_seed(base, rank), B, layer=l)
+        qs.append((to_dev(qi, s.act_dtype, dev), torch.from_numpy(wl).to(dev), to_dev(ql, s.act_dtype, dev)))
+    ld = (dc.max_len + 3) // 4 * 4
+    scores = torch.empty((B, ld), dtype=torch.float32, device=dev)
+    kept = [torch.empty((B, n_sel), dtype=torch.int32, device=dev) for _ in range(2)]
+    staged = [torch.empty((B * n_sel, bs, s.qk_dim), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    table = [torch.empty((B, n_sel), dtype=torch.int32, device=dev) for _ in range(2)]
+    sidx = [torch.empty((B, n_sel * bs), dtype=torch.int32, device=dev) for _ in range(2)]
+    lens = torch.full((B,), n_sel * bs, dtype=torch.int32, device=dev)
+    scache = [lsa.staged_cache(staged[i], table[i], lens, n_sel, bs) for i in range(2)]
+    ad = make_dims(s, top_k=n_sel * bs)
+    out = torch.empty((B, s.n_heads, s.v_dim), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, s.n_heads), dtype=torch.float32, device=dev)
+    ws_c = lsa.workspace(max(lsa.workspace_size(dc.dims, B, dc.max_len, lsa.LSA_OP_SCORES),
+                             lsa.block_select_workspace_size(B, dc.max_len, bs, n_sel),
+                             lsa.workspace_size(ad, B, n_sel * bs, lsa.LSA_OP_ATTN)), device=dev)
+    ws_x = lsa.workspace(256, device=dev)
+    comp = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+
+    def select(l):
+        qi, wl, _ = qs[l]
+        lsa.indexer_scores(dc.dims, dc.cache, qi, wl, scores, ld, ws_c, stream=comp)
+        lsa.block_select(scores, bs, n_sel, kept[l % 2], ws_c, valid_len=dc.seq_lens, n_cols=dc.max_len, ld=ld,
+                         stream=comp)
+
+    def stage(l, st):
+        lsa.stage_blocks(dc.dims, hcache, kept[l % 2], bs, staged[l % 2], table[l % 2], sidx[l % 2], ws_x, stream=st)
+
+    def attend(l):
+        lsa.sparse_attn_decode(ad, scache[l % 2], qs[l][2], sidx[l % 2], out, lse, ws_c, stream=comp)
+
+    def step(overlap):
+        select(0)
+        stage(0, comp)
+        for l in range(n_layers):
+            if l + 1 < n_layers:
+                select(l + 1)  # the forecast of the next layer's blocks
+                ev = torch.cuda.Event()
+                ev.record(comp)
+                st = copy if overlap else comp
+                if overlap:
+                    copy.wait_event(ev)
+                stage(l + 1, st)
+                done = torch.cuda.Event()
+                done.record(st)
+            attend(l)
+            if l + 1 < n_layers:
+                comp.wait_event(done)
+
+    res = {}
+    for overlap in (True, False):
+        for _ in range(args.warmup):
+            step(overlap)
+        torch.cuda.synchronize(dev)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(comp)
+        for _ in range(args.steps):
+            step(overlap)
+        b_.record(comp)
+        torch.cuda.synchronize(dev)
+        res[overlap] = reduce_max(a.elapsed_time(b_)) / args.steps
+    assert lsa.read_device_status(ws_c) == lsa.LSA_OK and lsa.read_device_status(ws_x) == lsa.LSA_OK
+    # the host link's copy rate for reference: one large page-locked copy
+    probe = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    dprobe = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    dprobe.copy_(probe, non_blocking=True)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    for _ in range(4):
+        dprobe.copy_(probe, non_blocking=True)
+    b_.record(comp)
+    torch.cuda.synchronize(dev)
+    h2d_gbs = 4 * probe.numel() / (a.elapsed_time(b_) / 1e3) / 1e9
+    L = case.seq_lens.astype(np.int64)
+    staged_bytes = int(np.minimum((L + bs - 1) // bs, n_sel).sum()) * bs * s.qk_dim * 2
+    ms = res[True]
+    line = {"metric": f"decode steps/s over {n_layers} layers attending {n_sel} KV blocks each, blocks of the next "
+                      f"layer staged from host memory during the current one",
+            "value": world / (ms / 1e3), "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_copy_in_line": res[False],
+            "overlap_gain": res[False] / ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded); KV in page-locked host memory",
+            "config": dict(workload_config(case), layers=n_layers, n_sel=n_sel, block_size=bs),
+            "staged_bytes_per_layer": staged_bytes,
+            "host_link_gbs_achieved": staged_bytes * (n_layers) / (ms / 1e3) / 1e9,
+            "host_link_gbs_plain_copy": h2d_gbs,
+            # per layer: scan, block maximum, top-k (histogram + select), staging copy, attention
+            "gpu_launches": args.steps * n_layers * 6,
+            }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def to_dev(arr, dtype, dev):
     from sparse_attention_decode_scan_b200.device import to_device
     return to_device(arr, dtype, dev)
@@ -762,6 +887,8 @@ def main(argv=None):
     ap.add_argument("--route", default="own", choices=["own", "prev"],
                     help="layers: attend the latest indexer layer at or before (own) or before (prev, MLI) a layer")
     ap.add_argument("--retention", type=int, default=1, help="layers: every retention-th layer keeps an indexer")
+    ap.add_argument("--blocks", type=int, default=0, metavar="N_SEL",
+                    help="layers attending N_SEL KV blocks each, staged from host memory a layer ahead")
     ap.add_argument("--two-stage", type=int, default=0, metavar="N_CAND",
                     help="decode steps whose selection is the two-stage search with a list of N_CAND")
     ap.add_argument("--fused", action="store_true",
@@ -785,6 +912,8 @@ def main(argv=None):
         else:
             if args.two_stage:
                 run_two_stage(args, world, rank, local)
+            elif args.blocks:
+                run_blocks(args, world, rank, local)
             elif args.layers > 1:
                 run_layers(args, world, rank, local)
             else:

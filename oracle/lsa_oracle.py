@@ -351,14 +351,16 @@ def block_positions(blocks: np.ndarray, block_size: int, valid_len: int) -> np.n
     return np.array(sorted(pos), np.int64)
 
 
-def row_block_step(case, r: int, n_blocks: int, q_row=None):
-    """Row r of a case: its kept blocks (by its indexer scores), the positions
-    they cover, and the attention of q_row (default the row's own attention
-    query, decoded) over those positions."""
+def row_block_step(case, r: int, n_blocks: int, q_row=None, block_size: int = None):
+    """Row r of a case: its kept blocks of block_size positions (default the
+    cache's page size) by its indexer scores, the positions they cover, and the
+    attention of q_row (default the row's own attention query, decoded) over
+    those positions."""
     s = case.spec
+    bs = s.block_size if block_size is None else block_size
     L = row_visible(case, r)
-    blocks = block_select(row_scores(case, r), L, s.block_size, n_blocks)
-    pos = block_positions(blocks, s.block_size, L)
+    blocks = block_select(row_scores(case, r), L, bs, n_blocks)
+    pos = block_positions(blocks, bs, L)
     q = decode(case.q[r], s.act_dtype) if q_row is None else q_row
     o, lse = sparse_attention(q, case.kv, int(case.row_seq[r]), pos, case.block_table, s.block_size, s.stride,
                               s.act_dtype, s.v_dim, s.softmax_scale)

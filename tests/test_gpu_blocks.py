@@ -98,7 +98,7 @@ def test_block_selection_and_staged_attention_vs_oracle(name, n_sel):
     # the staged copy and the attention over it, on the oracle's kept blocks
     _, o, l = _stage_and_attend(lsa, dc, ref, bs)
     for r in rows:
-        _, pos, o_ref, l_ref = O.row_block_step(case, r, n_sel)
+        _, pos, o_ref, l_ref = O.row_block_step(case, r, n_sel, block_size=bs)
         check_attention(o[r], o_ref, l[r], l_ref, what=f"{name} row {r}")
 
 
