@@ -861,6 +861,81 @@ def run_blocks(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_prefill_layers(args, world, rank, local):
+    """The prefill workload through several layers (lsa_prefill_layers), each
+    layer's history (131072 KV rows) in page-locked host memory and streamed
+    through two alternating device buffers, rows in blocks of --row-block.
+    Every layer uses layer 0's data (one host copy of the history; the copy
+    and the compute are what is timed).  Also times the same layers with the
+    history already on the device (no copy), for the overlap."""
+    import torch
+
+    from sparse_attention_decode_scan_b200 import lsa
+    from sparse_attention_decode_scan_b200.device import DeviceCase
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = synth.workload(args.workload)
+    if not base.causal:  # the mode runs the causal prefill workload
+        base = synth.workload(synth.PREFILL)
+    spec = synth.scaled(base, chunk=args.chunk) if args.chunk else base
+    case = synth.make_case(spec, rank_seed(base, rank))
+    dc = DeviceCase(case, device=dev)
+    s = case.spec
+    R, L = dc.rows, dc.max_len
+    n = args.layers if args.layers > 1 else 3
+    hist_len = int(case.row_pos[0])
+    host_hist = dc.kv[0, :hist_len].cpu().pin_memory()
+    dev_hist = dc.kv[0, :hist_len].contiguous()
+    chunk = dc.kv[0, hist_len:L].contiguous()
+    outs = [torch.empty((R, s.n_heads, s.v_dim), dtype=torch.bfloat16, device=dev) for _ in range(n)]
+    bufs = [torch.empty((L, s.qk_dim), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    rb = args.row_block if args.row_block else R
+    ws = lsa.workspace(lsa.prefill_layers_workspace_size(dc.dims, R, L, rb), device=dev)
+    events = [torch.cuda.Event() for _ in range(4)]
+    copy = torch.cuda.Stream(dev)
+    comp = torch.cuda.current_stream(dev)
+
+    def run(hist):
+        caches = []
+        for _ in range(n):
+            c = dc.make_cache()
+            c.kv = hist.data_ptr()
+            caches.append(c)
+        lsa.prefill_layers(dc.dims, caches, hist_len, [chunk] * n, dc.row_pos, [dc.q_idx] * n, [dc.w] * n,
+                           [dc.q] * n, outs, None, bufs, ws, rb, events, stream=comp, copy_stream=copy)
+
+    res = {}
+    for name, hist in (("host", host_hist), ("device", dev_hist)):
+        for _ in range(args.warmup):
+            run(hist)
+        torch.cuda.synchronize(dev)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(comp)
+        for _ in range(args.steps):
+            run(hist)
+        b_.record(comp)
+        torch.cuda.synchronize(dev)
+        res[name] = reduce_max(a.elapsed_time(b_)) / args.steps
+    assert lsa.read_device_status(ws) == lsa.LSA_OK
+    ms = res["host"]
+    kv_row = s.qk_dim * 2
+    line = {"metric": f"prefill chunk rows/s through {n} layers, history streamed from host memory through two "
+                      f"device buffers", "value": world * R * n / (ms / 1e3), "unit": "chunk rows x layers / s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "ms_per_layer": ms / n, "ms_per_step_history_on_device": res["device"],
+            "copy_hidden_frac": res["device"] / ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded); history in page-locked host memory",
+            "config": dict(workload_config(case), layers=n, row_block=rb, history_rows=hist_len),
+            "history_bytes_per_layer": hist_len * kv_row,
+            "device_history_bytes": 2 * L * kv_row, "device_history_bytes_all_layers_resident": n * L * kv_row,
+            "score_workspace_bytes": rb * ((L + 3) // 4 * 4) * 4,
+            "score_workspace_bytes_unblocked": R * ((L + 3) // 4 * 4) * 4,
+            "gpu_launches": args.steps * n * ((R + rb - 1) // rb) * 4}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def to_dev(arr, dtype, dev):
     from sparse_attention_decode_scan_b200.device import to_device
     return to_device(arr, dtype, dev)
@@ -887,6 +962,9 @@ def main(argv=None):
     ap.add_argument("--route", default="own", choices=["own", "prev"],
                     help="layers: attend the latest indexer layer at or before (own) or before (prev, MLI) a layer")
     ap.add_argument("--retention", type=int, default=1, help="layers: every retention-th layer keeps an indexer")
+    ap.add_argument("--prefill-layers", action="store_true",
+                    help="the prefill workload through --layers layers, history streamed from host memory")
+    ap.add_argument("--row-block", type=int, default=0, help="prefill layers: query rows per block (0: all)")
     ap.add_argument("--blocks", type=int, default=0, metavar="N_SEL",
                     help="layers attending N_SEL KV blocks each, staged from host memory a layer ahead")
     ap.add_argument("--two-stage", type=int, default=0, metavar="N_CAND",
@@ -914,6 +992,8 @@ def main(argv=None):
                 run_two_stage(args, world, rank, local)
             elif args.blocks:
                 run_blocks(args, world, rank, local)
+            elif args.prefill_layers:
+                run_prefill_layers(args, world, rank, local)
             elif args.layers > 1:
                 run_layers(args, world, rank, local)
             else:

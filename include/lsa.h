@@ -352,6 +352,45 @@ lsa_status lsa_stage_blocks(const lsa_dims* d, const lsa_cache* c, int32_t rows,
                             lsa_stream_t stream);
 
 /*
+ * Prefill of a chunk of query rows through several layers with each layer's
+ * history streamed through two alternating device buffers (LeanSparse episode
+ * page, summary: during prefill, stream each layer's history through two GPU
+ * buffers that alternate, so the prefill does not need every layer's KV
+ * resident, nor the large temporary workspace that forces).  Layer l runs on
+ * buffer l % 2 while the copy of layer l+1's history into the other buffer
+ * proceeds on the copy stream.
+ *   caches[l]  (HOST array of n_layers) layer l's cache of ONE sequence
+ *              (batch 1, contiguous: d->block_size = 0), every layer with the
+ *              same max_len = L (the visible sequence, history and chunk) and
+ *              seq_lens; idx_keys on the device (the indexer keys stay on the
+ *              GPU); kv = the layer's history rows [0, hist_len), in
+ *              page-locked host memory (an offloaded cache) or device memory.
+ *   chunk_kv[l] device [L - hist_len, D]: the chunk's own KV rows of layer l.
+ *   rows, row_pos [rows] device: the chunk's query rows and their positions.
+ *   q_idx[l], w[l], q[l], out[l], lse[l] (lse may be NULL or hold NULL),
+ *   idx_out[l] ([rows, k], may be NULL or hold NULL): per layer, as
+ *              lsa_indexer_scores / lsa_topk / lsa_sparse_attn_decode.
+ *   row_block  rows scored, selected and attended at a time: the score
+ *              workspace is row_block x L fp32 instead of rows x L.
+ *   kv_buf[2]  device [L, D] each: the alternating history buffers.
+ *   compute, copy: two streams (the copies run on `copy`, everything else on
+ *              `compute`); events[4]: cudaEvent_t created by the caller
+ *              (timing disabled is best): buffer 0 and 1 filled, buffer 0 and 1
+ *              released.  The call enqueues and returns; `compute` holds the
+ *              last layer's work.
+ * Each layer's results equal lsa_indexer_scores -> lsa_topk -> lsa_sparse_attn_decode
+ * on its whole cache (bit for bit with row_block >= rows).
+ * Workspace: lsa_prefill_layers_workspace_size(d, rows, L, row_block).
+ */
+size_t lsa_prefill_layers_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t row_block);
+lsa_status lsa_prefill_layers(const lsa_dims* d, int32_t n_layers, const lsa_cache* caches, int64_t hist_len,
+                              const void* const* chunk_kv, int32_t rows, const int32_t* row_pos,
+                              const void* const* q_idx, const float* const* w, const void* const* q,
+                              void* const* out, float* const* lse, int32_t* const* idx_out, int32_t row_block,
+                              void* const* kv_buf, void* ws, size_t ws_bytes, lsa_stream_t compute,
+                              lsa_stream_t copy, void* const* events);
+
+/*
  * Copies the workspace status word to *status (an lsa_status value), clears it,
  * and synchronises `stream`.  Returns LSA_ERR_CUDA if a CUDA call fails.
  */

@@ -177,6 +177,31 @@ TwoStageLayout two_stage_layout(const lsa_dims* d, int32_t rows, int64_t max_len
   return L;
 }
 
+// Layer-streamed prefill (lsa_prefill_layers): the rows' sequence map (all
+// zero), one block of rows' scores and selection, and the scan / top-k /
+// attention scratch of a block.
+struct PrefillLayout {
+  size_t rowseq_off, scores_off, idx_off, inner_off, inner_bytes, total;
+  int64_t ld;
+};
+
+PrefillLayout prefill_layout(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t row_block) {
+  PrefillLayout L;
+  const int32_t rb = row_block < rows ? row_block : rows;
+  L.ld = score_ld(max_len);
+  L.rowseq_off = kStatusBytes;
+  L.scores_off = L.rowseq_off + align_up(static_cast<size_t>(rows) * 4);
+  L.idx_off = L.scores_off + align_up(static_cast<size_t>(rb) * L.ld * 4);
+  L.inner_off = L.idx_off + align_up(static_cast<size_t>(rb) * d->top_k * 4);
+  size_t inner = topk_ws_bytes(rb, max_len, d->top_k);
+  const size_t a = attn_ws(d, rb), sc = scores_ws(rb, true);
+  if (a > inner) inner = a;
+  if (sc > inner) inner = sc;
+  L.inner_bytes = align_up(inner);
+  L.total = L.inner_off + L.inner_bytes;
+  return L;
+}
+
 lsa_status ws_check(void* ws, size_t have, size_t need) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LSA_ERR_WORKSPACE;
   if (have < need) return LSA_ERR_WORKSPACE;
@@ -699,6 +724,88 @@ lsa_status lsa_stage_blocks(const lsa_dims* d, const lsa_cache* c, int32_t rows,
   return cuda_status(launch_stage_blocks(v, rows, row_seq, row_pos, kept, n_sel, block_size, row_bytes, staged_kv,
                                          staged_table, staged_idx, status_of(ws),
                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t lsa_prefill_layers_workspace_size(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t row_block) {
+  if (!valid_dims(d) || rows < 0 || max_len < 0 || row_block < 1) return 0;
+  return prefill_layout(d, rows, max_len, row_block).total;
+}
+
+lsa_status lsa_prefill_layers(const lsa_dims* d, int32_t n_layers, const lsa_cache* caches, int64_t hist_len,
+                              const void* const* chunk_kv, int32_t rows, const int32_t* row_pos,
+                              const void* const* q_idx, const float* const* w, const void* const* q,
+                              void* const* out, float* const* lse, int32_t* const* idx_out, int32_t row_block,
+                              void* const* kv_buf, void* ws, size_t ws_bytes, lsa_stream_t compute,
+                              lsa_stream_t copy, void* const* events) {
+  if (!valid_dims(d) || n_layers < 1 || !caches || rows < 0 || row_block < 1) return LSA_ERR_INVALID_ARG;
+  if (d->block_size != 0) return LSA_ERR_INVALID_ARG;  // the streamed history is one contiguous sequence
+  const int64_t L = caches[0].max_len;
+  if (hist_len < 0 || hist_len > L) return LSA_ERR_INVALID_ARG;
+  const int64_t row_bytes = static_cast<int64_t>(d->qk_dim) * (d->act_dtype == LSA_F32 ? 4 : 2);
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const lsa_cache& c = caches[l];
+    if (!valid_cache(d, &c, true, false) || c.batch != 1 || c.max_len != L || !c.kv) return LSA_ERR_INVALID_ARG;
+    if (rows > 0) {
+      if (!q_idx || !w || !q || !out || !q_idx[l] || !w[l] || !q[l] || !out[l]) return LSA_ERR_INVALID_ARG;
+      if (!aligned16(q_idx[l]) || !aligned16(q[l]) || !aligned16(out[l])) return LSA_ERR_INVALID_ARG;
+      if (hist_len < L && (!chunk_kv || !chunk_kv[l])) return LSA_ERR_INVALID_ARG;
+    }
+  }
+  if (rows > 0 && (!row_pos || !kv_buf || !kv_buf[0] || !kv_buf[1] || !aligned16(kv_buf[0]) || !aligned16(kv_buf[1]) ||
+                   !events || !events[0] || !events[1] || !events[2] || !events[3]))
+    return LSA_ERR_INVALID_ARG;
+  if (rows > 65535) return LSA_ERR_UNSUPPORTED;
+  const PrefillLayout P = prefill_layout(d, rows, L, row_block);
+  lsa_status st = ws_check(ws, ws_bytes, P.total);
+  if (st != LSA_OK) return st;
+  if (rows == 0) return LSA_OK;
+  cudaStream_t sc = reinterpret_cast<cudaStream_t>(compute), sx = reinterpret_cast<cudaStream_t>(copy);
+  cudaEvent_t ready[2] = {static_cast<cudaEvent_t>(events[0]), static_cast<cudaEvent_t>(events[1])};
+  cudaEvent_t freed[2] = {static_cast<cudaEvent_t>(events[2]), static_cast<cudaEvent_t>(events[3])};
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* row_seq = reinterpret_cast<int32_t*>(base + P.rowseq_off);
+  float* scores = reinterpret_cast<float*>(base + P.scores_off);
+  int32_t* idx = reinterpret_cast<int32_t*>(base + P.idx_off);
+  void* inner = base + P.inner_off;
+  if (cudaMemsetAsync(row_seq, 0, static_cast<size_t>(rows) * 4, sc) != cudaSuccess) return LSA_ERR_CUDA;
+  const size_t qi_row = static_cast<size_t>(d->n_idx_heads) * d->idx_dim * (d->act_dtype == LSA_F32 ? 4 : 2);
+  const size_t q_row = static_cast<size_t>(d->n_heads) * d->qk_dim * (d->act_dtype == LSA_F32 ? 4 : 2);
+  const size_t o_row = static_cast<size_t>(d->n_heads) * d->v_dim * (d->act_dtype == LSA_F32 ? 4 : 2);
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const int b = l & 1;
+    // copy side: this layer's history into buffer b once the layer two back
+    // has finished reading it, then the chunk's own rows after it
+    if (l >= 2 && cudaStreamWaitEvent(sx, freed[b], 0) != cudaSuccess) return LSA_ERR_CUDA;
+    uint8_t* buf = static_cast<uint8_t*>(kv_buf[b]);
+    if (hist_len > 0 &&
+        cudaMemcpyAsync(buf, caches[l].kv, static_cast<size_t>(hist_len * row_bytes), cudaMemcpyDefault, sx) != cudaSuccess)
+      return LSA_ERR_CUDA;
+    if (hist_len < L && cudaMemcpyAsync(buf + hist_len * row_bytes, chunk_kv[l],
+                                        static_cast<size_t>((L - hist_len) * row_bytes), cudaMemcpyDefault,
+                                        sx) != cudaSuccess)
+      return LSA_ERR_CUDA;
+    if (cudaEventRecord(ready[b], sx) != cudaSuccess) return LSA_ERR_CUDA;
+    // compute side: the layer's rows, row_block at a time, on buffer b
+    if (cudaStreamWaitEvent(sc, ready[b], 0) != cudaSuccess) return LSA_ERR_CUDA;
+    lsa_cache cl = caches[l];
+    cl.kv = buf;
+    for (int32_t r0 = 0; r0 < rows; r0 += row_block) {
+      const int32_t nr = rows - r0 < row_block ? rows - r0 : row_block;
+      st = do_scores(d, &cl, nr, row_seq, row_pos + r0, static_cast<const uint8_t*>(q_idx[l]) + r0 * qi_row,
+                     w[l] + static_cast<int64_t>(r0) * d->n_idx_heads, scores, P.ld, ws, inner, P.inner_bytes, sc);
+      if (st != LSA_OK) return st;
+      int32_t* sel = idx_out && idx_out[l] ? idx_out[l] + static_cast<int64_t>(r0) * d->top_k : idx;
+      st = do_topk(scores, P.ld, nr, nullptr, L, d->top_k, sel, ws, inner, sc);
+      if (st != LSA_OK) return st;
+      st = do_attn(d, &cl, nr, row_seq, static_cast<const uint8_t*>(q[l]) + r0 * q_row, sel,
+                   static_cast<uint8_t*>(out[l]) + r0 * o_row,
+                   lse && lse[l] ? lse[l] + static_cast<int64_t>(r0) * d->n_heads : nullptr, ws, inner,
+                   P.inner_bytes, sc);
+      if (st != LSA_OK) return st;
+    }
+    if (cudaEventRecord(freed[b], sc) != cudaSuccess) return LSA_ERR_CUDA;
+  }
+  return LSA_OK;
 }
 
 lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream) {

@@ -485,6 +485,7 @@ int cluster_capacity(int nseg, size_t smem) {
 tk::ClPlan cluster_plan(int32_t rows, int64_t n_cols) {
   for (int cap = tk::kClMaxSeg; cap >= 1; cap /= 2) {
     const tk::ClPlan p = tk::cl_plan(n_cols, cap);
+    if (p.nseg == 0) break;                 // fewer segments would exceed what a CTA stages
     if (p.nseg < cap && cap > 1) continue;  // the row is too short for this many segments
     if (static_cast<int64_t>(rows) <= cluster_capacity(p.nseg, tk::cl_smem(p.seg_len))) return p;
   }

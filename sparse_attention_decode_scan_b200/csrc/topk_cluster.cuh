@@ -34,6 +34,8 @@ struct ClHdr {
   uint32_t gt;  // selected keys above T in the segment
   uint32_t eq;  // keys equal to T in the segment
   uint32_t pad;
+  uint64_t staged;  // mbarrier: the segment's scores and the row's histogram are in shared memory
+  uint64_t pad2;
 };
 
 struct ClPlan {
@@ -41,13 +43,21 @@ struct ClPlan {
   int64_t seg_len;  // multiple of kColRound
 };
 
+constexpr int64_t kClMaxSegLen = 32768;  // positions a CTA stages in shared memory (128 KB)
+
 // Segments of a row: up to max_seg CTAs (at most kClMaxSeg), at least one
-// collect round (kColRound positions) each.
+// collect round (kColRound positions) each.  nseg = 0: the row needs more
+// segments than max_seg to keep each within kClMaxSegLen.
 __host__ __device__ inline ClPlan cl_plan(int64_t n_cols, int max_seg = kClMaxSeg) {
   ClPlan p;
   int64_t rounds = (n_cols + kColRound - 1) / kColRound;
   if (rounds < 1) rounds = 1;
   const int64_t cap = max_seg < kClMaxSeg ? (max_seg < 1 ? 1 : max_seg) : kClMaxSeg;
+  if ((rounds + cap - 1) / cap * kColRound > kClMaxSegLen) {
+    p.nseg = 0;
+    p.seg_len = 0;
+    return p;
+  }
   const int64_t ns = rounds < cap ? rounds : cap;
   const int64_t per = (rounds + ns - 1) / ns;
   p.seg_len = per * kColRound;
@@ -55,17 +65,19 @@ __host__ __device__ inline ClPlan cl_plan(int64_t n_cols, int max_seg = kClMaxSe
   return p;
 }
 
-// Shared memory of the body: header | bitmap of the segment | tie bitmap |
-// candidates | every CTA's candidate keys, gathered.  The bitmaps are padded
-// per thread (tk_pad) so the ordered walk over each thread's own words hits
-// distinct banks.
+// Shared memory of the body: header | the segment's scores | the row's
+// first-digit histogram | bitmap of the segment | tie bitmap | candidates |
+// every CTA's candidate keys, gathered.  The bitmaps are padded per thread
+// (tk_pad) so the ordered walk over each thread's own words hits distinct
+// banks.
 __host__ __device__ inline int cl_bm_words(int64_t seg_len) {
   const TkPad p = tk_pad(seg_len, kClThreads);
   return (kClThreads * p.stride + 3) / 4 * 4;
 }
 
 __host__ __device__ inline size_t cl_smem(int64_t seg_len) {
-  return sizeof(ClHdr) + 2 * static_cast<size_t>(cl_bm_words(seg_len)) * 4 + static_cast<size_t>(kClCandCap) * 8 +
+  return sizeof(ClHdr) + static_cast<size_t>(seg_len) * 4 + static_cast<size_t>(kB1) * 4 +
+         2 * static_cast<size_t>(cl_bm_words(seg_len)) * 4 + static_cast<size_t>(kClCandCap) * 8 +
          static_cast<size_t>(kClMaxSeg) * kClCandCap * 4;
 }
 
@@ -82,7 +94,9 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
   const TkPad pad = tk_pad(seg_len, NT);
   const int bm_words = cl_bm_words(seg_len);
   ClHdr* hdr = reinterpret_cast<ClHdr*>(dsm);
-  uint32_t* bm = reinterpret_cast<uint32_t*>(dsm + sizeof(ClHdr));
+  float* seg = reinterpret_cast<float*>(dsm + sizeof(ClHdr));               // [seg_len]
+  uint32_t* hsm = reinterpret_cast<uint32_t*>(seg + seg_len);               // [kB1]
+  uint32_t* bm = hsm + kB1;
   uint32_t* tb = bm + bm_words;
   uint2* cs = reinterpret_cast<uint2*>(tb + bm_words);
   uint32_t* allk = reinterpret_cast<uint32_t*>(cs + kClCandCap);  // [kClMaxSeg * kClCandCap]
@@ -103,14 +117,39 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
   const int lim = ((n + 3) & ~3) < a.ld ? ((n + 3) & ~3) : static_cast<int>(a.ld);
   for (int i = t; i < bm_words; i += NT) tb[i] = 0;
+  // The segment's scores (up to the row's length rounded to 16 bytes) and the
+  // row's histogram come in by bulk copies, all in flight at once: the collect
+  // then reads shared memory, and the L2 round trips are paid once.
+  const int s1r = (s1 + 3) & ~3;  // 16-byte granules: the copy sizes must be multiples of 16
+  const int s_hi = s1r < lim ? s1r : lim;
+  const uint32_t seg_bytes = s_hi > s0 ? static_cast<uint32_t>(s_hi - s0) * 4u : 0u;
+  bool staged_ok = true;
+  const bool staging = live;
+  if (staging) {
+    if (t == 0) {
+      tc::mbar_init(&hdr->staged, 1);
+      tc::fence_mbar_init();
+    }
+    tk_sync<NT, ID>();
+    if (t == 0) {
+      tc::mbar_arrive_expect_tx(&hdr->staged, seg_bytes + static_cast<uint32_t>(kB1) * 4u);
+      tc::bulk_load(hsm, L.hist + static_cast<int64_t>(r) * kB1, static_cast<uint32_t>(kB1) * 4u, &hdr->staged);
+      for (uint32_t off = 0; off < seg_bytes; off += 32768u) {
+        const uint32_t nb = seg_bytes - off < 32768u ? seg_bytes - off : 32768u;
+        tc::bulk_load(reinterpret_cast<uint8_t*>(seg) + off, reinterpret_cast<const uint8_t*>(row + s0) + off, nb,
+                      &hdr->staged);
+      }
+    }
+    staged_ok = tc::mbar_wait(&hdr->staged, 0, nullptr);
+    if (!staged_ok && t == 0) record_error(a.status, LSA_ERR_TIMEOUT, r, 23);
+  }
   // ---------------------------------------------------------------- collect
   uint32_t keff = 0, b1 = 0xffffffffu, rank1 = 0;
   int nc = 0, above = 0;
-  if (live) {
-    ColRound cur;
-    if (s0 < s1) tk_round_load(row, s0, lim, cur);
+  if (live && staged_ok) {
     uint32_t hv[kB1 / NT];
-    tk_load_bins<NT, kB1>(L.hist + static_cast<int64_t>(r) * kB1, t, hv);
+#pragma unroll
+    for (int i = 0; i < kB1 / NT; ++i) hv[i] = hsm[t * (kB1 / NT) + i];
     const uint32_t total = tk_find<NT, ID, kB1>(hv, static_cast<uint32_t>(a.k), S, true);
     keff = total < static_cast<uint32_t>(a.k) ? total : static_cast<uint32_t>(a.k);
     if (keff > 0) {
@@ -124,12 +163,13 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
 #pragma unroll
       for (int v = 0; v < 8; ++v) {
         const int p = p0 + v * 128;
-        key[v][0] = p < n ? order_key(cur.x[v].x) : 0u;
-        key[v][1] = p + 1 < n ? order_key(cur.x[v].y) : 0u;
-        key[v][2] = p + 2 < n ? order_key(cur.x[v].z) : 0u;
-        key[v][3] = p + 3 < n ? order_key(cur.x[v].w) : 0u;
+        const float4 x = p < s_hi ? *reinterpret_cast<const float4*>(seg + (p - s0))
+                                  : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        key[v][0] = p < n ? order_key(x.x) : 0u;
+        key[v][1] = p + 1 < n ? order_key(x.y) : 0u;
+        key[v][2] = p + 2 < n ? order_key(x.z) : 0u;
+        key[v][3] = p + 3 < n ? order_key(x.w) : 0u;
       }
-      if (base + kColRound < s1) tk_round_load(row, base + kColRound, lim, cur);
       // bitmap word of lane l: positions 32 l .. 32 l + 31 of the warp's 1024
       uint32_t bal[4] = {0u, 0u, 0u, 0u};
       int ncl = 0;
@@ -168,6 +208,7 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
       nc += tot;
     }
   }
+  if (!staged_ok) live = false;
   // words of the bitmap the rounds did not write (a segment without a selectable key)
   if (!live || keff == 0)
     for (int i = t; i < bm_words; i += NT) bm[i] = 0;
@@ -248,7 +289,7 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
       }
     } else {
       for (int p = s0 + t; p < s1 && p < n; p += NT) {
-        const uint32_t key = order_key(__ldcg(row + p));
+        const uint32_t key = order_key(seg[p - s0]);
         if ((key >> 20) != b1) continue;
         const uint32_t w = static_cast<uint32_t>(p - s0) >> 5;
         if (key > T) atomicOr(&bm[pw(w)], 1u << (p & 31));
@@ -336,6 +377,7 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
     }
   }
   tc::cluster_wait();  // ---- the others have read this CTA's shared memory
+  if (t == 0 && staging && staged_ok) tc::mbar_inval(&hdr->staged);
 }
 
 }  // namespace tk

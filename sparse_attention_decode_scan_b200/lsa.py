@@ -104,7 +104,11 @@ def lib() -> ctypes.CDLL:
     L.lsa_block_select_workspace_size.restype = sz
     L.lsa_block_select.argtypes = [vp, i64, i32, vp, i64, i32, i32, vp, vp, sz, vp]
     L.lsa_stage_blocks.argtypes = [D, C, i32, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]
-    names = ["lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode", "lsa_decode_step",
+    L.lsa_prefill_layers_workspace_size.argtypes = [D, i32, i64, i32]
+    L.lsa_prefill_layers_workspace_size.restype = sz
+    L.lsa_prefill_layers.argtypes = [D, i32, C, i64, PV, i32, vp, PV, PV, PV, PV, PV, PV, i32, PV, vp, sz, vp, vp, PV]
+    names = ["lsa_prefill_layers", "lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode",
+             "lsa_decode_step",
              "lsa_decode_step_profiled", "lsa_decode_layers", "lsa_read_device_status", "lsa_candidate_scores",
              "lsa_two_stage_select", "lsa_block_select", "lsa_stage_blocks"]
     if path == TEST_LIB_PATH:
@@ -294,6 +298,35 @@ def staged_cache(staged_kv, staged_table, staged_lens, n_sel: int, block_size: i
     c.seq_lens = staged_lens.data_ptr()
     c.batch = int(staged_table.shape[0])
     return c
+
+
+def prefill_layers_workspace_size(dims: Dims, rows: int, max_len: int, row_block: int) -> int:
+    return int(lib().lsa_prefill_layers_workspace_size(ctypes.byref(dims), rows, max_len, row_block))
+
+
+def prefill_layers(dims: Dims, caches, hist_len: int, chunk_kv, row_pos, q_idx, w, q, out, lse, kv_buf, ws,
+                   row_block: int, events, idx_out=None, stream=None, copy_stream=None, raise_on_error=True) -> int:
+    """lsa_prefill_layers: per-layer lists of Cache structs (kv = the history, host or device) and tensors;
+    kv_buf: two device buffers; events: four torch.cuda.Event (created here if needed)."""
+    import torch
+    n = len(caches)
+    arr = (Cache * n)(*caches)
+
+    def ptrs(ts):
+        return (ctypes.c_void_p * n)(*[_ptr(t) for t in ts]) if ts is not None else None
+
+    for e in events:  # torch creates the CUDA event at its first record
+        if e.cuda_event == 0:
+            e.record()
+    ev = (ctypes.c_void_p * 4)(*[int(e.cuda_event) for e in events])
+    bufs = (ctypes.c_void_p * 2)(*[_ptr(t) for t in kv_buf])
+    cs = copy_stream if copy_stream is not None else torch.cuda.Stream()
+    rows = int(row_pos.shape[0])
+    return _check(lib().lsa_prefill_layers(ctypes.byref(dims), n, arr, int(hist_len), ptrs(chunk_kv), rows,
+                                           _ptr(row_pos), ptrs(q_idx), ptrs(w), ptrs(q), ptrs(out), ptrs(lse),
+                                           ptrs(idx_out), int(row_block), bufs, _ptr(ws),
+                                           ws.numel() if ws is not None else 0, _stream(stream), _stream(cs), ev),
+                  "lsa_prefill_layers", raise_on_error)
 
 
 def read_device_status(ws, stream=None) -> int:
