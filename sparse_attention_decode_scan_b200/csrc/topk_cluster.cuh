@@ -28,22 +28,21 @@ constexpr int kClThreads = kCollectThreads;        // the round shape of tk_roun
 constexpr int kClMaxSeg = 8;                       // CTAs per cluster (portable cluster size)
 constexpr int64_t kClMaxCols = int64_t(1) << 18;   // longer rows take the collect + select bodies
 constexpr int kClCandCap = 1024;                   // threshold-bin keys a CTA keeps
+constexpr int64_t kClMaxSegLen = 32768;            // positions a CTA stages in shared memory (128 KB)
 
 struct ClHdr {
   uint32_t nc;  // keys of the threshold bin in the segment (> kClCandCap: the list overflowed)
   uint32_t gt;  // selected keys above T in the segment
   uint32_t eq;  // keys equal to T in the segment
   uint32_t pad;
-  uint64_t staged;  // mbarrier: the segment's scores and the row's histogram are in shared memory
-  uint64_t pad2;
 };
+// the segment's scores follow the header: 16-byte loads and bulk copies need it aligned
+static_assert(sizeof(ClHdr) % 16 == 0, "header size");
 
 struct ClPlan {
   int nseg;
   int64_t seg_len;  // multiple of kColRound
 };
-
-constexpr int64_t kClMaxSegLen = 32768;  // positions a CTA stages in shared memory (128 KB)
 
 // Segments of a row: up to max_seg CTAs (at most kClMaxSeg), at least one
 // collect round (kColRound positions) each.  nseg = 0: the row needs more
@@ -89,7 +88,7 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
                                bool live) {
   constexpr int NT = kClThreads;
   const int t = threadIdx.x;
-  const int lane = t & 31, warp = t >> 5;
+  const int lane = t & 31;
   const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
   const TkPad pad = tk_pad(seg_len, NT);
   const int bm_words = cl_bm_words(seg_len);
@@ -117,31 +116,46 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
   const int lim = ((n + 3) & ~3) < a.ld ? ((n + 3) & ~3) : static_cast<int>(a.ld);
   for (int i = t; i < bm_words; i += NT) tb[i] = 0;
-  // The segment's scores (up to the row's length rounded to 16 bytes) and the
-  // row's histogram come in by bulk copies, all in flight at once: the collect
-  // then reads shared memory, and the L2 round trips are paid once.
-  const int s1r = (s1 + 3) & ~3;  // 16-byte granules: the copy sizes must be multiples of 16
+  // The row's histogram and the segment's scores (up to the row's length
+  // rounded to 16 bytes) come into shared memory by 16-byte cp.async copies of
+  // every thread, consecutive threads on consecutive bytes: one commit group
+  // for the histogram, one per collect round, all in flight at once, so each
+  // round starts as soon as its own group has landed.  (Large bulk copies were
+  // measured to deliver far fewer bytes per microsecond here.)
+  const int s1r = (s1 + 3) & ~3;  // whole 16-byte groups
   const int s_hi = s1r < lim ? s1r : lim;
-  const uint32_t seg_bytes = s_hi > s0 ? static_cast<uint32_t>(s_hi - s0) * 4u : 0u;
+  const int n_rounds = s1 > s0 ? (s1 - s0 + kColRound - 1) / kColRound : 0;
   bool staged_ok = true;
   const bool staging = live;
   if (staging) {
-    if (t == 0) {
-      tc::mbar_init(&hdr->staged, 1);
-      tc::fence_mbar_init();
-    }
-    tk_sync<NT, ID>();
-    if (t == 0) {
-      tc::mbar_arrive_expect_tx(&hdr->staged, seg_bytes + static_cast<uint32_t>(kB1) * 4u);
-      tc::bulk_load(hsm, L.hist + static_cast<int64_t>(r) * kB1, static_cast<uint32_t>(kB1) * 4u, &hdr->staged);
-      for (uint32_t off = 0; off < seg_bytes; off += 32768u) {
-        const uint32_t nb = seg_bytes - off < 32768u ? seg_bytes - off : 32768u;
-        tc::bulk_load(reinterpret_cast<uint8_t*>(seg) + off, reinterpret_cast<const uint8_t*>(row + s0) + off, nb,
-                      &hdr->staged);
+    const uint32_t* hsrc = L.hist + static_cast<int64_t>(r) * kB1;
+#pragma unroll
+    for (int k = 0; k < kB1 / 4 / NT; ++k)
+      tc::cp_async16_zfill(hsm + 4 * (k * NT + t), hsrc + 4 * (k * NT + t), 16u);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int i = 0; i < n_rounds; ++i) {
+#pragma unroll
+      for (int k = 0; k < kColRound / 4 / NT; ++k) {
+        const int p = s0 + i * kColRound + 4 * (k * NT + t);
+        // groups past the staged range are zero-filled (read nothing)
+        tc::cp_async16_zfill(seg + (p - s0), row + (p < s_hi ? p : s0), p < s_hi ? 16u : 0u);
       }
+      asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    staged_ok = tc::mbar_wait(&hdr->staged, 0, nullptr);
-    if (!staged_ok && t == 0) record_error(a.status, LSA_ERR_TIMEOUT, r, 23);
+  }
+  // waits until at most `pending` of this thread's newest groups are in flight
+  auto wait_groups = [&](int pending) {
+    switch (pending) {
+      case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+      case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+      case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+      case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+      default: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    }
+  };
+  if (staging) {
+    wait_groups(n_rounds);  // the histogram
+    tk_sync<NT, ID>();      // every thread's part of it
   }
   // ---------------------------------------------------------------- collect
   uint32_t keff = 0, b1 = 0xffffffffu, rank1 = 0;
@@ -157,53 +171,42 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
       rank1 = S.s_rank;
     }
 #pragma unroll 1
-    for (int base = s0; keff > 0 && base < s1; base += kColRound) {
-      const int p0 = base + warp * 1024 + lane * 4;
-      uint32_t key[8][4];
+    for (int rd = 0; keff > 0 && rd < n_rounds; ++rd) {
+      wait_groups(n_rounds - 1 - rd);  // this round's scores (later rounds may still be in flight)
+      tk_sync<NT, ID>();                // every thread's part of them
+      // thread t builds bitmap word t of the round (positions 32 t .. 32 t + 31)
+      // from its own 16-byte groups, read in a rotated order so that the
+      // warp's reads spread over the banks; every bit is independent work
+      const int base = s0 + rd * kColRound;
+      const int q = base + 32 * t;
+      const float4* g4 = reinterpret_cast<const float4*>(seg + (q - s0));
+      uint32_t above_w = 0u, bin_w = 0u;
 #pragma unroll
       for (int v = 0; v < 8; ++v) {
-        const int p = p0 + v * 128;
-        const float4 x = p < s_hi ? *reinterpret_cast<const float4*>(seg + (p - s0))
-                                  : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-        key[v][0] = p < n ? order_key(x.x) : 0u;
-        key[v][1] = p + 1 < n ? order_key(x.y) : 0u;
-        key[v][2] = p + 2 < n ? order_key(x.z) : 0u;
-        key[v][3] = p + 3 < n ? order_key(x.w) : 0u;
-      }
-      // bitmap word of lane l: positions 32 l .. 32 l + 31 of the warp's 1024
-      uint32_t bal[4] = {0u, 0u, 0u, 0u};
-      int ncl = 0;
+        const int vv = (v + lane) & 7;
+        const int p = q + 4 * vv;
+        const float4 x = p < s_hi ? g4[vv] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t k = key[v][c];
-          const uint32_t bb = __ballot_sync(0xffffffffu, k != 0u && (k >> 20) > b1);
-          bal[c] = (lane >> 2) == v ? bb : bal[c];
-          ncl += (k != 0u && (k >> 20) == b1) ? 1 : 0;
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t k = p + e < n ? order_key(xs[e]) : 0u;
+          const uint32_t hi = k >> 20;
+          above_w |= static_cast<uint32_t>(k != 0u && hi > b1) << (4 * vv + e);
+          bin_w |= static_cast<uint32_t>(k != 0u && hi == b1) << (4 * vv + e);
         }
       }
-      const int sh = 8 * (lane & 3);
-      const uint32_t word = spread8(bal[0] >> sh) | (spread8(bal[1] >> sh) << 1) | (spread8(bal[2] >> sh) << 2) |
-                            (spread8(bal[3] >> sh) << 3);
-      const int wi = (base - s0) / kWordElems + warp * 32 + lane;
-      if (wi < nw_seg) bm[pw(static_cast<uint32_t>(wi))] = word;
-      above += __popc(word);
+      const int wi = rd * (kColRound / kWordElems) + t;
+      if (wi < nw_seg) bm[pw(static_cast<uint32_t>(wi))] = above_w;
+      above += __popc(above_w);
+      const int ncl = __popc(bin_w);
       int tot;
       const int off = tk_excl_scan<NT, ID>(ncl, S.warp_sums, &tot);
       int o = nc + off;
-      if (ncl) {
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t k = key[v][c];
-            if (k != 0u && (k >> 20) == b1) {
-              if (o < kClCandCap) cs[o] = make_uint2(k, static_cast<uint32_t>(p0 + v * 128 + c));
-              ++o;
-            }
-          }
-        }
+      while (bin_w) {  // this thread's candidates, in position order
+        const int b = __ffs(bin_w) - 1;
+        bin_w &= bin_w - 1;
+        if (o < kClCandCap) cs[o] = make_uint2(order_key(seg[q - s0 + b]), static_cast<uint32_t>(q + b));
+        ++o;
       }
       nc += tot;
     }
@@ -377,7 +380,7 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
     }
   }
   tc::cluster_wait();  // ---- the others have read this CTA's shared memory
-  if (t == 0 && staging && staged_ok) tc::mbar_inval(&hdr->staged);
+  if (staging) asm volatile("cp.async.wait_all;" ::: "memory");  // nothing in flight when the CTA leaves
 }
 
 }  // namespace tk
