@@ -21,9 +21,14 @@
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0  TMA producer: 64-row boxes of the key cache (block-table gather)
-//   warp 1  MMA issuer (one thread) + TMEM owner
+//   warp 1  MMA issuer of the even tiles (one thread) + TMEM owner
 //   warp 2  query staging: query rows -> swizzled smem operand, weights
 //   warps 3-6 epilogue: TMEM -> registers, ReLU-weighted sum, score stores
+//            (warps 3-10 with two epilogue groups)
+//   last    MMA issuer of the odd tiles (one thread)
+// Two issuers, one per accumulator: an MMA of this size occupies the tensor
+// pipe for about as long as its issuer spends on the waits and bookkeeping of
+// a tile, so with one issuer the pipe idled half of the time.
 // Every wait is bounded; a timeout records LSA_ERR_TIMEOUT and unwinds.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -43,11 +48,14 @@ constexpr int kBoxRows = 64;     // rows per TMA box (one 64-token page or half 
 constexpr int kBoxX = 32;        // 4-byte TMA elements per 128-byte K block
 constexpr int kScaleBox = 68;    // FP8 scales per box load: 64 + up to 3 for the 16-byte aligned start
 constexpr int kScaleSlot = 96;   // floats per scale slot: a TMA destination starts on a 128-byte boundary
-constexpr int kThreads = 224;    // 7 warps (one epilogue group)
+constexpr int kThreads = 256;    // 8 warps (one epilogue group)
 // Threads of a scan CTA with EG epilogue groups of 4 warps (warps 3.., the
-// groups taking alternate tiles, i.e. one accumulator buffer each).
+// groups taking alternate tiles, i.e. one accumulator buffer each), the
+// second MMA issuer's warp last.
 template <int EG>
 constexpr int scan_threads() { return kThreads + (EG - 1) * 128; }
+template <int EG>
+constexpr int warp_mma2() { return 3 + 4 * EG; }
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpQ = 2, kWarpEpi = 3;
 constexpr int kSmemLimit = 232448;
 constexpr int kBarrierId = 1;    // named barrier of the scan's threads (a fused block holds more threads)
@@ -583,13 +591,13 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     }
     for (int s = 0; s < C::kNQ; ++s) {
       tc::mbar_init(&qfull[s], 1);
-      tc::mbar_init(&qempty[s], 1 + 4 * EG);  // MMA commit + every epilogue warp
+      tc::mbar_init(&qempty[s], 2 + 4 * EG);  // both MMA issuers' commits + every epilogue warp
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&tfull[s], 1);
       tc::mbar_init(&tempty[s], 4);
     }
-    tc::mbar_init(done, 1);
+    tc::mbar_init(done, 2);  // both MMA issuers
     tc::mbar_init(ebar, 4 * EG);
     *abort_flag = 0;
     tc::fence_mbar_init();
@@ -725,41 +733,63 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
           tc::mbar_wait(&full[i % C::kNS], static_cast<uint32_t>((i / C::kNS) & 1), nullptr);
       }
     }
-  } else if (warp == kWarpMma) {
+  } else if (warp == kWarpMma || warp == warp_mma2<EG>()) {
+    // issuer `who` takes the tiles it with it % 2 == who into accumulator who
+    const int who = warp == kWarpMma ? 0 : 1;
     if (lane == 0 && plan.n_items > 0) {
       Walker<QB> W;
       W.start(a, plan.r_first, plan.j_first);
       int gi = -1;
       int qi = 0;
+      // An issuer shares its SM sub-partition with epilogue warps, so its
+      // per-tile work is kept small: the stage and its phase advance
+      // incrementally (no 64-bit
+      // division per tile), and a tile's descriptors are the first stage's
+      // and query buffer's plus constant offsets in the start-address field
+      // (shared-memory addresses stay below 256 KB: adding never carries out
+      // of that 14-bit field).
+      int s = 0;
+      uint32_t sph = 0;
+      uint32_t aph = 0;  // phase of this issuer's accumulator
+      const uint64_t a_desc0 = tc::desc_sw128(tc::smem_u32(stages));
+      const uint64_t b_desc0 = tc::desc_sw128(tc::smem_u32(qbufs));
       for (int64_t it = 0; it < plan.n_items; ++it) {
         if (it == 0 || W.j == 0) {
           ++gi;
           qi = gi % C::kNQ;
           if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) goto mma_fail;
         }
-        {
-          const int s = static_cast<int>(it % C::kNS);
-          if (!tc::mbar_wait(&full[s], static_cast<uint32_t>((it / C::kNS) & 1), abort_flag)) goto mma_fail;
+        if (static_cast<int>(it & 1) == who) {
+          if (!tc::mbar_wait(&full[s], sph, abort_flag)) goto mma_fail;
           // gathered rows were written by cp.async (generic proxy); the MMA reads them through the async proxy
           if (GATHER) tc::fence_proxy_async_smem();
-          const int acc = static_cast<int>(it & 1);
-          if (!tc::mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag)) goto mma_fail;
+          const int acc = who;
+          if (!tc::mbar_wait(&tempty[acc], aph ^ 1u, abort_flag)) goto mma_fail;
+          aph ^= 1u;
           tc::tc_fence_after();
           const uint32_t d = tmem_base + acc * C::kAccCols;
-          const uint32_t a_base = tc::smem_u32(stages + s * C::kTileBytes);
-          const uint32_t b_base = tc::smem_u32(qbufs + qi * C::kQBytes);
+          const uint64_t ad0 = a_desc0 + static_cast<uint64_t>((s * C::kTileBytes) >> 4);
+          const uint64_t bd0 = b_desc0 + static_cast<uint64_t>((qi * C::kQBytes) >> 4);
 #pragma unroll
           for (int kb = 0; kb < C::kKBlocks; ++kb) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const uint64_t ad_ = tc::desc_sw128(a_base + kb * C::kKBlockBytes + k * 32);
-              const uint64_t bd_ = tc::desc_sw128(b_base + kb * C::kQKBlockBytes + k * 32);
+              const uint64_t ad_ = ad0 + static_cast<uint64_t>((kb * C::kKBlockBytes + k * 32) >> 4);
+              const uint64_t bd_ = bd0 + static_cast<uint64_t>((kb * C::kQKBlockBytes + k * 32) >> 4);
               if (C::kFp8) tc::mma_f8(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
               else tc::mma_f16(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
             }
           }
           tc::mma_commit(&empty[s]);
           tc::mma_commit(&tfull[acc]);
+        }
+        {
+          if (++s == C::kNS) {
+            s = 0;
+            sph ^= 1u;
+          }
+          // both issuers release the group's query buffer after its last tile
+          // (a commit covers every MMA its thread issued before it)
           const int jn = W.j + 1;
           if (it + 1 == plan.n_items || jn >= W.g.tiles) tc::mma_commit(&qempty[qi]);
           W.next(a);
@@ -771,10 +801,10 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
         break;
       }
       tc::mma_commit(done);
-      tc::mbar_wait(done, 0, nullptr);
+      tc::mbar_wait(done, 0, nullptr);  // both issuers' MMAs complete
       // The releases of the last stages and query buffer arrive asynchronously
       // too; they must land before the barriers are invalidated.
-      if (!*abort_flag) {
+      if (who == 0 && !*abort_flag) {
         const int64_t n = plan.n_items;
         for (int64_t i = n > C::kNS ? n - C::kNS : 0; i < n; ++i)
           tc::mbar_wait(&empty[i % C::kNS], static_cast<uint32_t>((i / C::kNS) & 1), abort_flag);
@@ -808,7 +838,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
         W.next(a);
       }
     }
-  } else {
+  } else if (warp < kWarpEpi + 4 * EG) {
     // epilogue: warp % 4 selects the TMEM lane quarter = token rows of the
     // tile; group eg (warps 3 + 4 eg ..) takes the tiles it with it % EG == eg
     const int quarter = warp & 3;
@@ -877,6 +907,8 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       int gi = -1, qi = 0;
       int hist_row = -1;
       int64_t vis_r[QB];
+      int stg = 0;        // stage of item it
+      uint32_t sph = 0;   // and its phase
       for (int64_t it = 0; it < plan.n_items; ++it) {
         if (it == 0 || W.j == 0) {
           ++gi;
@@ -923,8 +955,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
           int32_t mrow = 0;  // contiguous bf16: every visible position has a key row
           float kscale = 1.f;
           if (stage_meta) {
-            const int stg = static_cast<int>(it % C::kNS);
-            if (!tc::mbar_wait(&full[stg], static_cast<uint32_t>((it / C::kNS) & 1), abort_flag)) {
+            if (!tc::mbar_wait(&full[stg], sph, abort_flag)) {
               if (lane == 0) {
                 record_error(a.status, LSA_ERR_TIMEOUT, 0, 8);
                 *abort_flag = 1;
@@ -1003,6 +1034,10 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
         if (last) {
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&qempty[qi]);
+        }
+        if (++stg == C::kNS) {
+          stg = 0;
+          sph ^= 1u;
         }
         W.next(a);
       }
