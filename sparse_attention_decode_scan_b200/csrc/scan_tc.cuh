@@ -17,7 +17,9 @@
 // each key tile 4 times.  FP8 keys go straight to kind::f8f6f4 MMAs: the bf16
 // query is split into two e4m3 terms (hi + lo, per-head power-of-two scale
 // folded into w; exact for entries within 2^10 of the head's largest, see
-// stage_query_fp8), so N doubles and no key conversion is needed.
+// stage_query_fp8), so no key conversion is needed: the decode accumulates
+// both terms into one column per head (twice the K-steps), the prefill keeps
+// them as separate columns (twice the N).
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0  TMA producer: 64-row boxes of the key cache (block-table gather)
@@ -68,7 +70,7 @@ __device__ __forceinline__ void scan_sync() {
 template <int KDT, int QB, bool GATHER = false>
 struct Cfg {
   static constexpr bool kFp8 = KDT == LSA_FP8_E4M3;
-  static constexpr int kN = (kFp8 ? 2 * kHeads : kHeads) * QB;    // MMA N (columns per accumulator)
+  static constexpr int kN = (kFp8 ? 2 * kHeads : kHeads) * QB;    // query operand rows
   static constexpr int kKBlocks = kFp8 ? 1 : 2;                    // 128-byte K blocks per row
   static constexpr int kKBlockBytes = kTile * 128;                 // A: 128 rows x 128 B
   static constexpr int kTileBytes = kKBlocks * kKBlockBytes;
@@ -88,12 +90,22 @@ struct Cfg {
                                 1024 /*align*/;
   static constexpr int kNSmax = (kSmemLimit - kFixed) / (kTileBytes + kMetaBytes);
   static constexpr int kNS = kNSmax > 12 ? 12 : kNSmax;            // key stages
-  static constexpr int kAccCols = kN;
-  static constexpr int kTmemCols = 2 * kN <= 32 ? 32 : 2 * kN <= 64 ? 64 : 2 * kN <= 128 ? 128
-                                   : 2 * kN <= 256 ? 256 : 512;
+  // FP8 decode: the query's hi and lo terms (rows 0-63 and 64-127 of the
+  // query operand) accumulate into the same 64 columns, one per head, as
+  // K-steps 5-8 over the same key tile: the epilogue reads half the columns.
+  static constexpr bool kCat = kFp8 && QB == 1;
+  static constexpr int kNmma = kCat ? kHeads : kN;                 // MMA N
+  static constexpr int kAccCols = kNmma;
+  // Accumulators in TMEM, used round robin: an accumulator's turn spans its
+  // MMAs, the commit's arrival, the epilogue's reads and the release back to
+  // the issuer, so four (where they fit) keep the MMAs of a tile from waiting
+  // for the epilogue of the tile two before it.
+  static constexpr int kAcc = 4 * kAccCols <= 512 ? 4 : 2;
+  static constexpr int kTmemCols = kAcc * kAccCols <= 32 ? 32 : kAcc * kAccCols <= 64 ? 64
+                                   : kAcc * kAccCols <= 128 ? 128 : kAcc * kAccCols <= 256 ? 256 : 512;
   static constexpr int kSmemBytes = kNS * (kTileBytes + kMetaBytes) + kFixed;
   static constexpr uint32_t kIdesc = tc::idesc(kFp8 ? tc::kFmtE4M3 : tc::kFmtBF16,
-                                               kFp8 ? tc::kFmtE4M3 : tc::kFmtBF16, kTile, kN);
+                                               kFp8 ? tc::kFmtE4M3 : tc::kFmtBF16, kTile, kNmma);
   static_assert(kNS >= 3, "too few key stages");
   static_assert(2 * kN <= 512, "accumulators exceed TMEM");
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
@@ -568,8 +580,8 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   uint64_t* qfull = empty + C::kNS;
   uint64_t* qempty = qfull + C::kNQ;
   uint64_t* tfull = qempty + C::kNQ;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* done = tempty + 2;
+  uint64_t* tempty = tfull + C::kAcc;
+  uint64_t* done = tempty + C::kAcc;
   uint64_t* ebar = done + 1;  // epilogue warps' rendezvous around histogram flushes
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ebar + 1);
   int* sfound = const_cast<int*>(abort_flag) + 1;                       // 2 ints
@@ -593,7 +605,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       tc::mbar_init(&qfull[s], 1);
       tc::mbar_init(&qempty[s], 2 + 4 * EG);  // both MMA issuers' commits + every epilogue warp
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < C::kAcc; ++s) {
       tc::mbar_init(&tfull[s], 1);
       tc::mbar_init(&tempty[s], 4);
     }
@@ -734,7 +746,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       }
     }
   } else if (warp == kWarpMma || warp == warp_mma2<EG>()) {
-    // issuer `who` takes the tiles it with it % 2 == who into accumulator who
+    // issuer `who` takes the tiles it with it % 2 == who, into accumulator it % kAcc
     const int who = warp == kWarpMma ? 0 : 1;
     if (lane == 0 && plan.n_items > 0) {
       Walker<QB> W;
@@ -750,7 +762,6 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       // of that 14-bit field).
       int s = 0;
       uint32_t sph = 0;
-      uint32_t aph = 0;  // phase of this issuer's accumulator
       const uint64_t a_desc0 = tc::desc_sw128(tc::smem_u32(stages));
       const uint64_t b_desc0 = tc::desc_sw128(tc::smem_u32(qbufs));
       for (int64_t it = 0; it < plan.n_items; ++it) {
@@ -763,21 +774,33 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
           if (!tc::mbar_wait(&full[s], sph, abort_flag)) goto mma_fail;
           // gathered rows were written by cp.async (generic proxy); the MMA reads them through the async proxy
           if (GATHER) tc::fence_proxy_async_smem();
-          const int acc = who;
-          if (!tc::mbar_wait(&tempty[acc], aph ^ 1u, abort_flag)) goto mma_fail;
-          aph ^= 1u;
+          const int acc = static_cast<int>(it % C::kAcc);
+          if (!tc::mbar_wait(&tempty[acc], static_cast<uint32_t>(((it / C::kAcc) & 1) ^ 1), abort_flag)) goto mma_fail;
           tc::tc_fence_after();
           const uint32_t d = tmem_base + acc * C::kAccCols;
           const uint64_t ad0 = a_desc0 + static_cast<uint64_t>((s * C::kTileBytes) >> 4);
           const uint64_t bd0 = b_desc0 + static_cast<uint64_t>((qi * C::kQBytes) >> 4);
+          if (C::kCat) {
+            // D = K q_hi + K q_lo: the query operand's rows 64-127 start 8 KB in
 #pragma unroll
-          for (int kb = 0; kb < C::kKBlocks; ++kb) {
+            for (int part = 0; part < 2; ++part) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t ad_ = ad0 + static_cast<uint64_t>((kb * C::kKBlockBytes + k * 32) >> 4);
-              const uint64_t bd_ = bd0 + static_cast<uint64_t>((kb * C::kQKBlockBytes + k * 32) >> 4);
-              if (C::kFp8) tc::mma_f8(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
-              else tc::mma_f16(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t ad_ = ad0 + static_cast<uint64_t>((k * 32) >> 4);
+                const uint64_t bd_ = bd0 + static_cast<uint64_t>((part * kHeads * 128 + k * 32) >> 4);
+                tc::mma_f8(d, ad_, bd_, C::kIdesc, (part | k) != 0);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int kb = 0; kb < C::kKBlocks; ++kb) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t ad_ = ad0 + static_cast<uint64_t>((kb * C::kKBlockBytes + k * 32) >> 4);
+                const uint64_t bd_ = bd0 + static_cast<uint64_t>((kb * C::kQKBlockBytes + k * 32) >> 4);
+                if (C::kFp8) tc::mma_f8(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
+                else tc::mma_f16(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
+              }
             }
           }
           tc::mma_commit(&empty[s]);
@@ -940,8 +963,8 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
         // every query buffer: the weights are read by either)
         const bool mine = EG == 1 || static_cast<int>(it % EG) == eg;
         if (mine) {
-          const int acc = static_cast<int>(it & 1);
-          if (!tc::mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1), abort_flag)) {
+          const int acc = static_cast<int>(it % C::kAcc);
+          if (!tc::mbar_wait(&tfull[acc], static_cast<uint32_t>((it / C::kAcc) & 1), abort_flag)) {
             if (lane == 0) {
               record_error(a.status, LSA_ERR_TIMEOUT, 0, 5);
               *abort_flag = 1;
@@ -985,10 +1008,11 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   #pragma unroll
             for (int c = 0; c < 2; ++c) {
               float v[32];
-              const uint32_t col = acc * C::kAccCols + (C::kFp8 ? qq * 2 * kHeads : qq * kHeads) + c * 32;
+              const uint32_t col =
+                  acc * C::kAccCols + (C::kFp8 && !C::kCat ? qq * 2 * kHeads : qq * kHeads) + c * 32;
               tc::tmem_ld32(tmem_base + lane_base + col, v);
               const float4* w4 = reinterpret_cast<const float4*>(wb + qq * kHeads + c * 32);
-              if (C::kFp8) {
+              if (C::kFp8 && !C::kCat) {
                 float u[32];
                 tc::tmem_ld32(tmem_base + lane_base + col + kHeads, u);
                 tc::tmem_wait_ld();
