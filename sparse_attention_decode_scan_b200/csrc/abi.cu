@@ -464,13 +464,16 @@ static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const 
   // only makes the row's bitmap exact and stores per-segment offsets; each
   // attention CTA compacts its own entries from the segments holding them
   // (and writes them to idx only if the caller asked for the selection).
-  // It pays for long rows (the full select walks the whole row's bitmap in one
-  // CTA: about 27 us at 512K positions, against a few microseconds of
-  // compaction per attention CTA); for rows up to about 128K the full select
-  // is as fast or faster (measured at 32K and 128K).
+  // It pays for long rows the one-cluster-per-row top-k cannot take (the
+  // full select walks the whole row's bitmap in one CTA: about 27 us at 512K
+  // positions, against a few microseconds of compaction per attention CTA);
+  // for rows up to about 128K the full select is as fast or faster (measured
+  // at 32K and 128K), and rows whose clusters fit take the cluster top-k.
   AttnArgs split;
   bool split_sel = false;
-  if (handoff && !force_simt() && c->max_len >= split_select_min_cols() && attn_tc_split_fits(B, d->top_k) &&
+  const bool cluster = allow_cluster_topk() && !force_simt() && topk_cluster_planned(B, c->max_len);
+  if (handoff && !cluster && !force_simt() && c->max_len >= split_select_min_cols() &&
+      attn_tc_split_fits(B, d->top_k) &&
       attn_tc_supported(attn_args(d, c, B, nullptr, q, idx, out, lse, ws, inner, inner_bytes)) &&
       topk_rows_plan(B, c->max_len, &split.tk_nseg, &split.tk_seg_len)) {
     split_sel = true;

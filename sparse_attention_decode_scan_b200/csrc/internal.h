@@ -129,9 +129,11 @@ bool topk_rows_plan(int32_t rows, int64_t n_cols, int* nseg, int64_t* seg_len);
 // histogram then sits at the start of the top-k workspace, followed by the
 // list counters; topk_hist_zero_bytes of them must be zero before the scan.
 bool topk_v2_ok(int64_t n_cols);
-// Rows this short take the one-cluster-per-row top-k (unless a decode step's
-// split select applies).
+// Rows this short may take the one-cluster-per-row top-k.
 bool topk_cluster_ok(int64_t n_cols);
+// True if these rows take the one-cluster-per-row top-k (their clusters fit
+// on the device at once); a decode step then skips the split select.
+bool topk_cluster_planned(int32_t rows, int64_t n_cols);
 size_t topk_hist_zero_bytes(int32_t rows);
 // true if the scan can accumulate the top-k histogram itself
 bool scores_tc_fused_hist_ok(const ScoresArgs& a);

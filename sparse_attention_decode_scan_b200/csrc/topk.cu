@@ -408,7 +408,9 @@ __global__ void __launch_bounds__(tk::kCollectThreads, 2) k_tk_rows(TopkArgs a, 
 
 // One row per thread-block cluster (rows up to tk::kClMaxCols positions): CTA
 // blockIdx.x of the cluster collects segment blockIdx.x of row blockIdx.y and
-// the cluster selects the row together (topk_cluster.cuh).
+// the cluster selects the row together (topk_cluster.cuh).  MAXSEG: the body
+// for clusters of up to 8 CTAs, or of 9 to 16.
+template <int MAXSEG>
 __global__ void __launch_bounds__(tk::kClThreads, 2) k_tk_cluster(TopkArgs a, int64_t seg_len, int nseg) {
   extern __shared__ __align__(16) uint8_t csm[];
   __shared__ tk::TkScratch S;
@@ -439,7 +441,23 @@ __global__ void __launch_bounds__(tk::kClThreads, 2) k_tk_cluster(TopkArgs a, in
   __syncthreads();
   tc::griddep_launch_dependents();
   // every CTA of the cluster reaches the cluster barriers, live or not
-  tk::tk_cluster_row<2>(a, r, static_cast<int>(tc::cluster_ctarank()), nseg, seg_len, csm, S, s_live != 0);
+  tk::tk_cluster_row<2, MAXSEG>(a, r, static_cast<int>(tc::cluster_ctarank()), nseg, seg_len, csm, S, s_live != 0);
+}
+
+// The cluster kernel for clusters of nseg CTAs, its dynamic shared memory
+// raised to `smem` and, above 8 CTAs, non-portable cluster sizes allowed.
+using ClusterKernel = void (*)(TopkArgs, int64_t, int);
+cudaError_t cluster_kernel(int nseg, size_t smem, ClusterKernel* out) {
+  const bool big = tk::cl_maxseg(nseg) > tk::kClPortableSeg;
+  ClusterKernel fn = big ? k_tk_cluster<tk::kClMaxSeg> : k_tk_cluster<tk::kClPortableSeg>;
+  cudaError_t e = ensure_dyn_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  if (big) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  *out = fn;
+  return cudaSuccess;
 }
 
 // Clusters of `nseg` k_tk_cluster CTAs (with `smem` bytes each) the current
@@ -457,7 +475,8 @@ int cluster_capacity(int nseg, size_t smem) {
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   int n = 0;
-  if (ensure_dyn_smem(k_tk_cluster, smem) == cudaSuccess) {
+  ClusterKernel fn = nullptr;
+  if (cluster_kernel(nseg, smem, &fn) == cudaSuccess) {
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(nseg), 1, 1);
@@ -470,7 +489,7 @@ int cluster_capacity(int nseg, size_t smem) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, k_tk_cluster, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) n = 0;
   }
   (void)cudaGetLastError();
   cache[key] = n;
@@ -478,8 +497,8 @@ int cluster_capacity(int nseg, size_t smem) {
 }
 
 // The cluster plan of the one-cluster-per-row top-k for these sizes: the
-// largest cluster (8, 4, 2 CTAs, or 1) whose clusters for every row fit on the
-// device at once (a cluster that waits for a second wave costs a whole row's
+// largest cluster (16, 8, 4, 2 CTAs, or 1) whose clusters for every row fit on
+// the device at once (a cluster that waits for a second wave costs a whole row's
 // time again).  nseg = 0: too many rows for one wave; the collect + select
 // kernel takes them.
 tk::ClPlan cluster_plan(int32_t rows, int64_t n_cols) {
@@ -487,7 +506,7 @@ tk::ClPlan cluster_plan(int32_t rows, int64_t n_cols) {
     const tk::ClPlan p = tk::cl_plan(n_cols, cap);
     if (p.nseg == 0) break;                 // fewer segments would exceed what a CTA stages
     if (p.nseg < cap && cap > 1) continue;  // the row is too short for this many segments
-    if (static_cast<int64_t>(rows) <= cluster_capacity(p.nseg, tk::cl_smem(p.seg_len))) return p;
+    if (static_cast<int64_t>(rows) <= cluster_capacity(p.nseg, tk::cl_smem(p.seg_len, p.nseg))) return p;
   }
   tk::ClPlan none;
   none.nseg = 0;
@@ -537,6 +556,10 @@ TopkPlan topk_plan(int32_t rows, int64_t n_cols) {
 bool topk_v2_ok(int64_t n_cols) { return n_cols <= tk::kMaxBitmapCols; }
 
 bool topk_cluster_ok(int64_t n_cols) { return n_cols <= tk::kClMaxCols; }
+
+bool topk_cluster_planned(int32_t rows, int64_t n_cols) {
+  return topk_v2_ok(n_cols) && topk_cluster_ok(n_cols) && cluster_plan(rows, n_cols).nseg > 0;
+}
 
 size_t topk_hist_zero_bytes(int32_t rows) { return tk::tk_zero_bytes(rows); }
 
@@ -624,9 +647,10 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
                                ? cluster_plan(a.rows, a.n_cols) : tk::ClPlan{0, 0};
     if (clp.nseg > 0) {
       const tk::ClPlan& cp = clp;
-      // one cluster of up to 8 CTAs per row
-      const size_t smem = tk::cl_smem(cp.seg_len);
-      e = ensure_dyn_smem(k_tk_cluster, smem);
+      // one cluster of up to 16 CTAs per row
+      const size_t smem = tk::cl_smem(cp.seg_len, cp.nseg);
+      ClusterKernel fn = nullptr;
+      e = cluster_kernel(cp.nseg, smem, &fn);
       if (e != cudaSuccess) return e;
       cudaLaunchConfig_t cfg;
       memset(&cfg, 0, sizeof(cfg));
@@ -643,7 +667,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
       attr[1].val.programmaticStreamSerializationAllowed = 1;
       cfg.attrs = attr;
       cfg.numAttrs = a.pdl ? 2 : 1;
-      return cudaLaunchKernelEx(&cfg, k_tk_cluster, a, cp.seg_len, cp.nseg);
+      return cudaLaunchKernelEx(&cfg, fn, a, cp.seg_len, cp.nseg);
     }
     size_t smem;
     TopkPlan cp;

@@ -25,13 +25,18 @@ namespace lsa {
 namespace tk {
 
 constexpr int kClThreads = kCollectThreads;        // the round shape of tk_round_load
-constexpr int kClMaxSeg = 8;                       // CTAs per cluster (portable cluster size)
-constexpr int64_t kClMaxCols = int64_t(1) << 18;   // longer rows take the collect + select bodies
-constexpr int kClCandCap = 1024;                   // threshold-bin keys a CTA keeps
+constexpr int kClMaxSeg = 16;                      // CTAs per cluster (above 8: a non-portable cluster size)
+constexpr int kClPortableSeg = 8;
+constexpr int64_t kClMaxCols = int64_t(1) << 19;   // longer rows take the collect + select bodies
 constexpr int64_t kClMaxSegLen = 32768;            // positions a CTA stages in shared memory (128 KB)
+// Threshold-bin keys a CTA keeps, by the cluster's largest size: every CTA
+// gathers all CTAs' lists, so 16-CTA clusters keep half as many per CTA to
+// stay within shared memory.  (A bin holds a few hundred keys of a row at
+// these sizes; a longer list overflows into the whole-row path, still exact.)
+__host__ __device__ constexpr int cl_cap(int maxseg) { return maxseg > kClPortableSeg ? 512 : 1024; }
 
 struct ClHdr {
-  uint32_t nc;  // keys of the threshold bin in the segment (> kClCandCap: the list overflowed)
+  uint32_t nc;  // keys of the threshold bin in the segment (> cl_cap: the list overflowed)
   uint32_t gt;  // selected keys above T in the segment
   uint32_t eq;  // keys equal to T in the segment
   uint32_t pad;
@@ -74,19 +79,24 @@ __host__ __device__ inline int cl_bm_words(int64_t seg_len) {
   return (kClThreads * p.stride + 3) / 4 * 4;
 }
 
-__host__ __device__ inline size_t cl_smem(int64_t seg_len) {
+// Clusters of up to 8 CTAs run the MAXSEG = 8 body, larger ones MAXSEG = 16.
+__host__ __device__ constexpr int cl_maxseg(int nseg) { return nseg > kClPortableSeg ? kClMaxSeg : kClPortableSeg; }
+
+__host__ __device__ inline size_t cl_smem(int64_t seg_len, int nseg) {
+  const int maxseg = cl_maxseg(nseg);
+  const size_t cap = static_cast<size_t>(cl_cap(maxseg));
   return sizeof(ClHdr) + static_cast<size_t>(seg_len) * 4 + static_cast<size_t>(kB1) * 4 +
-         2 * static_cast<size_t>(cl_bm_words(seg_len)) * 4 + static_cast<size_t>(kClCandCap) * 8 +
-         static_cast<size_t>(kClMaxSeg) * kClCandCap * 4;
+         2 * static_cast<size_t>(cl_bm_words(seg_len)) * 4 + cap * 8 + static_cast<size_t>(maxseg) * cap * 4;
 }
 
 // Row r, segment s of ns (CTA rank s of the row's cluster).  `live` false (a
 // wait before it ran out): the CTA does no work but still takes part in the
 // cluster barriers.  ID: named barrier of the CTA's threads.
-template <int ID>
+template <int ID, int MAXSEG>
 __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t seg_len, uint8_t* dsm, TkScratch& S,
                                bool live) {
   constexpr int NT = kClThreads;
+  constexpr int CAP = cl_cap(MAXSEG);
   const int t = threadIdx.x;
   const int lane = t & 31;
   const TkLayout L = tk_layout(a.ws, a.rows, a.n_cols);
@@ -98,7 +108,7 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
   uint32_t* bm = hsm + kB1;
   uint32_t* tb = bm + bm_words;
   uint2* cs = reinterpret_cast<uint2*>(tb + bm_words);
-  uint32_t* allk = reinterpret_cast<uint32_t*>(cs + kClCandCap);  // [kClMaxSeg * kClCandCap]
+  uint32_t* allk = reinterpret_cast<uint32_t*>(cs + CAP);  // [MAXSEG * CAP]
   const DivU32 dper = make_divu32(static_cast<uint32_t>(pad.per));
   auto pw = [&](uint32_t w) -> int {  // padded index of segment word w
     const uint32_t q = divu32(dper, w);
@@ -205,7 +215,7 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
       while (bin_w) {  // this thread's candidates, in position order
         const int b = __ffs(bin_w) - 1;
         bin_w &= bin_w - 1;
-        if (o < kClCandCap) cs[o] = make_uint2(order_key(seg[q - s0 + b]), static_cast<uint32_t>(q + b));
+        if (o < CAP) cs[o] = make_uint2(order_key(seg[q - s0 + b]), static_cast<uint32_t>(q + b));
         ++o;
       }
       nc += tot;
@@ -222,24 +232,24 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
   // memory with all of the remote loads in flight at once (a remote load is a
   // round trip; one after another they would cost a round trip each)
   const uint32_t hdr_u = tc::smem_u32(hdr), cs_u = tc::smem_u32(cs);
-  uint32_t ncq[kClMaxSeg];
+  uint32_t ncq[MAXSEG];
 #pragma unroll
-  for (int q = 0; q < kClMaxSeg; ++q)
+  for (int q = 0; q < MAXSEG; ++q)
     ncq[q] = q < ns ? tc::ld_cluster_u32(tc::cluster_map(hdr_u, static_cast<uint32_t>(q))) : 0u;
   bool ovf = false;
   int n_all = 0;
-  uint32_t offq[kClMaxSeg];
+  uint32_t offq[MAXSEG];
 #pragma unroll
-  for (int q = 0; q < kClMaxSeg; ++q) {
-    ovf |= ncq[q] > static_cast<uint32_t>(kClCandCap);
+  for (int q = 0; q < MAXSEG; ++q) {
+    ovf |= ncq[q] > static_cast<uint32_t>(CAP);
     offq[q] = static_cast<uint32_t>(n_all);
     n_all += static_cast<int>(ncq[q]);
   }
   if (live && keff > 0 && !ovf) {
-    constexpr int U = kClCandCap / NT;
-    uint32_t kv[kClMaxSeg][U];
+    constexpr int U = CAP / NT;
+    uint32_t kv[MAXSEG][U];
 #pragma unroll
-    for (int q = 0; q < kClMaxSeg; ++q) {
+    for (int q = 0; q < MAXSEG; ++q) {
       const uint32_t base_q = tc::cluster_map(cs_u, static_cast<uint32_t>(q < ns ? q : 0));
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -248,7 +258,7 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
       }
     }
 #pragma unroll
-    for (int q = 0; q < kClMaxSeg; ++q) {
+    for (int q = 0; q < MAXSEG; ++q) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const uint32_t c = static_cast<uint32_t>(t + u * NT);
@@ -320,15 +330,15 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
   tc::cluster_sync();  // ---- every segment's counts published
   // entries before this segment and the ties left to it (lowest positions
   // first); the remote counts are loaded together
-  uint32_t gtq[kClMaxSeg], eqq[kClMaxSeg];
+  uint32_t gtq[MAXSEG], eqq[MAXSEG];
 #pragma unroll
-  for (int q = 0; q < kClMaxSeg; ++q) {
+  for (int q = 0; q < MAXSEG; ++q) {
     gtq[q] = q < ns ? tc::ld_cluster_u32(tc::cluster_map(hdr_u + 4u, static_cast<uint32_t>(q))) : 0u;
     eqq[q] = q < ns ? tc::ld_cluster_u32(tc::cluster_map(hdr_u + 8u, static_cast<uint32_t>(q))) : 0u;
   }
   uint32_t off = 0, ties_mine = 0, eq_seen = 0;
 #pragma unroll
-  for (int q = 0; q < kClMaxSeg; ++q) {
+  for (int q = 0; q < MAXSEG; ++q) {
     const uint32_t gt_q = gtq[q], eq_q = eqq[q];
     const uint32_t left = ties > eq_seen ? ties - eq_seen : 0u;
     const uint32_t take = left < eq_q ? left : eq_q;

@@ -258,14 +258,16 @@ def _split_case():
     return case
 
 
-@pytest.mark.parametrize("min_cols", [0, 100000000])
-def test_decode_step_split_select(min_cols, test_hooks):
-    """With the split select forced on (rows of any length) or off, the decode
-    step selects what lsa_indexer_scores + lsa_topk select, ties and the
-    fallback row included, and its outputs match the oracle."""
+@pytest.mark.parametrize("min_cols,no_cluster", [(0, True), (100000000, True), (100000000, False)])
+def test_decode_step_split_select(min_cols, no_cluster, test_hooks):
+    """With the split select forced on (rows of any length; the cluster top-k,
+    which rows that short would otherwise take, turned off) or off (the
+    collect + select or the cluster top-k), the decode step selects what
+    lsa_indexer_scores + lsa_topk select, ties and the fallback row included,
+    and its outputs match the oracle."""
     from sparse_attention_decode_scan_b200 import lsa
     from sparse_attention_decode_scan_b200.device import DeviceCase
-    test_hooks(split_select_min_cols=min_cols)
+    test_hooks(split_select_min_cols=min_cols, no_cluster_topk=no_cluster)
     case = _split_case()
     dc = DeviceCase(case)
     _, _, idx_step = _step(dc)

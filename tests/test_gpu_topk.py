@@ -24,6 +24,9 @@ CASES = [
     ("normal", 4, 3000, 64, "with_zero"),      # a row with no valid entry
     ("ties", 40, 139264, 2048, "ragged"),      # many rows
     ("equal", 1, 200000, 2048, "full"),        # one tie class spread over many segments
+    # 2^18 .. 2^19 positions: clusters of 16 CTAs (one overflowing every candidate list)
+    ("ties", 2, 400000, 2048, "ragged"),
+    ("equal", 1, 500000, 2048, "full"),
     # rows longer than 2^19 positions take the general five-launch path
     ("normal", 2, 600000, 2048, "full"),
     ("ties", 2, 600000, 2048, "ragged"),
@@ -67,10 +70,12 @@ def test_topk_exact(kind, rows, n, k, mode):
         assert np.array_equal(got[r], want), f"row {r}: first mismatch at {int(np.argmax(got[r] != want))}"
 
 
-@pytest.mark.parametrize("kind,rows,n,k,mode", [c for c in CASES if c[2] <= (1 << 18)][:10],
-                         ids=[f"{c[0]}-{c[1]}x{c[2]}-k{c[3]}-{c[4]}" for c in CASES if c[2] <= (1 << 18)][:10])
+_CL_CASES = [c for c in CASES if c[2] <= (1 << 19)]
+
+
+@pytest.mark.parametrize("kind,rows,n,k,mode", _CL_CASES, ids=[f"{c[0]}-{c[1]}x{c[2]}-k{c[3]}-{c[4]}" for c in _CL_CASES])
 def test_topk_collect_select_path_equals_cluster_path(kind, rows, n, k, mode, test_hooks):
-    """Rows of up to 2^18 positions take the one-cluster-per-row kernel; the
+    """Rows of up to 2^19 positions take the one-cluster-per-row kernel; the
     collect + per-row select kernel (the path of longer rows, forced here by
     the test build) gives the same index arrays."""
     from sparse_attention_decode_scan_b200 import lsa
