@@ -817,6 +817,14 @@ __device__ __forceinline__ void attn_cta(const TcAttnParams& P, uint8_t* smem_ra
         }
         l += lsum[0] + lsum[1];
       }
+      // P(j) may only be published once the MMA issuer has taken P(j-1)
+      // (P V(j-1) issued and done): S(j) can be issued before P V(j-1), so
+      // without this wait pfull could complete phases j-1 and j before the
+      // issuer tests it for j-1, its parity would read "not yet" and the
+      // issuer would stall.  The wait names its phase unambiguously: S(j)'s
+      // commit covered P V(j-2).  It rarely waits (P V(j-1) runs right after
+      // S(j), while this chunk's softmax is still busy).
+      if (j > 0 && !tc::mbar_wait(pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();

@@ -267,8 +267,56 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
     }
   }
   uint32_t T = 0, ties = 0;
-  if (live && keff > 0) {
-    if (!ovf) {
+  const bool work = live && keff > 0;
+  if (ovf) {
+    // Some CTA's list overflowed (many keys in the threshold bin, e.g. a
+    // large k or a flat score distribution).  T's lower two digits are then
+    // counted from every CTA's own segment, still in its shared memory, and
+    // the counts summed across the cluster through distributed shared memory:
+    // two rounds of two cluster barriers, every CTA taking part (the barriers
+    // are the cluster's, live or not).
+    T = b1 << 20;
+    uint32_t rank = rank1;
+    constexpr int PER = 1024 / NT;
+    static_assert(PER == 4, "one 16-byte word of bins per thread");
+    for (int pass = 0; pass < 2; ++pass) {
+      const uint32_t shift = pass == 0 ? 10 : 0;
+      const uint32_t pre_shift = pass == 0 ? 20 : 10;
+      const uint32_t prefix = T >> pre_shift;
+      for (int i = t; i < 1024; i += NT) S.h[i] = 0;
+      tk_sync<NT, ID>();
+      if (work) {
+        for (int p = s0 + t; p < s1 && p < n; p += NT) {
+          const uint32_t key = order_key(seg[p - s0]);
+          if (key != 0u && (key >> pre_shift) == prefix) atomicAdd(&S.h[(key >> shift) & 1023u], 1u);
+        }
+      }
+      tc::cluster_sync();  // every CTA's counts are complete
+      if (work) {
+        // bins 4t .. 4t+3 of every CTA, all loads in flight, then summed
+        const uint32_t h_u = tc::smem_u32(&S.h[t * PER]);
+        float4 part[MAXSEG];
+#pragma unroll
+        for (int q = 0; q < MAXSEG; ++q)
+          part[q] = q < ns ? tc::ld_cluster_f4(tc::cluster_map(h_u, static_cast<uint32_t>(q)))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        uint32_t hl[PER] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int q = 0; q < MAXSEG; ++q) {
+          hl[0] += __float_as_uint(part[q].x);
+          hl[1] += __float_as_uint(part[q].y);
+          hl[2] += __float_as_uint(part[q].z);
+          hl[3] += __float_as_uint(part[q].w);
+        }
+        tk_find<NT, ID, 1024>(hl, rank, S, false);
+        T |= static_cast<uint32_t>(S.s_bin) << shift;
+        rank = S.s_rank;
+      }
+      tc::cluster_sync();  // every CTA has read the others' counts before they are cleared
+    }
+    ties = rank;
+  } else if (work) {
+    {
       for (int pass = 0; pass < 2; ++pass) {
         for (int i = t; i < 1024; i += NT) S.h[i] = 0;
         tk_sync<NT, ID>();  // also: the gathered keys are complete
@@ -289,9 +337,9 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
         ties = S.s_rank;
         tk_sync<NT, ID>();
       }
-    } else {
-      tk_radix_T<NT, ID>(cs, 0, true, row, n, b1, rank1, S, &T, &ties);
     }
+  }
+  if (work) {
     // this segment's keys of bin b1: above T into the bitmap, equal to T into the tie bitmap
     if (!ovf) {
       for (int c = t; c < nc; c += NT) {

@@ -89,7 +89,7 @@ __host__ __device__ inline size_t tk_ws_bytes(int32_t rows, int64_t n_cols) {
 
 // Shared scratch of the bodies (static in the standalone kernels, carved from
 // dynamic shared memory in the fused step).
-struct TkScratch {
+struct __align__(16) TkScratch {  // h is read as 16-byte words (the cluster top-k's remote counts)
   int warp_sums[32];
   int s_bin;
   uint32_t s_rank;
