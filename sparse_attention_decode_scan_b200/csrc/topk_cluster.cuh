@@ -16,8 +16,10 @@
 // and publishes two counts.  After a second barrier each CTA knows the
 // selection entries before its segment and the ties left to it (the lowest
 // positions equal to T are taken first), and compacts its own segment into
-// the output.  If any CTA's candidates overflow its list, T is found from the
-// whole row and each segment is re-read to mark.
+// the output.  If any CTA's candidates overflow its list, T's lower digits are
+// counted by every CTA from its own staged segment, the counts summed across
+// the cluster through distributed shared memory, and each segment re-read
+// from shared memory to mark.
 #include "tc.cuh"
 #include "topk_sel.cuh"
 
