@@ -233,9 +233,11 @@ lsa_status lsa_decode_step_profiled(const lsa_dims* d, const lsa_cache* c, const
  * Order on `stream`: layer l+1 starts after layer l's attention has finished
  * (a layer's queries depend on the previous layer's output).  Within a layer
  * that keeps an indexer, LSA_ROUTE_OWN runs scan -> top-k -> attention as
- * lsa_decode_step does; LSA_ROUTE_PREV runs the attention (on the earlier
- * selection) first, then the layer's scan and top-k into a second selection
- * buffer.
+ * lsa_decode_step does; LSA_ROUTE_PREV launches the attention (on the earlier
+ * selection) first and the layer's scan as its programmatic dependent, so
+ * the scan runs on the SMs the attention leaves free while it runs (MLI
+ * abstract: each indexer runs concurrently with its layer's attention), then
+ * the top-k into a second selection buffer.
  * Results per layer equal lsa_decode_step / lsa_sparse_attn_decode on the
  * routed selection.
  * Workspace: lsa_workspace_size(d, B, max_len, LSA_OP_DECODE_LAYERS).

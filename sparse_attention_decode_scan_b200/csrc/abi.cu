@@ -25,6 +25,14 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Rows at least this long take the split select in a decode step.
 constexpr int64_t kSplitSelectMinCols = int64_t(1) << 18;
 
+// Timing model of the MLI layer's scan split (measured on B200 at 1965 MHz): a
+// tensor-core attention CTA takes about kAttnFixedUs plus kAttnChunkUs per
+// 64-entry chunk, and a scan CTA streams one 128-token bf16 tile per
+// kScanTileUs.  It only decides how many tiles the first scan launch takes.
+constexpr double kAttnFixedUs = 21.0;
+constexpr double kAttnChunkUs = 2.2;
+constexpr double kScanTileUs = 0.72;
+
 #ifdef LSA_TEST_HOOKS
 // Test build only (liblsa_test.so, include/lsa_test.h): switches that tests
 // set through lsa_test_set_hooks.  The product library has none of them, so
@@ -238,14 +246,24 @@ ScoresArgs scores_args(const lsa_dims* d, const lsa_cache* c, int32_t rows, cons
 lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const int32_t* row_seq,
                      const int32_t* row_pos, const void* q_idx, const float* w, float* scores,
                      int64_t ld, void* ws, void* inner_ws, size_t inner_bytes, cudaStream_t s,
-                     uint32_t* hist12 = nullptr, bool* hist_done = nullptr, uint32_t* done_ctr = nullptr) {
+                     uint32_t* hist12 = nullptr, bool* hist_done = nullptr, uint32_t* done_ctr = nullptr,
+                     bool zeroed = false, bool pdl = false, const ScoresArgs* split = nullptr) {
   ScoresArgs a = scores_args(d, c, rows, row_seq, row_pos, q_idx, w, scores, ld, ws, inner_ws, inner_bytes);
   if (hist_done) *hist_done = false;
   if (rows == 0 || ld == 0) return LSA_OK;
   if (!force_simt() && scores_tc_supported(a)) {
+    a.pdl = pdl;
+    if (split) {
+      a.grid = split->grid;
+      a.split_part = split->split_part;
+      a.split_free = split->split_free;
+      a.split_busy_us = split->split_busy_us;
+      a.split_tile_us = split->split_tile_us;
+    }
     if (hist12 && scores_tc_fused_hist_ok(a)) {
-      // the scan also counts the first top-k digit; the counters start at zero
-      cudaError_t e = cudaMemsetAsync(hist12, 0, topk_hist_zero_bytes(rows), s);
+      // the scan also counts the first top-k digit; the counters start at
+      // zero (cleared here unless the caller already did)
+      cudaError_t e = zeroed ? cudaSuccess : cudaMemsetAsync(hist12, 0, topk_hist_zero_bytes(rows), s);
       if (e != cudaSuccess) return LSA_ERR_CUDA;
       a.hist12 = hist12;
       a.done_ctr = done_ctr;  // zeroed with the histograms
@@ -553,15 +571,51 @@ lsa_status lsa_decode_layers(const lsa_dims* d, int32_t n_layers, const lsa_cach
       uint32_t *scan_done = nullptr, *sel_done = nullptr;
       if (hist12) topk_step_flags(tk, B, c->max_len, &scan_done, &sel_done);
       if (overlap) {
-        // The attention on the selection already made, then this layer's
-        // scan and top-k (which writes the other buffer), in stream order.
+        // The attention on the selection already made goes first.  The scan
+        // follows as its programmatic dependent (it reads nothing the
+        // attention writes) and takes the SMs the attention leaves; the
+        // top-k follows the scan.  The counters they share are cleared before
+        // the attention, so no copy-engine step separates the kernels.
+        const ScoresArgs sa =
+            scores_args(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes);
+        const bool fused_hist = hist12 && !force_simt() && scores_tc_supported(sa) && scores_tc_fused_hist_ok(sa);
+        if (fused_hist && cudaMemsetAsync(hist12, 0, topk_hist_zero_bytes(B), s) != cudaSuccess) return LSA_ERR_CUDA;
         st = do_attn(d, c, B, nullptr, q[l], sel[cur], out[l], lse_l, ws, at, L.at_bytes, s);
         if (st != LSA_OK) return st;
-        st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
-                       &hist_done, scan_done);
+        // The attention's CTAs (one per SM) leave some SMs free: a first scan
+        // launch of one CTA per free SM takes the tiles those SMs stream while
+        // the attention runs, a second (one CTA per SM) the rest as the
+        // attention's CTAs end (each CTA has a static share, so a single
+        // launch would end with its last-started CTAs).
+        const int sms = scan_tc_grid();
+        int cps = 0;
+        const bool tc_attn =
+            !force_simt() && attn_tc_supported(attn_args(d, c, B, nullptr, q[l], sel[cur], out[l], lse_l, ws, at,
+                                                         L.at_bytes));
+        const int free_sms = tc_attn ? sms - attn_tc_ctas(B, d->top_k, &cps) : 0;
+        uint32_t target = static_cast<uint32_t>(sms);
+        if (fused_hist && free_sms > 0) {
+          ScoresArgs sp;
+          sp.split_free = free_sms;
+          sp.split_busy_us = static_cast<float>(kAttnFixedUs + kAttnChunkUs * cps);
+          sp.split_tile_us = static_cast<float>(kScanTileUs);
+          sp.grid = free_sms;
+          sp.split_part = 1;
+          st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
+                         &hist_done, scan_done, true, true, &sp);
+          if (st != LSA_OK) return st;
+          sp.grid = sms;
+          sp.split_part = 2;
+          st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
+                         &hist_done, scan_done, true, true, &sp);
+          target = static_cast<uint32_t>(sms + free_sms);
+        } else {
+          st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s,
+                         fused_hist ? hist12 : nullptr, &hist_done, scan_done, fused_hist, true);
+        }
         if (st != LSA_OK) return st;
         st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, sel[nxt], ws, tk, s, hist_done, true,
-                     hist_done ? scan_done : nullptr, hist_done ? static_cast<uint32_t>(scan_tc_grid()) : 0u);
+                     hist_done ? scan_done : nullptr, hist_done ? target : 0u);
       } else {
         st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
                        &hist_done, scan_done);

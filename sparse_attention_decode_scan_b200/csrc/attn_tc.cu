@@ -20,6 +20,9 @@ using namespace attn;
 __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const TcAttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
+  // a programmatic dependent (the layer's scan under the MLI route, which
+  // reads nothing this kernel writes) may take the SMs this grid leaves free
+  tc::griddep_launch_dependents();
   if ((threadIdx.x >> 5) == kWarpMma) {
     tc::tmem_alloc(&tmem_slot, kTmemCols);
     tc::tc_fence_before();
@@ -92,6 +95,13 @@ bool attn_tc_shape_ok(int32_t dtype, int32_t H, int32_t D, int32_t Dv, int32_t) 
 }
 
 int attn_tc_launches(int32_t, int32_t, int32_t) { return 1; }
+
+int attn_tc_ctas(int32_t rows, int32_t k, int* chunks_per_cta) {
+  const int ns = tc_nsplit(rows, k);
+  const int chunks = (k + kChunk - 1) / kChunk;
+  if (chunks_per_cta) *chunks_per_cta = (chunks + ns - 1) / ns;
+  return ns * 2 * rows;
+}
 
 bool attn_tc_split_fits(int32_t rows, int32_t k) {
   const int ns = tc_nsplit(rows, k);

@@ -113,7 +113,23 @@ cudaError_t launch_t(const ScoresArgs& a, cudaStream_t s) {
   auto kern = k_scan_tc<KDT, QB, false, EG>;
   cudaError_t e = ensure_dyn_smem(kern, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<num_sms(), scan_threads<EG>(), C::kSmemBytes, s>>>(tmap, smap, a);
+  const unsigned grid = static_cast<unsigned>(a.grid > 0 ? a.grid : num_sms());
+  if (a.pdl) {
+    // a programmatic dependent: its CTAs take SMs as the kernel before frees them
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(scan_threads<EG>());
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmap, smap, a);
+  }
+  kern<<<grid, scan_threads<EG>(), C::kSmemBytes, s>>>(tmap, smap, a);
   return cudaGetLastError();
 }
 

@@ -53,6 +53,17 @@ struct ScoresArgs {
   // visible range or a bad block).  bf16 keys only.
   const int32_t* cand = nullptr;
   int32_t cand_ld = 0;
+  // Tensor-core scan launched as a programmatic dependent of the kernel before
+  // it, which writes nothing the scan reads (the scan never waits for it).
+  bool pdl = false;
+  // Tensor-core scan: `grid` CTAs (0: one per SM).  split_part 1 or 2: the
+  // launch covers the first or the second part of the rows' tiles, the first
+  // being what split_free CTAs stream in split_busy_us while the other SMs
+  // are held by another kernel (one tile per split_tile_us); 0: every tile.
+  int grid = 0;
+  int split_part = 0;
+  int split_free = 0;
+  float split_busy_us = 0.f, split_tile_us = 1.f;
 };
 
 // ---- indexer
@@ -185,6 +196,9 @@ bool attn_tc_supported(const AttnArgs& a);
 // Whether each split of the tensor-core attention holds at most one row table
 // of entries (needed for it to compact its entries itself).
 bool attn_tc_split_fits(int32_t rows, int32_t k);
+// CTAs of the tensor-core attention's launch for `rows` rows and k entries
+// (and the 64-entry chunks each CTA works through).
+int attn_tc_ctas(int32_t rows, int32_t k, int* chunks_per_cta);
 size_t attn_tc_ws_bytes(int32_t rows, int32_t H, int32_t D, int32_t Dv, int32_t k);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);
 // exact merge of per-split softmax partials (shared by both attention paths)

@@ -238,6 +238,18 @@ struct Plan {
   int64_t n_items;
 };
 
+// The tiles [lo, hi) of `tot` that this launch covers (ScoresArgs::split_part).
+__device__ __forceinline__ void launch_tiles(const ScoresArgs& a, int64_t tot, int64_t* lo, int64_t* hi) {
+  *lo = 0;
+  *hi = tot;
+  if (a.split_part == 0 || a.split_free <= 0) return;
+  // the first part: what split_free CTAs stream while the other SMs are busy
+  int64_t first = static_cast<int64_t>(a.split_busy_us / a.split_tile_us) * a.split_free;
+  first = first < 0 ? 0 : (first > tot ? tot : first);
+  if (a.split_part == 1) *hi = first;
+  else *lo = first;
+}
+
 // Every thread of the CTA takes part: total tiles, this CTA's share, and the
 // group holding its first tile.
 template <int QB, int NTH = kThreads>
@@ -251,8 +263,11 @@ __device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
     if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
     int64_t incl, tot;
     block_sum_i64_scan<NTH>(t, sbuf, &incl, &tot);
-    const int64_t t0 = tot * blockIdx.x / gridDim.x;
-    p.n_items = tot * (blockIdx.x + 1) / gridDim.x - t0;
+    // this launch's tiles [lo, hi), split evenly over its CTAs
+    int64_t lo, hi;
+    launch_tiles(a, tot, &lo, &hi);
+    const int64_t t0 = lo + (hi - lo) * blockIdx.x / gridDim.x;
+    p.n_items = lo + (hi - lo) * (blockIdx.x + 1) / gridDim.x - t0;
     if (p.n_items <= 0) return p;
     const int64_t start = incl - t;
     if (t > 0 && start <= t0 && t0 < start + t) {  // exactly one thread holds tile t0
@@ -273,8 +288,10 @@ __device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
     block_sum_i64_scan<NTH>(t, sbuf, &incl, &tot);
     total += tot;
   }
-  const int64_t t0 = total * blockIdx.x / gridDim.x;
-  const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
+  int64_t lo, hi;
+  launch_tiles(a, total, &lo, &hi);
+  const int64_t t0 = lo + (hi - lo) * blockIdx.x / gridDim.x;
+  const int64_t t1 = lo + (hi - lo) * (blockIdx.x + 1) / gridDim.x;
   p.n_items = t1 - t0;
   if (p.n_items <= 0) return p;
   if (threadIdx.x == 0) sfound[0] = -1;
