@@ -95,13 +95,14 @@ cudaError_t make_maps(const ScoresArgs& a, CUtensorMap* tmap_out, CUtensorMap* s
   return cudaSuccess;
 }
 
-// Epilogue groups: the per-tile epilogue (TMEM loads and the ReLU-weighted
-// head sums) of the FP8 decode scan and of the prefill scans is twice (FP8:
-// hi and lo terms) or four times (4 query rows) the bf16 decode scan's, so two
-// groups of epilogue warps take alternate tiles there; the bf16 decode scan
-// streams keys at the copy rate with one.
+// Epilogue groups: two groups of epilogue warps take alternate tiles.  The
+// per-tile epilogue (TMEM loads, the ReLU-weighted head sums, the score
+// stores and histogram counts) is the longest stage of the SM-side pipeline:
+// with the key loads taken out, the bf16 decode scan still needed 132 of its
+// 142 us with one group.  Two groups shorten the B=32 decode step by about
+// 2.5 us (the scan's CTAs end closer together).
 template <int KDT, int QB>
-constexpr int epi_groups() { return (KDT == LSA_FP8_E4M3 || QB > 1) ? 2 : 1; }
+constexpr int epi_groups() { return 2; }
 
 template <int KDT, int QB>
 cudaError_t launch_t(const ScoresArgs& a, cudaStream_t s) {
