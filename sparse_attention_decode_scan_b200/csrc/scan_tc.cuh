@@ -52,8 +52,7 @@ constexpr int kScaleBox = 68;    // FP8 scales per box load: 64 + up to 3 for th
 constexpr int kScaleSlot = 96;   // floats per scale slot: a TMA destination starts on a 128-byte boundary
 constexpr int kThreads = 256;    // 8 warps (one epilogue group)
 // Threads of a scan CTA with EG epilogue groups of 4 warps (warps 3.., the
-// groups taking alternate tiles, i.e. one accumulator buffer each), the
-// second MMA issuer's warp last.
+// groups taking alternate tiles), the second MMA issuer's warp last.
 template <int EG>
 constexpr int scan_threads() { return kThreads + (EG - 1) * 128; }
 template <int EG>
