@@ -131,29 +131,35 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
   // The row's histogram and the segment's scores (up to the row's length
   // rounded to 16 bytes) come into shared memory by 16-byte cp.async copies of
   // every thread, consecutive threads on consecutive bytes: one commit group
-  // for the histogram, one per collect round, all in flight at once, so each
-  // round starts as soon as its own group has landed.  (Large bulk copies were
-  // measured to deliver far fewer bytes per microsecond here.)
+  // for the histogram and one per collect round, each round's copies issued
+  // kAhead rounds before it is processed.  (Issuing every round at once made
+  // the first round's processing slow, its shared-memory reads meeting the
+  // later rounds' copies as they landed, and the issue itself stall on the
+  // copies in flight; large bulk copies delivered far fewer bytes per
+  // microsecond.)
+  constexpr int kAhead = 2;
   const int s1r = (s1 + 3) & ~3;  // whole 16-byte groups
   const int s_hi = s1r < lim ? s1r : lim;
   const int n_rounds = s1 > s0 ? (s1 - s0 + kColRound - 1) / kColRound : 0;
   bool staged_ok = true;
   const bool staging = live;
+  auto issue_round = [&](int i) {
+#pragma unroll
+    for (int k = 0; k < kColRound / 4 / NT; ++k) {
+      const int p = s0 + i * kColRound + 4 * (k * NT + t);
+      // groups past the staged range are zero-filled (read nothing)
+      tc::cp_async16_zfill(seg + (p - s0), row + (p < s_hi ? p : s0), p < s_hi ? 16u : 0u);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  const int first_rounds = n_rounds < kAhead ? n_rounds : kAhead;
   if (staging) {
     const uint32_t* hsrc = L.hist + static_cast<int64_t>(r) * kB1;
 #pragma unroll
     for (int k = 0; k < kB1 / 4 / NT; ++k)
       tc::cp_async16_zfill(hsm + 4 * (k * NT + t), hsrc + 4 * (k * NT + t), 16u);
     asm volatile("cp.async.commit_group;" ::: "memory");
-    for (int i = 0; i < n_rounds; ++i) {
-#pragma unroll
-      for (int k = 0; k < kColRound / 4 / NT; ++k) {
-        const int p = s0 + i * kColRound + 4 * (k * NT + t);
-        // groups past the staged range are zero-filled (read nothing)
-        tc::cp_async16_zfill(seg + (p - s0), row + (p < s_hi ? p : s0), p < s_hi ? 16u : 0u);
-      }
-      asm volatile("cp.async.commit_group;" ::: "memory");
-    }
+    for (int i = 0; i < first_rounds; ++i) issue_round(i);
   }
   // waits until at most `pending` of this thread's newest groups are in flight
   auto wait_groups = [&](int pending) {
@@ -166,8 +172,8 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
     }
   };
   if (staging) {
-    wait_groups(n_rounds);  // the histogram
-    tk_sync<NT, ID>();      // every thread's part of it
+    wait_groups(first_rounds);  // the histogram
+    tk_sync<NT, ID>();          // every thread's part of it
   }
   // ---------------------------------------------------------------- collect
   uint32_t keff = 0, b1 = 0xffffffffu, rank1 = 0;
@@ -184,8 +190,11 @@ __device__ void tk_cluster_row(const TopkArgs& a, int r, int s, int ns, int64_t 
     }
 #pragma unroll 1
     for (int rd = 0; keff > 0 && rd < n_rounds; ++rd) {
-      wait_groups(n_rounds - 1 - rd);  // this round's scores (later rounds may still be in flight)
-      tk_sync<NT, ID>();                // every thread's part of them
+      // round rd + kAhead's copies go out; this round's have had kAhead rounds to land
+      if (rd + kAhead < n_rounds) issue_round(rd + kAhead);
+      const int later = n_rounds - 1 - rd;  // rounds after this one, issued by now
+      wait_groups(later < kAhead ? later : kAhead);
+      tk_sync<NT, ID>();  // every thread's part of them
       // thread t builds bitmap word t of the round (positions 32 t .. 32 t + 31)
       // from its own 16-byte groups, read in a rotated order so that the
       // warp's reads spread over the banks; every bit is independent work
