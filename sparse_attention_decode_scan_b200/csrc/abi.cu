@@ -32,6 +32,12 @@ constexpr int64_t kSplitSelectMinCols = int64_t(1) << 18;
 constexpr double kAttnFixedUs = 21.0;
 constexpr double kAttnChunkUs = 2.2;
 constexpr double kScanTileUs = 0.72;
+// The decode scan's pooled schedule: each CTA's even share of the first
+// kPoolStaticPm thousandths of the tiles, then chunks of kPoolChunk tiles from
+// the pool until it is empty (the CTAs of a static split ended up to 8 us
+// apart at B = 32; a chunk takes a CTA about 3.4 us).
+constexpr int kPoolChunk = 4;
+constexpr int kPoolStaticPm = 900;
 
 #ifdef LSA_TEST_HOOKS
 // Test build only (liblsa_test.so, include/lsa_test.h): switches that tests
@@ -43,17 +49,23 @@ struct TestHooks {
   int64_t split_select_min_cols = kSplitSelectMinCols;
   uint32_t scan_wait_extra = 0;                    // raises the decode step's scan-CTA count
   bool no_cluster_topk = false;                    // the collect + select top-k for every row length
+  int pool_static_pm = kPoolStaticPm;              // > 1000: the decode scan without its pool
+  int pool_chunk = kPoolChunk;
 };
 TestHooks g_hooks;
 bool force_simt() { return g_hooks.force_simt; }
 int64_t split_select_min_cols() { return g_hooks.split_select_min_cols; }
 uint32_t test_scan_wait_extra() { return g_hooks.scan_wait_extra; }
 bool allow_cluster_topk() { return !g_hooks.no_cluster_topk; }
+int pool_static_pm() { return g_hooks.pool_static_pm; }
+int pool_chunk() { return g_hooks.pool_chunk; }
 #else
 constexpr bool force_simt() { return false; }
 constexpr int64_t split_select_min_cols() { return kSplitSelectMinCols; }
 constexpr uint32_t test_scan_wait_extra() { return 0u; }
 constexpr bool allow_cluster_topk() { return true; }
+constexpr int pool_static_pm() { return kPoolStaticPm; }
+constexpr int pool_chunk() { return kPoolChunk; }
 #endif
 
 bool valid_dims(const lsa_dims* d) {
@@ -247,7 +259,8 @@ lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const 
                      const int32_t* row_pos, const void* q_idx, const float* w, float* scores,
                      int64_t ld, void* ws, void* inner_ws, size_t inner_bytes, cudaStream_t s,
                      uint32_t* hist12 = nullptr, bool* hist_done = nullptr, uint32_t* done_ctr = nullptr,
-                     bool zeroed = false, bool pdl = false, const ScoresArgs* split = nullptr) {
+                     bool zeroed = false, bool pdl = false, const ScoresArgs* split = nullptr,
+                     int* pool = nullptr) {
   ScoresArgs a = scores_args(d, c, rows, row_seq, row_pos, q_idx, w, scores, ld, ws, inner_ws, inner_bytes);
   if (hist_done) *hist_done = false;
   if (rows == 0 || ld == 0) return LSA_OK;
@@ -268,6 +281,11 @@ lsa_status do_scores(const lsa_dims* d, const lsa_cache* c, int32_t rows, const 
       a.hist12 = hist12;
       a.done_ctr = done_ctr;  // zeroed with the histograms
       if (hist_done) *hist_done = true;
+      if (pool && pool_static_pm() <= 1000 && scores_tc_pool_ok(a)) {  // the pool counter too
+        a.pool = pool;
+        a.pool_chunk = pool_chunk();
+        a.pool_static_pm = pool_static_pm();
+      }
     }
     return cuda_status(launch_scores_tc(a, s));
   }
@@ -469,9 +487,10 @@ static lsa_status decode_step_impl(const lsa_dims* d, const lsa_cache* c, const 
   // zeroed with it: the top-k starts once every scan CTA has counted itself,
   // the attention of a row once that row's selection is written.
   uint32_t *scan_done = nullptr, *sel_done = nullptr;
-  if (hist12) topk_step_flags(inner, B, c->max_len, &scan_done, &sel_done);
+  int* scan_pool = nullptr;
+  if (hist12) topk_step_flags(inner, B, c->max_len, &scan_done, &sel_done, &scan_pool);
   st = do_scores(d, c, B, nullptr, nullptr, q_idx, w, scores, ld, ws, inner, inner_bytes, s, hist12, &hist_done,
-                 scan_done);
+                 scan_done, false, false, nullptr, scan_pool);
   if (st != LSA_OK) return st;
   if (!mark(1)) return LSA_ERR_CUDA;
   // The top-k and the attention are launched as programmatic dependents of the
@@ -569,7 +588,8 @@ lsa_status lsa_decode_layers(const lsa_dims* d, int32_t n_layers, const lsa_cach
       uint32_t* hist12 = (!force_simt() && topk_v2_ok(c->max_len)) ? static_cast<uint32_t*>(tk) : nullptr;
       bool hist_done = false;
       uint32_t *scan_done = nullptr, *sel_done = nullptr;
-      if (hist12) topk_step_flags(tk, B, c->max_len, &scan_done, &sel_done);
+      int* scan_pool = nullptr;
+      if (hist12) topk_step_flags(tk, B, c->max_len, &scan_done, &sel_done, &scan_pool);
       if (overlap) {
         // The attention on the selection already made goes first.  The scan
         // follows as its programmatic dependent (it reads nothing the
@@ -618,7 +638,7 @@ lsa_status lsa_decode_layers(const lsa_dims* d, int32_t n_layers, const lsa_cach
                      hist_done ? scan_done : nullptr, hist_done ? target : 0u);
       } else {
         st = do_scores(d, c, B, nullptr, nullptr, q_idx[l], w[l], scores, ld, ws, tk, L.tk_bytes, s, hist12,
-                       &hist_done, scan_done);
+                       &hist_done, scan_done, false, false, nullptr, scan_pool);
         if (st != LSA_OK) return st;
         st = do_topk(scores, ld, B, c->seq_lens, c->max_len, d->top_k, sel[nxt], ws, tk, s, hist_done, true,
                      hist_done ? scan_done : nullptr, hist_done ? static_cast<uint32_t>(scan_tc_grid()) : 0u);
@@ -935,6 +955,12 @@ lsa_status lsa_test_set_hooks(int32_t force_simt_path, int64_t split_select_min_
   g_hooks.force_simt = force_simt_path != 0;
   g_hooks.split_select_min_cols = split_select_min_cols_ < 0 ? kSplitSelectMinCols : split_select_min_cols_;
   g_hooks.scan_wait_extra = scan_wait_extra;
+  return LSA_OK;
+}
+
+lsa_status lsa_test_set_scan_pool(int32_t static_pm, int32_t chunk) {
+  g_hooks.pool_static_pm = static_pm < 0 ? kPoolStaticPm : static_pm;
+  g_hooks.pool_chunk = chunk <= 0 ? kPoolChunk : chunk;
   return LSA_OK;
 }
 #endif

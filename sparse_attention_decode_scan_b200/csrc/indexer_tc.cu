@@ -158,6 +158,13 @@ size_t scores_tc_ws_bytes(int32_t, bool) { return 0; }
 
 bool scores_tc_fused_hist_ok(const ScoresArgs& a) { return a.row_pos == nullptr && scores_tc_supported(a); }
 
+bool scores_tc_pool_ok(const ScoresArgs& a) {
+  // tile indices and row starts are kept as 32-bit integers
+  const int64_t tiles_max = static_cast<int64_t>(a.rows) * ((a.cache.max_len + kTile - 1) / kTile);
+  return a.row_pos == nullptr && a.cand == nullptr && a.rows <= kPoolRows && tiles_max < (1LL << 31) &&
+         scores_tc_supported(a);
+}
+
 cudaError_t scan_tc_maps(const ScoresArgs& a, CUtensorMap* tmap, CUtensorMap* smap) { return make_maps(a, tmap, smap); }
 
 int scan_tc_grid() { return num_sms(); }

@@ -64,6 +64,13 @@ struct ScoresArgs {
   int split_part = 0;
   int split_free = 0;
   float split_busy_us = 0.f, split_tile_us = 1.f;
+  // Tensor-core decode scan (one query row per tile, rows <= 256): if set
+  // (zeroed by the caller), the CTAs share the first pool_static_pm
+  // thousandths of the tiles evenly and claim the rest from this counter in
+  // chunks of pool_chunk tiles, so that they end together.
+  int* pool = nullptr;
+  int pool_chunk = 0;
+  int pool_static_pm = 1000;
 };
 
 // ---- indexer
@@ -72,6 +79,8 @@ cudaError_t launch_scores_simt(const ScoresArgs& a, cudaStream_t s);
 bool scores_tc_shape_ok(int32_t key_dtype, int32_t q_dtype, int32_t H, int32_t dI, int32_t block_size);
 int scores_tc_launches(bool causal);
 bool scores_tc_supported(const ScoresArgs& a);
+// the pooled tile schedule applies: one query row per tile, rows <= 256
+bool scores_tc_pool_ok(const ScoresArgs& a);
 size_t scores_tc_ws_bytes(int32_t rows, bool causal);
 cudaError_t launch_scores_tc(const ScoresArgs& a, cudaStream_t s);
 // Candidate re-scoring on the tensor cores (a.cand set): shape and alignment
@@ -131,8 +140,10 @@ struct TopkArgs {
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 // The decode step's handoff words inside the top-k workspace (zeroed with its
-// head): the count of finished scan CTAs and the per-row selection flags.
-void topk_step_flags(void* ws, int32_t rows, int64_t n_cols, uint32_t** scan_done, uint32_t** sel_done);
+// head): the count of finished scan CTAs, the per-row selection flags and the
+// scan's tile pool counter.
+void topk_step_flags(void* ws, int32_t rows, int64_t n_cols, uint32_t** scan_done, uint32_t** sel_done,
+                     int** scan_pool = nullptr);
 // Collect segments per row and their length of the one-launch top-k for these
 // sizes; false on a CUDA error.
 bool topk_rows_plan(int32_t rows, int64_t n_cols, int* nseg, int64_t* seg_len);

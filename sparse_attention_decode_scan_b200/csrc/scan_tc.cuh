@@ -60,6 +60,12 @@ constexpr int warp_mma2() { return 3 + 4 * EG; }
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpQ = 2, kWarpEpi = 3;
 constexpr int kSmemLimit = 232448;
 constexpr int kBarrierId = 1;    // named barrier of the scan's threads (a fused block holds more threads)
+// Pooled schedule (decode): tiles claimed from a global counter reach the
+// other roles as segments through a ring of kRing slots; a pooled launch has
+// at most kPoolRows query rows (the planner's one row per thread).
+constexpr int kRing = 8;
+constexpr int kSlotInts = 8;     // r0, j0, n, b, tiles, vis (2 ints), spare
+constexpr int kPoolRows = kThreads;
 
 template <int NTH = kThreads>
 __device__ __forceinline__ void scan_sync() {
@@ -76,7 +82,9 @@ struct Cfg {
   static constexpr int kBoxBytes = kBoxRows * 128;
   static constexpr int kQKBlockBytes = kN * 128;                   // B: N rows x 128 B per K block
   static constexpr int kQBytes = kKBlocks * kQKBlockBytes;
-  static constexpr int kNQ = (QB == 1 && kFp8) ? 2 : 1;            // query operand buffers
+  // query operand buffers: decode stages the next group's (or segment's)
+  // query while the MMAs of the current one run
+  static constexpr int kNQ = QB == 1 ? 2 : 1;
   static constexpr int kWBytes = QB * kHeads * 4;
   static constexpr int kHistBytes = QB == 1 ? kTopkBins1 * 4 : 0;  // fused first top-k histogram (decode)
   // Per stage besides the keys: the key rows of its two boxes (written by the
@@ -85,8 +93,12 @@ struct Cfg {
   // rows whose position or block was out of range (4 words).
   static constexpr int kMetaBytes = 2 * 4 + (kFp8 ? 2 * kScaleSlot * 4 : 0) + (GATHER ? 8 * 4 : 0);
   static constexpr int kRawBytes = kFp8 ? QB * kHeads * kDim * 2 : 0;  // FP8: bf16 query rows before the split
-  static constexpr int kFixed = kNQ * kQBytes + kNQ * kWBytes + kRawBytes + kHistBytes + 512 /*barriers, scratch*/ +
-                                1024 /*align*/;
+  // pooled schedule (decode, TMA producer): the ring's barriers and slots and
+  // the rows' first tiles and visible positions
+  static constexpr bool kPool = QB == 1 && !GATHER;
+  static constexpr int kPoolBytes = kPool ? kRing * (2 * 8 + kSlotInts * 4) + 2 * kPoolRows * 4 : 0;
+  static constexpr int kFixed = kNQ * kQBytes + kNQ * kWBytes + kRawBytes + kHistBytes + 640 /*barriers, scratch*/ +
+                                kPoolBytes + 1024 /*align*/;
   static constexpr int kNSmax = (kSmemLimit - kFixed) / (kTileBytes + kMetaBytes);
   static constexpr int kNS = kNSmax > 12 ? 12 : kNSmax;            // key stages
   // FP8 decode: the query's hi and lo terms (rows 0-63 and 64-127 of the
@@ -111,9 +123,9 @@ struct Cfg {
   static_assert(!GATHER || (KDT == LSA_BF16 && QB == 1), "candidate gather: bf16 keys, one row per tile");
 };
 
-// Stages of the configurations that run: decode 6 (bf16) and 9 (FP8) tiles in
+// Stages of the configurations that run: decode 5 (bf16) and 9 (FP8) tiles in
 // flight, the causal prefill 5 (bf16, 4 rows per tile) and 9 (FP8, 2 rows).
-static_assert(Cfg<LSA_BF16, 1>::kNS == 6 && Cfg<LSA_FP8_E4M3, 1>::kNS == 9, "decode stages");
+static_assert(Cfg<LSA_BF16, 1>::kNS == 5 && Cfg<LSA_FP8_E4M3, 1>::kNS == 9, "decode stages");
 static_assert(Cfg<LSA_BF16, 4>::kNS == 5 && Cfg<LSA_FP8_E4M3, 2>::kNS == 9, "prefill stages");
 
 // ---------------------------------------------------------------- work items
@@ -195,6 +207,10 @@ struct Walker {
     g = group_at<QB>(a, r0);
     j = j0;
   }
+  __device__ void start(const Group& g0, int j0) {
+    g = g0;
+    j = j0;
+  }
   __device__ void next(const ScoresArgs& a) {
     if (++j < g.tiles) return;
     j = 0;
@@ -235,6 +251,7 @@ struct Plan {
   int r_first;  // leader row of the CTA's first item
   int j_first;
   int64_t n_items;
+  int64_t pool_lo, pool_hi;  // pooled launch: the tiles claimed from the pool
 };
 
 // The tiles [lo, hi) of `tot` that this launch covers (ScoresArgs::split_part).
@@ -250,21 +267,41 @@ __device__ __forceinline__ void launch_tiles(const ScoresArgs& a, int64_t tot, i
 }
 
 // Every thread of the CTA takes part: total tiles, this CTA's share, and the
-// group holding its first tile.
+// group holding its first tile.  A pooled launch (pool_start set: one query
+// row per tile, at most kPoolRows rows) splits its first pool_static_pm
+// thousandths of the tiles evenly over the CTAs and leaves the rest to the
+// pool; pool_start[r] receives row r's first tile in the launch's order and
+// pool_start[kPoolRows + r] its visible positions.
 template <int QB, int NTH = kThreads>
-__device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound) {
+__device__ Plan plan_work(const ScoresArgs& a, int64_t* sbuf, int* sfound, int* pool_start = nullptr) {
   Plan p;
   p.r_first = 0;
   p.j_first = 0;
+  p.pool_lo = p.pool_hi = 0;
   if (a.rows <= NTH) {  // one row per thread: a single block scan
     const int r = threadIdx.x;
-    int64_t t = 0;
-    if (r < a.rows && is_leader<QB>(a, r)) t = group_at<QB>(a, r).tiles;
+    int64_t t = 0, vis = 0;
+    if (r < a.rows && is_leader<QB>(a, r)) {
+      const Group g = group_at<QB>(a, r);
+      t = g.tiles;
+      vis = g.vis;
+    }
     int64_t incl, tot;
     block_sum_i64_scan<NTH>(t, sbuf, &incl, &tot);
     // this launch's tiles [lo, hi), split evenly over its CTAs
     int64_t lo, hi;
     launch_tiles(a, tot, &lo, &hi);
+    if (pool_start) {
+      // row r's first tile, then (kPoolRows further on) its visible positions
+      if (r < a.rows) {
+        pool_start[r] = static_cast<int>(incl - t);
+        pool_start[kPoolRows + r] = static_cast<int>(vis);
+      }
+      lo = 0;
+      hi = tot * a.pool_static_pm / 1000;
+      p.pool_lo = hi;
+      p.pool_hi = tot;
+    }
     const int64_t t0 = lo + (hi - lo) * blockIdx.x / gridDim.x;
     p.n_items = lo + (hi - lo) * (blockIdx.x + 1) / gridDim.x - t0;
     if (p.n_items <= 0) return p;
@@ -548,14 +585,15 @@ __device__ void gather_producer(const ScoresArgs& a, const Plan& plan, const Cac
                                rv >= 0 ? 16u : 0u);
         }
       }
-      cp_async_arrive_noinc(&full[s]);
+      uint64_t* fb = &full[it % (2 * C::kNS)];  // the item's full barrier (see scan_cta)
+      cp_async_arrive_noinc(fb);
       if (lane == 0) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           smask[8 * s + m] = have[m];
           smask[8 * s + 4 + m] = bad[m];
         }
-        tc::mbar_arrive(&full[s]);  // release: the masks are visible to the epilogue's acquire
+        tc::mbar_arrive(fb);  // release: the masks are visible to the epilogue's acquire
       }
       ++it;
     }
@@ -591,8 +629,14 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   uint32_t* smask = reinterpret_cast<uint32_t*>(smeta + 2 * C::kNS);  // gather: [kNS][8]
   uint32_t* shist = smask + (GATHER ? 8 * C::kNS : 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(shist) + C::kHistBytes);
+  // Item it fills stage it % kNS and signals full[it % (2 kNS)]: with two MMA
+  // issuers (and two epilogue groups) taking alternate items, successive uses
+  // of one stage alternate between them whenever kNS is odd, and a waiter on
+  // a shared barrier could then test a phase one ahead of the one completing
+  // (the parity would read "done").  Over 2 kNS barriers each barrier's uses
+  // are 2 kNS items apart: the same issuer and group wait for every phase.
   uint64_t* full = bars;
-  uint64_t* empty = full + C::kNS;
+  uint64_t* empty = full + 2 * C::kNS;
   uint64_t* qfull = empty + C::kNS;
   uint64_t* qempty = qfull + C::kNQ;
   uint64_t* tfull = qempty + C::kNQ;
@@ -601,8 +645,15 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   uint64_t* ebar = done + 1;  // epilogue warps' rendezvous around histogram flushes
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ebar + 1);
   int* sfound = const_cast<int*>(abort_flag) + 1;                       // 2 ints
-  int64_t* sbuf = reinterpret_cast<int64_t*>(sfound + 2 + 1);           // kThreads/32 int64 (8-aligned below)
+  int64_t* sbuf = reinterpret_cast<int64_t*>(sfound + 2 + 1);           // NTH/32 int64 (8-aligned below)
   sbuf = reinterpret_cast<int64_t*>((reinterpret_cast<uintptr_t>(sbuf) + 7) & ~uintptr_t(7));
+  // pooled schedule: the ring (kRing segments: barriers, then slots of
+  // kSlotInts ints) and the rows' first tiles and visible positions
+  uint64_t* rfull = reinterpret_cast<uint64_t*>(sbuf + NTH / 32);
+  uint64_t* rempty = rfull + kRing;
+  int* rslot = reinterpret_cast<int*>(rempty + kRing);
+  int* pool_start = rslot + kRing * kSlotInts;  // [2][kPoolRows]
+  const bool pooled = C::kPool && a.pool != nullptr && a.pool_chunk > 0 && a.rows <= kPoolRows;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // a decode step's top-k may be scheduled onto SMs this launch frees (it
@@ -612,11 +663,12 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   // contiguous bf16 cache needs neither, and its stages free at MMA completion.
   const bool stage_meta = C::kFp8 || a.cache.block_size > 0 || GATHER;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kNS; ++s) {
+    for (int s = 0; s < 2 * C::kNS; ++s) {
       // gather: one cp.async completion per producer lane, plus lane 0's masks
       tc::mbar_init(&full[s], GATHER ? 32 + 1 : 1);
-      tc::mbar_init(&empty[s], stage_meta ? 1 + 4 : 1);  // MMA commit (+ 4 epilogue warps done with the stage)
     }
+    for (int s = 0; s < C::kNS; ++s)
+      tc::mbar_init(&empty[s], stage_meta ? 1 + 4 : 1);  // MMA commit (+ 4 epilogue warps done with the stage)
     for (int s = 0; s < C::kNQ; ++s) {
       tc::mbar_init(&qfull[s], 1);
       tc::mbar_init(&qempty[s], 2 + 4 * EG);  // both MMA issuers' commits + every epilogue warp
@@ -627,6 +679,12 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     }
     tc::mbar_init(done, 2);  // both MMA issuers
     tc::mbar_init(ebar, 4 * EG);
+    if (pooled) {
+      for (int s = 0; s < kRing; ++s) {
+        tc::mbar_init(&rfull[s], 1);            // the producer's publication
+        tc::mbar_init(&rempty[s], 3 + 4 * EG);  // both MMA issuers, the query warp, every epilogue warp
+      }
+    }
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -634,11 +692,29 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     tc::prefetch_tmap(&tmap);
     if (C::kFp8) tc::prefetch_tmap(&smap);
   }
-  const Plan plan = plan_work<QB, NTH>(a, sbuf, sfound);
+  const Plan plan = plan_work<QB, NTH>(a, sbuf, sfound, pooled ? pool_start : nullptr);
   scan_sync<NTH>();
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   CacheAddr ad{a.cache.block_table, a.cache.max_blocks, a.cache.block_size, a.cache.n_blocks, a.cache.max_len};
+  // Pooled segment k (k = 0, 1, ...) from the ring into a walker and its item
+  // count (0: no more); every calling thread reads it, and each consumer
+  // releases the slot afterwards (ring_release, once per consumer).
+  auto ring_take = [&](int k, Walker<QB>* w, int64_t* n) -> bool {
+    const int s = k % kRing;
+    if (!tc::mbar_wait(&rfull[s], static_cast<uint32_t>((k / kRing) & 1), abort_flag)) return false;
+    const volatile int* sl = rslot + s * kSlotInts;
+    Group g;
+    g.r0 = sl[0];
+    g.nrows = 1;
+    g.b = sl[3];
+    g.tiles = sl[4];
+    g.vis = static_cast<int64_t>(static_cast<uint32_t>(sl[5])) | (static_cast<int64_t>(sl[6]) << 32);
+    w->start(g, sl[1]);
+    *n = sl[2];
+    return true;
+  };
+  auto ring_release = [&](int k) { tc::mbar_arrive(&rempty[k % kRing]); };
 
   if (GATHER && warp == kWarpProd) {
     gather_producer<C>(a, plan, ad, stages, smask, full, empty, abort_flag, lane);
@@ -648,20 +724,28 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
     // entries are loaded before the current batch is issued and only read
     // after it, so their latency hides behind the 32 issues; a single thread
     // doing the lookups serially would wait one load latency per tile.
-    if (plan.n_items > 0) {
+    // A pooled launch continues past the CTA's static share with chunks of
+    // pool_chunk tiles claimed from the pool: the claim for the next chunk is
+    // made when the current segment's last batch starts, and the chunk is
+    // mapped to its row, published to the other roles and looked up halfway
+    // through that batch's issues.
+    if (plan.n_items > 0 || pooled) {
       struct Look {
         int64_t p0, vis;  // first position of the tile; visible positions of its group
         int b, r0;
         int32_t blk[2];   // block-table entries of the tile's two boxes (paged cache)
         bool live;
       };
-      auto look = [&](const Walker<QB>& base, int64_t base_item) -> Look {
-        Walker<QB> w = base;
-        if (w.j + lane < w.g.tiles) w.j += lane;  // same group: no walk
-        else
-          for (int i = 0; i < lane; ++i) w.next(a);
+      // lanes [0, left) take the items base, base + 1, ...
+      auto look = [&](const Walker<QB>& base, int64_t left) -> Look {
         Look L;
-        L.live = base_item + lane < plan.n_items;
+        L.live = lane < left;
+        Walker<QB> w = base;
+        if (L.live) {
+          if (w.j + lane < w.g.tiles) w.j += lane;  // same group: no walk
+          else
+            for (int i = 0; i < lane; ++i) w.next(a);
+        }
         L.p0 = static_cast<int64_t>(w.j) * kTile;
         L.vis = w.g.vis;
         L.b = w.g.b;
@@ -701,180 +785,288 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
           rows[h] = r;
         }
       };
+      int claim = 0;  // lane 0: the chunk index returned by the last claim
+      int k_pub = 0;  // pooled segments published
+      // The claimed chunk as the next segment (0 items: the pool is empty),
+      // published to the other roles; false on a timeout.
+      auto next_pooled = [&](Walker<QB>* w, int64_t* n) -> bool {
+        int r0 = 0, j0 = 0, nn = 0;
+        if (lane == 0) {
+          const int64_t t0 = plan.pool_lo + static_cast<int64_t>(claim) * a.pool_chunk;
+          if (t0 < plan.pool_hi) {
+            nn = plan.pool_hi - t0 < a.pool_chunk ? static_cast<int>(plan.pool_hi - t0) : a.pool_chunk;
+            // the row holding tile t0: the last row starting at or before it
+            int lo = 0, hi = a.rows - 1;
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (pool_start[mid] <= t0) lo = mid;
+              else hi = mid - 1;
+            }
+            r0 = lo;
+            j0 = static_cast<int>(t0 - pool_start[lo]);
+          }
+        }
+        r0 = __shfl_sync(0xffffffffu, r0, 0);
+        j0 = __shfl_sync(0xffffffffu, j0, 0);
+        nn = __shfl_sync(0xffffffffu, nn, 0);
+        Group g;
+        g.r0 = r0;
+        g.nrows = 1;
+        g.b = seq_of(a, r0);
+        g.vis = pool_start[kPoolRows + r0];
+        g.tiles = static_cast<int>((g.vis + kTile - 1) / kTile);
+        bool ok = true;
+        if (lane == 0) {
+          const int s = k_pub % kRing;
+          ok = tc::mbar_wait(&rempty[s], static_cast<uint32_t>(((k_pub / kRing) & 1) ^ 1), abort_flag);
+          if (ok) {
+            int* sl = rslot + s * kSlotInts;
+            sl[0] = g.r0;
+            sl[1] = j0;
+            sl[2] = nn;
+            sl[3] = g.b;
+            sl[4] = g.tiles;
+            sl[5] = static_cast<int>(static_cast<uint32_t>(g.vis));
+            sl[6] = static_cast<int>(g.vis >> 32);
+            tc::mbar_arrive(&rfull[s]);  // release: the slot is visible to the consumers' acquire
+          } else {
+            record_error(a.status, LSA_ERR_TIMEOUT, 0, 10);
+            *abort_flag = 1;
+          }
+        }
+        ++k_pub;
+        w->start(g, j0);
+        *n = nn;
+        return __shfl_sync(0xffffffffu, ok, 0);
+      };
       // decode streams each key once per step: evict it first; the causal
       // prefill reads every key once per group of query rows: keep it
       const uint64_t l2_policy = a.row_pos ? tc::l2_evict_last_policy() : tc::l2_evict_first_policy();
-      Walker<QB> Wb;
-      Wb.start(a, plan.r_first, plan.j_first);
-      Look cur = look(Wb, 0);
       int64_t it = 0;
       bool failed = false;
-      for (int64_t base_item = 0; base_item < plan.n_items && !failed; base_item += 32) {
+      // Issues item i of the batch whose key rows the lanes hold; false on a timeout.
+      auto issue = [&](const int64_t* cur_rows, int i) -> bool {
+        const int64_t rows[2] = {__shfl_sync(0xffffffffu, cur_rows[0], i), __shfl_sync(0xffffffffu, cur_rows[1], i)};
+        bool bad = false;
+        if (lane == 0) {
+          const int s = static_cast<int>(it % C::kNS);
+          const uint32_t ph = static_cast<uint32_t>((it / C::kNS) & 1);
+          uint64_t* fb = &full[it % (2 * C::kNS)];
+          if (!tc::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+            record_error(a.status, LSA_ERR_TIMEOUT, 0, 1);
+            *abort_flag = 1;
+            bad = true;
+          } else {
+            uint32_t bytes = 0;
+            for (int h = 0; h < 2; ++h)
+              if (rows[h] >= 0) bytes += C::kKBlocks * C::kBoxBytes + (C::kFp8 ? kScaleBox * 4 : 0);
+            smeta[2 * s] = static_cast<int32_t>(rows[0]);  // published to the epilogue by the full barrier
+            smeta[2 * s + 1] = static_cast<int32_t>(rows[1]);
+            tc::mbar_arrive_expect_tx(fb, bytes);
+            uint8_t* st = stages + s * C::kTileBytes;
+            for (int h = 0; h < 2; ++h) {
+              if (rows[h] < 0) continue;
+              for (int kb = 0; kb < C::kKBlocks; ++kb)
+                tc::tma_load_2d_hint(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * kBoxX,
+                                     static_cast<int32_t>(rows[h]), fb, l2_policy);
+              // the box's 64 scales, from the 16-byte aligned row at or below its first
+              if (C::kFp8)
+                tc::tma_load_1d(sscale + (2 * s + h) * kScaleSlot, &smap, static_cast<int32_t>(rows[h] & ~int64_t(3)),
+                                fb);
+            }
+            ++it;
+          }
+        }
+        return !__shfl_sync(0xffffffffu, bad, 0);
+      };
+      Walker<QB> Wb;
+      int64_t left = plan.n_items;  // items of the current segment from Wb on
+      if (left > 0) {
+        Wb.start(a, plan.r_first, plan.j_first);
+      } else {  // no static share: the first segment comes from the pool
+        if (lane == 0) claim = atomicAdd(a.pool, 1);
+        failed = !next_pooled(&Wb, &left);
+      }
+      Look cur = look(Wb, left);
+      while (left > 0 && !failed) {
         int64_t cur_rows[2];
         resolve(cur, cur_rows);
+        const int nb = static_cast<int>(left < 32 ? left : 32);
+        // The next batch: the rest of this segment, else the next pooled
+        // segment (claimed now, mapped after the first half of the issues).
+        const bool to_pool = pooled && nb == left;
+        if (to_pool && lane == 0) claim = atomicAdd(a.pool, 1);
+        const int h = to_pool ? (nb + 1) / 2 : 0;
+        for (int i = 0; i < h && !failed; ++i) failed = !issue(cur_rows, i);
         Walker<QB> Wn = Wb;
-        if (Wn.j + 32 < Wn.g.tiles) Wn.j += 32;
-        else
-          for (int i = 0; i < 32; ++i) Wn.next(a);
-        const Look nxt = look(Wn, base_item + 32);  // loads stay in flight during the issues below
-        const int nb = static_cast<int>(plan.n_items - base_item < 32 ? plan.n_items - base_item : 32);
-        for (int i = 0; i < nb; ++i) {
-          const int64_t rows[2] = {__shfl_sync(0xffffffffu, cur_rows[0], i), __shfl_sync(0xffffffffu, cur_rows[1], i)};
-          if (lane == 0) {
-            const int s = static_cast<int>(it % C::kNS);
-            const uint32_t ph = static_cast<uint32_t>((it / C::kNS) & 1);
-            if (!tc::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
-              record_error(a.status, LSA_ERR_TIMEOUT, 0, 1);
-              *abort_flag = 1;
-              failed = true;
-            } else {
-              uint32_t bytes = 0;
-              for (int h = 0; h < 2; ++h)
-                if (rows[h] >= 0) bytes += C::kKBlocks * C::kBoxBytes + (C::kFp8 ? kScaleBox * 4 : 0);
-              smeta[2 * s] = static_cast<int32_t>(rows[0]);  // published to the epilogue by full[s]
-              smeta[2 * s + 1] = static_cast<int32_t>(rows[1]);
-              tc::mbar_arrive_expect_tx(&full[s], bytes);
-              uint8_t* st = stages + s * C::kTileBytes;
-              for (int h = 0; h < 2; ++h) {
-                if (rows[h] < 0) continue;
-                for (int kb = 0; kb < C::kKBlocks; ++kb)
-                  tc::tma_load_2d_hint(st + kb * C::kKBlockBytes + h * C::kBoxBytes, &tmap, kb * kBoxX,
-                                       static_cast<int32_t>(rows[h]), &full[s], l2_policy);
-                // the box's 64 scales, from the 16-byte aligned row at or below its first
-                if (C::kFp8)
-                  tc::tma_load_1d(sscale + (2 * s + h) * kScaleSlot, &smap, static_cast<int32_t>(rows[h] & ~int64_t(3)),
-                                  &full[s]);
-              }
-              ++it;
-            }
-          }
-          failed = __shfl_sync(0xffffffffu, failed, 0);
-          if (failed) break;
+        int64_t nleft = left - nb;
+        if (failed) break;
+        if (nleft > 0) {
+          if (Wn.j + 32 < Wn.g.tiles) Wn.j += 32;
+          else
+            for (int i = 0; i < 32; ++i) Wn.next(a);
+        } else if (to_pool) {
+          if (!next_pooled(&Wn, &nleft)) break;
         }
+        const Look nxt = look(Wn, nleft);  // loads stay in flight during the issues below
+        for (int i = h; i < nb && !failed; ++i) failed = !issue(cur_rows, i);
         Wb = Wn;
+        left = nleft;
         cur = nxt;
       }
       // drain: the last load of every stage must land before the CTA exits
       if (lane == 0) {
         const int64_t n_issued = it;
         for (int64_t i = n_issued > C::kNS ? n_issued - C::kNS : 0; i < n_issued; ++i)
-          tc::mbar_wait(&full[i % C::kNS], static_cast<uint32_t>((i / C::kNS) & 1), nullptr);
+          tc::mbar_wait(&full[i % (2 * C::kNS)], static_cast<uint32_t>((i / (2 * C::kNS)) & 1), nullptr);
       }
     }
   } else if (warp == kWarpMma || warp == warp_mma2<EG>()) {
     // issuer `who` takes the tiles it with it % 2 == who, into accumulator it % kAcc
     const int who = warp == kWarpMma ? 0 : 1;
-    if (lane == 0 && plan.n_items > 0) {
+    if (lane == 0 && (plan.n_items > 0 || pooled)) {
       Walker<QB> W;
-      W.start(a, plan.r_first, plan.j_first);
+      int64_t n = plan.n_items;  // items of the current segment
+      if (n > 0) W.start(a, plan.r_first, plan.j_first);
       int gi = -1;
       int qi = 0;
       // An issuer shares its SM sub-partition with epilogue warps, so its
       // per-tile work is kept small: the stage and its phase advance
-      // incrementally (no 64-bit
-      // division per tile), and a tile's descriptors are the first stage's
-      // and query buffer's plus constant offsets in the start-address field
-      // (shared-memory addresses stay below 256 KB: adding never carries out
-      // of that 14-bit field).
-      int s = 0;
-      uint32_t sph = 0;
+      // incrementally (no 64-bit division per tile), and a tile's descriptors
+      // are the first stage's and query buffer's plus constant offsets in the
+      // start-address field (shared-memory addresses stay below 256 KB: adding
+      // never carries out of that 14-bit field).
+      int s = 0, fbi = 0;       // the item's stage and full barrier
+      uint32_t fph = 0;         // and the barrier's phase
       const uint64_t a_desc0 = tc::desc_sw128(tc::smem_u32(stages));
       const uint64_t b_desc0 = tc::desc_sw128(tc::smem_u32(qbufs));
-      for (int64_t it = 0; it < plan.n_items; ++it) {
-        if (it == 0 || W.j == 0) {
-          ++gi;
-          qi = gi % C::kNQ;
-          if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) goto mma_fail;
-        }
-        if (static_cast<int>(it & 1) == who) {
-          if (!tc::mbar_wait(&full[s], sph, abort_flag)) goto mma_fail;
-          // gathered rows were written by cp.async (generic proxy); the MMA reads them through the async proxy
-          if (GATHER) tc::fence_proxy_async_smem();
-          const int acc = static_cast<int>(it % C::kAcc);
-          if (!tc::mbar_wait(&tempty[acc], static_cast<uint32_t>(((it / C::kAcc) & 1) ^ 1), abort_flag)) goto mma_fail;
-          tc::tc_fence_after();
-          const uint32_t d = tmem_base + acc * C::kAccCols;
-          const uint64_t ad0 = a_desc0 + static_cast<uint64_t>((s * C::kTileBytes) >> 4);
-          const uint64_t bd0 = b_desc0 + static_cast<uint64_t>((qi * C::kQBytes) >> 4);
-          if (C::kCat) {
-            // D = K q_hi + K q_lo: the query operand's rows 64-127 start 8 KB in
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const uint64_t ad_ = ad0 + static_cast<uint64_t>((k * 32) >> 4);
-                const uint64_t bd_ = bd0 + static_cast<uint64_t>((part * kHeads * 128 + k * 32) >> 4);
-                tc::mma_f8(d, ad_, bd_, C::kIdesc, (part | k) != 0);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int kb = 0; kb < C::kKBlocks; ++kb) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const uint64_t ad_ = ad0 + static_cast<uint64_t>((kb * C::kKBlockBytes + k * 32) >> 4);
-                const uint64_t bd_ = bd0 + static_cast<uint64_t>((kb * C::kQKBlockBytes + k * 32) >> 4);
-                if (C::kFp8) tc::mma_f8(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
-                else tc::mma_f16(d, ad_, bd_, C::kIdesc, (kb | k) != 0);
-              }
+      int64_t it = 0;  // items of every segment so far
+      bool fail = false;
+      for (int k = 0;; ++k) {
+        for (int64_t i = 0; i < n; ++i, ++it) {
+          if (i == 0 || W.j == 0) {
+            ++gi;
+            qi = gi % C::kNQ;
+            if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) {
+              fail = true;
+              break;
             }
           }
-          tc::mma_commit(&empty[s]);
-          tc::mma_commit(&tfull[acc]);
-        }
-        {
-          if (++s == C::kNS) {
-            s = 0;
-            sph ^= 1u;
+          if (static_cast<int>(it & 1) == who) {
+            if (!tc::mbar_wait(&full[fbi], fph, abort_flag)) {
+              fail = true;
+              break;
+            }
+            // gathered rows were written by cp.async (generic proxy); the MMA reads them through the async proxy
+            if (GATHER) tc::fence_proxy_async_smem();
+            const int acc = static_cast<int>(it % C::kAcc);
+            if (!tc::mbar_wait(&tempty[acc], static_cast<uint32_t>(((it / C::kAcc) & 1) ^ 1), abort_flag)) {
+              fail = true;
+              break;
+            }
+            tc::tc_fence_after();
+            const uint32_t d = tmem_base + acc * C::kAccCols;
+            const uint64_t ad0 = a_desc0 + static_cast<uint64_t>((s * C::kTileBytes) >> 4);
+            const uint64_t bd0 = b_desc0 + static_cast<uint64_t>((qi * C::kQBytes) >> 4);
+            if (C::kCat) {
+              // D = K q_hi + K q_lo: the query operand's rows 64-127 start 8 KB in
+#pragma unroll
+              for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t ad_ = ad0 + static_cast<uint64_t>((kk * 32) >> 4);
+                  const uint64_t bd_ = bd0 + static_cast<uint64_t>((part * kHeads * 128 + kk * 32) >> 4);
+                  tc::mma_f8(d, ad_, bd_, C::kIdesc, (part | kk) != 0);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int kb = 0; kb < C::kKBlocks; ++kb) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t ad_ = ad0 + static_cast<uint64_t>((kb * C::kKBlockBytes + kk * 32) >> 4);
+                  const uint64_t bd_ = bd0 + static_cast<uint64_t>((kb * C::kQKBlockBytes + kk * 32) >> 4);
+                  if (C::kFp8) tc::mma_f8(d, ad_, bd_, C::kIdesc, (kb | kk) != 0);
+                  else tc::mma_f16(d, ad_, bd_, C::kIdesc, (kb | kk) != 0);
+                }
+              }
+            }
+            tc::mma_commit(&empty[s]);
+            tc::mma_commit(&tfull[acc]);
+          }
+          if (++s == C::kNS) s = 0;
+          if (++fbi == 2 * C::kNS) {
+            fbi = 0;
+            fph ^= 1u;
           }
           // both issuers release the group's query buffer after its last tile
-          // (a commit covers every MMA its thread issued before it)
-          const int jn = W.j + 1;
-          if (it + 1 == plan.n_items || jn >= W.g.tiles) tc::mma_commit(&qempty[qi]);
-          W.next(a);
+          // of the segment (a commit covers every MMA its thread issued before it)
+          if (i + 1 == n || W.j + 1 >= W.g.tiles) tc::mma_commit(&qempty[qi]);
+          if (i + 1 < n) W.next(a);
         }
-        continue;
-      mma_fail:
+        if (fail || !pooled) break;
+        if (!ring_take(k, &W, &n)) {
+          fail = true;
+          break;
+        }
+        ring_release(k);
+        if (n == 0) break;
+      }
+      if (fail) {
         record_error(a.status, LSA_ERR_TIMEOUT, 0, 2);
         *abort_flag = 1;
-        break;
       }
       tc::mma_commit(done);
       tc::mbar_wait(done, 0, nullptr);  // both issuers' MMAs complete
       // The releases of the last stages and query buffer arrive asynchronously
       // too; they must land before the barriers are invalidated.
       if (who == 0 && !*abort_flag) {
-        const int64_t n = plan.n_items;
-        for (int64_t i = n > C::kNS ? n - C::kNS : 0; i < n; ++i)
+        for (int64_t i = it > C::kNS ? it - C::kNS : 0; i < it; ++i)
           tc::mbar_wait(&empty[i % C::kNS], static_cast<uint32_t>((i / C::kNS) & 1), abort_flag);
         if (gi >= 0) tc::mbar_wait(&qempty[gi % C::kNQ], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag);
       }
     }
   } else if (warp == kWarpQ) {
-    if (plan.n_items > 0) {
+    if (plan.n_items > 0 || pooled) {
       Walker<QB> W;
-      W.start(a, plan.r_first, plan.j_first);
+      int64_t n = plan.n_items;  // items of the current segment
+      if (n > 0) W.start(a, plan.r_first, plan.j_first);
       int gi = -1;
-      for (int64_t it = 0; it < plan.n_items; ++it) {
-        if (it == 0 || W.j == 0) {
-          ++gi;
-          const int qi = gi % C::kNQ;
-          if (!tc::mbar_wait(&qempty[qi], static_cast<uint32_t>(((gi / C::kNQ) & 1) ^ 1), abort_flag)) {
-            if (lane == 0) {
-              record_error(a.status, LSA_ERR_TIMEOUT, 0, 3);
-              *abort_flag = 1;
+      bool fail = false;
+      for (int k = 0;; ++k) {
+        for (int64_t i = 0; i < n; ++i) {
+          if (i == 0 || W.j == 0) {
+            ++gi;
+            const int qi = gi % C::kNQ;
+            if (!tc::mbar_wait(&qempty[qi], static_cast<uint32_t>(((gi / C::kNQ) & 1) ^ 1), abort_flag)) {
+              if (lane == 0) {
+                record_error(a.status, LSA_ERR_TIMEOUT, 0, 3);
+                *abort_flag = 1;
+              }
+              fail = true;
+              break;
             }
-            break;
+            uint8_t* qb = qbufs + qi * C::kQBytes;
+            float* wb = wbufs + qi * (C::kWBytes / 4);
+            if (C::kFp8) stage_query_fp8<QB>(a, W.g, qb, wb, qraw, lane);
+            else stage_query_bf16<QB>(a, W.g, qb, wb, lane);
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&qfull[qi]);
           }
-          uint8_t* qb = qbufs + qi * C::kQBytes;
-          float* wb = wbufs + qi * (C::kWBytes / 4);
-          if (C::kFp8) stage_query_fp8<QB>(a, W.g, qb, wb, qraw, lane);
-          else stage_query_bf16<QB>(a, W.g, qb, wb, lane);
-          tc::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&qfull[qi]);
+          if (i + 1 < n) W.next(a);
         }
-        W.next(a);
+        if (fail || !pooled) break;
+        if (!ring_take(k, &W, &n)) {
+          if (lane == 0) {
+            record_error(a.status, LSA_ERR_TIMEOUT, 0, 11);
+            *abort_flag = 1;
+          }
+          break;
+        }
+        __syncwarp();
+        if (lane == 0) ring_release(k);
+        if (n == 0) break;
       }
     }
   } else if (warp < kWarpEpi + 4 * EG) {
@@ -940,146 +1132,173 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       for (int64_t i = et; i < nvec; i += 128 * EG) v4[i] = make_float4(val, val, val, val);
       for (int64_t p = head + nvec * 4 + et; p < a.ld; p += 128 * EG) row[p] = val;
     }
-    if (plan.n_items > 0) {
+    if (plan.n_items > 0 || pooled) {
       Walker<QB> W;
-      W.start(a, plan.r_first, plan.j_first);
+      int64_t n = plan.n_items;  // items of the current segment
+      if (n > 0) W.start(a, plan.r_first, plan.j_first);
       int gi = -1, qi = 0;
       int hist_row = -1;
       int64_t vis_r[QB];
-      int stg = 0;        // stage of item it
-      uint32_t sph = 0;   // and its phase
-      for (int64_t it = 0; it < plan.n_items; ++it) {
-        if (it == 0 || W.j == 0) {
-          ++gi;
-          qi = gi % C::kNQ;
-          if (use_hist && hist_row >= 0 && !flush_hist(hist_row)) {
-            if (lane == 0) {
-              record_error(a.status, LSA_ERR_TIMEOUT, 0, 6);
-              *abort_flag = 1;
-            }
-            hist_row = -1;
-            break;
-          }
-          hist_row = W.g.r0;
-          if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) {
-            if (lane == 0) {
-              record_error(a.status, LSA_ERR_TIMEOUT, 0, 4);
-              *abort_flag = 1;
-            }
-            hist_row = -1;
-            break;
-          }
-#pragma unroll
-          for (int qq = 0; qq < QB; ++qq) {
-            int bb;
-            vis_r[qq] = qq < W.g.nrows ? row_visible(a, W.g.r0 + qq, &bb) : 0;
-          }
-        }
-        // the other group's tiles are only walked past (both groups release
-        // every query buffer: the weights are read by either)
-        const bool mine = EG == 1 || static_cast<int>(it % EG) == eg;
-        if (mine) {
-          const int acc = static_cast<int>(it % C::kAcc);
-          if (!tc::mbar_wait(&tfull[acc], static_cast<uint32_t>((it / C::kAcc) & 1), abort_flag)) {
-            if (lane == 0) {
-              record_error(a.status, LSA_ERR_TIMEOUT, 0, 5);
-              *abort_flag = 1;
-            }
-            hist_row = -1;
-            break;
-          }
-          tc::tc_fence_after();
-          // The tile's key rows (and FP8 scales) come from the producer through
-          // the stage; the stage is released once all four warps have read them.
-          int32_t mrow = 0;  // contiguous bf16: every visible position has a key row
-          float kscale = 1.f;
-          if (stage_meta) {
-            if (!tc::mbar_wait(&full[stg], sph, abort_flag)) {
+      int stg = 0, fbi = 0;  // stage of item it and its full barrier
+      uint32_t fph = 0;      // and the barrier's phase
+      int64_t it = 0;     // items of every segment so far
+      bool fail = false;
+      for (int k = 0;; ++k) {
+        for (int64_t si = 0; si < n; ++si, ++it) {
+          if (si == 0 || W.j == 0) {
+            ++gi;
+            qi = gi % C::kNQ;
+            // a new row: the counts of the one before go to its histogram
+            if (use_hist && hist_row >= 0 && hist_row != W.g.r0 && !flush_hist(hist_row)) {
               if (lane == 0) {
-                record_error(a.status, LSA_ERR_TIMEOUT, 0, 8);
+                record_error(a.status, LSA_ERR_TIMEOUT, 0, 6);
                 *abort_flag = 1;
               }
               hist_row = -1;
+              fail = true;
               break;
             }
-            if (GATHER) {
-              // row t has a key (0), is a padding entry (-3: -inf) or an out-of-range one (-1: NaN)
-              const uint32_t* mk = smask + 8 * stg;
-              mrow = ((mk[t >> 5] >> (t & 31)) & 1u) ? 0 : (((mk[4 + (t >> 5)] >> (t & 31)) & 1u) ? -1 : -3);
-            } else {
-              const int box = 2 * stg + (t >> 6);
-              mrow = smeta[box];
-              if (C::kFp8 && mrow >= 0) kscale = sscale[box * kScaleSlot + (mrow & 3) + (t & 63)];
+            hist_row = W.g.r0;
+            if (!tc::mbar_wait(&qfull[qi], static_cast<uint32_t>((gi / C::kNQ) & 1), abort_flag)) {
+              if (lane == 0) {
+                record_error(a.status, LSA_ERR_TIMEOUT, 0, 4);
+                *abort_flag = 1;
+              }
+              hist_row = -1;
+              fail = true;
+              break;
             }
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty[stg]);
-          }
-          const int64_t p = static_cast<int64_t>(W.j) * kTile + t;
-          const int64_t prow = mrow >= 0 ? static_cast<int64_t>(mrow) + (t & 63) : (GATHER && mrow == -3 ? -3 : -1);
-          const float* wb = wbufs + qi * (C::kWBytes / 4);
-          float sc[QB];
-  #pragma unroll
-          for (int qq = 0; qq < QB; ++qq) {
-            float s = 0.f;
-  #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              float v[32];
-              const uint32_t col =
-                  acc * C::kAccCols + (C::kFp8 && !C::kCat ? qq * 2 * kHeads : qq * kHeads) + c * 32;
-              tc::tmem_ld32(tmem_base + lane_base + col, v);
-              const float4* w4 = reinterpret_cast<const float4*>(wb + qq * kHeads + c * 32);
-              if (C::kFp8 && !C::kCat) {
-                float u[32];
-                tc::tmem_ld32(tmem_base + lane_base + col + kHeads, u);
-                tc::tmem_wait_ld();
-  #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float4 w = w4[i];
-                  s = fmaf(w.x, fmaxf(v[4 * i] + u[4 * i], 0.f), s);
-                  s = fmaf(w.y, fmaxf(v[4 * i + 1] + u[4 * i + 1], 0.f), s);
-                  s = fmaf(w.z, fmaxf(v[4 * i + 2] + u[4 * i + 2], 0.f), s);
-                  s = fmaf(w.w, fmaxf(v[4 * i + 3] + u[4 * i + 3], 0.f), s);
-                }
-              } else {
-                tc::tmem_wait_ld();
-  #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float4 w = w4[i];
-                  s = fmaf(w.x, fmaxf(v[4 * i], 0.f), s);
-                  s = fmaf(w.y, fmaxf(v[4 * i + 1], 0.f), s);
-                  s = fmaf(w.z, fmaxf(v[4 * i + 2], 0.f), s);
-                  s = fmaf(w.w, fmaxf(v[4 * i + 3], 0.f), s);
-                }
+            if (QB == 1) {
+              vis_r[0] = W.g.vis;  // the group's one row
+            } else {
+#pragma unroll
+              for (int qq = 0; qq < QB; ++qq) {
+                int bb;
+                vis_r[qq] = qq < W.g.nrows ? row_visible(a, W.g.r0 + qq, &bb) : 0;
               }
             }
-            sc[qq] = s * kscale;
           }
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&tempty[acc]);
-          if (use_hist && p < vis_r[0] && prow >= 0) {
-            const uint32_t key = order_key(sc[0]);
-            if (key) atomicAdd(&shist[key >> 20], 1u);
-          }
-  #pragma unroll
-          for (int qq = 0; qq < QB; ++qq) {
-            if (qq < W.g.nrows && p < a.ld) {
-              float o = -INFINITY;
-              if (p < vis_r[qq]) o = prow >= 0 ? sc[qq] : (prow == -3 ? -INFINITY : NAN);
-              a.scores[static_cast<int64_t>(W.g.r0 + qq) * a.ld + p] = o;
+          // the other group's tiles are only walked past (both groups release
+          // every query buffer: the weights are read by either)
+          const bool mine = EG == 1 || static_cast<int>(it % EG) == eg;
+          if (mine) {
+            const int acc = static_cast<int>(it % C::kAcc);
+            if (!tc::mbar_wait(&tfull[acc], static_cast<uint32_t>((it / C::kAcc) & 1), abort_flag)) {
+              if (lane == 0) {
+                record_error(a.status, LSA_ERR_TIMEOUT, 0, 5);
+                *abort_flag = 1;
+              }
+              hist_row = -1;
+              fail = true;
+              break;
+            }
+            tc::tc_fence_after();
+            // The tile's key rows (and FP8 scales) come from the producer through
+            // the stage; the stage is released once all four warps have read them.
+            int32_t mrow = 0;  // contiguous bf16: every visible position has a key row
+            float kscale = 1.f;
+            if (stage_meta) {
+              if (!tc::mbar_wait(&full[fbi], fph, abort_flag)) {
+                if (lane == 0) {
+                  record_error(a.status, LSA_ERR_TIMEOUT, 0, 8);
+                  *abort_flag = 1;
+                }
+                hist_row = -1;
+                fail = true;
+                break;
+              }
+              if (GATHER) {
+                // row t has a key (0), is a padding entry (-3: -inf) or an out-of-range one (-1: NaN)
+                const uint32_t* mk = smask + 8 * stg;
+                mrow = ((mk[t >> 5] >> (t & 31)) & 1u) ? 0 : (((mk[4 + (t >> 5)] >> (t & 31)) & 1u) ? -1 : -3);
+              } else {
+                const int box = 2 * stg + (t >> 6);
+                mrow = smeta[box];
+                if (C::kFp8 && mrow >= 0) kscale = sscale[box * kScaleSlot + (mrow & 3) + (t & 63)];
+              }
+              __syncwarp();
+              if (lane == 0) tc::mbar_arrive(&empty[stg]);
+            }
+            const int64_t p = static_cast<int64_t>(W.j) * kTile + t;
+            const int64_t prow = mrow >= 0 ? static_cast<int64_t>(mrow) + (t & 63) : (GATHER && mrow == -3 ? -3 : -1);
+            const float* wb = wbufs + qi * (C::kWBytes / 4);
+            float sc[QB];
+#pragma unroll
+            for (int qq = 0; qq < QB; ++qq) {
+              float s = 0.f;
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                float v[32];
+                const uint32_t col =
+                    acc * C::kAccCols + (C::kFp8 && !C::kCat ? qq * 2 * kHeads : qq * kHeads) + c * 32;
+                tc::tmem_ld32(tmem_base + lane_base + col, v);
+                const float4* w4 = reinterpret_cast<const float4*>(wb + qq * kHeads + c * 32);
+                if (C::kFp8 && !C::kCat) {
+                  float u[32];
+                  tc::tmem_ld32(tmem_base + lane_base + col + kHeads, u);
+                  tc::tmem_wait_ld();
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) {
+                    const float4 w = w4[i];
+                    s = fmaf(w.x, fmaxf(v[4 * i] + u[4 * i], 0.f), s);
+                    s = fmaf(w.y, fmaxf(v[4 * i + 1] + u[4 * i + 1], 0.f), s);
+                    s = fmaf(w.z, fmaxf(v[4 * i + 2] + u[4 * i + 2], 0.f), s);
+                    s = fmaf(w.w, fmaxf(v[4 * i + 3] + u[4 * i + 3], 0.f), s);
+                  }
+                } else {
+                  tc::tmem_wait_ld();
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) {
+                    const float4 w = w4[i];
+                    s = fmaf(w.x, fmaxf(v[4 * i], 0.f), s);
+                    s = fmaf(w.y, fmaxf(v[4 * i + 1], 0.f), s);
+                    s = fmaf(w.z, fmaxf(v[4 * i + 2], 0.f), s);
+                    s = fmaf(w.w, fmaxf(v[4 * i + 3], 0.f), s);
+                  }
+                }
+              }
+              sc[qq] = s * kscale;
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+            if (use_hist && p < vis_r[0] && prow >= 0) {
+              const uint32_t key = order_key(sc[0]);
+              if (key) atomicAdd(&shist[key >> 20], 1u);
+            }
+#pragma unroll
+            for (int qq = 0; qq < QB; ++qq) {
+              if (qq < W.g.nrows && p < a.ld) {
+                float o = -INFINITY;
+                if (p < vis_r[qq]) o = prow >= 0 ? sc[qq] : (prow == -3 ? -INFINITY : NAN);
+                a.scores[static_cast<int64_t>(W.g.r0 + qq) * a.ld + p] = o;
+              }
             }
           }
+          const bool last = (si + 1 == n) || (W.j + 1 >= W.g.tiles);
+          if (last) {
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&qempty[qi]);
+          }
+          if (++stg == C::kNS) stg = 0;
+          if (++fbi == 2 * C::kNS) {
+            fbi = 0;
+            fph ^= 1u;
+          }
+          if (si + 1 < n) W.next(a);
         }
-        const bool last = (it + 1 == plan.n_items) || (W.j + 1 >= W.g.tiles);
-        if (last) {
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&qempty[qi]);
+        if (fail || !pooled) break;
+        if (!ring_take(k, &W, &n)) {
+          if (lane == 0) {
+            record_error(a.status, LSA_ERR_TIMEOUT, 0, 12);
+            *abort_flag = 1;
+          }
+          hist_row = -1;
+          break;
         }
-        if (++stg == C::kNS) {
-          stg = 0;
-          sph ^= 1u;
-        }
-        W.next(a);
+        __syncwarp();
+        if (lane == 0) ring_release(k);
+        if (n == 0) break;
       }
       if (use_hist && hist_row >= 0 && !flush_hist(hist_row) && lane == 0) {
         record_error(a.status, LSA_ERR_TIMEOUT, 0, 7);
@@ -1091,6 +1310,8 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
   scan_sync<NTH>();
   if (threadIdx.x == 0) {
     for (uint64_t* b = bars; b <= ebar; ++b) tc::mbar_inval(b);
+    if (pooled)
+      for (uint64_t* b = rfull; b < rempty + kRing; ++b) tc::mbar_inval(b);
   }
   scan_sync<NTH>();
   if (a.done_ctr) {

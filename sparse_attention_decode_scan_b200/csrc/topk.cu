@@ -587,10 +587,12 @@ bool topk_rows_plan(int32_t rows, int64_t n_cols, int* nseg, int64_t* seg_len) {
   return true;
 }
 
-void topk_step_flags(void* ws, int32_t rows, int64_t n_cols, uint32_t** scan_done, uint32_t** sel_done) {
+void topk_step_flags(void* ws, int32_t rows, int64_t n_cols, uint32_t** scan_done, uint32_t** sel_done,
+                     int** scan_pool) {
   const tk::TkLayout L = tk::tk_layout(ws, rows, n_cols);
   *scan_done = L.scan_done;
   *sel_done = L.sel_done;
+  if (scan_pool) *scan_pool = L.scan_pool;
 }
 
 size_t topk_ws_bytes(int32_t rows, int64_t n_cols, int32_t) {

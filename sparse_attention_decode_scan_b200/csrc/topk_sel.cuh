@@ -41,6 +41,7 @@ struct TkLayout {
   uint32_t* row_done;  // per row: collect CTAs finished (the last one selects)
   uint32_t* sel_done;  // per row: 1 once the row's selection is written (decode step)
   uint32_t* scan_done; // scan CTAs finished (decode step)
+  int* scan_pool;      // the scan's tile pool: chunks claimed so far (decode step)
   uint32_t* selready;  // per row: 1 once segoff and the marked bitmap are final, 2 once idx is (decode step)
   uint32_t* bitmap;
   uint2* cand;
@@ -69,6 +70,7 @@ __host__ __device__ inline TkLayout tk_layout(void* ws, int32_t rows, int64_t n_
   L.row_done = L.ctrl + kCtrlInts + 2 * rows;
   L.sel_done = L.ctrl + kCtrlInts + 3 * rows;
   L.scan_done = L.ctrl + 1;
+  L.scan_pool = reinterpret_cast<int*>(L.ctrl + 2);
   L.selready = L.ctrl + kCtrlInts + 4 * rows;
   b += tk_ctrl_bytes(rows);
   L.bitmap = reinterpret_cast<uint32_t*>(b);

@@ -68,6 +68,13 @@ def set_test_hooks(force_simt: bool = False, split_select_min_cols: int = -1, sc
                                     1 if no_cluster_topk else 0), "lsa_test_set_hooks")
 
 
+def set_test_scan_pool(static_pm: int = -1, chunk: int = 0) -> None:
+    """lsa_test_set_scan_pool of liblsa_test.so (include/lsa_test.h); needs use_test_library()."""
+    if not _use_test:
+        raise RuntimeError("test hooks exist only in liblsa_test.so: call use_test_library() first")
+    _check(lib().lsa_test_set_scan_pool(int(static_pm), int(chunk)), "lsa_test_set_scan_pool")
+
+
 def lib() -> ctypes.CDLL:
     """Loads liblsa.so (or, after use_test_library(), liblsa_test.so) once; raises if it is absent
     (no fallback path exists)."""
@@ -113,7 +120,8 @@ def lib() -> ctypes.CDLL:
              "lsa_two_stage_select", "lsa_block_select", "lsa_stage_blocks"]
     if path == TEST_LIB_PATH:
         L.lsa_test_set_hooks.argtypes = [i32, i64, ctypes.c_uint32, i32]
-        names.append("lsa_test_set_hooks")
+        L.lsa_test_set_scan_pool.argtypes = [i32, i32]
+        names += ["lsa_test_set_hooks", "lsa_test_set_scan_pool"]
     for f in names:
         getattr(L, f).restype = ctypes.c_int
     _libs[path] = L

@@ -38,3 +38,17 @@ def test_hooks():
     finally:
         lsa.set_test_hooks()
         lsa.use_test_library(False)
+
+
+@pytest.fixture
+def scan_pool():
+    """Routes the binding to liblsa_test.so and yields its scan-schedule setter
+    (lsa_test_set_scan_pool); restores the default schedule and the product
+    library afterwards."""
+    from sparse_attention_decode_scan_b200 import lsa
+    lsa.use_test_library(True)
+    try:
+        yield lsa.set_test_scan_pool
+    finally:
+        lsa.set_test_scan_pool()
+        lsa.use_test_library(False)

@@ -47,7 +47,7 @@ def test_test_library_exports_both_headers_and_the_product_no_switch(lsa):
     """liblsa_test.so exports lsa.h and lsa_test.h; liblsa.so exports nothing of lsa_test.h."""
     import ctypes as C
     test_only = declared_functions(TEST_HEADER)
-    assert test_only == ["lsa_test_set_hooks"]
+    assert test_only == ["lsa_test_set_hooks", "lsa_test_set_scan_pool"]
     prod = C.CDLL(lsa.LIB_PATH)
     for n in test_only:
         assert not hasattr(prod, n), f"{n} must exist only in the test build"
