@@ -43,12 +43,12 @@ lsa_status lsa_test_set_hooks(int32_t force_simt_path, int64_t split_select_min_
 /*
  * The decode scan's tile schedule inside lsa_decode_step and the DSA order of
  * lsa_decode_layers, for every later call in this process (process-wide, not
- * thread-safe).  Each scan CTA first takes its even share of the first
- * static_pm thousandths of the tiles, then claims chunks of `chunk` tiles from
- * a counter until none is left.
+ * thread-safe).  With a pool, each scan CTA first takes its even share of the
+ * first static_pm thousandths of the tiles, then claims chunks of `chunk`
+ * tiles from a counter until none is left.
  *   static_pm  0 .. 1000; > 1000: no pool (every tile in the static shares);
- *              < 0: the library's default (900).
- *   chunk      tiles per claim; <= 0: the library's default (4).
+ *              < 0: the library's default (no pool).
+ *   chunk      tiles per claim; <= 0: the default (4).
  * Every schedule computes each tile the same way, so the results are bitwise
  * the same; tests compare them.  Returns LSA_OK.
  */

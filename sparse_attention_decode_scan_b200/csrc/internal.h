@@ -67,7 +67,7 @@ struct ScoresArgs {
   // Tensor-core decode scan (one query row per tile, rows <= 256): if set
   // (zeroed by the caller), the CTAs share the first pool_static_pm
   // thousandths of the tiles evenly and claim the rest from this counter in
-  // chunks of pool_chunk tiles, so that they end together.
+  // chunks of pool_chunk tiles (a dynamic tail; off unless a test asks).
   int* pool = nullptr;
   int pool_chunk = 0;
   int pool_static_pm = 1000;

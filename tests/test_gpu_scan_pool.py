@@ -1,9 +1,10 @@
 """The decode scan's pooled tile schedule.
 
-Inside lsa_decode_step the scan's CTAs take an even share of most tiles and
-claim the rest from a counter in small chunks (so that they end together).
-Which CTA scores a tile does not change how the tile is scored, so every
-schedule must give bitwise the same step: selection, output and lse.  The
+With a pool (test build only: the library's default is the static split),
+the decode step's scan CTAs take an even share of most tiles and claim the
+rest from a counter in small chunks.  Which CTA scores a tile does not change
+how the tile is scored, so every schedule must give bitwise the same step:
+selection, output and lse.  The
 schedules below cover no pool at all, the default, every tile from the pool
 one at a time (the most segments, each CTA's first segment from the pool),
 chunks that cross rows, and a pool that is empty from the start (every CTA's
@@ -51,13 +52,13 @@ def test_pooled_step_bitwise_equals_static(name, scan_pool):
 
 
 def test_pooled_step_mid_size(scan_pool):
-    """Bitwise equality on the mid-size case, and the default schedule's
+    """Bitwise equality on the mid-size case, and a pooled schedule's
     selection on two rows against the oracle."""
     from sparse_attention_decode_scan_b200.device import DeviceCase
     case = _mid_case()
     dc = DeviceCase(case)
     _equal_steps(dc, scan_pool, SCHEDULES)
-    scan_pool()
+    scan_pool(900, 4)
     _, _, idx = _step(dc)
     idx_h = idx.cpu().numpy()
     for r in (0, case.rows - 1):
