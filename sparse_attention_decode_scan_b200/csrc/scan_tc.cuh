@@ -31,6 +31,10 @@
 // Two issuers, one per accumulator: an MMA of this size occupies the tensor
 // pipe for about as long as its issuer spends on the waits and bookkeeping of
 // a tile, so with one issuer the pipe idled half of the time.
+// Work: the query rows' tiles in row order, each CTA an even contiguous
+// share; every role walks the same sequence.  Optionally (decode) the CTAs
+// share only part of it and claim the rest in chunks from a counter, the
+// producer publishing each chunk to the other roles through a ring.
 // Every wait is bounded; a timeout records LSA_ERR_TIMEOUT and unwinds.
 #include <cuda.h>
 #include <cudaTypedefs.h>
