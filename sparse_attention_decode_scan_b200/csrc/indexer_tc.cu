@@ -150,6 +150,7 @@ bool scores_tc_supported(const ScoresArgs& a) {
   if (!aligned16(a.cache.idx_keys) || !aligned16(a.q_idx) || !aligned16(a.w)) return false;
   const int64_t kr = key_rows(a);
   if (kr <= 0 || kr >= (1LL << 31)) return false;
+  if (a.cache.max_len >= (1LL << 31)) return false;  // positions are kept as 32-bit integers
   if (a.key_dtype == LSA_FP8_E4M3 && (!a.cache.idx_key_scales || !aligned16(a.cache.idx_key_scales))) return false;
   return true;
 }

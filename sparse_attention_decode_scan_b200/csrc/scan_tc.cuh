@@ -940,8 +940,10 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       // are the first stage's and query buffer's plus constant offsets in the
       // start-address field (shared-memory addresses stay below 256 KB: adding
       // never carries out of that 14-bit field).
-      int s = 0, fbi = 0;       // the item's stage and full barrier
-      uint32_t fph = 0;         // and the barrier's phase
+      // the item's stage, and the passes over the stages so far (mod 4): its
+      // full barrier is s + kNS (sweep & 1), that barrier's phase sweep >> 1
+      int s = 0;
+      uint32_t sweep = 0;
       const uint64_t a_desc0 = tc::desc_sw128(tc::smem_u32(stages));
       const uint64_t b_desc0 = tc::desc_sw128(tc::smem_u32(qbufs));
       int64_t it = 0;  // items of every segment so far
@@ -957,7 +959,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
             }
           }
           if (static_cast<int>(it & 1) == who) {
-            if (!tc::mbar_wait(&full[fbi], fph, abort_flag)) {
+            if (!tc::mbar_wait(&full[s + C::kNS * (sweep & 1u)], sweep >> 1, abort_flag)) {
               fail = true;
               break;
             }
@@ -998,10 +1000,9 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
             tc::mma_commit(&empty[s]);
             tc::mma_commit(&tfull[acc]);
           }
-          if (++s == C::kNS) s = 0;
-          if (++fbi == 2 * C::kNS) {
-            fbi = 0;
-            fph ^= 1u;
+          if (++s == C::kNS) {
+            s = 0;
+            sweep = (sweep + 1u) & 3u;
           }
           // both issuers release the group's query buffer after its last tile
           // of the segment (a commit covers every MMA its thread issued before it)
@@ -1142,14 +1143,18 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
       if (n > 0) W.start(a, plan.r_first, plan.j_first);
       int gi = -1, qi = 0;
       int hist_row = -1;
-      int64_t vis_r[QB];
-      int stg = 0, fbi = 0;  // stage of item it and its full barrier
-      uint32_t fph = 0;      // and the barrier's phase
+      int32_t vis_r[QB];  // visible positions of the group's rows (below 2^31)
+      int stg = 0;          // stage of item it
+      uint32_t sweep = 0;   // passes over the stages (mod 4): full barrier and phase, as the issuers
       int64_t it = 0;     // items of every segment so far
       bool fail = false;
       for (int k = 0;; ++k) {
-        for (int64_t si = 0; si < n; ++si, ++it) {
-          if (si == 0 || W.j == 0) {
+        // `left` counts the segment's items down (fewer live 64-bit registers
+        // in the epilogue than an index and a bound)
+        bool seg_first = true;
+        for (int64_t left = n; left > 0; --left, ++it) {
+          if (seg_first || W.j == 0) {
+            seg_first = false;
             ++gi;
             qi = gi % C::kNQ;
             // a new row: the counts of the one before go to its histogram
@@ -1173,12 +1178,12 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
               break;
             }
             if (QB == 1) {
-              vis_r[0] = W.g.vis;  // the group's one row
+              vis_r[0] = static_cast<int32_t>(W.g.vis);  // the group's one row
             } else {
 #pragma unroll
               for (int qq = 0; qq < QB; ++qq) {
                 int bb;
-                vis_r[qq] = qq < W.g.nrows ? row_visible(a, W.g.r0 + qq, &bb) : 0;
+                vis_r[qq] = qq < W.g.nrows ? static_cast<int32_t>(row_visible(a, W.g.r0 + qq, &bb)) : 0;
               }
             }
           }
@@ -1202,7 +1207,7 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
             int32_t mrow = 0;  // contiguous bf16: every visible position has a key row
             float kscale = 1.f;
             if (stage_meta) {
-              if (!tc::mbar_wait(&full[fbi], fph, abort_flag)) {
+              if (!tc::mbar_wait(&full[stg + C::kNS * (sweep & 1u)], sweep >> 1, abort_flag)) {
                 if (lane == 0) {
                   record_error(a.status, LSA_ERR_TIMEOUT, 0, 8);
                   *abort_flag = 1;
@@ -1279,17 +1284,16 @@ __device__ __forceinline__ void scan_cta(const CUtensorMap* tmap_p, const CUtens
               }
             }
           }
-          const bool last = (si + 1 == n) || (W.j + 1 >= W.g.tiles);
+          const bool last = left == 1 || (W.j + 1 >= W.g.tiles);
           if (last) {
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&qempty[qi]);
           }
-          if (++stg == C::kNS) stg = 0;
-          if (++fbi == 2 * C::kNS) {
-            fbi = 0;
-            fph ^= 1u;
+          if (++stg == C::kNS) {
+            stg = 0;
+            sweep = (sweep + 1u) & 3u;
           }
-          if (si + 1 < n) W.next(a);
+          if (left > 1) W.next(a);
         }
         if (fail || !pooled) break;
         if (!ring_take(k, &W, &n)) {
