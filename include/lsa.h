@@ -30,8 +30,8 @@
  *     current device; structs (lsa_dims, lsa_cache) live in host memory and are
  *     read during the call only.  The caller owns every buffer.
  *   - The library never allocates device memory and never synchronises the
- *     stream, except lsa_read_device_status, which does both a copy and a
- *     stream synchronisation by design.
+ *     stream, except lsa_read_device_status and lsa_get_device_status, which
+ *     do both a copy and a stream synchronisation by design.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  A call returns after enqueueing.
  *   - Host-checkable argument errors return an error code and enqueue nothing.
@@ -397,6 +397,14 @@ lsa_status lsa_prefill_layers(const lsa_dims* d, int32_t n_layers, const lsa_cac
  * and synchronises `stream`.  Returns LSA_ERR_CUDA if a CUDA call fails.
  */
 lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream);
+
+/*
+ * The same read as a single status: the workspace status word (an lsa_status
+ * value, LSA_OK if no kernel recorded an error), which is cleared; or
+ * LSA_ERR_INVALID_ARG for a NULL workspace, or LSA_ERR_CUDA if a CUDA call of
+ * the read fails.  Synchronises `stream` like lsa_read_device_status.
+ */
+lsa_status lsa_get_device_status(void* ws, lsa_stream_t stream);
 
 /*
  * Top-k without a workspace argument, for callers that cannot allocate device

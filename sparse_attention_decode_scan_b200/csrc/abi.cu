@@ -900,6 +900,12 @@ lsa_status lsa_read_device_status(void* ws, int32_t* status, lsa_stream_t stream
   return LSA_OK;
 }
 
+lsa_status lsa_get_device_status(void* ws, lsa_stream_t stream) {
+  int32_t code = LSA_OK;
+  const lsa_status st = lsa_read_device_status(ws, &code, stream);
+  return st != LSA_OK ? st : static_cast<lsa_status>(code);
+}
+
 int32_t lsa_launch_count(const lsa_dims* d, int32_t rows, int64_t max_len, int32_t op, int32_t causal) {
   if (rows < 0 || max_len < 0) return -1;
   if (op == LSA_OP_TOPK ? (!d || d->top_k < 1) : !valid_dims(d)) return -1;

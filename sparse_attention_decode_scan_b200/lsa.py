@@ -98,6 +98,7 @@ def lib() -> ctypes.CDLL:
     PV = ctypes.POINTER(vp)
     L.lsa_decode_layers.argtypes = [D, i32, C, PV, PV, PV, PV, PV, i32, i32, vp, vp, sz, vp]
     L.lsa_read_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
+    L.lsa_get_device_status.argtypes = [vp, vp]
     L.lsa_status_string.argtypes = [ctypes.c_int]
     L.lsa_status_string.restype = ctypes.c_char_p
     L.lsa_version.restype = i32
@@ -116,7 +117,8 @@ def lib() -> ctypes.CDLL:
     L.lsa_prefill_layers.argtypes = [D, i32, C, i64, PV, i32, vp, PV, PV, PV, PV, PV, PV, i32, PV, vp, sz, vp, vp, PV]
     names = ["lsa_prefill_layers", "lsa_indexer_scores", "lsa_topk", "lsa_topk_noalloc", "lsa_sparse_attn_decode",
              "lsa_decode_step",
-             "lsa_decode_step_profiled", "lsa_decode_layers", "lsa_read_device_status", "lsa_candidate_scores",
+             "lsa_decode_step_profiled", "lsa_decode_layers", "lsa_read_device_status", "lsa_get_device_status",
+             "lsa_candidate_scores",
              "lsa_two_stage_select", "lsa_block_select", "lsa_stage_blocks"]
     if path == TEST_LIB_PATH:
         L.lsa_test_set_hooks.argtypes = [i32, i64, ctypes.c_uint32, i32]
@@ -341,6 +343,11 @@ def read_device_status(ws, stream=None) -> int:
     st = ctypes.c_int32(0)
     _check(lib().lsa_read_device_status(_ptr(ws), ctypes.byref(st), _stream(stream)), "lsa_read_device_status")
     return int(st.value)
+
+
+def get_device_status(ws, stream=None) -> int:
+    """lsa_get_device_status: the workspace status word (cleared), or the read's own error code."""
+    return int(lib().lsa_get_device_status(_ptr(ws), _stream(stream)))
 
 
 def launch_count(dims: Optional[Dims], rows: int, max_len: int, op: int, causal: bool = False) -> int:

@@ -106,3 +106,4 @@ def test_host_side_rejections_without_cuda(lsa):
                                None) == lsa.LSA_ERR_INVALID_ARG
     st = ctypes.c_int32(0)
     assert lib.lsa_read_device_status(None, ctypes.byref(st), None) == lsa.LSA_ERR_INVALID_ARG
+    assert lib.lsa_get_device_status(None, None) == lsa.LSA_ERR_INVALID_ARG

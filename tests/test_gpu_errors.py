@@ -78,6 +78,10 @@ def test_block_id_out_of_pool_is_reported(path, request):
     torch.cuda.synchronize()
     assert lsa.read_device_status(ws) == lsa.LSA_ERR_BOUNDS
     assert lsa.read_device_status(ws) == lsa.LSA_OK
+    # the single-status form reads and clears the same word
+    lsa.indexer_scores(dc.dims, dc.cache, dc.q_idx, dc.w, scores, ld, ws, row_seq=dc.row_seq)
+    assert lsa.get_device_status(ws) == lsa.LSA_ERR_BOUNDS
+    assert lsa.get_device_status(ws) == lsa.LSA_OK
 
 
 def test_length_above_max_len_is_reported():
